@@ -1,0 +1,222 @@
+/*
+ * tp_block.h -- C ABI of the tensor-parallel transformer block library (libtpblock.so).
+ *
+ * The library computes the Megatron-style tensor-parallel block on ONE GPU, with p as a logical
+ * partition of the weights:
+ *
+ *   MLP  ("How does tensor parallelism split a transformer feed-forward block's two matmuls
+ *         across devices?", sections "Column split, then row split", "The nonlinearity is free",
+ *         "Second matmul, row-parallel", "One collective"; "Tensor Parallelism" (klaylearn), Notes,
+ *         the column/row split paragraph):
+ *     shard i owns the column slice W1_i (and Wu_i for the gated form) and the matching row slice
+ *     W2_i;  h_i = act(x W1_i)  (column-parallel, activation local to the shard);
+ *     y_i = h_i W2_i  (row-parallel: a full-shape partial sum);  y = sum_i y_i  (the all-reduce's
+ *     arithmetic, done on the device in the fixed order i = 0 .. p-1 in fp32).
+ *   Backward ("The backward pass"): dY is replicated (the exit's backward is the identity); every
+ *     shard computes its own dW1_i, dW2_i with no exchange and a partial dx_i; dx = sum_i dx_i.
+ *   Attention ("Tensor Parallelism", Notes, grouped-query paragraph): Q/K/V column-parallel so a
+ *     shard owns n_q/p whole query heads and n_kv/p whole KV heads, attention runs locally over
+ *     them, the output projection is row-parallel and the p partials are summed.
+ *
+ * Conventions for every call:
+ *   - Every buffer is caller-owned device memory unless stated otherwise; the library allocates
+ *     nothing.  Matrices are row-major and densely packed.  "stream" is a cudaStream_t (NULL = the
+ *     legacy default stream); every call only enqueues work on it and returns without waiting.
+ *   - bf16 data (TP_BF16) is accumulated in fp32; results are rounded once to bf16 (round to
+ *     nearest even).  TP_F32 data is computed in fp32 throughout.
+ *   - Arguments are validated before anything is enqueued; on any error nothing is written and
+ *     the call returns a non-zero tp_status; tp_last_error() gives a message (per host thread).
+ *   - No call traps or aborts.  Device-side waits are bounded; a wait that runs out records an
+ *     error word that tp_check_device_error() reports as TP_ERR_TIMEOUT.
+ *   - Weights are taken in the pages' orientation Y = X W, i.e. W[in][out] row-major, and packed
+ *     once into a per-shard device layout (below) by the *_pack calls.
+ */
+#ifndef TP_BLOCK_H
+#define TP_BLOCK_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  TP_OK = 0,
+  TP_ERR_INVALID_ARG = 1,   /* null/misaligned pointer, negative size, bad enum value          */
+  TP_ERR_SHAPE = 2,         /* p does not divide d_ff, or n_q / n_kv; n_kv does not divide n_q  */
+  TP_ERR_UNSUPPORTED = 3,   /* valid but not implemented combination                            */
+  TP_ERR_WORKSPACE = 4,     /* workspace smaller than the *_workspace() query says              */
+  TP_ERR_CUDA = 5,          /* a CUDA runtime call failed (message in tp_last_error)            */
+  TP_ERR_TIMEOUT = 6        /* a bounded device-side wait ran out (tp_check_device_error)       */
+} tp_status;
+
+typedef enum { TP_F32 = 0, TP_BF16 = 1 } tp_dtype;
+
+/* The elementwise nonlinearity between the two MLP matmuls ("The nonlinearity is free":
+ * GELU, ReLU, or a gated variant computed from the same slice).  GELU is the exact erf form;
+ * SWIGLU is h = silu(x Wg) * (x Wu) with silu(z) = z / (1 + exp(-z)). */
+typedef enum { TP_ACT_IDENTITY = 0, TP_ACT_RELU = 1, TP_ACT_GELU = 2, TP_ACT_SWIGLU = 3 } tp_act;
+
+/* How the p partial sums are added ("One collective").
+ *   TP_REDUCE_SEPARATE: each shard's partial goes to fp32 workspace, then one vectorised
+ *                       reduce kernel adds them (order 0..p-1) and rounds once.
+ *   TP_REDUCE_FUSED:    the down-projection kernel adds the p shard partials of its output tile
+ *                       in the same order without writing them to memory.                      */
+typedef enum { TP_REDUCE_SEPARATE = 0, TP_REDUCE_FUSED = 1 } tp_reduce_mode;
+
+/* ------------------------------------------------------------------------------------------ */
+/* MLP block                                                                                   */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  int64_t T;            /* tokens (rows of x); 0 is allowed (empty batch)                     */
+  int64_t d;            /* hidden size                                                        */
+  int64_t d_ff;         /* intermediate size F; must be a multiple of p                       */
+  int32_t p;            /* logical shards, >= 1                                               */
+  int32_t act;          /* tp_act                                                             */
+  int32_t dtype;        /* tp_dtype of x, weights, y, dy, dx                                  */
+  int32_t reduce_mode;  /* tp_reduce_mode                                                     */
+} tp_mlp_desc;
+
+/* Packed layouts.  F_s = d_ff / p; F_sp = F_s rounded up to a multiple of 128 (padding rows and
+ * columns are zero).  R = 2*F_sp for SWIGLU, else F_sp.  Element type = desc.dtype.
+ *   w1p  [p][R][d]   SWIGLU: rows of shard i come in blocks of 256; rows 0..127 of block j hold
+ *                    gate features f = j*128 + r (column i*F_s + f of Wg), rows 128..255 the same
+ *                    features of Wu.  Other activations: row c of shard i is column i*F_s + c of
+ *                    W1.  (Each row is one column of the user's matrix: K-major for x W1.)
+ *   w2p  [p][d][F_sp] w2p[i][n][c] = W2[i*F_s + c][n]  (shard i's row slice, transposed).       */
+size_t tp_mlp_w1_packed_bytes(const tp_mlp_desc* desc);
+size_t tp_mlp_w2_packed_bytes(const tp_mlp_desc* desc);
+
+/* Pack user weights into the per-shard layout.  w1 = W1 (or Wg) [d][d_ff]; w_up = Wu [d][d_ff]
+ * for SWIGLU, NULL otherwise; w2 = W2 [d_ff][d].  All device pointers, element type desc.dtype.
+ * One-time setup; not part of the steady-state step. */
+tp_status tp_mlp_pack(const tp_mlp_desc* desc, const void* w1, const void* w_up, const void* w2,
+                      void* w1p, void* w2p, void* stream);
+
+/* Activations saved by the forward pass for the backward pass: z [T][p*R] (the pre-activations
+ * in w1p's row order) followed by h [T][p*F_sp] (the activated values), element type dtype. */
+size_t tp_mlp_saved_bytes(const tp_mlp_desc* desc);
+
+/* Workspace of tp_mlp_fwd in bytes (its contents need not survive between calls). */
+size_t tp_mlp_fwd_workspace(const tp_mlp_desc* desc);
+
+/* Forward: y = residual + sum_{i=0}^{p-1} act(x W1_i) W2_i.
+ *   x [T][d], y [T][d] (dtype).  residual: NULL, or [T][d] dtype added once after the sum
+ *   (the residual add that follows the reduction and stays replicated).  residual may equal y.
+ *   saved: NULL, or tp_mlp_saved_bytes() of device memory that receives z and h for
+ *   tp_mlp_bwd.  Adds 1 to the reduction counter.
+ *   Errors: TP_ERR_INVALID_ARG (null x/w1p/w2p/y/workspace with T>0, bad enum),
+ *   TP_ERR_SHAPE (p < 1, d < 1, d_ff % p), TP_ERR_WORKSPACE (ws_bytes too small). */
+tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p, const void* w2p,
+                     const void* residual, void* y, void* saved, void* workspace,
+                     size_t ws_bytes, void* stream);
+
+/* Workspace of tp_mlp_bwd in bytes. */
+size_t tp_mlp_bwd_workspace(const tp_mlp_desc* desc);
+
+/* Backward from the replicated output gradient dy [T][d] (dtype), the forward's x and saved.
+ *   dx  [T][d] dtype = sum_i dx_i (summed in order 0..p-1 in fp32, rounded once).
+ *   dw1p, dw2p: fp32 gradients in the packed layouts of w1p / w2p, one slice per shard with no
+ *   exchange between shards (padding entries are zero).  Adds 1 to the reduction counter. */
+tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const void* x, const void* saved,
+                     const void* w1p, const void* w2p, void* dx, void* dw1p, void* dw2p,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* Scatter packed fp32 gradients back to the user layout (fp32): dw1 [d][d_ff] (dWg for SWIGLU),
+ * dw_up [d][d_ff] (SWIGLU only, else NULL), dw2 [d_ff][d]. */
+tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw1p, const void* dw2p,
+                              void* dw1, void* dw_up, void* dw2, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Attention block                                                                             */
+/* ------------------------------------------------------------------------------------------ */
+
+typedef struct {
+  int64_t b;            /* sequences                                                          */
+  int64_t s;            /* tokens per sequence in this call (1 for decode)                    */
+  int64_t h;            /* hidden size                                                        */
+  int32_t n_q;          /* query heads                                                        */
+  int32_t n_kv;         /* key/value heads; must divide n_q                                   */
+  int32_t head_dim;     /* multiple of 8, <= 256                                              */
+  int32_t p;            /* logical shards; must divide n_q and n_kv (heads are never split)  */
+  int32_t causal;       /* 1: query t sees keys <= t                                          */
+  int32_t dtype;        /* tp_dtype                                                           */
+  int64_t kv_len;       /* 0: self-attention over the s tokens.  > 0: decode (s must be 1) over
+                           kv_len cached positions plus the new token                         */
+  int64_t kv_cap;       /* slots per head in the caches (>= kv_len + 1); 0 means kv_len + 1  */
+  int32_t reduce_mode;  /* tp_reduce_mode                                                     */
+  int32_t reserved;
+} tp_attn_desc;
+
+/* Packed layouts (element type dtype): qh = n_q/p, kh = n_kv/p, hd = head_dim,
+ * R_a = (qh + 2*kh) * hd.
+ *   wqkv_p [p][R_a][h]: shard i's rows are Wq columns i*qh*hd .. (qh*hd rows), then Wk columns
+ *                       i*kh*hd .. (kh*hd rows), then Wv columns likewise.
+ *   wo_p   [p][h][qh*hd]: wo_p[i][n][c] = Wo[i*qh*hd + c][n].                                 */
+size_t tp_attn_wqkv_packed_bytes(const tp_attn_desc* desc);
+size_t tp_attn_wo_packed_bytes(const tp_attn_desc* desc);
+
+/* wq [h][n_q*hd], wk and wv [h][n_kv*hd], wo [n_q*hd][h]; device pointers, dtype. */
+tp_status tp_attn_pack(const tp_attn_desc* desc, const void* wq, const void* wk, const void* wv,
+                       const void* wo, void* wqkv_p, void* wo_p, void* stream);
+
+size_t tp_attn_fwd_workspace(const tp_attn_desc* desc);
+
+/* y = residual + sum_i Attn_i(x) Wo_i.  x and y [b][s][h] dtype; residual NULL or [b][s][h].
+ * Query head j of shard i attends over KV head floor(j / (n_q/n_kv)); scale 1/sqrt(head_dim).
+ * Decode (kv_len > 0, s == 1): k_cache and v_cache are [b][n_kv][kv_cap][hd] dtype; the new
+ * token's key and value are written to slot kv_len and it attends to slots 0..kv_len.
+ * Self-attention (kv_len == 0): caches may be NULL.  Adds 1 to the reduction counter. */
+tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const void* wqkv_p,
+                      const void* wo_p, void* k_cache, void* v_cache, const void* residual,
+                      void* y, void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Reduction and glue                                                                          */
+/* ------------------------------------------------------------------------------------------ */
+
+/* out[j] = residual[j] + sum_{i=0}^{p-1} partials[i*n + j]: the all-reduce's arithmetic
+ * ("One collective"; "Tensor Parallelism", Notes: Y = sum_i Z_i).  Summed in fp32 in the order
+ * i = 0 .. p-1, residual (optional, out_dtype) added last, rounded once to out_dtype.
+ * partials: [p][n] of in_dtype.  Adds 1 to the reduction counter. */
+tp_status tp_reduce_partials(const void* partials, int32_t p, int64_t n, int32_t in_dtype,
+                             const void* residual, void* out, int32_t out_dtype, void* stream);
+
+/* Row-wise RMSNorm with unit weight: out = x / sqrt(mean(x^2) + eps), fp32 math, the
+ * normalization that follows the residual add and stays replicated ("One collective").
+ * x, out [rows][d] dtype (out may equal x). */
+tp_status tp_rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void* out,
+                     int32_t dtype, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
+/* Diagnostics                                                                                 */
+/* ------------------------------------------------------------------------------------------ */
+
+/* Reductions of p partials enqueued so far (one per tp_mlp_fwd / tp_mlp_bwd / tp_attn_fwd /
+ * tp_reduce_partials call that succeeded), process-wide. */
+uint64_t tp_reduction_count(void);
+void tp_reset_reduction_count(void);
+
+/* Kernels this library has launched so far, process-wide. */
+uint64_t tp_launch_count(void);
+
+/* Message of the last failed call on this host thread ("" if none). */
+const char* tp_last_error(void);
+const char* tp_status_string(int32_t status);
+
+/* Waits for the stream, then reports (and clears) the device error word: TP_ERR_TIMEOUT if a
+ * bounded device wait ran out since the last check, TP_ERR_CUDA on a CUDA error, else TP_OK. */
+tp_status tp_check_device_error(void* stream);
+
+/* 1 if this build contains the sm_100a tensor-core kernels and the current device runs them. */
+int32_t tp_tensor_core_path_available(void);
+
+/* Library version, major*10000 + minor*100 + patch. */
+int32_t tp_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+#endif /* TP_BLOCK_H */

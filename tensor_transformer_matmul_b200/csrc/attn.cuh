@@ -1,0 +1,450 @@
+// Attention block internals: layout, packing, QKV projection, local GQA attention per shard,
+// KV-cache append, row-parallel output projection and the partial-sum reduce.
+#pragma once
+
+#include <algorithm>
+
+#include "gemm_launch.cuh"
+#include "pack.cuh"
+#include "reduce.cuh"
+#include "simt.cuh"
+#include "tp_common.cuh"
+
+namespace tp {
+
+struct AttnLayout {
+  int64_t b, s, h, tokens, kv_len, kv_cap;
+  int n_q, n_kv, hd, p, qh, kh, causal, dtype, eb;
+  int64_t R_a;          // packed QKV rows per shard
+  size_t wqkv_bytes, wo_bytes;
+  size_t qkv_off, o_off, part_off, ml_off, ws_bytes;
+  int kv_splits;        // decode: key chunks per (sequence, KV head)
+};
+
+constexpr int kDecodeChunk = 256;   // keys per decode work item
+
+inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
+  if (!d) return set_error(TP_ERR_INVALID_ARG, "desc is null");
+  if (d->b < 0 || d->s < 0) return set_error(TP_ERR_SHAPE, "b and s must be >= 0");
+  if (d->h < 1 || d->n_q < 1 || d->n_kv < 1 || d->p < 1)
+    return set_error(TP_ERR_SHAPE, "h, n_q, n_kv and p must be >= 1");
+  if (d->n_q % d->n_kv) return set_error(TP_ERR_SHAPE, "n_kv must divide n_q");
+  if (d->n_q % d->p || d->n_kv % d->p)
+    return set_error(TP_ERR_SHAPE, "p must divide n_q and n_kv (heads are never split)");
+  if (d->head_dim < 8 || d->head_dim > 256 || d->head_dim % 8)
+    return set_error(TP_ERR_SHAPE, "head_dim must be a multiple of 8 in [8, 256]");
+  if (d->dtype != TP_F32 && d->dtype != TP_BF16) return set_error(TP_ERR_INVALID_ARG, "dtype");
+  if (d->reduce_mode != TP_REDUCE_SEPARATE && d->reduce_mode != TP_REDUCE_FUSED)
+    return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
+  if (d->kv_len < 0) return set_error(TP_ERR_SHAPE, "kv_len must be >= 0");
+  if (d->kv_len > 0 && d->s != 1) return set_error(TP_ERR_SHAPE, "decode (kv_len > 0) needs s == 1");
+  L->b = d->b; L->s = d->s; L->h = d->h; L->tokens = d->b * d->s;
+  L->n_q = d->n_q; L->n_kv = d->n_kv; L->hd = d->head_dim; L->p = d->p;
+  L->qh = d->n_q / d->p; L->kh = d->n_kv / d->p;
+  L->causal = d->causal ? 1 : 0; L->dtype = d->dtype; L->eb = elem_bytes(d->dtype);
+  L->kv_len = d->kv_len;
+  L->kv_cap = d->kv_cap > 0 ? d->kv_cap : d->kv_len + 1;
+  if (L->kv_len > 0 && L->kv_cap < L->kv_len + 1)
+    return set_error(TP_ERR_SHAPE, "kv_cap must be >= kv_len + 1");
+  L->R_a = static_cast<int64_t>(L->qh + 2 * L->kh) * L->hd;
+  const int64_t P = L->p;
+  L->wqkv_bytes = static_cast<size_t>(P * L->R_a * L->h) * L->eb;
+  L->wo_bytes = static_cast<size_t>(P * L->h * L->qh * L->hd) * L->eb;
+  L->kv_splits = L->kv_len > 0 ? static_cast<int>(ceil_div(L->kv_len + 1, kDecodeChunk)) : 0;
+  const size_t qkvb = static_cast<size_t>(L->tokens * P * L->R_a) * L->eb;
+  const size_t ob = static_cast<size_t>(L->tokens * L->n_q * L->hd) * L->eb;
+  const size_t partb = static_cast<size_t>(P * L->tokens * L->h) * 4;
+  // decode split-KV scratch: per (sequence, q head, split) an (m, l) pair and hd outputs
+  const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (2 + L->hd) * 4;
+  L->qkv_off = 0;
+  L->o_off = align256(qkvb);
+  L->part_off = L->o_off + align256(ob);
+  L->ml_off = L->part_off + align256(partb);
+  L->ws_bytes = L->ml_off + align256(mlb);
+  return TP_OK;
+}
+
+template <typename T>
+inline tp_status attn_pack_t(const AttnLayout& L, const void* wq, const void* wk, const void* wv,
+                             const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s) {
+  pack::ColMap cm{};
+  cm.kind = 2;
+  cm.R = L.R_a;
+  cm.q_rows = static_cast<int64_t>(L.qh) * L.hd;
+  cm.k_rows = static_cast<int64_t>(L.kh) * L.hd;
+  cm.src[0] = wq; cm.src[1] = wk; cm.src[2] = wv;
+  cm.ld[0] = static_cast<int64_t>(L.n_q) * L.hd;
+  cm.ld[1] = cm.ld[2] = static_cast<int64_t>(L.n_kv) * L.hd;
+  const int64_t rows = L.p * L.R_a;
+  dim3 blk(32, 8);
+  dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.h, 32)), 1);
+  if (!pack::grid_ok(g1.x, g1.y, 1)) return set_error(TP_ERR_UNSUPPORTED, "pack grid too large");
+  pack::pack_cols_kernel<T><<<g1, blk, 0, s>>>(static_cast<T*>(wqkv_p), rows, L.h, cm);
+  TP_LAUNCH_CHECK();
+  const int64_t K = static_cast<int64_t>(L.qh) * L.hd;
+  dim3 g2(static_cast<unsigned>(ceil_div(L.h, 32)), static_cast<unsigned>(ceil_div(K, 32)),
+          static_cast<unsigned>(L.p));
+  if (!pack::grid_ok(g2.x, g2.y, g2.z)) return set_error(TP_ERR_UNSUPPORTED, "pack grid too large");
+  pack::pack_rows_kernel<T><<<g2, blk, 0, s>>>(static_cast<T*>(wo_p), L.p, L.h, K, K,
+                                               static_cast<const T*>(wo), L.h);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+inline tp_status attn_pack(const AttnLayout& L, const void* wq, const void* wk, const void* wv,
+                           const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s) {
+  return L.dtype == TP_BF16 ? attn_pack_t<__nv_bfloat16>(L, wq, wk, wv, wo, wqkv_p, wo_p, s)
+                            : attn_pack_t<float>(L, wq, wk, wv, wo, wqkv_p, wo_p, s);
+}
+
+namespace attn {
+
+// Index helpers into the packed qkv activations [tokens][p * R_a].
+struct QkvIdx {
+  int64_t ld;     // p * R_a
+  int64_t R_a;
+  int qh, kh, hd, group;   // group = n_q / n_kv
+  __device__ __forceinline__ int64_t q(int64_t t, int j) const {   // global q head j
+    const int i = j / qh, jj = j - i * qh;
+    return t * ld + i * R_a + static_cast<int64_t>(jj) * hd;
+  }
+  __device__ __forceinline__ int64_t k(int64_t t, int g) const {   // global kv head g
+    const int i = g / kh, gg = g - i * kh;
+    return t * ld + i * R_a + static_cast<int64_t>(qh + gg) * hd;
+  }
+  __device__ __forceinline__ int64_t v(int64_t t, int g) const {
+    const int i = g / kh, gg = g - i * kh;
+    return t * ld + i * R_a + static_cast<int64_t>(qh + kh + gg) * hd;
+  }
+};
+
+// Prefill attention, one warp per (token, query head), online softmax over the visible keys.
+// o[t][j*hd + e]; lane l holds dims l, l+32, ... of q and of the running output.
+template <typename T>
+__global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, QkvIdx ix,
+                                                           int64_t b, int64_t s, int n_q,
+                                                           int causal, float scale) {
+  constexpr int kMaxPerLane = 8;  // head_dim <= 256
+  const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (wid >= b * s * n_q) return;
+  const int j = static_cast<int>(wid % n_q);
+  const int64_t t = wid / n_q;          // global token
+  const int64_t bi = t / s, pos = t - bi * s;
+  const int g = j / ix.group;
+  const int per = (ix.hd + 31) / 32;
+  float q[kMaxPerLane], acc[kMaxPerLane];
+#pragma unroll
+  for (int r = 0; r < kMaxPerLane; ++r) {
+    const int e = lane + 32 * r;
+    q[r] = (r < per && e < ix.hd) ? to_f(qkv[ix.q(t, j) + e]) * scale : 0.f;
+    acc[r] = 0.f;
+  }
+  float m = -INFINITY, l = 0.f;
+  const int64_t last = causal ? pos : s - 1;
+  for (int64_t kp = 0; kp <= last; ++kp) {
+    const int64_t tk = bi * s + kp;
+    const int64_t kb = ix.k(tk, g), vb = ix.v(tk, g);
+    float dot = 0.f;
+#pragma unroll
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int e = lane + 32 * r;
+      if (r < per && e < ix.hd) dot = fmaf(q[r], to_f(qkv[kb + e]), dot);
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+    const float mn = fmaxf(m, dot);
+    const float corr = expf(m - mn), pw = expf(dot - mn);
+    l = l * corr + pw;
+#pragma unroll
+    for (int r = 0; r < kMaxPerLane; ++r) {
+      const int e = lane + 32 * r;
+      if (r < per && e < ix.hd) acc[r] = acc[r] * corr + pw * to_f(qkv[vb + e]);
+    }
+    m = mn;
+  }
+  const float inv = 1.f / l;
+#pragma unroll
+  for (int r = 0; r < kMaxPerLane; ++r) {
+    const int e = lane + 32 * r;
+    if (r < per && e < ix.hd) o[t * static_cast<int64_t>(n_q) * ix.hd + j * ix.hd + e] = from_f<T>(acc[r] * inv);
+  }
+}
+
+// Decode: write the new token's keys and values into slot kv_len of the caches
+// [b][n_kv][kv_cap][hd].
+template <typename T>
+__global__ void kv_append_kernel(const T* qkv, QkvIdx ix, T* kc, T* vc, int64_t b, int n_kv,
+                                 int64_t kv_cap, int64_t slot) {
+  const int64_t total = b * n_kv * ix.hd;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int e = static_cast<int>(idx % ix.hd);
+    const int64_t bg = idx / ix.hd;
+    const int g = static_cast<int>(bg % n_kv);
+    const int64_t bi = bg / n_kv;
+    const int64_t dst = ((bi * n_kv + g) * kv_cap + slot) * ix.hd + e;
+    kc[dst] = qkv[ix.k(bi, g) + e];
+    vc[dst] = qkv[ix.v(bi, g) + e];
+  }
+}
+
+// Decode attention, split over keys.  Block = (split c, kv head g, sequence bi); its warps share
+// the chunk's keys; every query head of the group is handled in the same pass so each K/V row is
+// read once.  Output per (bi, q head, split): running max m, denominator l, unnormalised o[hd].
+template <typename T, int GROUP, int HD>
+__global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx ix, const T* kc,
+                                                           const T* vc, int64_t kv_cap,
+                                                           int64_t n_keys, int n_q, int n_kv,
+                                                           float scale, float* ml) {
+  constexpr int kWarps = 8;
+  constexpr int PER = HD / 32;           // dims per lane
+  __shared__ float s_m[kWarps][GROUP], s_l[kWarps][GROUP];
+  __shared__ float s_o[kWarps][GROUP][HD];
+  const int c = blockIdx.x, g = blockIdx.y;
+  const int64_t bi = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int64_t k0 = static_cast<int64_t>(c) * kDecodeChunk;
+  const int64_t k1 = min(n_keys, k0 + kDecodeChunk);
+  float q[GROUP][PER], acc[GROUP][PER], m[GROUP], l[GROUP];
+#pragma unroll
+  for (int a = 0; a < GROUP; ++a) {
+    const int j = g * GROUP + a;
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      q[a][r] = to_f(qkv[ix.q(bi, j) + lane + 32 * r]) * scale;
+      acc[a][r] = 0.f;
+    }
+    m[a] = -INFINITY;
+    l[a] = 0.f;
+  }
+  const T* kbase = kc + (bi * n_kv + g) * kv_cap * HD;
+  const T* vbase = vc + (bi * n_kv + g) * kv_cap * HD;
+  for (int64_t kp = k0 + warp; kp < k1; kp += kWarps) {
+    float kv[PER], vv[PER];
+#pragma unroll
+    for (int r = 0; r < PER; ++r) {
+      kv[r] = to_f(kbase[kp * HD + lane + 32 * r]);
+      vv[r] = to_f(vbase[kp * HD + lane + 32 * r]);
+    }
+#pragma unroll
+    for (int a = 0; a < GROUP; ++a) {
+      float dot = 0.f;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) dot = fmaf(q[a][r], kv[r], dot);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+      const float mn = fmaxf(m[a], dot);
+      const float corr = __expf(m[a] - mn), pw = __expf(dot - mn);
+      l[a] = l[a] * corr + pw;
+#pragma unroll
+      for (int r = 0; r < PER; ++r) acc[a][r] = acc[a][r] * corr + pw * vv[r];
+      m[a] = mn;
+    }
+  }
+#pragma unroll
+  for (int a = 0; a < GROUP; ++a) {
+    if (lane == 0) {
+      s_m[warp][a] = m[a];
+      s_l[warp][a] = l[a];
+    }
+#pragma unroll
+    for (int r = 0; r < PER; ++r) s_o[warp][a][lane + 32 * r] = acc[a][r];
+  }
+  __syncthreads();
+  // combine the warps: thread (a, e) for a < GROUP, e < HD
+  for (int idx = threadIdx.x; idx < GROUP * HD; idx += blockDim.x) {
+    const int a = idx / HD, e = idx - a * HD;
+    float mm = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, s_m[w][a]);
+    float ll = 0.f, oo = 0.f;
+    for (int w = 0; w < kWarps; ++w) {
+      const float f = s_m[w][a] == -INFINITY ? 0.f : __expf(s_m[w][a] - mm);
+      ll += s_l[w][a] * f;
+      oo += s_o[w][a][e] * f;
+    }
+    const int j = g * GROUP + a;
+    float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * (2 + HD);
+    if (e == 0) {
+      rec[0] = mm;
+      rec[1] = ll;
+    }
+    rec[2 + e] = oo;
+  }
+}
+
+// Merge the splits: o[bi][j*hd + e] = sum_c exp(m_c - M) o_c / sum_c exp(m_c - M) l_c.
+template <typename T>
+__global__ void decode_combine_kernel(const float* ml, int splits, int hd, int64_t rows, T* o) {
+  const int64_t total = rows * hd;
+  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
+       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
+    const int64_t r = idx / hd;
+    const int e = static_cast<int>(idx - r * hd);
+    const float* rec = ml + r * splits * (2 + hd);
+    float M = -INFINITY;
+    for (int c = 0; c < splits; ++c) M = fmaxf(M, rec[c * (2 + hd)]);
+    float L = 0.f, acc = 0.f;
+    for (int c = 0; c < splits; ++c) {
+      const float* rc = rec + c * (2 + hd);
+      const float f = rc[0] == -INFINITY ? 0.f : expf(rc[0] - M);
+      L += rc[1] * f;
+      acc += rc[2 + e] * f;
+    }
+    o[idx] = from_f<T>(acc / L);
+  }
+}
+
+}  // namespace attn
+
+template <typename T>
+inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, void* kc, void* vc,
+                           float* ml, cudaStream_t s) {
+  const T* qkv = static_cast<const T*>(qkv_v);
+  T* o = static_cast<T*>(o_v);
+  attn::QkvIdx ix{L.p * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
+  const float scale = 1.0f / sqrtf(static_cast<float>(L.hd));
+  if (L.kv_len == 0) {
+    const int64_t warps = L.tokens * L.n_q;
+    const int64_t blocks = ceil_div(warps * 32, 128);
+    if (blocks > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "attention grid too large");
+    attn::prefill_simt_kernel<T><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
+        qkv, o, ix, L.b, L.s, L.n_q, L.causal, scale);
+    TP_LAUNCH_CHECK();
+    return TP_OK;
+  }
+  // decode: append, split-KV attention, combine
+  {
+    const int64_t total = L.b * L.n_kv * L.hd;
+    attn::kv_append_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
+        qkv, ix, static_cast<T*>(kc), static_cast<T*>(vc), L.b, L.n_kv, L.kv_cap, L.kv_len);
+    TP_LAUNCH_CHECK();
+  }
+  const int group = L.n_q / L.n_kv;
+  dim3 grid(static_cast<unsigned>(L.kv_splits), static_cast<unsigned>(L.n_kv),
+            static_cast<unsigned>(L.b));
+  if (L.b > 65535) return set_error(TP_ERR_UNSUPPORTED, "decode batch above 65535");
+  const int64_t n_keys = L.kv_len + 1;
+#define TP_DECODE_CASE(G, H)                                                                  \
+  if (group == G && L.hd == H) {                                                              \
+    attn::decode_split_kernel<T, G, H><<<grid, 256, 0, s>>>(qkv, ix, static_cast<const T*>(kc),  \
+        static_cast<const T*>(vc), L.kv_cap, n_keys, L.n_q, L.n_kv, scale, ml);               \
+    TP_LAUNCH_CHECK();                                                                        \
+  } else
+  TP_DECODE_CASE(8, 128) TP_DECODE_CASE(4, 128) TP_DECODE_CASE(2, 128) TP_DECODE_CASE(1, 128)
+  TP_DECODE_CASE(8, 64) TP_DECODE_CASE(4, 64) TP_DECODE_CASE(2, 64) TP_DECODE_CASE(1, 64)
+  TP_DECODE_CASE(1, 32) TP_DECODE_CASE(2, 32) TP_DECODE_CASE(4, 32) TP_DECODE_CASE(8, 32)
+  {
+    return set_error(TP_ERR_UNSUPPORTED,
+                     "decode supports head_dim in {32, 64, 128} and n_q/n_kv in {1, 2, 4, 8}");
+  }
+#undef TP_DECODE_CASE
+  const int64_t rows = L.b * L.n_q;
+  attn::decode_combine_kernel<T><<<simt::elementwise_grid(rows * L.hd), 256, 0, s>>>(
+      ml, L.kv_splits, L.hd, rows, o);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+namespace attn_tc {
+using tc::Operand;
+template <int BN, int ASUB>
+using KK = tc::TileCfg<BN, ASUB, false, false,
+                       std::min(8, (200 * 1024) / (128 * ASUB * 64 * 2 + BN * 64 * 2))>;
+
+inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, void* qkv,
+                          cudaStream_t s) {
+  const int64_t rows = L.p * L.R_a;
+  tc::EpiHidden::Params ep;
+  ep.h = static_cast<__nv_bfloat16*>(qkv);
+  ep.z = nullptr;
+  ep.ld_h = rows;
+  ep.ld_z = 0;
+  ep.tokens = static_cast<int32_t>(L.tokens);
+  ep.rows = static_cast<int32_t>(rows);
+  ep.act = TP_ACT_IDENTITY;
+  const Operand xo{x, false, L.tokens, L.h, 1, L.h, 0};
+  const Operand wo{wqkv, false, rows, L.h, 1, L.h, 0};
+  if (L.tokens <= 128) {
+    ep.swap = 1;
+    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
+    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
+    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
+  }
+  ep.swap = 0;
+  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s);
+}
+
+inline tp_status out_proj_partials(const AttnLayout& L, const void* o, const void* wo_p,
+                                   float* part, cudaStream_t s) {
+  const int64_t K = static_cast<int64_t>(L.qh) * L.hd;
+  const Operand ao{o, false, L.tokens, K, L.p, static_cast<int64_t>(L.n_q) * L.hd, K};
+  const Operand wo{wo_p, false, L.h, K, L.p, K, L.h * K};
+  tc::EpiStoreF32::Params ep;
+  ep.out = part;
+  ep.ld = L.h;
+  ep.batch_stride = L.tokens * L.h;
+  ep.rows_valid = static_cast<int32_t>(L.tokens);
+  ep.cols_valid = static_cast<int32_t>(L.h);
+  if (L.tokens <= 128) {
+    ep.swap = 1;
+    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
+    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
+    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
+  }
+  ep.swap = 0;
+  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s);
+}
+}  // namespace attn_tc
+
+template <typename T>
+inline tp_status attn_simt_proj(const AttnLayout& L, const void* x, const void* wqkv, void* qkv,
+                                const void* o, const void* wo_p, float* part, cudaStream_t s,
+                                bool first) {
+  const int64_t P = L.p;
+  simt::GemmArgs g{};
+  if (first) {
+    g.a = x; g.a_bs = 0; g.a_sm = L.h; g.a_sk = 1;
+    g.b = wqkv; g.b_bs = 0; g.b_sm = L.h; g.b_sk = 1;
+    g.out = qkv; g.o_bs = 0; g.o_sm = P * L.R_a; g.o_sn = 1;
+    g.M = L.tokens; g.N = P * L.R_a; g.K = L.h; g.batch = 1; g.out_f32 = 0;
+    return simt::gemm<T>(g, s);
+  }
+  const int64_t K = static_cast<int64_t>(L.qh) * L.hd;
+  g.a = o; g.a_bs = K; g.a_sm = static_cast<int64_t>(L.n_q) * L.hd; g.a_sk = 1;
+  g.b = wo_p; g.b_bs = L.h * K; g.b_sm = K; g.b_sk = 1;
+  g.out = part; g.o_bs = L.tokens * L.h; g.o_sm = L.h; g.o_sn = 1;
+  g.M = L.tokens; g.N = L.h; g.K = K; g.batch = P; g.out_f32 = 1;
+  return simt::gemm<T>(g, s);
+}
+
+inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wqkv,
+                              const void* wo_p, void* kc, void* vc, const void* residual,
+                              void* y, void* ws, cudaStream_t s) {
+  uint8_t* w = static_cast<uint8_t*>(ws);
+  void* qkv = w + L.qkv_off;
+  void* o = w + L.o_off;
+  float* part = reinterpret_cast<float*>(w + L.part_off);
+  float* ml = reinterpret_cast<float*>(w + L.ml_off);
+  tp_status st;
+  const bool tc_ok = L.dtype == TP_BF16 && L.h % 8 == 0 && tensor_cores_usable();
+  if (tc_ok) {
+    for (const void* q : {x, wqkv, wo_p, residual, static_cast<const void*>(y)})
+      if (q && (reinterpret_cast<uintptr_t>(q) & 15))
+        return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, s)) != TP_OK) return st;
+    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_tc::out_proj_partials(L, o, wo_p, part, s)) != TP_OK) return st;
+  } else if (L.dtype == TP_BF16) {
+    if ((st = attn_simt_proj<__nv_bfloat16>(L, x, wqkv, qkv, o, wo_p, part, s, true)) != TP_OK) return st;
+    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_simt_proj<__nv_bfloat16>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
+  } else {
+    if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, true)) != TP_OK) return st;
+    if ((st = attn_core<float>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
+  }
+  return reduce::launch(part, TP_F32, L.p, L.tokens * L.h, residual, y, L.dtype, s);
+}
+
+}  // namespace tp

@@ -1,0 +1,576 @@
+// Persistent, warp-specialised tcgen05 GEMM core for sm_100a.
+//
+//   D[b][m][n] = sum_k A_b(m, k) * B_b(n, k)      (bf16 operands, fp32 accumulator in TMEM)
+//
+// Roles (192 threads):  warp 0 lane 0 -- TMA producer: fills a ring of shared-memory stages;
+//                       warp 1 lane 0 -- MMA issuer: tcgen05.mma into one of two TMEM
+//                                        accumulators, frees stages with tcgen05.commit;
+//                       warps 2..5    -- epilogue: tcgen05.ld the accumulator, apply the fused
+//                                        elementwise step, store to global memory.
+// Tiles are walked persistently (tile = blockIdx.x + i * gridDim.x), so the epilogue of one tile
+// overlaps the main loop of the next.
+//
+// Operands are 3-D TMA tensors (inner, outer, batch) with 128-byte swizzle.  A K-major operand has
+// K as its inner dimension (box 64 x rows); an MN-major operand has M (or N) as its inner
+// dimension and is loaded in 64-wide MN blocks (box 64 x 64), which lets the backward pass use
+// transposed operands without materialising transposes.  Out-of-range boxes are zero-filled by
+// TMA, so ragged M, N and K need no special casing in the main loop.
+//
+// Every wait is bounded (tp::kWaitTimeoutNs); a wait that runs out raises a shared abort flag,
+// records the site in the device error word, lets in-flight copies and MMAs land (bounded), frees
+// TMEM and returns.
+#pragma once
+
+#include <cuda.h>
+#include <stdint.h>
+
+#include "sm100.cuh"
+#include "tp_common.cuh"
+
+namespace tp {
+namespace tc {
+
+constexpr int kBK = 64;          // K per stage: 64 bf16 = one 128-byte swizzle row
+constexpr int kUmmaK = 16;       // K per tcgen05.mma (kind::f16)
+constexpr int kThreads = 192;
+constexpr int kEpiWarps = 4;
+
+// Compile-time tile configuration.
+//   BN     : N of each MMA (columns of the accumulator), 16..256, multiple of 16
+//   A_SUB  : 128-row MMAs per tile (1 or 2); A tile = 128*A_SUB rows, each sub-tile has its own
+//            accumulator (columns s*BN .. s*BN+BN-1)
+//   A_MN / B_MN : operand is MN-major (else K-major)
+//   STAGES : depth of the shared-memory ring
+template <int BN_, int A_SUB_, bool A_MN_, bool B_MN_, int STAGES_>
+struct TileCfg {
+  static constexpr int BN = BN_;
+  static constexpr int A_SUB = A_SUB_;
+  static constexpr bool A_MN = A_MN_;
+  static constexpr bool B_MN = B_MN_;
+  static constexpr int STAGES = STAGES_;
+  static constexpr int A_ROWS = 128 * A_SUB;
+  static constexpr int A_STAGE_BYTES = A_ROWS * kBK * 2;
+  static constexpr int B_STAGE_BYTES = BN * kBK * 2;
+  static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
+  static constexpr int ACC_COLS = A_SUB * BN;
+  static constexpr int TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
+                                   : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr uint32_t IDESC = sm100::make_idesc_bf16(128, BN, A_MN, B_MN);
+  static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 step 16");
+  static_assert(A_SUB == 1 || A_SUB == 2, "A_SUB");
+  static_assert(2 * ACC_COLS <= 512, "two accumulators must fit in TMEM");
+  static_assert(!B_MN || BN % 64 == 0, "MN-major operands are loaded in 64-wide blocks");
+  static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
+};
+
+struct GemmParams {
+  int32_t M, N, K;        // per problem
+  int32_t batch;          // independent problems (e.g. shards)
+  int32_t m_blocks, n_blocks, k_blocks;
+  int32_t m_fastest;      // tile order: walk M blocks first (1) or N blocks first (0)
+  int32_t a_batched, b_batched;  // operand's batch coordinate = problem index (else 0)
+  uint32_t* err;          // device error word
+};
+
+// What the epilogue of one tile sees.
+struct EpiCtx {
+  uint32_t taddr;   // TMEM address: this warp's 32 lanes, column 0 of the tile's accumulator
+  int row;          // accumulator row (A row within the tile) held by this thread, 0..127
+  int b;            // problem index
+  int m0;           // first A row of the tile
+  int n0;           // first B row of the tile
+};
+
+__device__ __forceinline__ void decode_tile(int t, const GemmParams& gp, int& b, int& mb,
+                                            int& nb) {
+  const int per = gp.m_blocks * gp.n_blocks;
+  b = t / per;
+  const int r = t - b * per;
+  if (gp.m_fastest) {
+    mb = r % gp.m_blocks;
+    nb = r / gp.m_blocks;
+  } else {
+    nb = r % gp.n_blocks;
+    mb = r / gp.n_blocks;
+  }
+}
+
+// Bounded wait used on the abort path only: ignores the abort flag.
+__device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint32_t* err) {
+  const uint64_t t0 = globaltimer_ns();
+  while (!sm100::mbar_try_wait(bar, parity)) {
+    if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      record_device_error(err, DEVERR_WAIT_DRAIN);
+      return false;
+    }
+  }
+  return true;
+}
+
+template <class Cfg, class Epi>
+__global__ void __launch_bounds__(kThreads, 1)
+    gemm_kernel(const __grid_constant__ CUtensorMap tma_a,
+                const __grid_constant__ CUtensorMap tma_b, const GemmParams gp,
+                const typename Epi::Params ep) {
+  using namespace sm100;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* a_smem = smem;
+  uint8_t* b_smem = smem + Cfg::STAGES * Cfg::A_STAGE_BYTES;
+  uint64_t* full = reinterpret_cast<uint64_t*>(b_smem + Cfg::STAGES * Cfg::B_STAGE_BYTES);
+  uint64_t* empty = full + Cfg::STAGES;
+  uint64_t* acc_full = empty + Cfg::STAGES;  // [2]
+  uint64_t* acc_empty = acc_full + 2;        // [2]
+  uint64_t* drain = acc_empty + 2;           // [1]
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < Cfg::STAGES; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int a = 0; a < 2; ++a) {
+      mbar_init(&acc_full[a], 1);
+      mbar_init(&acc_empty[a], kEpiWarps);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tma_a);
+    tma_prefetch_desc(&tma_b);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, Cfg::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int num_tiles = gp.batch * gp.m_blocks * gp.n_blocks;
+
+  if (warp == 0) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ TMA producer
+      int stage = 0;
+      uint32_t phase = 0;
+      uint32_t issued_mask = 0;   // stages that received at least one load
+      uint32_t last_parity = 0;   // parity of the last phase issued into each stage
+      bool ok = true;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
+        int b, mb, nb;
+        decode_tile(t, gp, b, mb, nb);
+        const int m0 = mb * Cfg::A_ROWS;
+        const int n0 = nb * Cfg::BN;
+        const int za = gp.a_batched ? b : 0;
+        const int zb = gp.b_batched ? b : 0;
+        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
+            ok = false;
+            break;
+          }
+          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+          const int k0 = kb * kBK;
+          uint8_t* sa = a_smem + stage * Cfg::A_STAGE_BYTES;
+          uint8_t* sb = b_smem + stage * Cfg::B_STAGE_BYTES;
+          if (Cfg::A_MN) {
+#pragma unroll
+            for (int j = 0; j < Cfg::A_ROWS / 64; ++j)
+              tma_load_3d(&tma_a, &full[stage], sa + j * 64 * kBK * 2, m0 + 64 * j, k0, za);
+          } else {
+            tma_load_3d(&tma_a, &full[stage], sa, k0, m0, za);
+          }
+          if (Cfg::B_MN) {
+#pragma unroll
+            for (int j = 0; j < Cfg::BN / 64; ++j)
+              tma_load_3d(&tma_b, &full[stage], sb + j * 64 * kBK * 2, n0 + 64 * j, k0, zb);
+          } else {
+            tma_load_3d(&tma_b, &full[stage], sb, k0, n0, zb);
+          }
+          issued_mask |= 1u << stage;
+          last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA can exit
+        for (int s = 0; s < Cfg::STAGES; ++s)
+          if (issued_mask & (1u << s)) drain_wait(&full[s], (last_parity >> s) & 1u, gp.err);
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      // ------------------------------------------------------------------ MMA issuer
+      int stage = 0;
+      uint32_t phase = 0;
+      int it = 0;
+      bool ok = true;
+      bool issued_any = false;
+      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
+        const int acc = it & 1;
+        const uint32_t acc_phase = (it >> 1) & 1;
+        if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, gp.err,
+                       DEVERR_WAIT_ACC_EMPTY)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const uint32_t d_base = tmem_base + acc * Cfg::ACC_COLS;
+        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, gp.err, DEVERR_WAIT_FULL)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t a_addr = smem_addr(a_smem + stage * Cfg::A_STAGE_BYTES);
+          const uint32_t b_addr = smem_addr(b_smem + stage * Cfg::B_STAGE_BYTES);
+#pragma unroll
+          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+            const uint64_t bdesc =
+                Cfg::B_MN ? make_sdesc_sw128(b_addr + kk * (kUmmaK * 128), 64 * kBK * 2, 1024)
+                          : make_sdesc_sw128(b_addr + kk * (kUmmaK * 2), 16, 1024);
+#pragma unroll
+            for (int s = 0; s < Cfg::A_SUB; ++s) {
+              const uint32_t a_sub = a_addr + s * 128 * kBK * 2;
+              const uint64_t adesc =
+                  Cfg::A_MN ? make_sdesc_sw128(a_sub + kk * (kUmmaK * 128), 64 * kBK * 2, 1024)
+                            : make_sdesc_sw128(a_sub + kk * (kUmmaK * 2), 16, 1024);
+              umma_f16(d_base + s * Cfg::BN, adesc, bdesc, Cfg::IDESC,
+                       (kb | kk) != 0 ? 1u : 0u);
+            }
+          }
+          issued_any = true;
+          umma_commit(&empty[stage]);
+          if (++stage == Cfg::STAGES) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        umma_commit(&acc_full[acc]);
+      }
+      if (!ok && issued_any) {
+        // every MMA issued so far must finish before TMEM is released
+        umma_commit(drain);
+        drain_wait(drain, 0, gp.err);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue warps
+    const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
+    const int row = quarter * 32 + lane;
+    int it = 0;
+    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
+      const int acc = it & 1;
+      const uint32_t acc_phase = (it >> 1) & 1;
+      int ok = 0;
+      if (lane == 0)
+        ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, gp.err, DEVERR_WAIT_ACC_FULL);
+      ok = __shfl_sync(0xffffffffu, ok, 0);
+      if (!ok) break;
+      tc_fence_after();
+      int b, mb, nb;
+      decode_tile(t, gp, b, mb, nb);
+      EpiCtx ctx;
+      ctx.taddr = tmem_base + acc * Cfg::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
+      ctx.row = row;
+      ctx.b = b;
+      ctx.m0 = mb * Cfg::A_ROWS;
+      ctx.n0 = nb * Cfg::BN;
+      Epi::template run<Cfg>(ep, gp, ctx);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&acc_empty[acc]);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem_base, Cfg::TMEM_COLS);
+}
+
+// ---------------------------------------------------------------------------------------------
+// Epilogue helpers
+// ---------------------------------------------------------------------------------------------
+
+// Load 32 consecutive fp32 accumulator columns of this thread's row.
+__device__ __forceinline__ void acc_load32(uint32_t taddr, int col, float (&v)[32]) {
+  uint32_t r[32];
+  sm100::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(col), r);
+  sm100::tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+}
+__device__ __forceinline__ void acc_load16(uint32_t taddr, int col, float (&v)[16]) {
+  uint32_t r[16];
+  sm100::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(col), r);
+  sm100::tmem_wait_ld();
+#pragma unroll
+  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 bf16 values to 64 contiguous bytes (16-byte aligned destination).
+__device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
+  uint4* d = reinterpret_cast<uint4*>(dst);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w;
+    w.x = pack_bf16x2(v[8 * q + 0], v[8 * q + 1]);
+    w.y = pack_bf16x2(v[8 * q + 2], v[8 * q + 3]);
+    w.z = pack_bf16x2(v[8 * q + 4], v[8 * q + 5]);
+    w.w = pack_bf16x2(v[8 * q + 6], v[8 * q + 7]);
+    d[q] = w;
+  }
+}
+__device__ __forceinline__ void load_bf16x32(const __nv_bfloat16* src, float (&v)[32]) {
+  const uint4* s = reinterpret_cast<const uint4*>(src);
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    uint4 w = s[q];
+    v[8 * q + 0] = bf16lo(w.x); v[8 * q + 1] = bf16hi(w.x);
+    v[8 * q + 2] = bf16lo(w.y); v[8 * q + 3] = bf16hi(w.y);
+    v[8 * q + 4] = bf16lo(w.z); v[8 * q + 5] = bf16hi(w.z);
+    v[8 * q + 6] = bf16lo(w.w); v[8 * q + 7] = bf16hi(w.w);
+  }
+}
+
+__device__ __forceinline__ float fast_silu(float z) { return z / (1.0f + __expf(-z)); }
+__device__ __forceinline__ float fast_sigmoid(float z) { return 1.0f / (1.0f + __expf(-z)); }
+
+// ---------------------------------------------------------------------------------------------
+// Forward up-projection epilogue: h = act(acc) (or silu(gate) * up), optional saved z.
+//   Non-swapped (A = x tokens, B = packed W1 rows): accumulator row = token, column = packed row.
+//   Swapped (A = packed W1 rows, B = x tokens):     accumulator row = packed row, column = token.
+// SwiGLU tiles hold 128 gate features and the same 128 up features: non-swapped BN = 256 with
+// gate in columns 0..127 and up in 128..255; swapped A_SUB = 2 with gate in sub-tile 0 and up in
+// sub-tile 1.  h column of feature (block j, offset o) is j*128 + o in the padded layout.
+// ---------------------------------------------------------------------------------------------
+struct EpiHidden {
+  struct Params {
+    __nv_bfloat16* h;   // [tokens][ld_h]
+    __nv_bfloat16* z;   // [tokens][ld_z] or null
+    int64_t ld_h, ld_z;
+    int32_t tokens;     // valid tokens
+    int32_t rows;       // valid packed rows (columns of z)
+    int32_t act;        // tp_act
+    int32_t swap;       // 1: A = weights, B = tokens
+  };
+
+  template <class Cfg>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+    const bool swiglu = p.act == TP_ACT_SWIGLU;
+    if (!p.swap) {
+      const int t = c.m0 + c.row;
+      const bool live = t < p.tokens;
+      if (swiglu) {
+        // BN == 256, n0 multiple of 256
+        const int blk = c.n0 >> 8;
+#pragma unroll 1
+        for (int col = 0; col < 128; col += 32) {
+          float g[32], u[32];
+          acc_load32(c.taddr, col, g);
+          acc_load32(c.taddr, 128 + col, u);
+          if (live) {
+            if (p.z) {
+              store_bf16x32(p.z + t * p.ld_z + c.n0 + col, g);
+              store_bf16x32(p.z + t * p.ld_z + c.n0 + 128 + col, u);
+            }
+            float hv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) hv[e] = fast_silu(g[e]) * u[e];
+            store_bf16x32(p.h + t * p.ld_h + blk * 128 + col, hv);
+          }
+        }
+      } else {
+#pragma unroll 1
+        for (int col = 0; col < Cfg::BN; col += 32) {
+          float v[32];
+          acc_load32(c.taddr, col, v);
+          const int r0 = c.n0 + col;
+          if (live && r0 + 32 <= p.rows) {
+            if (p.z) store_bf16x32(p.z + t * p.ld_z + r0, v);
+            float hv[32];
+#pragma unroll
+            for (int e = 0; e < 32; ++e) hv[e] = act_f(p.act, v[e]);
+            store_bf16x32(p.h + t * p.ld_h + r0, hv);
+          } else if (live) {
+#pragma unroll
+            for (int e = 0; e < 32; ++e) {
+              if (r0 + e < p.rows) {
+                if (p.z) p.z[t * p.ld_z + r0 + e] = __float2bfloat16_rn(v[e]);
+                p.h[t * p.ld_h + r0 + e] = __float2bfloat16_rn(act_f(p.act, v[e]));
+              }
+            }
+          }
+        }
+      }
+    } else {
+      // swapped: this thread owns packed row (m0 + row); columns are tokens n0 + col
+      if (swiglu) {
+        const int blk = c.m0 >> 8;
+        const int feat = blk * 128 + c.row;
+        const int zg = c.m0 + c.row, zu = c.m0 + 128 + c.row;
+#pragma unroll 1
+        for (int col = 0; col < Cfg::BN; col += 16) {
+          float g[16], u[16];
+          acc_load16(c.taddr, col, g);
+          acc_load16(c.taddr, Cfg::BN + col, u);
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = c.n0 + col + e;
+            if (t < p.tokens) {
+              p.h[t * p.ld_h + feat] = __float2bfloat16_rn(fast_silu(g[e]) * u[e]);
+              if (p.z) {
+                p.z[t * p.ld_z + zg] = __float2bfloat16_rn(g[e]);
+                p.z[t * p.ld_z + zu] = __float2bfloat16_rn(u[e]);
+              }
+            }
+          }
+        }
+      } else {
+        const int r = c.m0 + c.row;
+        const bool live = r < p.rows;
+#pragma unroll 1
+        for (int col = 0; col < Cfg::BN; col += 16) {
+          float v[16];
+          acc_load16(c.taddr, col, v);  // whole warp: tcgen05.ld is warp-collective
+          if (!live) continue;
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int t = c.n0 + col + e;
+            if (t < p.tokens) {
+              p.h[t * p.ld_h + r] = __float2bfloat16_rn(act_f(p.act, v[e]));
+              if (p.z) p.z[t * p.ld_z + r] = __float2bfloat16_rn(v[e]);
+            }
+          }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+// fp32 store of the accumulator: out[b][i][j] = D (or D^T when swapped), with i < rows_valid and
+// j < cols_valid.  Used for the row-parallel partial sums y_i, the dx partials and the weight
+// gradients.  Non-swapped: i = m (A row), j = n.  Swapped: i = n (token), j = m (feature).
+// ---------------------------------------------------------------------------------------------
+struct EpiStoreF32 {
+  // requires Cfg::A_SUB == 1
+  struct Params {
+    float* out;
+    int64_t ld;            // elements between rows
+    int64_t batch_stride;  // elements between problems
+    int32_t rows_valid, cols_valid;
+    int32_t swap;
+  };
+
+  template <class Cfg>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+    float* base = p.out + static_cast<int64_t>(c.b) * p.batch_stride;
+    if (!p.swap) {
+      const int i = c.m0 + c.row;
+      const bool live = i < p.rows_valid;
+#pragma unroll 1
+      for (int col = 0; col < Cfg::BN; col += 32) {
+        float v[32];
+        acc_load32(c.taddr, col, v);
+        const int j0 = c.n0 + col;
+        if (live) {
+          float* dst = base + i * p.ld + j0;
+          if (j0 + 32 <= p.cols_valid && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+            float4* d4 = reinterpret_cast<float4*>(dst);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          } else {
+#pragma unroll
+            for (int e = 0; e < 32; ++e)
+              if (j0 + e < p.cols_valid) dst[e] = v[e];
+          }
+        }
+      }
+    } else {
+      const int j = c.m0 + c.row;
+      const bool live = j < p.cols_valid;
+#pragma unroll 1
+      for (int col = 0; col < Cfg::BN; col += 16) {
+        float v[16];
+        acc_load16(c.taddr, col, v);
+        if (live) {
+#pragma unroll
+          for (int e = 0; e < 16; ++e) {
+            const int i = c.n0 + col + e;
+            if (i < p.rows_valid) base[i * p.ld + j] = v[e];
+          }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+// Backward epilogue of dH_i = dY W2_i^T (A = dY tokens, B = w2p[i] MN-major, problem = shard):
+// turns dH into the pre-activation gradient dz using the saved z, written in w1p's row order.
+//   SwiGLU: dg = dH * u * silu'(g), du = dH * silu(g);  other activations: dz = dH * act'(z).
+// ---------------------------------------------------------------------------------------------
+struct EpiActBwd {
+  struct Params {
+    const __nv_bfloat16* z;   // saved pre-activations [T][ld]
+    __nv_bfloat16* dz;        // [T][ld]
+    int64_t ld;               // p * R
+    int32_t R;                // packed rows per shard
+    int32_t tokens;
+    int32_t act;
+  };
+
+  template <class Cfg>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+    const int t = c.m0 + c.row;
+    const bool live = t < p.tokens;
+    const int64_t rowoff = static_cast<int64_t>(t) * p.ld + static_cast<int64_t>(c.b) * p.R;
+#pragma unroll 1
+    for (int col = 0; col < Cfg::BN; col += 32) {
+      float dh[32];
+      acc_load32(c.taddr, col, dh);
+      if (!live) continue;
+      const int f = c.n0 + col;                  // shard-local padded feature (multiple of 32)
+      if (p.act == TP_ACT_SWIGLU) {
+        const int zc = (f >> 7) * 256 + (f & 127);   // gate column; up column is zc + 128
+        float g[32], u[32], dg[32], du[32];
+        load_bf16x32(p.z + rowoff + zc, g);
+        load_bf16x32(p.z + rowoff + zc + 128, u);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) {
+          const float s = fast_sigmoid(g[e]);
+          dg[e] = dh[e] * u[e] * (s * (1.0f + g[e] * (1.0f - s)));
+          du[e] = dh[e] * g[e] * s;
+        }
+        store_bf16x32(p.dz + rowoff + zc, dg);
+        store_bf16x32(p.dz + rowoff + zc + 128, du);
+      } else {
+        float zv[32], d[32];
+        load_bf16x32(p.z + rowoff + f, zv);
+#pragma unroll
+        for (int e = 0; e < 32; ++e) d[e] = dh[e] * act_grad_f(p.act, zv[e]);
+        store_bf16x32(p.dz + rowoff + f, d);
+      }
+    }
+  }
+};
+
+}  // namespace tc
+}  // namespace tp

@@ -1,0 +1,146 @@
+// Partial-sum reduce and RMSNorm kernels (HBM-bound, vectorised, coalesced).
+#pragma once
+
+#include "tp_common.cuh"
+
+namespace tp {
+namespace reduce {
+
+template <typename T> struct Vec8;
+template <> struct Vec8<float> {
+  __device__ __forceinline__ static void load(const float* p, float (&v)[8]) {
+    const float4 a = reinterpret_cast<const float4*>(p)[0];
+    const float4 b = reinterpret_cast<const float4*>(p)[1];
+    v[0] = a.x; v[1] = a.y; v[2] = a.z; v[3] = a.w; v[4] = b.x; v[5] = b.y; v[6] = b.z; v[7] = b.w;
+  }
+  __device__ __forceinline__ static void store(float* p, const float (&v)[8]) {
+    reinterpret_cast<float4*>(p)[0] = make_float4(v[0], v[1], v[2], v[3]);
+    reinterpret_cast<float4*>(p)[1] = make_float4(v[4], v[5], v[6], v[7]);
+  }
+};
+template <> struct Vec8<__nv_bfloat16> {
+  __device__ __forceinline__ static void load(const __nv_bfloat16* p, float (&v)[8]) {
+    const uint4 w = *reinterpret_cast<const uint4*>(p);
+    v[0] = bf16lo(w.x); v[1] = bf16hi(w.x); v[2] = bf16lo(w.y); v[3] = bf16hi(w.y);
+    v[4] = bf16lo(w.z); v[5] = bf16hi(w.z); v[6] = bf16lo(w.w); v[7] = bf16hi(w.w);
+  }
+  __device__ __forceinline__ static void store(__nv_bfloat16* p, const float (&v)[8]) {
+    uint4 w;
+    w.x = pack_bf16x2(v[0], v[1]); w.y = pack_bf16x2(v[2], v[3]);
+    w.z = pack_bf16x2(v[4], v[5]); w.w = pack_bf16x2(v[6], v[7]);
+    *reinterpret_cast<uint4*>(p) = w;
+  }
+};
+
+// out[j] = res[j] + sum_{s=0}^{p-1} part[s*n + j]   (fp32, in order, one rounding)
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) reduce_vec8_kernel(const Tin* __restrict__ part, int p,
+                                                          int64_t n, const Tout* res,
+                                                          Tout* out) {
+  const int64_t nv = n >> 3;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+       i += stride) {
+    float acc[8];
+    Vec8<Tin>::load(part + 8 * i, acc);
+    for (int s = 1; s < p; ++s) {
+      float v[8];
+      Vec8<Tin>::load(part + static_cast<int64_t>(s) * n + 8 * i, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    }
+    if (res) {
+      float r[8];
+      Vec8<Tout>::load(res + 8 * i, r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = r[e] + acc[e];
+    }
+    Vec8<Tout>::store(out + 8 * i, acc);
+  }
+}
+
+template <typename Tin, typename Tout>
+__global__ void reduce_scalar_kernel(const Tin* part, int p, int64_t n, const Tout* res,
+                                     Tout* out) {
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < n; j += stride) {
+    float acc = to_f(part[j]);
+    for (int s = 1; s < p; ++s) acc += to_f(part[static_cast<int64_t>(s) * n + j]);
+    if (res) acc = to_f(res[j]) + acc;
+    out[j] = from_f<Tout>(acc);
+  }
+}
+
+template <typename Tin, typename Tout>
+inline tp_status launch_t(const void* part, int p, int64_t n, const void* res, void* out,
+                          cudaStream_t s) {
+  if (n == 0) return TP_OK;
+  const bool vec = (n % 8 == 0) && (reinterpret_cast<uintptr_t>(part) % 16 == 0) &&
+                   (reinterpret_cast<uintptr_t>(out) % 16 == 0) &&
+                   (!res || reinterpret_cast<uintptr_t>(res) % 16 == 0);
+  const int64_t work = vec ? n / 8 : n;
+  int64_t blocks = ceil_div(work, 256);
+  const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
+  if (blocks > cap) blocks = cap;
+  if (vec)
+    reduce_vec8_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
+        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+  else
+    reduce_scalar_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
+        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+inline tp_status launch(const void* part, int in_dtype, int p, int64_t n, const void* res,
+                        void* out, int out_dtype, cudaStream_t s) {
+  if (in_dtype == TP_F32 && out_dtype == TP_F32) return launch_t<float, float>(part, p, n, res, out, s);
+  if (in_dtype == TP_F32 && out_dtype == TP_BF16)
+    return launch_t<float, __nv_bfloat16>(part, p, n, res, out, s);
+  if (in_dtype == TP_BF16 && out_dtype == TP_F32)
+    return launch_t<__nv_bfloat16, float>(part, p, n, res, out, s);
+  return launch_t<__nv_bfloat16, __nv_bfloat16>(part, p, n, res, out, s);
+}
+
+// out[r] = x[r] / sqrt(mean(x[r]^2) + eps), one block per row.
+template <typename T>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* x, int64_t d, float eps, T* out) {
+  __shared__ float red[8];
+  const T* xr = x + blockIdx.x * d;
+  T* orow = out + blockIdx.x * d;
+  float ss = 0.f;
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
+    const float v = to_f(xr[j]);
+    ss = fmaf(v, v, ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) orow[j] = from_f<T>(to_f(xr[j]) * scale);
+}
+
+inline tp_status rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void* out, int dtype,
+                         cudaStream_t s) {
+  if (rows == 0) return TP_OK;
+  if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
+  if (dtype == TP_BF16)
+    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), 256, 0, s>>>(
+        static_cast<const __nv_bfloat16*>(x), d, eps, static_cast<__nv_bfloat16*>(out));
+  else
+    rmsnorm_kernel<float><<<static_cast<unsigned>(rows), 256, 0, s>>>(
+        static_cast<const float*>(x), d, eps, static_cast<float*>(out));
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+}  // namespace reduce
+}  // namespace tp

@@ -1,0 +1,143 @@
+// Library-wide state of libtpblock: error messages, counters, the device error word, device
+// queries and TMA tensor-map encoding.
+#include <cuda.h>
+#include <cudaTypedefs.h>
+#include <atomic>
+#include <mutex>
+#include <string>
+
+#include "tp_common.cuh"
+
+namespace tp {
+
+namespace {
+thread_local std::string t_last_error;
+std::atomic<uint64_t> g_reductions{0};
+std::atomic<uint64_t> g_launches{0};
+__device__ uint32_t d_error_word = 0;
+}  // namespace
+
+tp_status set_error(tp_status st, const std::string& msg) {
+  t_last_error = msg;
+  return st;
+}
+void clear_error() { t_last_error.clear(); }
+void count_launch(uint64_t n) { g_launches.fetch_add(n, std::memory_order_relaxed); }
+void count_reduction() { g_reductions.fetch_add(1, std::memory_order_relaxed); }
+
+uint32_t* device_error_word() {
+  static uint32_t* addr[64] = {nullptr};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return nullptr;
+  if (!addr[dev]) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, d_error_word) != cudaSuccess) return nullptr;
+    addr[dev] = static_cast<uint32_t*>(p);
+  }
+  return addr[dev];
+}
+
+int num_sms() {
+  static int cache[64] = {0};
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return 148;
+  if (!cache[dev]) {
+    int n = 0;
+    cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev);
+    cache[dev] = n > 0 ? n : 148;
+  }
+  return cache[dev];
+}
+
+bool tensor_cores_usable() {
+  static int cache[64] = {0};  // 0 unknown, 1 yes, 2 no
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= 64) return false;
+  if (!cache[dev]) {
+    int major = 0, minor = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cache[dev] = (major == 10 && minor == 0) ? 1 : 2;
+  }
+  return cache[dev] == 1;
+}
+
+static PFN_cuTensorMapEncodeTiled_v12000 get_encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) ==
+            cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+tp_status encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner, uint64_t outer,
+                              uint64_t batch, uint64_t outer_stride_bytes,
+                              uint64_t batch_stride_bytes, uint32_t box_inner, uint32_t box_outer) {
+  auto fn = get_encode_fn();
+  if (!fn) return set_error(TP_ERR_CUDA, "cuTensorMapEncodeTiled unavailable");
+  if (outer_stride_bytes % 16 || batch_stride_bytes % 16)
+    return set_error(TP_ERR_INVALID_ARG, "tensor-core operand row stride not a multiple of 16 bytes");
+  cuuint64_t dims[3] = {inner, outer, batch};
+  cuuint64_t strides[2] = {outer_stride_bytes, batch_stride_bytes};
+  cuuint32_t box[3] = {box_inner, box_outer, 1};
+  cuuint32_t estr[3] = {1, 1, 1};
+  CUresult r = fn(map, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void*>(base), dims, strides,
+                  box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                  CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS)
+    return set_error(TP_ERR_CUDA, "cuTensorMapEncodeTiled failed (code " + std::to_string(r) + ")");
+  return TP_OK;
+}
+
+}  // namespace tp
+
+extern "C" {
+
+uint64_t tp_reduction_count(void) { return tp::g_reductions.load(); }
+void tp_reset_reduction_count(void) { tp::g_reductions.store(0); }
+uint64_t tp_launch_count(void) { return tp::g_launches.load(); }
+const char* tp_last_error(void) { return tp::t_last_error.c_str(); }
+
+const char* tp_status_string(int32_t s) {
+  switch (s) {
+    case TP_OK: return "TP_OK";
+    case TP_ERR_INVALID_ARG: return "TP_ERR_INVALID_ARG";
+    case TP_ERR_SHAPE: return "TP_ERR_SHAPE";
+    case TP_ERR_UNSUPPORTED: return "TP_ERR_UNSUPPORTED";
+    case TP_ERR_WORKSPACE: return "TP_ERR_WORKSPACE";
+    case TP_ERR_CUDA: return "TP_ERR_CUDA";
+    case TP_ERR_TIMEOUT: return "TP_ERR_TIMEOUT";
+    default: return "TP_ERR_UNKNOWN";
+  }
+}
+
+tp_status tp_check_device_error(void* stream) {
+  cudaError_t e = cudaStreamSynchronize(static_cast<cudaStream_t>(stream));
+  if (e != cudaSuccess)
+    return tp::set_error(TP_ERR_CUDA, std::string("stream: ") + cudaGetErrorString(e));
+  uint32_t* w = tp::device_error_word();
+  if (!w) return tp::set_error(TP_ERR_CUDA, "device error word unavailable");
+  uint32_t v = 0;
+  e = cudaMemcpy(&v, w, sizeof(v), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess)
+    return tp::set_error(TP_ERR_CUDA, std::string("error word: ") + cudaGetErrorString(e));
+  if (v) {
+    const uint32_t zero = 0;
+    cudaMemcpy(w, &zero, sizeof(zero), cudaMemcpyHostToDevice);
+    return tp::set_error(TP_ERR_TIMEOUT,
+                         "a bounded device wait ran out (site bits " + std::to_string(v) + ")");
+  }
+  return TP_OK;
+}
+
+int32_t tp_tensor_core_path_available(void) { return tp::tensor_cores_usable() ? 1 : 0; }
+
+int32_t tp_version(void) { return 100; }  // 0.1.0
+
+}  // extern "C"

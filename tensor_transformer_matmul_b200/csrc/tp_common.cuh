@@ -1,0 +1,137 @@
+// Shared host/device helpers of libtpblock: status plumbing, the device error word, launch
+// accounting, bf16 conversions and the elementwise functions of the block.
+#pragma once
+
+#include <cuda_runtime.h>
+#include <cuda_bf16.h>
+#include <stdint.h>
+#include <stddef.h>
+#include <string>
+
+#include "tp_block.h"
+
+namespace tp {
+
+// ----------------------------------------------------------------------------------------------
+// host-side status helpers (defined in tp_abi.cu)
+// ----------------------------------------------------------------------------------------------
+tp_status set_error(tp_status st, const std::string& msg);
+void clear_error();
+void count_launch(uint64_t n = 1);
+void count_reduction();
+
+#define TP_CUDA_TRY(expr)                                                                       \
+  do {                                                                                          \
+    cudaError_t _e = (expr);                                                                    \
+    if (_e != cudaSuccess)                                                                      \
+      return ::tp::set_error(TP_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(_e));  \
+  } while (0)
+
+#define TP_LAUNCH_CHECK()                                                                       \
+  do {                                                                                          \
+    cudaError_t _e = cudaGetLastError();                                                        \
+    if (_e != cudaSuccess)                                                                      \
+      return ::tp::set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(_e)); \
+    ::tp::count_launch();                                                                       \
+  } while (0)
+
+inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
+inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
+inline size_t align256(size_t a) { return (a + 255) & ~size_t(255); }
+inline int elem_bytes(int dtype) { return dtype == TP_BF16 ? 2 : 4; }
+
+int num_sms();                    // SM count of the current device (cached per device)
+bool tensor_cores_usable();       // sm_100 device present
+
+// ----------------------------------------------------------------------------------------------
+// device error word: written by bounded waits that ran out, read by tp_check_device_error
+// ----------------------------------------------------------------------------------------------
+enum : uint32_t {
+  DEVERR_NONE = 0,
+  DEVERR_WAIT_FULL = 1u << 0,      // MMA warp waited too long for a TMA stage
+  DEVERR_WAIT_EMPTY = 1u << 1,     // producer waited too long for a free stage
+  DEVERR_WAIT_ACC_FULL = 1u << 2,  // epilogue waited too long for an accumulator
+  DEVERR_WAIT_ACC_EMPTY = 1u << 3, // MMA warp waited too long for the epilogue
+  DEVERR_WAIT_DRAIN = 1u << 4,     // abort path: in-flight copies did not land in time
+};
+
+// Device address of the error word of the current device (owned by tp_abi.cu).  Kernels get
+// it as a parameter; there is no cross-file device symbol.
+uint32_t* device_error_word();
+
+// Upper bound for a single device-side wait (nanoseconds of %globaltimer).
+constexpr uint64_t kWaitTimeoutNs = 2000000000ull;  // 2 s
+
+__device__ __forceinline__ uint64_t globaltimer_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
+  return t;
+}
+
+__device__ __forceinline__ void record_device_error(uint32_t* word, uint32_t bits) {
+  if (word) atomicOr(word, bits);
+}
+
+// ----------------------------------------------------------------------------------------------
+// element conversions
+// ----------------------------------------------------------------------------------------------
+template <typename T> struct Elem;
+template <> struct Elem<float> {
+  __device__ __forceinline__ static float load(const float* p) { return *p; }
+  __device__ __forceinline__ static float to_f(float v) { return v; }
+  __device__ __forceinline__ static float from_f(float v) { return v; }
+};
+template <> struct Elem<__nv_bfloat16> {
+  __device__ __forceinline__ static float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+  __device__ __forceinline__ static __nv_bfloat16 from_f(float v) { return __float2bfloat16_rn(v); }
+};
+
+__device__ __forceinline__ float to_f(float v) { return v; }
+__device__ __forceinline__ float to_f(__nv_bfloat16 v) { return __bfloat162float(v); }
+template <typename T> __device__ __forceinline__ T from_f(float v);
+template <> __device__ __forceinline__ float from_f<float>(float v) { return v; }
+template <> __device__ __forceinline__ __nv_bfloat16 from_f<__nv_bfloat16>(float v) {
+  return __float2bfloat16_rn(v);
+}
+
+// pack two floats into a bf16x2 word (low half = a)
+__device__ __forceinline__ uint32_t pack_bf16x2(float a, float b) {
+  __nv_bfloat162 v = __floats2bfloat162_rn(a, b);
+  return *reinterpret_cast<uint32_t*>(&v);
+}
+__device__ __forceinline__ float bf16lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16hi(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
+
+// ----------------------------------------------------------------------------------------------
+// the block's elementwise functions (CUDA's expf / erff are called, not re-derived)
+// ----------------------------------------------------------------------------------------------
+__device__ __forceinline__ float sigmoid_f(float z) { return 1.0f / (1.0f + expf(-z)); }
+__device__ __forceinline__ float silu_f(float z) { return z * sigmoid_f(z); }
+__device__ __forceinline__ float silu_grad_f(float z) {
+  float s = sigmoid_f(z);
+  return s * (1.0f + z * (1.0f - s));
+}
+__device__ __forceinline__ float gelu_f(float z) {
+  return 0.5f * z * (1.0f + erff(z * 0.70710678118654752440f));
+}
+__device__ __forceinline__ float gelu_grad_f(float z) {
+  float cdf = 0.5f * (1.0f + erff(z * 0.70710678118654752440f));
+  float pdf = 0.39894228040143267794f * expf(-0.5f * z * z);
+  return cdf + z * pdf;
+}
+__device__ __forceinline__ float act_f(int act, float z) {
+  switch (act) {
+    case TP_ACT_RELU: return z > 0.f ? z : 0.f;
+    case TP_ACT_GELU: return gelu_f(z);
+    default: return z;
+  }
+}
+__device__ __forceinline__ float act_grad_f(int act, float z) {
+  switch (act) {
+    case TP_ACT_RELU: return z > 0.f ? 1.f : 0.f;
+    case TP_ACT_GELU: return gelu_grad_f(z);
+    default: return 1.f;
+  }
+}
+
+}  // namespace tp

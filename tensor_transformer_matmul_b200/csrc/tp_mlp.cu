@@ -1,0 +1,451 @@
+// Tensor-parallel MLP block: packing, forward, backward.
+//
+// "How does tensor parallelism split a transformer feed-forward block's two matmuls across
+// devices?": column-parallel first matmul with the activation local to each shard, row-parallel
+// second matmul producing full-shape partial sums, one reduction; backward with per-shard weight
+// gradients and a reduced input gradient.  "Tensor Parallelism" (klaylearn), Notes: up/gate
+// projections sharded column-wise.
+//
+// All p shards live on this GPU.  Because x is replicated, the column-parallel matmuls of all
+// shards are one GEMM over the concatenated packed weights (their outputs are the column slices
+// h_i, laid side by side); the row-parallel matmul is a batched GEMM with one problem per shard,
+// each producing its own full-shape partial y_i; the partials are then summed in shard order.
+#include <algorithm>
+
+#include "gemm_launch.cuh"
+#include "pack.cuh"
+#include "reduce.cuh"
+#include "simt.cuh"
+#include "tp_common.cuh"
+
+namespace tp {
+namespace {
+
+using tc::Operand;
+using tc::TileCfg;
+
+constexpr int stages_for(int bn, int a_sub) {
+  return std::min(8, (200 * 1024) / (128 * a_sub * 64 * 2 + bn * 64 * 2));
+}
+
+struct MlpLayout {
+  int64_t T, d, F, Fs, Fsp, R;
+  int p, act, dtype, eb;
+  size_t w1p_bytes, w2p_bytes;
+  size_t saved_z_off, saved_h_off, saved_bytes;
+  size_t fz_off, fh_off, fpart_off, fwd_ws;
+  size_t bdh_off, bdz_off, bpart_off, bwd_ws;
+};
+
+tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
+  if (!desc) return set_error(TP_ERR_INVALID_ARG, "desc is null");
+  if (desc->T < 0) return set_error(TP_ERR_SHAPE, "T must be >= 0");
+  if (desc->d < 1 || desc->d_ff < 1) return set_error(TP_ERR_SHAPE, "d and d_ff must be >= 1");
+  if (desc->p < 1) return set_error(TP_ERR_SHAPE, "p must be >= 1");
+  if (desc->d_ff % desc->p) return set_error(TP_ERR_SHAPE, "p must divide d_ff");
+  if (desc->act < TP_ACT_IDENTITY || desc->act > TP_ACT_SWIGLU)
+    return set_error(TP_ERR_INVALID_ARG, "unknown activation");
+  if (desc->dtype != TP_F32 && desc->dtype != TP_BF16)
+    return set_error(TP_ERR_INVALID_ARG, "dtype must be TP_F32 or TP_BF16");
+  if (desc->reduce_mode != TP_REDUCE_SEPARATE && desc->reduce_mode != TP_REDUCE_FUSED)
+    return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
+  L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
+  L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
+  L->Fs = L->F / L->p;
+  L->Fsp = round_up(L->Fs, 128);
+  L->R = (L->act == TP_ACT_SWIGLU) ? 2 * L->Fsp : L->Fsp;
+  const int64_t P = L->p;
+  L->w1p_bytes = static_cast<size_t>(P * L->R * L->d) * L->eb;
+  L->w2p_bytes = static_cast<size_t>(P * L->d * L->Fsp) * L->eb;
+  const size_t zb = static_cast<size_t>(L->T * P * L->R) * L->eb;
+  const size_t hb = static_cast<size_t>(L->T * P * L->Fsp) * L->eb;
+  const size_t partb = static_cast<size_t>(P * L->T * L->d) * 4;
+  L->saved_z_off = 0;
+  L->saved_h_off = align256(zb);
+  L->saved_bytes = L->saved_h_off + align256(hb);
+  L->fz_off = 0;
+  L->fh_off = align256(zb);
+  L->fpart_off = L->fh_off + align256(hb);
+  L->fwd_ws = L->fpart_off + align256(partb);
+  const size_t dhb = static_cast<size_t>(L->T * P * L->Fsp) * 4;
+  L->bdh_off = 0;
+  L->bdz_off = align256(dhb);
+  L->bpart_off = L->bdz_off + align256(zb);
+  L->bwd_ws = L->bpart_off + align256(partb);
+  return TP_OK;
+}
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
+
+bool use_tensor_cores(const MlpLayout& L) {
+  return L.dtype == TP_BF16 && (L.d % 8 == 0) && tensor_cores_usable();
+}
+
+uint8_t* off(void* base, size_t o) { return static_cast<uint8_t*>(base) + o; }
+
+// ------------------------------------------------------------------------------ tensor cores
+template <int BN, int ASUB>
+using KK = TileCfg<BN, ASUB, false, false, stages_for(BN, ASUB)>;
+
+tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, void* z,
+                cudaStream_t s) {
+  const int64_t rows = L.p * L.R;
+  tc::EpiHidden::Params ep;
+  ep.h = static_cast<__nv_bfloat16*>(h);
+  ep.z = static_cast<__nv_bfloat16*>(z);
+  ep.ld_h = L.p * L.Fsp;
+  ep.ld_z = L.p * L.R;
+  ep.tokens = static_cast<int32_t>(L.T);
+  ep.rows = static_cast<int32_t>(rows);
+  ep.act = L.act;
+  const bool swiglu = L.act == TP_ACT_SWIGLU;
+  const Operand xo{x, false, L.T, L.d, 1, L.d, 0};
+  const Operand wo{w1p, false, rows, L.d, 1, L.d, 0};
+  if (L.T <= 128) {
+    ep.swap = 1;
+    if (swiglu) {
+      if (L.T <= 16) return tc::run_gemm<KK<16, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+      if (L.T <= 64) return tc::run_gemm<KK<64, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+      return tc::run_gemm<KK<128, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+    }
+    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+  }
+  ep.swap = 0;
+  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s);
+}
+
+// partial[i] = h_i W2_i  (fp32, [p][T][d])
+tp_status tc_down_partials(const MlpLayout& L, const void* h, const void* w2p, float* part,
+                           cudaStream_t s) {
+  const Operand ho{h, false, L.T, L.Fsp, L.p, L.p * L.Fsp, L.Fsp};
+  const Operand wo{w2p, false, L.d, L.Fsp, L.p, L.Fsp, L.d * L.Fsp};
+  tc::EpiStoreF32::Params ep;
+  ep.out = part;
+  ep.ld = L.d;
+  ep.batch_stride = L.T * L.d;
+  ep.rows_valid = static_cast<int32_t>(L.T);
+  ep.cols_valid = static_cast<int32_t>(L.d);
+  if (L.T <= 128) {
+    ep.swap = 1;
+    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
+    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
+    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
+  }
+  ep.swap = 0;
+  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s);
+}
+
+tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
+                      const void* h, const void* w1p, const void* w2p, void* dz, float* dw1p,
+                      float* dw2p, float* part, cudaStream_t s) {
+  const int64_t P = L.p;
+  tp_status st;
+  // (1) dH_i = dY W2_i^T with the activation backward fused: dz in w1p row order
+  {
+    const Operand a{dy, false, L.T, L.d, 1, L.d, 0};
+    const Operand b{w2p, true, L.Fsp, L.d, P, L.Fsp, L.d * L.Fsp};
+    tc::EpiActBwd::Params ep;
+    ep.z = static_cast<const __nv_bfloat16*>(z);
+    ep.dz = static_cast<__nv_bfloat16*>(dz);
+    ep.ld = P * L.R;
+    ep.R = static_cast<int32_t>(L.R);
+    ep.tokens = static_cast<int32_t>(L.T);
+    ep.act = L.act;
+    if (L.Fsp % 256 == 0)
+      st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiActBwd>(
+          a, b, L.T, L.Fsp, L.d, P, ep, s);
+    else
+      st = tc::run_gemm<TileCfg<128, 1, false, true, stages_for(128, 1)>, tc::EpiActBwd>(
+          a, b, L.T, L.Fsp, L.d, P, ep, s);
+    if (st != TP_OK) return st;
+  }
+  // (2) dW2_i[n][c] = sum_t dY[t][n] h_i[t][c]   (no exchange between shards)
+  {
+    const Operand a{dy, true, L.d, L.T, 1, L.d, 0};
+    const Operand b{h, true, L.Fsp, L.T, P, P * L.Fsp, L.Fsp};
+    tc::EpiStoreF32::Params ep;
+    ep.out = dw2p;
+    ep.ld = L.Fsp;
+    ep.batch_stride = L.d * L.Fsp;
+    ep.rows_valid = static_cast<int32_t>(L.d);
+    ep.cols_valid = static_cast<int32_t>(L.Fsp);
+    ep.swap = 0;
+    if (L.Fsp % 256 == 0)
+      st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
+          a, b, L.d, L.Fsp, L.T, P, ep, s);
+    else
+      st = tc::run_gemm<TileCfg<128, 1, true, true, stages_for(128, 1)>, tc::EpiStoreF32>(
+          a, b, L.d, L.Fsp, L.T, P, ep, s);
+    if (st != TP_OK) return st;
+  }
+  // (3) dW1_i[r][k] = sum_t dz_i[t][r] x[t][k]   (no exchange between shards)
+  {
+    const Operand a{dz, true, L.R, L.T, P, P * L.R, L.R};
+    const Operand b{x, true, L.d, L.T, 1, L.d, 0};
+    tc::EpiStoreF32::Params ep;
+    ep.out = dw1p;
+    ep.ld = L.d;
+    ep.batch_stride = L.R * L.d;
+    ep.rows_valid = static_cast<int32_t>(L.R);
+    ep.cols_valid = static_cast<int32_t>(L.d);
+    ep.swap = 0;
+    st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
+        a, b, L.R, L.d, L.T, P, ep, s);
+    if (st != TP_OK) return st;
+  }
+  // (4) dx_i = dz_i W1_i^T  (partials, summed by the caller)
+  {
+    const Operand a{dz, false, L.T, L.R, P, P * L.R, L.R};
+    const Operand b{w1p, true, L.d, L.R, P, L.d, L.R * L.d};
+    tc::EpiStoreF32::Params ep;
+    ep.out = part;
+    ep.ld = L.d;
+    ep.batch_stride = L.T * L.d;
+    ep.rows_valid = static_cast<int32_t>(L.T);
+    ep.cols_valid = static_cast<int32_t>(L.d);
+    ep.swap = 0;
+    st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiStoreF32>(
+        a, b, L.T, L.d, L.R, P, ep, s);
+  }
+  return st;
+}
+
+// ------------------------------------------------------------------------------ SIMT path
+template <typename T>
+tp_status simt_forward(const MlpLayout& L, const void* x, const void* w1p, const void* w2p,
+                       void* z, void* h, float* part, cudaStream_t s) {
+  const int64_t P = L.p;
+  simt::GemmArgs g{};
+  g.a = x; g.a_bs = 0; g.a_sm = L.d; g.a_sk = 1;
+  g.b = w1p; g.b_bs = 0; g.b_sm = L.d; g.b_sk = 1;
+  g.out = z; g.o_bs = 0; g.o_sm = P * L.R; g.o_sn = 1;
+  g.M = L.T; g.N = P * L.R; g.K = L.d; g.batch = 1; g.out_f32 = 0;
+  tp_status st = simt::gemm<T>(g, s);
+  if (st != TP_OK) return st;
+  const int64_t total = L.T * P * L.Fsp;
+  simt::act_fwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
+      static_cast<const T*>(z), static_cast<T*>(h), L.T, L.p, L.R, L.Fsp, L.act);
+  TP_LAUNCH_CHECK();
+  simt::GemmArgs g2{};
+  g2.a = h; g2.a_bs = L.Fsp; g2.a_sm = P * L.Fsp; g2.a_sk = 1;
+  g2.b = w2p; g2.b_bs = L.d * L.Fsp; g2.b_sm = L.Fsp; g2.b_sk = 1;
+  g2.out = part; g2.o_bs = L.T * L.d; g2.o_sm = L.d; g2.o_sn = 1;
+  g2.M = L.T; g2.N = L.d; g2.K = L.Fsp; g2.batch = P; g2.out_f32 = 1;
+  return simt::gemm<T>(g2, s);
+}
+
+template <typename T>
+tp_status simt_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
+                        const void* h, const void* w1p, const void* w2p, float* dh, void* dz,
+                        float* dw1p, float* dw2p, float* part, cudaStream_t s) {
+  const int64_t P = L.p;
+  tp_status st;
+  simt::GemmArgs g{};
+  // dH_i[t][c] = sum_n dY[t][n] w2p[i][n][c]
+  g.a = dy; g.a_bs = 0; g.a_sm = L.d; g.a_sk = 1;
+  g.b = w2p; g.b_bs = L.d * L.Fsp; g.b_sm = 1; g.b_sk = L.Fsp;
+  g.out = dh; g.o_bs = L.Fsp; g.o_sm = P * L.Fsp; g.o_sn = 1;
+  g.M = L.T; g.N = L.Fsp; g.K = L.d; g.batch = P; g.out_f32 = 1;
+  if ((st = simt::gemm<T>(g, s)) != TP_OK) return st;
+  const int64_t total = L.T * P * L.Fsp;
+  simt::act_bwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
+      dh, static_cast<const T*>(z), static_cast<T*>(dz), L.T, L.p, L.R, L.Fsp, L.act);
+  TP_LAUNCH_CHECK();
+  // dW2_i[n][c] = sum_t dY[t][n] h[t][i*Fsp + c]
+  g = simt::GemmArgs{};
+  g.a = dy; g.a_bs = 0; g.a_sm = 1; g.a_sk = L.d;
+  g.b = h; g.b_bs = L.Fsp; g.b_sm = 1; g.b_sk = P * L.Fsp;
+  g.out = dw2p; g.o_bs = L.d * L.Fsp; g.o_sm = L.Fsp; g.o_sn = 1;
+  g.M = L.d; g.N = L.Fsp; g.K = L.T; g.batch = P; g.out_f32 = 1;
+  if ((st = simt::gemm<T>(g, s)) != TP_OK) return st;
+  // dW1_i[r][k] = sum_t dz[t][i*R + r] x[t][k]
+  g = simt::GemmArgs{};
+  g.a = dz; g.a_bs = L.R; g.a_sm = 1; g.a_sk = P * L.R;
+  g.b = x; g.b_bs = 0; g.b_sm = 1; g.b_sk = L.d;
+  g.out = dw1p; g.o_bs = L.R * L.d; g.o_sm = L.d; g.o_sn = 1;
+  g.M = L.R; g.N = L.d; g.K = L.T; g.batch = P; g.out_f32 = 1;
+  if ((st = simt::gemm<T>(g, s)) != TP_OK) return st;
+  // dx_i[t][k] = sum_r dz[t][i*R + r] w1p[i][r][k]
+  g = simt::GemmArgs{};
+  g.a = dz; g.a_bs = L.R; g.a_sm = P * L.R; g.a_sk = 1;
+  g.b = w1p; g.b_bs = L.R * L.d; g.b_sm = 1; g.b_sk = L.d;
+  g.out = part; g.o_bs = L.T * L.d; g.o_sm = L.d; g.o_sn = 1;
+  g.M = L.T; g.N = L.d; g.K = L.R; g.batch = P; g.out_f32 = 1;
+  return simt::gemm<T>(g, s);
+}
+
+pack::ColMap w1_colmap(const MlpLayout& L, const void* w1, const void* wu) {
+  pack::ColMap cm{};
+  cm.kind = L.act == TP_ACT_SWIGLU ? 1 : 0;
+  cm.R = L.R;
+  cm.F_s = L.Fs;
+  cm.src[0] = w1; cm.src[1] = wu; cm.src[2] = nullptr;
+  cm.ld[0] = L.F; cm.ld[1] = L.F; cm.ld[2] = 0;
+  return cm;
+}
+
+template <typename T>
+tp_status pack_t(const MlpLayout& L, const void* w1, const void* wu, const void* w2, void* w1p,
+                 void* w2p, cudaStream_t s) {
+  const int64_t rows = L.p * L.R;
+  dim3 blk(32, 8);
+  dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.d, 32)), 1);
+  if (!pack::grid_ok(g1.x, g1.y, 1)) return set_error(TP_ERR_UNSUPPORTED, "pack grid too large");
+  pack::pack_cols_kernel<T><<<g1, blk, 0, s>>>(static_cast<T*>(w1p), rows, L.d, w1_colmap(L, w1, wu));
+  TP_LAUNCH_CHECK();
+  dim3 g2(static_cast<unsigned>(ceil_div(L.d, 32)), static_cast<unsigned>(ceil_div(L.Fsp, 32)),
+          static_cast<unsigned>(L.p));
+  if (!pack::grid_ok(g2.x, g2.y, g2.z)) return set_error(TP_ERR_UNSUPPORTED, "pack grid too large");
+  pack::pack_rows_kernel<T><<<g2, blk, 0, s>>>(static_cast<T*>(w2p), L.p, L.d, L.Fsp, L.Fs,
+                                               static_cast<const T*>(w2), L.d);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+}  // namespace
+}  // namespace tp
+
+using namespace tp;
+
+extern "C" size_t tp_mlp_w1_packed_bytes(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  return layout_of(desc, &L) == TP_OK ? L.w1p_bytes : 0;
+}
+extern "C" size_t tp_mlp_w2_packed_bytes(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  return layout_of(desc, &L) == TP_OK ? L.w2p_bytes : 0;
+}
+extern "C" size_t tp_mlp_saved_bytes(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  return layout_of(desc, &L) == TP_OK ? L.saved_bytes : 0;
+}
+extern "C" size_t tp_mlp_fwd_workspace(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  return layout_of(desc, &L) == TP_OK ? L.fwd_ws : 0;
+}
+extern "C" size_t tp_mlp_bwd_workspace(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  return layout_of(desc, &L) == TP_OK ? L.bwd_ws : 0;
+}
+
+extern "C" tp_status tp_mlp_pack(const tp_mlp_desc* desc, const void* w1, const void* w_up,
+                                 const void* w2, void* w1p, void* w2p, void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (!w1 || !w2 || !w1p || !w2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if ((L.act == TP_ACT_SWIGLU) != (w_up != nullptr))
+    return set_error(TP_ERR_INVALID_ARG, "w_up must be given exactly for TP_ACT_SWIGLU");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return L.dtype == TP_BF16 ? pack_t<__nv_bfloat16>(L, w1, w_up, w2, w1p, w2p, s)
+                            : pack_t<float>(L, w1, w_up, w2, w1p, w2p, s);
+}
+
+extern "C" tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw1p,
+                                         const void* dw2p, void* dw1, void* dw_up, void* dw2,
+                                         void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (!dw1p || !dw2p || !dw1 || !dw2) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if ((L.act == TP_ACT_SWIGLU) != (dw_up != nullptr))
+    return set_error(TP_ERR_INVALID_ARG, "dw_up must be given exactly for TP_ACT_SWIGLU");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const int64_t rows = L.p * L.R;
+  dim3 blk(32, 8);
+  dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.d, 32)), 1);
+  pack::unpack_cols_kernel<<<g1, blk, 0, s>>>(static_cast<const float*>(dw1p), rows, L.d,
+                                               w1_colmap(L, dw1, dw_up), static_cast<float*>(dw1),
+                                               static_cast<float*>(dw_up));
+  TP_LAUNCH_CHECK();
+  dim3 g2(static_cast<unsigned>(ceil_div(L.d, 32)), static_cast<unsigned>(ceil_div(L.Fsp, 32)),
+          static_cast<unsigned>(L.p));
+  pack::unpack_rows_kernel<<<g2, blk, 0, s>>>(static_cast<const float*>(dw2p), L.p, L.d, L.Fsp,
+                                               L.Fs, static_cast<float*>(dw2), L.d);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p,
+                                const void* w2p, const void* residual, void* y, void* saved,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (desc->reduce_mode == TP_REDUCE_FUSED)
+    return set_error(TP_ERR_UNSUPPORTED, "TP_REDUCE_FUSED is not available for tp_mlp_fwd");
+  if (L.T == 0) {
+    count_reduction();
+    return TP_OK;
+  }
+  if (!x || !w1p || !w2p || !y) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < L.fwd_ws) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* z = saved ? off(saved, L.saved_z_off) : off(workspace, L.fz_off);
+  void* h = saved ? off(saved, L.saved_h_off) : off(workspace, L.fh_off);
+  float* part = reinterpret_cast<float*>(off(workspace, L.fpart_off));
+  if (use_tensor_cores(L)) {
+    for (const void* q : {x, w1p, w2p, residual, static_cast<const void*>(y),
+                          static_cast<const void*>(saved)})
+      if (q && !aligned16(q))
+        return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, s)) != TP_OK) return st;
+    if ((st = tc_down_partials(L, h, w2p, part, s)) != TP_OK) return st;
+  } else if (L.dtype == TP_BF16) {
+    if ((st = simt_forward<__nv_bfloat16>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
+  } else {
+    if ((st = simt_forward<float>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
+  }
+  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.dtype, s);
+  if (st == TP_OK) count_reduction();
+  return st;
+}
+
+extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const void* x,
+                                const void* saved, const void* w1p, const void* w2p, void* dx,
+                                void* dw1p, void* dw2p, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (desc->reduce_mode == TP_REDUCE_FUSED)
+    return set_error(TP_ERR_UNSUPPORTED, "TP_REDUCE_FUSED is not available for tp_mlp_bwd");
+  if (!w1p || !w2p || !dw1p || !dw2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L.T == 0) {  // no tokens: zero weight gradients, nothing else
+    TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(L.p * L.R * L.d) * 4, s));
+    TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(L.p * L.d * L.Fsp) * 4, s));
+    count_reduction();
+    return TP_OK;
+  }
+  if (!dy || !x || !saved || !dx) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < L.bwd_ws) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  const void* z = static_cast<const uint8_t*>(saved) + L.saved_z_off;
+  const void* h = static_cast<const uint8_t*>(saved) + L.saved_h_off;
+  float* dh = reinterpret_cast<float*>(off(workspace, L.bdh_off));
+  void* dz = off(workspace, L.bdz_off);
+  float* part = reinterpret_cast<float*>(off(workspace, L.bpart_off));
+  float* g1 = static_cast<float*>(dw1p);
+  float* g2 = static_cast<float*>(dw2p);
+  if (use_tensor_cores(L)) {
+    for (const void* q : {dy, x, saved, w1p, w2p, static_cast<const void*>(dx)})
+      if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, s);
+  } else if (L.dtype == TP_BF16) {
+    st = simt_backward<__nv_bfloat16>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
+  } else {
+    st = simt_backward<float>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
+  }
+  if (st != TP_OK) return st;
+  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, nullptr, dx, L.dtype, s);
+  if (st == TP_OK) count_reduction();
+  return st;
+}

@@ -1,0 +1,251 @@
+"""Python binding of libtpblock (ctypes): the C-ABI calls under the same names.
+
+Argument marshalling only: tensors are passed as device pointers with the current torch CUDA
+stream; every step of the block runs in the library's CUDA kernels.  There is no fallback: if the
+library is missing or a call fails, a ``TpError`` is raised.  The C declarations, layouts and
+error behaviour are documented in ``include/tp_block.h``.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libtpblock.so")
+
+TP_OK, TP_ERR_INVALID_ARG, TP_ERR_SHAPE, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA, \
+    TP_ERR_TIMEOUT = range(7)
+TP_F32, TP_BF16 = 0, 1
+ACT = {"identity": 0, "relu": 1, "gelu": 2, "swiglu": 3}
+DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
+TORCH_OF = {TP_F32: torch.float32, TP_BF16: torch.bfloat16}
+TP_REDUCE_SEPARATE, TP_REDUCE_FUSED = 0, 1
+
+# every symbol the header declares
+EXPORTS = (
+    "tp_mlp_w1_packed_bytes", "tp_mlp_w2_packed_bytes", "tp_mlp_pack", "tp_mlp_saved_bytes",
+    "tp_mlp_fwd_workspace", "tp_mlp_fwd", "tp_mlp_bwd_workspace", "tp_mlp_bwd",
+    "tp_mlp_unpack_grads", "tp_attn_wqkv_packed_bytes", "tp_attn_wo_packed_bytes",
+    "tp_attn_pack", "tp_attn_fwd_workspace", "tp_attn_fwd", "tp_reduce_partials", "tp_rmsnorm",
+    "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
+    "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
+)
+
+
+class TpError(RuntimeError):
+    def __init__(self, status, msg):
+        super().__init__(f"{_status_name(status)}: {msg}")
+        self.status = status
+
+
+class tp_mlp_desc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("d_ff", ctypes.c_int64),
+                ("p", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("reduce_mode", ctypes.c_int32)]
+
+
+class tp_attn_desc(ctypes.Structure):
+    _fields_ = [("b", ctypes.c_int64), ("s", ctypes.c_int64), ("h", ctypes.c_int64),
+                ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
+                ("p", ctypes.c_int32), ("causal", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("kv_len", ctypes.c_int64), ("kv_cap", ctypes.c_int64),
+                ("reduce_mode", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+_lib = None
+
+
+def load():
+    """Load libtpblock.so (fails loudly if it was not built)."""
+    global _lib
+    if _lib is not None:
+        return _lib
+    if not os.path.exists(LIB_PATH):
+        raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                           "`python -m tensor_transformer_matmul_b200.build`")
+    lib = ctypes.CDLL(LIB_PATH)
+    P, S, I32, I64, F32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
+    MD, AD = ctypes.POINTER(tp_mlp_desc), ctypes.POINTER(tp_attn_desc)
+    sig = {
+        "tp_mlp_w1_packed_bytes": (S, [MD]), "tp_mlp_w2_packed_bytes": (S, [MD]),
+        "tp_mlp_pack": (I32, [MD, P, P, P, P, P, P]), "tp_mlp_saved_bytes": (S, [MD]),
+        "tp_mlp_fwd_workspace": (S, [MD]),
+        "tp_mlp_fwd": (I32, [MD, P, P, P, P, P, P, P, S, P]),
+        "tp_mlp_bwd_workspace": (S, [MD]),
+        "tp_mlp_bwd": (I32, [MD, P, P, P, P, P, P, P, P, P, S, P]),
+        "tp_mlp_unpack_grads": (I32, [MD, P, P, P, P, P, P]),
+        "tp_attn_wqkv_packed_bytes": (S, [AD]), "tp_attn_wo_packed_bytes": (S, [AD]),
+        "tp_attn_pack": (I32, [AD, P, P, P, P, P, P, P]), "tp_attn_fwd_workspace": (S, [AD]),
+        "tp_attn_fwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
+        "tp_reduce_partials": (I32, [P, I32, I64, I32, P, P, I32, P]),
+        "tp_rmsnorm": (I32, [P, I64, I64, F32, P, I32, P]),
+        "tp_reduction_count": (ctypes.c_uint64, []), "tp_reset_reduction_count": (None, []),
+        "tp_launch_count": (ctypes.c_uint64, []), "tp_last_error": (ctypes.c_char_p, []),
+        "tp_status_string": (ctypes.c_char_p, [I32]), "tp_check_device_error": (I32, [P]),
+        "tp_tensor_core_path_available": (I32, []), "tp_version": (I32, []),
+    }
+    for name, (res, args) in sig.items():
+        fn = getattr(lib, name)
+        fn.restype = res
+        fn.argtypes = args
+    _lib = lib
+    return lib
+
+
+def _status_name(st):
+    try:
+        return load().tp_status_string(st).decode()
+    except Exception:  # pragma: no cover
+        return f"status {st}"
+
+
+def _check(st):
+    if st != TP_OK:
+        raise TpError(st, load().tp_last_error().decode())
+
+
+def _ptr(t):
+    if t is None:
+        return None
+    if not isinstance(t, torch.Tensor):
+        raise TypeError("expected a torch.Tensor")
+    if t.numel() > 0 and not t.is_cuda:
+        raise ValueError("tensor must live on the GPU")
+    if not t.is_contiguous():
+        raise ValueError("tensor must be contiguous")
+    return t.data_ptr() if t.numel() > 0 else None
+
+
+def _stream(stream):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _nbytes(t):
+    return 0 if t is None else t.numel() * t.element_size()
+
+
+# ------------------------------------------------------------------------------------ MLP
+def mlp_desc(T, d, d_ff, p, act="swiglu", dtype="bf16", reduce_mode=TP_REDUCE_SEPARATE):
+    return tp_mlp_desc(int(T), int(d), int(d_ff), int(p), ACT[act] if isinstance(act, str) else int(act),
+                       DTYPE[dtype] if isinstance(dtype, str) else int(dtype), int(reduce_mode))
+
+
+def tp_mlp_w1_packed_bytes(desc):
+    return load().tp_mlp_w1_packed_bytes(ctypes.byref(desc))
+
+
+def tp_mlp_w2_packed_bytes(desc):
+    return load().tp_mlp_w2_packed_bytes(ctypes.byref(desc))
+
+
+def tp_mlp_saved_bytes(desc):
+    return load().tp_mlp_saved_bytes(ctypes.byref(desc))
+
+
+def tp_mlp_fwd_workspace(desc):
+    return load().tp_mlp_fwd_workspace(ctypes.byref(desc))
+
+
+def tp_mlp_bwd_workspace(desc):
+    return load().tp_mlp_bwd_workspace(ctypes.byref(desc))
+
+
+def tp_mlp_pack(desc, w1, w_up, w2, w1p, w2p, stream=None):
+    _check(load().tp_mlp_pack(ctypes.byref(desc), _ptr(w1), _ptr(w_up), _ptr(w2), _ptr(w1p),
+                              _ptr(w2p), _stream(stream)))
+
+
+def tp_mlp_fwd(desc, x, w1p, w2p, y, residual=None, saved=None, workspace=None, stream=None):
+    _check(load().tp_mlp_fwd(ctypes.byref(desc), _ptr(x), _ptr(w1p), _ptr(w2p), _ptr(residual),
+                             _ptr(y), _ptr(saved), _ptr(workspace), _nbytes(workspace),
+                             _stream(stream)))
+
+
+def tp_mlp_bwd(desc, dy, x, saved, w1p, w2p, dx, dw1p, dw2p, workspace=None, stream=None):
+    _check(load().tp_mlp_bwd(ctypes.byref(desc), _ptr(dy), _ptr(x), _ptr(saved), _ptr(w1p),
+                             _ptr(w2p), _ptr(dx), _ptr(dw1p), _ptr(dw2p), _ptr(workspace),
+                             _nbytes(workspace), _stream(stream)))
+
+
+def tp_mlp_unpack_grads(desc, dw1p, dw2p, dw1, dw_up, dw2, stream=None):
+    _check(load().tp_mlp_unpack_grads(ctypes.byref(desc), _ptr(dw1p), _ptr(dw2p), _ptr(dw1),
+                                      _ptr(dw_up), _ptr(dw2), _stream(stream)))
+
+
+# ------------------------------------------------------------------------------ attention
+def attn_desc(b, s, h, n_q, n_kv, head_dim, p, causal=True, dtype="bf16", kv_len=0, kv_cap=0,
+              reduce_mode=TP_REDUCE_SEPARATE):
+    return tp_attn_desc(int(b), int(s), int(h), int(n_q), int(n_kv), int(head_dim), int(p),
+                        int(bool(causal)), DTYPE[dtype] if isinstance(dtype, str) else int(dtype),
+                        int(kv_len), int(kv_cap), int(reduce_mode), 0)
+
+
+def tp_attn_wqkv_packed_bytes(desc):
+    return load().tp_attn_wqkv_packed_bytes(ctypes.byref(desc))
+
+
+def tp_attn_wo_packed_bytes(desc):
+    return load().tp_attn_wo_packed_bytes(ctypes.byref(desc))
+
+
+def tp_attn_fwd_workspace(desc):
+    return load().tp_attn_fwd_workspace(ctypes.byref(desc))
+
+
+def tp_attn_pack(desc, wq, wk, wv, wo, wqkv_p, wo_p, stream=None):
+    _check(load().tp_attn_pack(ctypes.byref(desc), _ptr(wq), _ptr(wk), _ptr(wv), _ptr(wo),
+                               _ptr(wqkv_p), _ptr(wo_p), _stream(stream)))
+
+
+def tp_attn_fwd(desc, x, wqkv_p, wo_p, y, k_cache=None, v_cache=None, residual=None,
+                workspace=None, stream=None):
+    _check(load().tp_attn_fwd(ctypes.byref(desc), _ptr(x), _ptr(wqkv_p), _ptr(wo_p),
+                              _ptr(k_cache), _ptr(v_cache), _ptr(residual), _ptr(y),
+                              _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------------------------- reduce and glue
+def tp_reduce_partials(partials, p, n, out, residual=None, stream=None):
+    in_t = TP_BF16 if partials.dtype == torch.bfloat16 else TP_F32
+    out_t = TP_BF16 if out.dtype == torch.bfloat16 else TP_F32
+    _check(load().tp_reduce_partials(_ptr(partials), int(p), int(n), in_t, _ptr(residual),
+                                     _ptr(out), out_t, _stream(stream)))
+
+
+def tp_rmsnorm(x, out, eps=1e-5, stream=None):
+    dt = TP_BF16 if x.dtype == torch.bfloat16 else TP_F32
+    rows = x.numel() // x.shape[-1] if x.numel() else 0
+    _check(load().tp_rmsnorm(_ptr(x), int(rows), int(x.shape[-1]), float(eps), _ptr(out), dt,
+                             _stream(stream)))
+
+
+# ------------------------------------------------------------------------------ diagnostics
+def tp_reduction_count():
+    return load().tp_reduction_count()
+
+
+def tp_reset_reduction_count():
+    load().tp_reset_reduction_count()
+
+
+def tp_launch_count():
+    return load().tp_launch_count()
+
+
+def tp_last_error():
+    return load().tp_last_error().decode()
+
+
+def tp_check_device_error(stream=None):
+    _check(load().tp_check_device_error(_stream(stream)))
+
+
+def tp_tensor_core_path_available():
+    return bool(load().tp_tensor_core_path_available())
+
+
+def tp_version():
+    return load().tp_version()

@@ -1,0 +1,136 @@
+"""The C-ABI library without a GPU: it builds, loads, exports every declared symbol, and its
+host-side logic (layout queries, argument validation, status strings) behaves as documented.
+No kernel is launched here."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "tp_block.h")
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"^\s*(?:const\s+)?[A-Za-z_][A-Za-z0-9_]*\s*\*?\s+(tp_[a-z0-9_]+)\s*\(",
+                       src, flags=re.M)
+    return sorted(set(names))
+
+
+def test_header_declares_the_boundary():
+    names = _declared_functions()
+    for required in ("tp_mlp_fwd", "tp_mlp_bwd", "tp_attn_fwd", "tp_reduce_partials"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    so = lib.load()
+    for name in _declared_functions():
+        assert hasattr(so, name), name
+    assert set(_declared_functions()) == set(lib.EXPORTS)
+
+
+def test_version_and_status_strings(lib):
+    assert lib.tp_version() >= 100
+    so = lib.load()
+    assert so.tp_status_string(0) == b"TP_OK"
+    assert so.tp_status_string(2) == b"TP_ERR_SHAPE"
+    assert so.tp_status_string(6) == b"TP_ERR_TIMEOUT"
+
+
+def test_mlp_layout_sizes(lib):
+    # decode MLP shape: T=64, d=8192, d_ff=28672, p=8, SwiGLU, bf16
+    d = lib.mlp_desc(64, 8192, 28672, 8, "swiglu", "bf16")
+    fs = 28672 // 8
+    assert lib.tp_mlp_w1_packed_bytes(d) == 8 * 2 * fs * 8192 * 2
+    assert lib.tp_mlp_w2_packed_bytes(d) == 8 * 8192 * fs * 2
+    # weights total 1,409,286,144 bytes (3 matrices of 8192 x 28672 bf16)
+    assert lib.tp_mlp_w1_packed_bytes(d) + lib.tp_mlp_w2_packed_bytes(d) == 1_409_286_144
+    # padding: F_s = 8 pads to 128 per shard
+    t = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32")
+    assert lib.tp_mlp_w1_packed_bytes(t) == 4 * 128 * 8 * 4
+    assert lib.tp_mlp_w2_packed_bytes(t) == 4 * 8 * 128 * 4
+    assert lib.tp_mlp_saved_bytes(t) >= (4 * 4 * 128 + 4 * 4 * 128) * 4
+    assert lib.tp_mlp_fwd_workspace(t) >= 4 * 4 * 8 * 4
+    assert lib.tp_mlp_bwd_workspace(t) >= 4 * 4 * 8 * 4
+
+
+def test_attn_layout_sizes(lib):
+    a = lib.attn_desc(1, 2048, 8192, 64, 8, 128, 8)
+    assert lib.tp_attn_wqkv_packed_bytes(a) == 8 * (1024 + 128 + 128) * 8192 * 2
+    assert lib.tp_attn_wo_packed_bytes(a) == 8 * 8192 * 1024 * 2
+    assert lib.tp_attn_fwd_workspace(a) > 0
+
+
+@pytest.mark.parametrize("T,d,F,p,status", [
+    (4, 8, 30, 4, "TP_ERR_SHAPE"),     # p does not divide d_ff
+    (4, 8, 32, 0, "TP_ERR_SHAPE"),     # p < 1
+    (-1, 8, 32, 4, "TP_ERR_SHAPE"),    # negative T
+    (4, 0, 32, 4, "TP_ERR_SHAPE"),     # d < 1
+])
+def test_mlp_shape_errors(lib, T, d, F, p, status):
+    desc = lib.mlp_desc(T, d, F, p, "gelu", "f32")
+    so = lib.load()
+    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None)
+    assert so.tp_status_string(st).decode() == status
+    assert lib.tp_mlp_fwd_workspace(desc) == 0
+    assert lib.tp_last_error() != ""
+
+
+def test_mlp_argument_errors(lib):
+    so = lib.load()
+    desc = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32")
+    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None)
+    assert st == lib.TP_ERR_INVALID_ARG  # null x
+    fake = ctypes.c_void_p(0x1000)
+    st = so.tp_mlp_fwd(ctypes.byref(desc), fake, fake, fake, None, fake, None, fake, 16, None)
+    assert st == lib.TP_ERR_WORKSPACE
+    bad = lib.mlp_desc(4, 8, 32, 4, 9, "f32")
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+                         None) == lib.TP_ERR_INVALID_ARG
+    bad = lib.mlp_desc(4, 8, 32, 4, "gelu", 7)
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+                         None) == lib.TP_ERR_INVALID_ARG
+    # SwiGLU needs w_up; the other activations must not get one
+    sw = lib.mlp_desc(4, 8, 32, 4, "swiglu", "f32")
+    assert so.tp_mlp_pack(ctypes.byref(sw), fake, None, fake, fake, fake, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_mlp_pack(ctypes.byref(desc), fake, fake, fake, fake, fake, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None) != 0
+
+
+def test_attn_shape_errors(lib):
+    so = lib.load()
+    fake = ctypes.c_void_p(0x1000)
+
+    def st(desc):
+        return so.tp_attn_fwd(ctypes.byref(desc), fake, fake, fake, None, None, None, fake, fake,
+                              1 << 40, None)
+    # "Tensor Parallelism", Notes: with 8 KV heads, p = 16 cannot give every rank a whole KV head
+    assert st(lib.attn_desc(1, 4, 64, 16, 8, 8, 16)) == lib.TP_ERR_SHAPE
+    assert st(lib.attn_desc(1, 4, 64, 8, 3, 8, 1)) == lib.TP_ERR_SHAPE     # n_kv does not divide n_q
+    assert st(lib.attn_desc(1, 4, 64, 8, 8, 12, 1)) == lib.TP_ERR_SHAPE    # head_dim not a multiple of 8
+    assert st(lib.attn_desc(1, 2, 64, 8, 8, 8, 1, kv_len=5)) == lib.TP_ERR_SHAPE   # decode needs s=1
+    assert st(lib.attn_desc(1, 1, 64, 8, 8, 8, 1, kv_len=5, kv_cap=5)) == lib.TP_ERR_SHAPE
+
+
+def test_reduce_argument_errors(lib):
+    so = lib.load()
+    fake = ctypes.c_void_p(0x1000)
+    assert so.tp_reduce_partials(fake, 0, 16, 0, None, fake, 0, None) == lib.TP_ERR_SHAPE
+    assert so.tp_reduce_partials(fake, 2, -1, 0, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_reduce_partials(None, 2, 16, 0, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_reduce_partials(fake, 2, 16, 5, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_rmsnorm(fake, 2, 0, 1e-5, fake, 0, None) == lib.TP_ERR_SHAPE
+
+
+def test_empty_batch_counts_one_reduction(lib):
+    # T = 0 is a valid, empty call: nothing is launched, the block still has its one reduction
+    so = lib.load()
+    lib.tp_reset_reduction_count()
+    desc = lib.mlp_desc(0, 8, 32, 4, "gelu", "f32")
+    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None) == 0
+    assert lib.tp_reduction_count() == 1
+    lib.tp_reset_reduction_count()

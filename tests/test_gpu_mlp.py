@@ -1,0 +1,158 @@
+"""MLP block on the GPU through the C ABI, element by element against the float64 oracle.
+
+Tolerance (rel-L2 of each output tensor): 2e-2 for bf16, 1e-5 for fp32.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from oracle import mlp as omlp
+from tensor_transformer_matmul_b200 import inputs
+from tests.helpers import TOL, Mlp, dev, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _oracle_fwd(inp, act):
+    wu = None if inp["w_up"] is None else f64(inp["w_up"])
+    return omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), act, wu)
+
+
+def test_tiny_config_fp32(lib):
+    # T=4 tokens, d=8, d_ff=32, p=4 logical shards, GELU, fp32; W ~ N(0, 1/sqrt(fan_in)), seed 0
+    inp = inputs.mlp_inputs(4, 8, 32, "gelu", "f32", seed=0)
+    m = Mlp(lib, inp, 4, "gelu", "f32")
+    lib.tp_reset_reduction_count()
+    y = m.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    ref = _oracle_fwd(inp, "gelu")
+    assert rel_l2(f64(y), ref) <= TOL["f32"]
+    # the sharded sum equals the unsharded result for every p dividing d_ff
+    for p in (1, 2, 8, 16, 32):
+        mp = Mlp(lib, inp, p, "gelu", "f32")
+        assert rel_l2(f64(mp.forward(inp["x"])), ref) <= TOL["f32"], p
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu", "relu", "identity"])
+@pytest.mark.parametrize("T", [1, 17, 64, 100, 200, 300])
+def test_bf16_forward_parity(lib, act, T):
+    # several tiles and ragged tails in every dimension: d = 328 (5 K-blocks + 8), F_s = 136
+    # (padded to 256 per shard), p = 3 (not a power of two, as in the h=2/d_ff=3 worked example)
+    d, F, p = 328, 408, 3
+    inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=1, w_std=0.05)
+    m = Mlp(lib, inp, p, act, "bf16")
+    y = m.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert rel_l2(f64(y), _oracle_fwd(inp, act)) <= TOL["bf16"]
+
+
+def test_bf16_residual_and_saved(lib):
+    T, d, F, p = 150, 256, 1024, 4
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=2, w_std=0.05)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    res = inputs.normal((T, d), 1.0, 2, 99, "bf16", "cpu").to(dev())
+    y = m.forward(inp["x"], residual=res)
+    torch.cuda.synchronize()
+    ref = _oracle_fwd(inp, "swiglu") + f64(res)
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
+    # residual may alias the output
+    y2 = res.clone()
+    m.lib.tp_mlp_fwd(m.desc, inp["x"].to(dev()), m.w1p, m.w2p, y2, residual=y2, workspace=m.ws_f)
+    torch.cuda.synchronize()
+    assert rel_l2(f64(y2), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+@pytest.mark.parametrize("dtype,T", [("bf16", 200), ("bf16", 37), ("f32", 9)])
+def test_backward_parity(lib, act, dtype, T):
+    d, F, p = (328, 408, 3) if dtype == "bf16" else (24, 48, 4)
+    inp = inputs.mlp_inputs(T, d, F, act, dtype, seed=3, w_std=0.05, backward=True)
+    m = Mlp(lib, inp, p, act, dtype)
+    lib.tp_reset_reduction_count()
+    m.forward(inp["x"])
+    dx, dw1, dwu, dw2, dw1p, _ = m.backward(inp["dy"], inp["x"])
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 2   # one forward, one backward
+    wu = None if inp["w_up"] is None else f64(inp["w_up"])
+    ref = omlp.mlp_backward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), f64(inp["dy"]), act, wu)
+    tol = TOL[dtype]
+    assert rel_l2(f64(dx), ref["dx"]) <= tol
+    assert rel_l2(f64(dw1), ref["dw1"]) <= tol
+    assert rel_l2(f64(dw2), ref["dw2"]) <= tol
+    if act == "swiglu":
+        assert rel_l2(f64(dwu), ref["dw_up"]) <= tol
+
+
+def test_backward_padding_gradients_are_zero(lib):
+    # F_s = 136 pads to 256 per shard: the padding rows of the packed gradient must be exactly 0
+    d, F, p, T = 64, 408, 3, 40
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=4, w_std=0.05, backward=True)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    m.forward(inp["x"])
+    _, _, _, _, dw1p, dw2p = m.backward(inp["dy"], inp["x"])
+    torch.cuda.synchronize()
+    g1 = dw1p.view(p, 2, 256, d)         # [shard][block][gate|up rows][d]
+    g2 = dw2p.view(p, d, 256)
+    # block 1 holds features 128..255 (gate rows 0..127, up rows 128..255); 136.. are padding
+    pad = np.concatenate([f64(g1[:, 1, 8:128]), f64(g1[:, 1, 136:256])], axis=1)
+    assert np.count_nonzero(pad) == 0
+    assert np.count_nonzero(np.asarray(f64(g2[:, :, 136:]))) == 0
+
+
+def test_empty_batch(lib):
+    inp = inputs.mlp_inputs(0, 64, 256, "swiglu", "bf16", seed=5, backward=True)
+    desc = lib.mlp_desc(0, 64, 256, 2, "swiglu", "bf16")
+    w1p = torch.full((lib.tp_mlp_w1_packed_bytes(desc) // 2,), 1.0, dtype=torch.bfloat16, device=dev())
+    w2p = torch.full((lib.tp_mlp_w2_packed_bytes(desc) // 2,), 1.0, dtype=torch.bfloat16, device=dev())
+    y = torch.empty(0, 64, dtype=torch.bfloat16, device=dev())
+    lib.tp_mlp_fwd(desc, inp["x"].to(dev()), w1p, w2p, y)
+    dw1p = torch.full((w1p.numel(),), 7.0, device=dev())
+    dw2p = torch.full((w2p.numel(),), 7.0, device=dev())
+    dx = torch.empty(0, 64, dtype=torch.bfloat16, device=dev())
+    lib.tp_mlp_bwd(desc, inp["dy"].to(dev()), inp["x"].to(dev()), None, w1p, w2p, dx, dw1p, dw2p)
+    torch.cuda.synchronize()
+    assert float(dw1p.abs().sum()) == 0.0 and float(dw2p.abs().sum()) == 0.0
+
+
+def test_deterministic(lib):
+    # fixed-order reduction: two runs give identical bytes
+    inp = inputs.mlp_inputs(130, 256, 1024, "swiglu", "bf16", seed=6, w_std=0.05)
+    m = Mlp(lib, inp, 8, "swiglu", "bf16")
+    a = m.forward(inp["x"]).clone()
+    b = m.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+
+
+def test_full_size_decode_mlp_sampled(lib):
+    # T=64 (batch 64, s=1), d=8192, d_ff=28672, p=8, bf16 x ~ N(0,1), W ~ N(0, 0.02)
+    T, d, F, p = 64, 8192, 28672, 8
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    y = m.forward(inp["x"], save=False)
+    torch.cuda.synchronize()
+    rows = [0, 1, 31, 63]
+    ref = omlp.mlp_forward_rows(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu", rows,
+                                f64(inp["w_up"]))
+    assert rel_l2(f64(y)[rows], ref) <= TOL["bf16"]
+
+
+def test_full_size_prefill_mlp_sampled(lib):
+    # T=4096 (b=1, s=4096), d=8192, d_ff=28672, p=8: forward rows, then backward samples
+    T, d, F, p = 4096, 8192, 28672, 8
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02,
+                            backward=True)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    y = m.forward(inp["x"])
+    dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
+    torch.cuda.synchronize()
+    x, wg, wu, w2, dy = (f64(inp[k]) for k in ("x", "w1", "w_up", "w2", "dy"))
+    rows, cols, w2rows = [0, 777, 2048, 4095], [0, 3583, 3584, 28671], [5, 14000]
+    assert rel_l2(f64(y)[rows], omlp.mlp_forward_rows(x, wg, w2, "swiglu", rows, wu)) <= TOL["bf16"]
+    s = omlp.mlp_backward_samples(x, wg, w2, dy, "swiglu", rows, cols, w2rows, wu)
+    assert rel_l2(f64(dx)[rows], s["dx"]) <= TOL["bf16"]
+    assert rel_l2(f64(dw1)[:, cols], s["dw1_cols"]) <= TOL["bf16"]
+    assert rel_l2(f64(dwu)[:, cols], s["dw_up_cols"]) <= TOL["bf16"]
+    assert rel_l2(f64(dw2)[w2rows], s["dw2_rows"]) <= TOL["bf16"]
