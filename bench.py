@@ -1,0 +1,487 @@
+"""Benchmark of the tensor-parallel block on B200 (one JSON line on rank 0).
+
+Headline workload (the decode configuration): one step = the whole decode TP SwiGLU MLP over a
+batch of T=64 single-token sequences, d=8192, d_ff=28672, p=8 logical shards, bf16, weights
+N(0, 0.02), x N(0, 1): column-parallel up/gate GEMM with the fused SwiGLU, row-parallel down GEMM
+giving 8 full-shape partials, in-order partial-sum reduce.  Weight packing is one-time setup.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--no-extras]
+
+For N > 1 launch with torch.distributed.run (one process per GPU).  The path has no exchange
+between GPUs (all p shards live on one GPU), so N GPUs run N independent replicas ("weak"
+scaling); value = tokens of all ranks / the slowest rank's time.
+
+Also reported (N = 1 only, under "extras"): prefill SwiGLU MLP forward+backward (T=4096),
+GQA attention block (s=2048, 64 Q / 8 KV heads), and the 16-layer decode stack.
+"""
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "TP block TFLOP/s (prefill/bwd) and decode tokens/s at 1 B200; % of roofline"
+DECODE = dict(T=64, d=8192, F=28672, p=8)
+PREFILL = dict(T=4096, d=8192, F=28672, p=8)
+ATTN = dict(b=1, s=2048, h=8192, n_q=64, n_kv=8, hd=128, p=8)
+STACK = dict(layers=16, h=8192, F=28672, n_q=64, n_kv=8, hd=128, p=8, kv_len=4096)
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return {"hbm_gbs": float(pk["hbm_gbs"]), "bf16_tflops": float(pk["bf16_tflops"]),
+                "bf16_tflops_sustained": float(pk.get("bf16_tflops_sustained", pk["bf16_tflops"])),
+                "source": "measured"}
+    except Exception:
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "source": "fallback"}
+
+
+# ------------------------------------------------------------------------------ plumbing
+class Dist:
+    def __init__(self):
+        self.world = int(os.environ.get("WORLD_SIZE", "1"))
+        self.rank = int(os.environ.get("RANK", "0"))
+        self.local = int(os.environ.get("LOCAL_RANK", "0"))
+        self.pg = None
+
+    def init(self, backend):
+        if self.world > 1:
+            import datetime
+            import torch.distributed as dist
+            os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+            self.pg = dist
+
+    def barrier(self):
+        if self.pg:
+            import torch
+            if torch.cuda.is_available():
+                self.pg.barrier(device_ids=[self.local])
+            else:
+                self.pg.barrier()
+
+    def max(self, v):
+        if not self.pg:
+            return v
+        import torch
+        t = torch.tensor([float(v)], device="cuda" if torch.cuda.is_available() else "cpu")
+        self.pg.all_reduce(t, op=self.pg.ReduceOp.MAX)
+        return float(t.item())
+
+    def close(self):
+        if self.pg:
+            self.pg.destroy_process_group()
+
+
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while a timed region runs."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100"],
+                stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if not self.proc:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return None
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        smax = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i].lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None, "reasons": reasons,
+                "samples": len(rows)}
+
+
+def _cuda_time(fn, steps, stream):
+    import torch
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for _ in range(steps):
+        fn()
+    b.record(stream)
+    torch.cuda.synchronize()
+    return a.elapsed_time(b)
+
+
+def _profile(tp, fn, steps):
+    import torch
+    tp.tp_profile_reset()
+    tp.tp_profile_enable(True)
+    for _ in range(steps):
+        fn()
+    torch.cuda.synchronize()
+    tp.tp_profile_enable(False)
+    prof = tp.tp_profile_read()
+    tp.tp_profile_reset()
+    return prof
+
+
+def _threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("user_api") == "blas"]
+        if n:
+            return int(max(n))
+    except Exception:
+        pass
+    return os.cpu_count()
+
+
+# ------------------------------------------------------------------------- workloads
+def decode_mlp_bytes():
+    c = DECODE
+    Fs = c["F"] // c["p"]
+    w1 = 2 * c["F"] * c["d"] * 2          # gate + up, bf16
+    w2 = c["F"] * c["d"] * 2
+    x = c["T"] * c["d"] * 2
+    h = c["T"] * c["F"] * 2
+    part = c["p"] * c["T"] * c["d"] * 4
+    y = c["T"] * c["d"] * 2
+    return {"mlp_up_gemm": w1 + x + h, "mlp_down_gemm": w2 + h + part,
+            "reduce_partials": part + y, "step": w1 + w2 + x + y, "weights": w1 + w2, "Fs": Fs}
+
+
+def setup_mlp(tp, inputs, torch, cfg, backward=False, seed=0):
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = inputs.mlp_inputs(cfg["T"], cfg["d"], cfg["F"], "swiglu", "bf16", seed=seed,
+                            device=dev, w_std=0.02, backward=backward)
+    desc = tp.mlp_desc(cfg["T"], cfg["d"], cfg["F"], cfg["p"], "swiglu", "bf16")
+    st = {"desc": desc, "x": inp["x"], "dy": inp.get("dy")}
+    st["w1p"] = torch.empty(tp.tp_mlp_w1_packed_bytes(desc) // 2, dtype=torch.bfloat16, device=dev)
+    st["w2p"] = torch.empty(tp.tp_mlp_w2_packed_bytes(desc) // 2, dtype=torch.bfloat16, device=dev)
+    tp.tp_mlp_pack(desc, inp["w1"], inp["w_up"], inp["w2"], st["w1p"], st["w2p"])
+    st["y"] = torch.empty(cfg["T"], cfg["d"], dtype=torch.bfloat16, device=dev)
+    st["ws"] = torch.empty(tp.tp_mlp_fwd_workspace(desc), dtype=torch.uint8, device=dev)
+    if backward:
+        st["saved"] = torch.empty(tp.tp_mlp_saved_bytes(desc), dtype=torch.uint8, device=dev)
+        st["wsb"] = torch.empty(tp.tp_mlp_bwd_workspace(desc), dtype=torch.uint8, device=dev)
+        st["dx"] = torch.empty_like(st["y"])
+        st["dw1p"] = torch.empty(st["w1p"].numel(), dtype=torch.float32, device=dev)
+        st["dw2p"] = torch.empty(st["w2p"].numel(), dtype=torch.float32, device=dev)
+    del inp
+    return st
+
+
+def run_ours(args, dist):
+    import torch
+
+    from tensor_transformer_matmul_b200 import build, inputs
+    from tensor_transformer_matmul_b200 import tpblock as tp
+
+    if not os.path.exists(tp.LIB_PATH):
+        build.build()
+    tp.load()
+    torch.cuda.set_device(dist.local)
+    dist.init("nccl")
+    stream = torch.cuda.current_stream()
+    peaks = _peaks()
+    c = DECODE
+
+    st = setup_mlp(tp, inputs, torch, c, seed=dist.rank)
+
+    def step():
+        tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], workspace=st["ws"])
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+
+    clk = ClockSampler(dist.local)
+    dist.barrier()
+    torch.cuda.synchronize()
+    clk.start()
+    l0 = tp.tp_launch_count()
+    ms = _cuda_time(step, args.steps, stream)
+    launches = tp.tp_launch_count() - l0
+    clocks = clk.stop()
+    dist.barrier()
+    ms = dist.max(ms)
+    ms_step = ms / args.steps
+    tokens = c["T"] * args.steps * dist.world
+    value = tokens / (ms / 1e3)
+
+    # per-kernel durations, measured with events on the launching stream over K more steps
+    prof = _profile(tp, step, args.steps)
+    nbytes = decode_mlp_bytes()
+    dom = max(prof, key=lambda k: prof[k][1])
+    dom_ms = prof[dom][1] / prof[dom][0]
+    achieved = nbytes.get(dom, 0) / (dom_ms / 1e3) / 1e9
+    roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
+                "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(achieved / peaks["hbm_gbs"], 4),
+                "traffic": None, "peak_source": peaks["source"],
+                "algorithmic_bytes_per_launch": nbytes.get(dom, 0),
+                "kernel_ms": round(dom_ms, 5)}
+    step_gbs = nbytes["step"] / (ms_step / 1e3) / 1e9
+    kernels = {k: {"launches_per_step": v[0] / args.steps, "ms_per_launch": round(v[1] / v[0], 5),
+                   "GB_per_s": round(nbytes[k] / (v[1] / v[0] / 1e3) / 1e9, 1) if k in nbytes else None}
+               for k, v in prof.items()}
+
+    # end to end through the public API: pinned host x -> device, block, y -> pinned host
+    xh = st["x"].cpu().pin_memory()
+    yh = torch.empty_like(st["y"], device="cpu").pin_memory()
+    xd = torch.empty_like(st["x"])
+
+    def e2e_step():
+        xd.copy_(xh, non_blocking=True)
+        tp.tp_mlp_fwd(st["desc"], xd, st["w1p"], st["w2p"], st["y"], workspace=st["ws"])
+        yh.copy_(st["y"], non_blocking=True)
+
+    for _ in range(3):
+        e2e_step()
+    dist.barrier()
+    e2e_ms = dist.max(_cuda_time(e2e_step, args.steps, stream))
+    e2e = {"value": round(tokens / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": xh.numel() * xh.element_size(),
+           "d2h_bytes_per_step": yh.numel() * yh.element_size()}
+
+    out = {
+        "metric": METRIC, "value": round(value, 1), "unit": "tokens/s", "n_gpus": dist.world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 5),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic (seeded N(0,0.02) weights, N(0,1) activations, drawn on the GPU)",
+        "config": {"workload": "decode TP SwiGLU MLP: T=64 (batch 64, s=1), d=8192, d_ff=28672, "
+                               "p=8 logical shards, bf16, fp32 accumulate",
+                   "global_batch": c["T"] * dist.world, "seq_len": 1,
+                   "parallelism": f"replicas x{dist.world} (p=8 logical shards per GPU)",
+                   "l2": "inputs larger than L2: 1.41 GB of weights streamed per step",
+                   "step_GB_per_s": round(step_gbs, 1),
+                   "step_frac_of_hbm": round(step_gbs / peaks["hbm_gbs"], 4)},
+        "roofline": roofline, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
+        "kernels": kernels,
+    }
+
+    if dist.world == 1 and not args.no_extras:
+        del st
+        torch.cuda.empty_cache()
+        out["extras"] = run_extras(args, tp, inputs, torch, stream, peaks)
+
+    if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+    elif dist.rank == 0:
+        out["cpu_baseline"] = None
+    dist.close()
+    if dist.rank == 0:
+        print(json.dumps(out), flush=True)
+
+
+def run_extras(args, tp, inputs, torch, stream, peaks):
+    ex = {}
+    steps = max(3, min(args.steps, args.extra_steps))
+    # prefill SwiGLU MLP forward + backward: 6 T d F flops per direction pair x 3 matmuls
+    c = PREFILL
+    st = setup_mlp(tp, inputs, torch, c, backward=True)
+
+    def fwd():
+        tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], saved=st["saved"],
+                      workspace=st["ws"])
+
+    def bwd():
+        tp.tp_mlp_bwd(st["desc"], st["dy"], st["x"], st["saved"], st["w1p"], st["w2p"], st["dx"],
+                      st["dw1p"], st["dw2p"], workspace=st["wsb"])
+
+    def both():
+        fwd()
+        bwd()
+
+    for _ in range(3):
+        both()
+    f_fl = 2.0 * c["T"] * c["d"] * c["F"] * 3
+    b_fl = 2 * f_fl
+    ms_f = _cuda_time(fwd, steps, stream) / steps
+    ms_b = _cuda_time(bwd, steps, stream) / steps
+    prof = _profile(tp, both, steps)
+    gemm_fl = {"mlp_up_gemm": 2.0 * c["T"] * c["d"] * 2 * c["F"],
+               "mlp_down_gemm": 2.0 * c["T"] * c["d"] * c["F"],
+               "mlp_dh_gemm": 2.0 * c["T"] * c["d"] * c["F"],
+               "mlp_dw2_gemm": 2.0 * c["T"] * c["d"] * c["F"],
+               "mlp_dw1_gemm": 2.0 * c["T"] * c["d"] * 2 * c["F"],
+               "mlp_dx_gemm": 2.0 * c["T"] * c["d"] * 2 * c["F"]}
+    kern = {}
+    for k, (n, ms) in prof.items():
+        e = {"ms_per_launch": round(ms / n, 4)}
+        if k in gemm_fl:
+            tf = gemm_fl[k] / (ms / n / 1e3) / 1e12
+            e["TFLOP_per_s"] = round(tf, 1)
+            e["frac_of_sustained_peak"] = round(tf / peaks["bf16_tflops_sustained"], 3)
+        kern[k] = e
+    tot = (ms_f + ms_b)
+    ex["prefill_mlp_fwd_bwd"] = {
+        "workload": "prefill TP SwiGLU MLP fwd+bwd: T=4096, d=8192, d_ff=28672, p=8, bf16",
+        "ms_fwd": round(ms_f, 3), "ms_bwd": round(ms_b, 3),
+        "TFLOP_per_s": round((f_fl + b_fl) / (tot / 1e3) / 1e12, 1),
+        "TFLOP_per_s_fwd": round(f_fl / (ms_f / 1e3) / 1e12, 1),
+        "TFLOP_per_s_bwd": round(b_fl / (ms_b / 1e3) / 1e12, 1),
+        "frac_of_burst_peak": round((f_fl + b_fl) / (tot / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
+        "frac_of_sustained_peak": round((f_fl + b_fl) / (tot / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 3),
+        "tokens_per_s": round(c["T"] / (tot / 1e3), 1), "kernels": kern, "steps": steps}
+    del st
+    torch.cuda.empty_cache()
+
+    # GQA attention block (prefill): QKV + causal local attention + O-proj + reduce
+    a = ATTN
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ai = inputs.attn_inputs(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], "bf16", seed=0,
+                            device=dev)
+    ad = tp.attn_desc(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], a["p"])
+    wqkv = torch.empty(tp.tp_attn_wqkv_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
+    wo = torch.empty(tp.tp_attn_wo_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
+    tp.tp_attn_pack(ad, ai["wq"], ai["wk"], ai["wv"], ai["wo"], wqkv, wo)
+    ya = torch.empty_like(ai["x"])
+    wsa = torch.empty(tp.tp_attn_fwd_workspace(ad), dtype=torch.uint8, device=dev)
+
+    def attn():
+        tp.tp_attn_fwd(ad, ai["x"], wqkv, wo, ya, workspace=wsa)
+
+    for _ in range(3):
+        attn()
+    ms_a = _cuda_time(attn, steps, stream) / steps
+    s, h = a["s"], a["h"]
+    fl_qkv = 2.0 * s * h * (a["n_q"] + 2 * a["n_kv"]) * a["hd"]
+    fl_att = 2.0 * 2 * a["n_q"] * a["hd"] * s * (s + 1) / 2
+    fl_o = 2.0 * s * a["n_q"] * a["hd"] * h
+    prof = _profile(tp, attn, steps)
+    ex["attention_block"] = {
+        "workload": "TP GQA attention: b=1, s=2048, h=8192, 64 Q / 8 KV heads, hd=128, p=8, causal",
+        "ms": round(ms_a, 3),
+        "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12, 1),
+        "frac_of_burst_peak": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
+        "tokens_per_s": round(s / (ms_a / 1e3), 1),
+        "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
+        "steps": steps}
+    return ex
+
+
+# -------------------------------------------------------------------------- CPU side
+ORACLE_CHUNK = 512   # d_ff features per oracle step
+
+
+def _oracle_decode_setup():
+    """Host float64 copies of the decode workload's weights (drawn on the CPU)."""
+    from tensor_transformer_matmul_b200 import inputs
+    c = DECODE
+    inp = inputs.mlp_inputs(c["T"], c["d"], c["F"], "swiglu", "bf16", seed=0, device="cpu",
+                            w_std=0.02)
+    return {k: inputs.to_f64(v) for k, v in inp.items() if v is not None}
+
+
+def _oracle_step(a, i):
+    """One bounded sample of the decode MLP on the oracle: all 64 tokens through a 512-feature
+    slice of d_ff (its contribution to y).  Worth 64 * 512 / d_ff token-equivalents."""
+    from oracle import mlp as omlp
+    n = DECODE["F"] // ORACLE_CHUNK
+    c = slice((i % n) * ORACLE_CHUNK, (i % n + 1) * ORACLE_CHUNK)
+    return omlp.mlp_forward(a["x"], a["w1"][:, c], a["w2"][c, :], "swiglu", a["w_up"][:, c])
+
+
+TOKENS_PER_ORACLE_STEP = DECODE["T"] * ORACLE_CHUNK / DECODE["F"]
+
+
+def cpu_baseline(seconds=10.0, arrays=None):
+    """The oracle (float64 numpy, as it stands) on the host cores, in decode tokens/s."""
+    a = arrays if arrays is not None else _oracle_decode_setup()
+    n, t0 = 0, time.perf_counter()
+    while True:
+        _oracle_step(a, n)
+        n += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return {"value": round(n * TOKENS_PER_ORACLE_STEP / el, 3), "unit": "tokens/s",
+            "cores": _threads(), "kind": "oracle",
+            "sample": f"{n} oracle calls, each all 64 tokens through a {ORACLE_CHUNK}-feature slice "
+                      f"of d_ff ({TOKENS_PER_ORACLE_STEP:.3f} token-equivalents), {el:.1f} s"}
+
+
+def run_reference(args, dist):
+    """The oracle as the reference arm: same workload, metric and unit, on the host cores."""
+    if dist.rank != 0:
+        return
+    a = _oracle_decode_setup()
+    for i in range(max(1, args.warmup)):
+        _oracle_step(a, i)
+    t0 = time.perf_counter()
+    for i in range(args.steps):
+        _oracle_step(a, i)
+    el = time.perf_counter() - t0
+    value = TOKENS_PER_ORACLE_STEP * args.steps / el
+    sample = (f"{args.steps} steps, each all 64 tokens through a {ORACLE_CHUNK}-feature slice of "
+              f"d_ff ({TOKENS_PER_ORACLE_STEP:.3f} token-equivalents)")
+    out = {"impl": "reference", "metric": METRIC, "value": round(value, 3), "unit": "tokens/s",
+           "n_gpus": dist.world, "steps": args.steps, "warmup": args.warmup,
+           "ms_per_step": round(el / args.steps * 1e3, 3), "higher_is_better": True,
+           "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+           "config": {"workload": "decode TP SwiGLU MLP: T=64 (batch 64, s=1), d=8192, "
+                                  "d_ff=28672, p=8 logical shards",
+                      "global_batch": 64, "seq_len": 1, "parallelism": "host oracle"},
+           "cpu_baseline": {"value": round(value, 3), "unit": "tokens/s", "cores": _threads(),
+                            "kind": "oracle", "sample": sample},
+           "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                   "d2h_bytes_per_step": 0}}
+    print(json.dumps(out), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=2000)
+    ap.add_argument("--warmup", type=int, default=20)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-extras", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--extra-steps", type=int, default=20)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    args = ap.parse_args()
+    args.warmup = max(3, args.warmup)
+    dist = Dist()
+    if args.impl == "reference":
+        run_reference(args, dist)
+        return
+    run_ours(args, dist)
+
+
+if __name__ == "__main__":
+    main()

@@ -213,6 +213,16 @@ tp_status tp_check_device_error(void* stream);
 /* 1 if this build contains the sm_100a tensor-core kernels and the current device runs them. */
 int32_t tp_tensor_core_path_available(void);
 
+/* Per-kernel timing.  While enabled, every kernel the library launches is bracketed by two CUDA
+ * events recorded on the launching stream (skipped while the stream is being captured into a
+ * graph).  tp_profile_read synchronizes the device and returns, for entry i (0-based, in order
+ * of first appearance), the kernel label, its launch count and the summed event time in ms;
+ * it returns 0 once i is past the last entry.  tp_profile_reset drops all records. */
+void tp_profile_enable(int32_t on);
+int32_t tp_profile_read(int32_t i, char* label, int32_t label_len, uint64_t* launches,
+                        double* total_ms);
+void tp_profile_reset(void);
+
 /* Library version, major*10000 + minor*100 + patch. */
 int32_t tp_version(void);
 

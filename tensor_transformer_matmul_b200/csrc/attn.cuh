@@ -308,6 +308,7 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
     const int64_t warps = L.tokens * L.n_q;
     const int64_t blocks = ceil_div(warps * 32, 128);
     if (blocks > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "attention grid too large");
+    ProfScope prof(s, "attn_prefill");
     attn::prefill_simt_kernel<T><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
         qkv, o, ix, L.b, L.s, L.n_q, L.causal, scale);
     TP_LAUNCH_CHECK();
@@ -316,6 +317,7 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   // decode: append, split-KV attention, combine
   {
     const int64_t total = L.b * L.n_kv * L.hd;
+    ProfScope prof(s, "kv_append");
     attn::kv_append_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
         qkv, ix, static_cast<T*>(kc), static_cast<T*>(vc), L.b, L.n_kv, L.kv_cap, L.kv_len);
     TP_LAUNCH_CHECK();
@@ -327,6 +329,7 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   const int64_t n_keys = L.kv_len + 1;
 #define TP_DECODE_CASE(G, H)                                                                  \
   if (group == G && L.hd == H) {                                                              \
+    ProfScope prof(s, "attn_decode");                                                         \
     attn::decode_split_kernel<T, G, H><<<grid, 256, 0, s>>>(qkv, ix, static_cast<const T*>(kc),  \
         static_cast<const T*>(vc), L.kv_cap, n_keys, L.n_q, L.n_kv, scale, ml);               \
     TP_LAUNCH_CHECK();                                                                        \
@@ -340,6 +343,7 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   }
 #undef TP_DECODE_CASE
   const int64_t rows = L.b * L.n_q;
+  ProfScope prof(s, "attn_decode_combine");
   attn::decode_combine_kernel<T><<<simt::elementwise_grid(rows * L.hd), 256, 0, s>>>(
       ml, L.kv_splits, L.hd, rows, o);
   TP_LAUNCH_CHECK();
@@ -367,12 +371,12 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
   const Operand wo{wqkv, false, rows, L.h, 1, L.h, 0};
   if (L.tokens <= 128) {
     ep.swap = 1;
-    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
-    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
-    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s);
+    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
+    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
+    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s);
+  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s, "attn_qkv_gemm");
 }
 
 inline tp_status out_proj_partials(const AttnLayout& L, const void* o, const void* wo_p,
@@ -388,12 +392,12 @@ inline tp_status out_proj_partials(const AttnLayout& L, const void* o, const voi
   ep.cols_valid = static_cast<int32_t>(L.h);
   if (L.tokens <= 128) {
     ep.swap = 1;
-    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
-    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
-    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s);
+    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
+    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
+    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s);
+  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s, "attn_out_gemm");
 }
 }  // namespace attn_tc
 

@@ -45,7 +45,7 @@ inline tp_status encode_operand(CUtensorMap* map, const Operand& o, int tile_mn)
 template <class Cfg, class Epi>
 tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int64_t K,
                    int64_t batch, const typename Epi::Params& ep, cudaStream_t stream,
-                   int m_fastest = -1) {
+                   const char* label = "gemm", int m_fastest = -1) {
   static_assert(Cfg::A_MN == false || Cfg::A_ROWS % 64 == 0, "A tile");
   if (a.mn_major != Cfg::A_MN || b.mn_major != Cfg::B_MN)
     return set_error(TP_ERR_INVALID_ARG, "operand major does not match the tile config");
@@ -83,6 +83,7 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   }
   const int64_t tiles = static_cast<int64_t>(gp.batch) * gp.m_blocks * gp.n_blocks;
   const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  ProfScope prof(stream, label);
   gemm_kernel<Cfg, Epi><<<grid, kThreads, Cfg::SMEM_BYTES, stream>>>(ta, tb, gp, ep);
   TP_LAUNCH_CHECK();
   return TP_OK;

@@ -82,6 +82,7 @@ inline tp_status launch_t(const void* part, int p, int64_t n, const void* res, v
   int64_t blocks = ceil_div(work, 256);
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
+  ProfScope prof(s, "reduce_partials");
   if (vec)
     reduce_vec8_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
         static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
@@ -132,6 +133,7 @@ inline tp_status rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void
                          cudaStream_t s) {
   if (rows == 0) return TP_OK;
   if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
+  ProfScope prof(s, "rmsnorm");
   if (dtype == TP_BF16)
     rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), 256, 0, s>>>(
         static_cast<const __nv_bfloat16*>(x), d, eps, static_cast<__nv_bfloat16*>(out));

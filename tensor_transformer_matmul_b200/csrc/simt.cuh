@@ -62,6 +62,7 @@ inline tp_status gemm(const GemmArgs& g, cudaStream_t s) {
     return set_error(TP_ERR_UNSUPPORTED, "SIMT GEMM grid too large");
   dim3 grid(static_cast<unsigned>(ceil_div(g.N, kTile)), static_cast<unsigned>(ceil_div(g.M, kTile)),
             static_cast<unsigned>(g.batch));
+  ProfScope prof(s, "simt_gemm");
   gemm_kernel<T><<<grid, 256, 0, s>>>(g);
   TP_LAUNCH_CHECK();
   return TP_OK;

@@ -2,7 +2,10 @@
 // queries and TMA tensor-map encoding.
 #include <cuda.h>
 #include <cudaTypedefs.h>
+#include <algorithm>
 #include <atomic>
+#include <cstdio>
+#include <vector>
 #include <mutex>
 #include <string>
 
@@ -95,9 +98,77 @@ tp_status encode_tmap_bf16_3d(CUtensorMap* map, const void* base, uint64_t inner
   return TP_OK;
 }
 
+namespace {
+struct ProfRec {
+  std::string label;
+  cudaEvent_t a, b;
+};
+std::mutex g_prof_mu;
+std::atomic<int> g_prof_on{0};
+std::vector<ProfRec> g_prof;
+}  // namespace
+
+ProfScope::ProfScope(cudaStream_t s, const char* label) : s_(s), label_(label) {
+  if (!g_prof_on.load(std::memory_order_relaxed)) return;
+  cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+  if (cudaStreamIsCapturing(s, &cs) != cudaSuccess || cs != cudaStreamCaptureStatusNone) return;
+  if (cudaEventCreate(&start_) != cudaSuccess) {
+    start_ = nullptr;
+    return;
+  }
+  cudaEventRecord(start_, s_);
+}
+
+ProfScope::~ProfScope() {
+  if (!start_) return;
+  cudaEvent_t end = nullptr;
+  if (cudaEventCreate(&end) != cudaSuccess) {
+    cudaEventDestroy(start_);
+    return;
+  }
+  cudaEventRecord(end, s_);
+  std::lock_guard<std::mutex> g(g_prof_mu);
+  g_prof.push_back({label_, start_, end});
+}
+
 }  // namespace tp
 
 extern "C" {
+
+void tp_profile_enable(int32_t on) { tp::g_prof_on.store(on ? 1 : 0); }
+
+void tp_profile_reset(void) {
+  std::lock_guard<std::mutex> g(tp::g_prof_mu);
+  for (auto& r : tp::g_prof) {
+    cudaEventDestroy(r.a);
+    cudaEventDestroy(r.b);
+  }
+  tp::g_prof.clear();
+}
+
+int32_t tp_profile_read(int32_t i, char* label, int32_t label_len, uint64_t* launches,
+                        double* total_ms) {
+  cudaDeviceSynchronize();
+  std::lock_guard<std::mutex> g(tp::g_prof_mu);
+  std::vector<std::string> order;
+  for (auto& r : tp::g_prof)
+    if (std::find(order.begin(), order.end(), r.label) == order.end()) order.push_back(r.label);
+  if (i < 0 || i >= static_cast<int32_t>(order.size())) return 0;
+  uint64_t n = 0;
+  double ms = 0.0;
+  for (auto& r : tp::g_prof) {
+    if (r.label != order[i]) continue;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) == cudaSuccess) ms += t;
+    ++n;
+  }
+  if (label && label_len > 0) {
+    std::snprintf(label, static_cast<size_t>(label_len), "%s", order[i].c_str());
+  }
+  if (launches) *launches = n;
+  if (total_ms) *total_ms = ms;
+  return 1;
+}
 
 uint64_t tp_reduction_count(void) { return tp::g_reductions.load(); }
 void tp_reset_reduction_count(void) { tp::g_reductions.store(0); }

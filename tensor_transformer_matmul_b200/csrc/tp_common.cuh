@@ -35,6 +35,19 @@ void count_reduction();
     ::tp::count_launch();                                                                       \
   } while (0)
 
+// Brackets one kernel launch with CUDA events when tp_profile_enable(1) is in effect.
+class ProfScope {
+ public:
+  ProfScope(cudaStream_t s, const char* label);
+  ~ProfScope();
+  ProfScope(const ProfScope&) = delete;
+  ProfScope& operator=(const ProfScope&) = delete;
+ private:
+  cudaStream_t s_;
+  const char* label_;
+  cudaEvent_t start_ = nullptr;
+};
+
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t a) { return (a + 255) & ~size_t(255); }

@@ -104,16 +104,16 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
   if (L.T <= 128) {
     ep.swap = 1;
     if (swiglu) {
-      if (L.T <= 16) return tc::run_gemm<KK<16, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
-      if (L.T <= 64) return tc::run_gemm<KK<64, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
-      return tc::run_gemm<KK<128, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+      if (L.T <= 16) return tc::run_gemm<KK<16, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
+      if (L.T <= 64) return tc::run_gemm<KK<64, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
+      return tc::run_gemm<KK<128, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
     }
-    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
-    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
-    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s);
+    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
+    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
+    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s);
+  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s, "mlp_up_gemm");
 }
 
 // partial[i] = h_i W2_i  (fp32, [p][T][d])
@@ -129,12 +129,12 @@ tp_status tc_down_partials(const MlpLayout& L, const void* h, const void* w2p, f
   ep.cols_valid = static_cast<int32_t>(L.d);
   if (L.T <= 128) {
     ep.swap = 1;
-    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
-    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
-    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s);
+    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
+    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
+    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s);
+  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s, "mlp_down_gemm");
 }
 
 tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
@@ -155,10 +155,10 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.act = L.act;
     if (L.Fsp % 256 == 0)
       st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiActBwd>(
-          a, b, L.T, L.Fsp, L.d, P, ep, s);
+          a, b, L.T, L.Fsp, L.d, P, ep, s, "mlp_dh_gemm");
     else
       st = tc::run_gemm<TileCfg<128, 1, false, true, stages_for(128, 1)>, tc::EpiActBwd>(
-          a, b, L.T, L.Fsp, L.d, P, ep, s);
+          a, b, L.T, L.Fsp, L.d, P, ep, s, "mlp_dh_gemm");
     if (st != TP_OK) return st;
   }
   // (2) dW2_i[n][c] = sum_t dY[t][n] h_i[t][c]   (no exchange between shards)
@@ -174,10 +174,10 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.swap = 0;
     if (L.Fsp % 256 == 0)
       st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-          a, b, L.d, L.Fsp, L.T, P, ep, s);
+          a, b, L.d, L.Fsp, L.T, P, ep, s, "mlp_dw2_gemm");
     else
       st = tc::run_gemm<TileCfg<128, 1, true, true, stages_for(128, 1)>, tc::EpiStoreF32>(
-          a, b, L.d, L.Fsp, L.T, P, ep, s);
+          a, b, L.d, L.Fsp, L.T, P, ep, s, "mlp_dw2_gemm");
     if (st != TP_OK) return st;
   }
   // (3) dW1_i[r][k] = sum_t dz_i[t][r] x[t][k]   (no exchange between shards)
@@ -192,7 +192,7 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.cols_valid = static_cast<int32_t>(L.d);
     ep.swap = 0;
     st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-        a, b, L.R, L.d, L.T, P, ep, s);
+        a, b, L.R, L.d, L.T, P, ep, s, "mlp_dw1_gemm");
     if (st != TP_OK) return st;
   }
   // (4) dx_i = dz_i W1_i^T  (partials, summed by the caller)
@@ -207,7 +207,7 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.cols_valid = static_cast<int32_t>(L.d);
     ep.swap = 0;
     st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-        a, b, L.T, L.d, L.R, P, ep, s);
+        a, b, L.T, L.d, L.R, P, ep, s, "mlp_dx_gemm");
   }
   return st;
 }
@@ -225,9 +225,12 @@ tp_status simt_forward(const MlpLayout& L, const void* x, const void* w1p, const
   tp_status st = simt::gemm<T>(g, s);
   if (st != TP_OK) return st;
   const int64_t total = L.T * P * L.Fsp;
-  simt::act_fwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
-      static_cast<const T*>(z), static_cast<T*>(h), L.T, L.p, L.R, L.Fsp, L.act);
-  TP_LAUNCH_CHECK();
+  {
+    ProfScope prof(s, "simt_act");
+    simt::act_fwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
+        static_cast<const T*>(z), static_cast<T*>(h), L.T, L.p, L.R, L.Fsp, L.act);
+    TP_LAUNCH_CHECK();
+  }
   simt::GemmArgs g2{};
   g2.a = h; g2.a_bs = L.Fsp; g2.a_sm = P * L.Fsp; g2.a_sk = 1;
   g2.b = w2p; g2.b_bs = L.d * L.Fsp; g2.b_sm = L.Fsp; g2.b_sk = 1;
@@ -250,9 +253,12 @@ tp_status simt_backward(const MlpLayout& L, const void* dy, const void* x, const
   g.M = L.T; g.N = L.Fsp; g.K = L.d; g.batch = P; g.out_f32 = 1;
   if ((st = simt::gemm<T>(g, s)) != TP_OK) return st;
   const int64_t total = L.T * P * L.Fsp;
-  simt::act_bwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
-      dh, static_cast<const T*>(z), static_cast<T*>(dz), L.T, L.p, L.R, L.Fsp, L.act);
-  TP_LAUNCH_CHECK();
+  {
+    ProfScope prof(s, "simt_act_bwd");
+    simt::act_bwd_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
+        dh, static_cast<const T*>(z), static_cast<T*>(dz), L.T, L.p, L.R, L.Fsp, L.act);
+    TP_LAUNCH_CHECK();
+  }
   // dW2_i[n][c] = sum_t dY[t][n] h[t][i*Fsp + c]
   g = simt::GemmArgs{};
   g.a = dy; g.a_bs = 0; g.a_sm = 1; g.a_sk = L.d;

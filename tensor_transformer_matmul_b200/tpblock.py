@@ -30,6 +30,7 @@ EXPORTS = (
     "tp_attn_pack", "tp_attn_fwd_workspace", "tp_attn_fwd", "tp_reduce_partials", "tp_rmsnorm",
     "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
+    "tp_profile_enable", "tp_profile_read", "tp_profile_reset",
 )
 
 
@@ -84,6 +85,9 @@ def load():
         "tp_launch_count": (ctypes.c_uint64, []), "tp_last_error": (ctypes.c_char_p, []),
         "tp_status_string": (ctypes.c_char_p, [I32]), "tp_check_device_error": (I32, [P]),
         "tp_tensor_core_path_available": (I32, []), "tp_version": (I32, []),
+        "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
+        "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
+                                  ctypes.POINTER(ctypes.c_double)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -249,3 +253,25 @@ def tp_tensor_core_path_available():
 
 def tp_version():
     return load().tp_version()
+
+
+def tp_profile_enable(on=True):
+    load().tp_profile_enable(1 if on else 0)
+
+
+def tp_profile_reset():
+    load().tp_profile_reset()
+
+
+def tp_profile_read():
+    """{label: (launches, total_ms)} of the kernels recorded while profiling was enabled."""
+    lib = load()
+    out = {}
+    buf = ctypes.create_string_buffer(128)
+    n = ctypes.c_uint64()
+    ms = ctypes.c_double()
+    i = 0
+    while lib.tp_profile_read(i, buf, 128, ctypes.byref(n), ctypes.byref(ms)):
+        out[buf.value.decode()] = (int(n.value), float(ms.value))
+        i += 1
+    return out
