@@ -159,6 +159,33 @@ def _profile(tp, fn, steps):
     return prof
 
 
+GEMM_SOURCES = ("gemm_tc.cuh", "sm100.cuh", "gemm_launch.cuh", "tp_mlp.cu")
+
+
+def _gemm_source_hash():
+    import hashlib
+    h = hashlib.sha256()
+    for f in GEMM_SOURCES:
+        with open(os.path.join(ROOT, "tensor_transformer_matmul_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def _measured_traffic(label, workload):
+    """ncu DRAM bytes per launch for (label, workload), or None if absent or stale."""
+    try:
+        cur = _gemm_source_hash()
+        with open(os.path.join(ROOT, "profiles", "traffic.txt")) as f:
+            for line in f:
+                parts = line.split()
+                if len(parts) >= 4 and not parts[0].startswith("#") and parts[0] == label \
+                        and parts[1] == workload:
+                    return int(parts[2]) if parts[3] == cur else None
+    except Exception:
+        pass
+    return None
+
+
 def _threads():
     try:
         from threadpoolctl import threadpool_info
@@ -252,7 +279,7 @@ def run_ours(args, dist):
     roofline = {"bound": "hbm", "kernel": dom, "achieved": round(achieved, 1),
                 "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(achieved / peaks["hbm_gbs"], 4),
-                "traffic": None, "peak_source": peaks["source"],
+                "traffic": _measured_traffic(dom, "decode_mlp"), "peak_source": peaks["source"],
                 "algorithmic_bytes_per_launch": nbytes.get(dom, 0),
                 "kernel_ms": round(dom_ms, 5)}
     step_gbs = nbytes["step"] / (ms_step / 1e3) / 1e9
@@ -310,7 +337,16 @@ def run_ours(args, dist):
 
 def run_extras(args, tp, inputs, torch, stream, peaks):
     ex = {}
+    which = set(args.extras.split(","))
     steps = max(3, min(args.steps, args.extra_steps))
+    if "prefill" in which:
+        ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
+    if "attention" in which:
+        ex["attention_block"] = extra_attention(tp, inputs, torch, stream, peaks, steps)
+    return ex
+
+
+def extra_prefill(tp, inputs, torch, stream, peaks, steps):
     # prefill SwiGLU MLP forward + backward: 6 T d F flops per direction pair x 3 matmuls
     c = PREFILL
     st = setup_mlp(tp, inputs, torch, c, backward=True)
@@ -349,7 +385,7 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
             e["frac_of_sustained_peak"] = round(tf / peaks["bf16_tflops_sustained"], 3)
         kern[k] = e
     tot = (ms_f + ms_b)
-    ex["prefill_mlp_fwd_bwd"] = {
+    res = {
         "workload": "prefill TP SwiGLU MLP fwd+bwd: T=4096, d=8192, d_ff=28672, p=8, bf16",
         "ms_fwd": round(ms_f, 3), "ms_bwd": round(ms_b, 3),
         "TFLOP_per_s": round((f_fl + b_fl) / (tot / 1e3) / 1e12, 1),
@@ -360,8 +396,11 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
         "tokens_per_s": round(c["T"] / (tot / 1e3), 1), "kernels": kern, "steps": steps}
     del st
     torch.cuda.empty_cache()
+    return res
 
-    # GQA attention block (prefill): QKV + causal local attention + O-proj + reduce
+
+def extra_attention(tp, inputs, torch, stream, peaks, steps):
+    """GQA attention block (prefill): QKV + causal local attention + O-proj + reduce."""
     a = ATTN
     dev = torch.device("cuda", torch.cuda.current_device())
     ai = inputs.attn_inputs(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], "bf16", seed=0,
@@ -384,7 +423,7 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     fl_att = 2.0 * 2 * a["n_q"] * a["hd"] * s * (s + 1) / 2
     fl_o = 2.0 * s * a["n_q"] * a["hd"] * h
     prof = _profile(tp, attn, steps)
-    ex["attention_block"] = {
+    return {
         "workload": "TP GQA attention: b=1, s=2048, h=8192, 64 Q / 8 KV heads, hd=128, p=8, causal",
         "ms": round(ms_a, 3),
         "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12, 1),
@@ -392,7 +431,6 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
         "tokens_per_s": round(s / (ms_a / 1e3), 1),
         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
         "steps": steps}
-    return ex
 
 
 # -------------------------------------------------------------------------- CPU side
@@ -473,6 +511,8 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=20)
+    ap.add_argument("--extras", default="prefill,attention,stack",
+                    help="comma list of extra workloads to measure at N=1")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)
