@@ -124,6 +124,27 @@ tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const void* x, con
                      const void* w1p, const void* w2p, void* dx, void* dw1p, void* dw2p,
                      void* workspace, size_t ws_bytes, void* stream);
 
+/* tp_mlp_fwd for callers that cannot allocate device memory (the pages have no counterpart:
+ * this is a deployment convenience, not part of the method).  Some callers cannot call
+ * cudaMalloc -- a plug-in inside a host application that owns all device memory and gives its
+ * plug-ins no allocator, or a latency-critical loop where an allocation, which may synchronize
+ * the device, is not allowed.  This variant takes only inputs and outputs (same meaning as in
+ * tp_mlp_fwd, no `saved`) and runs in scratch held in a fixed array of TP_MLP_STATIC_WS_BYTES
+ * (32 MiB) of the library's own device memory, which every GPU that loads the library keeps
+ * until exit.  It allocates nothing.
+ *   - A shape whose tp_mlp_fwd_workspace() exceeds TP_MLP_STATIC_WS_BYTES returns
+ *     TP_ERR_WORKSPACE before anything is enqueued (e.g. T <= 64 fits for d = 8192,
+ *     d_ff = 28672, p = 8).
+ *   - The first call on a device looks up the array's device address once for that device; make
+ *     it before any stream capture.
+ *   - All calls share the array: calls that overlap on the GPU race and must be serialised by
+ *     the caller.  The array keeps the last call's contents; nothing in it needs to start at
+ *     zero, since every scratch byte a call reads is written by that call first.
+ * Same errors, results and reduction count as tp_mlp_fwd otherwise. */
+#define TP_MLP_STATIC_WS_BYTES ((size_t)32 << 20)
+tp_status tp_mlp_fwd_static_ws(const tp_mlp_desc* desc, const void* x, const void* w1p,
+                               const void* w2p, const void* residual, void* y, void* stream);
+
 /* Scatter packed fp32 gradients back to the user layout (fp32): dw1 [d][d_ff] (dWg for SWIGLU),
  * dw_up [d][d_ff] (SWIGLU only, else NULL), dw2 [d_ff][d]. */
 tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw1p, const void* dw2p,

@@ -30,7 +30,7 @@ EXPORTS = (
     "tp_attn_pack", "tp_attn_fwd_workspace", "tp_attn_fwd", "tp_reduce_partials", "tp_rmsnorm",
     "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
-    "tp_profile_enable", "tp_profile_read", "tp_profile_reset",
+    "tp_profile_enable", "tp_profile_read", "tp_profile_reset", "tp_mlp_fwd_static_ws",
 )
 
 
@@ -76,6 +76,7 @@ def load():
         "tp_mlp_bwd_workspace": (S, [MD]),
         "tp_mlp_bwd": (I32, [MD, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_mlp_unpack_grads": (I32, [MD, P, P, P, P, P, P]),
+        "tp_mlp_fwd_static_ws": (I32, [MD, P, P, P, P, P, P]),
         "tp_attn_wqkv_packed_bytes": (S, [AD]), "tp_attn_wo_packed_bytes": (S, [AD]),
         "tp_attn_pack": (I32, [AD, P, P, P, P, P, P, P]), "tp_attn_fwd_workspace": (S, [AD]),
         "tp_attn_fwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
@@ -172,6 +173,13 @@ def tp_mlp_bwd(desc, dy, x, saved, w1p, w2p, dx, dw1p, dw2p, workspace=None, str
     _check(load().tp_mlp_bwd(ctypes.byref(desc), _ptr(dy), _ptr(x), _ptr(saved), _ptr(w1p),
                              _ptr(w2p), _ptr(dx), _ptr(dw1p), _ptr(dw2p), _ptr(workspace),
                              _nbytes(workspace), _stream(stream)))
+
+
+def tp_mlp_fwd_static_ws(desc, x, w1p, w2p, y, residual=None, stream=None):
+    """tp_mlp_fwd without a workspace argument, for callers that cannot allocate device memory:
+    the scratch is the library's fixed 32 MiB device array (see include/tp_block.h)."""
+    _check(load().tp_mlp_fwd_static_ws(ctypes.byref(desc), _ptr(x), _ptr(w1p), _ptr(w2p),
+                                       _ptr(residual), _ptr(y), _stream(stream)))
 
 
 def tp_mlp_unpack_grads(desc, dw1p, dw2p, dw1, dw_up, dw2, stream=None):
