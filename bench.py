@@ -343,7 +343,47 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
         ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
     if "attention" in which:
         ex["attention_block"] = extra_attention(tp, inputs, torch, stream, peaks, steps)
+    if "stack" in which:
+        ex["decode_stack"] = extra_stack(tp, torch, stream, peaks, steps)
     return ex
+
+
+def extra_stack(tp, torch, stream, peaks, steps):
+    """16 Llama-70B-shaped decode layers, b=1, KV length 4096, replayed as one CUDA graph."""
+    from tensor_transformer_matmul_b200.decode_stack import DecodeStack
+    c = STACK
+    st = DecodeStack(c["layers"], c["h"], c["F"], c["n_q"], c["n_kv"], c["hd"], c["p"],
+                     c["kv_len"], b=1, seed=0)
+    dev = torch.device("cuda", torch.cuda.current_device())
+    x = torch.randn(1, 1, c["h"], device=dev)   # float32 residual stream
+    st.capture(x)
+    for _ in range(3):
+        st.replay()
+    torch.cuda.synchronize()
+    ms = _cuda_time(st.replay, steps, stream) / steps
+    # eager steps with the event profiler: per-kernel split and per-reduction latency
+    tp.tp_reset_reduction_count()
+    prof = _profile(tp, lambda: st.step(x), max(3, steps // 4))
+    per_layer_w = (tp.tp_attn_wqkv_packed_bytes(st.adesc) + tp.tp_attn_wo_packed_bytes(st.adesc)
+                   + tp.tp_mlp_w1_packed_bytes(st.mdesc) + tp.tp_mlp_w2_packed_bytes(st.mdesc))
+    kv = 2 * c["n_kv"] * (c["kv_len"] + 1) * c["hd"] * 2
+    nbytes = c["layers"] * (per_layer_w + kv)
+    gbs = nbytes / (ms / 1e3) / 1e9
+    red = prof.get("reduce_partials", (0, 0.0))
+    out = {"workload": "decode stack: 16 layers (GQA attention s=1 over KV 4096+1, SwiGLU MLP "
+                       "d_ff=28672), b=1, p=8, 2 reductions of 1x8192 per layer, CUDA graph",
+           "ms_per_token": round(ms, 4), "tokens_per_s": round(1e3 / ms, 1),
+           "GB_per_s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
+           "bytes_per_step": nbytes,
+           "reductions_per_step": red[0] // max(1, max(3, steps // 4)),
+           "reduce_us_mean": round(red[1] / max(1, red[0]) * 1e3, 2),
+           "kernels": {k: {"launches_per_step": v[0] / max(3, steps // 4),
+                           "ms_per_step": round(v[1] / max(3, steps // 4), 4)}
+                       for k, v in prof.items()},
+           "steps": steps}
+    del st
+    torch.cuda.empty_cache()
+    return out
 
 
 def extra_prefill(tp, inputs, torch, stream, peaks, steps):

@@ -65,6 +65,12 @@ typedef enum { TP_ACT_IDENTITY = 0, TP_ACT_RELU = 1, TP_ACT_GELU = 2, TP_ACT_SWI
  *                       in the same order without writing them to memory.                      */
 typedef enum { TP_REDUCE_SEPARATE = 0, TP_REDUCE_FUSED = 1 } tp_reduce_mode;
 
+/* Descriptor flags.
+ *   TP_FLAG_F32_RESIDUAL: y and residual are float32 (a float32 residual stream) while x and the
+ *   weights stay in dtype.  The residual plus the sum of the partials is then rounded to fp32
+ *   instead of bf16, so a deep stack of bf16 layers never rounds its skip path to bf16. */
+#define TP_FLAG_F32_RESIDUAL 1
+
 /* ------------------------------------------------------------------------------------------ */
 /* MLP block                                                                                   */
 /* ------------------------------------------------------------------------------------------ */
@@ -77,6 +83,7 @@ typedef struct {
   int32_t act;          /* tp_act                                                             */
   int32_t dtype;        /* tp_dtype of x, weights, y, dy, dx                                  */
   int32_t reduce_mode;  /* tp_reduce_mode                                                     */
+  int32_t flags;        /* TP_FLAG_* (0 = none)                                               */
 } tp_mlp_desc;
 
 /* Packed layouts.  F_s = d_ff / p; F_sp = F_s rounded up to a multiple of 128 (padding rows and
@@ -168,7 +175,7 @@ typedef struct {
                            kv_len cached positions plus the new token                         */
   int64_t kv_cap;       /* slots per head in the caches (>= kv_len + 1); 0 means kv_len + 1  */
   int32_t reduce_mode;  /* tp_reduce_mode                                                     */
-  int32_t reserved;
+  int32_t flags;        /* TP_FLAG_* (0 = none)                                               */
 } tp_attn_desc;
 
 /* Packed layouts (element type dtype): qh = n_q/p, kh = n_kv/p, hd = head_dim,
@@ -207,9 +214,9 @@ tp_status tp_reduce_partials(const void* partials, int32_t p, int64_t n, int32_t
 
 /* Row-wise RMSNorm with unit weight: out = x / sqrt(mean(x^2) + eps), fp32 math, the
  * normalization that follows the residual add and stays replicated ("One collective").
- * x, out [rows][d] dtype (out may equal x). */
-tp_status tp_rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void* out,
-                     int32_t dtype, void* stream);
+ * x [rows][d] of x_dtype, out [rows][d] of out_dtype (out may equal x when the dtypes match). */
+tp_status tp_rmsnorm(const void* x, int32_t x_dtype, int64_t rows, int64_t d, float eps,
+                     void* out, int32_t out_dtype, void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
 /* Diagnostics                                                                                 */

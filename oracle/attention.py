@@ -89,6 +89,24 @@ def attention_forward(x, wq, wk, wv, wo, n_q, n_kv, head_dim, causal=True):
     return np.stack(ys)
 
 
+def attention_forward_rows(x, wq, wk, wv, wo, n_q, n_kv, head_dim, rows, causal=True):
+    """Rows ``rows`` (positions) of the unsharded block output for a single sequence x (s, h):
+    keys and values over every position, queries only at the chosen rows.  Each sampled output
+    row is computed over its full contraction, so it equals that row of attention_forward."""
+    x = _f64(x)
+    if x.ndim == 3:
+        x = x[0]
+    S = x.shape[0]
+    k = (x @ _f64(wk)).reshape(S, n_kv, head_dim)
+    v = (x @ _f64(wv)).reshape(S, n_kv, head_dim)
+    out = []
+    for r in rows:
+        q = (x[r:r + 1] @ _f64(wq)).reshape(1, n_q, head_dim)
+        o = attention_heads(q, k, v, n_q, n_kv, causal, q_pos0=r)
+        out.append(o @ _f64(wo))
+    return np.concatenate(out, axis=0)
+
+
 def attention_forward_sharded(x, wq, wk, wv, wo, n_q, n_kv, head_dim, p, causal=True):
     """Sharded reference mode (invariant tests only).
 

@@ -14,14 +14,14 @@ namespace tp {
 
 struct AttnLayout {
   int64_t b, s, h, tokens, kv_len, kv_cap;
-  int n_q, n_kv, hd, p, qh, kh, causal, dtype, eb;
+  int n_q, n_kv, hd, p, qh, kh, causal, dtype, eb, y_dtype;
   int64_t R_a;          // packed QKV rows per shard
   size_t wqkv_bytes, wo_bytes;
   size_t qkv_off, o_off, part_off, ml_off, ws_bytes;
   int kv_splits;        // decode: key chunks per (sequence, KV head)
 };
 
-constexpr int kDecodeChunk = 256;   // keys per decode work item
+constexpr int kDecodeChunk = 128;   // keys per decode work item
 
 inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (!d) return set_error(TP_ERR_INVALID_ARG, "desc is null");
@@ -36,12 +36,14 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (d->dtype != TP_F32 && d->dtype != TP_BF16) return set_error(TP_ERR_INVALID_ARG, "dtype");
   if (d->reduce_mode != TP_REDUCE_SEPARATE && d->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
+  if (d->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
   if (d->kv_len < 0) return set_error(TP_ERR_SHAPE, "kv_len must be >= 0");
   if (d->kv_len > 0 && d->s != 1) return set_error(TP_ERR_SHAPE, "decode (kv_len > 0) needs s == 1");
   L->b = d->b; L->s = d->s; L->h = d->h; L->tokens = d->b * d->s;
   L->n_q = d->n_q; L->n_kv = d->n_kv; L->hd = d->head_dim; L->p = d->p;
   L->qh = d->n_q / d->p; L->kh = d->n_kv / d->p;
   L->causal = d->causal ? 1 : 0; L->dtype = d->dtype; L->eb = elem_bytes(d->dtype);
+  L->y_dtype = (d->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : d->dtype;
   L->kv_len = d->kv_len;
   L->kv_cap = d->kv_cap > 0 ? d->kv_cap : d->kv_len + 1;
   if (L->kv_len > 0 && L->kv_cap < L->kv_len + 1)
@@ -189,70 +191,125 @@ __global__ void kv_append_kernel(const T* qkv, QkvIdx ix, T* kc, T* vc, int64_t 
   }
 }
 
-// Decode attention, split over keys.  Block = (split c, kv head g, sequence bi); its warps share
-// the chunk's keys; every query head of the group is handled in the same pass so each K/V row is
-// read once.  Output per (bi, q head, split): running max m, denominator l, unnormalised o[hd].
+// Decode attention, split over keys.  Block = (split c, kv head g, sequence bi); 8 warps share the
+// split's keys.  A group of HD/8 lanes handles one key: each lane holds 8 consecutive dims (one
+// 16-byte load of K and of V), so a warp covers 32/(HD/8) keys per pass and keeps kUnroll passes
+// of loads in flight.  Every query head of the KV group is handled in the same pass, so each K/V
+// row is read once.  Output per (bi, q head, split): running max m, denominator l and the
+// unnormalised o[hd].
 template <typename T, int GROUP, int HD>
 __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx ix, const T* kc,
                                                            const T* vc, int64_t kv_cap,
                                                            int64_t n_keys, int n_q, int n_kv,
                                                            float scale, float* ml) {
   constexpr int kWarps = 8;
-  constexpr int PER = HD / 32;           // dims per lane
+  constexpr int LPK = HD / 8;            // lanes per key
+  constexpr int KPW = 32 / LPK;          // keys per warp pass
+  constexpr int kUnroll = 4;
   __shared__ float s_m[kWarps][GROUP], s_l[kWarps][GROUP];
   __shared__ float s_o[kWarps][GROUP][HD];
   const int c = blockIdx.x, g = blockIdx.y;
   const int64_t bi = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int kslot = lane / LPK;          // which key of the pass this lane works on
+  const int d0 = (lane % LPK) * 8;       // first of this lane's 8 dims
   const int64_t k0 = static_cast<int64_t>(c) * kDecodeChunk;
   const int64_t k1 = min(n_keys, k0 + kDecodeChunk);
-  float q[GROUP][PER], acc[GROUP][PER], m[GROUP], l[GROUP];
+  float q[GROUP][8], acc[GROUP][8], m[GROUP], l[GROUP];
 #pragma unroll
   for (int a = 0; a < GROUP; ++a) {
     const int j = g * GROUP + a;
 #pragma unroll
-    for (int r = 0; r < PER; ++r) {
-      q[a][r] = to_f(qkv[ix.q(bi, j) + lane + 32 * r]) * scale;
-      acc[a][r] = 0.f;
+    for (int e = 0; e < 8; ++e) {
+      q[a][e] = to_f(qkv[ix.q(bi, j) + d0 + e]) * scale;
+      acc[a][e] = 0.f;
     }
     m[a] = -INFINITY;
     l[a] = 0.f;
   }
-  const T* kbase = kc + (bi * n_kv + g) * kv_cap * HD;
-  const T* vbase = vc + (bi * n_kv + g) * kv_cap * HD;
-  for (int64_t kp = k0 + warp; kp < k1; kp += kWarps) {
-    float kv[PER], vv[PER];
+  const T* kbase = kc + (bi * n_kv + g) * kv_cap * HD + d0;
+  const T* vbase = vc + (bi * n_kv + g) * kv_cap * HD + d0;
+  const int64_t stride = static_cast<int64_t>(kWarps) * KPW;
+  // the trip count depends on the warp only (every lane runs every pass: the shuffles below
+  // need the whole warp); lanes whose key is past the end mask themselves out with ok[]
+  for (int64_t wbase = k0 + warp * KPW; wbase < k1; wbase += stride * kUnroll) {
+    float kv[kUnroll][8], vv[kUnroll][8];
+    bool ok[kUnroll];
 #pragma unroll
-    for (int r = 0; r < PER; ++r) {
-      kv[r] = to_f(kbase[kp * HD + lane + 32 * r]);
-      vv[r] = to_f(vbase[kp * HD + lane + 32 * r]);
+    for (int u = 0; u < kUnroll; ++u) {
+      const int64_t kp = wbase + kslot + u * stride;
+      ok[u] = kp < k1;
+      if (ok[u]) {
+        if constexpr (sizeof(T) == 2) {
+          const uint4 wk = *reinterpret_cast<const uint4*>(kbase + kp * HD);
+          const uint4 wv = *reinterpret_cast<const uint4*>(vbase + kp * HD);
+          const uint32_t kw[4] = {wk.x, wk.y, wk.z, wk.w}, vw[4] = {wv.x, wv.y, wv.z, wv.w};
+#pragma unroll
+          for (int h2 = 0; h2 < 4; ++h2) {
+            kv[u][2 * h2] = bf16lo(kw[h2]); kv[u][2 * h2 + 1] = bf16hi(kw[h2]);
+            vv[u][2 * h2] = bf16lo(vw[h2]); vv[u][2 * h2 + 1] = bf16hi(vw[h2]);
+          }
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            kv[u][e] = to_f(kbase[kp * HD + e]);
+            vv[u][e] = to_f(vbase[kp * HD + e]);
+          }
+        }
+      }
     }
 #pragma unroll
-    for (int a = 0; a < GROUP; ++a) {
-      float dot = 0.f;
+    for (int u = 0; u < kUnroll; ++u) {
 #pragma unroll
-      for (int r = 0; r < PER; ++r) dot = fmaf(q[a][r], kv[r], dot);
+      for (int a = 0; a < GROUP; ++a) {
+        float dot = 0.f;
 #pragma unroll
-      for (int off = 16; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-      const float mn = fmaxf(m[a], dot);
-      const float corr = __expf(m[a] - mn), pw = __expf(dot - mn);
-      l[a] = l[a] * corr + pw;
+        for (int e = 0; e < 8; ++e) dot = fmaf(q[a][e], kv[u][e], dot);
 #pragma unroll
-      for (int r = 0; r < PER; ++r) acc[a][r] = acc[a][r] * corr + pw * vv[r];
+        for (int off = LPK / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
+        if (ok[u]) {
+          const float mn = fmaxf(m[a], dot);
+          const float corr = __expf(m[a] - mn), pw = __expf(dot - mn);
+          l[a] = l[a] * corr + pw;
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[a][e] = acc[a][e] * corr + pw * vv[u][e];
+          m[a] = mn;
+        }
+      }
+    }
+  }
+  // combine the warp's key slots (lanes that hold the same dims) with a fixed butterfly, then
+  // the warps in a fixed order: deterministic from run to run
+#pragma unroll
+  for (int a = 0; a < GROUP; ++a) {
+#pragma unroll
+    for (int off = LPK; off < 32; off <<= 1) {
+      const float mo = __shfl_xor_sync(0xffffffffu, m[a], off);
+      const float lo = __shfl_xor_sync(0xffffffffu, l[a], off);
+      const float mn = fmaxf(m[a], mo);
+      const float f1 = m[a] == -INFINITY ? 0.f : __expf(m[a] - mn);
+      const float f2 = mo == -INFINITY ? 0.f : __expf(mo - mn);
+      l[a] = l[a] * f1 + lo * f2;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) {
+        const float ao = __shfl_xor_sync(0xffffffffu, acc[a][e], off);
+        acc[a][e] = acc[a][e] * f1 + ao * f2;
+      }
       m[a] = mn;
     }
   }
+  if (lane < LPK) {
 #pragma unroll
-  for (int a = 0; a < GROUP; ++a) {
-    if (lane == 0) {
-      s_m[warp][a] = m[a];
-      s_l[warp][a] = l[a];
+    for (int a = 0; a < GROUP; ++a) {
+      if (lane == 0) {
+        s_m[warp][a] = m[a];
+        s_l[warp][a] = l[a];
+      }
+#pragma unroll
+      for (int e = 0; e < 8; ++e) s_o[warp][a][d0 + e] = acc[a][e];
     }
-#pragma unroll
-    for (int r = 0; r < PER; ++r) s_o[warp][a][lane + 32 * r] = acc[a][r];
   }
   __syncthreads();
-  // combine the warps: thread (a, e) for a < GROUP, e < HD
   for (int idx = threadIdx.x; idx < GROUP * HD; idx += blockDim.x) {
     const int a = idx / HD, e = idx - a * HD;
     float mm = -INFINITY;
@@ -448,7 +505,7 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
     if ((st = attn_core<float>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
     if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
   }
-  return reduce::launch(part, TP_F32, L.p, L.tokens * L.h, residual, y, L.dtype, s);
+  return reduce::launch(part, TP_F32, L.p, L.tokens * L.h, residual, y, L.y_dtype, s);
 }
 
 }  // namespace tp

@@ -104,11 +104,12 @@ inline tp_status launch(const void* part, int in_dtype, int p, int64_t n, const 
 }
 
 // out[r] = x[r] / sqrt(mean(x[r]^2) + eps), one block per row.
-template <typename T>
-__global__ void __launch_bounds__(256) rmsnorm_kernel(const T* x, int64_t d, float eps, T* out) {
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* x, int64_t d, float eps,
+                                                      Tout* out) {
   __shared__ float red[8];
-  const T* xr = x + blockIdx.x * d;
-  T* orow = out + blockIdx.x * d;
+  const Tin* xr = x + blockIdx.x * d;
+  Tout* orow = out + blockIdx.x * d;
   float ss = 0.f;
   for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
     const float v = to_f(xr[j]);
@@ -126,20 +127,26 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const T* x, int64_t d, flo
   }
   __syncthreads();
   const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
-  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) orow[j] = from_f<T>(to_f(xr[j]) * scale);
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) orow[j] = from_f<Tout>(to_f(xr[j]) * scale);
 }
 
-inline tp_status rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void* out, int dtype,
-                         cudaStream_t s) {
+template <typename Tin, typename Tout>
+inline void rmsnorm_launch(const void* x, int64_t rows, int64_t d, float eps, void* out,
+                           cudaStream_t s) {
+  rmsnorm_kernel<Tin, Tout><<<static_cast<unsigned>(rows), 256, 0, s>>>(
+      static_cast<const Tin*>(x), d, eps, static_cast<Tout*>(out));
+}
+
+inline tp_status rmsnorm(const void* x, int in_dtype, int64_t rows, int64_t d, float eps,
+                         void* out, int out_dtype, cudaStream_t s) {
   if (rows == 0) return TP_OK;
   if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
   ProfScope prof(s, "rmsnorm");
-  if (dtype == TP_BF16)
-    rmsnorm_kernel<__nv_bfloat16><<<static_cast<unsigned>(rows), 256, 0, s>>>(
-        static_cast<const __nv_bfloat16*>(x), d, eps, static_cast<__nv_bfloat16*>(out));
-  else
-    rmsnorm_kernel<float><<<static_cast<unsigned>(rows), 256, 0, s>>>(
-        static_cast<const float*>(x), d, eps, static_cast<float*>(out));
+  const bool ib = in_dtype == TP_BF16, ob = out_dtype == TP_BF16;
+  if (ib && ob) rmsnorm_launch<__nv_bfloat16, __nv_bfloat16>(x, rows, d, eps, out, s);
+  else if (ib) rmsnorm_launch<__nv_bfloat16, float>(x, rows, d, eps, out, s);
+  else if (ob) rmsnorm_launch<float, __nv_bfloat16>(x, rows, d, eps, out, s);
+  else rmsnorm_launch<float, float>(x, rows, d, eps, out, s);
   TP_LAUNCH_CHECK();
   return TP_OK;
 }

@@ -30,7 +30,7 @@ constexpr int stages_for(int bn, int a_sub) {
 
 struct MlpLayout {
   int64_t T, d, F, Fs, Fsp, R;
-  int p, act, dtype, eb;
+  int p, act, dtype, eb, y_dtype;
   size_t w1p_bytes, w2p_bytes;
   size_t saved_z_off, saved_h_off, saved_bytes;
   size_t fz_off, fh_off, fpart_off, fwd_ws;
@@ -49,6 +49,8 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
     return set_error(TP_ERR_INVALID_ARG, "dtype must be TP_F32 or TP_BF16");
   if (desc->reduce_mode != TP_REDUCE_SEPARATE && desc->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
+  if (desc->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  L->y_dtype = (desc->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : desc->dtype;
   L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
   L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
   L->Fs = L->F / L->p;
@@ -408,7 +410,7 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
   } else {
     if ((st = simt_forward<float>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
   }
-  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.dtype, s);
+  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.y_dtype, s);
   if (st == TP_OK) count_reduction();
   return st;
 }

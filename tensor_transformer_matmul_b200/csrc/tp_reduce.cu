@@ -19,12 +19,14 @@ extern "C" tp_status tp_reduce_partials(const void* partials, int32_t p, int64_t
   return st;
 }
 
-extern "C" tp_status tp_rmsnorm(const void* x, int64_t rows, int64_t d, float eps, void* out,
-                                int32_t dtype, void* stream) {
+extern "C" tp_status tp_rmsnorm(const void* x, int32_t x_dtype, int64_t rows, int64_t d,
+                                float eps, void* out, int32_t out_dtype, void* stream) {
   tp::clear_error();
   if (rows < 0 || d < 1) return tp::set_error(TP_ERR_SHAPE, "rows >= 0 and d >= 1 required");
-  if (dtype != TP_F32 && dtype != TP_BF16) return tp::set_error(TP_ERR_INVALID_ARG, "dtype");
+  if ((x_dtype != TP_F32 && x_dtype != TP_BF16) || (out_dtype != TP_F32 && out_dtype != TP_BF16))
+    return tp::set_error(TP_ERR_INVALID_ARG, "dtype");
   if (!(eps >= 0.f)) return tp::set_error(TP_ERR_INVALID_ARG, "eps must be >= 0");
   if (rows > 0 && (!x || !out)) return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
-  return tp::reduce::rmsnorm(x, rows, d, eps, out, dtype, static_cast<cudaStream_t>(stream));
+  return tp::reduce::rmsnorm(x, x_dtype, rows, d, eps, out, out_dtype,
+                             static_cast<cudaStream_t>(stream));
 }

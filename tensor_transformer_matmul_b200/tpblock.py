@@ -21,6 +21,7 @@ ACT = {"identity": 0, "relu": 1, "gelu": 2, "swiglu": 3}
 DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
 TORCH_OF = {TP_F32: torch.float32, TP_BF16: torch.bfloat16}
 TP_REDUCE_SEPARATE, TP_REDUCE_FUSED = 0, 1
+TP_FLAG_F32_RESIDUAL = 1
 
 # every symbol the header declares
 EXPORTS = (
@@ -43,7 +44,7 @@ class TpError(RuntimeError):
 class tp_mlp_desc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("d_ff", ctypes.c_int64),
                 ("p", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("reduce_mode", ctypes.c_int32)]
+                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 class tp_attn_desc(ctypes.Structure):
@@ -51,7 +52,7 @@ class tp_attn_desc(ctypes.Structure):
                 ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("p", ctypes.c_int32), ("causal", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("kv_len", ctypes.c_int64), ("kv_cap", ctypes.c_int64),
-                ("reduce_mode", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32)]
 
 
 _lib = None
@@ -81,7 +82,7 @@ def load():
         "tp_attn_pack": (I32, [AD, P, P, P, P, P, P, P]), "tp_attn_fwd_workspace": (S, [AD]),
         "tp_attn_fwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
         "tp_reduce_partials": (I32, [P, I32, I64, I32, P, P, I32, P]),
-        "tp_rmsnorm": (I32, [P, I64, I64, F32, P, I32, P]),
+        "tp_rmsnorm": (I32, [P, I32, I64, I64, F32, P, I32, P]),
         "tp_reduction_count": (ctypes.c_uint64, []), "tp_reset_reduction_count": (None, []),
         "tp_launch_count": (ctypes.c_uint64, []), "tp_last_error": (ctypes.c_char_p, []),
         "tp_status_string": (ctypes.c_char_p, [I32]), "tp_check_device_error": (I32, [P]),
@@ -133,9 +134,10 @@ def _nbytes(t):
 
 
 # ------------------------------------------------------------------------------------ MLP
-def mlp_desc(T, d, d_ff, p, act="swiglu", dtype="bf16", reduce_mode=TP_REDUCE_SEPARATE):
+def mlp_desc(T, d, d_ff, p, act="swiglu", dtype="bf16", reduce_mode=TP_REDUCE_SEPARATE, flags=0):
     return tp_mlp_desc(int(T), int(d), int(d_ff), int(p), ACT[act] if isinstance(act, str) else int(act),
-                       DTYPE[dtype] if isinstance(dtype, str) else int(dtype), int(reduce_mode))
+                       DTYPE[dtype] if isinstance(dtype, str) else int(dtype), int(reduce_mode),
+                       int(flags))
 
 
 def tp_mlp_w1_packed_bytes(desc):
@@ -189,10 +191,10 @@ def tp_mlp_unpack_grads(desc, dw1p, dw2p, dw1, dw_up, dw2, stream=None):
 
 # ------------------------------------------------------------------------------ attention
 def attn_desc(b, s, h, n_q, n_kv, head_dim, p, causal=True, dtype="bf16", kv_len=0, kv_cap=0,
-              reduce_mode=TP_REDUCE_SEPARATE):
+              reduce_mode=TP_REDUCE_SEPARATE, flags=0):
     return tp_attn_desc(int(b), int(s), int(h), int(n_q), int(n_kv), int(head_dim), int(p),
                         int(bool(causal)), DTYPE[dtype] if isinstance(dtype, str) else int(dtype),
-                        int(kv_len), int(kv_cap), int(reduce_mode), 0)
+                        int(kv_len), int(kv_cap), int(reduce_mode), int(flags))
 
 
 def tp_attn_wqkv_packed_bytes(desc):
@@ -228,9 +230,10 @@ def tp_reduce_partials(partials, p, n, out, residual=None, stream=None):
 
 
 def tp_rmsnorm(x, out, eps=1e-5, stream=None):
-    dt = TP_BF16 if x.dtype == torch.bfloat16 else TP_F32
+    xt = TP_BF16 if x.dtype == torch.bfloat16 else TP_F32
+    ot = TP_BF16 if out.dtype == torch.bfloat16 else TP_F32
     rows = x.numel() // x.shape[-1] if x.numel() else 0
-    _check(load().tp_rmsnorm(_ptr(x), int(rows), int(x.shape[-1]), float(eps), _ptr(out), dt,
+    _check(load().tp_rmsnorm(_ptr(x), xt, int(rows), int(x.shape[-1]), float(eps), _ptr(out), ot,
                              _stream(stream)))
 
 

@@ -64,3 +64,29 @@ class Mlp:
         dw2 = torch.empty(self.F, self.d, dtype=torch.float32, device=g)
         self.lib.tp_mlp_unpack_grads(self.desc, dw1p, dw2p, dw1, dwu, dw2)
         return dx, dw1, dwu, dw2, dw1p, dw2p
+
+
+class Attn:
+    """Packs one attention block's weights with the library and runs tp_attn_fwd."""
+
+    def __init__(self, lib, inp, p, dtype, causal=True, kv_len=0, n_q=None, n_kv=None, hd=None):
+        self.lib = lib
+        x = inp["x"]
+        self.b, self.s, self.h = x.shape
+        self.n_q, self.n_kv, self.hd = n_q, n_kv, hd
+        self.dtype = dtype
+        self.desc = lib.attn_desc(self.b, self.s, self.h, n_q, n_kv, hd, p, causal, dtype, kv_len)
+        tdt = inputs.TORCH_DTYPE[dtype]
+        eb = 2 if dtype == "bf16" else 4
+        g = dev()
+        self.wqkv = torch.empty(lib.tp_attn_wqkv_packed_bytes(self.desc) // eb, dtype=tdt, device=g)
+        self.wo = torch.empty(lib.tp_attn_wo_packed_bytes(self.desc) // eb, dtype=tdt, device=g)
+        lib.tp_attn_pack(self.desc, inp["wq"].to(g), inp["wk"].to(g), inp["wv"].to(g),
+                         inp["wo"].to(g), self.wqkv, self.wo)
+        self.ws = torch.empty(lib.tp_attn_fwd_workspace(self.desc), dtype=torch.uint8, device=g)
+
+    def forward(self, x, k_cache=None, v_cache=None, residual=None):
+        y = torch.empty(self.b, self.s, self.h, dtype=inputs.TORCH_DTYPE[self.dtype], device=dev())
+        self.lib.tp_attn_fwd(self.desc, x.to(dev()), self.wqkv, self.wo, y, k_cache=k_cache,
+                             v_cache=v_cache, residual=residual, workspace=self.ws)
+        return y

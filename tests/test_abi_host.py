@@ -123,7 +123,11 @@ def test_reduce_argument_errors(lib):
     assert so.tp_reduce_partials(fake, 2, -1, 0, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
     assert so.tp_reduce_partials(None, 2, 16, 0, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
     assert so.tp_reduce_partials(fake, 2, 16, 5, None, fake, 0, None) == lib.TP_ERR_INVALID_ARG
-    assert so.tp_rmsnorm(fake, 2, 0, 1e-5, fake, 0, None) == lib.TP_ERR_SHAPE
+    assert so.tp_rmsnorm(fake, 0, 2, 0, 1e-5, fake, 0, None) == lib.TP_ERR_SHAPE
+    assert so.tp_rmsnorm(fake, 3, 2, 8, 1e-5, fake, 0, None) == lib.TP_ERR_INVALID_ARG
+    bad = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32", flags=4)
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+                         None) == lib.TP_ERR_INVALID_ARG
 
 
 def test_empty_batch_counts_one_reduction(lib):

@@ -156,3 +156,17 @@ def test_full_size_prefill_mlp_sampled(lib):
     assert rel_l2(f64(dw1)[:, cols], s["dw1_cols"]) <= TOL["bf16"]
     assert rel_l2(f64(dwu)[:, cols], s["dw_up_cols"]) <= TOL["bf16"]
     assert rel_l2(f64(dw2)[w2rows], s["dw2_rows"]) <= TOL["bf16"]
+
+
+def test_f32_residual_stream(lib):
+    # TP_FLAG_F32_RESIDUAL: bf16 inputs and weights, float32 residual and output
+    T, d, F, p = 33, 256, 1024, 4
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=7, w_std=0.05)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    desc = lib.mlp_desc(T, d, F, p, "swiglu", "bf16", flags=lib.TP_FLAG_F32_RESIDUAL)
+    res = torch.randn(T, d, device=dev())
+    y = torch.empty(T, d, device=dev())
+    lib.tp_mlp_fwd(desc, inp["x"].to(dev()), m.w1p, m.w2p, y, residual=res, workspace=m.ws_f)
+    torch.cuda.synchronize()
+    assert y.dtype == torch.float32
+    assert rel_l2(f64(y), _oracle_fwd(inp, "swiglu") + f64(res)) <= TOL["bf16"]

@@ -145,3 +145,12 @@ def test_decode_layer_equals_prefill_layer_last_row():
     vc = (a[0, :L] @ w["wv"]).reshape(L, n_kv, hd).transpose(1, 0, 2)[None]
     out, _, _ = decode.decode_layer(xs[:, L], w, kc, vc, n_q, n_kv, hd)
     np.testing.assert_allclose(out, full[:, L], rtol=1e-12, atol=1e-13)
+
+
+def test_rows_match_full_forward():
+    n_q, n_kv, hd = 8, 2, 8
+    x, wq, wk, wv, wo = _case(1, 11, 32, n_q, n_kv, hd, seed=10)
+    full = attention.attention_forward(x, wq, wk, wv, wo, n_q, n_kv, hd, causal=True)[0]
+    rows = [0, 5, 10]
+    got = attention.attention_forward_rows(x, wq, wk, wv, wo, n_q, n_kv, hd, rows, causal=True)
+    np.testing.assert_allclose(got, full[rows], rtol=1e-12, atol=1e-13)
