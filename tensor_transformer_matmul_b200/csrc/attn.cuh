@@ -4,6 +4,7 @@
 
 #include <algorithm>
 
+#include "flash_attn.cuh"
 #include "gemm_launch.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
@@ -362,6 +363,14 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   attn::QkvIdx ix{L.p * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
   const float scale = 1.0f / sqrtf(static_cast<float>(L.hd));
   if (L.kv_len == 0) {
+    const bool tc = sizeof(T) == 2 && tensor_cores_usable() && (L.hd == 64 || L.hd == 128) &&
+                    L.s <= INT32_MAX && L.b <= 65535 && ceil_div(L.s, fa::kRows) <= 65535;
+    if (tc) {
+      const int group = L.n_q / L.n_kv;
+      if (L.hd == 128)
+        return fa::launch<128>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s);
+      return fa::launch<64>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s);
+    }
     const int64_t warps = L.tokens * L.n_q;
     const int64_t blocks = ceil_div(warps * 32, 128);
     if (blocks > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "attention grid too large");

@@ -36,6 +36,19 @@ def test_prefill_bf16(lib, causal, b, s, h, n_q, n_kv, hd, p):
     assert rel_l2(f64(y), _ref(inp, n_q, n_kv, hd, causal)) <= TOL["bf16"]
 
 
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("b,s,hd", [(2, 300, 128), (1, 257, 64), (3, 128, 128), (1, 1, 128)])
+def test_prefill_tensor_core_kernel(lib, causal, b, s, hd):
+    # head_dim 64/128 runs the tcgen05 flash kernel: several 128-row query tiles, ragged last
+    # tile, sequences packed back to back, a single-token sequence
+    h, n_q, n_kv, p = 256, 8, 2, 2
+    inp = inputs.attn_inputs(b, s, h, n_q, n_kv, hd, "bf16", seed=9, w_std=0.05)
+    a = Attn(lib, inp, p, "bf16", causal, n_q=n_q, n_kv=n_kv, hd=hd)
+    y = a.forward(inp["x"])
+    torch.cuda.synchronize()
+    assert rel_l2(f64(y), _ref(inp, n_q, n_kv, hd, causal)) <= TOL["bf16"]
+
+
 def test_prefill_fp32(lib):
     inp = inputs.attn_inputs(2, 21, 48, 6, 2, 8, "f32", seed=2, w_std=0.1)
     a = Attn(lib, inp, 2, "f32", True, n_q=6, n_kv=2, hd=8)
