@@ -208,14 +208,15 @@ def decode_mlp_bytes():
     part = c["p"] * c["T"] * c["d"] * 4
     y = c["T"] * c["d"] * 2
     return {"mlp_up_gemm": w1 + x + h, "mlp_down_gemm": w2 + h + part,
+            "mlp_down_gemm_fused": w2 + h + y,
             "reduce_partials": part + y, "step": w1 + w2 + x + y, "weights": w1 + w2, "Fs": Fs}
 
 
-def setup_mlp(tp, inputs, torch, cfg, backward=False, seed=0):
+def setup_mlp(tp, inputs, torch, cfg, backward=False, seed=0, reduce_mode=0):
     dev = torch.device("cuda", torch.cuda.current_device())
     inp = inputs.mlp_inputs(cfg["T"], cfg["d"], cfg["F"], "swiglu", "bf16", seed=seed,
                             device=dev, w_std=0.02, backward=backward)
-    desc = tp.mlp_desc(cfg["T"], cfg["d"], cfg["F"], cfg["p"], "swiglu", "bf16")
+    desc = tp.mlp_desc(cfg["T"], cfg["d"], cfg["F"], cfg["p"], "swiglu", "bf16", reduce_mode)
     st = {"desc": desc, "x": inp["x"], "dy": inp.get("dy")}
     st["w1p"] = torch.empty(tp.tp_mlp_w1_packed_bytes(desc) // 2, dtype=torch.bfloat16, device=dev)
     st["w2p"] = torch.empty(tp.tp_mlp_w2_packed_bytes(desc) // 2, dtype=torch.bfloat16, device=dev)
@@ -247,7 +248,8 @@ def run_ours(args, dist):
     peaks = _peaks()
     c = DECODE
 
-    st = setup_mlp(tp, inputs, torch, c, seed=dist.rank)
+    mode = tp.TP_REDUCE_FUSED if args.reduce_mode == "fused" else tp.TP_REDUCE_SEPARATE
+    st = setup_mlp(tp, inputs, torch, c, seed=dist.rank, reduce_mode=mode)
 
     def step():
         tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], workspace=st["ws"])
@@ -273,6 +275,8 @@ def run_ours(args, dist):
     # per-kernel durations, measured with events on the launching stream over K more steps
     prof = _profile(tp, step, args.steps)
     nbytes = decode_mlp_bytes()
+    if mode == tp.TP_REDUCE_FUSED:
+        nbytes["mlp_down_gemm"] = nbytes["mlp_down_gemm_fused"]
     dom = max(prof, key=lambda k: prof[k][1])
     dom_ms = prof[dom][1] / prof[dom][0]
     achieved = nbytes.get(dom, 0) / (dom_ms / 1e3) / 1e9
@@ -283,6 +287,8 @@ def run_ours(args, dist):
                 "algorithmic_bytes_per_launch": nbytes.get(dom, 0),
                 "kernel_ms": round(dom_ms, 5)}
     step_gbs = nbytes["step"] / (ms_step / 1e3) / 1e9
+    if mode == tp.TP_REDUCE_FUSED:
+        nbytes["mlp_down_gemm"] = nbytes["mlp_down_gemm_fused"]
     kernels = {k: {"launches_per_step": v[0] / args.steps, "ms_per_launch": round(v[1] / v[0], 5),
                    "GB_per_s": round(nbytes[k] / (v[1] / v[0] / 1e3) / 1e9, 1) if k in nbytes else None}
                for k, v in prof.items()}
@@ -312,6 +318,7 @@ def run_ours(args, dist):
         "data": "synthetic (seeded N(0,0.02) weights, N(0,1) activations, drawn on the GPU)",
         "config": {"workload": "decode TP SwiGLU MLP: T=64 (batch 64, s=1), d=8192, d_ff=28672, "
                                "p=8 logical shards, bf16, fp32 accumulate",
+                   "reduce_mode": args.reduce_mode,
                    "global_batch": c["T"] * dist.world, "seq_len": 1,
                    "parallelism": f"replicas x{dist.world} (p=8 logical shards per GPU)",
                    "l2": "inputs larger than L2: 1.41 GB of weights streamed per step",
@@ -344,16 +351,17 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     if "attention" in which:
         ex["attention_block"] = extra_attention(tp, inputs, torch, stream, peaks, steps)
     if "stack" in which:
-        ex["decode_stack"] = extra_stack(tp, torch, stream, peaks, steps)
+        ex["decode_stack"] = extra_stack(tp, torch, stream, peaks, steps, args.reduce_mode)
     return ex
 
 
-def extra_stack(tp, torch, stream, peaks, steps):
+def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
     """16 Llama-70B-shaped decode layers, b=1, KV length 4096, replayed as one CUDA graph."""
     from tensor_transformer_matmul_b200.decode_stack import DecodeStack
     c = STACK
     st = DecodeStack(c["layers"], c["h"], c["F"], c["n_q"], c["n_kv"], c["hd"], c["p"],
-                     c["kv_len"], b=1, seed=0)
+                     c["kv_len"], b=1, seed=0,
+                     reduce_mode=tp.TP_REDUCE_FUSED if reduce_mode == "fused" else tp.TP_REDUCE_SEPARATE)
     dev = torch.device("cuda", torch.cuda.current_device())
     x = torch.randn(1, 1, c["h"], device=dev)   # float32 residual stream
     st.capture(x)
@@ -553,6 +561,8 @@ def main():
     ap.add_argument("--extra-steps", type=int, default=20)
     ap.add_argument("--extras", default="prefill,attention,stack",
                     help="comma list of extra workloads to measure at N=1")
+    ap.add_argument("--reduce-mode", choices=["separate", "fused"], default="separate",
+                    help="how the p partial sums are added in the decode workloads")
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     args = ap.parse_args()
     args.warmup = max(3, args.warmup)

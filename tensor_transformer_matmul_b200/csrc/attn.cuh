@@ -18,9 +18,49 @@ struct AttnLayout {
   int n_q, n_kv, hd, p, qh, kh, causal, dtype, eb, y_dtype;
   int64_t R_a;          // packed QKV rows per shard
   size_t wqkv_bytes, wo_bytes;
-  size_t qkv_off, o_off, part_off, ml_off, ws_bytes;
+  size_t qkv_off, o_off, part_off, ml_off, sk_off, ws_bytes;
   int kv_splits;        // decode: key chunks per (sequence, KV head)
+  int reduce_mode;
+  bool tc;              // bf16 with 16-byte rows: tensor-core projections
 };
+
+namespace attn_tc {
+using tc::Operand;
+template <int BN, int ASUB>
+using KK = tc::TileCfg<BN, ASUB, false, false,
+                       std::min(8, (200 * 1024) / (128 * ASUB * 64 * 2 + BN * 64 * 2))>;
+template <class C> struct Tag { using type = C; };
+constexpr int64_t kSwapMaxT = 128;
+template <class F>
+auto by_tokens(int64_t T, F&& f) {
+  if (T <= 16) return f(Tag<KK<16, 1>>{});
+  if (T <= 64) return f(Tag<KK<64, 1>>{});
+  return f(Tag<KK<128, 1>>{});
+}
+}  // namespace attn_tc
+
+inline int64_t qkv_tiles(const AttnLayout& L) { return ceil_div(L.p * L.R_a, 128); }
+inline int64_t out_tiles(const AttnLayout& L) { return L.p * ceil_div(L.h, 128); }
+
+// stream-K bytes of the QKV projection and of the output projection (0 when not stream-K)
+inline size_t attn_sk_bytes(const AttnLayout& L) {
+  using namespace attn_tc;
+  if (!L.tc || L.tokens == 0) return 0;
+  const int64_t rows = L.p * L.R_a, K = static_cast<int64_t>(L.qh) * L.hd;
+  const bool fused = L.reduce_mode == TP_REDUCE_FUSED;
+  size_t a = 0, b = 0;
+  if (L.tokens <= kSwapMaxT) {
+    if (decode_stream_k(qkv_tiles(L))) a = by_tokens(L.tokens, [&](auto t) {
+      return tc::plan_stream_k<typename decltype(t)::type>(rows, L.tokens, L.h, 1, false, num_sms()).bytes();
+    });
+    if (decode_stream_k(out_tiles(L)) || fused) b = by_tokens(L.tokens, [&](auto t) {
+      return tc::plan_stream_k<typename decltype(t)::type>(L.h, L.tokens, K, L.p, fused, num_sms()).bytes();
+    });
+  } else if (fused) {
+    b = tc::plan_stream_k<KK<256, 1>>(L.tokens, L.h, K, L.p, true, num_sms()).bytes();
+  }
+  return std::max(a, b);
+}
 
 constexpr int kDecodeChunk = 128;   // keys per decode work item
 
@@ -59,11 +99,15 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   const size_t partb = static_cast<size_t>(P * L->tokens * L->h) * 4;
   // decode split-KV scratch: per (sequence, q head, split) an (m, l) pair and hd outputs
   const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (2 + L->hd) * 4;
+  L->reduce_mode = d->reduce_mode;
+  L->tc = d->dtype == TP_BF16 && d->h % 8 == 0;
   L->qkv_off = 0;
   L->o_off = align256(qkvb);
   L->part_off = L->o_off + align256(ob);
-  L->ml_off = L->part_off + align256(partb);
-  L->ws_bytes = L->ml_off + align256(mlb);
+  const size_t pb = (L->tc && L->reduce_mode == TP_REDUCE_FUSED) ? 0 : partb;
+  L->ml_off = L->part_off + align256(pb);
+  L->sk_off = L->ml_off + align256(mlb);
+  L->ws_bytes = L->sk_off + align256(attn_sk_bytes(*L));
   return TP_OK;
 }
 
@@ -417,13 +461,9 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
 }
 
 namespace attn_tc {
-using tc::Operand;
-template <int BN, int ASUB>
-using KK = tc::TileCfg<BN, ASUB, false, false,
-                       std::min(8, (200 * 1024) / (128 * ASUB * 64 * 2 + BN * 64 * 2))>;
 
 inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, void* qkv,
-                          cudaStream_t s) {
+                          void* sk_ws, size_t sk_bytes, cudaStream_t s) {
   const int64_t rows = L.p * L.R_a;
   tc::EpiHidden::Params ep;
   ep.h = static_cast<__nv_bfloat16*>(qkv);
@@ -435,32 +475,67 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
   ep.act = TP_ACT_IDENTITY;
   const Operand xo{x, false, L.tokens, L.h, 1, L.h, 0};
   const Operand wo{wqkv, false, rows, L.h, 1, L.h, 0};
-  if (L.tokens <= 128) {
+  if (L.tokens <= kSwapMaxT) {
     ep.swap = 1;
-    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
-    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
-    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1, ep, s, "attn_qkv_gemm");
+    const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = decode_stream_k(qkv_tiles(L)) ? &sk : nullptr;
+    opt.rotate_k = true;
+    return by_tokens(L.tokens, [&](auto t) {
+      return tc::run_gemm<typename decltype(t)::type, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1,
+                                                                     ep, s, "attn_qkv_gemm", opt);
+    });
   }
   ep.swap = 0;
   return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s, "attn_qkv_gemm");
 }
 
-inline tp_status out_proj_partials(const AttnLayout& L, const void* o, const void* wo_p,
-                                   float* part, cudaStream_t s) {
+// Row-parallel output projection: fp32 partials [p][tokens][h] (separate reduce), or the fused
+// in-order sum plus residual written straight to y.
+inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, float* part,
+                          const void* residual, void* y, void* sk_ws, size_t sk_bytes,
+                          cudaStream_t s) {
   const int64_t K = static_cast<int64_t>(L.qh) * L.hd;
   const Operand ao{o, false, L.tokens, K, L.p, static_cast<int64_t>(L.n_q) * L.hd, K};
   const Operand wo{wo_p, false, L.h, K, L.p, K, L.h * K};
+  const bool swap = L.tokens <= kSwapMaxT;
+  if (L.reduce_mode == TP_REDUCE_FUSED) {
+    tc::EpiReduceOut::Params ep;
+    ep.out = y;
+    ep.residual = residual;
+    ep.ld = L.h;
+    ep.rows_valid = static_cast<int32_t>(L.tokens);
+    ep.cols_valid = static_cast<int32_t>(L.h);
+    ep.out_bf16 = L.y_dtype == TP_BF16 ? 1 : 0;
+    ep.swap = swap ? 1 : 0;
+    const tc::StreamKArgs sk{true, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = &sk;
+    opt.rotate_k = swap;
+    if (swap)
+      return by_tokens(L.tokens, [&](auto t) {
+        return tc::run_gemm<typename decltype(t)::type, tc::EpiReduceOut>(
+            wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm", opt);
+      });
+    return tc::run_gemm<KK<256, 1>, tc::EpiReduceOut>(ao, wo, L.tokens, L.h, K, L.p, ep, s,
+                                                       "attn_out_gemm", opt);
+  }
   tc::EpiStoreF32::Params ep;
   ep.out = part;
   ep.ld = L.h;
   ep.batch_stride = L.tokens * L.h;
   ep.rows_valid = static_cast<int32_t>(L.tokens);
   ep.cols_valid = static_cast<int32_t>(L.h);
-  if (L.tokens <= 128) {
+  if (swap) {
     ep.swap = 1;
-    if (L.tokens <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
-    if (L.tokens <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
-    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm");
+    const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = decode_stream_k(out_tiles(L)) ? &sk : nullptr;
+    opt.rotate_k = true;
+    return by_tokens(L.tokens, [&](auto t) {
+      return tc::run_gemm<typename decltype(t)::type, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p,
+                                                                       ep, s, "attn_out_gemm", opt);
+    });
   }
   ep.swap = 0;
   return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s, "attn_out_gemm");
@@ -497,14 +572,18 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
   float* part = reinterpret_cast<float*>(w + L.part_off);
   float* ml = reinterpret_cast<float*>(w + L.ml_off);
   tp_status st;
-  const bool tc_ok = L.dtype == TP_BF16 && L.h % 8 == 0 && tensor_cores_usable();
-  if (tc_ok) {
+  if (L.tc) {
+    if (!tensor_cores_usable())
+      return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {x, wqkv, wo_p, residual, static_cast<const void*>(y)})
       if (q && (reinterpret_cast<uintptr_t>(q) & 15))
         return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, s)) != TP_OK) return st;
+    void* sk = w + L.sk_off;
+    const size_t skb = L.ws_bytes - L.sk_off;
+    if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, sk, skb, s)) != TP_OK) return st;
     if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
-    if ((st = attn_tc::out_proj_partials(L, o, wo_p, part, s)) != TP_OK) return st;
+    if ((st = attn_tc::out_proj(L, o, wo_p, part, residual, y, sk, skb, s)) != TP_OK) return st;
+    if (L.reduce_mode == TP_REDUCE_FUSED) return TP_OK;
   } else if (L.dtype == TP_BF16) {
     if ((st = attn_simt_proj<__nv_bfloat16>(L, x, wqkv, qkv, o, wo_p, part, s, true)) != TP_OK) return st;
     if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;

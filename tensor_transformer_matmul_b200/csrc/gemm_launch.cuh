@@ -3,6 +3,7 @@
 
 #include <cuda.h>
 #include <algorithm>
+#include <vector>
 
 #include "gemm_tc.cuh"
 #include "tp_common.cuh"
@@ -41,11 +42,80 @@ inline tp_status encode_operand(CUtensorMap* map, const Operand& o, int tile_mn)
   return encode_tmap_bf16_3d(map, o.ptr, o.mn_ext, o.k_ext, o.batch, rs, bs, 64, 64);
 }
 
+// Stream-K schedule of one GEMM: every CTA gets an equal contiguous range of the k-blocks of all
+// output tiles.  Computed on the host by walking each CTA's segments exactly as the kernel does.
+struct SkPlan {
+  int grid = 0;             // CTAs (<= SMs, <= k-blocks)
+  int slots_per_cta = 0;    // partial-tile slots per CTA
+  int max_group_segs = 0;   // most segments any output tile is cut into
+  int64_t units = 0;        // k-blocks over all output tiles
+  int64_t groups = 0;       // output tiles
+  size_t counter_bytes = 0; // arrival counters (256-aligned)
+  size_t slot_bytes = 0;    // partial slots
+  size_t bytes() const { return counter_bytes + slot_bytes; }
+};
+
+template <class Cfg>
+SkPlan plan_stream_k(int64_t M, int64_t N, int64_t K, int64_t batch, bool sum_batch, int sms) {
+  SkPlan pl;
+  const int64_t mb = ceil_div(M, Cfg::A_ROWS), nb = ceil_div(N, Cfg::BN), kb = ceil_div(K, kBK);
+  if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return pl;
+  pl.groups = sum_batch ? mb * nb : batch * mb * nb;
+  const int64_t U = sum_batch ? batch * kb : kb;
+  pl.units = pl.groups * U;
+  std::vector<int> per_group(static_cast<size_t>(pl.groups), 0);
+  // fewer, longer ranges when a tile would otherwise be cut into too many segments (tiny
+  // problems spread over many SMs)
+  for (int grid = static_cast<int>(std::min<int64_t>(sms, pl.units)); grid >= 1; grid = grid / 2) {
+    std::fill(per_group.begin(), per_group.end(), 0);
+    int spc = 0;
+    for (int c = 0; c < grid; ++c) {
+      int64_t u = static_cast<int64_t>(c) * pl.units / grid;
+      const int64_t end = static_cast<int64_t>(c + 1) * pl.units / grid;
+      int n = 0;
+      while (u < end) {
+        const int64_t g = u / U, o = u - g * U;
+        const int64_t lim = sum_batch ? (o / kb + 1) * kb : U;
+        const int64_t seg_end = std::min(lim, end - g * U);
+        ++n;
+        ++per_group[static_cast<size_t>(g)];
+        u = g * U + seg_end;
+      }
+      spc = std::max(spc, n);
+    }
+    int mx = 0;
+    for (int v : per_group) mx = std::max(mx, v);
+    pl.grid = grid;
+    pl.slots_per_cta = spc;
+    pl.max_group_segs = mx;
+    if (mx <= kMaxGroupSegs || grid == 1) break;
+  }
+  pl.counter_bytes = align256(static_cast<size_t>(pl.groups) * sizeof(int32_t));
+  pl.slot_bytes = static_cast<size_t>(pl.grid) * pl.slots_per_cta * Cfg::SLOT_FLOATS * sizeof(float);
+  return pl;
+}
+
+// Where a stream-K launch keeps its counters and partial slots.
+struct StreamKArgs {
+  bool sum_batch;     // add the problems (shards) into one output: the fused reduce
+  void* ws;           // at least plan_stream_k(...).bytes(), 256-byte aligned
+  size_t ws_bytes;
+};
+
+// Launch options beyond the shapes.
+struct GemmOpts {
+  const StreamKArgs* sk = nullptr;   // stream-K schedule (else whole tiles)
+  bool rotate_k = false;             // tile-dependent k-loop start (weight streaming)
+};
+
 // Launch gemm_kernel<Cfg, Epi> over ``batch`` problems of D = A B^T (M x N, contraction K).
+// With ``sk`` the stream-K schedule is used (and its counters are zeroed on the stream first).
 template <class Cfg, class Epi>
 tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int64_t K,
                    int64_t batch, const typename Epi::Params& ep, cudaStream_t stream,
-                   const char* label = "gemm", int m_fastest = -1) {
+                   const char* label = "gemm", const GemmOpts& opts = GemmOpts(),
+                   int m_fastest = -1) {
+  const StreamKArgs* sk = opts.sk;
   static_assert(Cfg::A_MN == false || Cfg::A_ROWS % 64 == 0, "A tile");
   if (a.mn_major != Cfg::A_MN || b.mn_major != Cfg::B_MN)
     return set_error(TP_ERR_INVALID_ARG, "operand major does not match the tile config");
@@ -71,6 +141,29 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   gp.b_batched = b.batch > 1 ? 1 : 0;
   gp.err = device_error_word();
   if (gp.k_blocks == 0) return set_error(TP_ERR_INVALID_ARG, "GEMM with K == 0");
+  gp.stream_k = 0;
+  gp.sum_batch = 0;
+  gp.units = 0;
+  gp.slots_per_cta = 0;
+  gp.slots = nullptr;
+  gp.counters = nullptr;
+  gp.rotate_k = opts.rotate_k ? 1 : 0;
+  int grid_sk = 0;
+  if (sk) {
+    const SkPlan pl = plan_stream_k<Cfg>(M, N, K, batch, sk->sum_batch, num_sms());
+    if (pl.max_group_segs > kMaxGroupSegs)
+      return set_error(TP_ERR_UNSUPPORTED, "stream-K: an output tile would need too many segments");
+    if (!sk->ws || sk->ws_bytes < pl.bytes())
+      return set_error(TP_ERR_WORKSPACE, "stream-K workspace too small");
+    gp.stream_k = 1;
+    gp.sum_batch = sk->sum_batch ? 1 : 0;
+    gp.units = pl.units;
+    gp.slots_per_cta = pl.slots_per_cta;
+    gp.counters = static_cast<int32_t*>(sk->ws);
+    gp.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(sk->ws) + pl.counter_bytes);
+    grid_sk = pl.grid;
+    TP_CUDA_TRY(cudaMemsetAsync(sk->ws, 0, pl.counter_bytes, stream));
+  }
 
   static int attr_set[64] = {0};
   int dev = 0;
@@ -82,7 +175,7 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
     attr_set[dev] = 1;
   }
   const int64_t tiles = static_cast<int64_t>(gp.batch) * gp.m_blocks * gp.n_blocks;
-  const int grid = static_cast<int>(std::min<int64_t>(tiles, num_sms()));
+  const int grid = sk ? grid_sk : static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   ProfScope prof(stream, label);
   gemm_kernel<Cfg, Epi><<<grid, kThreads, Cfg::SMEM_BYTES, stream>>>(ta, tb, gp, ep);
   TP_LAUNCH_CHECK();

@@ -5,10 +5,19 @@
 // Roles (192 threads):  warp 0 lane 0 -- TMA producer: fills a ring of shared-memory stages;
 //                       warp 1 lane 0 -- MMA issuer: tcgen05.mma into one of two TMEM
 //                                        accumulators, frees stages with tcgen05.commit;
-//                       warps 2..5    -- epilogue: tcgen05.ld the accumulator, apply the fused
+//                       warps 2..5    -- epilogue: read the accumulator, apply the fused
 //                                        elementwise step, store to global memory.
-// Tiles are walked persistently (tile = blockIdx.x + i * gridDim.x), so the epilogue of one tile
-// overlaps the main loop of the next.
+//
+// Work is cut into segments, each one accumulator's worth of k-blocks.  Two schedules:
+//   * tiles: segment = one whole output tile (all of K); tile = blockIdx.x + i * gridDim.x.
+//   * stream-K: the k-blocks of all tiles, in order, are split into gridDim.x equal contiguous
+//     ranges, one per CTA, so every SM streams the same number of k-blocks.  A tile whose
+//     k-blocks fall in several segments ("split") is finished by whichever CTA arrives last:
+//     each writes its fp32 partial to a slot, and the last one adds the slots in k order and
+//     applies the epilogue.  No CTA ever waits for another.
+//   With sum_batch, the problem index (the shard) is part of the k space of an output tile:
+//   each shard's k-range is its own segment, and the finishing CTA adds the shards' partial
+//   tiles in shard order 0..p-1 -- the partial-sum reduce fused into the GEMM.
 //
 // Operands are 3-D TMA tensors (inner, outer, batch) with 128-byte swizzle.  A K-major operand has
 // K as its inner dimension (box 64 x rows); an MN-major operand has M (or N) as its inner
@@ -34,6 +43,7 @@ constexpr int kBK = 64;          // K per stage: 64 bf16 = one 128-byte swizzle 
 constexpr int kUmmaK = 16;       // K per tcgen05.mma (kind::f16)
 constexpr int kThreads = 192;
 constexpr int kEpiWarps = 4;
+constexpr int kMaxGroupSegs = 16;   // segments one split tile may have (checked on the host)
 
 // Compile-time tile configuration.
 //   BN     : N of each MMA (columns of the accumulator), 16..256, multiple of 16
@@ -55,9 +65,10 @@ struct TileCfg {
   static constexpr int ACC_COLS = A_SUB * BN;
   static constexpr int TMEM_COLS = (2 * ACC_COLS <= 32) ? 32 : (2 * ACC_COLS <= 64) ? 64
                                    : (2 * ACC_COLS <= 128) ? 128 : (2 * ACC_COLS <= 256) ? 256 : 512;
-  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 16;
+  static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 32;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
   static constexpr uint32_t IDESC = sm100::make_idesc_bf16(128, BN, A_MN, B_MN);
+  static constexpr int SLOT_FLOATS = 128 * ACC_COLS;   // one partial accumulator tile
   static_assert(BN % 16 == 0 && BN >= 16 && BN <= 256, "UMMA N for M=128 is 16..256 step 16");
   static_assert(A_SUB == 1 || A_SUB == 2, "A_SUB");
   static_assert(2 * ACC_COLS <= 512, "two accumulators must fit in TMEM");
@@ -72,22 +83,39 @@ struct GemmParams {
   int32_t m_fastest;      // tile order: walk M blocks first (1) or N blocks first (0)
   int32_t a_batched, b_batched;  // operand's batch coordinate = problem index (else 0)
   uint32_t* err;          // device error word
+  // stream-K schedule
+  int32_t stream_k;       // 0: whole tiles; 1: equal contiguous k-block ranges per CTA
+  int32_t sum_batch;      // stream-K: the problems are summed into one output (fused reduce)
+  int64_t units;          // total k-blocks over all output tiles
+  int32_t slots_per_cta;  // partial-tile slots reserved per CTA
+  float* slots;           // [gridDim.x][slots_per_cta][SLOT_FLOATS]
+  int32_t* counters;      // [output tiles] arrivals of split tiles (zero before the launch)
+  // Start each segment's k loop at a tile-dependent k-block (wrapping around).  Weight-streaming
+  // GEMMs set it: concurrent CTAs then read different column offsets of their row-major tiles,
+  // which spreads the loads over the HBM channels instead of having every CTA hit the same
+  // offset within the row pitch at the same moment.
+  int32_t rotate_k;
+};
+
+// One accumulator's worth of work.
+struct Seg {
+  int g;          // output tile (group)
+  int b;          // problem of this segment (for operand coordinates)
+  int mb, nb;     // tile coordinates in blocks
+  int kb0, kb1;   // k-block range
+  int local;      // index of this segment within its CTA (slot index)
+  int rot;        // the k loop visits kb0 + (i + rot) % (kb1 - kb0), i = 0, 1, ...
 };
 
 // What the epilogue of one tile sees.
 struct EpiCtx {
-  uint32_t taddr;   // TMEM address: this warp's 32 lanes, column 0 of the tile's accumulator
   int row;          // accumulator row (A row within the tile) held by this thread, 0..127
-  int b;            // problem index
+  int b;            // problem index (0 when the problems were summed)
   int m0;           // first A row of the tile
   int n0;           // first B row of the tile
 };
 
-__device__ __forceinline__ void decode_tile(int t, const GemmParams& gp, int& b, int& mb,
-                                            int& nb) {
-  const int per = gp.m_blocks * gp.n_blocks;
-  b = t / per;
-  const int r = t - b * per;
+__device__ __forceinline__ void decode_mn(int r, const GemmParams& gp, int& mb, int& nb) {
   if (gp.m_fastest) {
     mb = r % gp.m_blocks;
     nb = r / gp.m_blocks;
@@ -95,6 +123,100 @@ __device__ __forceinline__ void decode_tile(int t, const GemmParams& gp, int& b,
     nb = r % gp.n_blocks;
     mb = r / gp.n_blocks;
   }
+}
+
+__device__ __forceinline__ int64_t units_per_group(const GemmParams& gp) {
+  return gp.sum_batch ? static_cast<int64_t>(gp.batch) * gp.k_blocks : gp.k_blocks;
+}
+__device__ __forceinline__ int num_groups(const GemmParams& gp) {
+  return gp.sum_batch ? gp.m_blocks * gp.n_blocks : gp.batch * gp.m_blocks * gp.n_blocks;
+}
+__device__ __forceinline__ int64_t cta_start(int c, const GemmParams& gp, int grid) {
+  return static_cast<int64_t>(c) * gp.units / grid;
+}
+// the CTA whose range holds unit u (the largest c with cta_start(c) <= u)
+__device__ __forceinline__ int cta_of(int64_t u, const GemmParams& gp, int grid) {
+  const int64_t c = ((u + 1) * grid + gp.units - 1) / gp.units - 1;
+  return static_cast<int>(c < grid - 1 ? c : grid - 1);
+}
+
+// Segment iterator over one CTA's work (both schedules); all roles walk the same sequence.
+struct SegIter {
+  int64_t u, end;   // stream-K: unit cursor and end; tiles: tile cursor and count
+  int local;
+  __device__ __forceinline__ void init(const GemmParams& gp, int cta, int grid) {
+    local = 0;
+    if (gp.stream_k) {
+      u = cta_start(cta, gp, grid);
+      end = cta_start(cta + 1, gp, grid);
+    } else {
+      u = cta;
+      end = num_groups(gp);
+    }
+  }
+  __device__ __forceinline__ bool next(const GemmParams& gp, int grid, Seg& s) {
+    if (u >= end) return false;
+    if (!gp.stream_k) {
+      const int per = gp.m_blocks * gp.n_blocks;
+      s.g = static_cast<int>(u);
+      s.b = s.g / per;
+      decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
+      s.kb0 = 0;
+      s.kb1 = gp.k_blocks;
+      s.local = local++;
+      s.rot = gp.rotate_k ? static_cast<int>((static_cast<int64_t>(s.g) * 37) % gp.k_blocks) : 0;
+      u += grid;
+      return true;
+    }
+    const int64_t U = units_per_group(gp);
+    const int64_t g = u / U, o = u - g * U;
+    s.g = static_cast<int>(g);
+    int64_t lim;
+    if (gp.sum_batch) {
+      s.b = static_cast<int>(o / gp.k_blocks);
+      s.kb0 = static_cast<int>(o - static_cast<int64_t>(s.b) * gp.k_blocks);
+      lim = static_cast<int64_t>(s.b + 1) * gp.k_blocks;
+      decode_mn(s.g, gp, s.mb, s.nb);
+    } else {
+      const int per = gp.m_blocks * gp.n_blocks;
+      s.b = s.g / per;
+      decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
+      s.kb0 = static_cast<int>(o);
+      lim = U;
+    }
+    const int64_t seg_end = lim < end - g * U ? lim : end - g * U;
+    s.kb1 = s.kb0 + static_cast<int>(seg_end - o);
+    s.local = local++;
+    s.rot = gp.rotate_k ? static_cast<int>((static_cast<int64_t>(s.g) * 37) % (s.kb1 - s.kb0)) : 0;
+    u = g * U + seg_end;
+    return true;
+  }
+};
+
+// All segments of output tile g, in k order: slot pointer and problem index of each.  Returns the
+// count (0 if more than kMaxGroupSegs, which the host rules out).
+template <int SLOT_FLOATS>
+__device__ __forceinline__ int group_segments(const GemmParams& gp, int grid, int g,
+                                              const float* (&ptr)[kMaxGroupSegs],
+                                              int (&bs)[kMaxGroupSegs]) {
+  const int64_t U = units_per_group(gp);
+  const int c0 = cta_of(static_cast<int64_t>(g) * U, gp, grid);
+  const int c1 = cta_of(static_cast<int64_t>(g) * U + U - 1, gp, grid);
+  int n = 0;
+  for (int c = c0; c <= c1; ++c) {
+    SegIter it;
+    it.init(gp, c, grid);
+    Seg s;
+    while (it.next(gp, grid, s)) {
+      if (s.g < g) continue;
+      if (s.g > g) break;
+      if (n == kMaxGroupSegs) return 0;
+      ptr[n] = gp.slots + (static_cast<int64_t>(c) * gp.slots_per_cta + s.local) * SLOT_FLOATS;
+      bs[n] = s.b;
+      ++n;
+    }
+  }
+  return n;
 }
 
 // Bounded wait used on the abort path only: ignores the abort flag.
@@ -108,6 +230,89 @@ __device__ __forceinline__ bool drain_wait(uint64_t* bar, uint32_t parity, uint3
   }
   return true;
 }
+
+// barrier among the four epilogue warps (barrier 0 is __syncthreads)
+__device__ __forceinline__ void epi_bar() { asm volatile("bar.sync 1, 128;" ::: "memory"); }
+// the same barrier, returning the AND of v over the 128 epilogue threads
+__device__ __forceinline__ int epi_bar_and(int v) {
+  int r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, 128, p;\n\t"
+      "selp.s32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(r)
+      : "r"(v)
+      : "memory");
+  return r;
+}
+
+// ---------------------------------------------------------------------------------------------
+// Accumulator value sources for the epilogues
+// ---------------------------------------------------------------------------------------------
+// From TMEM: 32 lanes x consecutive fp32 columns (warp-collective).
+struct TmemSrc {
+  uint32_t taddr;   // this warp's 32 lanes, column 0 of the tile's accumulator
+  __device__ __forceinline__ void load32(int col, float (&v)[32]) const {
+    uint32_t r[32];
+    sm100::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(col), r);
+    sm100::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
+  }
+  __device__ __forceinline__ void load16(int col, float (&v)[16]) const {
+    uint32_t r[16];
+    sm100::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(col), r);
+    sm100::tmem_wait_ld();
+#pragma unroll
+    for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
+  }
+};
+
+// From the partial slots of a split tile: the sum over its segments, in k order; with several
+// problems (shards), each shard's segments are added first, then the shards in order.
+template <int ACC_COLS>
+struct FixupSrc {
+  const float* const* ptr;
+  const int* bs;
+  int n;
+  int row;
+  template <int W>
+  __device__ __forceinline__ void load(int col, float (&v)[W]) const {
+    float tot[W], cur[W];
+#pragma unroll
+    for (int e = 0; e < W; ++e) {
+      tot[e] = 0.f;
+      cur[e] = 0.f;
+    }
+    int cur_b = -1;
+    for (int s = 0; s < n; ++s) {
+      const float4* p4 = reinterpret_cast<const float4*>(ptr[s] + row * ACC_COLS + col);
+      float x[W];
+#pragma unroll
+      for (int q = 0; q < W / 4; ++q) {
+        const float4 f = __ldcg(p4 + q);
+        x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
+      }
+      if (bs[s] != cur_b) {
+        if (cur_b >= 0) {
+#pragma unroll
+          for (int e = 0; e < W; ++e) tot[e] += cur[e];
+        }
+#pragma unroll
+        for (int e = 0; e < W; ++e) cur[e] = x[e];
+        cur_b = bs[s];
+      } else {
+#pragma unroll
+        for (int e = 0; e < W; ++e) cur[e] += x[e];
+      }
+    }
+#pragma unroll
+    for (int e = 0; e < W; ++e) v[e] = tot[e] + cur[e];
+  }
+  __device__ __forceinline__ void load32(int col, float (&v)[32]) const { load<32>(col, v); }
+  __device__ __forceinline__ void load16(int col, float (&v)[16]) const { load<16>(col, v); }
+};
 
 template <class Cfg, class Epi>
 __global__ void __launch_bounds__(kThreads, 1)
@@ -127,9 +332,11 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  volatile int* last_flag = reinterpret_cast<volatile int*>(tmem_slot + 2);
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  const int grid = gridDim.x;
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -157,8 +364,6 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
 
-  const int num_tiles = gp.batch * gp.m_blocks * gp.n_blocks;
-
   if (warp == 0) {
     if (lane == 0) {
       // ------------------------------------------------------------------ TMA producer
@@ -167,14 +372,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0;   // stages that received at least one load
       uint32_t last_parity = 0;   // parity of the last phase issued into each stage
       bool ok = true;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x) {
-        int b, mb, nb;
-        decode_tile(t, gp, b, mb, nb);
-        const int m0 = mb * Cfg::A_ROWS;
-        const int n0 = nb * Cfg::BN;
-        const int za = gp.a_batched ? b : 0;
-        const int zb = gp.b_batched ? b : 0;
-        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+      SegIter it;
+      it.init(gp, blockIdx.x, grid);
+      Seg sg;
+      while (ok && it.next(gp, grid, sg)) {
+        const int m0 = sg.mb * Cfg::A_ROWS;
+        const int n0 = sg.nb * Cfg::BN;
+        const int za = gp.a_batched ? sg.b : 0;
+        const int zb = gp.b_batched ? sg.b : 0;
+        const int nk = sg.kb1 - sg.kb0;
+        for (int i = 0; i < nk; ++i) {
+          int kb = sg.kb0 + i + sg.rot;
+          if (kb >= sg.kb1) kb -= nk;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
             ok = false;
             break;
@@ -216,12 +425,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       // ------------------------------------------------------------------ MMA issuer
       int stage = 0;
       uint32_t phase = 0;
-      int it = 0;
+      int it_n = 0;
       bool ok = true;
       bool issued_any = false;
-      for (int t = blockIdx.x; t < num_tiles && ok; t += gridDim.x, ++it) {
-        const int acc = it & 1;
-        const uint32_t acc_phase = (it >> 1) & 1;
+      SegIter it;
+      it.init(gp, blockIdx.x, grid);
+      Seg sg;
+      while (ok && it.next(gp, grid, sg)) {
+        const int acc = it_n & 1;
+        const uint32_t acc_phase = (it_n >> 1) & 1;
+        ++it_n;
         if (!mbar_wait(&acc_empty[acc], acc_phase ^ 1u, abort_flag, gp.err,
                        DEVERR_WAIT_ACC_EMPTY)) {
           ok = false;
@@ -229,7 +442,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_base = tmem_base + acc * Cfg::ACC_COLS;
-        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+        const int nk = sg.kb1 - sg.kb0;
+        for (int i = 0; i < nk; ++i) {
           if (!mbar_wait(&full[stage], phase, abort_flag, gp.err, DEVERR_WAIT_FULL)) {
             ok = false;
             break;
@@ -249,7 +463,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                   Cfg::A_MN ? make_sdesc_sw128(a_sub + kk * (kUmmaK * 128), 64 * kBK * 2, 1024)
                             : make_sdesc_sw128(a_sub + kk * (kUmmaK * 2), 16, 1024);
               umma_f16(d_base + s * Cfg::BN, adesc, bdesc, Cfg::IDESC,
-                       (kb | kk) != 0 ? 1u : 0u);
+                       (i > 0 || kk != 0) ? 1u : 0u);
             }
           }
           issued_any = true;
@@ -272,28 +486,77 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ epilogue warps
     const int quarter = warp & 3;            // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
-    int it = 0;
-    for (int t = blockIdx.x; t < num_tiles; t += gridDim.x, ++it) {
-      const int acc = it & 1;
-      const uint32_t acc_phase = (it >> 1) & 1;
+    const int64_t U = units_per_group(gp);
+    const int64_t my_start = gp.stream_k ? cta_start(blockIdx.x, gp, grid) : 0;
+    const int64_t my_end = gp.stream_k ? cta_start(blockIdx.x + 1, gp, grid) : 0;
+    int it_n = 0;
+    SegIter it;
+    it.init(gp, blockIdx.x, grid);
+    Seg sg;
+    while (it.next(gp, grid, sg)) {
+      const int acc = it_n & 1;
+      const uint32_t acc_phase = (it_n >> 1) & 1;
+      ++it_n;
       int ok = 0;
       if (lane == 0)
         ok = mbar_wait(&acc_full[acc], acc_phase, abort_flag, gp.err, DEVERR_WAIT_ACC_FULL);
       ok = __shfl_sync(0xffffffffu, ok, 0);
-      if (!ok) break;
+      // all four epilogue warps agree, so none of them can be left waiting at a named barrier
+      if (!epi_bar_and(ok)) break;
       tc_fence_after();
-      int b, mb, nb;
-      decode_tile(t, gp, b, mb, nb);
+      TmemSrc tsrc;
+      tsrc.taddr = tmem_base + acc * Cfg::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
       EpiCtx ctx;
-      ctx.taddr = tmem_base + acc * Cfg::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
       ctx.row = row;
-      ctx.b = b;
-      ctx.m0 = mb * Cfg::A_ROWS;
-      ctx.n0 = nb * Cfg::BN;
-      Epi::template run<Cfg>(ep, gp, ctx);
+      ctx.b = gp.sum_batch ? 0 : sg.b;
+      ctx.m0 = sg.mb * Cfg::A_ROWS;
+      ctx.n0 = sg.nb * Cfg::BN;
+      // the tile is whole when all its k-blocks lie in this CTA's range (then it is one segment)
+      const int64_t g0 = static_cast<int64_t>(sg.g) * U;
+      const bool whole = !gp.stream_k ||
+                         (g0 >= my_start && g0 + U <= my_end && (!gp.sum_batch || gp.batch == 1));
+      if (whole) {
+        Epi::template run<Cfg>(ep, gp, ctx, tsrc);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&acc_empty[acc]);
+        continue;
+      }
+      // split tile: park the partial in this CTA's slot and free the accumulator
+      float* slot = gp.slots +
+                    (static_cast<int64_t>(blockIdx.x) * gp.slots_per_cta + sg.local) * Cfg::SLOT_FLOATS +
+                    static_cast<int64_t>(row) * Cfg::ACC_COLS;
+#pragma unroll 1
+      for (int col = 0; col < Cfg::ACC_COLS; col += 16) {
+        float v[16];
+        tsrc.load16(col, v);
+        float4* d4 = reinterpret_cast<float4*>(slot + col);
+#pragma unroll
+        for (int q = 0; q < 4; ++q)
+          __stcg(d4 + q, make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
+      }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&acc_empty[acc]);
+      __threadfence();
+      epi_bar();
+      const float* ptrs[kMaxGroupSegs];
+      int bs[kMaxGroupSegs];
+      const int nseg = group_segments<Cfg::SLOT_FLOATS>(gp, grid, sg.g, ptrs, bs);
+      if (threadIdx.x == 64) {
+        const int old = atomicAdd(&gp.counters[sg.g], 1);
+        const int last = (old == nseg - 1) ? 1 : 0;
+        if (last) gp.counters[sg.g] = 0;   // ready for the next launch
+        *last_flag = last;
+      }
+      epi_bar();
+      const int last = *last_flag;
+      epi_bar();   // every thread has read the flag before it can be rewritten
+      if (last) {
+        __threadfence();
+        FixupSrc<Cfg::ACC_COLS> fsrc{ptrs, bs, nseg, row};
+        Epi::template run<Cfg>(ep, gp, ctx, fsrc);
+      }
     }
   }
 
@@ -306,22 +569,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 // ---------------------------------------------------------------------------------------------
 // Epilogue helpers
 // ---------------------------------------------------------------------------------------------
-
-// Load 32 consecutive fp32 accumulator columns of this thread's row.
-__device__ __forceinline__ void acc_load32(uint32_t taddr, int col, float (&v)[32]) {
-  uint32_t r[32];
-  sm100::tmem_ld_32x32b_x32(taddr + static_cast<uint32_t>(col), r);
-  sm100::tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 32; ++i) v[i] = __uint_as_float(r[i]);
-}
-__device__ __forceinline__ void acc_load16(uint32_t taddr, int col, float (&v)[16]) {
-  uint32_t r[16];
-  sm100::tmem_ld_32x32b_x16(taddr + static_cast<uint32_t>(col), r);
-  sm100::tmem_wait_ld();
-#pragma unroll
-  for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(r[i]);
-}
 
 // 32 bf16 values to 64 contiguous bytes (16-byte aligned destination).
 __device__ __forceinline__ void store_bf16x32(__nv_bfloat16* dst, const float (&v)[32]) {
@@ -370,8 +617,9 @@ struct EpiHidden {
     int32_t swap;       // 1: A = weights, B = tokens
   };
 
-  template <class Cfg>
-  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+  template <class Cfg, class Src>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
+                                             const Src& src) {
     const bool swiglu = p.act == TP_ACT_SWIGLU;
     if (!p.swap) {
       const int t = c.m0 + c.row;
@@ -382,8 +630,8 @@ struct EpiHidden {
 #pragma unroll 1
         for (int col = 0; col < 128; col += 32) {
           float g[32], u[32];
-          acc_load32(c.taddr, col, g);
-          acc_load32(c.taddr, 128 + col, u);
+          src.load32(col, g);
+          src.load32(128 + col, u);
           if (live) {
             if (p.z) {
               store_bf16x32(p.z + t * p.ld_z + c.n0 + col, g);
@@ -399,7 +647,7 @@ struct EpiHidden {
 #pragma unroll 1
         for (int col = 0; col < Cfg::BN; col += 32) {
           float v[32];
-          acc_load32(c.taddr, col, v);
+          src.load32(col, v);
           const int r0 = c.n0 + col;
           if (live && r0 + 32 <= p.rows) {
             if (p.z) store_bf16x32(p.z + t * p.ld_z + r0, v);
@@ -427,8 +675,8 @@ struct EpiHidden {
 #pragma unroll 1
         for (int col = 0; col < Cfg::BN; col += 16) {
           float g[16], u[16];
-          acc_load16(c.taddr, col, g);
-          acc_load16(c.taddr, Cfg::BN + col, u);
+          src.load16(col, g);
+          src.load16(Cfg::BN + col, u);
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int t = c.n0 + col + e;
@@ -447,7 +695,7 @@ struct EpiHidden {
 #pragma unroll 1
         for (int col = 0; col < Cfg::BN; col += 16) {
           float v[16];
-          acc_load16(c.taddr, col, v);  // whole warp: tcgen05.ld is warp-collective
+          src.load16(col, v);  // whole warp: a TMEM source is warp-collective
           if (!live) continue;
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
@@ -478,8 +726,9 @@ struct EpiStoreF32 {
     int32_t swap;
   };
 
-  template <class Cfg>
-  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+  template <class Cfg, class Src>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
+                                             const Src& src) {
     float* base = p.out + static_cast<int64_t>(c.b) * p.batch_stride;
     if (!p.swap) {
       const int i = c.m0 + c.row;
@@ -487,7 +736,7 @@ struct EpiStoreF32 {
 #pragma unroll 1
       for (int col = 0; col < Cfg::BN; col += 32) {
         float v[32];
-        acc_load32(c.taddr, col, v);
+        src.load32(col, v);
         const int j0 = c.n0 + col;
         if (live) {
           float* dst = base + i * p.ld + j0;
@@ -509,13 +758,70 @@ struct EpiStoreF32 {
 #pragma unroll 1
       for (int col = 0; col < Cfg::BN; col += 16) {
         float v[16];
-        acc_load16(c.taddr, col, v);
+        src.load16(col, v);
         if (live) {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int i = c.n0 + col + e;
             if (i < p.rows_valid) base[i * p.ld + j] = v[e];
           }
+        }
+      }
+    }
+  }
+};
+
+// ---------------------------------------------------------------------------------------------
+// Fused partial-sum reduce: with sum_batch the source already holds sum_i y_i (shards added in
+// order 0..p-1 in fp32); this adds the residual once and rounds to the output dtype.
+// out[i][j] with i = token, j = output feature (swapped: i = n, j = m).  Requires A_SUB == 1.
+// ---------------------------------------------------------------------------------------------
+struct EpiReduceOut {
+  struct Params {
+    void* out;
+    const void* residual;   // same dtype and layout as out, or null
+    int64_t ld;
+    int32_t rows_valid, cols_valid;
+    int32_t out_bf16;
+    int32_t swap;
+  };
+
+  __device__ __forceinline__ static void put(const Params& p, int64_t idx, float v) {
+    if (p.residual)
+      v = (p.out_bf16 ? __bfloat162float(static_cast<const __nv_bfloat16*>(p.residual)[idx])
+                      : static_cast<const float*>(p.residual)[idx]) + v;
+    if (p.out_bf16) static_cast<__nv_bfloat16*>(p.out)[idx] = __float2bfloat16_rn(v);
+    else static_cast<float*>(p.out)[idx] = v;
+  }
+
+  template <class Cfg, class Src>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
+                                             const Src& src) {
+    if (!p.swap) {
+      const int i = c.m0 + c.row;
+      const bool live = i < p.rows_valid;
+#pragma unroll 1
+      for (int col = 0; col < Cfg::BN; col += 32) {
+        float v[32];
+        src.load32(col, v);
+        if (!live) continue;
+        const int j0 = c.n0 + col;
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (j0 + e < p.cols_valid) put(p, static_cast<int64_t>(i) * p.ld + j0 + e, v[e]);
+      }
+    } else {
+      const int j = c.m0 + c.row;
+      const bool live = j < p.cols_valid;
+#pragma unroll 1
+      for (int col = 0; col < Cfg::BN; col += 16) {
+        float v[16];
+        src.load16(col, v);
+        if (!live) continue;
+#pragma unroll
+        for (int e = 0; e < 16; ++e) {
+          const int i = c.n0 + col + e;
+          if (i < p.rows_valid) put(p, static_cast<int64_t>(i) * p.ld + j, v[e]);
         }
       }
     }
@@ -537,15 +843,16 @@ struct EpiActBwd {
     int32_t act;
   };
 
-  template <class Cfg>
-  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c) {
+  template <class Cfg, class Src>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
+                                             const Src& src) {
     const int t = c.m0 + c.row;
     const bool live = t < p.tokens;
     const int64_t rowoff = static_cast<int64_t>(t) * p.ld + static_cast<int64_t>(c.b) * p.R;
 #pragma unroll 1
     for (int col = 0; col < Cfg::BN; col += 32) {
       float dh[32];
-      acc_load32(c.taddr, col, dh);
+      src.load32(col, dh);
       if (!live) continue;
       const int f = c.n0 + col;                  // shard-local padded feature (multiple of 32)
       if (p.act == TP_ACT_SWIGLU) {

@@ -59,6 +59,39 @@ __global__ void __launch_bounds__(256) reduce_vec8_kernel(const Tin* __restrict_
   }
 }
 
+// Same sum for p <= PMAX: all p loads are issued before the first add (more bytes in flight);
+// the additions still run in the order 0..p-1.
+template <typename Tin, typename Tout, int PMAX>
+__global__ void __launch_bounds__(256) reduce_vec8_small_kernel(const Tin* __restrict__ part,
+                                                                int p, int64_t n,
+                                                                const Tout* res, Tout* out) {
+  const int64_t nv = n >> 3;
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
+       i += stride) {
+    float v[PMAX][8];
+#pragma unroll
+    for (int s = 0; s < PMAX; ++s)
+      if (s < p) Vec8<Tin>::load(part + static_cast<int64_t>(s) * n + 8 * i, v[s]);
+    float r[8];
+    if (res) Vec8<Tout>::load(res + 8 * i, r);
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = v[0][e];
+#pragma unroll
+    for (int s = 1; s < PMAX; ++s)
+      if (s < p) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += v[s][e];
+      }
+    if (res) {
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = r[e] + acc[e];
+    }
+    Vec8<Tout>::store(out + 8 * i, acc);
+  }
+}
+
 template <typename Tin, typename Tout>
 __global__ void reduce_scalar_kernel(const Tin* part, int p, int64_t n, const Tout* res,
                                      Tout* out) {
@@ -83,7 +116,10 @@ inline tp_status launch_t(const void* part, int p, int64_t n, const void* res, v
   const int64_t cap = static_cast<int64_t>(num_sms()) * 8;
   if (blocks > cap) blocks = cap;
   ProfScope prof(s, "reduce_partials");
-  if (vec)
+  if (vec && p <= 8)
+    reduce_vec8_small_kernel<Tin, Tout, 8><<<static_cast<int>(blocks), 256, 0, s>>>(
+        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+  else if (vec)
     reduce_vec8_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
         static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
   else

@@ -37,8 +37,9 @@ extern "C" tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const 
   tp::AttnLayout L;
   tp_status st = tp::attn_layout_of(desc, &L);
   if (st != TP_OK) return st;
-  if (desc->reduce_mode == TP_REDUCE_FUSED)
-    return tp::set_error(TP_ERR_UNSUPPORTED, "TP_REDUCE_FUSED is not available for tp_attn_fwd");
+  if (desc->reduce_mode == TP_REDUCE_FUSED && !L.tc)
+    return tp::set_error(TP_ERR_UNSUPPORTED,
+                         "TP_REDUCE_FUSED needs the tensor-core path (bf16, h a multiple of 8)");
   if (L.tokens == 0) {
     tp::count_reduction();
     return TP_OK;

@@ -48,12 +48,16 @@ class ProfScope {
   cudaEvent_t start_ = nullptr;
 };
 
+int num_sms();                    // SM count of the current device (cached per device)
+// Decode (swapped, weight-streaming) GEMMs use whole tiles with rotated k order when there are at
+// least as many tiles as SMs; with fewer tiles, stream-K gives every SM an equal share.
+inline bool decode_stream_k(int64_t tiles) { return tiles < num_sms(); }
+
 inline int64_t round_up(int64_t a, int64_t b) { return (a + b - 1) / b * b; }
 inline int64_t ceil_div(int64_t a, int64_t b) { return (a + b - 1) / b; }
 inline size_t align256(size_t a) { return (a + 255) & ~size_t(255); }
 inline int elem_bytes(int dtype) { return dtype == TP_BF16 ? 2 : 4; }
 
-int num_sms();                    // SM count of the current device (cached per device)
 bool tensor_cores_usable();       // sm_100 device present
 
 // ----------------------------------------------------------------------------------------------

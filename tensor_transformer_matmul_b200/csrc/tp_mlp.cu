@@ -30,12 +30,54 @@ constexpr int stages_for(int bn, int a_sub) {
 
 struct MlpLayout {
   int64_t T, d, F, Fs, Fsp, R;
-  int p, act, dtype, eb, y_dtype;
+  int p, act, dtype, eb, y_dtype, reduce_mode;
+  bool tc;                      // bf16 with 16-byte rows: the tensor-core path
   size_t w1p_bytes, w2p_bytes;
   size_t saved_z_off, saved_h_off, saved_bytes;
-  size_t fz_off, fh_off, fpart_off, fwd_ws;
+  size_t fz_off, fh_off, fpart_off, fsk_off, fwd_ws;
   size_t bdh_off, bdz_off, bpart_off, bwd_ws;
 };
+
+template <class C> struct Tag { using type = C; };
+template <int BN, int ASUB>
+using KK = TileCfg<BN, ASUB, false, false, stages_for(BN, ASUB)>;
+
+// Swapped GEMMs put the weights on the 128-row M side and the T tokens on N: pick N by T.
+template <int ASUB, class F>
+auto by_tokens(int64_t T, F&& f) {
+  if (T <= 16) return f(Tag<KK<16, ASUB>>{});
+  if (T <= 64) return f(Tag<KK<64, ASUB>>{});
+  return f(Tag<KK<128, ASUB>>{});
+}
+
+constexpr int64_t kSwapMaxT = 128;   // token counts up to this use the swapped (decode) tiles
+
+// stream-K plans of the forward GEMMs (bytes of counters + partial slots); empty if unused
+// output tiles of the swapped (decode) up and down GEMMs
+int64_t up_tiles(const MlpLayout& L) {
+  return ceil_div(L.p * L.R, L.act == TP_ACT_SWIGLU ? 256 : 128);
+}
+int64_t down_tiles(const MlpLayout& L) { return L.p * ceil_div(L.d, 128); }
+
+size_t up_sk_bytes(const MlpLayout& L) {
+  if (L.T > kSwapMaxT || !decode_stream_k(up_tiles(L))) return 0;
+  const int64_t rows = L.p * L.R;
+  auto f = [&](auto tag) {
+    return tc::plan_stream_k<typename decltype(tag)::type>(rows, L.T, L.d, 1, false, num_sms()).bytes();
+  };
+  return L.act == TP_ACT_SWIGLU ? by_tokens<2>(L.T, f) : by_tokens<1>(L.T, f);
+}
+size_t down_sk_bytes(const MlpLayout& L) {
+  const bool fused = L.reduce_mode == TP_REDUCE_FUSED;
+  if (L.T > kSwapMaxT) {
+    if (!fused) return 0;
+    return tc::plan_stream_k<KK<256, 1>>(L.T, L.d, L.Fsp, L.p, true, num_sms()).bytes();
+  }
+  if (!fused && !decode_stream_k(down_tiles(L))) return 0;
+  return by_tokens<1>(L.T, [&](auto tag) {
+    return tc::plan_stream_k<typename decltype(tag)::type>(L.d, L.T, L.Fsp, L.p, fused, num_sms()).bytes();
+  });
+}
 
 tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   if (!desc) return set_error(TP_ERR_INVALID_ARG, "desc is null");
@@ -53,6 +95,8 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   L->y_dtype = (desc->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : desc->dtype;
   L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
   L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
+  L->reduce_mode = desc->reduce_mode;
+  L->tc = desc->dtype == TP_BF16 && desc->d % 8 == 0;
   L->Fs = L->F / L->p;
   L->Fsp = round_up(L->Fs, 128);
   L->R = (L->act == TP_ACT_SWIGLU) ? 2 * L->Fsp : L->Fsp;
@@ -65,10 +109,23 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   L->saved_z_off = 0;
   L->saved_h_off = align256(zb);
   L->saved_bytes = L->saved_h_off + align256(hb);
-  L->fz_off = 0;
-  L->fh_off = align256(zb);
-  L->fpart_off = L->fh_off + align256(hb);
-  L->fwd_ws = L->fpart_off + align256(partb);
+  if (L->tc) {
+    // h, the stream-K region (shared by the up and down GEMMs, which run one after the other),
+    // then the fp32 partials when they are reduced by a separate kernel
+    L->fz_off = 0;
+    L->fh_off = 0;
+    L->fsk_off = align256(hb);
+    const size_t sk = L->T > 0 ? std::max(up_sk_bytes(*L), down_sk_bytes(*L)) : 0;
+    L->fpart_off = L->fsk_off + align256(sk);
+    const size_t pb = L->reduce_mode == TP_REDUCE_FUSED ? 0 : partb;
+    L->fwd_ws = L->fpart_off + align256(pb);
+  } else {
+    L->fz_off = 0;
+    L->fh_off = align256(zb);
+    L->fpart_off = L->fh_off + align256(hb);
+    L->fsk_off = L->fpart_off;
+    L->fwd_ws = L->fpart_off + align256(partb);
+  }
   const size_t dhb = static_cast<size_t>(L->T * P * L->Fsp) * 4;
   L->bdh_off = 0;
   L->bdz_off = align256(dhb);
@@ -79,18 +136,12 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15) == 0; }
 
-bool use_tensor_cores(const MlpLayout& L) {
-  return L.dtype == TP_BF16 && (L.d % 8 == 0) && tensor_cores_usable();
-}
-
 uint8_t* off(void* base, size_t o) { return static_cast<uint8_t*>(base) + o; }
 
 // ------------------------------------------------------------------------------ tensor cores
-template <int BN, int ASUB>
-using KK = TileCfg<BN, ASUB, false, false, stages_for(BN, ASUB)>;
 
 tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, void* z,
-                cudaStream_t s) {
+                void* sk_ws, size_t sk_bytes, cudaStream_t s) {
   const int64_t rows = L.p * L.R;
   tc::EpiHidden::Params ep;
   ep.h = static_cast<__nv_bfloat16*>(h);
@@ -100,40 +151,69 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
   ep.tokens = static_cast<int32_t>(L.T);
   ep.rows = static_cast<int32_t>(rows);
   ep.act = L.act;
-  const bool swiglu = L.act == TP_ACT_SWIGLU;
   const Operand xo{x, false, L.T, L.d, 1, L.d, 0};
   const Operand wo{w1p, false, rows, L.d, 1, L.d, 0};
-  if (L.T <= 128) {
+  if (L.T <= kSwapMaxT) {
+    // decode: weights stream once, every SM takes an equal share of their k-blocks
     ep.swap = 1;
-    if (swiglu) {
-      if (L.T <= 16) return tc::run_gemm<KK<16, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
-      if (L.T <= 64) return tc::run_gemm<KK<64, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
-      return tc::run_gemm<KK<128, 2>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
-    }
-    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
-    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
-    return tc::run_gemm<KK<128, 1>, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep, s, "mlp_up_gemm");
+    const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = decode_stream_k(up_tiles(L)) ? &sk : nullptr;
+    opt.rotate_k = true;
+    auto f = [&](auto tag) {
+      return tc::run_gemm<typename decltype(tag)::type, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep,
+                                                                       s, "mlp_up_gemm", opt);
+    };
+    return L.act == TP_ACT_SWIGLU ? by_tokens<2>(L.T, f) : by_tokens<1>(L.T, f);
   }
   ep.swap = 0;
   return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s, "mlp_up_gemm");
 }
 
-// partial[i] = h_i W2_i  (fp32, [p][T][d])
-tp_status tc_down_partials(const MlpLayout& L, const void* h, const void* w2p, float* part,
-                           cudaStream_t s) {
+// Row-parallel down projection.  Separate reduce: partial[i] = h_i W2_i (fp32, [p][T][d]).
+// Fused reduce: y = residual + sum_i h_i W2_i written directly (shards added in order).
+tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* part,
+                  const void* residual, void* y, void* sk_ws, size_t sk_bytes, cudaStream_t s) {
   const Operand ho{h, false, L.T, L.Fsp, L.p, L.p * L.Fsp, L.Fsp};
   const Operand wo{w2p, false, L.d, L.Fsp, L.p, L.Fsp, L.d * L.Fsp};
+  const bool swap = L.T <= kSwapMaxT;
+  if (L.reduce_mode == TP_REDUCE_FUSED) {
+    tc::EpiReduceOut::Params ep;
+    ep.out = y;
+    ep.residual = residual;
+    ep.ld = L.d;
+    ep.rows_valid = static_cast<int32_t>(L.T);
+    ep.cols_valid = static_cast<int32_t>(L.d);
+    ep.out_bf16 = L.y_dtype == TP_BF16 ? 1 : 0;
+    ep.swap = swap ? 1 : 0;
+    const tc::StreamKArgs sk{true, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = &sk;
+    opt.rotate_k = swap;
+    if (swap)
+      return by_tokens<1>(L.T, [&](auto tag) {
+        return tc::run_gemm<typename decltype(tag)::type, tc::EpiReduceOut>(
+            wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm", opt);
+      });
+    return tc::run_gemm<KK<256, 1>, tc::EpiReduceOut>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s,
+                                                       "mlp_down_gemm", opt);
+  }
   tc::EpiStoreF32::Params ep;
   ep.out = part;
   ep.ld = L.d;
   ep.batch_stride = L.T * L.d;
   ep.rows_valid = static_cast<int32_t>(L.T);
   ep.cols_valid = static_cast<int32_t>(L.d);
-  if (L.T <= 128) {
+  if (swap) {
     ep.swap = 1;
-    if (L.T <= 16) return tc::run_gemm<KK<16, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
-    if (L.T <= 64) return tc::run_gemm<KK<64, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
-    return tc::run_gemm<KK<128, 1>, tc::EpiStoreF32>(wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm");
+    const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
+    tc::GemmOpts opt;
+    opt.sk = decode_stream_k(down_tiles(L)) ? &sk : nullptr;
+    opt.rotate_k = true;
+    return by_tokens<1>(L.T, [&](auto tag) {
+      return tc::run_gemm<typename decltype(tag)::type, tc::EpiStoreF32>(
+          wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm", opt);
+    });
   }
   ep.swap = 0;
   return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s, "mlp_down_gemm");
@@ -385,8 +465,9 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
   MlpLayout L;
   tp_status st = layout_of(desc, &L);
   if (st != TP_OK) return st;
-  if (desc->reduce_mode == TP_REDUCE_FUSED)
-    return set_error(TP_ERR_UNSUPPORTED, "TP_REDUCE_FUSED is not available for tp_mlp_fwd");
+  if (desc->reduce_mode == TP_REDUCE_FUSED && !L.tc)
+    return set_error(TP_ERR_UNSUPPORTED,
+                     "TP_REDUCE_FUSED needs the tensor-core path (bf16, d a multiple of 8)");
   if (L.T == 0) {
     count_reduction();
     return TP_OK;
@@ -398,13 +479,21 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
   void* z = saved ? off(saved, L.saved_z_off) : off(workspace, L.fz_off);
   void* h = saved ? off(saved, L.saved_h_off) : off(workspace, L.fh_off);
   float* part = reinterpret_cast<float*>(off(workspace, L.fpart_off));
-  if (use_tensor_cores(L)) {
+  if (L.tc) {
+    if (!tensor_cores_usable())
+      return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {x, w1p, w2p, residual, static_cast<const void*>(y),
                           static_cast<const void*>(saved)})
       if (q && !aligned16(q))
         return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, s)) != TP_OK) return st;
-    if ((st = tc_down_partials(L, h, w2p, part, s)) != TP_OK) return st;
+    void* sk = off(workspace, L.fsk_off);
+    const size_t skb = L.fpart_off - L.fsk_off;
+    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
+    if ((st = tc_down(L, h, w2p, part, residual, y, sk, skb, s)) != TP_OK) return st;
+    if (L.reduce_mode == TP_REDUCE_FUSED) {
+      count_reduction();
+      return TP_OK;
+    }
   } else if (L.dtype == TP_BF16) {
     if ((st = simt_forward<__nv_bfloat16>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
   } else {
@@ -423,8 +512,6 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
   MlpLayout L;
   tp_status st = layout_of(desc, &L);
   if (st != TP_OK) return st;
-  if (desc->reduce_mode == TP_REDUCE_FUSED)
-    return set_error(TP_ERR_UNSUPPORTED, "TP_REDUCE_FUSED is not available for tp_mlp_bwd");
   if (!w1p || !w2p || !dw1p || !dw2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (L.T == 0) {  // no tokens: zero weight gradients, nothing else
@@ -443,7 +530,9 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
   float* part = reinterpret_cast<float*>(off(workspace, L.bpart_off));
   float* g1 = static_cast<float*>(dw1p);
   float* g2 = static_cast<float*>(dw2p);
-  if (use_tensor_cores(L)) {
+  if (L.tc) {
+    if (!tensor_cores_usable())
+      return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {dy, x, saved, w1p, w2p, static_cast<const void*>(dx)})
       if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
     st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, s);

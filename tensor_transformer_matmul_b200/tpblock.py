@@ -12,7 +12,8 @@ import os
 import torch
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
-LIB_PATH = os.path.join(_HERE, "libtpblock.so")
+# TPBLOCK_LIBRARY may point at another build of the same library (e.g. a tuning variant)
+LIB_PATH = os.environ.get("TPBLOCK_LIBRARY") or os.path.join(_HERE, "libtpblock.so")
 
 TP_OK, TP_ERR_INVALID_ARG, TP_ERR_SHAPE, TP_ERR_UNSUPPORTED, TP_ERR_WORKSPACE, TP_ERR_CUDA, \
     TP_ERR_TIMEOUT = range(7)

@@ -69,13 +69,15 @@ class Mlp:
 class Attn:
     """Packs one attention block's weights with the library and runs tp_attn_fwd."""
 
-    def __init__(self, lib, inp, p, dtype, causal=True, kv_len=0, n_q=None, n_kv=None, hd=None):
+    def __init__(self, lib, inp, p, dtype, causal=True, kv_len=0, n_q=None, n_kv=None, hd=None,
+                 reduce_mode=0):
         self.lib = lib
         x = inp["x"]
         self.b, self.s, self.h = x.shape
         self.n_q, self.n_kv, self.hd = n_q, n_kv, hd
         self.dtype = dtype
-        self.desc = lib.attn_desc(self.b, self.s, self.h, n_q, n_kv, hd, p, causal, dtype, kv_len)
+        self.desc = lib.attn_desc(self.b, self.s, self.h, n_q, n_kv, hd, p, causal, dtype, kv_len,
+                                  reduce_mode=reduce_mode)
         tdt = inputs.TORCH_DTYPE[dtype]
         eb = 2 if dtype == "bf16" else 4
         g = dev()

@@ -28,7 +28,7 @@ def _ref(inp, n_q, n_kv, hd, causal):
 ])
 def test_prefill_bf16(lib, causal, b, s, h, n_q, n_kv, hd, p):
     inp = inputs.attn_inputs(b, s, h, n_q, n_kv, hd, "bf16", seed=1, w_std=0.05)
-    a = Attn(lib, inp, p, "bf16", causal, n_q=n_q, n_kv=n_kv, hd=hd)
+    a = Attn(lib, inp, p, "bf16", causal, n_q=n_q, n_kv=n_kv, hd=hd, reduce_mode=int(causal))
     lib.tp_reset_reduction_count()
     y = a.forward(inp["x"])
     torch.cuda.synchronize()
@@ -66,15 +66,16 @@ def test_residual(lib):
     assert rel_l2(f64(y), _ref(inp, 8, 2, 32, True) + f64(res)) <= TOL["bf16"]
 
 
-@pytest.mark.parametrize("dtype,b,kv_len,h,n_q,n_kv,hd,p", [
-    ("bf16", 3, 300, 256, 8, 2, 64, 2),     # two key chunks
-    ("bf16", 1, 4096, 512, 16, 2, 128, 2),  # 17 chunks, group of 8 query heads per KV head
-    ("bf16", 2, 1, 128, 4, 4, 32, 4),       # a single cached key
-    ("f32", 2, 37, 64, 4, 2, 32, 2),
+@pytest.mark.parametrize("dtype,b,kv_len,h,n_q,n_kv,hd,p,mode", [
+    ("bf16", 3, 300, 256, 8, 2, 64, 2, 0),     # three key chunks
+    ("bf16", 3, 300, 256, 8, 2, 64, 2, 1),     # same, shard reduce fused into the O projection
+    ("bf16", 1, 4096, 512, 16, 2, 128, 2, 1),  # 33 chunks, group of 8 query heads per KV head
+    ("bf16", 2, 1, 128, 4, 4, 32, 4, 0),       # a single cached key
+    ("f32", 2, 37, 64, 4, 2, 32, 2, 0),
 ])
-def test_decode(lib, dtype, b, kv_len, h, n_q, n_kv, hd, p):
+def test_decode(lib, dtype, b, kv_len, h, n_q, n_kv, hd, p, mode):
     inp = inputs.attn_inputs(b, 1, h, n_q, n_kv, hd, dtype, seed=4, w_std=0.05, kv_len=kv_len)
-    a = Attn(lib, inp, p, dtype, True, kv_len=kv_len, n_q=n_q, n_kv=n_kv, hd=hd)
+    a = Attn(lib, inp, p, dtype, True, kv_len=kv_len, n_q=n_q, n_kv=n_kv, hd=hd, reduce_mode=mode)
     kc, vc = inp["k_cache"].to(dev()), inp["v_cache"].to(dev())
     y = a.forward(inp["x"], k_cache=kc, v_cache=vc)
     torch.cuda.synchronize()

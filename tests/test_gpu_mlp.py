@@ -35,14 +35,16 @@ def test_tiny_config_fp32(lib):
         assert rel_l2(f64(mp.forward(inp["x"])), ref) <= TOL["f32"], p
 
 
+@pytest.mark.parametrize("reduce_mode", [0, 1])
 @pytest.mark.parametrize("act", ["swiglu", "gelu", "relu", "identity"])
 @pytest.mark.parametrize("T", [1, 17, 64, 100, 200, 300])
-def test_bf16_forward_parity(lib, act, T):
+def test_bf16_forward_parity(lib, act, T, reduce_mode):
     # several tiles and ragged tails in every dimension: d = 328 (5 K-blocks + 8), F_s = 136
-    # (padded to 256 per shard), p = 3 (not a power of two, as in the h=2/d_ff=3 worked example)
+    # (padded to 256 per shard), p = 3 (not a power of two, as in the h=2/d_ff=3 worked example);
+    # T <= 128 runs the stream-K decode schedule, reduce_mode 1 fuses the shard reduce into it
     d, F, p = 328, 408, 3
     inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=1, w_std=0.05)
-    m = Mlp(lib, inp, p, act, "bf16")
+    m = Mlp(lib, inp, p, act, "bf16", reduce_mode)
     y = m.forward(inp["x"])
     torch.cuda.synchronize()
     assert rel_l2(f64(y), _oracle_fwd(inp, act)) <= TOL["bf16"]
@@ -170,3 +172,30 @@ def test_f32_residual_stream(lib):
     torch.cuda.synchronize()
     assert y.dtype == torch.float32
     assert rel_l2(f64(y), _oracle_fwd(inp, "swiglu") + f64(res)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("T,d,F,p", [(64, 2048, 8192, 8), (16, 4096, 4096, 4), (128, 1024, 16384, 16),
+                                     (1, 8192, 3584, 8)])
+def test_stream_k_splits_fused_vs_separate(lib, T, d, F, p):
+    # decode shapes whose k-blocks split tiles across CTAs at many different points; the fused
+    # reduce (shards added inside the GEMM) and the separate reduce both match the oracle
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=8, w_std=0.02)
+    ref = _oracle_fwd(inp, "swiglu")
+    outs = []
+    for mode in (0, 1):
+        m = Mlp(lib, inp, p, "swiglu", "bf16", mode)
+        lib.tp_reset_reduction_count()
+        outs.append(m.forward(inp["x"], save=False))
+        torch.cuda.synchronize()
+        assert lib.tp_reduction_count() == 1
+        assert rel_l2(f64(outs[-1]), ref) <= TOL["bf16"]
+    assert rel_l2(f64(outs[0]), f64(outs[1])) <= 1e-2
+
+
+def test_fused_reduce_deterministic(lib):
+    inp = inputs.mlp_inputs(64, 1024, 4096, "swiglu", "bf16", seed=9, w_std=0.02)
+    m = Mlp(lib, inp, 8, "swiglu", "bf16", 1)
+    a = m.forward(inp["x"], save=False).clone()
+    b = m.forward(inp["x"], save=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
