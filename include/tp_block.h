@@ -84,6 +84,7 @@ typedef struct {
   int32_t dtype;        /* tp_dtype of x, weights, y, dy, dx                                  */
   int32_t reduce_mode;  /* tp_reduce_mode                                                     */
   int32_t flags;        /* TP_FLAG_* (0 = none)                                               */
+  float norm_eps;       /* eps of the RMSNorm written to y_norm (0 means 1e-5)                */
 } tp_mlp_desc;
 
 /* Packed layouts.  F_s = d_ff / p; F_sp = F_s rounded up to a multiple of 128 (padding rows and
@@ -110,14 +111,17 @@ size_t tp_mlp_saved_bytes(const tp_mlp_desc* desc);
 size_t tp_mlp_fwd_workspace(const tp_mlp_desc* desc);
 
 /* Forward: y = residual + sum_{i=0}^{p-1} act(x W1_i) W2_i.
- *   x [T][d], y [T][d] (dtype).  residual: NULL, or [T][d] dtype added once after the sum
- *   (the residual add that follows the reduction and stays replicated).  residual may equal y.
+ *   x [T][d], y [T][d] (dtype; float32 with TP_FLAG_F32_RESIDUAL).  residual: NULL, or like y,
+ *   added once after the sum (the residual add that follows the reduction and stays
+ *   replicated).  residual may equal y.
+ *   y_norm: NULL, or [T][d] dtype that receives RMSNorm(y) (unit weight, eps desc.norm_eps):
+ *   the replicated normalization that follows the residual add, fused into the reduction.
  *   saved: NULL, or tp_mlp_saved_bytes() of device memory that receives z and h for
  *   tp_mlp_bwd.  Adds 1 to the reduction counter.
  *   Errors: TP_ERR_INVALID_ARG (null x/w1p/w2p/y/workspace with T>0, bad enum),
  *   TP_ERR_SHAPE (p < 1, d < 1, d_ff % p), TP_ERR_WORKSPACE (ws_bytes too small). */
 tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p, const void* w2p,
-                     const void* residual, void* y, void* saved, void* workspace,
+                     const void* residual, void* y, void* y_norm, void* saved, void* workspace,
                      size_t ws_bytes, void* stream);
 
 /* Workspace of tp_mlp_bwd in bytes. */
@@ -176,6 +180,8 @@ typedef struct {
   int64_t kv_cap;       /* slots per head in the caches (>= kv_len + 1); 0 means kv_len + 1  */
   int32_t reduce_mode;  /* tp_reduce_mode                                                     */
   int32_t flags;        /* TP_FLAG_* (0 = none)                                               */
+  float norm_eps;       /* eps of the RMSNorm written to y_norm (0 means 1e-5)                */
+  int32_t reserved;
 } tp_attn_desc;
 
 /* Packed layouts (element type dtype): qh = n_q/p, kh = n_kv/p, hd = head_dim,
@@ -192,14 +198,15 @@ tp_status tp_attn_pack(const tp_attn_desc* desc, const void* wq, const void* wk,
 
 size_t tp_attn_fwd_workspace(const tp_attn_desc* desc);
 
-/* y = residual + sum_i Attn_i(x) Wo_i.  x and y [b][s][h] dtype; residual NULL or [b][s][h].
+/* y = residual + sum_i Attn_i(x) Wo_i.  x [b][s][h] dtype; y and residual as in tp_mlp_fwd
+ * (residual NULL or like y); y_norm NULL or [b][s][h] dtype receiving RMSNorm(y).
  * Query head j of shard i attends over KV head floor(j / (n_q/n_kv)); scale 1/sqrt(head_dim).
  * Decode (kv_len > 0, s == 1): k_cache and v_cache are [b][n_kv][kv_cap][hd] dtype; the new
  * token's key and value are written to slot kv_len and it attends to slots 0..kv_len.
  * Self-attention (kv_len == 0): caches may be NULL.  Adds 1 to the reduction counter. */
 tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const void* wqkv_p,
                       const void* wo_p, void* k_cache, void* v_cache, const void* residual,
-                      void* y, void* workspace, size_t ws_bytes, void* stream);
+                      void* y, void* y_norm, void* workspace, size_t ws_bytes, void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
 /* Reduction and glue                                                                          */

@@ -16,10 +16,13 @@ namespace tp {
 struct AttnLayout {
   int64_t b, s, h, tokens, kv_len, kv_cap;
   int n_q, n_kv, hd, p, qh, kh, causal, dtype, eb, y_dtype;
+  float norm_eps;
   int64_t R_a;          // packed QKV rows per shard
   size_t wqkv_bytes, wo_bytes;
   size_t qkv_off, o_off, part_off, ml_off, sk_off, ws_bytes;
   int kv_splits;        // decode: key chunks per (sequence, KV head)
+  int kv_chunk;         // decode: keys per chunk
+  size_t cnt_off;       // decode: arrival counters [b][n_kv]
   int reduce_mode;
   bool tc;              // bf16 with 16-byte rows: tensor-core projections
 };
@@ -62,7 +65,6 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
   return std::max(a, b);
 }
 
-constexpr int kDecodeChunk = 128;   // keys per decode work item
 
 inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (!d) return set_error(TP_ERR_INVALID_ARG, "desc is null");
@@ -85,6 +87,7 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   L->qh = d->n_q / d->p; L->kh = d->n_kv / d->p;
   L->causal = d->causal ? 1 : 0; L->dtype = d->dtype; L->eb = elem_bytes(d->dtype);
   L->y_dtype = (d->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : d->dtype;
+  L->norm_eps = d->norm_eps > 0.f ? d->norm_eps : 1e-5f;
   L->kv_len = d->kv_len;
   L->kv_cap = d->kv_cap > 0 ? d->kv_cap : d->kv_len + 1;
   if (L->kv_len > 0 && L->kv_cap < L->kv_len + 1)
@@ -93,7 +96,24 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   const int64_t P = L->p;
   L->wqkv_bytes = static_cast<size_t>(P * L->R_a * L->h) * L->eb;
   L->wo_bytes = static_cast<size_t>(P * L->h * L->qh * L->hd) * L->eb;
-  L->kv_splits = L->kv_len > 0 ? static_cast<int>(ceil_div(L->kv_len + 1, kDecodeChunk)) : 0;
+  if (L->kv_len > 0) {
+    // about one wave of blocks over (split, KV head, sequence); chunks a multiple of 16 keys
+    const int64_t n_keys = L->kv_len + 1;
+    // at most one wave: splits * n_kv * b <= SMs when possible; a split's K and V rows must fit
+    // in shared memory (staged by bulk copies)
+    const int64_t max_chunk = std::min<int64_t>(
+        512, (200 * 1024) / (2 * static_cast<int64_t>(L->hd) * L->eb + 4 * (L->n_q / L->n_kv)) / 16 * 16);
+    const int64_t want = std::max<int64_t>(1, num_sms() / std::max<int64_t>(1, L->b * L->n_kv));
+    int64_t splits = std::min<int64_t>(std::min<int64_t>(want, 64), ceil_div(n_keys, 16));
+    splits = std::max<int64_t>(splits, ceil_div(n_keys, max_chunk));
+    L->kv_chunk = static_cast<int>(round_up(ceil_div(n_keys, splits), 16));
+    L->kv_splits = static_cast<int>(ceil_div(n_keys, L->kv_chunk));
+    if (L->kv_chunk > max_chunk || L->kv_splits > 64)
+      return set_error(TP_ERR_UNSUPPORTED, "decode KV length too long for the split-KV kernel");
+  } else {
+    L->kv_chunk = 0;
+    L->kv_splits = 0;
+  }
   const size_t qkvb = static_cast<size_t>(L->tokens * P * L->R_a) * L->eb;
   const size_t ob = static_cast<size_t>(L->tokens * L->n_q * L->hd) * L->eb;
   const size_t partb = static_cast<size_t>(P * L->tokens * L->h) * 4;
@@ -106,7 +126,9 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   L->part_off = L->o_off + align256(ob);
   const size_t pb = (L->tc && L->reduce_mode == TP_REDUCE_FUSED) ? 0 : partb;
   L->ml_off = L->part_off + align256(pb);
-  L->sk_off = L->ml_off + align256(mlb);
+  L->cnt_off = L->ml_off + align256(mlb);
+  const size_t cntb = L->kv_len > 0 ? static_cast<size_t>(L->b * L->n_kv) * sizeof(int32_t) : 0;
+  L->sk_off = L->cnt_off + align256(cntb);
   L->ws_bytes = L->sk_off + align256(attn_sk_bytes(*L));
   return TP_OK;
 }
@@ -218,182 +240,231 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, Q
   }
 }
 
-// Decode: write the new token's keys and values into slot kv_len of the caches
-// [b][n_kv][kv_cap][hd].
-template <typename T>
-__global__ void kv_append_kernel(const T* qkv, QkvIdx ix, T* kc, T* vc, int64_t b, int n_kv,
-                                 int64_t kv_cap, int64_t slot) {
-  const int64_t total = b * n_kv * ix.hd;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int e = static_cast<int>(idx % ix.hd);
-    const int64_t bg = idx / ix.hd;
-    const int g = static_cast<int>(bg % n_kv);
-    const int64_t bi = bg / n_kv;
-    const int64_t dst = ((bi * n_kv + g) * kv_cap + slot) * ix.hd + e;
-    kc[dst] = qkv[ix.k(bi, g) + e];
-    vc[dst] = qkv[ix.v(bi, g) + e];
+// Decode attention, split over keys.  Block = (split c, KV head g, sequence bi), 256 threads.
+// The split's K and V rows (contiguous in the cache) are staged into shared memory by two bulk
+// async copies, then three phases run over the staged keys (all query heads of the KV group
+// together, so each K and V row is read from HBM once):
+//   1. scores: a group of HD/8 lanes per key, each lane holding 8 consecutive dims;
+//      s[key][a] = (q_a . k) * log2(e)/sqrt(hd)
+//   2. softmax statistics: one warp per query head, m_a = max s, p = exp2(s - m_a), l_a = sum p
+//   3. o_a[d] = sum_key p[key][a] v[key][d]: each thread owns one dim d and GROUP*HD/256 heads
+// The new token (position kv_len) takes its key and value from the projection; the split that
+// holds it patches them into its staged rows and stores them into cache slot kv_len.
+// Output per (bi, q head, split): m (log2 units), l, o[hd].
+template <int HD, int GROUP, typename T>
+struct DecodeSmem {
+  static size_t bytes(int chunk) {
+    return static_cast<size_t>(chunk) * HD * sizeof(T) * 2 + static_cast<size_t>(chunk) * GROUP * 4 +
+           64;
   }
-}
+};
 
-// Decode attention, split over keys.  Block = (split c, kv head g, sequence bi); 8 warps share the
-// split's keys.  A group of HD/8 lanes handles one key: each lane holds 8 consecutive dims (one
-// 16-byte load of K and of V), so a warp covers 32/(HD/8) keys per pass and keeps kUnroll passes
-// of loads in flight.  Every query head of the KV group is handled in the same pass, so each K/V
-// row is read once.  Output per (bi, q head, split): running max m, denominator l and the
-// unnormalised o[hd].
 template <typename T, int GROUP, int HD>
-__global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx ix, const T* kc,
-                                                           const T* vc, int64_t kv_cap,
-                                                           int64_t n_keys, int n_q, int n_kv,
-                                                           float scale, float* ml) {
+__global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx ix, T* kc, T* vc,
+                                                           int64_t kv_cap, int64_t kv_len,
+                                                           int chunk, int n_q, int n_kv,
+                                                           float scale, float* ml, int* counters,
+                                                           T* o, uint32_t* err) {
   constexpr int kWarps = 8;
   constexpr int LPK = HD / 8;            // lanes per key
   constexpr int KPW = 32 / LPK;          // keys per warp pass
-  constexpr int kUnroll = 4;
-  __shared__ float s_m[kWarps][GROUP], s_l[kWarps][GROUP];
-  __shared__ float s_o[kWarps][GROUP][HD];
+  constexpr int APT = (GROUP * HD + 255) / 256;   // heads per thread in phase 3
+  extern __shared__ __align__(16) uint8_t dsm[];
+  T* sK = reinterpret_cast<T*>(dsm);
+  T* sV = sK + static_cast<size_t>(chunk) * HD;
+  float* s_p = reinterpret_cast<float*>(sV + static_cast<size_t>(chunk) * HD);   // [chunk][GROUP]
+  __shared__ float s_m[GROUP], s_l[GROUP];
+  __shared__ __align__(8) uint64_t bar;
+  __shared__ int s_ok;
   const int c = blockIdx.x, g = blockIdx.y;
   const int64_t bi = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int kslot = lane / LPK;          // which key of the pass this lane works on
-  const int d0 = (lane % LPK) * 8;       // first of this lane's 8 dims
-  const int64_t k0 = static_cast<int64_t>(c) * kDecodeChunk;
-  const int64_t k1 = min(n_keys, k0 + kDecodeChunk);
-  float q[GROUP][8], acc[GROUP][8], m[GROUP], l[GROUP];
-#pragma unroll
-  for (int a = 0; a < GROUP; ++a) {
-    const int j = g * GROUP + a;
-#pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      q[a][e] = to_f(qkv[ix.q(bi, j) + d0 + e]) * scale;
-      acc[a][e] = 0.f;
-    }
-    m[a] = -INFINITY;
-    l[a] = 0.f;
+  const int64_t n_keys = kv_len + 1;       // the cached positions plus the new token
+  const int64_t k0 = static_cast<int64_t>(c) * chunk;
+  const int nk = static_cast<int>(min(n_keys, k0 + chunk) - k0);
+  T* kbase = kc + (bi * n_kv + g) * kv_cap * HD;
+  T* vbase = vc + (bi * n_kv + g) * kv_cap * HD;
+  const T* knew = qkv + ix.k(bi, g);
+  const T* vnew = qkv + ix.v(bi, g);
+  const float sl2 = scale * 1.4426950408889634f;
+
+  // ---- stage the split's K and V rows
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    sm100::fence_barrier_init();
   }
-  const T* kbase = kc + (bi * n_kv + g) * kv_cap * HD + d0;
-  const T* vbase = vc + (bi * n_kv + g) * kv_cap * HD + d0;
-  const int64_t stride = static_cast<int64_t>(kWarps) * KPW;
-  // the trip count depends on the warp only (every lane runs every pass: the shuffles below
-  // need the whole warp); lanes whose key is past the end mask themselves out with ok[]
-  for (int64_t wbase = k0 + warp * KPW; wbase < k1; wbase += stride * kUnroll) {
-    float kv[kUnroll][8], vv[kUnroll][8];
-    bool ok[kUnroll];
-#pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
-      const int64_t kp = wbase + kslot + u * stride;
-      ok[u] = kp < k1;
-      if (ok[u]) {
-        if constexpr (sizeof(T) == 2) {
-          const uint4 wk = *reinterpret_cast<const uint4*>(kbase + kp * HD);
-          const uint4 wv = *reinterpret_cast<const uint4*>(vbase + kp * HD);
-          const uint32_t kw[4] = {wk.x, wk.y, wk.z, wk.w}, vw[4] = {wv.x, wv.y, wv.z, wv.w};
-#pragma unroll
-          for (int h2 = 0; h2 < 4; ++h2) {
-            kv[u][2 * h2] = bf16lo(kw[h2]); kv[u][2 * h2 + 1] = bf16hi(kw[h2]);
-            vv[u][2 * h2] = bf16lo(vw[h2]); vv[u][2 * h2 + 1] = bf16hi(vw[h2]);
-          }
-        } else {
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            kv[u][e] = to_f(kbase[kp * HD + e]);
-            vv[u][e] = to_f(vbase[kp * HD + e]);
-          }
-        }
+  __syncthreads();
+  const uint32_t rows_bytes = static_cast<uint32_t>(nk) * HD * sizeof(T);
+  if (threadIdx.x == 0) {
+    sm100::mbar_arrive_expect_tx(&bar, 2 * rows_bytes);
+    sm100::bulk_load(sK, kbase + k0 * HD, rows_bytes, &bar);
+    sm100::bulk_load(sV, vbase + k0 * HD, rows_bytes, &bar);
+  }
+  {
+    // every thread waits (bounded); on a timeout the copies must still land before the block
+    // leaves, so wait again without the abort shortcut (also bounded)
+    int dummy_abort = 0;
+    bool ok = sm100::mbar_wait(&bar, 0, &dummy_abort, err, DEVERR_WAIT_FULL);
+    if (!ok) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!sm100::mbar_try_wait(&bar, 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
       }
     }
+    if (threadIdx.x == 0) s_ok = 1;
+    __syncthreads();
+    if (!ok) s_ok = 0;
+    __syncthreads();
+    if (!s_ok) return;
+  }
+  // the new token: patch its staged rows from the projection and append it to the cache
+  if (kv_len >= k0 && kv_len < k0 + nk) {
+    const int r = static_cast<int>(kv_len - k0);
+    for (int e = threadIdx.x; e < HD; e += blockDim.x) {
+      const T kvv = knew[e], vvv = vnew[e];
+      sK[static_cast<size_t>(r) * HD + e] = kvv;
+      sV[static_cast<size_t>(r) * HD + e] = vvv;
+      kbase[kv_len * HD + e] = kvv;
+      vbase[kv_len * HD + e] = vvv;
+    }
+  }
+  __syncthreads();
+
+  // ---- phase 1: scores
+  {
+    const int kslot = lane / LPK;
+    const int d0 = (lane % LPK) * 8;
+    float q[GROUP][8];
 #pragma unroll
-    for (int u = 0; u < kUnroll; ++u) {
+    for (int a = 0; a < GROUP; ++a) {
+      const T* qp = qkv + ix.q(bi, g * GROUP + a) + d0;
+#pragma unroll
+      for (int e = 0; e < 8; ++e) q[a][e] = to_f(qp[e]) * sl2;
+    }
+    const int stride = kWarps * KPW;
+    for (int wb = warp * KPW; wb < nk; wb += stride) {   // warp-uniform trip count
+      const int i = wb + kslot;
+      const bool ok = i < nk;
+      float kv[8];
+      const int ii = ok ? i : 0;
+      if constexpr (sizeof(T) == 2) {
+        const uint4 w = *reinterpret_cast<const uint4*>(sK + static_cast<size_t>(ii) * HD + d0);
+        const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
+#pragma unroll
+        for (int h2 = 0; h2 < 4; ++h2) {
+          kv[2 * h2] = bf16lo(ww[h2]);
+          kv[2 * h2 + 1] = bf16hi(ww[h2]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) kv[e] = to_f(sK[static_cast<size_t>(ii) * HD + d0 + e]);
+      }
 #pragma unroll
       for (int a = 0; a < GROUP; ++a) {
         float dot = 0.f;
 #pragma unroll
-        for (int e = 0; e < 8; ++e) dot = fmaf(q[a][e], kv[u][e], dot);
+        for (int e = 0; e < 8; ++e) dot = fmaf(q[a][e], kv[e], dot);
 #pragma unroll
         for (int off = LPK / 2; off > 0; off >>= 1) dot += __shfl_xor_sync(0xffffffffu, dot, off);
-        if (ok[u]) {
-          const float mn = fmaxf(m[a], dot);
-          const float corr = __expf(m[a] - mn), pw = __expf(dot - mn);
-          l[a] = l[a] * corr + pw;
+        if (ok && (lane % LPK) == 0) s_p[i * GROUP + a] = dot;
+      }
+    }
+  }
+  __syncthreads();
+  // ---- phase 2: per query head, max and exp over the chunk (one warp per head)
+  for (int a = warp; a < GROUP; a += kWarps) {
+    float mx = -INFINITY;
+    for (int i = lane; i < nk; i += 32) mx = fmaxf(mx, s_p[i * GROUP + a]);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[a][e] = acc[a][e] * corr + pw * vv[u][e];
-          m[a] = mn;
+    for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
+    float sum = 0.f;
+    for (int i = lane; i < nk; i += 32) {
+      const float pv = exp2f(s_p[i * GROUP + a] - mx);
+      s_p[i * GROUP + a] = pv;
+      sum += pv;
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
+    if (lane == 0) {
+      s_m[a] = mx;
+      s_l[a] = sum;
+    }
+  }
+  __syncthreads();
+  // ---- phase 3: o_a[d] = sum_key p[key][a] v[key][d]
+  {
+    const int d = threadIdx.x % HD;
+    const int a0 = (threadIdx.x / HD) * APT;
+    float acc[APT];
+#pragma unroll
+    for (int t = 0; t < APT; ++t) acc[t] = 0.f;
+    if (a0 < GROUP) {
+#pragma unroll 8
+      for (int i = 0; i < nk; ++i) {
+        const float v = to_f(sV[static_cast<size_t>(i) * HD + d]);
+#pragma unroll
+        for (int t = 0; t < APT; ++t)
+          if (a0 + t < GROUP) acc[t] = fmaf(s_p[i * GROUP + a0 + t], v, acc[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < APT; ++t) {
+        const int a = a0 + t;
+        if (a < GROUP) {
+          const int j = g * GROUP + a;
+          float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * (2 + HD);
+          if (d == 0) {
+            rec[0] = s_m[a];   // in log2 units (the scores carry log2(e))
+            rec[1] = s_l[a];
+          }
+          rec[2 + d] = acc[t];
         }
       }
     }
   }
-  // combine the warp's key slots (lanes that hold the same dims) with a fixed butterfly, then
-  // the warps in a fixed order: deterministic from run to run
-#pragma unroll
-  for (int a = 0; a < GROUP; ++a) {
-#pragma unroll
-    for (int off = LPK; off < 32; off <<= 1) {
-      const float mo = __shfl_xor_sync(0xffffffffu, m[a], off);
-      const float lo = __shfl_xor_sync(0xffffffffu, l[a], off);
-      const float mn = fmaxf(m[a], mo);
-      const float f1 = m[a] == -INFINITY ? 0.f : __expf(m[a] - mn);
-      const float f2 = mo == -INFINITY ? 0.f : __expf(mo - mn);
-      l[a] = l[a] * f1 + lo * f2;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) {
-        const float ao = __shfl_xor_sync(0xffffffffu, acc[a][e], off);
-        acc[a][e] = acc[a][e] * f1 + ao * f2;
-      }
-      m[a] = mn;
-    }
+  // the last block of this (sequence, KV head) to finish merges all splits, in split order:
+  // o = sum_c exp(m_c - M) o_c / sum_c exp(m_c - M) l_c   (no block waits for another)
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* cnt = counters + bi * n_kv + g;
+    const int last = atomicAdd(cnt, 1) == static_cast<int>(gridDim.x) - 1;
+    if (last) *cnt = 0;
+    s_last = last;
   }
-  if (lane < LPK) {
-#pragma unroll
-    for (int a = 0; a < GROUP; ++a) {
-      if (lane == 0) {
-        s_m[warp][a] = m[a];
-        s_l[warp][a] = l[a];
-      }
-#pragma unroll
-      for (int e = 0; e < 8; ++e) s_o[warp][a][d0 + e] = acc[a][e];
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // weights w[a][c] = exp(m_c - M_a) / L_a of every split, then independent loads of the o_c
+  constexpr int kMaxSplits = 64;
+  __shared__ float s_w[GROUP][kMaxSplits];
+  const int splits = gridDim.x;   // <= kMaxSplits (host)
+  const float* recs = ml + (bi * n_q + static_cast<int64_t>(g) * GROUP) * splits * (2 + HD);
+  for (int idx = threadIdx.x; idx < GROUP * splits; idx += blockDim.x) {
+    const int a = idx / splits, sp = idx - a * splits;
+    s_w[a][sp] = __ldcg(recs + (static_cast<int64_t>(a) * splits + sp) * (2 + HD));   // m
+  }
+  __syncthreads();
+  if (threadIdx.x < GROUP) {
+    const int a = threadIdx.x;
+    float M = -INFINITY;
+    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, s_w[a][sp]);
+    float Ls = 0.f;
+    for (int sp = 0; sp < splits; ++sp) {
+      const float f = s_w[a][sp] == -INFINITY ? 0.f : exp2f(s_w[a][sp] - M);
+      s_w[a][sp] = f;
+      Ls += __ldcg(recs + (static_cast<int64_t>(a) * splits + sp) * (2 + HD) + 1) * f;
     }
+    const float inv = 1.f / Ls;
+    for (int sp = 0; sp < splits; ++sp) s_w[a][sp] *= inv;
   }
   __syncthreads();
   for (int idx = threadIdx.x; idx < GROUP * HD; idx += blockDim.x) {
     const int a = idx / HD, e = idx - a * HD;
-    float mm = -INFINITY;
-    for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, s_m[w][a]);
-    float ll = 0.f, oo = 0.f;
-    for (int w = 0; w < kWarps; ++w) {
-      const float f = s_m[w][a] == -INFINITY ? 0.f : __expf(s_m[w][a] - mm);
-      ll += s_l[w][a] * f;
-      oo += s_o[w][a][e] * f;
-    }
-    const int j = g * GROUP + a;
-    float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * (2 + HD);
-    if (e == 0) {
-      rec[0] = mm;
-      rec[1] = ll;
-    }
-    rec[2 + e] = oo;
-  }
-}
-
-// Merge the splits: o[bi][j*hd + e] = sum_c exp(m_c - M) o_c / sum_c exp(m_c - M) l_c.
-template <typename T>
-__global__ void decode_combine_kernel(const float* ml, int splits, int hd, int64_t rows, T* o) {
-  const int64_t total = rows * hd;
-  for (int64_t idx = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; idx < total;
-       idx += static_cast<int64_t>(gridDim.x) * blockDim.x) {
-    const int64_t r = idx / hd;
-    const int e = static_cast<int>(idx - r * hd);
-    const float* rec = ml + r * splits * (2 + hd);
-    float M = -INFINITY;
-    for (int c = 0; c < splits; ++c) M = fmaxf(M, rec[c * (2 + hd)]);
-    float L = 0.f, acc = 0.f;
-    for (int c = 0; c < splits; ++c) {
-      const float* rc = rec + c * (2 + hd);
-      const float f = rc[0] == -INFINITY ? 0.f : expf(rc[0] - M);
-      L += rc[1] * f;
-      acc += rc[2 + e] * f;
-    }
-    o[idx] = from_f<T>(acc / L);
+    const float* r = recs + static_cast<int64_t>(a) * splits * (2 + HD) + 2 + e;
+    float acc2 = 0.f;
+#pragma unroll 8
+    for (int sp = 0; sp < splits; ++sp) acc2 += s_w[a][sp] * __ldcg(r + static_cast<int64_t>(sp) * (2 + HD));
+    o[bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + e] = from_f<T>(acc2);
   }
 }
 
@@ -401,7 +472,7 @@ __global__ void decode_combine_kernel(const float* ml, int splits, int hd, int64
 
 template <typename T>
 inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, void* kc, void* vc,
-                           float* ml, cudaStream_t s) {
+                           float* ml, int* counters, cudaStream_t s) {
   const T* qkv = static_cast<const T*>(qkv_v);
   T* o = static_cast<T*>(o_v);
   attn::QkvIdx ix{L.p * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
@@ -424,24 +495,22 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
     TP_LAUNCH_CHECK();
     return TP_OK;
   }
-  // decode: append, split-KV attention, combine
-  {
-    const int64_t total = L.b * L.n_kv * L.hd;
-    ProfScope prof(s, "kv_append");
-    attn::kv_append_kernel<T><<<simt::elementwise_grid(total), 256, 0, s>>>(
-        qkv, ix, static_cast<T*>(kc), static_cast<T*>(vc), L.b, L.n_kv, L.kv_cap, L.kv_len);
-    TP_LAUNCH_CHECK();
-  }
+  // decode: split-KV attention that also appends the new key/value and merges its splits
   const int group = L.n_q / L.n_kv;
   dim3 grid(static_cast<unsigned>(L.kv_splits), static_cast<unsigned>(L.n_kv),
             static_cast<unsigned>(L.b));
   if (L.b > 65535) return set_error(TP_ERR_UNSUPPORTED, "decode batch above 65535");
-  const int64_t n_keys = L.kv_len + 1;
+  TP_CUDA_TRY(cudaMemsetAsync(counters, 0, static_cast<size_t>(L.b * L.n_kv) * sizeof(int), s));
 #define TP_DECODE_CASE(G, H)                                                                  \
   if (group == G && L.hd == H) {                                                              \
+    const size_t smem = attn::DecodeSmem<H, G, T>::bytes(L.kv_chunk);                         \
+    TP_CUDA_TRY(cudaFuncSetAttribute(attn::decode_split_kernel<T, G, H>,                      \
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize,             \
+                                     static_cast<int>(smem)));                                \
     ProfScope prof(s, "attn_decode");                                                         \
-    attn::decode_split_kernel<T, G, H><<<grid, 256, 0, s>>>(qkv, ix, static_cast<const T*>(kc),  \
-        static_cast<const T*>(vc), L.kv_cap, n_keys, L.n_q, L.n_kv, scale, ml);               \
+    attn::decode_split_kernel<T, G, H><<<grid, 256, smem, s>>>(qkv, ix, static_cast<T*>(kc),  \
+        static_cast<T*>(vc), L.kv_cap, L.kv_len, L.kv_chunk, L.n_q, L.n_kv, scale, ml,        \
+        counters, o, device_error_word());                                                    \
     TP_LAUNCH_CHECK();                                                                        \
   } else
   TP_DECODE_CASE(8, 128) TP_DECODE_CASE(4, 128) TP_DECODE_CASE(2, 128) TP_DECODE_CASE(1, 128)
@@ -452,11 +521,6 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
                      "decode supports head_dim in {32, 64, 128} and n_q/n_kv in {1, 2, 4, 8}");
   }
 #undef TP_DECODE_CASE
-  const int64_t rows = L.b * L.n_q;
-  ProfScope prof(s, "attn_decode_combine");
-  attn::decode_combine_kernel<T><<<simt::elementwise_grid(rows * L.hd), 256, 0, s>>>(
-      ml, L.kv_splits, L.hd, rows, o);
-  TP_LAUNCH_CHECK();
   return TP_OK;
 }
 
@@ -565,12 +629,13 @@ inline tp_status attn_simt_proj(const AttnLayout& L, const void* x, const void* 
 
 inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wqkv,
                               const void* wo_p, void* kc, void* vc, const void* residual,
-                              void* y, void* ws, cudaStream_t s) {
+                              void* y, void* y_norm, void* ws, cudaStream_t s) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   void* qkv = w + L.qkv_off;
   void* o = w + L.o_off;
   float* part = reinterpret_cast<float*>(w + L.part_off);
   float* ml = reinterpret_cast<float*>(w + L.ml_off);
+  int* counters = reinterpret_cast<int*>(w + L.cnt_off);
   tp_status st;
   if (L.tc) {
     if (!tensor_cores_usable())
@@ -581,18 +646,23 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
     void* sk = w + L.sk_off;
     const size_t skb = L.ws_bytes - L.sk_off;
     if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, sk, skb, s)) != TP_OK) return st;
-    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
     if ((st = attn_tc::out_proj(L, o, wo_p, part, residual, y, sk, skb, s)) != TP_OK) return st;
-    if (L.reduce_mode == TP_REDUCE_FUSED) return TP_OK;
+    if (L.reduce_mode == TP_REDUCE_FUSED)
+      return y_norm ? reduce::rmsnorm(y, L.y_dtype, L.tokens, L.h, L.norm_eps, y_norm, L.dtype, s)
+                    : TP_OK;
   } else if (L.dtype == TP_BF16) {
     if ((st = attn_simt_proj<__nv_bfloat16>(L, x, wqkv, qkv, o, wo_p, part, s, true)) != TP_OK) return st;
-    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
     if ((st = attn_simt_proj<__nv_bfloat16>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
   } else {
     if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, true)) != TP_OK) return st;
-    if ((st = attn_core<float>(L, qkv, o, kc, vc, ml, s)) != TP_OK) return st;
+    if ((st = attn_core<float>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
     if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
   }
+  if (y_norm)
+    return reduce::reduce_norm(part, L.p, L.tokens, L.h, residual, y, L.y_dtype, y_norm, L.dtype,
+                               L.norm_eps, s);
   return reduce::launch(part, TP_F32, L.p, L.tokens * L.h, residual, y, L.y_dtype, s);
 }
 

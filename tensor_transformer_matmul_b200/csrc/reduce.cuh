@@ -139,6 +139,104 @@ inline tp_status launch(const void* part, int in_dtype, int p, int64_t n, const 
   return launch_t<__nv_bfloat16, __nv_bfloat16>(part, p, n, res, out, s);
 }
 
+// Reduce and normalize one row per block (512 threads): out = res + sum_s part[s] (in order,
+// fp32, one rounding), then norm = out / sqrt(mean(out^2) + eps) from the stored out values.
+// VEC (p <= 8): 8 consecutive elements per thread, all p loads issued before the in-order adds.
+template <typename Tin, typename Tout, typename Tn, bool VEC>
+__global__ void __launch_bounds__(512) reduce_norm_rows_kernel(const Tin* __restrict__ part, int p,
+                                                                int64_t rows, int64_t d,
+                                                                const Tout* res, Tout* out,
+                                                                Tn* norm, float eps) {
+  __shared__ float red[16];
+  const int64_t n = rows * d;
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * d;
+  float ss = 0.f;
+  if (VEC) {
+    for (int64_t j = 8 * static_cast<int64_t>(threadIdx.x); j < d; j += 8 * blockDim.x) {
+      float v[8][8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (q < p) Vec8<Tin>::load(part + static_cast<int64_t>(q) * n + base + j, v[q]);
+      float acc[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = v[0][e];
+#pragma unroll
+      for (int t = 1; t < 8; ++t)
+        if (t < p) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += v[t][e];
+        }
+      if (res) {
+        float r[8];
+        Vec8<Tout>::load(res + base + j, r);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = r[e] + acc[e];
+      }
+      Vec8<Tout>::store(out + base + j, acc);
+      float st[8];
+      Vec8<Tout>::load(out + base + j, st);   // the stored (rounded) values
+#pragma unroll
+      for (int e = 0; e < 8; ++e) ss = fmaf(st[e], st[e], ss);
+    }
+  } else {
+    for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
+      float acc = to_f(part[base + j]);
+      for (int q = 1; q < p; ++q) acc += to_f(part[static_cast<int64_t>(q) * n + base + j]);
+      if (res) acc = to_f(res[base + j]) + acc;
+      const Tout y = from_f<Tout>(acc);
+      out[base + j] = y;
+      const float yv = to_f(y);
+      ss = fmaf(yv, yv, ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  for (int64_t j = threadIdx.x; j < d; j += blockDim.x)
+    norm[base + j] = from_f<Tn>(to_f(out[base + j]) * scale);
+}
+
+template <typename Tin, typename Tout, typename Tn>
+inline void reduce_norm_launch(const void* part, int p, int64_t rows, int64_t d, const void* res,
+                               void* out, void* norm, float eps, cudaStream_t s) {
+  const bool vec = p <= 8 && d % 8 == 0 && (reinterpret_cast<uintptr_t>(part) & 31) == 0 &&
+                   (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
+                   (!res || (reinterpret_cast<uintptr_t>(res) & 15) == 0);
+  if (vec)
+    reduce_norm_rows_kernel<Tin, Tout, Tn, true><<<static_cast<unsigned>(rows), 512, 0, s>>>(
+        static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
+        static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
+  else
+    reduce_norm_rows_kernel<Tin, Tout, Tn, false><<<static_cast<unsigned>(rows), 512, 0, s>>>(
+        static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
+        static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
+}
+
+// y = res + sum of fp32 partials [p][rows][d]; norm = RMSNorm(y) in norm_dtype
+inline tp_status reduce_norm(const float* part, int p, int64_t rows, int64_t d, const void* res,
+                             void* out, int out_dtype, void* norm, int norm_dtype, float eps,
+                             cudaStream_t s) {
+  if (rows == 0) return TP_OK;
+  if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
+  ProfScope prof(s, "reduce_partials");
+  const bool ob = out_dtype == TP_BF16, nb = norm_dtype == TP_BF16;
+  if (ob && nb) reduce_norm_launch<float, __nv_bfloat16, __nv_bfloat16>(part, p, rows, d, res, out, norm, eps, s);
+  else if (ob) reduce_norm_launch<float, __nv_bfloat16, float>(part, p, rows, d, res, out, norm, eps, s);
+  else if (nb) reduce_norm_launch<float, float, __nv_bfloat16>(part, p, rows, d, res, out, norm, eps, s);
+  else reduce_norm_launch<float, float, float>(part, p, rows, d, res, out, norm, eps, s);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
 // out[r] = x[r] / sqrt(mean(x[r]^2) + eps), one block per row.
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* x, int64_t d, float eps,

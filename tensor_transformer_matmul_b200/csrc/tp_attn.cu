@@ -31,8 +31,8 @@ extern "C" tp_status tp_attn_pack(const tp_attn_desc* desc, const void* wq, cons
 
 extern "C" tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const void* wqkv_p,
                                  const void* wo_p, void* k_cache, void* v_cache,
-                                 const void* residual, void* y, void* workspace, size_t ws_bytes,
-                                 void* stream) {
+                                 const void* residual, void* y, void* y_norm, void* workspace,
+                                 size_t ws_bytes, void* stream) {
   tp::clear_error();
   tp::AttnLayout L;
   tp_status st = tp::attn_layout_of(desc, &L);
@@ -47,9 +47,11 @@ extern "C" tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const 
   if (!x || !wqkv_p || !wo_p || !y) return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
   if (L.kv_len > 0 && (!k_cache || !v_cache))
     return tp::set_error(TP_ERR_INVALID_ARG, "decode needs k_cache and v_cache");
+  if (L.kv_len > 0 && ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15))
+    return tp::set_error(TP_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
   if (!workspace) return tp::set_error(TP_ERR_INVALID_ARG, "workspace is null");
   if (ws_bytes < L.ws_bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
-  st = tp::attn_forward(L, x, wqkv_p, wo_p, k_cache, v_cache, residual, y, workspace,
+  st = tp::attn_forward(L, x, wqkv_p, wo_p, k_cache, v_cache, residual, y, y_norm, workspace,
                         static_cast<cudaStream_t>(stream));
   if (st == TP_OK) tp::count_reduction();
   return st;

@@ -31,6 +31,7 @@ constexpr int stages_for(int bn, int a_sub) {
 struct MlpLayout {
   int64_t T, d, F, Fs, Fsp, R;
   int p, act, dtype, eb, y_dtype, reduce_mode;
+  float norm_eps;
   bool tc;                      // bf16 with 16-byte rows: the tensor-core path
   size_t w1p_bytes, w2p_bytes;
   size_t saved_z_off, saved_h_off, saved_bytes;
@@ -96,6 +97,7 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
   L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
   L->reduce_mode = desc->reduce_mode;
+  L->norm_eps = desc->norm_eps > 0.f ? desc->norm_eps : 1e-5f;
   L->tc = desc->dtype == TP_BF16 && desc->d % 8 == 0;
   L->Fs = L->F / L->p;
   L->Fsp = round_up(L->Fs, 128);
@@ -459,8 +461,8 @@ extern "C" tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw
 }
 
 extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p,
-                                const void* w2p, const void* residual, void* y, void* saved,
-                                void* workspace, size_t ws_bytes, void* stream) {
+                                const void* w2p, const void* residual, void* y, void* y_norm,
+                                void* saved, void* workspace, size_t ws_bytes, void* stream) {
   clear_error();
   MlpLayout L;
   tp_status st = layout_of(desc, &L);
@@ -491,6 +493,8 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
     if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
     if ((st = tc_down(L, h, w2p, part, residual, y, sk, skb, s)) != TP_OK) return st;
     if (L.reduce_mode == TP_REDUCE_FUSED) {
+      if (y_norm && (st = reduce::rmsnorm(y, L.y_dtype, L.T, L.d, L.norm_eps, y_norm, L.dtype, s)) != TP_OK)
+        return st;
       count_reduction();
       return TP_OK;
     }
@@ -499,7 +503,9 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
   } else {
     if ((st = simt_forward<float>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
   }
-  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.y_dtype, s);
+  st = y_norm ? reduce::reduce_norm(part, L.p, L.T, L.d, residual, y, L.y_dtype, y_norm, L.dtype,
+                                    L.norm_eps, s)
+              : reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.y_dtype, s);
   if (st == TP_OK) count_reduction();
   return st;
 }

@@ -66,7 +66,7 @@ extern "C" tp_status tp_mlp_fwd_static_ws(const tp_mlp_desc* desc, const void* x
   if (need == 0) {
     // an invalid shape (reported by tp_mlp_fwd) or an empty batch (T = 0, nothing to compute):
     // neither touches scratch
-    return tp_mlp_fwd(desc, x, w1p, w2p, residual, y, nullptr, nullptr, 0, stream);
+    return tp_mlp_fwd(desc, x, w1p, w2p, residual, y, nullptr, nullptr, nullptr, 0, stream);
   }
   if (need > kStaticWsBytes)
     return tp::set_error(TP_ERR_WORKSPACE,
@@ -76,5 +76,5 @@ extern "C" tp_status tp_mlp_fwd_static_ws(const tp_mlp_desc* desc, const void* x
   void* ws = nullptr;
   tp_status st = static_ws_address(&ws);
   if (st != TP_OK) return st;
-  return tp_mlp_fwd(desc, x, w1p, w2p, residual, y, nullptr, ws, kStaticWsBytes, stream);
+  return tp_mlp_fwd(desc, x, w1p, w2p, residual, y, nullptr, nullptr, ws, kStaticWsBytes, stream);
 }

@@ -2,8 +2,11 @@
 
 Each layer, for a batch of b single-token sequences x (b, h):
 
-    x <- x + sum_i Attn_i(RMSNorm(x))        (tp_rmsnorm, then tp_attn_fwd with residual = x)
-    x <- x + sum_i MLP_i(RMSNorm(x))         (tp_rmsnorm, then tp_mlp_fwd with residual = x)
+    x <- x + sum_i Attn_i(RMSNorm(x))        (tp_attn_fwd with residual = x)
+    x <- x + sum_i MLP_i(RMSNorm(x))         (tp_mlp_fwd with residual = x)
+
+Each reduction also writes RMSNorm of its result (the y_norm output), which is the next
+sublayer's input, so the only separate normalization is the first one of a step.
 
 "How does tensor parallelism split a transformer feed-forward block's two matmuls", "One
 collective": after the reduction the full y is "ready for the residual add and the following
@@ -60,19 +63,21 @@ class DecodeStack:
         ws = max(tp.tp_attn_fwd_workspace(self.adesc), tp.tp_mlp_fwd_workspace(self.mdesc))
         self.ws = torch.empty(ws, dtype=torch.uint8, device=self.device)
         self.normed = torch.empty(b, 1, h, dtype=torch.bfloat16, device=self.device)
+        self.normed2 = torch.empty(b, 1, h, dtype=torch.bfloat16, device=self.device)
         self.graph = None
 
     def step(self, x):
         """One decode step over all layers; x (b, 1, h) float32 on the device, updated in place."""
-        for lay in self.layers:
-            tp.tp_rmsnorm(x, self.normed)
+        tp.tp_rmsnorm(x, self.normed)
+        for li, lay in enumerate(self.layers):
             tp.tp_attn_fwd(self.adesc, self.normed, lay["wqkv"], lay["wo"], x,
                            k_cache=lay["k_cache"], v_cache=lay["v_cache"], residual=x,
-                           workspace=self.ws)
-            tp.tp_rmsnorm(x, self.normed)
-            tp.tp_mlp_fwd(self.mdesc, self.normed.view(self.b, self.h), lay["w1p"], lay["w2p"],
+                           workspace=self.ws, y_norm=self.normed2)
+            last = li == len(self.layers) - 1
+            tp.tp_mlp_fwd(self.mdesc, self.normed2.view(self.b, self.h), lay["w1p"], lay["w2p"],
                           x.view(self.b, self.h), residual=x.view(self.b, self.h),
-                          workspace=self.ws)
+                          workspace=self.ws,
+                          y_norm=None if last else self.normed.view(self.b, self.h))
         return x
 
     def capture(self, x):

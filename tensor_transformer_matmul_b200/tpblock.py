@@ -45,7 +45,8 @@ class TpError(RuntimeError):
 class tp_mlp_desc(ctypes.Structure):
     _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("d_ff", ctypes.c_int64),
                 ("p", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
-                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("norm_eps", ctypes.c_float)]
 
 
 class tp_attn_desc(ctypes.Structure):
@@ -53,7 +54,8 @@ class tp_attn_desc(ctypes.Structure):
                 ("n_q", ctypes.c_int32), ("n_kv", ctypes.c_int32), ("head_dim", ctypes.c_int32),
                 ("p", ctypes.c_int32), ("causal", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("kv_len", ctypes.c_int64), ("kv_cap", ctypes.c_int64),
-                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32)]
+                ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32),
+                ("norm_eps", ctypes.c_float), ("reserved", ctypes.c_int32)]
 
 
 _lib = None
@@ -74,14 +76,14 @@ def load():
         "tp_mlp_w1_packed_bytes": (S, [MD]), "tp_mlp_w2_packed_bytes": (S, [MD]),
         "tp_mlp_pack": (I32, [MD, P, P, P, P, P, P]), "tp_mlp_saved_bytes": (S, [MD]),
         "tp_mlp_fwd_workspace": (S, [MD]),
-        "tp_mlp_fwd": (I32, [MD, P, P, P, P, P, P, P, S, P]),
+        "tp_mlp_fwd": (I32, [MD, P, P, P, P, P, P, P, P, S, P]),
         "tp_mlp_bwd_workspace": (S, [MD]),
         "tp_mlp_bwd": (I32, [MD, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_mlp_unpack_grads": (I32, [MD, P, P, P, P, P, P]),
         "tp_mlp_fwd_static_ws": (I32, [MD, P, P, P, P, P, P]),
         "tp_attn_wqkv_packed_bytes": (S, [AD]), "tp_attn_wo_packed_bytes": (S, [AD]),
         "tp_attn_pack": (I32, [AD, P, P, P, P, P, P, P]), "tp_attn_fwd_workspace": (S, [AD]),
-        "tp_attn_fwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_fwd": (I32, [AD, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_reduce_partials": (I32, [P, I32, I64, I32, P, P, I32, P]),
         "tp_rmsnorm": (I32, [P, I32, I64, I64, F32, P, I32, P]),
         "tp_reduction_count": (ctypes.c_uint64, []), "tp_reset_reduction_count": (None, []),
@@ -138,7 +140,7 @@ def _nbytes(t):
 def mlp_desc(T, d, d_ff, p, act="swiglu", dtype="bf16", reduce_mode=TP_REDUCE_SEPARATE, flags=0):
     return tp_mlp_desc(int(T), int(d), int(d_ff), int(p), ACT[act] if isinstance(act, str) else int(act),
                        DTYPE[dtype] if isinstance(dtype, str) else int(dtype), int(reduce_mode),
-                       int(flags))
+                       int(flags), 0.0)
 
 
 def tp_mlp_w1_packed_bytes(desc):
@@ -166,10 +168,11 @@ def tp_mlp_pack(desc, w1, w_up, w2, w1p, w2p, stream=None):
                               _ptr(w2p), _stream(stream)))
 
 
-def tp_mlp_fwd(desc, x, w1p, w2p, y, residual=None, saved=None, workspace=None, stream=None):
+def tp_mlp_fwd(desc, x, w1p, w2p, y, residual=None, saved=None, workspace=None, stream=None,
+               y_norm=None):
     _check(load().tp_mlp_fwd(ctypes.byref(desc), _ptr(x), _ptr(w1p), _ptr(w2p), _ptr(residual),
-                             _ptr(y), _ptr(saved), _ptr(workspace), _nbytes(workspace),
-                             _stream(stream)))
+                             _ptr(y), _ptr(y_norm), _ptr(saved), _ptr(workspace),
+                             _nbytes(workspace), _stream(stream)))
 
 
 def tp_mlp_bwd(desc, dy, x, saved, w1p, w2p, dx, dw1p, dw2p, workspace=None, stream=None):
@@ -195,7 +198,7 @@ def attn_desc(b, s, h, n_q, n_kv, head_dim, p, causal=True, dtype="bf16", kv_len
               reduce_mode=TP_REDUCE_SEPARATE, flags=0):
     return tp_attn_desc(int(b), int(s), int(h), int(n_q), int(n_kv), int(head_dim), int(p),
                         int(bool(causal)), DTYPE[dtype] if isinstance(dtype, str) else int(dtype),
-                        int(kv_len), int(kv_cap), int(reduce_mode), int(flags))
+                        int(kv_len), int(kv_cap), int(reduce_mode), int(flags), 0.0, 0)
 
 
 def tp_attn_wqkv_packed_bytes(desc):
@@ -216,10 +219,11 @@ def tp_attn_pack(desc, wq, wk, wv, wo, wqkv_p, wo_p, stream=None):
 
 
 def tp_attn_fwd(desc, x, wqkv_p, wo_p, y, k_cache=None, v_cache=None, residual=None,
-                workspace=None, stream=None):
+                workspace=None, stream=None, y_norm=None):
     _check(load().tp_attn_fwd(ctypes.byref(desc), _ptr(x), _ptr(wqkv_p), _ptr(wo_p),
                               _ptr(k_cache), _ptr(v_cache), _ptr(residual), _ptr(y),
-                              _ptr(workspace), _nbytes(workspace), _stream(stream)))
+                              _ptr(y_norm), _ptr(workspace), _nbytes(workspace),
+                              _stream(stream)))
 
 
 # ------------------------------------------------------------------------- reduce and glue

@@ -74,7 +74,7 @@ def test_attn_layout_sizes(lib):
 def test_mlp_shape_errors(lib, T, d, F, p, status):
     desc = lib.mlp_desc(T, d, F, p, "gelu", "f32")
     so = lib.load()
-    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None)
+    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, None, 0, None)
     assert so.tp_status_string(st).decode() == status
     assert lib.tp_mlp_fwd_workspace(desc) == 0
     assert lib.tp_last_error() != ""
@@ -83,22 +83,22 @@ def test_mlp_shape_errors(lib, T, d, F, p, status):
 def test_mlp_argument_errors(lib):
     so = lib.load()
     desc = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32")
-    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None)
+    st = so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, None, 0, None)
     assert st == lib.TP_ERR_INVALID_ARG  # null x
     fake = ctypes.c_void_p(0x1000)
-    st = so.tp_mlp_fwd(ctypes.byref(desc), fake, fake, fake, None, fake, None, fake, 16, None)
+    st = so.tp_mlp_fwd(ctypes.byref(desc), fake, fake, fake, None, fake, None, None, fake, 16, None)
     assert st == lib.TP_ERR_WORKSPACE
     bad = lib.mlp_desc(4, 8, 32, 4, 9, "f32")
-    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, None, fake, 1 << 30,
                          None) == lib.TP_ERR_INVALID_ARG
     bad = lib.mlp_desc(4, 8, 32, 4, "gelu", 7)
-    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, None, fake, 1 << 30,
                          None) == lib.TP_ERR_INVALID_ARG
     # SwiGLU needs w_up; the other activations must not get one
     sw = lib.mlp_desc(4, 8, 32, 4, "swiglu", "f32")
     assert so.tp_mlp_pack(ctypes.byref(sw), fake, None, fake, fake, fake, None) == lib.TP_ERR_INVALID_ARG
     assert so.tp_mlp_pack(ctypes.byref(desc), fake, fake, fake, fake, fake, None) == lib.TP_ERR_INVALID_ARG
-    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None) != 0
+    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, None, 0, None) != 0
 
 
 def test_attn_shape_errors(lib):
@@ -106,8 +106,8 @@ def test_attn_shape_errors(lib):
     fake = ctypes.c_void_p(0x1000)
 
     def st(desc):
-        return so.tp_attn_fwd(ctypes.byref(desc), fake, fake, fake, None, None, None, fake, fake,
-                              1 << 40, None)
+        return so.tp_attn_fwd(ctypes.byref(desc), fake, fake, fake, None, None, None, fake, None,
+                              fake, 1 << 40, None)
     # "Tensor Parallelism", Notes: with 8 KV heads, p = 16 cannot give every rank a whole KV head
     assert st(lib.attn_desc(1, 4, 64, 16, 8, 8, 16)) == lib.TP_ERR_SHAPE
     assert st(lib.attn_desc(1, 4, 64, 8, 3, 8, 1)) == lib.TP_ERR_SHAPE     # n_kv does not divide n_q
@@ -126,7 +126,7 @@ def test_reduce_argument_errors(lib):
     assert so.tp_rmsnorm(fake, 0, 2, 0, 1e-5, fake, 0, None) == lib.TP_ERR_SHAPE
     assert so.tp_rmsnorm(fake, 3, 2, 8, 1e-5, fake, 0, None) == lib.TP_ERR_INVALID_ARG
     bad = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32", flags=4)
-    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, fake, 1 << 30,
+    assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, None, fake, 1 << 30,
                          None) == lib.TP_ERR_INVALID_ARG
 
 
@@ -135,6 +135,6 @@ def test_empty_batch_counts_one_reduction(lib):
     so = lib.load()
     lib.tp_reset_reduction_count()
     desc = lib.mlp_desc(0, 8, 32, 4, "gelu", "f32")
-    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, 0, None) == 0
+    assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, None, 0, None) == 0
     assert lib.tp_reduction_count() == 1
     lib.tp_reset_reduction_count()

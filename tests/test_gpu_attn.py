@@ -159,3 +159,30 @@ def test_rmsnorm_dtypes(lib):
         lib.tp_rmsnorm(x, out)
         torch.cuda.synchronize()
         assert rel_l2(f64(out), odec.rmsnorm(f64(x))) <= tol
+
+
+@pytest.mark.parametrize("kv_len", [0, 200])
+def test_y_norm_output(lib, kv_len):
+    from oracle import decode as odec
+    s_len = 1 if kv_len else 40
+    inp = inputs.attn_inputs(2, s_len, 256, 8, 2, 64, "bf16", seed=11, w_std=0.05, kv_len=kv_len)
+    a = Attn(lib, inp, 2, "bf16", True, kv_len=kv_len, n_q=8, n_kv=2, hd=64)
+    res = torch.randn(2, s_len, 256, device=dev())
+    desc = lib.attn_desc(2, s_len, 256, 8, 2, 64, 2, True, "bf16", kv_len,
+                         flags=lib.TP_FLAG_F32_RESIDUAL)
+    y = torch.empty(2, s_len, 256, device=dev())
+    yn = torch.empty(2, s_len, 256, dtype=torch.bfloat16, device=dev())
+    kc = inp["k_cache"].to(dev()) if kv_len else None
+    vc = inp["v_cache"].to(dev()) if kv_len else None
+    lib.tp_attn_fwd(desc, inp["x"].to(dev()), a.wqkv, a.wo, y, k_cache=kc, v_cache=vc,
+                    residual=res, workspace=a.ws, y_norm=yn)
+    torch.cuda.synchronize()
+    if kv_len:
+        ref, _, _ = oattn.attention_decode(f64(inp["x"])[:, 0], *(f64(inp[k]) for k in ("wq", "wk", "wv", "wo")),
+                                           f64(inp["k_cache"])[:, :, :kv_len], f64(inp["v_cache"])[:, :, :kv_len],
+                                           8, 2, 64)
+        ref = ref[:, None] + f64(res)
+    else:
+        ref = _ref(inp, 8, 2, 64, True) + f64(res)
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
+    assert rel_l2(f64(yn), odec.rmsnorm(ref)) <= TOL["bf16"]

@@ -199,3 +199,22 @@ def test_fused_reduce_deterministic(lib):
     b = m.forward(inp["x"], save=False)
     torch.cuda.synchronize()
     assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("reduce_mode", [0, 1])
+@pytest.mark.parametrize("T", [1, 150])
+def test_y_norm_output(lib, reduce_mode, T):
+    # the reduction also writes RMSNorm(y): the replicated normalization after the residual add
+    from oracle import decode as odec
+    d, F, p = 256, 1024, 4
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=10, w_std=0.05)
+    m = Mlp(lib, inp, p, "swiglu", "bf16", reduce_mode)
+    res = inputs.normal((T, d), 1.0, 10, 99, "bf16", "cpu").to(dev())
+    y = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+    yn = torch.empty_like(y)
+    lib.tp_mlp_fwd(m.desc, inp["x"].to(dev()), m.w1p, m.w2p, y, residual=res, workspace=m.ws_f,
+                   y_norm=yn)
+    torch.cuda.synchronize()
+    ref = _oracle_fwd(inp, "swiglu") + f64(res)
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
+    assert rel_l2(f64(yn), odec.rmsnorm(ref)) <= TOL["bf16"]
