@@ -11,7 +11,10 @@
 //   out = O / l
 //
 // 128 threads: thread t owns query row t of the tile (TMEM lane t).  Thread 0 also issues the TMA
-// loads and the MMAs.  K/V blocks of 128 keys are double buffered.  All waits are bounded.
+// loads and the MMAs.  K/V blocks of 64 keys are double buffered; with head_dim 128 the bf16 P of
+// a block is written over that block's K tile (K is dead once S is computed), which keeps a CTA
+// under 100 KB of shared memory so two CTAs share an SM and one's softmax overlaps the other's
+// MMAs.  All waits are bounded.
 #pragma once
 
 #include <cuda.h>
@@ -23,21 +26,25 @@
 namespace tp {
 namespace fa {
 
-constexpr int kRows = 128;   // query rows per tile = keys per block
+constexpr int kRows = 128;   // query rows per tile
+constexpr int kKeys = 64;    // keys per K/V block
 constexpr int kThreads = 128;
 
 template <int HD>
 struct Smem {
   static constexpr int SUB = HD / 64;                 // 64-wide swizzle sub-tiles along the head dim
-  static constexpr int TILE = kRows * 128;            // one sub-tile: 128 rows x 128 bytes
+  static constexpr int QTILE = kRows * 128;           // Q sub-tile: 128 rows x 128 bytes
+  static constexpr int KTILE = kKeys * 128;           // K or V sub-tile: 64 rows x 128 bytes
+  static constexpr int PTILE = kRows * 128;           // P: 128 rows x 64 keys (bf16)
+  static constexpr bool P_IN_K = SUB * KTILE >= PTILE;   // P reuses the block's K buffer
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + SUB * TILE;    // 2 buffers
-  static constexpr int V_OFF = K_OFF + 2 * SUB * TILE;
-  static constexpr int P_OFF = V_OFF + 2 * SUB * TILE;  // 2 sub-tiles (128 keys)
-  static constexpr int BAR_OFF = P_OFF + 2 * TILE;
+  static constexpr int K_OFF = Q_OFF + SUB * QTILE;   // 2 buffers
+  static constexpr int V_OFF = K_OFF + 2 * SUB * KTILE;
+  static constexpr int P_OFF = V_OFF + 2 * SUB * KTILE;   // used only when !P_IN_K
+  static constexpr int BAR_OFF = P_OFF + (P_IN_K ? 0 : PTILE);
   static constexpr int BYTES = BAR_OFF + 128 + 1024;  // barriers + alignment slack
-  static constexpr int KV_BYTES = 2 * SUB * TILE;     // one K block + one V block
-  static constexpr uint32_t TMEM_COLS = 256;          // S (128 cols) + O (up to 128 cols)
+  static constexpr int KV_BYTES = 2 * SUB * KTILE;    // one K block + one V block
+  static constexpr uint32_t TMEM_COLS = 256;          // S (64 cols) + O (from col 128)
 };
 
 struct Params {
@@ -72,7 +79,7 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(kThreads, 2)
     flash_fwd_kernel(const __grid_constant__ CUtensorMap tma_qkv, const Params P) {
   using namespace sm100;
   using L = Smem<HD>;
@@ -99,8 +106,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_col = shard * P.R_a + (P.qh + gl) * HD;
   const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
   const int q0 = qt * kRows;
-  const int n_kb_all = (P.s + kRows - 1) / kRows;
-  const int nkb = P.causal ? min(qt + 1, n_kb_all) : n_kb_all;
+  const int n_kb_all = (P.s + kKeys - 1) / kKeys;
+  const int nkb = P.causal ? min((q0 + kRows) / kKeys, n_kb_all) : n_kb_all;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
@@ -127,26 +134,27 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
   uint8_t* sV = smem + L::V_OFF;
-  uint8_t* sP = smem + L::P_OFF;
 
   auto load_kv = [&](int kb) {
     const int buf = kb & 1;
     mbar_arrive_expect_tx(&kv_full[buf], L::KV_BYTES);
 #pragma unroll
     for (int c = 0; c < L::SUB; ++c) {
-      tma_load_3d(&tma_qkv, &kv_full[buf], sK + (buf * L::SUB + c) * L::TILE, k_col + 64 * c,
-                  kb * kRows, bi);
-      tma_load_3d(&tma_qkv, &kv_full[buf], sV + (buf * L::SUB + c) * L::TILE, v_col + 64 * c,
-                  kb * kRows, bi);
+      tma_load_3d(&tma_qkv, &kv_full[buf], sK + (buf * L::SUB + c) * L::KTILE, k_col + 64 * c,
+                  kb * kKeys, bi);
+      tma_load_3d(&tma_qkv, &kv_full[buf], sV + (buf * L::SUB + c) * L::KTILE, v_col + 64 * c,
+                  kb * kKeys, bi);
     }
   };
 
   uint32_t issued_kv = 0;       // blocks whose loads were issued (thread 0 only)
   if (tid == 0) {
-    mbar_arrive_expect_tx(q_full, L::SUB * L::TILE);
+    mbar_arrive_expect_tx(q_full, L::SUB * L::QTILE);
 #pragma unroll
-    for (int c = 0; c < L::SUB; ++c)
-      tma_load_3d(&tma_qkv, q_full, sQ + c * L::TILE, q_col + 64 * c, q0, bi);
+    for (int c = 0; c < L::SUB; ++c) {   // a Q sub-tile is two 64-row boxes
+      tma_load_3d(&tma_qkv, q_full, sQ + c * L::QTILE, q_col + 64 * c, q0, bi);
+      tma_load_3d(&tma_qkv, q_full, sQ + c * L::QTILE + L::KTILE, q_col + 64 * c, q0 + 64, bi);
+    }
     load_kv(0);
     issued_kv = 1;
     if (nkb > 1) {
@@ -156,7 +164,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
 
   // instruction descriptors: S = Q K^T (both K-major); O += P V (P K-major, V MN-major)
-  constexpr uint32_t IDESC_S = make_idesc_bf16(128, 128, false, false);
+  constexpr uint32_t IDESC_S = make_idesc_bf16(128, kKeys, false, false);
   constexpr uint32_t IDESC_O = make_idesc_bf16(128, HD, false, true);
 
   const int row = tid;                 // query row within the tile
@@ -173,35 +181,36 @@ __global__ void __launch_bounds__(kThreads, 1)
                         mbar_wait(&kv_full[buf], (kb >> 1) & 1, abort_flag, P.err, DEVERR_WAIT_FULL));
     if (w && tid == 0) {
       tc_fence_after();
-      const uint32_t qa = smem_addr(sQ), ka = smem_addr(sK + buf * L::SUB * L::TILE);
+      const uint32_t qa = smem_addr(sQ), ka = smem_addr(sK + buf * L::SUB * L::KTILE);
 #pragma unroll
       for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
-        umma_f16(tS, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                 IDESC_S, kk > 0 ? 1u : 0u);
+        const uint32_t koff = (kk & 3) * 32;
+        umma_f16(tS, make_sdesc_sw128(qa + (kk >> 2) * L::QTILE + koff, 16, 1024),
+                 make_sdesc_sw128(ka + (kk >> 2) * L::KTILE + koff, 16, 1024), IDESC_S,
+                 kk > 0 ? 1u : 0u);
       }
       umma_commit(s_done);
       issued_mma = true;
     }
     if (w) w = __all_sync(0xffffffffu, mbar_wait(s_done, kb & 1, abort_flag, P.err,
                                                    DEVERR_WAIT_ACC_FULL));
-    float sv[128];
+    float sv[kKeys];
     if (w) {
       tc_fence_after();
       // ---- online softmax on this thread's row of S
 #pragma unroll
-      for (int c = 0; c < 4; ++c) {
+      for (int c = 0; c < kKeys / 32; ++c) {
         uint32_t r[32];
         tmem_ld_32x32b_x32(tS + lane_base + c * 32, r);
         tmem_wait_ld();
 #pragma unroll
         for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
       }
-      const int k_base = kb * kRows;
-      const bool need_mask = (k_base + kRows > P.s) || (P.causal && k_base + kRows - 1 > q0);
+      const int k_base = kb * kKeys;
+      const bool need_mask = (k_base + kKeys > P.s) || (P.causal && k_base + kKeys - 1 > q0);
       float mx = -INFINITY;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < kKeys; ++c) {
         if (need_mask) {
           const int k_abs = k_base + c;
           if (k_abs >= P.s || (P.causal && k_abs > q_abs)) sv[c] = -INFINITY;
@@ -213,7 +222,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       const float mscaled = (m_new == -INFINITY) ? 0.f : m_new * P.scale_log2;
       float rs = 0.f;
 #pragma unroll
-      for (int c = 0; c < 128; ++c) {
+      for (int c = 0; c < kKeys; ++c) {
         const float pv = exp2f(sv[c] * P.scale_log2 - mscaled);   // exp2(-inf) = 0 when masked
         sv[c] = pv;
         rs += pv;
@@ -247,17 +256,18 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    // P of this block: over its K tile (dead after S) or in its own buffer
+    uint8_t* sP = L::P_IN_K ? sK + buf * L::SUB * L::KTILE : smem + L::P_OFF;
     if (w) {
-      // ---- P (bf16) into smem, K-major with the 128-byte swizzle: row `row`, 2 key sub-tiles
+      // ---- P (bf16) into smem, K-major with the 128-byte swizzle: row `row`, 64 keys
 #pragma unroll
-      for (int ch = 0; ch < 16; ++ch) {
-        const int sub = ch >> 3, q16 = ch & 7;
+      for (int ch = 0; ch < kKeys / 8; ++ch) {
         uint4 v4;
         v4.x = pack_bf16x2(sv[ch * 8 + 0], sv[ch * 8 + 1]);
         v4.y = pack_bf16x2(sv[ch * 8 + 2], sv[ch * 8 + 3]);
         v4.z = pack_bf16x2(sv[ch * 8 + 4], sv[ch * 8 + 5]);
         v4.w = pack_bf16x2(sv[ch * 8 + 6], sv[ch * 8 + 7]);
-        *reinterpret_cast<uint4*>(sP + sub * L::TILE + row * 128 + ((q16 ^ (row & 7)) << 4)) = v4;
+        *reinterpret_cast<uint4*>(sP + row * 128 + ((ch ^ (row & 7)) << 4)) = v4;
       }
       fence_proxy_async_smem();
     }
@@ -268,12 +278,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     if (tid == 0) {
       tc_fence_after();
-      const uint32_t pa = smem_addr(sP), va = smem_addr(sV + buf * L::SUB * L::TILE);
+      const uint32_t pa = smem_addr(sP), va = smem_addr(sV + buf * L::SUB * L::KTILE);
 #pragma unroll
-      for (int kk = 0; kk < kRows / 16; ++kk) {
-        const uint64_t adesc = make_sdesc_sw128(pa + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024);
-        // V tile: 64-dim blocks of 128 key rows (LBO = one sub-tile), 16 keys per MMA
-        const uint64_t bdesc = make_sdesc_sw128(va + kk * 16 * 128, L::TILE, 1024);
+      for (int kk = 0; kk < kKeys / 16; ++kk) {
+        const uint64_t adesc = make_sdesc_sw128(pa + kk * 32, 16, 1024);
+        // V tile: 64-dim blocks of 64 key rows (LBO = one sub-tile), 16 keys per MMA
+        const uint64_t bdesc = make_sdesc_sw128(va + kk * 16 * 128, L::KTILE, 1024);
         umma_f16(tO, adesc, bdesc, IDESC_O, (kb > 0 || kk > 0) ? 1u : 0u);
       }
       umma_commit(o_done);
@@ -339,7 +349,7 @@ inline tp_status launch(const void* qkv, int64_t b, int64_t s, int n_q, int qh, 
   const uint64_t cols = static_cast<uint64_t>(p) * R_a;
   tp_status r = encode_tmap_bf16_3d(&map, qkv, cols, static_cast<uint64_t>(s),
                                     static_cast<uint64_t>(b), cols * 2,
-                                    cols * 2 * static_cast<uint64_t>(s), 64, kRows);
+                                    cols * 2 * static_cast<uint64_t>(s), 64, kKeys);
   if (r != TP_OK) return r;
   static int attr_set[64] = {0};
   int dev = 0;
