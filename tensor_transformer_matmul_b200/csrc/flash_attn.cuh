@@ -4,17 +4,25 @@
 // FlashAttention's tiling of QK, softmax and V as the way to cut its HBM traffic).
 //
 //   S  = Q K_b^T                (tcgen05.mma, Q and K K-major in smem, S fp32 in TMEM)
-//   m' = max(m, rowmax(S)),  P = exp(S - m') (bf16, written to smem in the UMMA K-major layout),
-//   l  = l * exp(m - m') + rowsum(P),  O = O * exp(m - m')  (O fp32 in TMEM, rescaled only when
-//        some row's maximum moved)
+//   m' = max(m, rowmax(S)),  P = exp(S - m') (bf16),
+//   l  = l * exp(m - m') + rowsum(P),  O = O * exp(m - m')  (O fp32 in TMEM; m is only moved when
+//        the row maximum grew by more than 2^8, so the rescale is rare)
 //   O += P V_b                  (tcgen05.mma, V read MN-major straight from its [key][dim] tile)
 //   out = O / l
 //
-// 128 threads: thread t owns query row t of the tile (TMEM lane t).  Thread 0 also issues the TMA
-// loads and the MMAs.  K/V blocks of 64 keys are double buffered; with head_dim 128 the bf16 P of
-// a block is written over that block's K tile (K is dead once S is computed), which keeps a CTA
-// under 100 KB of shared memory so two CTAs share an SM and one's softmax overlaps the other's
-// MMAs.  All waits are bounded.
+// 128 threads, thread t owning query row t of the tile (TMEM lane t).  Thread 0 also issues the
+// TMA loads and the MMAs.  Key blocks are 128 keys, so every MMA is 128 x 128.  S and P share 128
+// TMEM columns (the bf16 P of a block is written over its S and read from there as the A operand
+// of P V, so P never touches shared memory) and O takes the other 128.  Q, K and V each have one
+// shared-memory buffer: K(kb+1) is fetched as soon as S(kb) is done, V(kb+1) as soon as P(kb)
+// V(kb) is done, each well ahead of its use.  A CTA needs 96 KB of shared memory and 256 TMEM
+// columns, so two CTAs share an SM and one's softmax runs while the other's MMAs do.
+//
+// The special-function unit computes 16 exponentials per clock per SM, which for this tile shape
+// is as slow as the tensor core, so three pairs of P values in eight are computed on the FMA pipe:
+// 2^x = 2^n * 2^f with n = round(x), f in [-1/2, 1/2], 2^f by a degree-3 polynomial (minimax fit
+// for relative error, max error 7.5e-5, below bf16's rounding of P), and n added to the exponent.
+// All waits are bounded; a timeout sets the abort flag, drains what was issued and leaves.
 #pragma once
 
 #include <cuda.h>
@@ -27,25 +35,30 @@ namespace tp {
 namespace fa {
 
 constexpr int kRows = 128;   // query rows per tile
-constexpr int kKeys = 64;    // keys per K/V block
+constexpr int kKeys = 128;   // keys per K/V block
 constexpr int kThreads = 128;
 
 template <int HD>
 struct Smem {
   static constexpr int SUB = HD / 64;                 // 64-wide swizzle sub-tiles along the head dim
-  static constexpr int QTILE = kRows * 128;           // Q sub-tile: 128 rows x 128 bytes
-  static constexpr int KTILE = kKeys * 128;           // K or V sub-tile: 64 rows x 128 bytes
-  static constexpr int PTILE = kRows * 128;           // P: 128 rows x 64 keys (bf16)
-  static constexpr bool P_IN_K = SUB * KTILE >= PTILE;   // P reuses the block's K buffer
+  static constexpr int TILE = 128 * 128;              // one sub-tile: 128 rows x 128 bytes
+  static constexpr int BLOCK = SUB * TILE;            // Q tile, or one K or V block
   static constexpr int Q_OFF = 0;
-  static constexpr int K_OFF = Q_OFF + SUB * QTILE;   // 2 buffers
-  static constexpr int V_OFF = K_OFF + 2 * SUB * KTILE;
-  static constexpr int P_OFF = V_OFF + 2 * SUB * KTILE;   // used only when !P_IN_K
-  static constexpr int BAR_OFF = P_OFF + (P_IN_K ? 0 : PTILE);
+  static constexpr int K_OFF = Q_OFF + BLOCK;
+  static constexpr int V_OFF = K_OFF + BLOCK;
+  static constexpr int BAR_OFF = V_OFF + BLOCK;
   static constexpr int BYTES = BAR_OFF + 128 + 1024;  // barriers + alignment slack
-  static constexpr int KV_BYTES = 2 * SUB * KTILE;    // one K block + one V block
-  static constexpr uint32_t TMEM_COLS = 256;          // S (64 cols) + O (from col 128)
+  static constexpr uint32_t TMEM_COLS = 256;          // S/P at column 0, O at column 128
 };
+
+constexpr float kRescaleLog2 = 8.f;   // growth of a row maximum (log2 units) that forces a rescale
+// 2^f ~= kP0 + f (kP1 + f (kP2 + f kP3)) on [-1/2, 1/2]
+constexpr float kP0 = 0.9999281168f, kP1 = 0.6932609677f, kP2 = 0.2426105440f, kP3 = 0.0551713221f;
+constexpr float kRoundMagic = 12582912.f;   // 1.5 * 2^23: x + magic has round(x) in its low bits
+// pairs of P values (index mod 8) computed on the FMA pipe; the rest use the special-function unit.
+// Three of eight balances the two when two warps share a sub-partition: a pair costs 16 cycles
+// of the 4-lane-per-clock unit, or about twice the issue slots on the FMA pipe.
+constexpr uint32_t kPolyPairs = (1u << 1) | (1u << 4) | (1u << 6);
 
 struct Params {
   int32_t s;          // tokens per sequence
@@ -74,8 +87,71 @@ __device__ __forceinline__ void tmem_st_32x32b_x32(uint32_t taddr, const uint32_
       "r"(r[29]), "r"(r[30]), "r"(r[31])
       : "memory");
 }
+// 2^x with the special-function unit (PTX ex2.approx.ftz.f32: results below 2^-126 flush to 0,
+// 2^-inf = 0); a softmax term that small does not change the sum.
+__device__ __forceinline__ float ex2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
+  return y;
+}
+// Packed pairs of fp32 (PTX .f32x2 arithmetic, sm_100): one instruction for two lanes of work.
+__device__ __forceinline__ uint64_t f2_pack(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t r, float& a, float& b) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(r));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float fmax3(float a, float b, float c) {
+  float d;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(d) : "f"(a), "f"(b), "f"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+// (2^x0, 2^x1) on the FMA pipe; inputs below -125 (masked keys at -inf included) give about
+// 2^-125, which no softmax sum notices.
+__device__ __forceinline__ void exp2_poly_x2(float x0, float x1, float& y0, float& y1) {
+  const uint64_t x = f2_pack(fmaxf(x0, -125.f), fmaxf(x1, -125.f));
+  const uint64_t magic = f2_pack(kRoundMagic, kRoundMagic);
+  const uint64_t j = fadd2(x, magic);
+  const uint64_t f = fsub2(x, fsub2(j, magic));
+  uint64_t q = ffma2(f2_pack(kP3, kP3), f, f2_pack(kP2, kP2));
+  q = ffma2(q, f, f2_pack(kP1, kP1));
+  q = ffma2(q, f, f2_pack(kP0, kP0));
+  float j0, j1, q0, q1;
+  f2_unpack(j, j0, j1);
+  f2_unpack(q, q0, q1);
+  y0 = __uint_as_float(__float_as_uint(q0) + __float_as_uint(j0) * (1u << 23));
+  y1 = __uint_as_float(__float_as_uint(q1) + __float_as_uint(j1) * (1u << 23));
+}
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+// D[tmem] (+)= A[tmem] * B[smem]^T, kind::f16: A (M x 16, K-major) sits in TMEM, row i in lane i,
+// two bf16 per 32-bit column (lower k in the low half).  Issued by a single thread.
+__device__ __forceinline__ void umma_f16_tmem_a(uint32_t d_tmem, uint32_t a_tmem, uint64_t b_desc,
+                                                uint32_t idesc, uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f16 [%0], [%1], %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "r"(a_tmem), "l"(b_desc), "r"(idesc), "r"(accumulate)
+      : "memory");
 }
 
 template <int HD>
@@ -88,11 +164,13 @@ __global__ void __launch_bounds__(kThreads, 2)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint64_t* bar = reinterpret_cast<uint64_t*>(smem + L::BAR_OFF);
   uint64_t* q_full = bar + 0;
-  uint64_t* kv_full = bar + 1;   // [2]
-  uint64_t* s_done = bar + 3;
-  uint64_t* o_done = bar + 4;
-  uint64_t* drain = bar + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* k_full = bar + 1;    // K block landed (one phase per block)
+  uint64_t* v_full = bar + 2;    // V block landed
+  uint64_t* s_full = bar + 3;    // S = Q K^T done
+  uint64_t* p_full = bar + 4;    // P stored in TMEM and O rescaled (128 arrivals)
+  uint64_t* pv_done = bar + 5;   // O += P V done: S/P columns and the V buffer are free again
+  uint64_t* drain = bar + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -107,14 +185,15 @@ __global__ void __launch_bounds__(kThreads, 2)
   const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
   const int q0 = qt * kRows;
   const int n_kb_all = (P.s + kKeys - 1) / kKeys;
-  const int nkb = P.causal ? min((q0 + kRows) / kKeys, n_kb_all) : n_kb_all;
+  const int nkb = P.causal ? min(qt + 1, n_kb_all) : n_kb_all;
 
   if (tid == 0) {
     mbar_init(q_full, 1);
-    mbar_init(&kv_full[0], 1);
-    mbar_init(&kv_full[1], 1);
-    mbar_init(s_done, 1);
-    mbar_init(o_done, 1);
+    mbar_init(k_full, 1);
+    mbar_init(v_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_full, kThreads);
+    mbar_init(pv_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -134,164 +213,168 @@ __global__ void __launch_bounds__(kThreads, 2)
   uint8_t* sQ = smem + L::Q_OFF;
   uint8_t* sK = smem + L::K_OFF;
   uint8_t* sV = smem + L::V_OFF;
-
-  auto load_kv = [&](int kb) {
-    const int buf = kb & 1;
-    mbar_arrive_expect_tx(&kv_full[buf], L::KV_BYTES);
-#pragma unroll
-    for (int c = 0; c < L::SUB; ++c) {
-      tma_load_3d(&tma_qkv, &kv_full[buf], sK + (buf * L::SUB + c) * L::KTILE, k_col + 64 * c,
-                  kb * kKeys, bi);
-      tma_load_3d(&tma_qkv, &kv_full[buf], sV + (buf * L::SUB + c) * L::KTILE, v_col + 64 * c,
-                  kb * kKeys, bi);
-    }
+  auto wait = [&](uint64_t* b, uint32_t par, uint32_t site) {
+    return mbar_wait(b, par, abort_flag, P.err, site);
   };
 
-  uint32_t issued_kv = 0;       // blocks whose loads were issued (thread 0 only)
-  if (tid == 0) {
-    mbar_arrive_expect_tx(q_full, L::SUB * L::QTILE);
+  // ---- thread 0: loads and MMAs
+  uint32_t n_k = 0, n_v = 0;    // K / V loads issued (thread 0)
+  bool issued_mma = false;
+  auto load_block = [&](uint64_t* full, uint8_t* dst, int col, int row) {
+    mbar_arrive_expect_tx(full, L::BLOCK);
 #pragma unroll
-    for (int c = 0; c < L::SUB; ++c) {   // a Q sub-tile is two 64-row boxes
-      tma_load_3d(&tma_qkv, q_full, sQ + c * L::QTILE, q_col + 64 * c, q0, bi);
-      tma_load_3d(&tma_qkv, q_full, sQ + c * L::QTILE + L::KTILE, q_col + 64 * c, q0 + 64, bi);
+    for (int c = 0; c < L::SUB; ++c) tma_load_3d(&tma_qkv, full, dst + c * L::TILE, col + 64 * c, row, bi);
+  };
+  auto issue_s = [&]() {
+    constexpr uint32_t IDESC_S = make_idesc_bf16(128, kKeys, false, false);
+    tc_fence_after();
+    const uint32_t qa = smem_addr(sQ), ka = smem_addr(sK);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
+      umma_f16(tS, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+               IDESC_S, kk > 0 ? 1u : 0u);
     }
-    load_kv(0);
-    issued_kv = 1;
-    if (nkb > 1) {
-      load_kv(1);
-      issued_kv = 2;
+    umma_commit(s_full);
+    issued_mma = true;
+  };
+  auto issue_pv = [&](int kb) {
+    constexpr uint32_t IDESC_O = make_idesc_bf16(128, HD, false, true);
+    tc_fence_after();
+    const uint32_t va = smem_addr(sV);
+#pragma unroll
+    for (int kk = 0; kk < kKeys / 16; ++kk) {
+      // P: 16 keys = 8 TMEM columns; V: 64-dim blocks of 128 key rows (LBO = one sub-tile)
+      umma_f16_tmem_a(tO, tS + kk * 8, make_sdesc_sw128(va + kk * 16 * 128, L::TILE, 1024),
+                      IDESC_O, (kb > 0 || kk > 0) ? 1u : 0u);
     }
+    umma_commit(pv_done);
+  };
+
+  bool ok = true;
+  if (tid == 0) {
+    load_block(q_full, sQ, q_col, q0);
+    load_block(k_full, sK, k_col, 0);
+    ++n_k;
+    load_block(v_full, sV, v_col, 0);
+    ++n_v;
+    if (wait(q_full, 0, DEVERR_WAIT_FULL) && wait(k_full, 0, DEVERR_WAIT_FULL)) issue_s();
   }
 
-  // instruction descriptors: S = Q K^T (both K-major); O += P V (P K-major, V MN-major)
-  constexpr uint32_t IDESC_S = make_idesc_bf16(128, kKeys, false, false);
-  constexpr uint32_t IDESC_O = make_idesc_bf16(128, HD, false, true);
-
-  const int row = tid;                 // query row within the tile
-  const int q_abs = q0 + row;
+  // ---- softmax: every thread one row; wait results are made warp-uniform (the TMEM loads and
+  // stores are warp-collective)
+  const int q_abs = q0 + tid;
   float m_run = -INFINITY, l_run = 0.f;
-  bool issued_mma = false;
-  // every wait result is made warp-uniform (the TMEM loads are warp-collective) and, once per
-  // key block, CTA-uniform, so on a timeout all threads leave the loop together
-  bool ok = __syncthreads_and(mbar_wait(q_full, 0, abort_flag, P.err, DEVERR_WAIT_FULL) ? 1 : 0);
-
-  for (int kb = 0; kb < nkb && ok; ++kb) {
-    const int buf = kb & 1;
-    bool w = __all_sync(0xffffffffu,
-                        mbar_wait(&kv_full[buf], (kb >> 1) & 1, abort_flag, P.err, DEVERR_WAIT_FULL));
-    if (w && tid == 0) {
-      tc_fence_after();
-      const uint32_t qa = smem_addr(sQ), ka = smem_addr(sK + buf * L::SUB * L::KTILE);
-#pragma unroll
-      for (int kk = 0; kk < HD / 16; ++kk) {
-        const uint32_t koff = (kk & 3) * 32;
-        umma_f16(tS, make_sdesc_sw128(qa + (kk >> 2) * L::QTILE + koff, 16, 1024),
-                 make_sdesc_sw128(ka + (kk >> 2) * L::KTILE + koff, 16, 1024), IDESC_S,
-                 kk > 0 ? 1u : 0u);
-      }
-      umma_commit(s_done);
-      issued_mma = true;
+  for (int kb = 0; kb < nkb; ++kb) {
+    const uint32_t par = kb & 1;
+    ok = __all_sync(0xffffffffu, wait(s_full, par, DEVERR_WAIT_ACC_FULL));
+    // O holds P(kb-1) V(kb-1) (S(kb) was issued after it completed; waited here for ordering)
+    if (ok && kb > 0)
+      ok = __all_sync(0xffffffffu, wait(pv_done, par ^ 1, DEVERR_WAIT_ACC_EMPTY));
+    if (!ok) break;
+    tc_fence_after();
+    if (tid == 0 && kb + 1 < nkb) {   // K buffer is free once S(kb) is done
+      load_block(k_full, sK, k_col, (kb + 1) * kKeys);
+      ++n_k;
     }
-    if (w) w = __all_sync(0xffffffffu, mbar_wait(s_done, kb & 1, abort_flag, P.err,
-                                                   DEVERR_WAIT_ACC_FULL));
     float sv[kKeys];
-    if (w) {
-      tc_fence_after();
-      // ---- online softmax on this thread's row of S
+    {
+      uint32_t r[4][32];
 #pragma unroll
-      for (int c = 0; c < kKeys / 32; ++c) {
+      for (int c = 0; c < 4; ++c) tmem_ld_32x32b_x32(tS + lane_base + c * 32, r[c]);
+      tmem_wait_ld();
+#pragma unroll
+      for (int c = 0; c < 4; ++c)
+#pragma unroll
+        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[c][e]);
+    }
+    const int k_base = kb * kKeys;
+    if ((k_base + kKeys > P.s) || (P.causal && k_base + kKeys - 1 > q0)) {
+      // keys of this row inside the block: beyond the sequence or the causal limit -> -inf
+      const int lim = (P.causal ? min(P.s, q_abs + 1) : P.s) - k_base;
+#pragma unroll
+      for (int c = 0; c < kKeys; ++c) sv[c] = c < lim ? sv[c] : -INFINITY;
+    }
+    float mx;
+    {   // row maximum: 8 partial maxima, two new keys per three-input max
+      float m8[8];
+#pragma unroll
+      for (int i = 0; i < 8; ++i) m8[i] = sv[i];
+#pragma unroll
+      for (int c = 8; c < kKeys; c += 16)
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m8[i] = fmax3(m8[i], sv[c + i], sv[c + 8 + i]);
+      mx = fmax3(fmax3(m8[0], m8[1], m8[2]), fmax3(m8[3], m8[4], m8[5]), fmaxf(m8[6], m8[7]));
+    }
+    // The reference maximum m moves only on the first block or when the block's maximum
+    // exceeds it by more than 2^8 in the exp2 domain, so O and l are rarely rescaled; P then
+    // stays below 2^8 and O / l is the same whichever m was used.
+    float alpha = 1.f;
+    if (m_run == -INFINITY || (mx - m_run) * P.scale_log2 > kRescaleLog2) {
+      alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - mx) * P.scale_log2);
+      m_run = mx;
+    }
+    const float mscaled = (m_run == -INFINITY) ? 0.f : m_run * P.scale_log2;
+    uint32_t pk[kKeys / 2];
+    float rs;
+    {   // P = 2^(s*scale - m) two keys at a time; row sum in 4 packed partial sums
+      const uint64_t scale2 = f2_pack(P.scale_log2, P.scale_log2);
+      const uint64_t negm2 = f2_pack(-mscaled, -mscaled);
+      uint64_t acc[4] = {0, 0, 0, 0};
+#pragma unroll
+      for (int c = 0; c < kKeys / 2; ++c) {
+        float x0, x1, p0, p1;
+        f2_unpack(ffma2(f2_pack(sv[2 * c], sv[2 * c + 1]), scale2, negm2), x0, x1);
+        if (kPolyPairs & (1u << (c & 7))) {
+          exp2_poly_x2(x0, x1, p0, p1);
+        } else {
+          p0 = ex2_approx(x0);   // 2^-inf = 0 for masked keys
+          p1 = ex2_approx(x1);
+        }
+        acc[c & 3] = fadd2(acc[c & 3], f2_pack(p0, p1));
+        pk[c] = pack_bf16x2(p0, p1);
+      }
+      const uint64_t a2 = fadd2(fadd2(acc[0], acc[1]), fadd2(acc[2], acc[3]));
+      float a, bb;
+      f2_unpack(a2, a, bb);
+      rs = a + bb;
+    }
+    l_run = l_run * alpha + rs;
+    // P(kb) as bf16 over the first half of the S columns
+    tmem_st_32x32b_x32(tS + lane_base, *reinterpret_cast<uint32_t(*)[32]>(&pk[0]));
+    tmem_st_32x32b_x32(tS + lane_base + 32, *reinterpret_cast<uint32_t(*)[32]>(&pk[32]));
+    if (kb > 0 && __any_sync(0xffffffffu, alpha != 1.f)) {
+#pragma unroll
+      for (int c = 0; c < HD / 32; ++c) {
         uint32_t r[32];
-        tmem_ld_32x32b_x32(tS + lane_base + c * 32, r);
+        tmem_ld_32x32b_x32(tO + lane_base + c * 32, r);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 32; ++e) sv[c * 32 + e] = __uint_as_float(r[e]);
-      }
-      const int k_base = kb * kKeys;
-      const bool need_mask = (k_base + kKeys > P.s) || (P.causal && k_base + kKeys - 1 > q0);
-      float mx = -INFINITY;
-#pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        if (need_mask) {
-          const int k_abs = k_base + c;
-          if (k_abs >= P.s || (P.causal && k_abs > q_abs)) sv[c] = -INFINITY;
-        }
-        mx = fmaxf(mx, sv[c]);
-      }
-      const float m_new = fmaxf(m_run, mx);
-      const float alpha = (m_run == -INFINITY) ? 0.f : exp2f((m_run - m_new) * P.scale_log2);
-      const float mscaled = (m_new == -INFINITY) ? 0.f : m_new * P.scale_log2;
-      float rs = 0.f;
-#pragma unroll
-      for (int c = 0; c < kKeys; ++c) {
-        const float pv = exp2f(sv[c] * P.scale_log2 - mscaled);   // exp2(-inf) = 0 when masked
-        sv[c] = pv;
-        rs += pv;
-      }
-      l_run = l_run * alpha + rs;
-      m_run = m_new;
-
-      // ---- the previous P V must be finished before P and O are touched again
-      if (kb > 0) {
-        w = __all_sync(0xffffffffu, mbar_wait(o_done, (kb - 1) & 1, abort_flag, P.err,
-                                              DEVERR_WAIT_ACC_EMPTY));
-        if (w) {
-          tc_fence_after();
-          if (tid == 0 && kb + 1 < nkb) {
-            load_kv(kb + 1);   // buffer (kb+1)&1 held block kb-1, whose MMAs are complete
-            issued_kv = kb + 2;
-          }
-          // rescale O only in warps where some row's maximum moved
-          if (__any_sync(0xffffffffu, alpha != 1.f)) {
-#pragma unroll
-            for (int c = 0; c < HD / 32; ++c) {
-              uint32_t r[32];
-              tmem_ld_32x32b_x32(tO + lane_base + c * 32, r);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
-              tmem_st_32x32b_x32(tO + lane_base + c * 32, r);
-            }
-            tmem_wait_st();
-          }
-        }
+        for (int e = 0; e < 32; ++e) r[e] = __float_as_uint(__uint_as_float(r[e]) * alpha);
+        tmem_st_32x32b_x32(tO + lane_base + c * 32, r);
       }
     }
-    // P of this block: over its K tile (dead after S) or in its own buffer
-    uint8_t* sP = L::P_IN_K ? sK + buf * L::SUB * L::KTILE : smem + L::P_OFF;
-    if (w) {
-      // ---- P (bf16) into smem, K-major with the 128-byte swizzle: row `row`, 64 keys
-#pragma unroll
-      for (int ch = 0; ch < kKeys / 8; ++ch) {
-        uint4 v4;
-        v4.x = pack_bf16x2(sv[ch * 8 + 0], sv[ch * 8 + 1]);
-        v4.y = pack_bf16x2(sv[ch * 8 + 2], sv[ch * 8 + 3]);
-        v4.z = pack_bf16x2(sv[ch * 8 + 4], sv[ch * 8 + 5]);
-        v4.w = pack_bf16x2(sv[ch * 8 + 6], sv[ch * 8 + 7]);
-        *reinterpret_cast<uint4*>(sP + row * 128 + ((ch ^ (row & 7)) << 4)) = v4;
-      }
-      fence_proxy_async_smem();
-    }
+    tmem_wait_st();
     tc_fence_before();
-    if (!__syncthreads_and(w ? 1 : 0)) {
-      ok = false;
-      break;
-    }
+    mbar_arrive(p_full);
     if (tid == 0) {
-      tc_fence_after();
-      const uint32_t pa = smem_addr(sP), va = smem_addr(sV + buf * L::SUB * L::KTILE);
-#pragma unroll
-      for (int kk = 0; kk < kKeys / 16; ++kk) {
-        const uint64_t adesc = make_sdesc_sw128(pa + kk * 32, 16, 1024);
-        // V tile: 64-dim blocks of 64 key rows (LBO = one sub-tile), 16 keys per MMA
-        const uint64_t bdesc = make_sdesc_sw128(va + kk * 16 * 128, L::KTILE, 1024);
-        umma_f16(tO, adesc, bdesc, IDESC_O, (kb > 0 || kk > 0) ? 1u : 0u);
+      // every row has stored P(kb) and rescaled O: O += P(kb) V(kb); then, once that is done
+      // (it reads P from the S columns), V(kb+1) and S(kb+1)
+      bool t = wait(p_full, par, DEVERR_WAIT_ACC_FULL) && wait(v_full, par, DEVERR_WAIT_FULL);
+      if (t) issue_pv(kb);
+      if (t && kb + 1 < nkb) {
+        t = wait(pv_done, par, DEVERR_WAIT_ACC_EMPTY) &&
+            wait(k_full, (kb + 1) & 1, DEVERR_WAIT_FULL);
+        if (t) {
+          issue_s();
+          load_block(v_full, sV, v_col, (kb + 1) * kKeys);   // V is free once P(kb) V(kb) is done
+          ++n_v;
+        }
       }
-      umma_commit(o_done);
     }
   }
-
-  if (ok) ok = __all_sync(0xffffffffu, mbar_wait(o_done, (nkb - 1) & 1, abort_flag, P.err,
-                                                 DEVERR_WAIT_ACC_EMPTY));
+  tmem_wait_st();
+  if (ok) ok = __all_sync(0xffffffffu, wait(pv_done, (nkb - 1) & 1, DEVERR_WAIT_ACC_EMPTY));
   if (ok) {
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
@@ -315,20 +398,22 @@ __global__ void __launch_bounds__(kThreads, 2)
         }
       }
     }
-  } else if (tid == 0) {
-    // abort path: let issued copies and MMAs land before the CTA leaves (bounded waits)
+  }
+  __syncthreads();
+  if (*abort_flag && tid == 0) {
+    // let issued copies and MMAs land before the CTA leaves (bounded waits); each buffer has at
+    // most its latest load in flight
     const uint64_t t0 = globaltimer_ns();
-    auto bounded = [&](uint64_t* b, uint32_t par) {
-      while (!mbar_try_wait(b, par))
+    auto bounded = [&](uint64_t* bb, uint32_t pp) {
+      while (!mbar_try_wait(bb, pp))
         if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
           record_device_error(P.err, DEVERR_WAIT_DRAIN);
           return;
         }
     };
     bounded(q_full, 0);
-    // only the most recent load into each buffer can still be in flight
-    for (uint32_t kb = issued_kv >= 2 ? issued_kv - 2 : 0; kb < issued_kv; ++kb)
-      bounded(&kv_full[kb & 1], (kb >> 1) & 1);
+    if (n_k) bounded(k_full, (n_k - 1) & 1);
+    if (n_v) bounded(v_full, (n_v - 1) & 1);
     if (issued_mma) {
       umma_commit(drain);
       bounded(drain, 0);
@@ -349,7 +434,7 @@ inline tp_status launch(const void* qkv, int64_t b, int64_t s, int n_q, int qh, 
   const uint64_t cols = static_cast<uint64_t>(p) * R_a;
   tp_status r = encode_tmap_bf16_3d(&map, qkv, cols, static_cast<uint64_t>(s),
                                     static_cast<uint64_t>(b), cols * 2,
-                                    cols * 2 * static_cast<uint64_t>(s), 64, kKeys);
+                                    cols * 2 * static_cast<uint64_t>(s), 64, 128);
   if (r != TP_OK) return r;
   static int attr_set[64] = {0};
   int dev = 0;
