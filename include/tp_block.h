@@ -248,6 +248,15 @@ tp_status tp_check_device_error(void* stream);
 /* 1 if this build contains the sm_100a tensor-core kernels and the current device runs them. */
 int32_t tp_tensor_core_path_available(void);
 
+/* Failure-detection self-test (the pages have no counterpart; it exercises the timeout path
+ * behind TP_ERR_TIMEOUT without any fault).  Enqueues one small kernel that waits, through the
+ * same bounded mbarrier wait the tensor-core kernels use, on a barrier that nothing completes;
+ * after limit_us microseconds (1 .. 1000000) the wait gives up, records the timeout in the device
+ * error word and the kernel returns.  A following tp_check_device_error() reports TP_ERR_TIMEOUT
+ * and clears the word; the CUDA context stays usable.  Returns TP_ERR_INVALID_ARG for a limit
+ * out of range (checked before anything is enqueued). */
+tp_status tp_selftest_wait_timeout(uint32_t limit_us, void* stream);
+
 /* Per-kernel timing.  While enabled, every kernel the library launches is bracketed by two CUDA
  * events recorded on the launching stream (skipped while the stream is being captured into a
  * graph).  tp_profile_read synchronizes the device and returns, for entry i (0-based, in order

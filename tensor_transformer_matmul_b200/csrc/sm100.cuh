@@ -45,10 +45,11 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
 }
 
 // Wait for the phase with the given parity to complete.  Gives up when *abort becomes non-zero
-// (another role gave up) or after kWaitTimeoutNs, in which case it raises *abort, records
-// ``site`` in the device error word and returns false.
+// (another role gave up) or after ``limit_ns`` (kWaitTimeoutNs unless given), in which case it
+// raises *abort, records ``site`` in the device error word and returns false.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
-                                          uint32_t* err, uint32_t site) {
+                                          uint32_t* err, uint32_t site,
+                                          uint64_t limit_ns = kWaitTimeoutNs) {
   if (mbar_try_wait(bar, parity)) return true;
   const uint64_t t0 = globaltimer_ns();
   uint32_t n = 0;
@@ -56,7 +57,7 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
     if (mbar_try_wait(bar, parity)) return true;
     if ((++n & 31u) == 0) {
       if (*abort) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+      if (globaltimer_ns() - t0 > limit_ns) {
         *abort = 1;
         record_device_error(err, site);
         return false;

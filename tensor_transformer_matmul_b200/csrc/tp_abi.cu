@@ -9,6 +9,7 @@
 #include <mutex>
 #include <string>
 
+#include "sm100.cuh"
 #include "tp_common.cuh"
 
 namespace tp {
@@ -133,6 +134,25 @@ ProfScope::~ProfScope() {
 
 }  // namespace tp
 
+namespace tp {
+// One warp waits, through the same bounded mbarrier wait the tensor-core kernels use, on a
+// barrier that nothing ever completes; after limit_ns the wait gives up, raises the abort flag
+// and records DEVERR_WAIT_FULL in the device error word, and the kernel returns.
+__global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    sm100::mbar_init(&bar, 1);
+    abort_flag = 0;
+    sm100::fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0)
+    sm100::mbar_wait(&bar, 0, &abort_flag, err, DEVERR_WAIT_FULL, limit_ns);
+  __syncthreads();
+}
+}  // namespace tp
+
 extern "C" {
 
 void tp_profile_enable(int32_t on) { tp::g_prof_on.store(on ? 1 : 0); }
@@ -208,6 +228,18 @@ tp_status tp_check_device_error(void* stream) {
 }
 
 int32_t tp_tensor_core_path_available(void) { return tp::tensor_cores_usable() ? 1 : 0; }
+
+tp_status tp_selftest_wait_timeout(uint32_t limit_us, void* stream) {
+  tp::clear_error();
+  if (limit_us == 0 || limit_us > 1000000u)
+    return tp::set_error(TP_ERR_INVALID_ARG, "limit_us must be in 1 .. 1000000");
+  uint32_t* w = tp::device_error_word();
+  if (!w) return tp::set_error(TP_ERR_CUDA, "device error word unavailable");
+  tp::wait_selftest_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(
+      static_cast<uint64_t>(limit_us) * 1000ull, w);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
 
 int32_t tp_version(void) { return 100; }  // 0.1.0
 

@@ -33,6 +33,7 @@ EXPORTS = (
     "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
     "tp_profile_enable", "tp_profile_read", "tp_profile_reset", "tp_mlp_fwd_static_ws",
+    "tp_selftest_wait_timeout",
 )
 
 
@@ -90,6 +91,7 @@ def load():
         "tp_launch_count": (ctypes.c_uint64, []), "tp_last_error": (ctypes.c_char_p, []),
         "tp_status_string": (ctypes.c_char_p, [I32]), "tp_check_device_error": (I32, [P]),
         "tp_tensor_core_path_available": (I32, []), "tp_version": (I32, []),
+        "tp_selftest_wait_timeout": (I32, [ctypes.c_uint32, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
@@ -261,6 +263,10 @@ def tp_last_error():
 
 def tp_check_device_error(stream=None):
     _check(load().tp_check_device_error(_stream(stream)))
+
+
+def tp_selftest_wait_timeout(limit_us, stream=None):
+    _check(load().tp_selftest_wait_timeout(limit_us, _stream(stream)))
 
 
 def tp_tensor_core_path_available():

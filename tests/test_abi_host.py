@@ -128,6 +128,9 @@ def test_reduce_argument_errors(lib):
     bad = lib.mlp_desc(4, 8, 32, 4, "gelu", "f32", flags=4)
     assert so.tp_mlp_fwd(ctypes.byref(bad), fake, fake, fake, None, fake, None, None, fake, 1 << 30,
                          None) == lib.TP_ERR_INVALID_ARG
+    # the failure-detection self-test checks its limit before enqueueing anything
+    assert so.tp_selftest_wait_timeout(0, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_selftest_wait_timeout(1000001, None) == lib.TP_ERR_INVALID_ARG
 
 
 def test_empty_batch_counts_one_reduction(lib):
