@@ -221,12 +221,24 @@ inline void reduce_norm_launch(const void* part, int p, int64_t rows, int64_t d,
         static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
 }
 
+inline tp_status rmsnorm(const void* x, int in_dtype, int64_t rows, int64_t d, float eps,
+                         void* out, int out_dtype, cudaStream_t s);
+inline bool rmsnorm_split_ok(const void* x, int64_t rows, int64_t d, const void* out);
+
 // y = res + sum of fp32 partials [p][rows][d]; norm = RMSNorm(y) in norm_dtype
 inline tp_status reduce_norm(const float* part, int p, int64_t rows, int64_t d, const void* res,
                              void* out, int out_dtype, void* norm, int norm_dtype, float eps,
                              cudaStream_t s) {
   if (rows == 0) return TP_OK;
   if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
+  if (rmsnorm_split_ok(out, rows, d, norm)) {
+    // few rows: one row per block would leave most SMs idle, so the sum runs as the plain
+    // vectorised reduce over all rows*d elements and the norm as the row-split kernel (both read
+    // the stored, rounded y, as the one-kernel path does)
+    tp_status st = launch(part, TP_F32, p, rows * d, res, out, out_dtype, s);
+    if (st != TP_OK) return st;
+    return rmsnorm(out, out_dtype, rows, d, eps, norm, norm_dtype, s);
+  }
   ProfScope prof(s, "reduce_partials");
   const bool ob = out_dtype == TP_BF16, nb = norm_dtype == TP_BF16;
   if (ob && nb) reduce_norm_launch<float, __nv_bfloat16, __nv_bfloat16>(part, p, rows, d, res, out, norm, eps, s);
@@ -271,13 +283,71 @@ inline void rmsnorm_launch(const void* x, int64_t rows, int64_t d, float eps, vo
       static_cast<const Tin*>(x), d, eps, static_cast<Tout*>(out));
 }
 
+// RMSNorm for few rows (fewer than SMs): block (c, r) recomputes the sum of squares of the whole
+// row r, vectorised and in a fixed order (so every block of a row gets the same scale), and
+// normalises columns [c*W, (c+1)*W) of it.  Needs d % 8 == 0 and 16-byte aligned rows.
+constexpr int kSplitW = 512;
+template <typename Tin, typename Tout>
+__global__ void __launch_bounds__(256) rmsnorm_split_kernel(const Tin* __restrict__ x, int64_t d,
+                                                            float eps, Tout* __restrict__ out) {
+  __shared__ float red[8];
+  const Tin* xr = x + static_cast<int64_t>(blockIdx.y) * d;
+  Tout* orow = out + static_cast<int64_t>(blockIdx.y) * d;
+  float ss = 0.f;
+  for (int64_t j = 8 * static_cast<int64_t>(threadIdx.x); j < d; j += 8 * blockDim.x) {
+    float v[8];
+    Vec8<Tin>::load(xr + j, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) ss = fmaf(v[e], v[e], ss);
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x < 32) {
+    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    if (threadIdx.x == 0) red[0] = v;
+  }
+  __syncthreads();
+  const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
+  const int64_t c0 = static_cast<int64_t>(blockIdx.x) * kSplitW;
+  const int64_t c1 = c0 + kSplitW < d ? c0 + kSplitW : d;
+  for (int64_t j = c0 + 8 * static_cast<int64_t>(threadIdx.x); j < c1; j += 8 * blockDim.x) {
+    float v[8];
+    Vec8<Tin>::load(xr + j, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] *= scale;
+    Vec8<Tout>::store(orow + j, v);
+  }
+}
+
+template <typename Tin, typename Tout>
+inline void rmsnorm_split_launch(const void* x, int64_t rows, int64_t d, float eps, void* out,
+                                 cudaStream_t s) {
+  const dim3 grid(static_cast<unsigned>(ceil_div(d, kSplitW)), static_cast<unsigned>(rows));
+  rmsnorm_split_kernel<Tin, Tout><<<grid, 256, 0, s>>>(static_cast<const Tin*>(x), d, eps,
+                                                       static_cast<Tout*>(out));
+}
+
+inline bool rmsnorm_split_ok(const void* x, int64_t rows, int64_t d, const void* out) {
+  return rows > 0 && rows < num_sms() && d % 8 == 0 && rows <= 65535 &&
+         ((reinterpret_cast<uintptr_t>(x) | reinterpret_cast<uintptr_t>(out)) & 15) == 0;
+}
+
 inline tp_status rmsnorm(const void* x, int in_dtype, int64_t rows, int64_t d, float eps,
                          void* out, int out_dtype, cudaStream_t s) {
   if (rows == 0) return TP_OK;
   if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
   ProfScope prof(s, "rmsnorm");
   const bool ib = in_dtype == TP_BF16, ob = out_dtype == TP_BF16;
-  if (ib && ob) rmsnorm_launch<__nv_bfloat16, __nv_bfloat16>(x, rows, d, eps, out, s);
+  if (rmsnorm_split_ok(x, rows, d, out)) {   // few rows: spread each row over many blocks
+    if (ib && ob) rmsnorm_split_launch<__nv_bfloat16, __nv_bfloat16>(x, rows, d, eps, out, s);
+    else if (ib) rmsnorm_split_launch<__nv_bfloat16, float>(x, rows, d, eps, out, s);
+    else if (ob) rmsnorm_split_launch<float, __nv_bfloat16>(x, rows, d, eps, out, s);
+    else rmsnorm_split_launch<float, float>(x, rows, d, eps, out, s);
+  } else if (ib && ob) rmsnorm_launch<__nv_bfloat16, __nv_bfloat16>(x, rows, d, eps, out, s);
   else if (ib) rmsnorm_launch<__nv_bfloat16, float>(x, rows, d, eps, out, s);
   else if (ob) rmsnorm_launch<float, __nv_bfloat16>(x, rows, d, eps, out, s);
   else rmsnorm_launch<float, float>(x, rows, d, eps, out, s);

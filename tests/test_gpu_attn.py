@@ -151,11 +151,18 @@ def test_f32_residual_stream(lib):
     assert rel_l2(f64(y), _ref(inp, 8, 2, 32, True) + f64(res)) <= TOL["bf16"]
 
 
-def test_rmsnorm_dtypes(lib):
+@pytest.mark.parametrize("rows,d", [
+    (5, 300),      # d not a multiple of 8: one block per row
+    (1, 8192),     # few rows: each row spread over 16 blocks of 512 columns
+    (3, 1000),     # few rows, ragged last 512-column block
+    (200, 64),     # more rows than SMs: one block per row
+])
+@pytest.mark.parametrize("in_dtype", [torch.float32, torch.bfloat16])
+def test_rmsnorm_dtypes(lib, rows, d, in_dtype):
     from oracle import decode as odec
-    x = torch.randn(5, 300, device=dev())
+    x = torch.randn(rows, d, device=dev()).to(in_dtype)
     for out_dtype, tol in ((torch.bfloat16, TOL["bf16"]), (torch.float32, TOL["f32"])):
-        out = torch.empty(5, 300, dtype=out_dtype, device=dev())
+        out = torch.empty(rows, d, dtype=out_dtype, device=dev())
         lib.tp_rmsnorm(x, out)
         torch.cuda.synchronize()
         assert rel_l2(f64(out), odec.rmsnorm(f64(x))) <= tol
