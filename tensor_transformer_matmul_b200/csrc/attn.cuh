@@ -287,6 +287,8 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
   const T* knew = qkv + ix.k(bi, g);
   const T* vnew = qkv + ix.v(bi, g);
   const float sl2 = scale * 1.4426950408889634f;
+  pdl_wait();   // global memory only from here on (programmatic dependent launch)
+  pdl_trigger();
 
   // ---- stage the split's K and V rows
   if (threadIdx.x == 0) {
@@ -500,7 +502,11 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   dim3 grid(static_cast<unsigned>(L.kv_splits), static_cast<unsigned>(L.n_kv),
             static_cast<unsigned>(L.b));
   if (L.b > 65535) return set_error(TP_ERR_UNSUPPORTED, "decode batch above 65535");
-  TP_CUDA_TRY(cudaMemsetAsync(counters, 0, static_cast<size_t>(L.b * L.n_kv) * sizeof(int), s));
+  {
+    const int64_t words = L.b * L.n_kv;
+    TP_LAUNCH_PDL(zero_words_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words, 256), 64))),
+                  dim3(256), 0, s, reinterpret_cast<uint32_t*>(counters), words);
+  }
 #define TP_DECODE_CASE(G, H)                                                                  \
   if (group == G && L.hd == H) {                                                              \
     const size_t smem = attn::DecodeSmem<H, G, T>::bytes(L.kv_chunk);                         \
@@ -508,10 +514,10 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
                                      cudaFuncAttributeMaxDynamicSharedMemorySize,             \
                                      static_cast<int>(smem)));                                \
     ProfScope prof(s, "attn_decode");                                                         \
-    attn::decode_split_kernel<T, G, H><<<grid, 256, smem, s>>>(qkv, ix, static_cast<T*>(kc),  \
-        static_cast<T*>(vc), L.kv_cap, L.kv_len, L.kv_chunk, L.n_q, L.n_kv, scale, ml,        \
-        counters, o, device_error_word());                                                    \
-    TP_LAUNCH_CHECK();                                                                        \
+    auto* kern = attn::decode_split_kernel<T, G, H>;                                          \
+    TP_LAUNCH_PDL(kern, grid, dim3(256), smem, s, qkv, ix, static_cast<T*>(kc),               \
+                  static_cast<T*>(vc), L.kv_cap, L.kv_len, L.kv_chunk, L.n_q, L.n_kv, scale,  \
+                  ml, counters, o, device_error_word());                                      \
   } else
   TP_DECODE_CASE(8, 128) TP_DECODE_CASE(4, 128) TP_DECODE_CASE(2, 128) TP_DECODE_CASE(1, 128)
   TP_DECODE_CASE(8, 64) TP_DECODE_CASE(4, 64) TP_DECODE_CASE(2, 64) TP_DECODE_CASE(1, 64)

@@ -109,7 +109,8 @@ struct GemmOpts {
 };
 
 // Launch gemm_kernel<Cfg, Epi> over ``batch`` problems of D = A B^T (M x N, contraction K).
-// With ``sk`` the stream-K schedule is used (and its counters are zeroed on the stream first).
+// With ``sk`` the stream-K schedule is used (and its counters are zeroed on the stream first, by
+// a small kernel).  Both kernels are launched with programmatic dependent launch.
 template <class Cfg, class Epi>
 tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int64_t K,
                    int64_t batch, const typename Epi::Params& ep, cudaStream_t stream,
@@ -162,7 +163,9 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
     gp.counters = static_cast<int32_t*>(sk->ws);
     gp.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(sk->ws) + pl.counter_bytes);
     grid_sk = pl.grid;
-    TP_CUDA_TRY(cudaMemsetAsync(sk->ws, 0, pl.counter_bytes, stream));
+    const int64_t words = static_cast<int64_t>(pl.counter_bytes / 4);
+    TP_LAUNCH_PDL(zero_words_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words, 256), 64))),
+                  dim3(256), 0, stream, static_cast<uint32_t*>(sk->ws), words);
   }
 
   static int attr_set[64] = {0};
@@ -177,8 +180,8 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   const int64_t tiles = static_cast<int64_t>(gp.batch) * gp.m_blocks * gp.n_blocks;
   const int grid = sk ? grid_sk : static_cast<int>(std::min<int64_t>(tiles, num_sms()));
   ProfScope prof(stream, label);
-  gemm_kernel<Cfg, Epi><<<grid, kThreads, Cfg::SMEM_BYTES, stream>>>(ta, tb, gp, ep);
-  TP_LAUNCH_CHECK();
+  auto* kern = gemm_kernel<Cfg, Epi>;
+  TP_LAUNCH_PDL(kern, dim3(grid), dim3(kThreads), Cfg::SMEM_BYTES, stream, ta, tb, gp, ep);
   return TP_OK;
 }
 

@@ -37,6 +37,8 @@ template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) reduce_vec8_kernel(const Tin* __restrict__ part, int p,
                                                           int64_t n, const Tout* res,
                                                           Tout* out) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   const int64_t nv = n >> 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
@@ -65,6 +67,8 @@ template <typename Tin, typename Tout, int PMAX>
 __global__ void __launch_bounds__(256) reduce_vec8_small_kernel(const Tin* __restrict__ part,
                                                                 int p, int64_t n,
                                                                 const Tout* res, Tout* out) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   const int64_t nv = n >> 3;
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t i = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; i < nv;
@@ -95,6 +99,8 @@ __global__ void __launch_bounds__(256) reduce_vec8_small_kernel(const Tin* __res
 template <typename Tin, typename Tout>
 __global__ void reduce_scalar_kernel(const Tin* part, int p, int64_t n, const Tout* res,
                                      Tout* out) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
   for (int64_t j = blockIdx.x * static_cast<int64_t>(blockDim.x) + threadIdx.x; j < n; j += stride) {
     float acc = to_f(part[j]);
@@ -117,14 +123,17 @@ inline tp_status launch_t(const void* part, int p, int64_t n, const void* res, v
   if (blocks > cap) blocks = cap;
   ProfScope prof(s, "reduce_partials");
   if (vec && p <= 8)
-    reduce_vec8_small_kernel<Tin, Tout, 8><<<static_cast<int>(blocks), 256, 0, s>>>(
-        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+    (void)launch_pdl(reduce_vec8_small_kernel<Tin, Tout, 8>, dim3(static_cast<unsigned>(blocks)),
+                     dim3(256), 0, s, static_cast<const Tin*>(part), p, n,
+                     static_cast<const Tout*>(res), static_cast<Tout*>(out));
   else if (vec)
-    reduce_vec8_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
-        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+    (void)launch_pdl(reduce_vec8_kernel<Tin, Tout>, dim3(static_cast<unsigned>(blocks)), dim3(256),
+                     0, s, static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res),
+                     static_cast<Tout*>(out));
   else
-    reduce_scalar_kernel<Tin, Tout><<<static_cast<int>(blocks), 256, 0, s>>>(
-        static_cast<const Tin*>(part), p, n, static_cast<const Tout*>(res), static_cast<Tout*>(out));
+    (void)launch_pdl(reduce_scalar_kernel<Tin, Tout>, dim3(static_cast<unsigned>(blocks)),
+                     dim3(256), 0, s, static_cast<const Tin*>(part), p, n,
+                     static_cast<const Tout*>(res), static_cast<Tout*>(out));
   TP_LAUNCH_CHECK();
   return TP_OK;
 }
@@ -147,6 +156,8 @@ __global__ void __launch_bounds__(512) reduce_norm_rows_kernel(const Tin* __rest
                                                                 int64_t rows, int64_t d,
                                                                 const Tout* res, Tout* out,
                                                                 Tn* norm, float eps) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   __shared__ float red[16];
   const int64_t n = rows * d;
   const int64_t base = static_cast<int64_t>(blockIdx.x) * d;
@@ -212,13 +223,15 @@ inline void reduce_norm_launch(const void* part, int p, int64_t rows, int64_t d,
                    (reinterpret_cast<uintptr_t>(out) & 15) == 0 &&
                    (!res || (reinterpret_cast<uintptr_t>(res) & 15) == 0);
   if (vec)
-    reduce_norm_rows_kernel<Tin, Tout, Tn, true><<<static_cast<unsigned>(rows), 512, 0, s>>>(
-        static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
-        static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
+    (void)launch_pdl(reduce_norm_rows_kernel<Tin, Tout, Tn, true>, dim3(static_cast<unsigned>(rows)),
+                     dim3(512), 0, s, static_cast<const Tin*>(part), p, rows, d,
+                     static_cast<const Tout*>(res), static_cast<Tout*>(out),
+                     static_cast<Tn*>(norm), eps);
   else
-    reduce_norm_rows_kernel<Tin, Tout, Tn, false><<<static_cast<unsigned>(rows), 512, 0, s>>>(
-        static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
-        static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
+    (void)launch_pdl(reduce_norm_rows_kernel<Tin, Tout, Tn, false>,
+                     dim3(static_cast<unsigned>(rows)), dim3(512), 0, s,
+                     static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
+                     static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
 }
 
 inline tp_status rmsnorm(const void* x, int in_dtype, int64_t rows, int64_t d, float eps,
@@ -253,6 +266,8 @@ inline tp_status reduce_norm(const float* part, int p, int64_t rows, int64_t d, 
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* x, int64_t d, float eps,
                                                       Tout* out) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   __shared__ float red[8];
   const Tin* xr = x + blockIdx.x * d;
   Tout* orow = out + blockIdx.x * d;
@@ -279,8 +294,8 @@ __global__ void __launch_bounds__(256) rmsnorm_kernel(const Tin* x, int64_t d, f
 template <typename Tin, typename Tout>
 inline void rmsnorm_launch(const void* x, int64_t rows, int64_t d, float eps, void* out,
                            cudaStream_t s) {
-  rmsnorm_kernel<Tin, Tout><<<static_cast<unsigned>(rows), 256, 0, s>>>(
-      static_cast<const Tin*>(x), d, eps, static_cast<Tout*>(out));
+  (void)launch_pdl(rmsnorm_kernel<Tin, Tout>, dim3(static_cast<unsigned>(rows)), dim3(256), 0, s,
+                   static_cast<const Tin*>(x), d, eps, static_cast<Tout*>(out));
 }
 
 // RMSNorm for few rows (fewer than SMs): block (c, r) recomputes the sum of squares of the whole
@@ -290,6 +305,8 @@ constexpr int kSplitW = 512;
 template <typename Tin, typename Tout>
 __global__ void __launch_bounds__(256) rmsnorm_split_kernel(const Tin* __restrict__ x, int64_t d,
                                                             float eps, Tout* __restrict__ out) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
   __shared__ float red[8];
   const Tin* xr = x + static_cast<int64_t>(blockIdx.y) * d;
   Tout* orow = out + static_cast<int64_t>(blockIdx.y) * d;
@@ -327,8 +344,8 @@ template <typename Tin, typename Tout>
 inline void rmsnorm_split_launch(const void* x, int64_t rows, int64_t d, float eps, void* out,
                                  cudaStream_t s) {
   const dim3 grid(static_cast<unsigned>(ceil_div(d, kSplitW)), static_cast<unsigned>(rows));
-  rmsnorm_split_kernel<Tin, Tout><<<grid, 256, 0, s>>>(static_cast<const Tin*>(x), d, eps,
-                                                       static_cast<Tout*>(out));
+  (void)launch_pdl(rmsnorm_split_kernel<Tin, Tout>, grid, dim3(256), 0, s,
+                   static_cast<const Tin*>(x), d, eps, static_cast<Tout*>(out));
 }
 
 inline bool rmsnorm_split_ok(const void* x, int64_t rows, int64_t d, const void* out) {

@@ -27,6 +27,42 @@ void count_reduction();
       return ::tp::set_error(TP_ERR_CUDA, std::string(#expr) + ": " + cudaGetErrorString(_e));  \
   } while (0)
 
+// Programmatic dependent launch.  A kernel launched with launch_pdl() may start, and run up to
+// its pdl_wait(), while the previous kernel on the stream is still finishing (its launch latency
+// and set-up overlap that kernel's tail); pdl_wait() returns once the previous kernel has
+// completed and its memory is visible, so stream order is kept for everything after it.  Every
+// kernel launched this way calls pdl_wait() before it touches global memory, and pdl_trigger()
+// to let the next kernel start launching.  Both are no-ops for an ordinary launch.
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+__device__ __forceinline__ void pdl_trigger() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+template <typename... KArgs, typename... Args>
+inline cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem,
+                              cudaStream_t s, Args... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
+// launch_pdl + error check + launch count (inside a function returning tp_status)
+#define TP_LAUNCH_PDL(kern, grid, block, smem, stream, ...)                                     \
+  do {                                                                                          \
+    cudaError_t _e = ::tp::launch_pdl(kern, grid, block, smem, stream, __VA_ARGS__);           \
+    if (_e != cudaSuccess)                                                                      \
+      return ::tp::set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(_e)); \
+    ::tp::count_launch();                                                                       \
+  } while (0)
+
 #define TP_LAUNCH_CHECK()                                                                       \
   do {                                                                                          \
     cudaError_t _e = cudaGetLastError();                                                        \
@@ -34,6 +70,17 @@ void count_reduction();
       return ::tp::set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(_e)); \
     ::tp::count_launch();                                                                       \
   } while (0)
+
+// Zero n 32-bit words.  Used instead of a memset for the small counter arrays in front of a
+// kernel, so that the stream keeps a chain of programmatically launched kernels.
+static __global__ void zero_words_kernel(uint32_t* p, int64_t n) {
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n;
+       i += static_cast<int64_t>(gridDim.x) * blockDim.x)
+    p[i] = 0u;
+}
+
 
 // Brackets one kernel launch with CUDA events when tp_profile_enable(1) is in effect.
 class ProfScope {
