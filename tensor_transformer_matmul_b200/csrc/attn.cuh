@@ -97,7 +97,7 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   L->wqkv_bytes = static_cast<size_t>(P * L->R_a * L->h) * L->eb;
   L->wo_bytes = static_cast<size_t>(P * L->h * L->qh * L->hd) * L->eb;
   if (L->kv_len > 0) {
-    // about one wave of blocks over (split, KV head, sequence); chunks a multiple of 16 keys
+    // blocks over (split, KV head, sequence); chunks a multiple of 16 keys
     const int64_t n_keys = L->kv_len + 1;
     // at most one wave: splits * n_kv * b <= SMs when possible; a split's K and V rows must fit
     // in shared memory (staged by bulk copies)
@@ -118,7 +118,7 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   const size_t ob = static_cast<size_t>(L->tokens * L->n_q * L->hd) * L->eb;
   const size_t partb = static_cast<size_t>(P * L->tokens * L->h) * 4;
   // decode split-KV scratch: per (sequence, q head, split) an (m, l) pair and hd outputs
-  const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (2 + L->hd) * 4;
+  const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (L->hd + 4) * 4;
   L->reduce_mode = d->reduce_mode;
   L->tc = d->dtype == TP_BF16 && d->h % 8 == 0;
   L->qkv_off = 0;
@@ -250,7 +250,8 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, Q
 //   3. o_a[d] = sum_key p[key][a] v[key][d]: each thread owns one dim d and GROUP*HD/256 heads
 // The new token (position kv_len) takes its key and value from the projection; the split that
 // holds it patches them into its staged rows and stores them into cache slot kv_len.
-// Output per (bi, q head, split): m (log2 units), l, o[hd].
+// Output per (bi, q head, split): a record of hd + 4 floats, o[hd] then m (log2 units) and l
+// (16-byte aligned records, so the merge reads o with vector loads).
 template <int HD, int GROUP, typename T>
 struct DecodeSmem {
   static size_t bytes(int chunk) {
@@ -269,6 +270,7 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
   constexpr int LPK = HD / 8;            // lanes per key
   constexpr int KPW = 32 / LPK;          // keys per warp pass
   constexpr int APT = (GROUP * HD + 255) / 256;   // heads per thread in phase 3
+  constexpr int kRec = HD + 4;                    // floats per split record: o[HD], m, l, pad
   extern __shared__ __align__(16) uint8_t dsm[];
   T* sK = reinterpret_cast<T*>(dsm);
   T* sV = sK + static_cast<size_t>(chunk) * HD;
@@ -333,14 +335,22 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
 
   // ---- phase 1: scores
   {
+    // the group's query vectors, scaled, staged once per block in shared memory
+    __shared__ __align__(16) float s_q[GROUP][HD];
+    for (int idx = threadIdx.x; idx < GROUP * HD; idx += blockDim.x) {
+      const int a = idx / HD, e = idx - a * HD;
+      s_q[a][e] = to_f(qkv[ix.q(bi, g * GROUP + a) + e]) * sl2;
+    }
+    __syncthreads();
     const int kslot = lane / LPK;
     const int d0 = (lane % LPK) * 8;
     float q[GROUP][8];
 #pragma unroll
     for (int a = 0; a < GROUP; ++a) {
-      const T* qp = qkv + ix.q(bi, g * GROUP + a) + d0;
-#pragma unroll
-      for (int e = 0; e < 8; ++e) q[a][e] = to_f(qp[e]) * sl2;
+      const float4 q0 = *reinterpret_cast<const float4*>(&s_q[a][d0]);
+      const float4 q1 = *reinterpret_cast<const float4*>(&s_q[a][d0 + 4]);
+      q[a][0] = q0.x; q[a][1] = q0.y; q[a][2] = q0.z; q[a][3] = q0.w;
+      q[a][4] = q1.x; q[a][5] = q1.y; q[a][6] = q1.z; q[a][7] = q1.w;
     }
     const int stride = kWarps * KPW;
     for (int wb = warp * KPW; wb < nk; wb += stride) {   // warp-uniform trip count
@@ -412,17 +422,17 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
         const int a = a0 + t;
         if (a < GROUP) {
           const int j = g * GROUP + a;
-          float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * (2 + HD);
+          float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * kRec;
           if (d == 0) {
-            rec[0] = s_m[a];   // in log2 units (the scores carry log2(e))
-            rec[1] = s_l[a];
+            rec[HD] = s_m[a];   // in log2 units (the scores carry log2(e))
+            rec[HD + 1] = s_l[a];
           }
-          rec[2 + d] = acc[t];
+          rec[d] = acc[t];
         }
       }
     }
   }
-  // the last block of this (sequence, KV head) to finish merges all splits, in split order:
+  // the last block of this (sequence, KV head) to finish merges all splits (fixed order):
   // o = sum_c exp(m_c - M) o_c / sum_c exp(m_c - M) l_c   (no block waits for another)
   __shared__ int s_last;
   __threadfence();
@@ -436,37 +446,59 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  // weights w[a][c] = exp(m_c - M_a) / L_a of every split, then independent loads of the o_c
+  // weights w[a][c] = exp(m_c - M_a) / L_a of every split: all (m, l) pairs are loaded at once,
+  // then one warp per query head reduces over the splits with shuffles; then independent loads
+  // of the o_c
   constexpr int kMaxSplits = 64;
-  __shared__ float s_w[GROUP][kMaxSplits];
+  __shared__ float s_w[GROUP][kMaxSplits], s_lc[GROUP][kMaxSplits];
   const int splits = gridDim.x;   // <= kMaxSplits (host)
-  const float* recs = ml + (bi * n_q + static_cast<int64_t>(g) * GROUP) * splits * (2 + HD);
+  const float* recs = ml + (bi * n_q + static_cast<int64_t>(g) * GROUP) * splits * kRec;
   for (int idx = threadIdx.x; idx < GROUP * splits; idx += blockDim.x) {
     const int a = idx / splits, sp = idx - a * splits;
-    s_w[a][sp] = __ldcg(recs + (static_cast<int64_t>(a) * splits + sp) * (2 + HD));   // m
+    const float* r = recs + (static_cast<int64_t>(a) * splits + sp) * kRec;
+    s_w[a][sp] = __ldcg(r + HD);        // m (log2 units)
+    s_lc[a][sp] = __ldcg(r + HD + 1);   // l
   }
   __syncthreads();
-  if (threadIdx.x < GROUP) {
-    const int a = threadIdx.x;
-    float M = -INFINITY;
-    for (int sp = 0; sp < splits; ++sp) M = fmaxf(M, s_w[a][sp]);
-    float Ls = 0.f;
-    for (int sp = 0; sp < splits; ++sp) {
-      const float f = s_w[a][sp] == -INFINITY ? 0.f : exp2f(s_w[a][sp] - M);
-      s_w[a][sp] = f;
-      Ls += __ldcg(recs + (static_cast<int64_t>(a) * splits + sp) * (2 + HD) + 1) * f;
-    }
+  for (int a = warp; a < GROUP; a += kWarps) {
+    // splits <= 64: lane handles splits lane and lane + 32
+    const float m0 = lane < splits ? s_w[a][lane] : -INFINITY;
+    const float m1 = lane + 32 < splits ? s_w[a][lane + 32] : -INFINITY;
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+    const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    float Ls = (lane < splits ? s_lc[a][lane] * f0 : 0.f) +
+               (lane + 32 < splits ? s_lc[a][lane + 32] * f1 : 0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
     const float inv = 1.f / Ls;
-    for (int sp = 0; sp < splits; ++sp) s_w[a][sp] *= inv;
+    if (lane < splits) s_w[a][lane] = f0 * inv;
+    if (lane + 32 < splits) s_w[a][lane + 32] = f1 * inv;
   }
   __syncthreads();
-  for (int idx = threadIdx.x; idx < GROUP * HD; idx += blockDim.x) {
-    const int a = idx / HD, e = idx - a * HD;
-    const float* r = recs + static_cast<int64_t>(a) * splits * (2 + HD) + 2 + e;
-    float acc2 = 0.f;
-#pragma unroll 8
-    for (int sp = 0; sp < splits; ++sp) acc2 += s_w[a][sp] * __ldcg(r + static_cast<int64_t>(sp) * (2 + HD));
-    o[bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + e] = from_f<T>(acc2);
+  // o: four consecutive dims per thread, every split's 16-byte load issued before the adds,
+  // which run in split order
+  constexpr int V4 = HD / 4;
+  for (int idx = threadIdx.x; idx < GROUP * V4; idx += blockDim.x) {
+    const int a = idx / V4, e4 = idx - a * V4;
+    const float4* r = reinterpret_cast<const float4*>(recs + static_cast<int64_t>(a) * splits * kRec) + e4;
+    float4 acc2 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 16
+    for (int sp = 0; sp < splits; ++sp) {
+      const float4 v = __ldcg(r + static_cast<int64_t>(sp) * (kRec / 4));
+      const float w = s_w[a][sp];
+      acc2.x += w * v.x;
+      acc2.y += w * v.y;
+      acc2.z += w * v.z;
+      acc2.w += w * v.w;
+    }
+    T* op = o + bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + 4 * e4;
+    op[0] = from_f<T>(acc2.x);
+    op[1] = from_f<T>(acc2.y);
+    op[2] = from_f<T>(acc2.z);
+    op[3] = from_f<T>(acc2.w);
   }
 }
 
