@@ -84,6 +84,14 @@ class Dist:
             self.pg.destroy_process_group()
 
 
+def job_throughput(dist, ms_local, units_per_rank):
+    """Whole-job rate of N replicas: every rank processed ``units_per_rank`` units; the job took
+    as long as the slowest rank (max over ranks of the device-timed ``ms_local``).  Returns
+    (max ms, units of all ranks per second)."""
+    ms = dist.max(ms_local)
+    return ms, units_per_rank * dist.world / (ms / 1e3)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while a timed region runs."""
 
@@ -267,10 +275,9 @@ def run_ours(args, dist):
     launches = tp.tp_launch_count() - l0
     clocks = clk.stop()
     dist.barrier()
-    ms = dist.max(ms)
+    ms, value = job_throughput(dist, ms, c["T"] * args.steps)
     ms_step = ms / args.steps
     tokens = c["T"] * args.steps * dist.world
-    value = tokens / (ms / 1e3)
 
     # per-kernel durations, measured with events on the launching stream over K more steps
     prof = _profile(tp, step, args.steps)
