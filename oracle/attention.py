@@ -160,3 +160,78 @@ def attention_decode(x, wq, wk, wv, wo, k_cache, v_cache, n_q, n_kv, head_dim):
         kn.append(k[0])
         vn.append(v[0])
     return np.concatenate(ys, axis=0), np.stack(kn), np.stack(vn)
+
+
+# ----------------------------------------------------------------------------------- backward
+# "Tensor Parallelism" (klaylearn), Notes: the attention block is column-parallel Q/K/V, local
+# attention and a row-parallel output projection, so its backward has the same shape as the
+# MLP's ("How does tensor parallelism split a transformer feed-forward block's two matmuls",
+# "The backward pass"; the same page notes the pattern applies to multi-head attention): dY is
+# replicated, each shard's weight gradients need no exchange, and dX is the sum of per-shard
+# partials.  Here the block is unsharded; the chain rule is written out step by step.
+
+
+def attend_backward(q, k, v, do, causal, q_pos0=0):
+    """Gradients of one head's attention o = softmax(q k^T / sqrt(hd) [masked]) v.
+
+    q (Sq, hd), k and v (Sk, hd), do (Sq, hd) = dL/do.  Returns dq, dk, dv.
+      P = softmax(S), dV = P^T dO, dP = dO V^T,
+      dS = P * (dP - D) with D = rowsum(dO * O) (= rowsum(P * dP)),
+      dQ = dS K / sqrt(hd), dK = dS^T Q / sqrt(hd).
+    """
+    q, k, v, do = _f64(q), _f64(k), _f64(v), _f64(do)
+    hd = q.shape[-1]
+    scale = 1.0 / np.sqrt(hd)
+    s = (q @ k.T) * scale
+    if causal:
+        qpos = q_pos0 + np.arange(q.shape[0])[:, None]
+        kpos = np.arange(k.shape[0])[None, :]
+        s = np.where(kpos <= qpos, s, -np.inf)
+    p = softmax_rows(s)
+    o = p @ v
+    dv = p.T @ do
+    dp = do @ v.T
+    d = np.sum(do * o, axis=-1, keepdims=True)
+    ds = p * (dp - d)
+    dq = (ds @ k) * scale
+    dk = (ds.T @ q) * scale
+    return dq, dk, dv
+
+
+def attention_backward(x, wq, wk, wv, wo, dy, n_q, n_kv, head_dim, causal=True):
+    """Unsharded block backward.  x and dy (b, s, h).  Returns dx (b, s, h) and the weight
+    gradients dWq (h, n_q hd), dWk and dWv (h, n_kv hd), dWo (n_q hd, h), summed over the batch.
+
+      O = attention(x Wq, x Wk, x Wv),  y = O Wo
+      dWo = O^T dY,  dO = dY Wo^T,  (dQ, dK, dV) per head by attend_backward (a KV head collects
+      the dK, dV of every query head that reads it),
+      dWq = x^T dQ,  dWk = x^T dK,  dWv = x^T dV,  dx = dQ Wq^T + dK Wk^T + dV Wv^T.
+    """
+    x, dy = _f64(x), _f64(dy)
+    if x.ndim == 2:
+        x, dy = x[None], dy[None]
+    wq, wk, wv, wo = _f64(wq), _f64(wk), _f64(wv), _f64(wo)
+    dwq, dwk, dwv, dwo = (np.zeros_like(wq), np.zeros_like(wk), np.zeros_like(wv),
+                          np.zeros_like(wo))
+    dxs = []
+    for bi in range(x.shape[0]):
+        S = x.shape[1]
+        q, k, v = project_qkv(x[bi], wq, wk, wv, n_q, n_kv, head_dim)
+        o = attention_heads(q, k, v, n_q, n_kv, causal)               # (S, n_q hd)
+        dwo += o.T @ dy[bi]
+        do = (dy[bi] @ wo.T).reshape(S, n_q, head_dim)
+        dq = np.zeros((S, n_q, head_dim))
+        dk = np.zeros((S, n_kv, head_dim))
+        dv = np.zeros((S, n_kv, head_dim))
+        for j in range(n_q):
+            g = kv_head_of(j, n_q, n_kv)
+            a, b_, c = attend_backward(q[:, j], k[:, g], v[:, g], do[:, j], causal)
+            dq[:, j] = a
+            dk[:, g] += b_
+            dv[:, g] += c
+        dq, dk, dv = (t.reshape(S, -1) for t in (dq, dk, dv))
+        dwq += x[bi].T @ dq
+        dwk += x[bi].T @ dk
+        dwv += x[bi].T @ dv
+        dxs.append(dq @ wq.T + dk @ wk.T + dv @ wv.T)
+    return np.stack(dxs), dwq, dwk, dwv, dwo

@@ -154,3 +154,65 @@ def test_rows_match_full_forward():
     rows = [0, 5, 10]
     got = attention.attention_forward_rows(x, wq, wk, wv, wo, n_q, n_kv, hd, rows, causal=True)
     np.testing.assert_allclose(got, full[rows], rtol=1e-12, atol=1e-13)
+
+
+# ------------------------------------------------------------------------------ backward pins
+def _torch_grads(x, wq, wk, wv, wo, dy, n_q, n_kv, hd, causal):
+    """Library routine: torch autograd through SDPA in float64 with repeat-interleaved KV heads."""
+    T = [torch.tensor(a, requires_grad=True) for a in (x, wq, wk, wv, wo)]
+    X, Wq, Wk, Wv, Wo = T
+    b, s, _ = x.shape
+    Q = (X @ Wq).reshape(b, s, n_q, hd).transpose(1, 2)
+    K = (X @ Wk).reshape(b, s, n_kv, hd).transpose(1, 2).repeat_interleave(n_q // n_kv, 1)
+    V = (X @ Wv).reshape(b, s, n_kv, hd).transpose(1, 2).repeat_interleave(n_q // n_kv, 1)
+    O = torch.nn.functional.scaled_dot_product_attention(Q, K, V, is_causal=causal)
+    Y = O.transpose(1, 2).reshape(b, s, n_q * hd) @ Wo
+    (Y * torch.tensor(dy)).sum().backward()
+    return [t.grad.numpy() for t in T]
+
+
+@pytest.mark.parametrize("causal", [True, False])
+@pytest.mark.parametrize("n_q,n_kv", [(4, 2), (4, 4), (8, 1)])
+def test_backward_matches_torch_autograd(causal, n_q, n_kv):
+    hd = 8
+    x, wq, wk, wv, wo = _case(2, 9, 24, n_q, n_kv, hd, seed=20)
+    dy = np.random.default_rng(21).standard_normal(x.shape)
+    got = attention.attention_backward(x, wq, wk, wv, wo, dy, n_q, n_kv, hd, causal)
+    ref = _torch_grads(x, wq, wk, wv, wo, dy, n_q, n_kv, hd, causal)
+    for g, r in zip(got, ref):
+        np.testing.assert_allclose(g, r, rtol=1e-10, atol=1e-12)
+
+
+def test_backward_central_differences():
+    # L = sum(y * dY); every gradient entry checked against (L(w+e) - L(w-e)) / 2e in float64
+    n_q, n_kv, hd = 4, 2, 3
+    x, wq, wk, wv, wo = _case(1, 5, 6, n_q, n_kv, hd, seed=22)
+    dy = np.random.default_rng(23).standard_normal(x.shape)
+    grads = attention.attention_backward(x, wq, wk, wv, wo, dy, n_q, n_kv, hd, True)
+    args = [x, wq, wk, wv, wo]
+    eps = 1e-6
+
+    def loss(a):
+        return float(np.sum(attention.attention_forward(*a, n_q, n_kv, hd, True) * dy))
+
+    for which, g in enumerate(grads):
+        base = args[which]
+        for idx in np.ndindex(base.shape):
+            plus = [a.copy() for a in args]
+            minus = [a.copy() for a in args]
+            plus[which][idx] += eps
+            minus[which][idx] -= eps
+            fd = (loss(plus) - loss(minus)) / (2 * eps)
+            assert abs(fd - g[idx]) <= 1e-6 * max(1.0, abs(fd)), (which, idx, fd, g[idx])
+
+
+def test_backward_single_key_closed_form():
+    # one position: the softmax has a single entry, so o = v and the scores get no gradient:
+    # dq = dk = 0 and dv = do for every head (summed over the heads sharing a KV head)
+    n_q, n_kv, hd = 4, 2, 5
+    q, k, v = (np.random.default_rng(24 + i).standard_normal((1, hd)) for i in range(3))
+    do = np.random.default_rng(27).standard_normal((1, hd))
+    dq, dk, dv = attention.attend_backward(q, k, v, do, causal=True)
+    # dS = P (dP - D) with dP = do.v and D = sum(do * o), o = v: zero up to summation order
+    assert np.abs(dq).max() < 1e-14 and np.abs(dk).max() < 1e-14
+    np.testing.assert_allclose(dv, do, rtol=0, atol=0)
