@@ -208,6 +208,30 @@ tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const void* wqkv_
                       const void* wo_p, void* k_cache, void* v_cache, const void* residual,
                       void* y, void* y_norm, void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of the self-attention block (kv_len == 0; bf16 with h a multiple of 8; no flags).
+ * ("Tensor Parallelism" (klaylearn), Notes: Q/K/V column-parallel, local attention, row-parallel
+ * output projection; "How does tensor parallelism split a transformer feed-forward block's two
+ * matmuls", "The backward pass": dY replicated, per-shard weight gradients with no exchange,
+ * the input gradient summed from per-shard partials.)
+ *   dy [b][s][h] bf16 = dL/dy (the output of tp_attn_fwd without residual);
+ *   dx [b][s][h] bf16 = sum_i dx_i, summed in shard order in fp32 (adds 1 to the reduction
+ *      counter);
+ *   dwqkv_p, dwo_p: fp32 gradients of wqkv_p and wo_p in their packed per-shard layouts
+ *      (tp_attn_wqkv_packed_bytes / tp_attn_wo_packed_bytes * 2 bytes; tp_attn_unpack_grads
+ *      scatters them back), summed over the batch.
+ * The forward's q, k, v, o and row log-sum-exp are recomputed from x inside the call (the
+ * forward keeps no activations).  workspace: tp_attn_bwd_workspace(desc) bytes (0 for an
+ * unsupported descriptor).  Returns TP_ERR_UNSUPPORTED for decode, fp32, flags or head_dim > 256. */
+size_t tp_attn_bwd_workspace(const tp_attn_desc* desc);
+tp_status tp_attn_bwd(const tp_attn_desc* desc, const void* x, const void* wqkv_p,
+                      const void* wo_p, const void* dy, void* dx, void* dwqkv_p, void* dwo_p,
+                      void* workspace, size_t ws_bytes, void* stream);
+
+/* Scatter packed fp32 attention gradients back to the user layout (fp32): dwq [h][n_q*hd],
+ * dwk and dwv [h][n_kv*hd], dwo [n_q*hd][h]. */
+tp_status tp_attn_unpack_grads(const tp_attn_desc* desc, const void* dwqkv_p, const void* dwo_p,
+                               void* dwq, void* dwk, void* dwv, void* dwo, void* stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* Reduction and glue                                                                          */
 /* ------------------------------------------------------------------------------------------ */

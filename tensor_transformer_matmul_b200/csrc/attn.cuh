@@ -192,7 +192,7 @@ struct QkvIdx {
 template <typename T>
 __global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, QkvIdx ix,
                                                            int64_t b, int64_t s, int n_q,
-                                                           int causal, float scale) {
+                                                           int causal, float scale, float* lse) {
   constexpr int kMaxPerLane = 8;  // head_dim <= 256
   const int64_t wid = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
   const int lane = threadIdx.x & 31;
@@ -238,6 +238,8 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, Q
     const int e = lane + 32 * r;
     if (r < per && e < ix.hd) o[t * static_cast<int64_t>(n_q) * ix.hd + j * ix.hd + e] = from_f<T>(acc[r] * inv);
   }
+  // log2 of the softmax denominator in units of the log2-scaled scores (backward pass)
+  if (lse && lane == 0) lse[t * n_q + j] = (m + logf(l)) * 1.4426950408889634f;
 }
 
 // Decode attention, split over keys.  Block = (split c, KV head g, sequence bi), 256 threads.
@@ -506,7 +508,7 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
 
 template <typename T>
 inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, void* kc, void* vc,
-                           float* ml, int* counters, cudaStream_t s) {
+                           float* ml, int* counters, cudaStream_t s, float* lse = nullptr) {
   const T* qkv = static_cast<const T*>(qkv_v);
   T* o = static_cast<T*>(o_v);
   attn::QkvIdx ix{L.p * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
@@ -517,15 +519,17 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
     if (tc) {
       const int group = L.n_q / L.n_kv;
       if (L.hd == 128)
-        return fa::launch<128>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s);
-      return fa::launch<64>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s);
+        return fa::launch<128>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s,
+                               lse);
+      return fa::launch<64>(qkv, L.b, L.s, L.n_q, L.qh, L.kh, group, L.R_a, L.p, L.causal, o, s,
+                            lse);
     }
     const int64_t warps = L.tokens * L.n_q;
     const int64_t blocks = ceil_div(warps * 32, 128);
     if (blocks > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "attention grid too large");
     ProfScope prof(s, "attn_prefill");
     attn::prefill_simt_kernel<T><<<static_cast<unsigned>(blocks), 128, 0, s>>>(
-        qkv, o, ix, L.b, L.s, L.n_q, L.causal, scale);
+        qkv, o, ix, L.b, L.s, L.n_q, L.causal, scale, lse);
     TP_LAUNCH_CHECK();
     return TP_OK;
   }

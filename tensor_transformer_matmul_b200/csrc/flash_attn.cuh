@@ -68,6 +68,7 @@ struct Params {
   int32_t causal;
   float scale_log2;   // log2(e) / sqrt(hd)
   __nv_bfloat16* o;   // [b*s][n_q*hd]
+  float* lse;         // optional [b*s][n_q]: log2 of each row's softmax denominator (scaled units)
   uint32_t* err;
 };
 
@@ -378,6 +379,10 @@ __global__ void __launch_bounds__(kThreads, 2)
   if (ok) {
     tc_fence_after();
     const float inv = l_run > 0.f ? 1.f / l_run : 0.f;
+    // p = 2^(s * scale_log2 - lse) reproduces the softmax (used by the backward pass)
+    if (P.lse && q_abs < P.s)
+      P.lse[(static_cast<int64_t>(bi) * P.s + q_abs) * P.n_q + j] =
+          (m_run == -INFINITY ? 0.f : m_run * P.scale_log2) + log2f(l_run);
     const bool live = q_abs < P.s;
     __nv_bfloat16* dst = P.o + (static_cast<int64_t>(bi) * P.s + q_abs) * (P.n_q * HD) + j * HD;
 #pragma unroll
@@ -428,7 +433,8 @@ __global__ void __launch_bounds__(kThreads, 2)
 // Host launcher: qkv [b][s][p*R_a] bf16 (packed per shard: Q heads, K heads, V heads), o out.
 template <int HD>
 inline tp_status launch(const void* qkv, int64_t b, int64_t s, int n_q, int qh, int kh, int group,
-                        int64_t R_a, int p, int causal, void* o, cudaStream_t st) {
+                        int64_t R_a, int p, int causal, void* o, cudaStream_t st,
+                        float* lse = nullptr) {
   using L = Smem<HD>;
   CUtensorMap map;
   const uint64_t cols = static_cast<uint64_t>(p) * R_a;
@@ -452,6 +458,7 @@ inline tp_status launch(const void* qkv, int64_t b, int64_t s, int n_q, int qh, 
   P.causal = causal;
   P.scale_log2 = 1.4426950408889634f / sqrtf(static_cast<float>(HD));
   P.o = static_cast<__nv_bfloat16*>(o);
+  P.lse = lse;
   P.err = device_error_word();
   dim3 grid(static_cast<unsigned>(n_q), static_cast<unsigned>(P.n_qt), static_cast<unsigned>(b));
   ProfScope prof(st, "attn_prefill");

@@ -882,5 +882,43 @@ struct EpiActBwd {
   }
 };
 
+// ---------------------------------------------------------------------------------------------
+// bf16 store of the accumulator, problem b's columns placed b * col_off to the right:
+// out[i][b * col_off + j] = D[i][j] for i < rows_valid, j < cols_valid (not swapped).  Used for
+// the attention backward's dO_i = dY Wo_i^T, which lands in the [tokens][n_q hd] layout of o.
+// ---------------------------------------------------------------------------------------------
+struct EpiStoreBf16 {
+  struct Params {
+    __nv_bfloat16* out;
+    int64_t ld;        // elements between rows
+    int64_t col_off;   // column offset per problem
+    int32_t rows_valid, cols_valid;
+  };
+
+  template <class Cfg, class Src>
+  __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
+                                             const Src& src) {
+    const int i = c.m0 + c.row;
+    const bool live = i < p.rows_valid;
+    __nv_bfloat16* base =
+        p.out + static_cast<int64_t>(i) * p.ld + static_cast<int64_t>(c.b) * p.col_off;
+#pragma unroll 1
+    for (int col = 0; col < Cfg::BN; col += 32) {
+      float v[32];
+      src.load32(col, v);   // warp-collective: every lane loads
+      const int j0 = c.n0 + col;
+      if (!live) continue;
+      __nv_bfloat16* dst = base + j0;
+      if (j0 + 32 <= p.cols_valid && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
+        store_bf16x32(dst, v);
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e)
+          if (j0 + e < p.cols_valid) dst[e] = __float2bfloat16_rn(v[e]);
+      }
+    }
+  }
+};
+
 }  // namespace tc
 }  // namespace tp

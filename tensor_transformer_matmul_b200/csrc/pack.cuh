@@ -87,7 +87,7 @@ __global__ void pack_rows_kernel(T* out, int p, int64_t nrows, int64_t Kp, int64
 // Inverse of pack_cols for fp32 gradients: dst_s[k][col] = in[r][k] for every valid packed row r
 // (each valid (s, col) is hit by exactly one r).  Tiles run over packed rows.
 static __global__ void unpack_cols_kernel(const float* in, int64_t rows, int64_t K, ColMap cm,
-                                   float* dst0, float* dst1) {
+                                   float* dst0, float* dst1, float* dst2) {
   __shared__ float tile[kT][kT + 1];
   const int64_t r0 = static_cast<int64_t>(blockIdx.x) * kT, k0 = static_cast<int64_t>(blockIdx.y) * kT;
   const int tx = threadIdx.x, ty = threadIdx.y;
@@ -101,7 +101,7 @@ static __global__ void unpack_cols_kernel(const float* in, int64_t rows, int64_t
     if (r < rows && k < K) {
       int s; int64_t col;
       cm.map(r, s, col);
-      float* d = s == 0 ? dst0 : (s == 1 ? dst1 : nullptr);
+      float* d = s == 0 ? dst0 : (s == 1 ? dst1 : (s == 2 ? dst2 : nullptr));
       if (d) d[k * cm.ld[s] + col] = tile[tx][j];
     }
   }

@@ -56,3 +56,66 @@ extern "C" tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const 
   if (st == TP_OK) tp::count_reduction();
   return st;
 }
+
+// ------------------------------------------------------------------------------------ backward
+#include "attn_bwd.cuh"
+
+namespace {
+tp_status attn_bwd_check(const tp_attn_desc* desc, tp::AttnLayout* L) {
+  tp_status st = tp::attn_layout_of(desc, L);
+  if (st != TP_OK) return st;
+  if (L->kv_len != 0) return tp::set_error(TP_ERR_UNSUPPORTED, "backward is for self-attention (kv_len == 0)");
+  if (!L->tc) return tp::set_error(TP_ERR_UNSUPPORTED, "backward needs bf16 with h a multiple of 8");
+  if (L->hd > 256) return tp::set_error(TP_ERR_UNSUPPORTED, "backward needs head_dim <= 256");
+  if (desc->flags != 0) return tp::set_error(TP_ERR_UNSUPPORTED, "backward takes no flags");
+  return TP_OK;
+}
+}  // namespace
+
+extern "C" size_t tp_attn_bwd_workspace(const tp_attn_desc* desc) {
+  tp::AttnLayout L;
+  if (attn_bwd_check(desc, &L) != TP_OK) return 0;
+  return tp::attn_bwd_layout(L).bytes;
+}
+
+extern "C" tp_status tp_attn_bwd(const tp_attn_desc* desc, const void* x, const void* wqkv_p,
+                                 const void* wo_p, const void* dy, void* dx, void* dwqkv_p,
+                                 void* dwo_p, void* workspace, size_t ws_bytes, void* stream) {
+  tp::clear_error();
+  tp::AttnLayout L;
+  tp_status st = attn_bwd_check(desc, &L);
+  if (st != TP_OK) return st;
+  if (L.tokens == 0) {
+    tp::count_reduction();
+    return TP_OK;
+  }
+  if (!x || !wqkv_p || !wo_p || !dy || !dx || !dwqkv_p || !dwo_p || !workspace)
+    return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  for (const void* q : {x, wqkv_p, wo_p, dy, static_cast<const void*>(dx),
+                        static_cast<const void*>(dwqkv_p), static_cast<const void*>(dwo_p)})
+    if (reinterpret_cast<uintptr_t>(q) & 15)
+      return tp::set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const tp::AttnBwdLayout B = tp::attn_bwd_layout(L);
+  if (ws_bytes < B.bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tp::tensor_cores_usable())
+    return tp::set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  st = tp::attn_backward(L, x, wqkv_p, wo_p, dy, dx, static_cast<float*>(dwqkv_p),
+                         static_cast<float*>(dwo_p), workspace, static_cast<cudaStream_t>(stream));
+  if (st == TP_OK) tp::count_reduction();
+  return st;
+}
+
+extern "C" tp_status tp_attn_unpack_grads(const tp_attn_desc* desc, const void* dwqkv_p,
+                                          const void* dwo_p, void* dwq, void* dwk, void* dwv,
+                                          void* dwo, void* stream) {
+  tp::clear_error();
+  tp::AttnLayout L;
+  tp_status st = tp::attn_layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (!dwqkv_p || !dwo_p || !dwq || !dwk || !dwv || !dwo)
+    return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  return tp::attn_unpack_grads(L, static_cast<const float*>(dwqkv_p),
+                               static_cast<const float*>(dwo_p), static_cast<float*>(dwq),
+                               static_cast<float*>(dwk), static_cast<float*>(dwv),
+                               static_cast<float*>(dwo), static_cast<cudaStream_t>(stream));
+}

@@ -450,7 +450,7 @@ extern "C" tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw
   dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.d, 32)), 1);
   pack::unpack_cols_kernel<<<g1, blk, 0, s>>>(static_cast<const float*>(dw1p), rows, L.d,
                                                w1_colmap(L, dw1, dw_up), static_cast<float*>(dw1),
-                                               static_cast<float*>(dw_up));
+                                               static_cast<float*>(dw_up), nullptr);
   TP_LAUNCH_CHECK();
   dim3 g2(static_cast<unsigned>(ceil_div(L.d, 32)), static_cast<unsigned>(ceil_div(L.Fsp, 32)),
           static_cast<unsigned>(L.p));

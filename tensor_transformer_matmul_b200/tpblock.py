@@ -33,7 +33,7 @@ EXPORTS = (
     "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
     "tp_profile_enable", "tp_profile_read", "tp_profile_reset", "tp_mlp_fwd_static_ws",
-    "tp_selftest_wait_timeout",
+    "tp_selftest_wait_timeout", "tp_attn_bwd_workspace", "tp_attn_bwd", "tp_attn_unpack_grads",
 )
 
 
@@ -92,6 +92,9 @@ def load():
         "tp_status_string": (ctypes.c_char_p, [I32]), "tp_check_device_error": (I32, [P]),
         "tp_tensor_core_path_available": (I32, []), "tp_version": (I32, []),
         "tp_selftest_wait_timeout": (I32, [ctypes.c_uint32, P]),
+        "tp_attn_bwd_workspace": (S, [AD]),
+        "tp_attn_bwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_unpack_grads": (I32, [AD, P, P, P, P, P, P, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
@@ -226,6 +229,21 @@ def tp_attn_fwd(desc, x, wqkv_p, wo_p, y, k_cache=None, v_cache=None, residual=N
                               _ptr(k_cache), _ptr(v_cache), _ptr(residual), _ptr(y),
                               _ptr(y_norm), _ptr(workspace), _nbytes(workspace),
                               _stream(stream)))
+
+
+def tp_attn_bwd_workspace(desc):
+    return load().tp_attn_bwd_workspace(ctypes.byref(desc))
+
+
+def tp_attn_bwd(desc, x, wqkv_p, wo_p, dy, dx, dwqkv_p, dwo_p, workspace=None, stream=None):
+    _check(load().tp_attn_bwd(ctypes.byref(desc), _ptr(x), _ptr(wqkv_p), _ptr(wo_p), _ptr(dy),
+                              _ptr(dx), _ptr(dwqkv_p), _ptr(dwo_p), _ptr(workspace),
+                              _nbytes(workspace), _stream(stream)))
+
+
+def tp_attn_unpack_grads(desc, dwqkv_p, dwo_p, dwq, dwk, dwv, dwo, stream=None):
+    _check(load().tp_attn_unpack_grads(ctypes.byref(desc), _ptr(dwqkv_p), _ptr(dwo_p), _ptr(dwq),
+                                       _ptr(dwk), _ptr(dwv), _ptr(dwo), _stream(stream)))
 
 
 # ------------------------------------------------------------------------- reduce and glue

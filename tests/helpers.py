@@ -92,3 +92,20 @@ class Attn:
         self.lib.tp_attn_fwd(self.desc, x.to(dev()), self.wqkv, self.wo, y, k_cache=k_cache,
                              v_cache=v_cache, residual=residual, workspace=self.ws)
         return y
+
+    def backward(self, x, dy):
+        """tp_attn_bwd; returns dx and the unpacked fp32 weight gradients dwq, dwk, dwv, dwo."""
+        g = dev()
+        lib = self.lib
+        dx = torch.empty(self.b, self.s, self.h, dtype=inputs.TORCH_DTYPE[self.dtype], device=g)
+        dwqkv_p = torch.empty(self.wqkv.numel(), dtype=torch.float32, device=g)
+        dwo_p = torch.empty(self.wo.numel(), dtype=torch.float32, device=g)
+        ws = torch.empty(lib.tp_attn_bwd_workspace(self.desc), dtype=torch.uint8, device=g)
+        lib.tp_attn_bwd(self.desc, x.to(g), self.wqkv, self.wo, dy.to(g), dx, dwqkv_p, dwo_p,
+                        workspace=ws)
+        dwq = torch.empty(self.h, self.n_q * self.hd, dtype=torch.float32, device=g)
+        dwk = torch.empty(self.h, self.n_kv * self.hd, dtype=torch.float32, device=g)
+        dwv = torch.empty(self.h, self.n_kv * self.hd, dtype=torch.float32, device=g)
+        dwo = torch.empty(self.n_q * self.hd, self.h, dtype=torch.float32, device=g)
+        lib.tp_attn_unpack_grads(self.desc, dwqkv_p, dwo_p, dwq, dwk, dwv, dwo)
+        return dx, dwq, dwk, dwv, dwo
