@@ -361,6 +361,9 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     if "attention" in which:
         ex["attention_block"] = extra_attention(tp, inputs, torch, stream, peaks, steps)
         time.sleep(1.0)
+        ex["attention_block_bwd"] = extra_attention_bwd(tp, inputs, torch, stream, peaks,
+                                                        max(3, steps // 4))
+        time.sleep(1.0)
     if "prefill" in which:
         ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
     return ex
@@ -488,6 +491,48 @@ def extra_attention(tp, inputs, torch, stream, peaks, steps):
         "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12, 1),
         "frac_of_burst_peak": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "tokens_per_s": round(s / (ms_a / 1e3), 1),
+        "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
+        "steps": steps}
+
+
+def extra_attention_bwd(tp, inputs, torch, stream, peaks, steps):
+    """Backward of the GQA attention block (prefill): recomputed forward, dO and dWo GEMMs,
+    dQ/dK/dV, dWqkv and dX GEMMs, dX reduce."""
+    a = ATTN
+    dev = torch.device("cuda", torch.cuda.current_device())
+    ai = inputs.attn_inputs(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], "bf16", seed=0,
+                            device=dev)
+    ad = tp.attn_desc(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], a["p"])
+    wqkv = torch.empty(tp.tp_attn_wqkv_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
+    wo = torch.empty(tp.tp_attn_wo_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
+    tp.tp_attn_pack(ad, ai["wq"], ai["wk"], ai["wv"], ai["wo"], wqkv, wo)
+    dy = inputs.normal((a["b"], a["s"], a["h"]), 1.0, 0, 97, "bf16", dev)
+    dx = torch.empty_like(ai["x"])
+    dwqkv = torch.empty(wqkv.numel(), dtype=torch.float32, device=dev)
+    dwo = torch.empty(wo.numel(), dtype=torch.float32, device=dev)
+    ws = torch.empty(tp.tp_attn_bwd_workspace(ad), dtype=torch.uint8, device=dev)
+
+    def bwd():
+        tp.tp_attn_bwd(ad, ai["x"], wqkv, wo, dy, dx, dwqkv, dwo, workspace=ws)
+
+    for _ in range(3):
+        bwd()
+    ms = _cuda_time(bwd, steps, stream) / steps
+    s, h = a["s"], a["h"]
+    rqkv = (a["n_q"] + 2 * a["n_kv"]) * a["hd"]
+    fl_proj = 2.0 * s * h * rqkv            # one projection-sized GEMM (QKV)
+    fl_o = 2.0 * s * a["n_q"] * a["hd"] * h  # one O-projection-sized GEMM
+    fl_att = 2.0 * 2 * a["n_q"] * a["hd"] * s * (s + 1) / 2
+    # recomputed forward (QKV GEMM + attention), dO and dWo, dQ/dK/dV (2.5x the forward's
+    # attention matmuls), dWqkv and dX
+    flops = fl_proj + fl_att + 2 * fl_o + 2.5 * fl_att + 2 * fl_proj
+    prof = _profile(tp, bwd, steps)
+    return {
+        "workload": "TP GQA attention backward: b=1, s=2048, h=8192, 64 Q / 8 KV heads, hd=128, "
+                    "p=8, causal (forward recomputed inside)",
+        "ms": round(ms, 3),
+        "TFLOP_per_s": round(flops / (ms / 1e3) / 1e12, 1),
+        "frac_of_burst_peak": round(flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
         "steps": steps}
 

@@ -57,3 +57,17 @@ def test_backward_rejects_unsupported(lib):
     assert lib.tp_attn_bwd_workspace(a.desc) == 0      # decode has no backward
     with pytest.raises(lib.TpError):
         a.backward(inp["x"], torch.zeros(1, 1, 64, dtype=torch.bfloat16))
+
+
+def test_backward_llama_heads(lib):
+    # the full head structure of the attention configuration (h=8192, 64 query / 8 KV heads,
+    # head_dim 128, p=8) at 512 tokens: four query tiles of the flash forward, every shard
+    inp = inputs.attn_inputs(1, 512, 8192, 64, 8, 128, "bf16", seed=34, w_std=0.02)
+    dy = inputs.normal((1, 512, 8192), 1.0, 34, 97, "bf16", "cpu")
+    a = Attn(lib, inp, 8, "bf16", True, n_q=64, n_kv=8, hd=128)
+    got = a.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    ref = _grads_ref(inp, dy, 64, 8, 128, True)
+    for name, g, r in zip(("dx", "dwq", "dwk", "dwv", "dwo"), got, ref):
+        err = rel_l2(f64(g), r)
+        assert err <= TOL["bf16"], (name, err)
