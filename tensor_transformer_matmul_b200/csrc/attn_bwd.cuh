@@ -17,12 +17,14 @@
 //   dx = sum_i [dQ dK dV]_i Wqkv_i         (per-shard partials, summed in shard order)
 //
 // The forward quantities Q, K, V, O and the log-sum-exp are recomputed from x (the forward call
-// keeps no activations).  The GEMMs run on the tcgen05 core; dQ, dK and dV run in SIMT kernels
-// (one warp per query row and head for dQ, one per key row and KV head for dK and dV, so each
-// output is summed by one warp in a fixed order; no atomics).
+// keeps no activations).  The GEMMs run on the tcgen05 core.  dQ, dK and dV run in the tcgen05
+// kernels of flash_bwd.cuh for head_dim 64 and 128, otherwise in SIMT kernels (one warp per query
+// row and head for dQ, one per key row and KV head for dK and dV).  Each output is summed by one
+// CTA or warp in a fixed order; no atomics.
 #pragma once
 
 #include "attn.cuh"
+#include "flash_bwd.cuh"
 
 namespace tp {
 namespace attn {
@@ -248,24 +250,43 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
                    a, bo, L.h, K, T, P, ep, s, "attn_dwo_gemm");
     if (st != TP_OK) return st;
   }
-  // dQ, dK, dV of every head
+  // dQ, dK, dV of every head: tcgen05 kernels for head_dim 64/128, SIMT kernels otherwise
   {
+#define return_if_error(expr)          \
+  do {                                 \
+    tp_status _r = (expr);             \
+    if (_r != TP_OK) return _r;        \
+  } while (0)
     attn::QkvIdx ix{P * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
     const float scale = 1.0f / sqrtf(static_cast<float>(L.hd));
     const float scale_log2 = scale * 1.4426950408889634f;
     const int64_t rows = T * L.n_q, krows = T * L.n_kv;
     if (ceil_div(rows * 32, 128) > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "grid too large");
+    {
+      ProfScope prof(s, "attn_bwd_rowdot");
+      attn::bwd_rowdot_kernel<BF><<<static_cast<unsigned>(ceil_div(rows * 32, 128)), 128, 0, s>>>(
+          o, dO, T, L.n_q, L.hd, D);
+      TP_LAUNCH_CHECK();
+    }
+    const int group = L.n_q / L.n_kv;
+    if ((L.hd == 128 || L.hd == 64) && L.b <= 65535 && L.s <= INT32_MAX) {
+      if (L.hd == 128)
+        return_if_error(fb::launch_bwd<128>(qkv, dO, lse, D, dqkv, L.b, L.s, L.n_q, L.qh, L.kh,
+                                            group, L.R_a, L.p, L.causal, s));
+      else
+        return_if_error(fb::launch_bwd<64>(qkv, dO, lse, D, dqkv, L.b, L.s, L.n_q, L.qh, L.kh,
+                                           group, L.R_a, L.p, L.causal, s));
+    } else {
     ProfScope prof(s, "attn_bwd_core");
-    attn::bwd_rowdot_kernel<BF><<<static_cast<unsigned>(ceil_div(rows * 32, 128)), 128, 0, s>>>(
-        o, dO, T, L.n_q, L.hd, D);
-    TP_LAUNCH_CHECK();
     attn::bwd_dq_kernel<BF><<<static_cast<unsigned>(ceil_div(rows * 32, 128)), 128, 0, s>>>(
         qkv, dO, ix, lse, D, L.b, L.s, L.n_q, L.causal, scale_log2, scale, dqkv);
     TP_LAUNCH_CHECK();
     attn::bwd_dkv_kernel<BF><<<static_cast<unsigned>(ceil_div(krows * 32, 128)), 128, 0, s>>>(
         qkv, dO, ix, lse, D, L.b, L.s, L.n_q, L.n_kv, L.causal, scale_log2, scale, dqkv);
     TP_LAUNCH_CHECK();
+    }
   }
+#undef return_if_error
   // dWqkv_i[r][k] = sum_t dqkv_i[t][r] x[t][k]   (no exchange between shards)
   {
     const Operand a{dqkv, true, L.R_a, T, P, P * L.R_a, L.R_a};

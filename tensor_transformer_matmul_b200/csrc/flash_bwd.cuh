@@ -1,0 +1,556 @@
+// Attention backward on the tensor cores (sm_100a), head_dim 64 or 128, bf16.
+//
+//   With P = softmax(S), S = Q K^T / sqrt(hd) (causal mask), O = P V, the row log-sum-exp of
+//   the forward and D = rowsum(dO * O):
+//     dV = P^T dO,  dP = dO V^T,  dS = P * (dP - D),  dK = dS^T Q / sqrt(hd),  dQ = dS K / sqrt(hd)
+//   ("Tensor Parallelism" (klaylearn), Notes: attention is local to the shard's heads, so each
+//   shard differentiates its own heads; a KV head collects dK and dV from every query head of
+//   its group.)
+//
+// Two kernels, neither with atomics (each output tile is summed by one CTA in a fixed order):
+//   * dK/dV: one CTA per (128-key block, KV head, sequence).  It walks the group's query heads
+//     and the query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in TMEM,
+//     the 128 threads (one key row each) turn them into P^T and dS^T (bf16, shared memory, K-major),
+//     and dV += P^T dO, dK += dS^T Q accumulate in TMEM (dO and Q read MN-major from the same tiles).
+//   * dQ: one CTA per (128-query block, query head, sequence).  It walks the key blocks its
+//     queries see; per step S = Q K^T and dP = dO V^T land in TMEM, the threads (one query row
+//     each) form dS (bf16, shared memory), and dQ += dS K accumulates in TMEM (K read MN-major).
+// Thread 0 issues the TMA loads and the MMAs; TMEM holds four (three) 128-column fp32 tiles.
+// Every wait is bounded; a timeout sets the abort flag, drains what was issued and leaves, and
+// the loop exit is CTA-uniform.
+#pragma once
+
+#include <cuda.h>
+
+#include "gemm_launch.cuh"
+#include "sm100.cuh"
+#include "tp_common.cuh"
+
+namespace tp {
+namespace fb {
+
+constexpr int kBlk = 128;       // query rows and key rows per block
+constexpr int kThreads = 128;
+
+struct Params {
+  int32_t s;                    // tokens per sequence
+  int32_t n_q, qh, kh, group;   // heads: total Q, per shard Q, per shard KV, n_q / n_kv
+  int32_t R_a;                  // packed qkv columns per shard
+  int32_t n_blk;                // 128-row blocks per sequence
+  int32_t causal;
+  int64_t ld;                   // qkv and dqkv row length (p * R_a)
+  float scale_log2, scale;      // log2(e) / sqrt(hd), 1 / sqrt(hd)
+  const float* lse;             // [b*s][n_q], log2 units of the scaled scores
+  const float* D;               // [b*s][n_q]
+  __nv_bfloat16* dqkv;
+  uint32_t* err;
+};
+
+template <int HD>
+struct Tiles {
+  static constexpr int SUB = HD / 64;           // 64-column swizzle sub-tiles along the head dim
+  static constexpr int TILE = kBlk * 128;       // one sub-tile: 128 rows x 128 bytes
+  static constexpr int BLOCK = SUB * TILE;      // one 128-row head tile
+  static constexpr int PTILE = 2 * TILE;        // a 128 x 128 bf16 tile (two sub-tiles)
+};
+
+__device__ __forceinline__ void fence_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
+// 32 bf16 (16 words) of row ``row`` at K-columns c0..c0+31 of a K-major 128B-swizzled tile made
+// of two 64-column sub-tiles of ``tile`` bytes each.
+__device__ __forceinline__ void st_kmajor32(uint8_t* base, int tile, int row, int c0,
+                                            const uint32_t (&w)[16]) {
+  uint8_t* sub = base + (c0 >> 6) * tile + row * 128;
+  const int ch0 = (c0 & 63) >> 3;
+#pragma unroll
+  for (int q = 0; q < 4; ++q)
+    *reinterpret_cast<uint4*>(sub + (((ch0 + q) ^ (row & 7)) << 4)) =
+        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
+}
+
+__device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
+  uint32_t r[32];
+  sm100::tmem_ld_32x32b_x32(taddr, r);
+  sm100::tmem_wait_ld();
+#pragma unroll
+  for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+}
+
+// bounded drain of what thread 0 issued, on the abort path
+struct Drain {
+  uint64_t t0;
+  uint32_t* err;
+  __device__ void operator()(uint64_t* bar, uint32_t par) const {
+    while (!sm100::mbar_try_wait(bar, par))
+      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+        record_device_error(err, DEVERR_WAIT_DRAIN);
+        return;
+      }
+  }
+};
+
+// ================================================================================ dK and dV
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    flash_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tma_qkv,
+                         const __grid_constant__ CUtensorMap tma_do, const Params P) {
+  using namespace sm100;
+  using L = Tiles<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sK = smem;
+  uint8_t* sV = sK + L::BLOCK;
+  uint8_t* sQ = sV + L::BLOCK;
+  uint8_t* sDO = sQ + L::BLOCK;
+  uint8_t* sPT = sDO + L::BLOCK;     // P^T  [key][query], K-major (K = query)
+  uint8_t* sDST = sPT + L::PTILE;    // dS^T [key][query]
+  float* lse_s = reinterpret_cast<float*>(sDST + L::PTILE);
+  float* D_s = lse_s + kBlk;
+  uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + kBlk);
+  uint64_t* kv_full = bar + 0;
+  uint64_t* qd_full = bar + 1;
+  uint64_t* s_full = bar + 2;
+  uint64_t* p_ready = bar + 3;
+  uint64_t* m_done = bar + 4;
+  uint64_t* drain = bar + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int kb = blockIdx.x, g = blockIdx.y, bi = blockIdx.z;
+  const int shard = g / P.kh, gl = g - shard * P.kh;
+  const int k_col = shard * P.R_a + (P.qh + gl) * HD;
+  const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
+  const int k0 = kb * kBlk;
+  const int qb0 = P.causal ? kb : 0;
+  const int nqb = P.n_blk - qb0;
+  const int n_iter = P.group * nqb;
+
+  if (tid == 0) {
+    mbar_init(kv_full, 1);
+    mbar_init(qd_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, kThreads);
+    mbar_init(m_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tma_qkv);
+    tma_prefetch_desc(&tma_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const int row = tid;
+  const int k_abs = k0 + row;
+  auto wait = [&](uint64_t* b, uint32_t par, uint32_t site) {
+    return mbar_wait(b, par, abort_flag, P.err, site);
+  };
+  constexpr uint32_t IDESC_KK = make_idesc_bf16(128, 128, false, false);   // S^T, dP^T
+  constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);     // dV, dK
+
+  uint32_t issued = 0;   // Q/dO loads issued (thread 0)
+  bool any_mma = false;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
+#pragma unroll
+    for (int c = 0; c < L::SUB; ++c) {
+      tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
+      tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
+    }
+  }
+  bool ok = true;
+  for (int it = 0; it < n_iter; ++it) {
+    if (!__syncthreads_and(ok ? 1 : 0)) {   // everyone is done with the previous step
+      ok = false;
+      break;
+    }
+    const int a = it / nqb, qb = qb0 + it % nqb;
+    const int j = g * P.group + a;
+    const int jl = j - shard * P.qh;
+    const int q_col = shard * P.R_a + jl * HD;
+    const int q0 = qb * kBlk;
+    {
+      const int t_abs = q0 + tid;
+      const bool valid = t_abs < P.s;
+      const int64_t ri = (static_cast<int64_t>(bi) * P.s + t_abs) * P.n_q + j;
+      lse_s[tid] = valid ? P.lse[ri] : 0.f;
+      D_s[tid] = valid ? P.D[ri] : 0.f;
+    }
+    __syncthreads();
+    if (tid == 0 && ok) {
+      if (it > 0) ok = wait(m_done, (it - 1) & 1, DEVERR_WAIT_ACC_EMPTY);   // Q, dO, P^T, dS^T free
+      if (ok) {
+        mbar_arrive_expect_tx(qd_full, 2 * L::BLOCK);
+#pragma unroll
+        for (int c = 0; c < L::SUB; ++c) {
+          tma_load_3d(&tma_qkv, qd_full, sQ + c * L::TILE, q_col + 64 * c, q0, bi);
+          tma_load_3d(&tma_do, qd_full, sDO + c * L::TILE, j * HD + 64 * c, q0, bi);
+        }
+        ++issued;
+        ok = wait(qd_full, it & 1, DEVERR_WAIT_FULL) &&
+             (it > 0 || wait(kv_full, 0, DEVERR_WAIT_FULL));
+      }
+      if (ok) {
+        tc_fence_after();
+        const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ),
+                       da = smem_addr(sDO);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
+          umma_f16(tS, make_sdesc_sw128(ka + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
+                   IDESC_KK, kk > 0 ? 1u : 0u);
+          umma_f16(tdP, make_sdesc_sw128(va + off, 16, 1024),
+                   make_sdesc_sw128(da + off, 16, 1024), IDESC_KK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        any_mma = true;
+      }
+    }
+    // ---- P^T and dS^T for this key row against the block's 128 queries
+    ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+        float sv[32], dp[32];
+        ld32(tS + lane_base + c0, sv);
+        ld32(tdP + lane_base + c0, dp);
+        uint32_t pw[16], dw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float pr[2], ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int qi = c0 + e + u, q_abs = q0 + qi;
+            const bool masked = q_abs >= P.s || k_abs >= P.s || (P.causal && k_abs > q_abs);
+            pr[u] = masked ? 0.f : exp2f(sv[e + u] * P.scale_log2 - lse_s[qi]);
+            ds[u] = pr[u] * (dp[e + u] - D_s[qi]);
+          }
+          pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+          dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+        st_kmajor32(sPT, L::TILE, row, c0, pw);
+        st_kmajor32(sDST, L::TILE, row, c0, dw);
+      }
+      fence_async_smem();
+    }
+    tc_fence_before();
+    mbar_arrive(p_ready);
+    if (tid == 0 && ok) {
+      ok = wait(p_ready, it & 1, DEVERR_WAIT_ACC_FULL);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t pa = smem_addr(sPT), sa = smem_addr(sDST), qa = smem_addr(sQ),
+                       da = smem_addr(sDO);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          const uint32_t aoff = (kk >> 2) * L::TILE + (kk & 3) * 32;
+          // B: the [query][dim] tiles read MN-major (N = dim), 16 query rows per MMA
+          umma_f16(tdV, make_sdesc_sw128(pa + aoff, 16, 1024),
+                   make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+          umma_f16(tdK, make_sdesc_sw128(sa + aoff, 16, 1024),
+                   make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                   (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(m_done);
+      }
+    }
+  }
+  if (!__syncthreads_and(ok ? 1 : 0)) ok = false;
+  if (ok) ok = __all_sync(0xffffffffu, wait(m_done, (n_iter - 1) & 1, DEVERR_WAIT_ACC_EMPTY));
+  if (ok) {
+    tc_fence_after();
+    const bool live = k_abs < P.s;
+    __nv_bfloat16* rowp = P.dqkv + (static_cast<int64_t>(bi) * P.s + k_abs) * P.ld;
+#pragma unroll 1
+    for (int c = 0; c < HD; c += 32) {
+      float v[32];
+      ld32(tdK + lane_base + c, v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] *= P.scale;
+      if (live) tc::store_bf16x32(rowp + k_col + c, v);
+      ld32(tdV + lane_base + c, v);
+      if (live) tc::store_bf16x32(rowp + v_col + c, v);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && tid == 0) {
+    const Drain dr{globaltimer_ns(), P.err};
+    dr(kv_full, 0);
+    if (issued) dr(qd_full, (issued - 1) & 1);
+    if (any_mma) {
+      umma_commit(drain);
+      dr(drain, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+// ======================================================================================= dQ
+template <int HD>
+__global__ void __launch_bounds__(kThreads, 1)
+    flash_bwd_dq_kernel(const __grid_constant__ CUtensorMap tma_qkv,
+                        const __grid_constant__ CUtensorMap tma_do, const Params P) {
+  using namespace sm100;
+  using L = Tiles<HD>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>(
+      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
+  uint8_t* sQ = smem;
+  uint8_t* sDO = sQ + L::BLOCK;
+  uint8_t* sK = sDO + L::BLOCK;
+  uint8_t* sV = sK + L::BLOCK;
+  uint8_t* sDS = sV + L::BLOCK;      // dS [query][key], K-major (K = key)
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sDS + L::PTILE);
+  uint64_t* qd_full = bar + 0;
+  uint64_t* kv_full = bar + 1;
+  uint64_t* s_full = bar + 2;
+  uint64_t* p_ready = bar + 3;
+  uint64_t* m_done = bar + 4;
+  uint64_t* drain = bar + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int tid = threadIdx.x, warp = tid >> 5;
+  const int qb = P.causal ? P.n_blk - 1 - static_cast<int>(blockIdx.x) : blockIdx.x;
+  const int j = blockIdx.y, bi = blockIdx.z;
+  const int shard = j / P.qh, jl = j - shard * P.qh;
+  const int g = j / P.group, gl = g - shard * P.kh;
+  const int q_col = shard * P.R_a + jl * HD;
+  const int k_col = shard * P.R_a + (P.qh + gl) * HD;
+  const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
+  const int q0 = qb * kBlk;
+  const int nkb = P.causal ? qb + 1 : P.n_blk;
+
+  if (tid == 0) {
+    mbar_init(qd_full, 1);
+    mbar_init(kv_full, 1);
+    mbar_init(s_full, 1);
+    mbar_init(p_ready, kThreads);
+    mbar_init(m_done, 1);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    tma_prefetch_desc(&tma_qkv);
+    tma_prefetch_desc(&tma_do);
+  }
+  if (warp == 0) {
+    tmem_alloc(tmem_slot, 512);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
+  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
+  const int row = tid;
+  const int q_abs = q0 + row;
+  const bool q_live = q_abs < P.s;
+  const int64_t ri = (static_cast<int64_t>(bi) * P.s + q_abs) * P.n_q + j;
+  const float lse_r = q_live ? P.lse[ri] : 0.f;
+  const float D_r = q_live ? P.D[ri] : 0.f;
+  auto wait = [&](uint64_t* b, uint32_t par, uint32_t site) {
+    return mbar_wait(b, par, abort_flag, P.err, site);
+  };
+  constexpr uint32_t IDESC_KK = make_idesc_bf16(128, 128, false, false);   // S, dP
+  constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);     // dQ
+
+  uint32_t issued = 0;   // K/V loads issued (thread 0)
+  bool any_mma = false;
+  if (tid == 0) {
+    mbar_arrive_expect_tx(qd_full, 2 * L::BLOCK);
+#pragma unroll
+    for (int c = 0; c < L::SUB; ++c) {
+      tma_load_3d(&tma_qkv, qd_full, sQ + c * L::TILE, q_col + 64 * c, q0, bi);
+      tma_load_3d(&tma_do, qd_full, sDO + c * L::TILE, j * HD + 64 * c, q0, bi);
+    }
+  }
+  bool ok = true;
+  for (int kb = 0; kb < nkb; ++kb) {
+    if (!__syncthreads_and(ok ? 1 : 0)) {
+      ok = false;
+      break;
+    }
+    const int k0 = kb * kBlk;
+    if (tid == 0 && ok) {
+      if (kb > 0) ok = wait(m_done, (kb - 1) & 1, DEVERR_WAIT_ACC_EMPTY);   // K, V, dS free
+      if (ok) {
+        mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
+#pragma unroll
+        for (int c = 0; c < L::SUB; ++c) {
+          tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
+          tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
+        }
+        ++issued;
+        ok = wait(kv_full, kb & 1, DEVERR_WAIT_FULL) &&
+             (kb > 0 || wait(qd_full, 0, DEVERR_WAIT_FULL));
+      }
+      if (ok) {
+        tc_fence_after();
+        const uint32_t qa = smem_addr(sQ), da = smem_addr(sDO), ka = smem_addr(sK),
+                       va = smem_addr(sV);
+#pragma unroll
+        for (int kk = 0; kk < HD / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
+          umma_f16(tS, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+                   IDESC_KK, kk > 0 ? 1u : 0u);
+          umma_f16(tdP, make_sdesc_sw128(da + off, 16, 1024),
+                   make_sdesc_sw128(va + off, 16, 1024), IDESC_KK, kk > 0 ? 1u : 0u);
+        }
+        umma_commit(s_full);
+        any_mma = true;
+      }
+    }
+    ok = __all_sync(0xffffffffu, ok && wait(s_full, kb & 1, DEVERR_WAIT_ACC_FULL));
+    if (ok) {
+      tc_fence_after();
+#pragma unroll 1
+      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+        float sv[32], dp[32];
+        ld32(tS + lane_base + c0, sv);
+        ld32(tdP + lane_base + c0, dp);
+        uint32_t dw[16];
+#pragma unroll
+        for (int e = 0; e < 32; e += 2) {
+          float ds[2];
+#pragma unroll
+          for (int u = 0; u < 2; ++u) {
+            const int k_abs = k0 + c0 + e + u;
+            const bool masked = !q_live || k_abs >= P.s || (P.causal && k_abs > q_abs);
+            const float pr = masked ? 0.f : exp2f(sv[e + u] * P.scale_log2 - lse_r);
+            ds[u] = pr * (dp[e + u] - D_r);
+          }
+          dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+        }
+        st_kmajor32(sDS, L::TILE, row, c0, dw);
+      }
+      fence_async_smem();
+    }
+    tc_fence_before();
+    mbar_arrive(p_ready);
+    if (tid == 0 && ok) {
+      ok = wait(p_ready, kb & 1, DEVERR_WAIT_ACC_FULL);
+      if (ok) {
+        tc_fence_after();
+        const uint32_t sa = smem_addr(sDS), ka = smem_addr(sK);
+#pragma unroll
+        for (int kk = 0; kk < kBlk / 16; ++kk) {
+          // B: the [key][dim] K tile read MN-major (N = dim), 16 key rows per MMA
+          umma_f16(tdQ, make_sdesc_sw128(sa + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024),
+                   make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                   (kb > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(m_done);
+      }
+    }
+  }
+  if (!__syncthreads_and(ok ? 1 : 0)) ok = false;
+  if (ok) ok = __all_sync(0xffffffffu, wait(m_done, (nkb - 1) & 1, DEVERR_WAIT_ACC_EMPTY));
+  if (ok) {
+    tc_fence_after();
+    __nv_bfloat16* rowp = P.dqkv + (static_cast<int64_t>(bi) * P.s + q_abs) * P.ld + q_col;
+#pragma unroll 1
+    for (int c = 0; c < HD; c += 32) {
+      float v[32];
+      ld32(tdQ + lane_base + c, v);
+#pragma unroll
+      for (int e = 0; e < 32; ++e) v[e] *= P.scale;
+      if (q_live) tc::store_bf16x32(rowp + c, v);
+    }
+  }
+  __syncthreads();
+  if (*abort_flag && tid == 0) {
+    const Drain dr{globaltimer_ns(), P.err};
+    dr(qd_full, 0);
+    if (issued) dr(kv_full, (issued - 1) & 1);
+    if (any_mma) {
+      umma_commit(drain);
+      dr(drain, 0);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 0) tmem_dealloc(tmem, 512);
+}
+
+template <int HD>
+constexpr int dkv_smem() { return 4 * Tiles<HD>::BLOCK + 2 * Tiles<HD>::PTILE + 2 * kBlk * 4 + 128 + 1024; }
+// at least 120 KB, so that no second CTA (which would wait for the 512 TMEM columns) shares an SM
+template <int HD>
+constexpr int dq_smem() {
+  return 4 * Tiles<HD>::BLOCK + Tiles<HD>::PTILE + 128 + 1024 > 120 * 1024
+             ? 4 * Tiles<HD>::BLOCK + Tiles<HD>::PTILE + 128 + 1024
+             : 120 * 1024;
+}
+
+// Host launcher.  qkv and dqkv [b][s][p*R_a] bf16 (packed per shard: Q heads, K heads, V heads),
+// dO [b][s][n_q*HD] bf16, lse and D [b*s][n_q] fp32.
+template <int HD>
+inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, const float* D,
+                            void* dqkv, int64_t b, int64_t s, int n_q, int qh, int kh, int group,
+                            int64_t R_a, int p, int causal, cudaStream_t st) {
+  CUtensorMap mq, md;
+  const uint64_t cols = static_cast<uint64_t>(p) * R_a;
+  tp_status r = encode_tmap_bf16_3d(&mq, qkv, cols, static_cast<uint64_t>(s),
+                                    static_cast<uint64_t>(b), cols * 2,
+                                    cols * 2 * static_cast<uint64_t>(s), 64, kBlk);
+  if (r != TP_OK) return r;
+  const uint64_t dcols = static_cast<uint64_t>(n_q) * HD;
+  r = encode_tmap_bf16_3d(&md, dO, dcols, static_cast<uint64_t>(s), static_cast<uint64_t>(b),
+                          dcols * 2, dcols * 2 * static_cast<uint64_t>(s), 64, kBlk);
+  if (r != TP_OK) return r;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  TP_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    TP_CUDA_TRY(cudaFuncSetAttribute(flash_bwd_dkv_kernel<HD>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dkv_smem<HD>()));
+    TP_CUDA_TRY(cudaFuncSetAttribute(flash_bwd_dq_kernel<HD>,
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dq_smem<HD>()));
+    attr_set[dev] = 1;
+  }
+  Params P;
+  P.s = static_cast<int32_t>(s);
+  P.n_q = n_q; P.qh = qh; P.kh = kh; P.group = group;
+  P.R_a = static_cast<int32_t>(R_a);
+  P.n_blk = static_cast<int32_t>(ceil_div(s, kBlk));
+  P.causal = causal;
+  P.ld = static_cast<int64_t>(cols);
+  P.scale = 1.0f / sqrtf(static_cast<float>(HD));
+  P.scale_log2 = P.scale * 1.4426950408889634f;
+  P.lse = lse;
+  P.D = D;
+  P.dqkv = static_cast<__nv_bfloat16*>(dqkv);
+  P.err = device_error_word();
+  const int n_kv = n_q / group;
+  ProfScope prof(st, "attn_bwd_flash");
+  flash_bwd_dkv_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk), static_cast<unsigned>(n_kv),
+                                  static_cast<unsigned>(b)),
+                             kThreads, dkv_smem<HD>(), st>>>(mq, md, P);
+  TP_LAUNCH_CHECK();
+  flash_bwd_dq_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk), static_cast<unsigned>(n_q),
+                                 static_cast<unsigned>(b)),
+                            kThreads, dq_smem<HD>(), st>>>(mq, md, P);
+  TP_LAUNCH_CHECK();
+  return TP_OK;
+}
+
+}  // namespace fb
+}  // namespace tp
