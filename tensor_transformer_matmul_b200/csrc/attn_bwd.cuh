@@ -180,7 +180,9 @@ inline AttnBwdLayout attn_bwd_layout(const AttnLayout& L) {
   const size_t qkvb = static_cast<size_t>(L.tokens * L.p * L.R_a) * 2;
   const size_t ob = static_cast<size_t>(L.tokens * L.n_q * L.hd) * 2;
   const size_t rowb = static_cast<size_t>(L.tokens * L.n_q) * 4;
-  const size_t partb = static_cast<size_t>(L.p * L.tokens * L.h) * 4;
+  // the dX partials; before them, the per-query-head dK/dV shares of the flash kernels
+  const size_t partb = std::max(static_cast<size_t>(L.p * L.tokens * L.h),
+                                static_cast<size_t>(L.tokens * L.n_q * 2 * L.hd)) * 4;
   B.qkv = 0;
   B.o = B.qkv + align256(qkvb);
   B.dO = B.o + align256(ob);
@@ -272,10 +274,10 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
     if ((L.hd == 128 || L.hd == 64) && L.b <= 65535 && L.s <= INT32_MAX) {
       if (L.hd == 128)
         return_if_error(fb::launch_bwd<128>(qkv, dO, lse, D, dqkv, L.b, L.s, L.n_q, L.qh, L.kh,
-                                            group, L.R_a, L.p, L.causal, s));
+                                            group, L.R_a, L.p, L.causal, part, s));
       else
         return_if_error(fb::launch_bwd<64>(qkv, dO, lse, D, dqkv, L.b, L.s, L.n_q, L.qh, L.kh,
-                                           group, L.R_a, L.p, L.causal, s));
+                                           group, L.R_a, L.p, L.causal, part, s));
     } else {
     ProfScope prof(s, "attn_bwd_core");
     attn::bwd_dq_kernel<BF><<<static_cast<unsigned>(ceil_div(rows * 32, 128)), 128, 0, s>>>(

@@ -43,6 +43,8 @@ struct Params {
   const float* lse;             // [b*s][n_q], log2 units of the scaled scores
   const float* D;               // [b*s][n_q]
   __nv_bfloat16* dqkv;
+  float* part_kv;               // split > 1: fp32 partial dK, dV [split][b*s][n_kv][2][hd]
+  int32_t split;                // CTAs sharing one key block's query heads
   uint32_t* err;
 };
 
@@ -120,14 +122,16 @@ __global__ void __launch_bounds__(kThreads, 1)
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
-  const int kb = blockIdx.x, g = blockIdx.y, bi = blockIdx.z;
+  const int kb = blockIdx.x, bi = blockIdx.z;
+  const int g = blockIdx.y / P.split, sp = blockIdx.y - g * P.split;   // KV head, head slice
+  const int heads = P.group / P.split, a0 = sp * heads;                 // query heads of this CTA
   const int shard = g / P.kh, gl = g - shard * P.kh;
   const int k_col = shard * P.R_a + (P.qh + gl) * HD;
   const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
   const int k0 = kb * kBlk;
   const int qb0 = P.causal ? kb : 0;
   const int nqb = P.n_blk - qb0;
-  const int n_iter = P.group * nqb;
+  const int n_iter = heads * nqb;
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
@@ -175,7 +179,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
       break;
     }
-    const int a = it / nqb, qb = qb0 + it % nqb;
+    const int a = a0 + it / nqb, qb = qb0 + it % nqb;
     const int j = g * P.group + a;
     const int jl = j - shard * P.qh;
     const int q_col = shard * P.R_a + jl * HD;
@@ -273,16 +277,37 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (ok) {
     tc_fence_after();
     const bool live = k_abs < P.s;
-    __nv_bfloat16* rowp = P.dqkv + (static_cast<int64_t>(bi) * P.s + k_abs) * P.ld;
+    const int64_t t = static_cast<int64_t>(bi) * P.s + k_abs;
+    __nv_bfloat16* rowp = P.dqkv + t * P.ld;
+    // split > 1: this CTA's share of dK (unscaled) and dV, added up by the combine kernel
+    const int64_t n_tok = static_cast<int64_t>(gridDim.z) * P.s;
+    const int n_kv = static_cast<int>(gridDim.y) / P.split;
+    float* prow = P.part_kv + ((static_cast<int64_t>(sp) * n_tok + t) * n_kv + g) * 2 * HD;
 #pragma unroll 1
     for (int c = 0; c < HD; c += 32) {
       float v[32];
       ld32(tdK + lane_base + c, v);
+      if (P.split > 1) {
+        if (live) {
 #pragma unroll
-      for (int e = 0; e < 32; ++e) v[e] *= P.scale;
-      if (live) tc::store_bf16x32(rowp + k_col + c, v);
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(prow + c)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      } else {
+#pragma unroll
+        for (int e = 0; e < 32; ++e) v[e] *= P.scale;
+        if (live) tc::store_bf16x32(rowp + k_col + c, v);
+      }
       ld32(tdV + lane_base + c, v);
-      if (live) tc::store_bf16x32(rowp + v_col + c, v);
+      if (P.split > 1) {
+        if (live) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            reinterpret_cast<float4*>(prow + HD + c)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+        }
+      } else if (live) {
+        tc::store_bf16x32(rowp + v_col + c, v);
+      }
     }
   }
   __syncthreads();
@@ -490,6 +515,34 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 0) tmem_dealloc(tmem, 512);
 }
 
+// dK = scale * sum_sp partial dK, dV = sum_sp partial dV, slices added in order; bf16 into dqkv.
+// One thread per 4 consecutive dims of one (token, KV head).
+template <int HD>
+__global__ void __launch_bounds__(256) combine_kv_kernel(const float* part, int split,
+                                                         int64_t n_tok, int n_kv, int kh,
+                                                         int qh, int64_t R_a, int64_t ld,
+                                                         float scale, __nv_bfloat16* dqkv) {
+  const int64_t idx = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  constexpr int V4 = HD / 4;
+  if (idx >= n_tok * n_kv * 2 * V4) return;
+  const int e4 = static_cast<int>(idx % V4);
+  const int which = static_cast<int>((idx / V4) & 1);   // 0: dK, 1: dV
+  const int64_t tg = idx / (2 * V4);
+  const int g = static_cast<int>(tg % n_kv);
+  const int64_t t = tg / n_kv;
+  float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+  for (int sp = 0; sp < split; ++sp) {
+    const float4 v = reinterpret_cast<const float4*>(
+        part + ((static_cast<int64_t>(sp) * n_tok + t) * n_kv + g) * 2 * HD + which * HD)[e4];
+    acc.x += v.x; acc.y += v.y; acc.z += v.z; acc.w += v.w;
+  }
+  const float f = which == 0 ? scale : 1.f;
+  const int shard = g / kh, gl = g - shard * kh;
+  __nv_bfloat16* dst = dqkv + t * ld + shard * R_a + (qh + which * kh + gl) * HD + 4 * e4;
+  reinterpret_cast<uint2*>(dst)[0] = make_uint2(pack_bf16x2(acc.x * f, acc.y * f),
+                                                pack_bf16x2(acc.z * f, acc.w * f));
+}
+
 template <int HD>
 constexpr int dkv_smem() { return 4 * Tiles<HD>::BLOCK + 2 * Tiles<HD>::PTILE + 2 * kBlk * 4 + 128 + 1024; }
 // at least 120 KB, so that no second CTA (which would wait for the 512 TMEM columns) shares an SM
@@ -505,7 +558,7 @@ constexpr int dq_smem() {
 template <int HD>
 inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, const float* D,
                             void* dqkv, int64_t b, int64_t s, int n_q, int qh, int kh, int group,
-                            int64_t R_a, int p, int causal, cudaStream_t st) {
+                            int64_t R_a, int p, int causal, float* part_kv, cudaStream_t st) {
   CUtensorMap mq, md;
   const uint64_t cols = static_cast<uint64_t>(p) * R_a;
   tp_status r = encode_tmap_bf16_3d(&mq, qkv, cols, static_cast<uint64_t>(s),
@@ -540,11 +593,22 @@ inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, c
   P.dqkv = static_cast<__nv_bfloat16*>(dqkv);
   P.err = device_error_word();
   const int n_kv = n_q / group;
+  // one CTA per query head of the group when the workspace slice is given (more CTAs than the
+  // key blocks times KV heads alone); their fp32 shares are added in order afterwards
+  P.split = (part_kv && group > 1) ? group : 1;
+  P.part_kv = part_kv;
   ProfScope prof(st, "attn_bwd_flash");
-  flash_bwd_dkv_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk), static_cast<unsigned>(n_kv),
-                                  static_cast<unsigned>(b)),
+  flash_bwd_dkv_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk),
+                                  static_cast<unsigned>(n_kv * P.split), static_cast<unsigned>(b)),
                              kThreads, dkv_smem<HD>(), st>>>(mq, md, P);
   TP_LAUNCH_CHECK();
+  if (P.split > 1) {
+    const int64_t n_tok = b * s;
+    const int64_t work = n_tok * n_kv * 2 * (HD / 4);
+    combine_kv_kernel<HD><<<static_cast<unsigned>(ceil_div(work, 256)), 256, 0, st>>>(
+        part_kv, P.split, n_tok, n_kv, kh, qh, R_a, P.ld, P.scale, P.dqkv);
+    TP_LAUNCH_CHECK();
+  }
   flash_bwd_dq_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk), static_cast<unsigned>(n_q),
                                  static_cast<unsigned>(b)),
                             kThreads, dq_smem<HD>(), st>>>(mq, md, P);
