@@ -8,13 +8,16 @@
 //   its group.)
 //
 // Two kernels, neither with atomics (each output tile is summed by one CTA in a fixed order):
-//   * dK/dV: one CTA per (128-key block, KV head, sequence).  It walks the group's query heads
-//     and the query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in TMEM,
-//     the 128 threads (one key row each) turn them into P^T and dS^T (bf16, shared memory, K-major),
-//     and dV += P^T dO, dK += dS^T Q accumulate in TMEM (dO and Q read MN-major from the same tiles).
+//   * dK/dV: one CTA per (128-key block, KV head, query head of its group, sequence).  It walks
+//     the query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in TMEM,
+//     the 128 threads (one key row each) turn them into P^T and dS^T, written back as bf16 over
+//     their own TMEM columns, and dV += P^T dO, dK += dS^T Q accumulate in TMEM with P^T and
+//     dS^T as the TMEM A operands (dO and Q read MN-major).  Q and dO are double buffered, so
+//     the next step's tiles load during this one.  The per-head shares are added afterwards.
 //   * dQ: one CTA per (128-query block, query head, sequence).  It walks the key blocks its
 //     queries see; per step S = Q K^T and dP = dO V^T land in TMEM, the threads (one query row
-//     each) form dS (bf16, shared memory), and dQ += dS K accumulates in TMEM (K read MN-major).
+//     each) write dS back over S, and dQ += dS K accumulates in TMEM (K read MN-major).  K and
+//     V are double buffered.
 // Thread 0 issues the TMA loads and the MMAs; TMEM holds four (three) 128-column fp32 tiles.
 // Every wait is bounded; a timeout sets the abort flag, drains what was issued and leaves, and
 // the loop exit is CTA-uniform.
@@ -22,6 +25,7 @@
 
 #include <cuda.h>
 
+#include "flash_attn.cuh"
 #include "gemm_launch.cuh"
 #include "sm100.cuh"
 #include "tp_common.cuh"
@@ -53,24 +57,7 @@ struct Tiles {
   static constexpr int SUB = HD / 64;           // 64-column swizzle sub-tiles along the head dim
   static constexpr int TILE = kBlk * 128;       // one sub-tile: 128 rows x 128 bytes
   static constexpr int BLOCK = SUB * TILE;      // one 128-row head tile
-  static constexpr int PTILE = 2 * TILE;        // a 128 x 128 bf16 tile (two sub-tiles)
 };
-
-__device__ __forceinline__ void fence_async_smem() {
-  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
-}
-
-// 32 bf16 (16 words) of row ``row`` at K-columns c0..c0+31 of a K-major 128B-swizzled tile made
-// of two 64-column sub-tiles of ``tile`` bytes each.
-__device__ __forceinline__ void st_kmajor32(uint8_t* base, int tile, int row, int c0,
-                                            const uint32_t (&w)[16]) {
-  uint8_t* sub = base + (c0 >> 6) * tile + row * 128;
-  const int ch0 = (c0 & 63) >> 3;
-#pragma unroll
-  for (int q = 0; q < 4; ++q)
-    *reinterpret_cast<uint4*>(sub + (((ch0 + q) ^ (row & 7)) << 4)) =
-        make_uint4(w[4 * q], w[4 * q + 1], w[4 * q + 2], w[4 * q + 3]);
-}
 
 __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
   uint32_t r[32];
@@ -78,6 +65,17 @@ __device__ __forceinline__ void ld32(uint32_t taddr, float (&v)[32]) {
   sm100::tmem_wait_ld();
 #pragma unroll
   for (int e = 0; e < 32; ++e) v[e] = __uint_as_float(r[e]);
+}
+
+// 32 bf16 values (16 words) of this lane's row into TMEM columns taddr .. taddr+15
+__device__ __forceinline__ void st16(uint32_t taddr, const uint32_t (&w)[16]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16};" ::"r"(taddr),
+      "r"(w[0]), "r"(w[1]), "r"(w[2]), "r"(w[3]), "r"(w[4]), "r"(w[5]), "r"(w[6]), "r"(w[7]),
+      "r"(w[8]), "r"(w[9]), "r"(w[10]), "r"(w[11]), "r"(w[12]), "r"(w[13]), "r"(w[14]),
+      "r"(w[15])
+      : "memory");
 }
 
 // bounded drain of what thread 0 issued, on the abort path
@@ -105,20 +103,18 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + L::BLOCK;
-  uint8_t* sQ = sV + L::BLOCK;
-  uint8_t* sDO = sQ + L::BLOCK;
-  uint8_t* sPT = sDO + L::BLOCK;     // P^T  [key][query], K-major (K = query)
-  uint8_t* sDST = sPT + L::PTILE;    // dS^T [key][query]
-  float* lse_s = reinterpret_cast<float*>(sDST + L::PTILE);
+  uint8_t* sQ = sV + L::BLOCK;        // [2] buffers
+  uint8_t* sDO = sQ + 2 * L::BLOCK;   // [2] buffers
+  float* lse_s = reinterpret_cast<float*>(sDO + 2 * L::BLOCK);
   float* D_s = lse_s + kBlk;
   uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + kBlk);
   uint64_t* kv_full = bar + 0;
-  uint64_t* qd_full = bar + 1;
-  uint64_t* s_full = bar + 2;
-  uint64_t* p_ready = bar + 3;
-  uint64_t* m_done = bar + 4;
-  uint64_t* drain = bar + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* qd_full = bar + 1;   // [2]
+  uint64_t* s_full = bar + 3;
+  uint64_t* p_ready = bar + 4;
+  uint64_t* m_done = bar + 5;
+  uint64_t* drain = bar + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -135,7 +131,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(qd_full, 1);
+    mbar_init(&qd_full[0], 1);
+    mbar_init(&qd_full[1], 1);
     mbar_init(s_full, 1);
     mbar_init(p_ready, kThreads);
     mbar_init(m_done, 1);
@@ -163,8 +160,22 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t IDESC_KK = make_idesc_bf16(128, 128, false, false);   // S^T, dP^T
   constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);     // dV, dK
 
-  uint32_t issued = 0;   // Q/dO loads issued (thread 0)
+  // step it -> (query head, query block)
+  auto head_of = [&](int it) { return g * P.group + a0 + it / nqb; };
+  auto block_of = [&](int it) { return qb0 + it % nqb; };
+  uint32_t nq[2] = {0, 0};   // Q/dO loads issued per buffer (thread 0)
   bool any_mma = false;
+  auto load_qd = [&](int it) {
+    const int b = it & 1, j = head_of(it), jl = j - shard * P.qh;
+    const int q_col = shard * P.R_a + jl * HD, q0 = block_of(it) * kBlk;
+    mbar_arrive_expect_tx(&qd_full[b], 2 * L::BLOCK);
+#pragma unroll
+    for (int c = 0; c < L::SUB; ++c) {
+      tma_load_3d(&tma_qkv, &qd_full[b], sQ + b * L::BLOCK + c * L::TILE, q_col + 64 * c, q0, bi);
+      tma_load_3d(&tma_do, &qd_full[b], sDO + b * L::BLOCK + c * L::TILE, j * HD + 64 * c, q0, bi);
+    }
+    ++nq[b];
+  };
   if (tid == 0) {
     mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
 #pragma unroll
@@ -172,6 +183,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
       tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
     }
+    load_qd(0);
+    if (n_iter > 1) load_qd(1);
   }
   bool ok = true;
   for (int it = 0; it < n_iter; ++it) {
@@ -179,11 +192,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
       break;
     }
-    const int a = a0 + it / nqb, qb = qb0 + it % nqb;
-    const int j = g * P.group + a;
-    const int jl = j - shard * P.qh;
-    const int q_col = shard * P.R_a + jl * HD;
-    const int q0 = qb * kBlk;
+    const int b = it & 1;
+    const int j = head_of(it);
+    const int q0 = block_of(it) * kBlk;
     {
       const int t_abs = q0 + tid;
       const bool valid = t_abs < P.s;
@@ -193,22 +204,16 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     __syncthreads();
     if (tid == 0 && ok) {
-      if (it > 0) ok = wait(m_done, (it - 1) & 1, DEVERR_WAIT_ACC_EMPTY);   // Q, dO, P^T, dS^T free
-      if (ok) {
-        mbar_arrive_expect_tx(qd_full, 2 * L::BLOCK);
-#pragma unroll
-        for (int c = 0; c < L::SUB; ++c) {
-          tma_load_3d(&tma_qkv, qd_full, sQ + c * L::TILE, q_col + 64 * c, q0, bi);
-          tma_load_3d(&tma_do, qd_full, sDO + c * L::TILE, j * HD + 64 * c, q0, bi);
-        }
-        ++issued;
-        ok = wait(qd_full, it & 1, DEVERR_WAIT_FULL) &&
-             (it > 0 || wait(kv_full, 0, DEVERR_WAIT_FULL));
-      }
+      // S^T and dP^T overwrite P^T, dS^T of the previous step: wait for its MMAs (which also
+      // frees the other Q/dO buffer for the step after this one)
+      if (it > 0) ok = wait(m_done, (it - 1) & 1, DEVERR_WAIT_ACC_EMPTY);
+      if (ok && it >= 1 && it + 1 < n_iter) load_qd(it + 1);
+      if (ok) ok = wait(&qd_full[b], (it >> 1) & 1, DEVERR_WAIT_FULL) &&
+                   (it > 0 || wait(kv_full, 0, DEVERR_WAIT_FULL));
       if (ok) {
         tc_fence_after();
-        const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ),
-                       da = smem_addr(sDO);
+        const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ + b * L::BLOCK),
+                       da = smem_addr(sDO + b * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
@@ -221,7 +226,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         any_mma = true;
       }
     }
-    // ---- P^T and dS^T for this key row against the block's 128 queries
+    // ---- P^T and dS^T for this key row against the block's 128 queries, written as bf16 over
+    // the first half of their own TMEM columns (chunks in ascending order: a chunk's S and dP
+    // are read before any later chunk's columns are overwritten)
     ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
     if (ok) {
       tc_fence_after();
@@ -244,10 +251,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        st_kmajor32(sPT, L::TILE, row, c0, pw);
-        st_kmajor32(sDST, L::TILE, row, c0, dw);
+        st16(tS + lane_base + c0 / 2, pw);
+        st16(tdP + lane_base + c0 / 2, dw);
       }
-      fence_async_smem();
+      fa::tmem_wait_st();
     }
     tc_fence_before();
     mbar_arrive(p_ready);
@@ -255,18 +262,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait(p_ready, it & 1, DEVERR_WAIT_ACC_FULL);
       if (ok) {
         tc_fence_after();
-        const uint32_t pa = smem_addr(sPT), sa = smem_addr(sDST), qa = smem_addr(sQ),
-                       da = smem_addr(sDO);
+        const uint32_t qa = smem_addr(sQ + b * L::BLOCK), da = smem_addr(sDO + b * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          const uint32_t aoff = (kk >> 2) * L::TILE + (kk & 3) * 32;
-          // B: the [query][dim] tiles read MN-major (N = dim), 16 query rows per MMA
-          umma_f16(tdV, make_sdesc_sw128(pa + aoff, 16, 1024),
-                   make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                   (it > 0 || kk > 0) ? 1u : 0u);
-          umma_f16(tdK, make_sdesc_sw128(sa + aoff, 16, 1024),
-                   make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                   (it > 0 || kk > 0) ? 1u : 0u);
+          // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
+          // MN-major (N = dim), 16 query rows per MMA
+          fa::umma_f16_tmem_a(tdV, tS + kk * 8, make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024),
+                              IDESC_KN, (it > 0 || kk > 0) ? 1u : 0u);
+          fa::umma_f16_tmem_a(tdK, tdP + kk * 8, make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024),
+                              IDESC_KN, (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
       }
@@ -314,7 +318,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_flag && tid == 0) {
     const Drain dr{globaltimer_ns(), P.err};
     dr(kv_full, 0);
-    if (issued) dr(qd_full, (issued - 1) & 1);
+    for (int b = 0; b < 2; ++b)
+      if (nq[b]) dr(&qd_full[b], (nq[b] - 1) & 1);
     if (any_mma) {
       umma_commit(drain);
       dr(drain, 0);
@@ -338,17 +343,16 @@ __global__ void __launch_bounds__(kThreads, 1)
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sQ = smem;
   uint8_t* sDO = sQ + L::BLOCK;
-  uint8_t* sK = sDO + L::BLOCK;
-  uint8_t* sV = sK + L::BLOCK;
-  uint8_t* sDS = sV + L::BLOCK;      // dS [query][key], K-major (K = key)
-  uint64_t* bar = reinterpret_cast<uint64_t*>(sDS + L::PTILE);
+  uint8_t* sK = sDO + L::BLOCK;      // [2] buffers
+  uint8_t* sV = sK + 2 * L::BLOCK;   // [2] buffers
+  uint64_t* bar = reinterpret_cast<uint64_t*>(sV + 2 * L::BLOCK);
   uint64_t* qd_full = bar + 0;
-  uint64_t* kv_full = bar + 1;
-  uint64_t* s_full = bar + 2;
-  uint64_t* p_ready = bar + 3;
-  uint64_t* m_done = bar + 4;
-  uint64_t* drain = bar + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* kv_full = bar + 1;       // [2]
+  uint64_t* s_full = bar + 3;
+  uint64_t* p_ready = bar + 4;
+  uint64_t* m_done = bar + 5;
+  uint64_t* drain = bar + 6;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 7);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -364,7 +368,8 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (tid == 0) {
     mbar_init(qd_full, 1);
-    mbar_init(kv_full, 1);
+    mbar_init(&kv_full[0], 1);
+    mbar_init(&kv_full[1], 1);
     mbar_init(s_full, 1);
     mbar_init(p_ready, kThreads);
     mbar_init(m_done, 1);
@@ -396,8 +401,20 @@ __global__ void __launch_bounds__(kThreads, 1)
   constexpr uint32_t IDESC_KK = make_idesc_bf16(128, 128, false, false);   // S, dP
   constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);     // dQ
 
-  uint32_t issued = 0;   // K/V loads issued (thread 0)
+  uint32_t nk[2] = {0, 0};   // K/V loads issued per buffer (thread 0)
   bool any_mma = false;
+  auto load_kv = [&](int kb) {
+    const int b = kb & 1;
+    mbar_arrive_expect_tx(&kv_full[b], 2 * L::BLOCK);
+#pragma unroll
+    for (int c = 0; c < L::SUB; ++c) {
+      tma_load_3d(&tma_qkv, &kv_full[b], sK + b * L::BLOCK + c * L::TILE, k_col + 64 * c,
+                  kb * kBlk, bi);
+      tma_load_3d(&tma_qkv, &kv_full[b], sV + b * L::BLOCK + c * L::TILE, v_col + 64 * c,
+                  kb * kBlk, bi);
+    }
+    ++nk[b];
+  };
   if (tid == 0) {
     mbar_arrive_expect_tx(qd_full, 2 * L::BLOCK);
 #pragma unroll
@@ -405,6 +422,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       tma_load_3d(&tma_qkv, qd_full, sQ + c * L::TILE, q_col + 64 * c, q0, bi);
       tma_load_3d(&tma_do, qd_full, sDO + c * L::TILE, j * HD + 64 * c, q0, bi);
     }
+    load_kv(0);
+    if (nkb > 1) load_kv(1);
   }
   bool ok = true;
   for (int kb = 0; kb < nkb; ++kb) {
@@ -412,24 +431,19 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = false;
       break;
     }
+    const int b = kb & 1;
     const int k0 = kb * kBlk;
     if (tid == 0 && ok) {
-      if (kb > 0) ok = wait(m_done, (kb - 1) & 1, DEVERR_WAIT_ACC_EMPTY);   // K, V, dS free
-      if (ok) {
-        mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
-#pragma unroll
-        for (int c = 0; c < L::SUB; ++c) {
-          tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
-          tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
-        }
-        ++issued;
-        ok = wait(kv_full, kb & 1, DEVERR_WAIT_FULL) &&
-             (kb > 0 || wait(qd_full, 0, DEVERR_WAIT_FULL));
-      }
+      // S and dP overwrite dS of the previous step: wait for its MMA (which also frees the
+      // other K/V buffer for the step after this one)
+      if (kb > 0) ok = wait(m_done, (kb - 1) & 1, DEVERR_WAIT_ACC_EMPTY);
+      if (ok && kb >= 1 && kb + 1 < nkb) load_kv(kb + 1);
+      if (ok) ok = wait(&kv_full[b], (kb >> 1) & 1, DEVERR_WAIT_FULL) &&
+                   (kb > 0 || wait(qd_full, 0, DEVERR_WAIT_FULL));
       if (ok) {
         tc_fence_after();
-        const uint32_t qa = smem_addr(sQ), da = smem_addr(sDO), ka = smem_addr(sK),
-                       va = smem_addr(sV);
+        const uint32_t qa = smem_addr(sQ), da = smem_addr(sDO), ka = smem_addr(sK + b * L::BLOCK),
+                       va = smem_addr(sV + b * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < HD / 16; ++kk) {
           const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
@@ -442,6 +456,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         any_mma = true;
       }
     }
+    // ---- dS for this query row against the block's 128 keys, bf16 over the first half of the
+    // S columns (ascending chunks: a chunk is read before any later chunk is overwritten)
     ok = __all_sync(0xffffffffu, ok && wait(s_full, kb & 1, DEVERR_WAIT_ACC_FULL));
     if (ok) {
       tc_fence_after();
@@ -463,9 +479,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        st_kmajor32(sDS, L::TILE, row, c0, dw);
+        st16(tS + lane_base + c0 / 2, dw);
       }
-      fence_async_smem();
+      fa::tmem_wait_st();
     }
     tc_fence_before();
     mbar_arrive(p_ready);
@@ -473,13 +489,12 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait(p_ready, kb & 1, DEVERR_WAIT_ACC_FULL);
       if (ok) {
         tc_fence_after();
-        const uint32_t sa = smem_addr(sDS), ka = smem_addr(sK);
+        const uint32_t ka = smem_addr(sK + b * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
-          // B: the [key][dim] K tile read MN-major (N = dim), 16 key rows per MMA
-          umma_f16(tdQ, make_sdesc_sw128(sa + (kk >> 2) * L::TILE + (kk & 3) * 32, 16, 1024),
-                   make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                   (kb > 0 || kk > 0) ? 1u : 0u);
+          // A: 16 keys = 8 TMEM columns of dS; B: the [key][dim] K tile read MN-major
+          fa::umma_f16_tmem_a(tdQ, tS + kk * 8, make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024),
+                              IDESC_KN, (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
       }
@@ -503,7 +518,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (*abort_flag && tid == 0) {
     const Drain dr{globaltimer_ns(), P.err};
     dr(qd_full, 0);
-    if (issued) dr(kv_full, (issued - 1) & 1);
+    for (int b = 0; b < 2; ++b)
+      if (nk[b]) dr(&kv_full[b], (nk[b] - 1) & 1);
     if (any_mma) {
       umma_commit(drain);
       dr(drain, 0);
@@ -544,14 +560,15 @@ __global__ void __launch_bounds__(256) combine_kv_kernel(const float* part, int 
 }
 
 template <int HD>
-constexpr int dkv_smem() { return 4 * Tiles<HD>::BLOCK + 2 * Tiles<HD>::PTILE + 2 * kBlk * 4 + 128 + 1024; }
+constexpr int dkv_smem() { return 6 * Tiles<HD>::BLOCK + 2 * kBlk * 4 + 128 + 1024; }
 // at least 120 KB, so that no second CTA (which would wait for the 512 TMEM columns) shares an SM
 template <int HD>
 constexpr int dq_smem() {
-  return 4 * Tiles<HD>::BLOCK + Tiles<HD>::PTILE + 128 + 1024 > 120 * 1024
-             ? 4 * Tiles<HD>::BLOCK + Tiles<HD>::PTILE + 128 + 1024
-             : 120 * 1024;
+  return 6 * Tiles<HD>::BLOCK + 128 + 1024 > 120 * 1024 ? 6 * Tiles<HD>::BLOCK + 128 + 1024
+                                                         : 120 * 1024;
 }
+template <int HD>
+constexpr int dkv_smem_padded() { return dkv_smem<HD>() > 120 * 1024 ? dkv_smem<HD>() : 120 * 1024; }
 
 // Host launcher.  qkv and dqkv [b][s][p*R_a] bf16 (packed per shard: Q heads, K heads, V heads),
 // dO [b][s][n_q*HD] bf16, lse and D [b*s][n_q] fp32.
@@ -574,7 +591,7 @@ inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, c
   TP_CUDA_TRY(cudaGetDevice(&dev));
   if (dev < 64 && !attr_set[dev]) {
     TP_CUDA_TRY(cudaFuncSetAttribute(flash_bwd_dkv_kernel<HD>,
-                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dkv_smem<HD>()));
+                                     cudaFuncAttributeMaxDynamicSharedMemorySize, dkv_smem_padded<HD>()));
     TP_CUDA_TRY(cudaFuncSetAttribute(flash_bwd_dq_kernel<HD>,
                                      cudaFuncAttributeMaxDynamicSharedMemorySize, dq_smem<HD>()));
     attr_set[dev] = 1;
@@ -600,7 +617,7 @@ inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, c
   ProfScope prof(st, "attn_bwd_flash");
   flash_bwd_dkv_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk),
                                   static_cast<unsigned>(n_kv * P.split), static_cast<unsigned>(b)),
-                             kThreads, dkv_smem<HD>(), st>>>(mq, md, P);
+                             kThreads, dkv_smem_padded<HD>(), st>>>(mq, md, P);
   TP_LAUNCH_CHECK();
   if (P.split > 1) {
     const int64_t n_tok = b * s;
