@@ -353,6 +353,8 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     ex = {}
     which = set(args.extras.split(","))
     steps = max(3, min(args.steps, args.extra_steps))
+    if "tiny" in which:
+        ex["tiny_mlp"] = extra_tiny(tp, inputs, torch, stream)
     # lightest first, with a short idle gap between workloads, so that no extra is timed at the
     # power-capped clocks a previous seconds-long tensor-core run leaves behind
     if "stack" in which:
@@ -367,6 +369,33 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     if "prefill" in which:
         ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
     return ex
+
+
+def extra_tiny(tp, inputs, torch, stream, calls=2000):
+    """The tiny configuration (T=4, d=8, d_ff=32, p=4, GELU, fp32): launch-latency bound, so it
+    is reported as microseconds per forward call (every call enqueues the up GEMM, the partial
+    GEMM and the reduce)."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    inp = inputs.mlp_inputs(4, 8, 32, "gelu", "f32", seed=0, device=dev)
+    d = tp.mlp_desc(4, 8, 32, 4, "gelu", "f32")
+    w1p = torch.empty(tp.tp_mlp_w1_packed_bytes(d) // 4, dtype=torch.float32, device=dev)
+    w2p = torch.empty(tp.tp_mlp_w2_packed_bytes(d) // 4, dtype=torch.float32, device=dev)
+    tp.tp_mlp_pack(d, inp["w1"], None, inp["w2"], w1p, w2p)
+    ws = torch.empty(tp.tp_mlp_fwd_workspace(d), dtype=torch.uint8, device=dev)
+    y = torch.empty(4, 8, dtype=torch.float32, device=dev)
+
+    def fwd():
+        tp.tp_mlp_fwd(d, inp["x"], w1p, w2p, y, workspace=ws)
+
+    for _ in range(20):
+        fwd()
+    ms = _cuda_time(fwd, calls, stream)
+    l0 = tp.tp_launch_count()
+    fwd()
+    launches = tp.tp_launch_count() - l0
+    return {"workload": "tiny MLP: T=4, d=8, d_ff=32, p=4 logical shards, GELU, fp32",
+            "us_per_call": round(ms / calls * 1e3, 2), "launches_per_call": int(launches),
+            "calls": calls}
 
 
 def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
@@ -615,7 +644,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=20)
-    ap.add_argument("--extras", default="prefill,attention,stack",
+    ap.add_argument("--extras", default="tiny,prefill,attention,stack",
                     help="comma list of extra workloads to measure at N=1")
     ap.add_argument("--reduce-mode", choices=["separate", "fused"], default="separate",
                     help="how the p partial sums are added in the decode workloads")
