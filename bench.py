@@ -279,6 +279,20 @@ def run_ours(args, dist):
     ms_step = ms / args.steps
     tokens = c["T"] * args.steps * dist.world
 
+    # distribution of single-step times (one event pair per step, 200 steps at most)
+    n_q = min(args.steps, 200)
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+           for _ in range(n_q)]
+    for a_ev, b_ev in evs:
+        a_ev.record(stream)
+        step()
+        b_ev.record(stream)
+    torch.cuda.synchronize()
+    one = sorted(a_ev.elapsed_time(b_ev) for a_ev, b_ev in evs)
+    step_quantiles = {"p10": round(one[int(0.1 * (n_q - 1))], 5),
+                      "p50": round(one[int(0.5 * (n_q - 1))], 5),
+                      "p90": round(one[int(0.9 * (n_q - 1))], 5), "steps": n_q}
+
     # per-kernel durations, measured with events on the launching stream over K more steps
     prof = _profile(tp, step, args.steps)
     nbytes = decode_mlp_bytes()
@@ -331,6 +345,7 @@ def run_ours(args, dist):
                    "l2": "inputs larger than L2: 1.41 GB of weights streamed per step",
                    "step_GB_per_s": round(step_gbs, 1),
                    "step_frac_of_hbm": round(step_gbs / peaks["hbm_gbs"], 4)},
+        "step_ms_quantiles": step_quantiles,
         "roofline": roofline, "e2e": e2e, "gpu_launches": int(launches), "clocks": clocks,
         "kernels": kernels,
     }

@@ -24,6 +24,8 @@ def _grads_ref(inp, dy, n_q, n_kv, hd, causal):
     (1, 130, 192, 4, 4, 64, 4),     # MHA, flash forward (head_dim 64), two query tiles
     (1, 200, 512, 8, 2, 128, 1),    # one shard, flash forward (head_dim 128), 200 tokens
     (3, 9, 64, 8, 8, 8, 8),         # tiny head_dim, p = n_kv
+    (2, 150, 256, 4, 2, 128, 2),    # tcgen05 backward, two sequences, ragged second block
+    (3, 70, 256, 8, 2, 64, 1),      # tcgen05 backward (head_dim 64), three short sequences
 ])
 def test_backward_parity(lib, causal, b, s, h, n_q, n_kv, hd, p):
     inp = inputs.attn_inputs(b, s, h, n_q, n_kv, hd, "bf16", seed=31, w_std=0.05)
