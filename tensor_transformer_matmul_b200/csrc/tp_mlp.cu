@@ -13,6 +13,7 @@
 #include <algorithm>
 
 #include "gemm_launch.cuh"
+#include "gemm_pair.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
 #include "simt.cuh"
@@ -40,6 +41,9 @@ struct MlpLayout {
 };
 
 template <class C> struct Tag { using type = C; };
+// 256 x 256 tiles on SM pairs (cta_group::2): the prefill and backward GEMMs
+template <bool A_MN, bool B_MN>
+using PP = tc::PairCfg<A_MN, B_MN, 6>;
 template <int BN, int ASUB>
 using KK = TileCfg<BN, ASUB, false, false, stages_for(BN, ASUB)>;
 
@@ -169,7 +173,8 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
     return L.act == TP_ACT_SWIGLU ? by_tokens<2>(L.T, f) : by_tokens<1>(L.T, f);
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s, "mlp_up_gemm");
+  return tc::run_gemm_pair<PP<false, false>, tc::EpiHidden>(xo, wo, L.T, rows, L.d, 1, ep, s,
+                                                            "mlp_up_gemm");
 }
 
 // Row-parallel down projection.  Separate reduce: partial[i] = h_i W2_i (fp32, [p][T][d]).
@@ -218,7 +223,8 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
     });
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s, "mlp_down_gemm");
+  return tc::run_gemm_pair<PP<false, false>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s,
+                                                              "mlp_down_gemm");
 }
 
 tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
@@ -238,8 +244,8 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.tokens = static_cast<int32_t>(L.T);
     ep.act = L.act;
     if (L.Fsp % 256 == 0)
-      st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiActBwd>(
-          a, b, L.T, L.Fsp, L.d, P, ep, s, "mlp_dh_gemm");
+      st = tc::run_gemm_pair<PP<false, true>, tc::EpiActBwd>(a, b, L.T, L.Fsp, L.d, P, ep, s,
+                                                             "mlp_dh_gemm");
     else
       st = tc::run_gemm<TileCfg<128, 1, false, true, stages_for(128, 1)>, tc::EpiActBwd>(
           a, b, L.T, L.Fsp, L.d, P, ep, s, "mlp_dh_gemm");
@@ -257,8 +263,8 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.cols_valid = static_cast<int32_t>(L.Fsp);
     ep.swap = 0;
     if (L.Fsp % 256 == 0)
-      st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-          a, b, L.d, L.Fsp, L.T, P, ep, s, "mlp_dw2_gemm");
+      st = tc::run_gemm_pair<PP<true, true>, tc::EpiStoreF32>(a, b, L.d, L.Fsp, L.T, P, ep, s,
+                                                              "mlp_dw2_gemm");
     else
       st = tc::run_gemm<TileCfg<128, 1, true, true, stages_for(128, 1)>, tc::EpiStoreF32>(
           a, b, L.d, L.Fsp, L.T, P, ep, s, "mlp_dw2_gemm");
@@ -275,8 +281,8 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.rows_valid = static_cast<int32_t>(L.R);
     ep.cols_valid = static_cast<int32_t>(L.d);
     ep.swap = 0;
-    st = tc::run_gemm<TileCfg<256, 1, true, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-        a, b, L.R, L.d, L.T, P, ep, s, "mlp_dw1_gemm");
+    st = tc::run_gemm_pair<PP<true, true>, tc::EpiStoreF32>(a, b, L.R, L.d, L.T, P, ep, s,
+                                                            "mlp_dw1_gemm");
     if (st != TP_OK) return st;
   }
   // (4) dx_i = dz_i W1_i^T  (partials, summed by the caller)
@@ -290,8 +296,8 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
     ep.rows_valid = static_cast<int32_t>(L.T);
     ep.cols_valid = static_cast<int32_t>(L.d);
     ep.swap = 0;
-    st = tc::run_gemm<TileCfg<256, 1, false, true, stages_for(256, 1)>, tc::EpiStoreF32>(
-        a, b, L.T, L.d, L.R, P, ep, s, "mlp_dx_gemm");
+    st = tc::run_gemm_pair<PP<false, true>, tc::EpiStoreF32>(a, b, L.T, L.d, L.R, P, ep, s,
+                                                             "mlp_dx_gemm");
   }
   return st;
 }

@@ -87,6 +87,27 @@ def test_backward_parity(lib, act, dtype, T):
         assert rel_l2(f64(dwu), ref["dw_up"]) <= tol
 
 
+@pytest.mark.parametrize("act", ["swiglu", "gelu"])
+def test_pair_tiles_forward_backward(lib, act):
+    # the prefill and backward GEMMs run 256 x 256 tiles on SM pairs: T = 520 gives three token
+    # tiles (the last one ragged, its second half empty), d = 776 a ragged K and N, F_s = 512 two
+    # feature tiles per shard; every GEMM of forward and backward has several tiles per dimension
+    T, d, F, p = 520, 776, 1536, 3
+    inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=11, w_std=0.05, backward=True)
+    m = Mlp(lib, inp, p, act, "bf16")
+    y = m.forward(inp["x"])
+    dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
+    torch.cuda.synchronize()
+    wu = None if inp["w_up"] is None else f64(inp["w_up"])
+    assert rel_l2(f64(y), _oracle_fwd(inp, act)) <= TOL["bf16"]
+    ref = omlp.mlp_backward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), f64(inp["dy"]), act, wu)
+    assert rel_l2(f64(dx), ref["dx"]) <= TOL["bf16"]
+    assert rel_l2(f64(dw1), ref["dw1"]) <= TOL["bf16"]
+    assert rel_l2(f64(dw2), ref["dw2"]) <= TOL["bf16"]
+    if act == "swiglu":
+        assert rel_l2(f64(dwu), ref["dw_up"]) <= TOL["bf16"]
+
+
 def test_backward_padding_gradients_are_zero(lib):
     # F_s = 136 pads to 256 per shard: the padding rows of the packed gradient must be exactly 0
     d, F, p, T = 64, 408, 3, 40
