@@ -454,8 +454,19 @@ def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
 
 def extra_prefill(tp, inputs, torch, stream, peaks, steps):
     # prefill SwiGLU MLP forward + backward: 6 T d F flops per direction pair x 3 matmuls
+    res = _prefill_mode(tp, inputs, torch, stream, peaks, steps, tp.TP_REDUCE_SEPARATE)
+    fused = _prefill_mode(tp, inputs, torch, stream, peaks, steps, tp.TP_REDUCE_FUSED)
+    res["reduce_fused"] = {k: fused[k] for k in ("ms_fwd", "ms_bwd", "TFLOP_per_s",
+                                                  "frac_of_burst_peak", "frac_of_sustained_peak",
+                                                  "tokens_per_s", "kernels")}
+    return res
+
+
+def _prefill_mode(tp, inputs, torch, stream, peaks, steps, mode):
+    """The prefill step with the shard partials summed by a separate reduce (TP_REDUCE_SEPARATE)
+    or inside the down and dx GEMMs' accumulators (TP_REDUCE_FUSED)."""
     c = PREFILL
-    st = setup_mlp(tp, inputs, torch, c, backward=True)
+    st = setup_mlp(tp, inputs, torch, c, backward=True, reduce_mode=mode)
 
     def fwd():
         tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], saved=st["saved"],
@@ -512,18 +523,26 @@ def extra_attention(tp, inputs, torch, stream, peaks, steps):
     ai = inputs.attn_inputs(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], "bf16", seed=0,
                             device=dev)
     ad = tp.attn_desc(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], a["p"])
+    adf = tp.attn_desc(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], a["p"],
+                       reduce_mode=tp.TP_REDUCE_FUSED)
     wqkv = torch.empty(tp.tp_attn_wqkv_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
     wo = torch.empty(tp.tp_attn_wo_packed_bytes(ad) // 2, dtype=torch.bfloat16, device=dev)
     tp.tp_attn_pack(ad, ai["wq"], ai["wk"], ai["wv"], ai["wo"], wqkv, wo)
     ya = torch.empty_like(ai["x"])
-    wsa = torch.empty(tp.tp_attn_fwd_workspace(ad), dtype=torch.uint8, device=dev)
+    wsa = torch.empty(max(tp.tp_attn_fwd_workspace(ad), tp.tp_attn_fwd_workspace(adf)),
+                      dtype=torch.uint8, device=dev)
 
     def attn():
         tp.tp_attn_fwd(ad, ai["x"], wqkv, wo, ya, workspace=wsa)
 
+    def attn_fused():
+        tp.tp_attn_fwd(adf, ai["x"], wqkv, wo, ya, workspace=wsa)
+
     for _ in range(3):
         attn()
+        attn_fused()
     ms_a = _cuda_time(attn, steps, stream) / steps
+    ms_af = _cuda_time(attn_fused, steps, stream) / steps
     s, h = a["s"], a["h"]
     fl_qkv = 2.0 * s * h * (a["n_q"] + 2 * a["n_kv"]) * a["hd"]
     fl_att = 2.0 * 2 * a["n_q"] * a["hd"] * s * (s + 1) / 2
@@ -536,6 +555,10 @@ def extra_attention(tp, inputs, torch, stream, peaks, steps):
         "frac_of_burst_peak": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "tokens_per_s": round(s / (ms_a / 1e3), 1),
         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
+        "reduce_fused": {"ms": round(ms_af, 3),
+                         "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_af / 1e3) / 1e12, 1),
+                         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)}
+                                     for k, v in _profile(tp, attn_fused, steps).items()}},
         "steps": steps}
 
 
@@ -554,14 +577,22 @@ def extra_attention_bwd(tp, inputs, torch, stream, peaks, steps):
     dx = torch.empty_like(ai["x"])
     dwqkv = torch.empty(wqkv.numel(), dtype=torch.float32, device=dev)
     dwo = torch.empty(wo.numel(), dtype=torch.float32, device=dev)
-    ws = torch.empty(tp.tp_attn_bwd_workspace(ad), dtype=torch.uint8, device=dev)
+    adf = tp.attn_desc(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], a["p"],
+                       reduce_mode=tp.TP_REDUCE_FUSED)
+    ws = torch.empty(max(tp.tp_attn_bwd_workspace(ad), tp.tp_attn_bwd_workspace(adf)),
+                     dtype=torch.uint8, device=dev)
 
     def bwd():
         tp.tp_attn_bwd(ad, ai["x"], wqkv, wo, dy, dx, dwqkv, dwo, workspace=ws)
 
+    def bwd_fused():
+        tp.tp_attn_bwd(adf, ai["x"], wqkv, wo, dy, dx, dwqkv, dwo, workspace=ws)
+
     for _ in range(3):
         bwd()
+        bwd_fused()
     ms = _cuda_time(bwd, steps, stream) / steps
+    ms_f = _cuda_time(bwd_fused, steps, stream) / steps
     s, h = a["s"], a["h"]
     rqkv = (a["n_q"] + 2 * a["n_kv"]) * a["hd"]
     fl_proj = 2.0 * s * h * rqkv            # one projection-sized GEMM (QKV)
@@ -578,6 +609,8 @@ def extra_attention_bwd(tp, inputs, torch, stream, peaks, steps):
         "TFLOP_per_s": round(flops / (ms / 1e3) / 1e12, 1),
         "frac_of_burst_peak": round(flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
+        "reduce_fused": {"ms": round(ms_f, 3),
+                         "TFLOP_per_s": round(flops / (ms_f / 1e3) / 1e12, 1)},
         "steps": steps}
 
 

@@ -61,8 +61,12 @@ typedef enum { TP_ACT_IDENTITY = 0, TP_ACT_RELU = 1, TP_ACT_GELU = 2, TP_ACT_SWI
 /* How the p partial sums are added ("One collective").
  *   TP_REDUCE_SEPARATE: each shard's partial goes to fp32 workspace, then one vectorised
  *                       reduce kernel adds them (order 0..p-1) and rounds once.
- *   TP_REDUCE_FUSED:    the down-projection kernel adds the p shard partials of its output tile
- *                       in the same order without writing them to memory.                      */
+ *   TP_REDUCE_FUSED:    the row-parallel GEMM adds the p shard partials of its output tile
+ *                       in the same order without writing them to memory: for up to 128
+ *                       tokens by a stream-K split over the shards' k-blocks, for more tokens
+ *                       by running shard 0, 1, ..., p-1's k-blocks into one fp32 accumulator.
+ *                       It applies to the forward's down / output projection and to the
+ *                       backward's dx GEMM (tp_mlp_bwd, tp_attn_bwd).                          */
 typedef enum { TP_REDUCE_SEPARATE = 0, TP_REDUCE_FUSED = 1 } tp_reduce_mode;
 
 /* Descriptor flags.

@@ -6,6 +6,7 @@
 
 #include "flash_attn.cuh"
 #include "gemm_launch.cuh"
+#include "gemm_pair.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
 #include "simt.cuh"
@@ -33,6 +34,9 @@ template <int BN, int ASUB>
 using KK = tc::TileCfg<BN, ASUB, false, false,
                        std::min(8, (200 * 1024) / (128 * ASUB * 64 * 2 + BN * 64 * 2))>;
 template <class C> struct Tag { using type = C; };
+// 256 x 256 tiles on SM pairs (cta_group::2): the prefill and backward projections
+template <bool A_MN, bool B_MN>
+using PP = tc::PairCfg<A_MN, B_MN, 6>;
 constexpr int64_t kSwapMaxT = 128;
 template <class F>
 auto by_tokens(int64_t T, F&& f) {
@@ -59,8 +63,6 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
     if (decode_stream_k(out_tiles(L)) || fused) b = by_tokens(L.tokens, [&](auto t) {
       return tc::plan_stream_k<typename decltype(t)::type>(L.h, L.tokens, K, L.p, fused, num_sms()).bytes();
     });
-  } else if (fused) {
-    b = tc::plan_stream_k<KK<256, 1>>(L.tokens, L.h, K, L.p, true, num_sms()).bytes();
   }
   return std::max(a, b);
 }
@@ -593,7 +595,8 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
     });
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s, "attn_qkv_gemm");
+  return tc::run_gemm_pair<PP<false, false>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s,
+                                                            "attn_qkv_gemm");
 }
 
 // Row-parallel output projection: fp32 partials [p][tokens][h] (separate reduce), or the fused
@@ -623,8 +626,10 @@ inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, 
         return tc::run_gemm<typename decltype(t)::type, tc::EpiReduceOut>(
             wo, ao, L.h, L.tokens, K, L.p, ep, s, "attn_out_gemm", opt);
       });
-    return tc::run_gemm<KK<256, 1>, tc::EpiReduceOut>(ao, wo, L.tokens, L.h, K, L.p, ep, s,
-                                                       "attn_out_gemm", opt);
+    // prefill: each 256 x 256 tile runs the k-blocks of shard 0, 1, ..., p-1 into one
+    // accumulator, so the shard sum never leaves TMEM
+    return tc::run_gemm_pair<PP<false, false>, tc::EpiReduceOut>(ao, wo, L.tokens, L.h, K, L.p, ep,
+                                                                 s, "attn_out_gemm", -1, true);
   }
   tc::EpiStoreF32::Params ep;
   ep.out = part;
@@ -644,7 +649,8 @@ inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, 
     });
   }
   ep.swap = 0;
-  return tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s, "attn_out_gemm");
+  return tc::run_gemm_pair<PP<false, false>, tc::EpiStoreF32>(ao, wo, L.tokens, L.h, K, L.p, ep, s,
+                                                              "attn_out_gemm");
 }
 }  // namespace attn_tc
 

@@ -228,7 +228,7 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
     ep.rows_valid = static_cast<int32_t>(T);
     ep.cols_valid = static_cast<int32_t>(K);
     st = K % 256 == 0
-             ? tc::run_gemm<TileCfg<256, 1, false, true, 4>, tc::EpiStoreBf16>(
+             ? tc::run_gemm_pair<attn_tc::PP<false, true>, tc::EpiStoreBf16>(
                    a, bo, T, K, L.h, P, ep, s, "attn_do_gemm")
              : tc::run_gemm<TileCfg<128, 1, false, true, 6>, tc::EpiStoreBf16>(
                    a, bo, T, K, L.h, P, ep, s, "attn_do_gemm");
@@ -246,7 +246,7 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
     ep.cols_valid = static_cast<int32_t>(K);
     ep.swap = 0;
     st = K % 256 == 0
-             ? tc::run_gemm<TileCfg<256, 1, true, true, 4>, tc::EpiStoreF32>(
+             ? tc::run_gemm_pair<attn_tc::PP<true, true>, tc::EpiStoreF32>(
                    a, bo, L.h, K, T, P, ep, s, "attn_dwo_gemm")
              : tc::run_gemm<TileCfg<128, 1, true, true, 6>, tc::EpiStoreF32>(
                    a, bo, L.h, K, T, P, ep, s, "attn_dwo_gemm");
@@ -300,14 +300,27 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
     ep.rows_valid = static_cast<int32_t>(L.R_a);
     ep.cols_valid = static_cast<int32_t>(L.h);
     ep.swap = 0;
-    st = tc::run_gemm<TileCfg<256, 1, true, true, 4>, tc::EpiStoreF32>(
+    st = tc::run_gemm_pair<attn_tc::PP<true, true>, tc::EpiStoreF32>(
         a, bx, L.R_a, L.h, T, P, ep, s, "attn_dwqkv_gemm");
     if (st != TP_OK) return st;
   }
-  // dx_i = dqkv_i Wqkv_i (partials), then dx = sum_i dx_i in shard order
+  // dx_i = dqkv_i Wqkv_i (partials), then dx = sum_i dx_i in shard order; with
+  // TP_REDUCE_FUSED the GEMM adds the shards in its accumulator and writes dx itself
   {
     const Operand a{dqkv, false, T, L.R_a, P, P * L.R_a, L.R_a};
     const Operand bw{wqkv, true, L.h, L.R_a, P, L.h, L.R_a * L.h};
+    if (L.reduce_mode == TP_REDUCE_FUSED) {
+      tc::EpiReduceOut::Params ep;
+      ep.out = dx;
+      ep.residual = nullptr;
+      ep.ld = L.h;
+      ep.rows_valid = static_cast<int32_t>(T);
+      ep.cols_valid = static_cast<int32_t>(L.h);
+      ep.out_bf16 = 1;
+      ep.swap = 0;
+      return tc::run_gemm_pair<attn_tc::PP<false, true>, tc::EpiReduceOut>(
+          a, bw, T, L.h, L.R_a, P, ep, s, "attn_dx_gemm", -1, true);
+    }
     tc::EpiStoreF32::Params ep;
     ep.out = part;
     ep.ld = L.h;
@@ -315,7 +328,7 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
     ep.rows_valid = static_cast<int32_t>(T);
     ep.cols_valid = static_cast<int32_t>(L.h);
     ep.swap = 0;
-    st = tc::run_gemm<TileCfg<256, 1, false, true, 4>, tc::EpiStoreF32>(
+    st = tc::run_gemm_pair<attn_tc::PP<false, true>, tc::EpiStoreF32>(
         a, bw, T, L.h, L.R_a, P, ep, s, "attn_dx_gemm");
     if (st != TP_OK) return st;
   }

@@ -10,15 +10,20 @@
 // Two kernels, neither with atomics (each output tile is summed by one CTA in a fixed order):
 //   * dK/dV: one CTA per (128-key block, KV head, query head of its group, sequence).  It walks
 //     the query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in TMEM,
-//     the 128 threads (one key row each) turn them into P^T and dS^T, written back as bf16 over
-//     their own TMEM columns, and dV += P^T dO, dK += dS^T Q accumulate in TMEM with P^T and
-//     dS^T as the TMEM A operands (dO and Q read MN-major).  Q and dO are double buffered, so
-//     the next step's tiles load during this one.  The per-head shares are added afterwards.
+//     the 256 threads (one key row and one half of the 128 queries each) turn them into P^T and
+//     dS^T, written back as bf16 over their own TMEM columns, and dV += P^T dO, dK += dS^T Q
+//     accumulate in TMEM with P^T and dS^T as the TMEM A operands (dO and Q read MN-major).
+//     Q and dO are double buffered, so the next step's tiles load during this one.  The
+//     per-head shares are added afterwards.
 //   * dQ: one CTA per (128-query block, query head, sequence).  It walks the key blocks its
 //     queries see; per step S = Q K^T and dP = dO V^T land in TMEM, the threads (one query row
-//     each) write dS back over S, and dQ += dS K accumulates in TMEM (K read MN-major).  K and
-//     V are double buffered.
+//     and one half of the 128 keys each) write dS back over S, and dQ += dS K accumulates in
+//     TMEM (K read MN-major).  K and V are double buffered.
 // Thread 0 issues the TMA loads and the MMAs; TMEM holds four (three) 128-column fp32 tiles.
+// The two thread halves (warps 0-3 and 4-7) read the same TMEM lanes, columns 0-63 and 64-127;
+// half h packs its 64 bf16 results into columns 64 h .. 64 h + 31, which only it reads, so the
+// halves need no ordering between them.  The MMA that consumes them takes queries (keys)
+// 0-63 from columns 0-31 and 64-127 from columns 64-95.
 // Every wait is bounded; a timeout sets the abort flag, drains what was issued and leaves, and
 // the loop exit is CTA-uniform.
 #pragma once
@@ -34,7 +39,17 @@ namespace tp {
 namespace fb {
 
 constexpr int kBlk = 128;       // query rows and key rows per block
-constexpr int kThreads = 128;
+constexpr int kThreads = 256;   // two threads per row: each takes half of the block's columns
+
+// TMEM column (from the tile's start) of the packed bf16 pair holding columns 2i and 2i+1 of a
+// 128-column block: half h = i / 32 of the threads writes its 32 packed columns at 64 h
+__device__ __forceinline__ uint32_t packed_col(int i) {
+  return static_cast<uint32_t>(i + (i >> 5) * 32);
+}
+
+// 2^x with the MUFU approximation (flushes subnormal results to zero); the probabilities it
+// feeds are rounded to bf16 right after
+__device__ __forceinline__ float exp2_fast(float x) { return fa::ex2_approx(x); }
 
 struct Params {
   int32_t s;                    // tokens per sequence
@@ -151,8 +166,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const int row = tid;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int row = tid & (kBlk - 1);
+  const int half = tid >> 7;   // columns 64 half .. 64 half + 63
   const int k_abs = k0 + row;
   auto wait = [&](uint64_t* b, uint32_t par, uint32_t site) {
     return mbar_wait(b, par, abort_flag, P.err, site);
@@ -195,7 +211,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int b = it & 1;
     const int j = head_of(it);
     const int q0 = block_of(it) * kBlk;
-    {
+    if (tid < kBlk) {
       const int t_abs = q0 + tid;
       const bool valid = t_abs < P.s;
       const int64_t ri = (static_cast<int64_t>(bi) * P.s + t_abs) * P.n_q + j;
@@ -226,14 +242,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         any_mma = true;
       }
     }
-    // ---- P^T and dS^T for this key row against the block's 128 queries, written as bf16 over
-    // the first half of their own TMEM columns (chunks in ascending order: a chunk's S and dP
-    // are read before any later chunk's columns are overwritten)
+    // ---- P^T and dS^T for this key row against this thread's 64 of the block's queries,
+    // written as bf16 over the first half of this half's TMEM columns (chunks in ascending
+    // order: a chunk's S and dP are read before any later chunk's columns are overwritten)
     ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
     if (ok) {
       tc_fence_after();
+      // no mask inside the block: every query is valid and (causal) after every key
+      const bool plain = q0 + kBlk <= P.s && k0 + kBlk <= P.s && (!P.causal || q0 > k0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+      for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
         float sv[32], dp[32];
         ld32(tS + lane_base + c0, sv);
         ld32(tdP + lane_base + c0, dp);
@@ -243,16 +261,19 @@ __global__ void __launch_bounds__(kThreads, 1)
           float pr[2], ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int qi = c0 + e + u, q_abs = q0 + qi;
-            const bool masked = q_abs >= P.s || k_abs >= P.s || (P.causal && k_abs > q_abs);
-            pr[u] = masked ? 0.f : exp2f(sv[e + u] * P.scale_log2 - lse_s[qi]);
+            const int qi = c0 + e + u;
+            pr[u] = exp2_fast(sv[e + u] * P.scale_log2 - lse_s[qi]);
+            if (!plain) {
+              const int q_abs = q0 + qi;
+              if (q_abs >= P.s || k_abs >= P.s || (P.causal && k_abs > q_abs)) pr[u] = 0.f;
+            }
             ds[u] = pr[u] * (dp[e + u] - D_s[qi]);
           }
           pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        st16(tS + lane_base + c0 / 2, pw);
-        st16(tdP + lane_base + c0 / 2, dw);
+        st16(tS + lane_base + packed_col(c0 / 2), pw);
+        st16(tdP + lane_base + packed_col(c0 / 2), dw);
       }
       fa::tmem_wait_st();
     }
@@ -267,10 +288,12 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kk = 0; kk < kBlk / 16; ++kk) {
           // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
           // MN-major (N = dim), 16 query rows per MMA
-          fa::umma_f16_tmem_a(tdV, tS + kk * 8, make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024),
-                              IDESC_KN, (it > 0 || kk > 0) ? 1u : 0u);
-          fa::umma_f16_tmem_a(tdK, tdP + kk * 8, make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024),
-                              IDESC_KN, (it > 0 || kk > 0) ? 1u : 0u);
+          fa::umma_f16_tmem_a(tdV, tS + packed_col(kk * 8),
+                              make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                              (it > 0 || kk > 0) ? 1u : 0u);
+          fa::umma_f16_tmem_a(tdK, tdP + packed_col(kk * 8),
+                              make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                              (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
       }
@@ -288,7 +311,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     const int n_kv = static_cast<int>(gridDim.y) / P.split;
     float* prow = P.part_kv + ((static_cast<int64_t>(sp) * n_tok + t) * n_kv + g) * 2 * HD;
 #pragma unroll 1
-    for (int c = 0; c < HD; c += 32) {
+    for (int c = half * (HD / 2); c < (half + 1) * (HD / 2); c += 32) {
       float v[32];
       ld32(tdK + lane_base + c, v);
       if (P.split > 1) {
@@ -388,8 +411,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const uint32_t tS = tmem, tdP = tmem + 128, tdQ = tmem + 256;
-  const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
-  const int row = tid;
+  const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
+  const int row = tid & (kBlk - 1);
+  const int half = tid >> 7;   // columns 64 half .. 64 half + 63
   const int q_abs = q0 + row;
   const bool q_live = q_abs < P.s;
   const int64_t ri = (static_cast<int64_t>(bi) * P.s + q_abs) * P.n_q + j;
@@ -456,13 +480,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         any_mma = true;
       }
     }
-    // ---- dS for this query row against the block's 128 keys, bf16 over the first half of the
-    // S columns (ascending chunks: a chunk is read before any later chunk is overwritten)
+    // ---- dS for this query row against this thread's 64 of the block's 128 keys, bf16 over
+    // the first half of this half's S columns (ascending chunks: a chunk is read before any
+    // later chunk is overwritten)
     ok = __all_sync(0xffffffffu, ok && wait(s_full, kb & 1, DEVERR_WAIT_ACC_FULL));
     if (ok) {
       tc_fence_after();
+      // no mask inside the block: every key is valid and (causal) before every query
+      const bool plain = q0 + kBlk <= P.s && k0 + kBlk <= P.s && (!P.causal || k0 < q0);
 #pragma unroll 1
-      for (int c0 = 0; c0 < kBlk; c0 += 32) {
+      for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
         float sv[32], dp[32];
         ld32(tS + lane_base + c0, sv);
         ld32(tdP + lane_base + c0, dp);
@@ -472,14 +499,16 @@ __global__ void __launch_bounds__(kThreads, 1)
           float ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            const int k_abs = k0 + c0 + e + u;
-            const bool masked = !q_live || k_abs >= P.s || (P.causal && k_abs > q_abs);
-            const float pr = masked ? 0.f : exp2f(sv[e + u] * P.scale_log2 - lse_r);
+            float pr = exp2_fast(sv[e + u] * P.scale_log2 - lse_r);
+            if (!plain) {
+              const int k_abs = k0 + c0 + e + u;
+              if (!q_live || k_abs >= P.s || (P.causal && k_abs > q_abs)) pr = 0.f;
+            }
             ds[u] = pr * (dp[e + u] - D_r);
           }
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
-        st16(tS + lane_base + c0 / 2, dw);
+        st16(tS + lane_base + packed_col(c0 / 2), dw);
       }
       fa::tmem_wait_st();
     }
@@ -493,8 +522,9 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
           // A: 16 keys = 8 TMEM columns of dS; B: the [key][dim] K tile read MN-major
-          fa::umma_f16_tmem_a(tdQ, tS + kk * 8, make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024),
-                              IDESC_KN, (kb > 0 || kk > 0) ? 1u : 0u);
+          fa::umma_f16_tmem_a(tdQ, tS + packed_col(kk * 8),
+                              make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                              (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
       }
@@ -506,7 +536,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     tc_fence_after();
     __nv_bfloat16* rowp = P.dqkv + (static_cast<int64_t>(bi) * P.s + q_abs) * P.ld + q_col;
 #pragma unroll 1
-    for (int c = 0; c < HD; c += 32) {
+    for (int c = half * (HD / 2); c < (half + 1) * (HD / 2); c += 32) {
       float v[32];
       ld32(tdQ + lane_base + c, v);
 #pragma unroll

@@ -20,7 +20,10 @@
 //   warps 2..5, both CTAs    -- epilogue of the CTA's 128 accumulator rows; each warp returns
 //                               the accumulator by arriving on CTA 0's "acc_empty" barrier.
 // Whole tiles only (no stream-K): cluster c takes tiles c, c + C, c + 2C, ... of the
-// batch x M x N tile space.  No copy is multicast: every CTA loads only its own halves.
+// batch x M x N tile space.  With sum_batch the problems (shards) are summed into one output:
+// the tile space is M x N and each tile's k loop runs over the k-blocks of problem 0, then of
+// problem 1, ... into the same TMEM accumulator -- the partial-sum reduce, shard by shard in
+// order, done in the accumulator.  No copy is multicast: every CTA loads only its own halves.
 //
 // Every wait is bounded as in the one-CTA kernel.  Both CTAs meet at a cluster barrier before
 // TMEM is released and before either exits, so neither CTA's shared memory goes away while the
@@ -129,9 +132,18 @@ __device__ __forceinline__ void umma_commit(uint64_t* bar) {
 }
 
 __device__ __forceinline__ void decode_tile(int t, const GemmParams& gp, int& b, int& mb, int& nb) {
+  if (gp.sum_batch) {
+    b = 0;
+    decode_mn(t, gp, mb, nb);
+    return;
+  }
   const int per = gp.m_blocks * gp.n_blocks;
   b = t / per;
   decode_mn(t - b * per, gp, mb, nb);
+}
+// k-blocks of one tile: all problems' with sum_batch
+__device__ __forceinline__ int tile_k_blocks(const GemmParams& gp) {
+  return gp.sum_batch ? gp.batch * gp.k_blocks : gp.k_blocks;
 }
 
 }  // namespace pair
@@ -160,7 +172,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   const uint32_t rank = pair::cluster_rank();
   const int cluster = static_cast<int>(blockIdx.x >> 1);
   const int nclusters = static_cast<int>(gridDim.x >> 1);
-  const int tiles = gp.batch * gp.m_blocks * gp.n_blocks;
+  const int tiles = (gp.sum_batch ? 1 : gp.batch) * gp.m_blocks * gp.n_blocks;
+  const int nk = pair::tile_k_blocks(gp);
 
   if (threadIdx.x == 0) {
     for (int s = 0; s < Cfg::STAGES; ++s) {
@@ -205,9 +218,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         pair::decode_tile(t, gp, b, mb, nb);
         const int m0 = mb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
         const int n0 = nb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
-        const int za = gp.a_batched ? b : 0;
-        const int zb = gp.b_batched ? b : 0;
-        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+        int bu = b, kb = 0;   // problem and k-block of step u
+        for (int u = 0; u < nk; ++u, ++kb) {
+          if (kb == gp.k_blocks) {   // sum_batch: on to the next problem's k-blocks
+            kb = 0;
+            ++bu;
+          }
+          const int za = gp.a_batched ? bu : 0;
+          const int zb = gp.b_batched ? bu : 0;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
             ok = false;
             break;
@@ -276,7 +294,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_tmem = tmem_base + acc * Cfg::ACC_COLS;
-        for (int kb = 0; kb < gp.k_blocks; ++kb) {
+        for (int u = 0; u < nk; ++u) {
           if (!mbar_wait(&full[stage], phase, abort_flag, gp.err, DEVERR_WAIT_FULL)) {
             ok = false;
             break;
@@ -292,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint64_t bdesc =
                 Cfg::B_MN ? make_sdesc_sw128(b_addr + kk * (kUmmaK * 128), 64 * kBK * 2, 1024)
                           : make_sdesc_sw128(b_addr + kk * (kUmmaK * 2), 16, 1024);
-            pair::umma_f16(d_tmem, adesc, bdesc, Cfg::IDESC, (kb > 0 || kk != 0) ? 1u : 0u);
+            pair::umma_f16(d_tmem, adesc, bdesc, Cfg::IDESC, (u > 0 || kk != 0) ? 1u : 0u);
           }
           issued_any = true;
           pair::umma_commit_mc(&empty[stage], 0x3);
@@ -397,7 +415,8 @@ tp_status pair_clusters(int* out) {
 template <class Cfg, class Epi>
 tp_status run_gemm_pair(const Operand& a, const Operand& b, int64_t M, int64_t N, int64_t K,
                         int64_t batch, const typename Epi::Params& ep, cudaStream_t stream,
-                        const char* label = "gemm", int m_fastest = -1) {
+                        const char* label = "gemm", int m_fastest = -1,
+                        bool sum_batch = false) {
   if (a.mn_major != Cfg::A_MN || b.mn_major != Cfg::B_MN)
     return set_error(TP_ERR_INVALID_ARG, "operand major does not match the tile config");
   if (M <= 0 || N <= 0 || batch <= 0) return TP_OK;
@@ -421,9 +440,11 @@ tp_status run_gemm_pair(const Operand& a, const Operand& b, int64_t M, int64_t N
   gp.a_batched = a.batch > 1 ? 1 : 0;
   gp.b_batched = b.batch > 1 ? 1 : 0;
   gp.err = device_error_word();
+  gp.sum_batch = sum_batch ? 1 : 0;
   if (gp.k_blocks == 0) return set_error(TP_ERR_INVALID_ARG, "GEMM with K == 0");
-  const int64_t tiles = static_cast<int64_t>(gp.batch) * gp.m_blocks * gp.n_blocks;
-  if (tiles > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many output tiles");
+  const int64_t tiles = static_cast<int64_t>(sum_batch ? 1 : gp.batch) * gp.m_blocks * gp.n_blocks;
+  if (tiles > INT32_MAX || static_cast<int64_t>(gp.batch) * gp.k_blocks > INT32_MAX)
+    return set_error(TP_ERR_UNSUPPORTED, "too many output tiles");
 
   int resident = 0;
   st = pair_clusters<Cfg, Epi>(&resident);

@@ -74,10 +74,7 @@ size_t up_sk_bytes(const MlpLayout& L) {
 }
 size_t down_sk_bytes(const MlpLayout& L) {
   const bool fused = L.reduce_mode == TP_REDUCE_FUSED;
-  if (L.T > kSwapMaxT) {
-    if (!fused) return 0;
-    return tc::plan_stream_k<KK<256, 1>>(L.T, L.d, L.Fsp, L.p, true, num_sms()).bytes();
-  }
+  if (L.T > kSwapMaxT) return 0;   // prefill: whole pair tiles, the fused sum in the accumulator
   if (!fused && !decode_stream_k(down_tiles(L))) return 0;
   return by_tokens<1>(L.T, [&](auto tag) {
     return tc::plan_stream_k<typename decltype(tag)::type>(L.d, L.T, L.Fsp, L.p, fused, num_sms()).bytes();
@@ -202,8 +199,10 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
         return tc::run_gemm<typename decltype(tag)::type, tc::EpiReduceOut>(
             wo, ho, L.d, L.T, L.Fsp, L.p, ep, s, "mlp_down_gemm", opt);
       });
-    return tc::run_gemm<KK<256, 1>, tc::EpiReduceOut>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s,
-                                                       "mlp_down_gemm", opt);
+    // prefill: each 256 x 256 tile runs the k-blocks of shard 0, 1, ..., p-1 into one
+    // accumulator, so the shard sum never leaves TMEM
+    return tc::run_gemm_pair<PP<false, false>, tc::EpiReduceOut>(ho, wo, L.T, L.d, L.Fsp, L.p, ep,
+                                                                 s, "mlp_down_gemm", -1, true);
   }
   tc::EpiStoreF32::Params ep;
   ep.out = part;
@@ -227,9 +226,11 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
                                                               "mlp_down_gemm");
 }
 
+// With TP_REDUCE_FUSED the dx GEMM sums the shards in its accumulator and writes dx itself
+// (``dx``); otherwise it writes the fp32 partials to ``part`` for the separate reduce.
 tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
                       const void* h, const void* w1p, const void* w2p, void* dz, float* dw1p,
-                      float* dw2p, float* part, cudaStream_t s) {
+                      float* dw2p, float* part, void* dx, cudaStream_t s) {
   const int64_t P = L.p;
   tp_status st;
   // (1) dH_i = dY W2_i^T with the activation backward fused: dz in w1p row order
@@ -285,10 +286,22 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
                                                             "mlp_dw1_gemm");
     if (st != TP_OK) return st;
   }
-  // (4) dx_i = dz_i W1_i^T  (partials, summed by the caller)
+  // (4) dx_i = dz_i W1_i^T  (partials, summed by the caller; or summed here when fused)
   {
     const Operand a{dz, false, L.T, L.R, P, P * L.R, L.R};
     const Operand b{w1p, true, L.d, L.R, P, L.d, L.R * L.d};
+    if (L.reduce_mode == TP_REDUCE_FUSED) {
+      tc::EpiReduceOut::Params ep;
+      ep.out = dx;
+      ep.residual = nullptr;
+      ep.ld = L.d;
+      ep.rows_valid = static_cast<int32_t>(L.T);
+      ep.cols_valid = static_cast<int32_t>(L.d);
+      ep.out_bf16 = 1;
+      ep.swap = 0;
+      return tc::run_gemm_pair<PP<false, true>, tc::EpiReduceOut>(a, b, L.T, L.d, L.R, P, ep, s,
+                                                                  "mlp_dx_gemm", -1, true);
+    }
     tc::EpiStoreF32::Params ep;
     ep.out = part;
     ep.ld = L.d;
@@ -547,7 +560,11 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
       return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {dy, x, saved, w1p, w2p, static_cast<const void*>(dx)})
       if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, s);
+    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, dx, s);
+    if (st == TP_OK && L.reduce_mode == TP_REDUCE_FUSED) {   // dx already summed
+      count_reduction();
+      return TP_OK;
+    }
   } else if (L.dtype == TP_BF16) {
     st = simt_backward<__nv_bfloat16>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
   } else {

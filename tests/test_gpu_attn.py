@@ -113,11 +113,13 @@ def test_decode_matches_prefill_last_row(lib):
     assert rel_l2(f64(y_dec)[0, 0], f64(y_pre)[0, L]) <= TOL["bf16"]
 
 
-def test_full_size_attention_sampled(lib):
-    # b=1, s=2048, h=8192, 64 Q / 8 KV heads, head_dim 128, p=8, causal, W ~ N(0, 0.02)
+@pytest.mark.parametrize("mode", [0, 1])
+def test_full_size_attention_sampled(lib, mode):
+    # b=1, s=2048, h=8192, 64 Q / 8 KV heads, head_dim 128, p=8, causal, W ~ N(0, 0.02);
+    # mode 1 adds the 8 shard partials inside the output projection's accumulator
     cfg = dict(b=1, s=2048, h=8192, n_q=64, n_kv=8, hd=128)
     inp = inputs.attn_inputs(*cfg.values(), "bf16", seed=0, device="cuda", w_std=0.02)
-    a = Attn(lib, inp, 8, "bf16", True, n_q=64, n_kv=8, hd=128)
+    a = Attn(lib, inp, 8, "bf16", True, n_q=64, n_kv=8, hd=128, reduce_mode=mode)
     y = a.forward(inp["x"])
     torch.cuda.synchronize()
     rows = [0, 1, 1023, 2047]

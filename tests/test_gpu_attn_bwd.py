@@ -42,6 +42,25 @@ def test_backward_parity(lib, causal, b, s, h, n_q, n_kv, hd, p):
         assert err <= TOL["bf16"], (name, err)
 
 
+@pytest.mark.parametrize("b,s,h,n_q,n_kv,hd,p", [
+    (2, 37, 256, 8, 2, 32, 2),
+    (2, 150, 264, 4, 2, 128, 2),    # h = 264: ragged K of the dx GEMM's second shard tile
+])
+def test_backward_fused_dx(lib, b, s, h, n_q, n_kv, hd, p):
+    # TP_REDUCE_FUSED: the dx GEMM adds the shards in its accumulator and writes dx directly
+    inp = inputs.attn_inputs(b, s, h, n_q, n_kv, hd, "bf16", seed=35, w_std=0.05)
+    dy = inputs.normal((b, s, h), 1.0, 35, 97, "bf16", "cpu")
+    a = Attn(lib, inp, p, "bf16", True, n_q=n_q, n_kv=n_kv, hd=hd, reduce_mode=1)
+    lib.tp_reset_reduction_count()
+    got = a.backward(inp["x"], dy)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    ref = _grads_ref(inp, dy, n_q, n_kv, hd, True)
+    for name, g, r in zip(("dx", "dwq", "dwk", "dwv", "dwo"), got, ref):
+        err = rel_l2(f64(g), r)
+        assert err <= TOL["bf16"], (name, err)
+
+
 def test_backward_deterministic(lib):
     inp = inputs.attn_inputs(1, 100, 256, 8, 2, 64, "bf16", seed=32, w_std=0.05)
     dy = inputs.normal((1, 100, 256), 1.0, 32, 97, "bf16", "cpu")

@@ -87,17 +87,21 @@ def test_backward_parity(lib, act, dtype, T):
         assert rel_l2(f64(dwu), ref["dw_up"]) <= tol
 
 
+@pytest.mark.parametrize("reduce_mode", [0, 1])
 @pytest.mark.parametrize("act", ["swiglu", "gelu"])
-def test_pair_tiles_forward_backward(lib, act):
+def test_pair_tiles_forward_backward(lib, act, reduce_mode):
     # the prefill and backward GEMMs run 256 x 256 tiles on SM pairs: T = 520 gives three token
     # tiles (the last one ragged, its second half empty), d = 776 a ragged K and N, F_s = 512 two
-    # feature tiles per shard; every GEMM of forward and backward has several tiles per dimension
+    # feature tiles per shard; every GEMM of forward and backward has several tiles per dimension.
+    # reduce_mode 1 sums the shards of the down and dx GEMMs in their accumulators.
     T, d, F, p = 520, 776, 1536, 3
     inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=11, w_std=0.05, backward=True)
-    m = Mlp(lib, inp, p, act, "bf16")
+    m = Mlp(lib, inp, p, act, "bf16", reduce_mode)
+    lib.tp_reset_reduction_count()
     y = m.forward(inp["x"])
     dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
     torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 2
     wu = None if inp["w_up"] is None else f64(inp["w_up"])
     assert rel_l2(f64(y), _oracle_fwd(inp, act)) <= TOL["bf16"]
     ref = omlp.mlp_backward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), f64(inp["dy"]), act, wu)
@@ -162,12 +166,14 @@ def test_full_size_decode_mlp_sampled(lib):
     assert rel_l2(f64(y)[rows], ref) <= TOL["bf16"]
 
 
-def test_full_size_prefill_mlp_sampled(lib):
-    # T=4096 (b=1, s=4096), d=8192, d_ff=28672, p=8: forward rows, then backward samples
+@pytest.mark.parametrize("mode", [0, 1])
+def test_full_size_prefill_mlp_sampled(lib, mode):
+    # T=4096 (b=1, s=4096), d=8192, d_ff=28672, p=8: forward rows, then backward samples;
+    # mode 1 adds the 8 shard partials of y and of dx inside the GEMM accumulators
     T, d, F, p = 4096, 8192, 28672, 8
     inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02,
                             backward=True)
-    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    m = Mlp(lib, inp, p, "swiglu", "bf16", mode)
     y = m.forward(inp["x"])
     dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
     torch.cuda.synchronize()
