@@ -18,6 +18,9 @@ What it computes, and where the method is stated:
                    "One collective": the residual add and the following normalization stay
                    replicated).
 * ``costmodel`` -- the pages' reduction-count and message-byte arithmetic.
+* ``seqpar``    -- the sequence-parallel form of the collective: reduce-scatter of the partials
+                   into token slices and all-gather of the slices ("Why tensor parallelism has to
+                   stay in scale-up", "Where the 320 comes from").
 
 Each function also has a *sharded reference mode* (loop over the p shards and add the partial
 results in order) used only by the invariant tests that check "the sharded sum equals the
@@ -27,4 +30,4 @@ Everything is float64 numpy; matrix products use numpy's matmul as a library pri
 error function comes from scipy.  No blocking, fusion or reordering beyond the stated formulas.
 """
 
-from . import mlp, attention, decode, costmodel  # noqa: F401
+from . import mlp, attention, decode, costmodel, seqpar  # noqa: F401
