@@ -383,7 +383,63 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
         time.sleep(1.0)
     if "prefill" in which:
         ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
+    if "seqpar" in which:
+        time.sleep(1.0)
+        ex["seqpar_prefill_mlp_fwd"] = extra_seqpar(tp, inputs, torch, stream, peaks, steps)
     return ex
+
+
+def extra_seqpar(tp, inputs, torch, stream, peaks, steps):
+    """Sequence-parallel prefill MLP forward (T=4096, d=8192, d_ff=28672, p=8): x arrives as the
+    8 shards' token slices and y leaves as slices -- all-gather, the two GEMMs, then the
+    reduce-scatter with the residual add and RMSNorm on the slices -- against the plain forward
+    with the same residual and norm."""
+    c = PREFILL
+    st = setup_mlp(tp, inputs, torch, c)
+    dev = st["x"].device
+    T, d, p = c["T"], c["d"], c["p"]
+    R = T // p
+    res = inputs.normal((T, d), 1.0, 0, 98, "bf16", dev)
+    yn = torch.empty_like(st["y"])
+    cut = lambda t: [t[i * R:(i + 1) * R].clone() for i in range(p)]
+    xs, rs = cut(st["x"]), cut(res)
+    ys = [torch.empty(R, d, dtype=torch.bfloat16, device=dev) for _ in range(p)]
+    yns = [torch.empty_like(ys[0]) for _ in range(p)]
+    ws = torch.empty(tp.tp_mlp_fwd_sp_workspace(st["desc"]), dtype=torch.uint8, device=dev)
+
+    def plain():
+        tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], residual=res,
+                      workspace=st["ws"], y_norm=yn)
+
+    def spf():
+        tp.tp_mlp_fwd_sp(st["desc"], xs, st["w1p"], st["w2p"], ys, residual_slices=rs,
+                         y_norm_slices=yns, workspace=ws)
+
+    for _ in range(3):
+        plain()
+        spf()
+    ms_plain = _cuda_time(plain, steps, stream) / steps
+    ms_sp = _cuda_time(spf, steps, stream) / steps
+    prof = _profile(tp, spf, steps)
+    # algorithmic bytes: the reduce-scatter reads the p fp32 partials and the residual slices
+    # and writes y and its norm (bf16); the all-gather reads and writes x once
+    coll = {"reduce_scatter": p * T * d * 4 + 3 * T * d * 2, "all_gather": 2 * T * d * 2}
+    kern = {}
+    for k, (n, ms) in prof.items():
+        e = {"ms_per_launch": round(ms / n, 4)}
+        if k in coll:
+            gbs = coll[k] / (ms / n / 1e3) / 1e9
+            e.update({"algorithmic_bytes": coll[k], "GB_per_s": round(gbs, 1),
+                      "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 3)})
+        kern[k] = e
+    same = bool(torch.equal(torch.cat(ys), st["y"]) and torch.equal(torch.cat(yns), yn))
+    del st
+    torch.cuda.empty_cache()
+    return {"workload": "sequence-parallel prefill TP SwiGLU MLP forward: T=4096 as 8 slices of "
+                        "512 tokens, d=8192, d_ff=28672, p=8, bf16, residual + RMSNorm on slices",
+            "ms": round(ms_sp, 3), "ms_plain_forward": round(ms_plain, 3),
+            "TFLOP_per_s": round(2.0 * T * d * c["F"] * 3 / (ms_sp / 1e3) / 1e12, 1),
+            "slices_equal_plain_rows": same, "kernels": kern, "steps": steps}
 
 
 def extra_tiny(tp, inputs, torch, stream, calls=2000):
@@ -692,7 +748,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=20)
-    ap.add_argument("--extras", default="tiny,prefill,attention,stack",
+    ap.add_argument("--extras", default="tiny,prefill,attention,stack,seqpar",
                     help="comma list of extra workloads to measure at N=1")
     ap.add_argument("--reduce-mode", choices=["separate", "fused"], default="separate",
                     help="how the p partial sums are added in the decode workloads")

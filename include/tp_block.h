@@ -254,11 +254,73 @@ tp_status tp_rmsnorm(const void* x, int32_t x_dtype, int64_t rows, int64_t d, fl
                      void* out, int32_t out_dtype, void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* Sequence parallelism                                                                        */
+/* ------------------------------------------------------------------------------------------ */
+/* "Why tensor parallelism has to stay in scale-up" (Keysight), "Where the 320 comes from": with
+ * sequence parallelism each all-reduce becomes a reduce-scatter plus an all-gather, moving the
+ * same bytes.  Between the row-parallel output of one block and the column-parallel input of the
+ * next, shard i owns token rows i*T/p .. (i+1)*T/p - 1 of the [T][d] activation (a "slice"),
+ * and the residual add and normalisation run on the slices.  Here every slice is its own device
+ * buffer [T/p][d]: the slice arguments are HOST arrays of p device pointers (p <= 64), each
+ * 16-byte aligned for the vectorised path (any alignment works).  p must divide T; a violation
+ * returns TP_ERR_SHAPE.  The block calls accept only TP_REDUCE_SEPARATE (TP_ERR_UNSUPPORTED
+ * otherwise). */
+
+/* Reduce-scatter: out_slices[i][r] = residual_slices[i][r] + sum_{s=0}^{p-1} partials[s][i*T/p + r]
+ * (fp32 in shard order, residual last, one rounding to out_dtype); with norm_slices, also
+ * norm_slices[i][r] = RMSNorm(out_slices[i][r]) (unit weight, eps; norm_dtype) computed from the
+ * stored values.  partials: [p][T][d] fp32.  residual_slices and norm_slices may be NULL.
+ * Adds 1 to the reduction counter. */
+tp_status tp_reduce_scatter_partials(const void* partials, int32_t p, int64_t T, int64_t d,
+                                     void* const* residual_slices, void* const* out_slices,
+                                     int32_t out_dtype, void* const* norm_slices,
+                                     int32_t norm_dtype, float eps, void* stream);
+
+/* All-gather: out[i*rows_per_slice + r] = slices[i][r]; out is [p*rows_per_slice][d] of dtype. */
+tp_status tp_all_gather_slices(const void* const* slices, int32_t p, int64_t rows_per_slice,
+                               int64_t d, int32_t dtype, void* out, void* stream);
+
+/* MLP forward, sequence-parallel.  The p slices of x ([T/p][d], dtype) are all-gathered, then
+ * the block runs as in tp_mlp_fwd (the same packed weights and saved activations).  The partials
+ * are then reduce-scattered into y_slices ([T/p][d], dtype, or fp32 with TP_FLAG_F32_RESIDUAL),
+ * adding residual_slices (optional).  y_norm_slices (optional) receive RMSNorm of the y rows
+ * (norm_eps).  workspace: tp_mlp_fwd_sp_workspace(desc) bytes (0 for an unsupported
+ * descriptor).  Adds 1 to the reduction counter. */
+size_t tp_mlp_fwd_sp_workspace(const tp_mlp_desc* desc);
+tp_status tp_mlp_fwd_sp(const tp_mlp_desc* desc, const void* const* x_slices, const void* w1p,
+                        const void* w2p, void* const* residual_slices, void* const* y_slices,
+                        void* const* y_norm_slices, void* saved, void* workspace,
+                        size_t ws_bytes, void* stream);
+
+/* MLP backward, sequence-parallel.  The dy and x slices are all-gathered (the reduce-scatter's
+ * gradient is an all-gather), and the backward runs as in tp_mlp_bwd.  The dx partials are then
+ * reduce-scattered into dx_slices ([T/p][d], dtype; the all-gather's gradient).  dw1p and dw2p
+ * are as in tp_mlp_bwd.  saved is the forward's saved activations.  workspace:
+ * tp_mlp_bwd_sp_workspace(desc) bytes.  Adds 1 to the reduction counter. */
+size_t tp_mlp_bwd_sp_workspace(const tp_mlp_desc* desc);
+tp_status tp_mlp_bwd_sp(const tp_mlp_desc* desc, const void* const* dy_slices,
+                        const void* const* x_slices, const void* saved, const void* w1p,
+                        const void* w2p, void* const* dx_slices, void* dw1p, void* dw2p,
+                        void* workspace, size_t ws_bytes, void* stream);
+
+/* Attention forward, sequence-parallel over the b*s token rows.  It all-gathers the x slices
+ * ([b*s/p][h]), runs tp_attn_fwd's block (KV caches as there), then reduce-scatters the output
+ * partials into y_slices with residual_slices and y_norm_slices as in tp_mlp_fwd_sp.
+ * workspace: tp_attn_fwd_sp_workspace(desc) bytes.  Adds 1 to the reduction counter. */
+size_t tp_attn_fwd_sp_workspace(const tp_attn_desc* desc);
+tp_status tp_attn_fwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
+                         const void* wqkv_p, const void* wo_p, void* k_cache, void* v_cache,
+                         void* const* residual_slices, void* const* y_slices,
+                         void* const* y_norm_slices, void* workspace, size_t ws_bytes,
+                         void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Diagnostics                                                                                 */
 /* ------------------------------------------------------------------------------------------ */
 
 /* Reductions of p partials enqueued so far (one per tp_mlp_fwd / tp_mlp_bwd / tp_attn_fwd /
- * tp_reduce_partials call that succeeded), process-wide. */
+ * tp_attn_bwd / tp_reduce_partials call that succeeded, and one per reduce-scatter of the
+ * sequence-parallel calls), process-wide. */
 uint64_t tp_reduction_count(void);
 void tp_reset_reduction_count(void);
 

@@ -9,6 +9,7 @@
 #include "gemm_pair.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
+#include "seqpar.cuh"
 #include "simt.cuh"
 #include "tp_common.cuh"
 
@@ -675,9 +676,12 @@ inline tp_status attn_simt_proj(const AttnLayout& L, const void* x, const void* 
   return simt::gemm<T>(g, s);
 }
 
+// With ``sp`` (sequence parallelism) the partials are reduce-scattered into the shards' token
+// slices instead of summed into y (which, like residual and y_norm, is then unused).
 inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wqkv,
                               const void* wo_p, void* kc, void* vc, const void* residual,
-                              void* y, void* y_norm, void* ws, cudaStream_t s) {
+                              void* y, void* y_norm, void* ws, cudaStream_t s,
+                              const seqpar::SpOut* sp = nullptr) {
   uint8_t* w = static_cast<uint8_t*>(ws);
   void* qkv = w + L.qkv_off;
   void* o = w + L.o_off;
@@ -708,6 +712,9 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
     if ((st = attn_core<float>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
     if ((st = attn_simt_proj<float>(L, x, wqkv, qkv, o, wo_p, part, s, false)) != TP_OK) return st;
   }
+  if (sp)
+    return seqpar::reduce_scatter(part, L.p, L.tokens, L.h, sp->res, sp->y, L.y_dtype, sp->norm,
+                                  L.dtype, L.norm_eps, s);
   if (y_norm)
     return reduce::reduce_norm(part, L.p, L.tokens, L.h, residual, y, L.y_dtype, y_norm, L.dtype,
                                L.norm_eps, s);

@@ -57,6 +57,72 @@ extern "C" tp_status tp_attn_fwd(const tp_attn_desc* desc, const void* x, const 
   return st;
 }
 
+// Sequence-parallel forward: the input arrives as the p shards' token slices and is all-gathered
+// before the QKV GEMM; the output partials are reduce-scattered into the slices (with the residual
+// add and the RMSNorm on the slices).  "Why tensor parallelism has to stay in scale-up"
+// (Keysight), "Where the 320 comes from".
+namespace {
+size_t sp_act_bytes(const tp::AttnLayout& L) {
+  return tp::align256(static_cast<size_t>(L.tokens * L.h) * tp::elem_bytes(L.dtype));
+}
+tp_status sp_layout(const tp_attn_desc* desc, tp::AttnLayout* L) {
+  tp_status st = tp::attn_layout_of(desc, L);
+  if (st != TP_OK) return st;
+  if (desc->reduce_mode != TP_REDUCE_SEPARATE)
+    return tp::set_error(TP_ERR_UNSUPPORTED,
+                         "the sequence-parallel calls reduce-scatter the partials: use TP_REDUCE_SEPARATE");
+  if (L->p > tp::seqpar::kMaxSlices) return tp::set_error(TP_ERR_SHAPE, "p must be <= 64 for slices");
+  if (L->tokens % L->p) return tp::set_error(TP_ERR_SHAPE, "sequence parallelism needs p to divide b*s");
+  return TP_OK;
+}
+}  // namespace
+
+extern "C" size_t tp_attn_fwd_sp_workspace(const tp_attn_desc* desc) {
+  tp::AttnLayout L;
+  if (sp_layout(desc, &L) != TP_OK) return 0;
+  return sp_act_bytes(L) + L.ws_bytes;
+}
+
+extern "C" tp_status tp_attn_fwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
+                                    const void* wqkv_p, const void* wo_p, void* k_cache,
+                                    void* v_cache, void* const* residual_slices,
+                                    void* const* y_slices, void* const* y_norm_slices,
+                                    void* workspace, size_t ws_bytes, void* stream) {
+  tp::clear_error();
+  tp::AttnLayout L;
+  tp_status st = sp_layout(desc, &L);
+  if (st != TP_OK) return st;
+  if (L.tokens == 0) {
+    tp::count_reduction();
+    return TP_OK;
+  }
+  using tp::seqpar::check_slices;
+  if ((st = check_slices(L.p, L.tokens, const_cast<void* const*>(x_slices), "x_slices")) != TP_OK ||
+      (st = check_slices(L.p, L.tokens, y_slices, "y_slices")) != TP_OK)
+    return st;
+  if (residual_slices && (st = check_slices(L.p, L.tokens, residual_slices, "residual_slices")) != TP_OK)
+    return st;
+  if (y_norm_slices && (st = check_slices(L.p, L.tokens, y_norm_slices, "y_norm_slices")) != TP_OK)
+    return st;
+  if (!wqkv_p || !wo_p) return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (L.kv_len > 0 && (!k_cache || !v_cache))
+    return tp::set_error(TP_ERR_INVALID_ARG, "decode needs k_cache and v_cache");
+  if (L.kv_len > 0 && ((reinterpret_cast<uintptr_t>(k_cache) | reinterpret_cast<uintptr_t>(v_cache)) & 15))
+    return tp::set_error(TP_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
+  if (!workspace) return tp::set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < sp_act_bytes(L) + L.ws_bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* x = workspace;
+  void* ws = static_cast<uint8_t*>(workspace) + sp_act_bytes(L);
+  st = tp::seqpar::all_gather(x_slices, L.p,
+                              (L.tokens / L.p) * L.h * tp::elem_bytes(L.dtype), x, s);
+  if (st != TP_OK) return st;
+  const tp::seqpar::SpOut sp{residual_slices, y_slices, y_norm_slices};
+  st = tp::attn_forward(L, x, wqkv_p, wo_p, k_cache, v_cache, nullptr, nullptr, nullptr, ws, s, &sp);
+  if (st == TP_OK) tp::count_reduction();
+  return st;
+}
+
 // ------------------------------------------------------------------------------------ backward
 #include "attn_bwd.cuh"
 

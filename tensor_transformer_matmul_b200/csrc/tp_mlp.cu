@@ -16,6 +16,7 @@
 #include "gemm_pair.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
+#include "seqpar.cuh"
 #include "simt.cuh"
 #include "tp_common.cuh"
 
@@ -572,6 +573,144 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
   }
   if (st != TP_OK) return st;
   st = reduce::launch(part, TP_F32, L.p, L.T * L.d, nullptr, dx, L.dtype, s);
+  if (st == TP_OK) count_reduction();
+  return st;
+}
+
+// ------------------------------------------------------------------ sequence-parallel variant
+// "Why tensor parallelism has to stay in scale-up" (Keysight), "Where the 320 comes from": with
+// sequence parallelism the block's all-reduce becomes a reduce-scatter of the partials into the
+// shards' token slices (residual add and norm then run on the slices) and an all-gather of the
+// slices before the column-parallel GEMM.  Backward: the all-gather's gradient is a
+// reduce-scatter (dx) and the reduce-scatter's an all-gather (dy).
+namespace {
+size_t act_bytes(const MlpLayout& L) { return align256(static_cast<size_t>(L.T * L.d) * L.eb); }
+
+tp_status sp_layout(const tp_mlp_desc* desc, MlpLayout* L) {
+  tp_status st = layout_of(desc, L);
+  if (st != TP_OK) return st;
+  if (desc->reduce_mode != TP_REDUCE_SEPARATE)
+    return set_error(TP_ERR_UNSUPPORTED,
+                     "the sequence-parallel calls reduce-scatter the partials: use TP_REDUCE_SEPARATE");
+  if (L->p > seqpar::kMaxSlices) return set_error(TP_ERR_SHAPE, "p must be <= 64 for slices");
+  if (L->T % L->p) return set_error(TP_ERR_SHAPE, "sequence parallelism needs p to divide T");
+  return TP_OK;
+}
+}  // namespace
+
+extern "C" size_t tp_mlp_fwd_sp_workspace(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  if (sp_layout(desc, &L) != TP_OK) return 0;
+  return act_bytes(L) + L.fwd_ws;
+}
+
+extern "C" tp_status tp_mlp_fwd_sp(const tp_mlp_desc* desc, const void* const* x_slices,
+                                   const void* w1p, const void* w2p,
+                                   void* const* residual_slices, void* const* y_slices,
+                                   void* const* y_norm_slices, void* saved, void* workspace,
+                                   size_t ws_bytes, void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = sp_layout(desc, &L);
+  if (st != TP_OK) return st;
+  if (L.T == 0) {
+    count_reduction();
+    return TP_OK;
+  }
+  void* const* xs = const_cast<void* const*>(x_slices);
+  if ((st = seqpar::check_slices(L.p, L.T, xs, "x_slices")) != TP_OK) return st;
+  if ((st = seqpar::check_slices(L.p, L.T, y_slices, "y_slices")) != TP_OK) return st;
+  if (residual_slices && (st = seqpar::check_slices(L.p, L.T, residual_slices, "residual_slices")) != TP_OK)
+    return st;
+  if (y_norm_slices && (st = seqpar::check_slices(L.p, L.T, y_norm_slices, "y_norm_slices")) != TP_OK)
+    return st;
+  if (!w1p || !w2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < act_bytes(L) + L.fwd_ws) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  void* x = workspace;                        // the gathered [T][d] input
+  void* ws = off(workspace, act_bytes(L));    // the forward's own workspace
+  void* z = saved ? off(saved, L.saved_z_off) : off(ws, L.fz_off);
+  void* h = saved ? off(saved, L.saved_h_off) : off(ws, L.fh_off);
+  float* part = reinterpret_cast<float*>(off(ws, L.fpart_off));
+  if ((st = seqpar::all_gather(x_slices, L.p, (L.T / L.p) * L.d * L.eb, x, s)) != TP_OK) return st;
+  if (L.tc) {
+    if (!tensor_cores_usable())
+      return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+    for (const void* q : {w1p, w2p, static_cast<const void*>(saved)})
+      if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    void* sk = off(ws, L.fsk_off);
+    const size_t skb = L.fpart_off - L.fsk_off;
+    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
+    if ((st = tc_down(L, h, w2p, part, nullptr, nullptr, sk, skb, s)) != TP_OK) return st;
+  } else if (L.dtype == TP_BF16) {
+    if ((st = simt_forward<__nv_bfloat16>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
+  } else {
+    if ((st = simt_forward<float>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
+  }
+  st = seqpar::reduce_scatter(part, L.p, L.T, L.d, residual_slices, y_slices, L.y_dtype,
+                              y_norm_slices, L.dtype, L.norm_eps, s);
+  if (st == TP_OK) count_reduction();
+  return st;
+}
+
+extern "C" size_t tp_mlp_bwd_sp_workspace(const tp_mlp_desc* desc) {
+  MlpLayout L;
+  if (sp_layout(desc, &L) != TP_OK) return 0;
+  return 2 * act_bytes(L) + L.bwd_ws;
+}
+
+extern "C" tp_status tp_mlp_bwd_sp(const tp_mlp_desc* desc, const void* const* dy_slices,
+                                   const void* const* x_slices, const void* saved,
+                                   const void* w1p, const void* w2p, void* const* dx_slices,
+                                   void* dw1p, void* dw2p, void* workspace, size_t ws_bytes,
+                                   void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = sp_layout(desc, &L);
+  if (st != TP_OK) return st;
+  if (!w1p || !w2p || !dw1p || !dw2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (L.T == 0) {
+    TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(L.p * L.R * L.d) * 4, s));
+    TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(L.p * L.d * L.Fsp) * 4, s));
+    count_reduction();
+    return TP_OK;
+  }
+  if ((st = seqpar::check_slices(L.p, L.T, const_cast<void* const*>(dy_slices), "dy_slices")) != TP_OK ||
+      (st = seqpar::check_slices(L.p, L.T, const_cast<void* const*>(x_slices), "x_slices")) != TP_OK ||
+      (st = seqpar::check_slices(L.p, L.T, dx_slices, "dx_slices")) != TP_OK)
+    return st;
+  if (!saved) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < 2 * act_bytes(L) + L.bwd_ws) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  void* dy = workspace;
+  void* x = off(workspace, act_bytes(L));
+  void* ws = off(workspace, 2 * act_bytes(L));
+  const int64_t slice_bytes = (L.T / L.p) * L.d * L.eb;
+  if ((st = seqpar::all_gather(dy_slices, L.p, slice_bytes, dy, s)) != TP_OK) return st;
+  if ((st = seqpar::all_gather(x_slices, L.p, slice_bytes, x, s)) != TP_OK) return st;
+  const void* z = static_cast<const uint8_t*>(saved) + L.saved_z_off;
+  const void* h = static_cast<const uint8_t*>(saved) + L.saved_h_off;
+  float* dh = reinterpret_cast<float*>(off(ws, L.bdh_off));
+  void* dz = off(ws, L.bdz_off);
+  float* part = reinterpret_cast<float*>(off(ws, L.bpart_off));
+  float* g1 = static_cast<float*>(dw1p);
+  float* g2 = static_cast<float*>(dw2p);
+  if (L.tc) {
+    if (!tensor_cores_usable())
+      return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+    for (const void* q : {saved, w1p, w2p})
+      if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
+    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, nullptr, s);
+  } else if (L.dtype == TP_BF16) {
+    st = simt_backward<__nv_bfloat16>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
+  } else {
+    st = simt_backward<float>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
+  }
+  if (st != TP_OK) return st;
+  st = seqpar::reduce_scatter(part, L.p, L.T, L.d, nullptr, dx_slices, L.dtype, nullptr, L.dtype,
+                              L.norm_eps, s);
   if (st == TP_OK) count_reduction();
   return st;
 }

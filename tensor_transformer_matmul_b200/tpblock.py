@@ -34,6 +34,9 @@ EXPORTS = (
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
     "tp_profile_enable", "tp_profile_read", "tp_profile_reset", "tp_mlp_fwd_static_ws",
     "tp_selftest_wait_timeout", "tp_attn_bwd_workspace", "tp_attn_bwd", "tp_attn_unpack_grads",
+    "tp_reduce_scatter_partials", "tp_all_gather_slices", "tp_mlp_fwd_sp_workspace",
+    "tp_mlp_fwd_sp", "tp_mlp_bwd_sp_workspace", "tp_mlp_bwd_sp", "tp_attn_fwd_sp_workspace",
+    "tp_attn_fwd_sp",
 )
 
 
@@ -95,6 +98,14 @@ def load():
         "tp_attn_bwd_workspace": (S, [AD]),
         "tp_attn_bwd": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
         "tp_attn_unpack_grads": (I32, [AD, P, P, P, P, P, P, P]),
+        "tp_reduce_scatter_partials": (I32, [P, I32, I64, I64, P, P, I32, P, I32, F32, P]),
+        "tp_all_gather_slices": (I32, [P, I32, I64, I64, I32, P, P]),
+        "tp_mlp_fwd_sp_workspace": (S, [MD]),
+        "tp_mlp_fwd_sp": (I32, [MD, P, P, P, P, P, P, P, P, S, P]),
+        "tp_mlp_bwd_sp_workspace": (S, [MD]),
+        "tp_mlp_bwd_sp": (I32, [MD, P, P, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_fwd_sp_workspace": (S, [AD]),
+        "tp_attn_fwd_sp": (I32, [AD, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
@@ -260,6 +271,89 @@ def tp_rmsnorm(x, out, eps=1e-5, stream=None):
     rows = x.numel() // x.shape[-1] if x.numel() else 0
     _check(load().tp_rmsnorm(_ptr(x), xt, int(rows), int(x.shape[-1]), float(eps), _ptr(out), ot,
                              _stream(stream)))
+
+
+# ------------------------------------------------------------------- sequence parallelism
+class _Slices:
+    """A host array of device pointers, one per shard's token slice (kept alive with the
+    tensors it points into)."""
+
+    def __init__(self, tensors):
+        self.tensors = list(tensors)
+        self.arr = (ctypes.c_void_p * len(self.tensors))(*[_ptr(t) for t in self.tensors])
+
+    @property
+    def ptr(self):
+        return ctypes.cast(self.arr, ctypes.c_void_p)
+
+
+def _slices(ts):
+    return None if ts is None else _Slices(ts)
+
+
+def _sp(s):
+    return None if s is None else s.ptr
+
+
+def _dt(t):
+    return TP_BF16 if t.dtype == torch.bfloat16 else TP_F32
+
+
+def tp_reduce_scatter_partials(partials, p, slices, residual=None, norm=None, eps=1e-5,
+                               stream=None):
+    """partials [p][T][d] fp32 -> slices[i] [T/p][d] (+ residual[i]; norm[i] = RMSNorm)."""
+    T, d = partials.shape[-2], partials.shape[-1]
+    so, sr, sn = _Slices(slices), _slices(residual), _slices(norm)
+    _check(load().tp_reduce_scatter_partials(
+        _ptr(partials), int(p), int(T), int(d), _sp(sr), so.ptr, _dt(slices[0]), _sp(sn),
+        _dt(norm[0]) if norm is not None else TP_F32, float(eps), _stream(stream)))
+
+
+def tp_all_gather_slices(slices, out, stream=None):
+    """slices[i] [R][d] -> out [p*R][d]."""
+    si = _Slices(slices)
+    R = slices[0].shape[0] if slices[0].dim() > 1 else 0
+    d = slices[0].shape[-1]
+    _check(load().tp_all_gather_slices(si.ptr, len(slices), int(R), int(d), _dt(out), _ptr(out),
+                                       _stream(stream)))
+
+
+def tp_mlp_fwd_sp_workspace(desc):
+    return load().tp_mlp_fwd_sp_workspace(ctypes.byref(desc))
+
+
+def tp_mlp_fwd_sp(desc, x_slices, w1p, w2p, y_slices, residual_slices=None, y_norm_slices=None,
+                  saved=None, workspace=None, stream=None):
+    xs, ys = _Slices(x_slices), _Slices(y_slices)
+    rs, ns = _slices(residual_slices), _slices(y_norm_slices)
+    _check(load().tp_mlp_fwd_sp(ctypes.byref(desc), xs.ptr, _ptr(w1p), _ptr(w2p), _sp(rs), ys.ptr,
+                                _sp(ns), _ptr(saved), _ptr(workspace), _nbytes(workspace),
+                                _stream(stream)))
+
+
+def tp_mlp_bwd_sp_workspace(desc):
+    return load().tp_mlp_bwd_sp_workspace(ctypes.byref(desc))
+
+
+def tp_mlp_bwd_sp(desc, dy_slices, x_slices, saved, w1p, w2p, dx_slices, dw1p, dw2p,
+                  workspace=None, stream=None):
+    dys, xs, dxs = _Slices(dy_slices), _Slices(x_slices), _Slices(dx_slices)
+    _check(load().tp_mlp_bwd_sp(ctypes.byref(desc), dys.ptr, xs.ptr, _ptr(saved), _ptr(w1p),
+                                _ptr(w2p), dxs.ptr, _ptr(dw1p), _ptr(dw2p), _ptr(workspace),
+                                _nbytes(workspace), _stream(stream)))
+
+
+def tp_attn_fwd_sp_workspace(desc):
+    return load().tp_attn_fwd_sp_workspace(ctypes.byref(desc))
+
+
+def tp_attn_fwd_sp(desc, x_slices, wqkv_p, wo_p, y_slices, k_cache=None, v_cache=None,
+                   residual_slices=None, y_norm_slices=None, workspace=None, stream=None):
+    xs, ys = _Slices(x_slices), _Slices(y_slices)
+    rs, ns = _slices(residual_slices), _slices(y_norm_slices)
+    _check(load().tp_attn_fwd_sp(ctypes.byref(desc), xs.ptr, _ptr(wqkv_p), _ptr(wo_p),
+                                 _ptr(k_cache), _ptr(v_cache), _sp(rs), ys.ptr, _sp(ns),
+                                 _ptr(workspace), _nbytes(workspace), _stream(stream)))
 
 
 # ------------------------------------------------------------------------------ diagnostics

@@ -141,3 +141,40 @@ def test_empty_batch_counts_one_reduction(lib):
     assert so.tp_mlp_fwd(ctypes.byref(desc), None, None, None, None, None, None, None, None, 0, None) == 0
     assert lib.tp_reduction_count() == 1
     lib.tp_reset_reduction_count()
+
+
+def test_sequence_parallel_argument_errors(lib):
+    # checked on the host before anything is enqueued
+    so = lib.load()
+    fake = ctypes.c_void_p(0x1000)
+    two = (ctypes.c_void_p * 2)(0x1000, 0x2000)
+    one_null = (ctypes.c_void_p * 2)(0x1000, None)
+    arr = lambda a: ctypes.cast(a, ctypes.c_void_p)
+    # p must divide T
+    assert so.tp_reduce_scatter_partials(fake, 2, 5, 8, None, arr(two), 1, None, 1, 1e-5,
+                                         None) == lib.TP_ERR_SHAPE
+    # every slice pointer must be given
+    assert so.tp_reduce_scatter_partials(fake, 2, 4, 8, None, arr(one_null), 1, None, 1, 1e-5,
+                                         None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_reduce_scatter_partials(fake, 2, 4, 8, None, None, 1, None, 1, 1e-5,
+                                         None) == lib.TP_ERR_INVALID_ARG
+    # at most 64 slices
+    assert so.tp_reduce_scatter_partials(fake, 65, 65, 8, None, arr(two), 1, None, 1, 1e-5,
+                                         None) == lib.TP_ERR_SHAPE
+    assert so.tp_all_gather_slices(arr(two), 2, 4, 8, 7, fake, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_all_gather_slices(arr(one_null), 2, 4, 8, 1, fake, None) == lib.TP_ERR_INVALID_ARG
+    # the block calls: p must divide the tokens; the fused reduce has no sequence-parallel form
+    d_ok = lib.mlp_desc(8, 64, 256, 2, "swiglu", "bf16")
+    d_rag = lib.mlp_desc(9, 64, 256, 2, "swiglu", "bf16")
+    d_fused = lib.mlp_desc(8, 64, 256, 2, "swiglu", "bf16", lib.TP_REDUCE_FUSED)
+    assert lib.tp_mlp_fwd_sp_workspace(d_ok) > lib.tp_mlp_fwd_workspace(d_ok)
+    assert lib.tp_mlp_fwd_sp_workspace(d_rag) == 0
+    assert lib.tp_mlp_bwd_sp_workspace(d_fused) == 0
+    assert so.tp_mlp_fwd_sp(ctypes.byref(d_rag), arr(two), fake, fake, None, arr(two), None, None,
+                            fake, 1 << 30, None) == lib.TP_ERR_SHAPE
+    assert so.tp_mlp_fwd_sp(ctypes.byref(d_fused), arr(two), fake, fake, None, arr(two), None,
+                            None, fake, 1 << 30, None) == lib.TP_ERR_UNSUPPORTED
+    a_rag = lib.attn_desc(1, 9, 64, 4, 2, 16, 2)
+    assert lib.tp_attn_fwd_sp_workspace(a_rag) == 0
+    a_ok = lib.attn_desc(1, 8, 64, 4, 2, 16, 2)
+    assert lib.tp_attn_fwd_sp_workspace(a_ok) > lib.tp_attn_fwd_workspace(a_ok)
