@@ -18,6 +18,10 @@ What it computes, and where the method is stated:
                    "One collective": the residual add and the following normalization stay
                    replicated).
 * ``costmodel`` -- the pages' reduction-count and message-byte arithmetic.
+* ``moe``       -- the tensor-parallel mixture-of-experts block: replicated top-k router, SwiGLU
+                   experts and shared expert sharded in place, one block-level sum, bias once
+                   ("Tensor-parallel all-reduce count per transformer layer in MLX shard_linear",
+                   facts on MoE layers).
 * ``seqpar``    -- the sequence-parallel form of the collective: reduce-scatter of the partials
                    into token slices and all-gather of the slices ("Why tensor parallelism has to
                    stay in scale-up", "Where the 320 comes from").
@@ -30,4 +34,4 @@ Everything is float64 numpy; matrix products use numpy's matmul as a library pri
 error function comes from scipy.  No blocking, fusion or reordering beyond the stated formulas.
 """
 
-from . import mlp, attention, decode, costmodel, seqpar  # noqa: F401
+from . import mlp, attention, decode, costmodel, seqpar, moe  # noqa: F401

@@ -1,0 +1,106 @@
+"""Oracle for the tensor-parallel mixture-of-experts block (float64, CPU).
+
+Test infrastructure only (see the package docstring).
+
+Source (page title, section): "Tensor-parallel all-reduce count per transformer layer in MLX
+shard_linear" (llms-explorer), facts:
+* a MoE layer shards its routed experts ("switch_mlp") and its shared expert in place and the
+  MoE block makes one all_sum on its output;
+* the router stays replicated (Qwen3-MoE);
+* sharding the shared expert in place folds its output into the routed experts' sum, so routed
+  plus shared experts need one all_sum, not two;
+* the sharded-to-all linear adds its bias once, after the sum.
+
+Readings where the pages leave a step open:
+
+* Each expert is a SwiGLU feed-forward block, h = silu(x Wg) * (x Wu), y = h W2 (the block of
+  the MLP oracle), with its intermediate width F_e split column-wise into p shards like the
+  dense MLP ("shard in place").
+* Router: logits = x Wr (Wr of shape (d, E)); each token takes the k experts with the largest
+  logits (ties: the lower expert index first) and weights them by the softmax of those k logits
+  (softmax over all experts renormalised over the chosen k -- the same numbers).
+* The shared expert (optional) sees every token with weight 1; an optional bias is added once
+  to the sum.
+* Block output: y = sum_{j<k} w_j expert_{e_j}(x) + shared(x) + bias.  Shard i's partial is
+  shared_i(x) + sum_j w_j expert_{e_j, i}(x); the block's one reduction adds the p partials.
+"""
+
+import numpy as np
+
+from . import mlp
+
+
+def _f64(a):
+    return np.asarray(a, dtype=np.float64)
+
+
+def route(x, wr, k):
+    """Top-k routing.  Returns (idx [T, k] int, weights [T, k]) with idx[t] in descending logit
+    order (lower index first among equal logits) and weights[t] = softmax(logits[t, idx[t]])."""
+    logits = _f64(x) @ _f64(wr)
+    T, E = logits.shape
+    if not 1 <= k <= E:
+        raise ValueError("k must be in 1..E")
+    idx = np.zeros((T, k), dtype=np.int64)
+    w = np.zeros((T, k))
+    for t in range(T):
+        # stable sort on the negated logits: equal logits keep ascending expert order
+        order = np.argsort(-logits[t], kind="stable")[:k]
+        idx[t] = order
+        sel = logits[t, order]
+        e = np.exp(sel - sel.max())
+        w[t] = e / e.sum()
+    return idx, w
+
+
+def moe_forward(x, wr, experts, k, shared=None, bias=None, routing=None):
+    """Unsharded MoE block.  experts: list of (wg, wu, w2) per expert; shared: (wg, wu, w2) or
+    None; routing: (idx, weights) to use instead of route(x, wr, k)."""
+    x = _f64(x)
+    idx, w = routing if routing is not None else route(x, wr, k)
+    y = np.zeros((x.shape[0], x.shape[1]))
+    for t in range(x.shape[0]):
+        for j in range(idx.shape[1]):
+            wg, wu, w2 = experts[int(idx[t, j])]
+            y[t] += w[t, j] * mlp.mlp_forward(x[t:t + 1], wg, w2, "swiglu", wu)[0]
+    if shared is not None:
+        wg, wu, w2 = shared
+        y = y + mlp.mlp_forward(x, wg, w2, "swiglu", wu)
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return y
+
+
+def moe_forward_sharded(x, wr, experts, k, p, shared=None, bias=None, routing=None):
+    """Sharded reference mode (invariant tests only).  Shard i runs every expert (and the shared
+    expert) on its column slice of Wg/Wu and row slice of W2.  Returns (y, partials): partials[i]
+    is shard i's output and y = sum of the partials in order i = 0..p-1, plus the bias once."""
+    x = _f64(x)
+    idx, w = routing if routing is not None else route(x, wr, k)
+    T, d = x.shape
+    partials = []
+    for i in range(p):
+        part = np.zeros((T, d))
+        for t in range(T):
+            for j in range(idx.shape[1]):
+                wg, wu, w2 = experts[int(idx[t, j])]
+                f = _f64(wg).shape[1]
+                if f % p:
+                    raise ValueError("p must divide every expert's width")
+                c = slice(i * f // p, (i + 1) * f // p)
+                part[t] += w[t, j] * mlp.mlp_forward(x[t:t + 1], _f64(wg)[:, c], _f64(w2)[c, :],
+                                                     "swiglu", _f64(wu)[:, c])[0]
+        if shared is not None:
+            wg, wu, w2 = shared
+            f = _f64(wg).shape[1]
+            if f % p:
+                raise ValueError("p must divide the shared expert's width")
+            c = slice(i * f // p, (i + 1) * f // p)
+            part += mlp.mlp_forward(x, _f64(wg)[:, c], _f64(w2)[c, :], "swiglu", _f64(wu)[:, c])
+        partials.append(part)
+    y = np.zeros((T, d))
+    for part in partials:
+        y = y + part
+    if bias is not None:
+        y = y + _f64(bias)[None, :]
+    return y, partials

@@ -1,0 +1,114 @@
+"""Pins for the MoE oracle ("Tensor-parallel all-reduce count per transformer layer in MLX
+shard_linear", facts on MoE layers: experts and shared expert sharded in place, one block-level
+sum, router replicated, bias added once after the sum).
+
+They use hand-computed routing, scipy's softmax, the dense MLP oracle (pinned on its own), brute
+force and the sharding invariants; none re-types the oracle's formulas.
+"""
+import math
+
+import numpy as np
+import pytest
+from scipy.special import softmax
+
+from oracle import mlp, moe
+
+
+def _case(T=6, d=8, E=4, F=8, seed=0, shared=True):
+    r = np.random.default_rng(seed)
+    x = r.standard_normal((T, d))
+    wr = r.standard_normal((d, E))
+    experts = [tuple(r.standard_normal(s) / math.sqrt(s[0]) for s in ((d, F), (d, F), (F, d)))
+               for _ in range(E)]
+    sh = tuple(r.standard_normal(s) / math.sqrt(s[0]) for s in ((d, F), (d, F), (F, d))) if shared else None
+    return x, wr, experts, sh
+
+
+def test_routing_by_hand():
+    # x picks rows of Wr: logits are known exactly
+    wr = np.array([[1.0, 3.0, 2.0, 0.0],
+                   [0.5, 0.5, 4.0, 1.0]])
+    x = np.array([[1.0, 0.0], [0.0, 1.0]])
+    idx, w = moe.route(x, wr, 2)
+    assert idx.tolist() == [[1, 2], [2, 3]]
+    # weights: softmax of the two chosen logits, e.g. e^3 / (e^3 + e^2)
+    assert abs(w[0, 0] - math.exp(3) / (math.exp(3) + math.exp(2))) < 1e-15
+    assert abs(w[1, 1] - math.exp(1) / (math.exp(4) + math.exp(1))) < 1e-15
+    np.testing.assert_allclose(w.sum(axis=1), 1.0, rtol=0, atol=1e-15)
+
+
+def test_routing_ties_take_lower_index():
+    wr = np.array([[2.0, 5.0, 5.0, 5.0]])
+    idx, w = moe.route(np.array([[1.0]]), wr, 2)
+    assert idx.tolist() == [[1, 2]]
+    assert w.tolist() == [[0.5, 0.5]]
+
+
+def test_k_equals_E_is_full_softmax_mixture():
+    x, wr, experts, _ = _case(shared=False)
+    E = len(experts)
+    y = moe.moe_forward(x, wr, experts, E)
+    g = softmax(x @ wr, axis=1)
+    want = sum(g[:, e:e + 1] * mlp.mlp_forward(x, ex[0], ex[2], "swiglu", ex[1])
+               for e, ex in enumerate(experts))
+    np.testing.assert_allclose(y, want, rtol=1e-12, atol=1e-13)
+
+
+def test_one_expert_is_the_dense_mlp():
+    x, wr, experts, _ = _case(E=1, shared=False)
+    y = moe.moe_forward(x, wr, experts, 1)
+    wg, wu, w2 = experts[0]
+    np.testing.assert_allclose(y, mlp.mlp_forward(x, wg, w2, "swiglu", wu), rtol=1e-13)
+
+
+def test_brute_force_top1():
+    # k = 1: each token's output is exactly its arg-max expert's block (weight 1)
+    x, wr, experts, _ = _case(shared=False, seed=3)
+    y = moe.moe_forward(x, wr, experts, 1)
+    for t in range(x.shape[0]):
+        logits = [sum(x[t, i] * wr[i, e] for i in range(x.shape[1])) for e in range(wr.shape[1])]
+        e = max(range(len(logits)), key=lambda j: (logits[j], -j))
+        wg, wu, w2 = experts[e]
+        np.testing.assert_allclose(y[t], mlp.mlp_forward(x[t:t + 1], wg, w2, "swiglu", wu)[0],
+                                   rtol=1e-13)
+
+
+@pytest.mark.parametrize("p", [1, 2, 4, 8])
+def test_sharded_sum_equals_unsharded(p):
+    x, wr, experts, sh = _case(seed=4)
+    bias = np.arange(x.shape[1], dtype=np.float64)
+    y, parts = moe.moe_forward_sharded(x, wr, experts, 2, p, shared=sh, bias=bias)
+    assert len(parts) == p   # one partial per shard: one block-level reduction
+    np.testing.assert_allclose(y, moe.moe_forward(x, wr, experts, 2, shared=sh, bias=bias),
+                               rtol=1e-12, atol=1e-12)
+
+
+def test_shared_expert_folds_into_the_one_sum():
+    x, wr, experts, sh = _case(seed=5)
+    routed = moe.moe_forward(x, wr, experts, 2)
+    both = moe.moe_forward(x, wr, experts, 2, shared=sh)
+    np.testing.assert_allclose(both - routed, mlp.mlp_forward(x, sh[0], sh[2], "swiglu", sh[1]),
+                               rtol=1e-12, atol=1e-13)
+    # sharded: the shared expert's slice is inside each shard's partial, no second sum
+    _, parts = moe.moe_forward_sharded(x, wr, experts, 2, 2, shared=sh)
+    _, parts_r = moe.moe_forward_sharded(x, wr, experts, 2, 2)
+    shared_parts = [p_ - q_ for p_, q_ in zip(parts, parts_r)]
+    np.testing.assert_allclose(sum(shared_parts), mlp.mlp_forward(x, sh[0], sh[2], "swiglu", sh[1]),
+                               rtol=1e-12, atol=1e-13)
+
+
+def test_bias_added_once_after_the_sum():
+    x, wr, experts, sh = _case(seed=6)
+    bias = np.full(x.shape[1], 0.25)
+    y0, _ = moe.moe_forward_sharded(x, wr, experts, 2, 4, shared=sh)
+    y1, _ = moe.moe_forward_sharded(x, wr, experts, 2, 4, shared=sh, bias=bias)
+    np.testing.assert_allclose(y1 - y0, np.broadcast_to(bias, y0.shape), rtol=0, atol=1e-14)
+
+
+def test_given_routing_is_used():
+    x, wr, experts, _ = _case(seed=7)
+    idx = np.tile(np.array([[3, 0]]), (x.shape[0], 1))
+    w = np.tile(np.array([[0.75, 0.25]]), (x.shape[0], 1))
+    y = moe.moe_forward(x, wr, experts, 2, routing=(idx, w))
+    f = lambda e: mlp.mlp_forward(x, experts[e][0], experts[e][2], "swiglu", experts[e][1])
+    np.testing.assert_allclose(y, 0.75 * f(3) + 0.25 * f(0), rtol=1e-13)
