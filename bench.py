@@ -386,7 +386,64 @@ def run_extras(args, tp, inputs, torch, stream, peaks):
     if "seqpar" in which:
         time.sleep(1.0)
         ex["seqpar_prefill_mlp_fwd"] = extra_seqpar(tp, inputs, torch, stream, peaks, steps)
+    if "moe" in which:
+        time.sleep(1.0)
+        ex["moe_layer"] = extra_moe(tp, inputs, torch, stream, peaks, steps)
     return ex
+
+
+def extra_moe(tp, inputs, torch, stream, peaks, steps):
+    """A DeepSeek-V3-shaped MoE layer (hidden 7168, 256 routed experts of width 2048, top-8, one
+    shared expert of width 2048; the pages' 7168 hidden size and MoE facts), p=8, bf16 weights
+    N(0, 0.02), router N(0, 1/sqrt(d)): the prefill forward at T=4096 and a decode step at T=64."""
+    dev = torch.device("cuda", torch.cuda.current_device())
+    d, E, k, F, Fs, p = 7168, 256, 8, 2048, 2048, 8
+    out = {"workload": "TP MoE layer: d=7168, 256 experts x d_ff 2048, top-8, shared expert "
+                       "d_ff 2048, p=8, bf16"}
+    desc0 = tp.moe_desc(4096, d, F, Fs, E, k, p)
+    w1p = torch.empty(E * tp.tp_moe_expert_w1_bytes(desc0) // 2, dtype=torch.bfloat16, device=dev)
+    w2p = torch.empty(E * tp.tp_moe_expert_w2_bytes(desc0) // 2, dtype=torch.bfloat16, device=dev)
+    w1s = torch.empty(tp.tp_moe_shared_w1_bytes(desc0) // 2, dtype=torch.bfloat16, device=dev)
+    w2s = torch.empty(tp.tp_moe_shared_w2_bytes(desc0) // 2, dtype=torch.bfloat16, device=dev)
+    e1, e2 = tp.tp_moe_expert_w1_bytes(desc0) // 2, tp.tp_moe_expert_w2_bytes(desc0) // 2
+    # each expert packs like the dense SwiGLU MLP (tp_moe_pack's layout); drawn and packed one at
+    # a time so that the unpacked weights never all sit on the device
+    ed = tp.mlp_desc(1, d, F, p, "swiglu", "bf16")
+    for e in range(E):
+        g_, u_, o_ = (inputs.normal(s_, 0.02, 0, 1000 + 3 * e + j, "bf16", dev)
+                      for j, s_ in enumerate(((d, F), (d, F), (F, d))))
+        tp.tp_mlp_pack(ed, g_, u_, o_, w1p[e * e1:(e + 1) * e1], w2p[e * e2:(e + 1) * e2])
+    sg, su, so = (inputs.normal(s_, 0.02, 0, 900 + j, "bf16", dev)
+                  for j, s_ in enumerate(((d, Fs), (d, Fs), (Fs, d))))
+    tp.tp_mlp_pack(tp.mlp_desc(1, d, Fs, p, "swiglu", "bf16"), sg, su, so, w1s, w2s)
+    del sg, su, so
+    wr = inputs.normal((d, E), 1.0 / d ** 0.5, 0, 901, "bf16", dev)
+    fl_per_row = 2.0 * d * 3 * F
+    for T, name in ((4096, "prefill"), (64, "decode")):
+        desc = tp.moe_desc(T, d, F, Fs, E, k, p)
+        x = inputs.normal((T, d), 1.0, 0, 902, "bf16", dev)
+        y = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+        ws = torch.empty(tp.tp_moe_fwd_workspace(desc), dtype=torch.uint8, device=dev)
+
+        def fwd():
+            tp.tp_moe_fwd(desc, x, wr, w1p, w2p, y, w1p_s=w1s, w2p_s=w2s, residual=x, workspace=ws)
+
+        for _ in range(3):
+            fwd()
+        ms = _cuda_time(fwd, steps, stream) / steps
+        prof = _profile(tp, fwd, steps)
+        flops = T * k * fl_per_row + T * 2.0 * d * 3 * Fs + 2.0 * T * d * E
+        out[name] = {"T": T, "ms": round(ms, 3),
+                     "TFLOP_per_s": round(flops / (ms / 1e3) / 1e12, 1),
+                     "frac_of_burst_peak": round(flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
+                     "tokens_per_s": round(T / (ms / 1e3), 1),
+                     "kernels": {kk: {"ms_per_launch": round(v[1] / v[0], 4)} for kk, v in prof.items()}}
+        del ws, x, y
+        torch.cuda.empty_cache()
+    out["steps"] = steps
+    del w1p, w2p, w1s, w2s
+    torch.cuda.empty_cache()
+    return out
 
 
 def extra_seqpar(tp, inputs, torch, stream, peaks, steps):

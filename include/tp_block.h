@@ -254,6 +254,56 @@ tp_status tp_rmsnorm(const void* x, int32_t x_dtype, int64_t rows, int64_t d, fl
                      void* out, int32_t out_dtype, void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* Mixture of experts                                                                          */
+/* ------------------------------------------------------------------------------------------ */
+/* "Tensor-parallel all-reduce count per transformer layer in MLX shard_linear" (llms-explorer),
+ * facts on MoE layers: the router is replicated; the routed experts and the shared expert are
+ * sharded in place; the block makes ONE sum of the shards' outputs (the shared expert's slice
+ * folded in); the bias is added once, after the sum.  Readings: every expert is a SwiGLU block,
+ * sharded over p like the dense MLP; a token takes the top_k experts with the largest router
+ * logits (ties: lower index) weighted by the softmax of those k logits.
+ *   y = residual + bias + sum_{i<p} [ shared_i(x) + sum_{j<k} w_j expert_{e_j,i}(x) ]
+ * bf16 only; d and n_experts multiples of 8; top_k <= 8; p divides d_ff and d_ff_shared. */
+typedef struct {
+  int64_t T;            /* tokens                                                             */
+  int64_t d;            /* hidden size                                                        */
+  int64_t d_ff;         /* each routed expert's intermediate size                             */
+  int64_t d_ff_shared;  /* the shared expert's intermediate size (0: no shared expert)        */
+  int32_t n_experts;    /* E                                                                  */
+  int32_t top_k;        /* experts per token                                                  */
+  int32_t p;            /* logical shards                                                     */
+  int32_t dtype;        /* TP_BF16                                                            */
+  int32_t flags;        /* 0                                                                  */
+  int32_t reserved;
+} tp_moe_desc;
+
+/* Packed bytes of ONE routed expert (the dense MLP's packed layout for d, d_ff, p, SWIGLU; the E
+ * experts' packings lie back to back: w1p [E][...], w2p [E][...]) and of the shared expert. */
+size_t tp_moe_expert_w1_bytes(const tp_moe_desc* desc);
+size_t tp_moe_expert_w2_bytes(const tp_moe_desc* desc);
+size_t tp_moe_shared_w1_bytes(const tp_moe_desc* desc);
+size_t tp_moe_shared_w2_bytes(const tp_moe_desc* desc);
+
+/* Pack the experts.  wg, wu, w2: HOST arrays of E device pointers to expert e's Wg, Wu [d][d_ff]
+ * and W2 [d_ff][d] (bf16, input-major); wg_s, wu_s, w2_s: the shared expert (ignored when
+ * d_ff_shared == 0).  w1p, w2p: E * tp_moe_expert_w{1,2}_bytes; w1p_s, w2p_s: the shared sizes. */
+tp_status tp_moe_pack(const tp_moe_desc* desc, const void* const* wg, const void* const* wu,
+                      const void* const* w2, const void* wg_s, const void* wu_s, const void* w2_s,
+                      void* w1p, void* w2p, void* w1p_s, void* w2p_s, void* stream);
+
+/* Forward of the MoE block.  x [T][d]; wr [d][E] router weights (bf16, replicated, not packed);
+ * bias [d] and residual [T][d] optional; y [T][d] bf16.  route_idx (int32 [T][top_k]) and route_w
+ * (fp32 [T][top_k]) receive the routing when non-null (descending logit order).  Routing,
+ * dispatch, the grouped expert GEMMs, the shared expert and the one reduction all run on the
+ * device; nothing is read back to the host.  workspace: tp_moe_fwd_workspace(desc) bytes.  Adds 1
+ * to the reduction counter. */
+size_t tp_moe_fwd_workspace(const tp_moe_desc* desc);
+tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr, const void* w1p,
+                     const void* w2p, const void* w1p_s, const void* w2p_s, const void* bias,
+                     const void* residual, void* y, void* route_idx, void* route_w,
+                     void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Sequence parallelism                                                                        */
 /* ------------------------------------------------------------------------------------------ */
 /* "Why tensor parallelism has to stay in scale-up" (Keysight), "Where the 320 comes from": with

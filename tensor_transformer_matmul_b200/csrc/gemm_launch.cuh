@@ -106,6 +106,14 @@ struct StreamKArgs {
 struct GemmOpts {
   const StreamKArgs* sk = nullptr;   // stream-K schedule (else whole tiles)
   bool rotate_k = false;             // tile-dependent k-loop start (weight streaming)
+  // grouped problems (see GemmParams): device arrays of the n groups' row counts, first rows
+  // and 128-row block prefix (n + 1 entries); M is then the largest group's row count
+  const int32_t* grp_cnt = nullptr;
+  const int32_t* grp_off = nullptr;
+  const int32_t* grp_mbp = nullptr;
+  int grp_n = 0;
+  int grp_div = 1;
+  bool grp_sum = false;   // sum each group's grp_div problems into one output (in order)
 };
 
 // Launch gemm_kernel<Cfg, Epi> over ``batch`` problems of D = A B^T (M x N, contraction K).
@@ -149,6 +157,16 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   gp.slots = nullptr;
   gp.counters = nullptr;
   gp.rotate_k = opts.rotate_k ? 1 : 0;
+  gp.grp_cnt = opts.grp_cnt;
+  gp.grp_off = opts.grp_off;
+  gp.grp_mbp = opts.grp_mbp;
+  gp.grp_n = opts.grp_n;
+  gp.grp_div = opts.grp_div > 0 ? opts.grp_div : 1;
+  if (opts.grp_cnt && opts.grp_sum) gp.sum_batch = 1;
+  if (opts.grp_cnt && (sk || Cfg::A_MN || Cfg::A_ROWS != 128 || !opts.grp_off || !opts.grp_mbp ||
+                       opts.grp_n < 1 || batch != static_cast<int64_t>(opts.grp_n) * gp.grp_div))
+    return set_error(TP_ERR_INVALID_ARG,
+                     "grouped GEMM: whole 128-row tiles, K-major A, n groups x grp_div problems");
   int grid_sk = 0;
   if (sk) {
     const SkPlan pl = plan_stream_k<Cfg>(M, N, K, batch, sk->sum_batch, num_sms());

@@ -95,6 +95,19 @@ struct GemmParams {
   // which spreads the loads over the HBM channels instead of having every CTA hit the same
   // offset within the row pitch at the same moment.
   int32_t rotate_k;
+  // Grouped problems (mixture of experts; whole tiles only): problem b belongs to group
+  // e = b / grp_div, whose A rows are rows grp_off[e] .. grp_off[e] + grp_cnt[e] - 1 of one
+  // K-major A, read at A batch coordinate b % grp_div.  grp_mbp[e] = sum over groups < e of
+  // their 128-row blocks (grp_mbp[grp_n] = all of them), so the tiles that hold rows are
+  // enumerated directly: tile t -> (block of all groups' blocks, shard, N block), its group found
+  // by binary search.  With sum_batch the grp_div problems of a group are summed into one output:
+  // a tile's k loop runs problem e*grp_div's k-blocks, then e*grp_div+1's, ... (the shard sum in
+  // the accumulator) and the tile space drops the problem index.  grp_cnt == nullptr: ungrouped.
+  const int32_t* grp_cnt;
+  const int32_t* grp_off;
+  const int32_t* grp_mbp;
+  int32_t grp_n;
+  int32_t grp_div;
 };
 
 // One accumulator's worth of work.
@@ -105,14 +118,18 @@ struct Seg {
   int kb0, kb1;   // k-block range
   int local;      // index of this segment within its CTA (slot index)
   int rot;        // the k loop visits kb0 + (i + rot) % (kb1 - kb0), i = 0, 1, ...
+  int ab;         // A batch coordinate
+  int row0;       // first A row of the problem (grouped), else 0
+  int row_end;    // end of the problem's A rows (grouped), else INT32_MAX
 };
 
 // What the epilogue of one tile sees.
 struct EpiCtx {
   int row;          // accumulator row (A row within the tile) held by this thread, 0..127
-  int b;            // problem index (0 when the problems were summed)
+  int b;            // problem index (0 when the problems were summed; A batch when grouped)
   int m0;           // first A row of the tile
   int n0;           // first B row of the tile
+  int row_end = 0x7fffffff;   // A rows at or past this belong to no problem of the tile
 };
 
 __device__ __forceinline__ void decode_mn(int r, const GemmParams& gp, int& mb, int& nb) {
@@ -149,6 +166,10 @@ struct SegIter {
     if (gp.stream_k) {
       u = cta_start(cta, gp, grid);
       end = cta_start(cta + 1, gp, grid);
+    } else if (gp.grp_cnt) {
+      u = cta;
+      end = static_cast<int64_t>(gp.grp_mbp[gp.grp_n]) * (gp.sum_batch ? 1 : gp.grp_div) *
+            gp.n_blocks;
     } else {
       u = cta;
       end = num_groups(gp);
@@ -157,17 +178,40 @@ struct SegIter {
   __device__ __forceinline__ bool next(const GemmParams& gp, int grid, Seg& s) {
     if (u >= end) return false;
     if (!gp.stream_k) {
-      const int per = gp.m_blocks * gp.n_blocks;
       s.g = static_cast<int>(u);
-      s.b = s.g / per;
-      decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
+      u += grid;
+      if (gp.grp_cnt) {
+        s.nb = s.g % gp.n_blocks;
+        const int r = s.g / gp.n_blocks;
+        const int i = gp.sum_batch ? 0 : r % gp.grp_div;
+        const int mbg = gp.sum_batch ? r : r / gp.grp_div;
+        int lo = 0, hi = gp.grp_n;   // the last group whose first block is <= mbg
+        while (hi - lo > 1) {
+          const int mid = (lo + hi) >> 1;
+          if (gp.grp_mbp[mid] <= mbg) lo = mid;
+          else hi = mid;
+        }
+        s.mb = mbg - gp.grp_mbp[lo];
+        s.b = lo * gp.grp_div + i;
+        s.ab = i;
+        s.row0 = gp.grp_off[lo];
+        s.row_end = s.row0 + gp.grp_cnt[lo];
+      } else {
+        const int per = gp.m_blocks * gp.n_blocks;
+        s.b = s.g / per;
+        decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
+        s.ab = s.b;
+        s.row0 = 0;
+        s.row_end = 0x7fffffff;
+      }
       s.kb0 = 0;
-      s.kb1 = gp.k_blocks;
+      s.kb1 = (gp.grp_cnt && gp.sum_batch) ? gp.grp_div * gp.k_blocks : gp.k_blocks;
       s.local = local++;
       s.rot = gp.rotate_k ? static_cast<int>((static_cast<int64_t>(s.g) * 37) % gp.k_blocks) : 0;
-      u += grid;
       return true;
     }
+    s.row0 = 0;
+    s.row_end = 0x7fffffff;
     const int64_t U = units_per_group(gp);
     const int64_t g = u / U, o = u - g * U;
     s.g = static_cast<int>(g);
@@ -188,6 +232,7 @@ struct SegIter {
     s.kb1 = s.kb0 + static_cast<int>(seg_end - o);
     s.local = local++;
     s.rot = gp.rotate_k ? static_cast<int>((static_cast<int64_t>(s.g) * 37) % (s.kb1 - s.kb0)) : 0;
+    s.ab = s.b;
     u = g * U + seg_end;
     return true;
   }
@@ -379,9 +424,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       it.init(gp, blockIdx.x, grid);
       Seg sg;
       while (ok && it.next(gp, grid, sg)) {
-        const int m0 = sg.mb * Cfg::A_ROWS;
+        const int m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
         const int n0 = sg.nb * Cfg::BN;
-        const int za = gp.a_batched ? sg.b : 0;
+        const int za = gp.a_batched ? sg.ab : 0;
         const int zb = gp.b_batched ? sg.b : 0;
         const int nk = sg.kb1 - sg.kb0;
         for (int i = 0; i < nk; ++i) {
@@ -392,22 +437,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             break;
           }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          const int k0 = kb * kBK;
+          // grouped sum: k steps past the first problem's k-blocks belong to the next problems
+          const int pi = kb / gp.k_blocks;
+          const int k0 = (kb - pi * gp.k_blocks) * kBK;
+          const int zai = gp.a_batched ? za + pi : 0;
+          const int zbi = gp.b_batched ? zb + pi : 0;
           uint8_t* sa = a_smem + stage * Cfg::A_STAGE_BYTES;
           uint8_t* sb = b_smem + stage * Cfg::B_STAGE_BYTES;
           if (Cfg::A_MN) {
 #pragma unroll
             for (int j = 0; j < Cfg::A_ROWS / 64; ++j)
-              tma_load_3d(&tma_a, &full[stage], sa + j * 64 * kBK * 2, m0 + 64 * j, k0, za);
+              tma_load_3d(&tma_a, &full[stage], sa + j * 64 * kBK * 2, m0 + 64 * j, k0, zai);
           } else {
-            tma_load_3d(&tma_a, &full[stage], sa, k0, m0, za);
+            tma_load_3d(&tma_a, &full[stage], sa, k0, m0, zai);
           }
           if (Cfg::B_MN) {
 #pragma unroll
             for (int j = 0; j < Cfg::BN / 64; ++j)
-              tma_load_3d(&tma_b, &full[stage], sb + j * 64 * kBK * 2, n0 + 64 * j, k0, zb);
+              tma_load_3d(&tma_b, &full[stage], sb + j * 64 * kBK * 2, n0 + 64 * j, k0, zbi);
           } else {
-            tma_load_3d(&tma_b, &full[stage], sb, k0, n0, zb);
+            tma_load_3d(&tma_b, &full[stage], sb, k0, n0, zbi);
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -511,9 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       tsrc.taddr = tmem_base + acc * Cfg::ACC_COLS + (static_cast<uint32_t>(quarter * 32) << 16);
       EpiCtx ctx;
       ctx.row = row;
-      ctx.b = gp.sum_batch ? 0 : sg.b;
-      ctx.m0 = sg.mb * Cfg::A_ROWS;
+      ctx.b = gp.sum_batch ? 0 : (gp.grp_cnt ? sg.ab : sg.b);
+      ctx.m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
       ctx.n0 = sg.nb * Cfg::BN;
+      ctx.row_end = sg.row_end;
       // the tile is whole when all its k-blocks lie in this CTA's range (then it is one segment)
       const int64_t g0 = static_cast<int64_t>(sg.g) * U;
       const bool whole = !gp.stream_k ||
@@ -626,7 +676,7 @@ struct EpiHidden {
     const bool swiglu = p.act == TP_ACT_SWIGLU;
     if (!p.swap) {
       const int t = c.m0 + c.row;
-      const bool live = t < p.tokens;
+      const bool live = t < p.tokens && t < c.row_end;
       if (swiglu) {
         // BN == 256, n0 multiple of 256
         const int blk = c.n0 >> 8;
@@ -735,7 +785,7 @@ struct EpiStoreF32 {
     float* base = p.out + static_cast<int64_t>(c.b) * p.batch_stride;
     if (!p.swap) {
       const int i = c.m0 + c.row;
-      const bool live = i < p.rows_valid;
+      const bool live = i < p.rows_valid && i < c.row_end;
 #pragma unroll 1
       for (int col = 0; col < Cfg::BN; col += 32) {
         float v[32];

@@ -1,0 +1,239 @@
+// Kernels of the tensor-parallel mixture-of-experts block (routing, dispatch, combine).
+//
+// "Tensor-parallel all-reduce count per transformer layer in MLX shard_linear" (llms-explorer),
+// facts on MoE layers: the router stays replicated, the routed experts and the shared expert are
+// sharded in place, and the block makes one sum of the shards' outputs (the shared expert's slice
+// folded in); a sharded-to-all linear adds its bias once, after the sum.
+//
+// Per call, on the device:
+//   logits = x Wr (tcgen05 GEMM, fp32)  ->  top-k per token, weights = softmax of the k chosen
+//   logits  ->  per expert, its (token, choice) entries in token order (counts, offsets, a stable
+//   position for every entry)  ->  gather of the routed token rows into expert order  ->  grouped
+//   up / down GEMMs over all experts (gemm_tc.cuh, grouped mode; the down GEMM runs the p shards'
+//   k-blocks of a row tile into one accumulator, so the shard sum -- the block's one reduction --
+//   happens there, as it does in the shared expert's fused down GEMM)  ->  one combine: shared
+//   expert + weighted routed rows (choices in order) + bias, then the residual.
+#pragma once
+
+#include "tp_common.cuh"
+
+namespace tp {
+namespace moe {
+
+constexpr int kMaxTopK = 8;
+
+// Router logits for few experts (E not a multiple of 64): block t, thread q*E + e sums
+// x[t][k] Wr[k][e] over k = q, q + Q, ... (Q = blockDim / E; consecutive threads read
+// consecutive Wr elements), then thread e adds the Q partial sums in order.  fp32.
+__global__ void __launch_bounds__(256) router_simt_kernel(const __nv_bfloat16* __restrict__ x,
+                                                          const __nv_bfloat16* __restrict__ wr,
+                                                          int64_t d, int E,
+                                                          float* __restrict__ logits) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ float part[256];
+  const int64_t t = blockIdx.x;
+  const int Q = static_cast<int>(blockDim.x) / E;
+  const int e = threadIdx.x % E, q = threadIdx.x / E;
+  float acc = 0.f;
+  if (q < Q)
+    for (int64_t k = q; k < d; k += Q)
+      acc = fmaf(__bfloat162float(x[t * d + k]), __bfloat162float(wr[k * E + e]), acc);
+  part[threadIdx.x] = acc;
+  __syncthreads();
+  if (threadIdx.x < E) {
+    float v = 0.f;
+    for (int j = 0; j < Q; ++j) v += part[j * E + threadIdx.x];
+    logits[t * E + threadIdx.x] = v;
+  }
+}
+
+// One thread per token: the k largest logits (descending; among equal logits the lower expert
+// index first) and their softmax.
+__global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
+                                                   int E, int k, int32_t* __restrict__ idx,
+                                                   float* __restrict__ w) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (t >= T) return;
+  const float* l = logits + t * E;
+  float best[kMaxTopK];
+  int bi[kMaxTopK];
+#pragma unroll
+  for (int j = 0; j < kMaxTopK; ++j) {
+    best[j] = -INFINITY;
+    bi[j] = j;
+  }
+  for (int e = 0; e < E; ++e) {
+    const float v = l[e];
+    if (!(v > best[k - 1]) && e >= k) continue;   // not above the k-th (ties keep the lower index)
+    // insertion: after every kept entry with a logit >= v
+    int pos = k - 1;
+    while (pos > 0 && best[pos - 1] < v) {
+      best[pos] = best[pos - 1];
+      bi[pos] = bi[pos - 1];
+      --pos;
+    }
+    best[pos] = v;
+    bi[pos] = e;
+  }
+  float s = 0.f, ex[kMaxTopK];
+  for (int j = 0; j < k; ++j) {
+    ex[j] = expf(best[j] - best[0]);
+    s += ex[j];
+  }
+  for (int j = 0; j < k; ++j) {
+    idx[t * k + j] = bi[j];
+    w[t * k + j] = ex[j] / s;
+  }
+}
+
+__device__ __forceinline__ int block_sum_int(int v, int* red) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = v;
+  __syncthreads();
+  int tot = 0;
+  for (int i = 0; i < static_cast<int>(blockDim.x >> 5); ++i) tot += red[i];
+  __syncthreads();
+  return tot;
+}
+
+// Block e: cnt[e] = number of entries routed to expert e.
+__global__ void __launch_bounds__(1024) count_kernel(const int32_t* __restrict__ idx,
+                                                     int64_t n_entries, int32_t* __restrict__ cnt) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int red[32];
+  const int e = blockIdx.x;
+  int c = 0;
+  for (int64_t i = threadIdx.x; i < n_entries; i += blockDim.x) c += idx[i] == e ? 1 : 0;
+  c = block_sum_int(c, red);
+  if (threadIdx.x == 0) cnt[e] = c;
+}
+
+// Block e: off[e] = sum of the counts of experts < e and mbp[e] = sum of their block_rows-row
+// blocks (the last block also writes mbp[E], the total); then every entry routed to e gets the
+// next position in entry order: perm[off + pos] = entry, inv[entry] = off + pos (a stable order,
+// so the dispatch is deterministic).
+__global__ void __launch_bounds__(1024) position_kernel(const int32_t* __restrict__ idx,
+                                                        int64_t n_entries,
+                                                        const int32_t* __restrict__ cnt,
+                                                        int block_rows,
+                                                        int32_t* __restrict__ off,
+                                                        int32_t* __restrict__ mbp,
+                                                        int32_t* __restrict__ perm,
+                                                        int32_t* __restrict__ inv) {
+  pdl_wait();
+  pdl_trigger();
+  __shared__ int red[32];
+  __shared__ int warp_pre[32];
+  const int e = blockIdx.x;
+  int o = 0, nb = 0;
+  for (int i = threadIdx.x; i < e; i += blockDim.x) {
+    o += cnt[i];
+    nb += (cnt[i] + block_rows - 1) / block_rows;
+  }
+  const int base0 = block_sum_int(o, red);
+  const int blocks0 = block_sum_int(nb, red);
+  if (threadIdx.x == 0) {
+    off[e] = base0;
+    mbp[e] = blocks0;
+    if (e == static_cast<int>(gridDim.x) - 1) mbp[e + 1] = blocks0 + (cnt[e] + block_rows - 1) / block_rows;
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int base = base0;
+  for (int64_t c0 = 0; c0 < n_entries; c0 += blockDim.x) {
+    const int64_t i = c0 + threadIdx.x;
+    const bool hit = i < n_entries && idx[i] == e;
+    const unsigned m = __ballot_sync(0xffffffffu, hit);
+    if (lane == 0) warp_pre[warp] = __popc(m);
+    __syncthreads();
+    int before = 0, total = 0;
+    for (int q = 0; q < nw; ++q) {
+      const int v = warp_pre[q];
+      if (q < warp) before += v;
+      total += v;
+    }
+    if (hit) {
+      const int slot = base + before + __popc(m & ((1u << lane) - 1u));
+      perm[slot] = static_cast<int32_t>(i);
+      inv[i] = slot;
+    }
+    base += total;
+    __syncthreads();   // warp_pre is rewritten by the next chunk
+  }
+}
+
+// xs[r] = x[perm[r] / k] for the n_rows routed rows: one block per row, 16-byte words (d % 8 == 0).
+__global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __restrict__ x,
+                                                     const int32_t* __restrict__ perm, int k,
+                                                     int64_t d, __nv_bfloat16* __restrict__ xs) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t r = blockIdx.x;
+  const int64_t t = perm[r] / k;
+  const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
+  uint4* dst = reinterpret_cast<uint4*>(xs + r * d);
+  for (int64_t j = threadIdx.x; j < d / 8; j += blockDim.x) dst[j] = src[j];
+}
+
+// y[t] = residual[t] + ((shared[t] + sum_{j<k} w[t][j] * routed[inv[t k + j]]) + bias): the
+// routed rows and the shared expert arrive with their p shards already summed (in order, inside
+// their GEMMs' accumulators); the choices are added in order, all in fp32 with one rounding.
+// 8 consecutive columns per thread (d % 8 == 0).
+__global__ void __launch_bounds__(256) combine_kernel(
+    const float* __restrict__ routed, const float* __restrict__ shared,
+    const int32_t* __restrict__ inv, const float* __restrict__ w, int k, int64_t T, int64_t d,
+    const __nv_bfloat16* __restrict__ bias, const __nv_bfloat16* residual, __nv_bfloat16* y) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t nv = T * (d / 8);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < nv; q += stride) {
+    const int64_t t = q / (d / 8);
+    const int64_t c = (q - t * (d / 8)) * 8;
+    float acc[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = 0.f;
+    if (shared) {
+      const float4* s4 = reinterpret_cast<const float4*>(shared + t * d + c);
+      const float4 a = s4[0], b = s4[1];
+      acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
+      acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
+    }
+    for (int j = 0; j < k; ++j) {
+      const float wt = w[t * k + j];
+      const int64_t rr = inv[t * k + j];
+      const float4* r4 = reinterpret_cast<const float4*>(routed + rr * d + c);
+      const float4 a = r4[0], b = r4[1];
+      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wt, v[e], acc[e]);
+    }
+    if (bias) {
+      const uint4 bw = *reinterpret_cast<const uint4*>(bias + c);
+      const float bv[8] = {bf16lo(bw.x), bf16hi(bw.x), bf16lo(bw.y), bf16hi(bw.y),
+                           bf16lo(bw.z), bf16hi(bw.z), bf16lo(bw.w), bf16hi(bw.w)};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += bv[e];
+    }
+    if (residual) {
+      const uint4 rw = *reinterpret_cast<const uint4*>(residual + t * d + c);
+      const float rv[8] = {bf16lo(rw.x), bf16hi(rw.x), bf16lo(rw.y), bf16hi(rw.y),
+                           bf16lo(rw.z), bf16hi(rw.z), bf16lo(rw.w), bf16hi(rw.w)};
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = rv[e] + acc[e];
+    }
+    uint4 o;
+    o.x = pack_bf16x2(acc[0], acc[1]);
+    o.y = pack_bf16x2(acc[2], acc[3]);
+    o.z = pack_bf16x2(acc[4], acc[5]);
+    o.w = pack_bf16x2(acc[6], acc[7]);
+    *reinterpret_cast<uint4*>(y + t * d + c) = o;
+  }
+}
+
+}  // namespace moe
+}  // namespace tp

@@ -14,6 +14,7 @@
 
 #include "gemm_launch.cuh"
 #include "gemm_pair.cuh"
+#include "moe.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
 #include "seqpar.cuh"
@@ -713,4 +714,260 @@ extern "C" tp_status tp_mlp_bwd_sp(const tp_mlp_desc* desc, const void* const* d
                               L.norm_eps, s);
   if (st == TP_OK) count_reduction();
   return st;
+}
+
+// ------------------------------------------------------------------ mixture of experts
+// "Tensor-parallel all-reduce count per transformer layer in MLX shard_linear" (llms-explorer),
+// facts on MoE layers: replicated router, routed and shared experts sharded in place, one
+// block-level sum, bias once after the sum.  Every expert is a SwiGLU block packed exactly like
+// the dense MLP (tp_mlp_pack's layout for d, d_ff, p); the E experts' packings lie back to back.
+namespace {
+struct MoeLayout {
+  int64_t T, d, F, Fsh, n_rows;
+  int E, k, p;
+  MlpLayout ex;       // one routed expert as an MLP block (T = routed rows)
+  MlpLayout sh;       // the shared expert over the T tokens (valid when Fsh > 0)
+  size_t logits_off, idx_off, w_off, cnt_off, off_off, mbp_off, perm_off, inv_off, xs_off,
+      hs_off, part_off, shared_off, shared_y_off, bytes;
+};
+
+tp_status moe_layout(const tp_moe_desc* desc, MoeLayout* M) {
+  if (!desc) return set_error(TP_ERR_INVALID_ARG, "desc is null");
+  if (desc->dtype != TP_BF16) return set_error(TP_ERR_UNSUPPORTED, "the MoE block is bf16");
+  if (desc->flags != 0) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  if (desc->T < 0 || desc->d < 8 || desc->d % 8) return set_error(TP_ERR_SHAPE, "T >= 0, d a multiple of 8");
+  if (desc->n_experts < 1 || desc->n_experts % 8 || (desc->n_experts % 64 && desc->n_experts > 256))
+    return set_error(TP_ERR_SHAPE, "n_experts: a multiple of 8, and of 64 above 256");
+  if (desc->top_k < 1 || desc->top_k > moe::kMaxTopK || desc->top_k > desc->n_experts)
+    return set_error(TP_ERR_SHAPE, "top_k must be 1..8 and <= n_experts");
+  if (desc->d_ff_shared < 0) return set_error(TP_ERR_SHAPE, "d_ff_shared must be >= 0");
+  M->T = desc->T; M->d = desc->d; M->F = desc->d_ff; M->Fsh = desc->d_ff_shared;
+  M->E = desc->n_experts; M->k = desc->top_k; M->p = desc->p;
+  M->n_rows = M->T * M->k;
+  if (M->n_rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many routed rows");
+  tp_mlp_desc me{M->n_rows, M->d, M->F, M->p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_SEPARATE, 0, 0.f};
+  tp_status st = layout_of(&me, &M->ex);
+  if (st != TP_OK) return st;
+  if (M->Fsh > 0) {
+    // the shared expert's shard sum is fused into its down GEMM, written as fp32
+    tp_mlp_desc ms{M->T, M->d, M->Fsh, M->p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_FUSED,
+                   TP_FLAG_F32_RESIDUAL, 0.f};
+    if ((st = layout_of(&ms, &M->sh)) != TP_OK) return st;
+  }
+  size_t o = 0;
+  auto take = [&](size_t& field, size_t bytes) {
+    field = o;
+    o += align256(bytes);
+  };
+  const size_t R = static_cast<size_t>(M->n_rows);
+  take(M->logits_off, static_cast<size_t>(M->T) * M->E * 4);
+  take(M->idx_off, R * 4);
+  take(M->w_off, R * 4);
+  take(M->cnt_off, static_cast<size_t>(M->E) * 4);
+  take(M->off_off, static_cast<size_t>(M->E) * 4);
+  take(M->mbp_off, static_cast<size_t>(M->E + 1) * 4);
+  take(M->perm_off, R * 4);
+  take(M->inv_off, R * 4);
+  take(M->xs_off, R * M->d * 2);
+  take(M->hs_off, R * M->p * M->ex.Fsp * 2);
+  take(M->part_off, R * M->d * 4);            // routed rows, the shards already summed
+  take(M->shared_off, M->Fsh > 0 ? M->sh.fwd_ws : 0);
+  take(M->shared_y_off, M->Fsh > 0 ? static_cast<size_t>(M->T) * M->d * 4 : 0);
+  M->bytes = o;
+  return TP_OK;
+}
+}  // namespace
+
+extern "C" size_t tp_moe_expert_w1_bytes(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK ? M.ex.w1p_bytes : 0;
+}
+extern "C" size_t tp_moe_expert_w2_bytes(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK ? M.ex.w2p_bytes : 0;
+}
+extern "C" size_t tp_moe_shared_w1_bytes(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK && M.Fsh > 0 ? M.sh.w1p_bytes : 0;
+}
+extern "C" size_t tp_moe_shared_w2_bytes(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK && M.Fsh > 0 ? M.sh.w2p_bytes : 0;
+}
+extern "C" size_t tp_moe_fwd_workspace(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK ? M.bytes : 0;
+}
+
+extern "C" tp_status tp_moe_pack(const tp_moe_desc* desc, const void* const* wg,
+                                 const void* const* wu, const void* const* w2, const void* wg_s,
+                                 const void* wu_s, const void* w2_s, void* w1p, void* w2p,
+                                 void* w1p_s, void* w2p_s, void* stream) {
+  clear_error();
+  MoeLayout M;
+  tp_status st = moe_layout(desc, &M);
+  if (st != TP_OK) return st;
+  if (!wg || !wu || !w2 || !w1p || !w2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  for (int e = 0; e < M.E; ++e) {
+    if (!wg[e] || !wu[e] || !w2[e]) return set_error(TP_ERR_INVALID_ARG, "null expert weight");
+    if ((st = pack_t<__nv_bfloat16>(M.ex, wg[e], wu[e], w2[e], off(w1p, e * M.ex.w1p_bytes),
+                                    off(w2p, e * M.ex.w2p_bytes), s)) != TP_OK)
+      return st;
+  }
+  if (M.Fsh > 0) {
+    if (!wg_s || !wu_s || !w2_s || !w1p_s || !w2p_s)
+      return set_error(TP_ERR_INVALID_ARG, "the shared expert's weights are null");
+    return pack_t<__nv_bfloat16>(M.sh, wg_s, wu_s, w2_s, w1p_s, w2p_s, s);
+  }
+  return TP_OK;
+}
+
+extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr,
+                                const void* w1p, const void* w2p, const void* w1p_s,
+                                const void* w2p_s, const void* bias, const void* residual,
+                                void* y, void* route_idx, void* route_w, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  clear_error();
+  MoeLayout M;
+  tp_status st = moe_layout(desc, &M);
+  if (st != TP_OK) return st;
+  if (M.T == 0) {
+    count_reduction();
+    return TP_OK;
+  }
+  if (!x || !wr || !w1p || !w2p || !y) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (M.Fsh > 0 && (!w1p_s || !w2p_s))
+    return set_error(TP_ERR_INVALID_ARG, "the shared expert's packed weights are null");
+  for (const void* q : {x, wr, w1p, w2p, w1p_s, w2p_s, bias, residual, static_cast<const void*>(y)})
+    if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < M.bytes) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tensor_cores_usable())
+    return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float* logits = reinterpret_cast<float*>(off(workspace, M.logits_off));
+  int32_t* idx = route_idx ? static_cast<int32_t*>(route_idx)
+                           : reinterpret_cast<int32_t*>(off(workspace, M.idx_off));
+  float* wts = route_w ? static_cast<float*>(route_w) : reinterpret_cast<float*>(off(workspace, M.w_off));
+  int32_t* cnt = reinterpret_cast<int32_t*>(off(workspace, M.cnt_off));
+  int32_t* offs = reinterpret_cast<int32_t*>(off(workspace, M.off_off));
+  int32_t* mbp = reinterpret_cast<int32_t*>(off(workspace, M.mbp_off));
+  int32_t* perm = reinterpret_cast<int32_t*>(off(workspace, M.perm_off));
+  int32_t* inv = reinterpret_cast<int32_t*>(off(workspace, M.inv_off));
+  auto* xs = reinterpret_cast<__nv_bfloat16*>(off(workspace, M.xs_off));
+  auto* hs = reinterpret_cast<__nv_bfloat16*>(off(workspace, M.hs_off));
+  float* part = reinterpret_cast<float*>(off(workspace, M.part_off));
+  const MlpLayout& L = M.ex;
+  // (1) router logits = x Wr (Wr [d][E] read MN-major), fp32
+  if (M.E % 64) {
+    ProfScope prof(s, "moe_router");
+    const int threads = (256 / M.E) * M.E;
+    TP_LAUNCH_PDL(moe::router_simt_kernel, dim3(static_cast<unsigned>(M.T)), dim3(threads), 0, s,
+                  static_cast<const __nv_bfloat16*>(x), static_cast<const __nv_bfloat16*>(wr),
+                  M.d, M.E, logits);
+  } else {
+    const Operand xo{x, false, M.T, M.d, 1, M.d, 0};
+    const Operand ro{wr, true, M.E, M.d, 1, M.E, 0};
+    tc::EpiStoreF32::Params ep;
+    ep.out = logits;
+    ep.ld = M.E;
+    ep.batch_stride = 0;
+    ep.rows_valid = static_cast<int32_t>(M.T);
+    ep.cols_valid = M.E;
+    ep.swap = 0;
+    st = M.E == 64 ? tc::run_gemm<TileCfg<64, 1, false, true, stages_for(64, 1)>, tc::EpiStoreF32>(
+                         xo, ro, M.T, M.E, M.d, 1, ep, s, "moe_router")
+                   : tc::run_gemm<TileCfg<128, 1, false, true, stages_for(128, 1)>, tc::EpiStoreF32>(
+                         xo, ro, M.T, M.E, M.d, 1, ep, s, "moe_router");
+    if (st != TP_OK) return st;
+  }
+  // (2) top-k and weights; (3) per-expert counts, offsets and stable positions; (4) gather
+  {
+    ProfScope prof(s, "moe_route");
+    TP_LAUNCH_PDL(moe::topk_kernel, dim3(static_cast<unsigned>(ceil_div(M.T, 256))), dim3(256), 0,
+                  s, logits, M.T, M.E, M.k, idx, wts);
+    TP_LAUNCH_PDL(moe::count_kernel, dim3(static_cast<unsigned>(M.E)), dim3(1024), 0, s,
+                  static_cast<const int32_t*>(idx), M.n_rows, cnt);
+    TP_LAUNCH_PDL(moe::position_kernel, dim3(static_cast<unsigned>(M.E)), dim3(1024), 0, s,
+                  static_cast<const int32_t*>(idx), M.n_rows, static_cast<const int32_t*>(cnt), 128,
+                  offs, mbp, perm, inv);
+    TP_LAUNCH_PDL(moe::gather_kernel, dim3(static_cast<unsigned>(M.n_rows)), dim3(128), 0, s,
+                  static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(perm), M.k,
+                  M.d, xs);
+  }
+  // (5) grouped up GEMM + SwiGLU over all experts: rows of expert e are xs[off[e] .. +cnt[e])
+  {
+    const int64_t rows = L.p * L.R;
+    tc::EpiHidden::Params ep;
+    ep.h = hs;
+    ep.z = nullptr;
+    ep.ld_h = L.p * L.Fsp;
+    ep.ld_z = 0;
+    ep.tokens = static_cast<int32_t>(M.n_rows);
+    ep.rows = static_cast<int32_t>(rows);
+    ep.act = TP_ACT_SWIGLU;
+    ep.swap = 0;
+    const Operand ao{xs, false, M.n_rows, M.d, 1, M.d, 0};
+    const Operand bo{w1p, false, rows, M.d, M.E, M.d, rows * M.d};
+    tc::GemmOpts opt;
+    opt.grp_cnt = cnt;
+    opt.grp_off = offs;
+    opt.grp_mbp = mbp;
+    opt.grp_n = M.E;
+    opt.grp_div = 1;
+    st = tc::run_gemm<KK<256, 1>, tc::EpiHidden>(ao, bo, M.T, rows, M.d, M.E, ep, s,
+                                                 "moe_up_gemm", opt);
+    if (st != TP_OK) return st;
+  }
+  // (6) grouped down GEMM: problem e * p + i = expert e, shard i; each tile runs shard 0..p-1's
+  // k-blocks into one accumulator, so the routed rows leave with their shards summed: [row][d]
+  {
+    const Operand ho{hs, false, M.n_rows, L.Fsp, L.p, L.p * L.Fsp, L.Fsp};
+    const Operand wo{w2p, false, M.d, L.Fsp, static_cast<int64_t>(M.E) * L.p, L.Fsp, M.d * L.Fsp};
+    tc::EpiStoreF32::Params ep;
+    ep.out = part;
+    ep.ld = M.d;
+    ep.batch_stride = 0;
+    ep.rows_valid = static_cast<int32_t>(M.n_rows);
+    ep.cols_valid = static_cast<int32_t>(M.d);
+    ep.swap = 0;
+    tc::GemmOpts opt;
+    opt.grp_cnt = cnt;
+    opt.grp_off = offs;
+    opt.grp_mbp = mbp;
+    opt.grp_n = M.E;
+    opt.grp_div = L.p;
+    opt.grp_sum = true;
+    st = tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, M.T, M.d, L.Fsp,
+                                                   static_cast<int64_t>(M.E) * L.p, ep, s,
+                                                   "moe_down_gemm", opt);
+    if (st != TP_OK) return st;
+  }
+  // (7) the shared expert over all tokens, its p shards summed in its down GEMM: [T][d] fp32
+  const float* shared_sum = nullptr;
+  if (M.Fsh > 0) {
+    void* ws = off(workspace, M.shared_off);
+    void* h = off(ws, M.sh.fh_off);
+    float* sy = reinterpret_cast<float*>(off(workspace, M.shared_y_off));
+    void* sk = off(ws, M.sh.fsk_off);
+    const size_t skb = M.sh.fpart_off - M.sh.fsk_off;
+    if ((st = tc_up(M.sh, x, w1p_s, h, nullptr, sk, skb, s)) != TP_OK) return st;
+    if ((st = tc_down(M.sh, h, w2p_s, nullptr, nullptr, sy, sk, skb, s)) != TP_OK) return st;
+    shared_sum = sy;
+  }
+  // (8) the block's sum: shared expert + the weighted routed rows (choices in order), bias
+  // once, residual
+  {
+    ProfScope prof(s, "moe_combine");
+    const int64_t nv = M.T * (M.d / 8);
+    const int64_t blocks = std::min<int64_t>(ceil_div(nv, 256), static_cast<int64_t>(num_sms()) * 8);
+    TP_LAUNCH_PDL(moe::combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                  static_cast<const float*>(part), shared_sum, static_cast<const int32_t*>(inv),
+                  static_cast<const float*>(wts), M.k, M.T, M.d,
+                  static_cast<const __nv_bfloat16*>(bias),
+                  static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y));
+  }
+  count_reduction();
+  return TP_OK;
 }

@@ -36,7 +36,9 @@ EXPORTS = (
     "tp_selftest_wait_timeout", "tp_attn_bwd_workspace", "tp_attn_bwd", "tp_attn_unpack_grads",
     "tp_reduce_scatter_partials", "tp_all_gather_slices", "tp_mlp_fwd_sp_workspace",
     "tp_mlp_fwd_sp", "tp_mlp_bwd_sp_workspace", "tp_mlp_bwd_sp", "tp_attn_fwd_sp_workspace",
-    "tp_attn_fwd_sp",
+    "tp_attn_fwd_sp", "tp_moe_expert_w1_bytes", "tp_moe_expert_w2_bytes",
+    "tp_moe_shared_w1_bytes", "tp_moe_shared_w2_bytes", "tp_moe_pack", "tp_moe_fwd_workspace",
+    "tp_moe_fwd",
 )
 
 
@@ -51,6 +53,13 @@ class tp_mlp_desc(ctypes.Structure):
                 ("p", ctypes.c_int32), ("act", ctypes.c_int32), ("dtype", ctypes.c_int32),
                 ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("norm_eps", ctypes.c_float)]
+
+
+class tp_moe_desc(ctypes.Structure):
+    _fields_ = [("T", ctypes.c_int64), ("d", ctypes.c_int64), ("d_ff", ctypes.c_int64),
+                ("d_ff_shared", ctypes.c_int64), ("n_experts", ctypes.c_int32),
+                ("top_k", ctypes.c_int32), ("p", ctypes.c_int32), ("dtype", ctypes.c_int32),
+                ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32)]
 
 
 class tp_attn_desc(ctypes.Structure):
@@ -76,6 +85,7 @@ def load():
     lib = ctypes.CDLL(LIB_PATH)
     P, S, I32, I64, F32 = ctypes.c_void_p, ctypes.c_size_t, ctypes.c_int32, ctypes.c_int64, ctypes.c_float
     MD, AD = ctypes.POINTER(tp_mlp_desc), ctypes.POINTER(tp_attn_desc)
+    ED = ctypes.POINTER(tp_moe_desc)
     sig = {
         "tp_mlp_w1_packed_bytes": (S, [MD]), "tp_mlp_w2_packed_bytes": (S, [MD]),
         "tp_mlp_pack": (I32, [MD, P, P, P, P, P, P]), "tp_mlp_saved_bytes": (S, [MD]),
@@ -106,6 +116,11 @@ def load():
         "tp_mlp_bwd_sp": (I32, [MD, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_attn_fwd_sp_workspace": (S, [AD]),
         "tp_attn_fwd_sp": (I32, [AD, P, P, P, P, P, P, P, P, P, S, P]),
+        "tp_moe_expert_w1_bytes": (S, [ED]), "tp_moe_expert_w2_bytes": (S, [ED]),
+        "tp_moe_shared_w1_bytes": (S, [ED]), "tp_moe_shared_w2_bytes": (S, [ED]),
+        "tp_moe_pack": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P]),
+        "tp_moe_fwd_workspace": (S, [ED]),
+        "tp_moe_fwd": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
@@ -354,6 +369,49 @@ def tp_attn_fwd_sp(desc, x_slices, wqkv_p, wo_p, y_slices, k_cache=None, v_cache
     _check(load().tp_attn_fwd_sp(ctypes.byref(desc), xs.ptr, _ptr(wqkv_p), _ptr(wo_p),
                                  _ptr(k_cache), _ptr(v_cache), _sp(rs), ys.ptr, _sp(ns),
                                  _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+# ------------------------------------------------------------------------ mixture of experts
+def moe_desc(T, d, d_ff, d_ff_shared, n_experts, top_k, p):
+    return tp_moe_desc(int(T), int(d), int(d_ff), int(d_ff_shared), int(n_experts), int(top_k),
+                       int(p), TP_BF16, 0, 0)
+
+
+def tp_moe_expert_w1_bytes(desc):
+    return load().tp_moe_expert_w1_bytes(ctypes.byref(desc))
+
+
+def tp_moe_expert_w2_bytes(desc):
+    return load().tp_moe_expert_w2_bytes(ctypes.byref(desc))
+
+
+def tp_moe_shared_w1_bytes(desc):
+    return load().tp_moe_shared_w1_bytes(ctypes.byref(desc))
+
+
+def tp_moe_shared_w2_bytes(desc):
+    return load().tp_moe_shared_w2_bytes(ctypes.byref(desc))
+
+
+def tp_moe_fwd_workspace(desc):
+    return load().tp_moe_fwd_workspace(ctypes.byref(desc))
+
+
+def tp_moe_pack(desc, wg, wu, w2, w1p, w2p, shared=None, w1p_s=None, w2p_s=None, stream=None):
+    """wg, wu, w2: lists of the E experts' weights; shared: (wg_s, wu_s, w2_s) or None."""
+    g, u, o = _Slices(wg), _Slices(wu), _Slices(w2)
+    sg, su, so = shared if shared is not None else (None, None, None)
+    _check(load().tp_moe_pack(ctypes.byref(desc), g.ptr, u.ptr, o.ptr, _ptr(sg), _ptr(su),
+                              _ptr(so), _ptr(w1p), _ptr(w2p), _ptr(w1p_s), _ptr(w2p_s),
+                              _stream(stream)))
+
+
+def tp_moe_fwd(desc, x, wr, w1p, w2p, y, w1p_s=None, w2p_s=None, bias=None, residual=None,
+               route_idx=None, route_w=None, workspace=None, stream=None):
+    _check(load().tp_moe_fwd(ctypes.byref(desc), _ptr(x), _ptr(wr), _ptr(w1p), _ptr(w2p),
+                             _ptr(w1p_s), _ptr(w2p_s), _ptr(bias), _ptr(residual), _ptr(y),
+                             _ptr(route_idx), _ptr(route_w), _ptr(workspace), _nbytes(workspace),
+                             _stream(stream)))
 
 
 # ------------------------------------------------------------------------------ diagnostics

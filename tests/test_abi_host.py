@@ -178,3 +178,28 @@ def test_sequence_parallel_argument_errors(lib):
     assert lib.tp_attn_fwd_sp_workspace(a_rag) == 0
     a_ok = lib.attn_desc(1, 8, 64, 4, 2, 16, 2)
     assert lib.tp_attn_fwd_sp_workspace(a_ok) > lib.tp_attn_fwd_workspace(a_ok)
+
+
+def test_moe_layout_and_argument_errors(lib):
+    so = lib.load()
+    d = lib.moe_desc(64, 256, 512, 256, 16, 2, 2)
+    # one expert packs like the dense SwiGLU MLP of the same d, d_ff, p
+    md = lib.mlp_desc(64, 256, 512, 2, "swiglu", "bf16")
+    assert lib.tp_moe_expert_w1_bytes(d) == lib.tp_mlp_w1_packed_bytes(md)
+    assert lib.tp_moe_expert_w2_bytes(d) == lib.tp_mlp_w2_packed_bytes(md)
+    md_s = lib.mlp_desc(64, 256, 256, 2, "swiglu", "bf16")
+    assert lib.tp_moe_shared_w1_bytes(d) == lib.tp_mlp_w1_packed_bytes(md_s)
+    assert lib.tp_moe_shared_w1_bytes(lib.moe_desc(64, 256, 512, 0, 16, 2, 2)) == 0
+    assert lib.tp_moe_fwd_workspace(d) > 0
+    for bad in (lib.moe_desc(64, 256, 512, 0, 12, 2, 2), lib.moe_desc(64, 256, 512, 0, 16, 0, 2),
+                lib.moe_desc(64, 250, 512, 0, 16, 2, 2), lib.moe_desc(64, 256, 512, 100, 16, 2, 8)):
+        assert lib.tp_moe_fwd_workspace(bad) == 0
+    fake = ctypes.c_void_p(0x1000)
+    lib.tp_reset_reduction_count()
+    empty = lib.moe_desc(0, 256, 512, 0, 16, 2, 2)
+    assert so.tp_moe_fwd(ctypes.byref(empty), None, None, None, None, None, None, None, None, None,
+                         None, None, None, 0, None) == 0
+    assert lib.tp_reduction_count() == 1
+    assert so.tp_moe_fwd(ctypes.byref(d), None, fake, fake, fake, fake, fake, None, None, fake,
+                         None, None, fake, 1 << 40, None) == lib.TP_ERR_INVALID_ARG
+    lib.tp_reset_reduction_count()

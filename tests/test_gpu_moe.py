@@ -1,0 +1,110 @@
+"""Tensor-parallel MoE block on the GPU through the C ABI, against the float64 oracle.
+
+The routing (which experts, a discrete decision) is compared where it is unique: tokens whose k-th
+and (k+1)-th oracle logits are apart by more than the fp32/bf16 rounding of the router.  The
+block's output is then compared with the oracle run on the GPU's own routing (the decision passed
+in), rel-L2 <= 2e-2 (bf16).
+"""
+import numpy as np
+import pytest
+import torch
+
+from oracle import moe as omoe
+from tensor_transformer_matmul_b200 import inputs
+from tests.helpers import TOL, dev, f64, rel_l2
+
+pytestmark = pytest.mark.gpu
+
+
+def _setup(lib, T, d, E, k, F, Fs, p, seed, with_bias=True, with_res=True):
+    g = dev()
+    rnd = lambda shape, std, salt: inputs.normal(shape, std, seed, salt, "bf16", "cpu")
+    x = rnd((T, d), 1.0, 1)
+    wr = rnd((d, E), 1.0 / np.sqrt(d), 2)
+    ex = [(rnd((d, F), 0.05, 10 + 3 * e), rnd((d, F), 0.05, 11 + 3 * e), rnd((F, d), 0.05, 12 + 3 * e))
+          for e in range(E)]
+    sh = (rnd((d, Fs), 0.05, 5), rnd((d, Fs), 0.05, 6), rnd((Fs, d), 0.05, 7)) if Fs else None
+    bias = rnd((d,), 0.5, 8) if with_bias else None
+    res = rnd((T, d), 1.0, 9) if with_res else None
+    desc = lib.moe_desc(T, d, F, Fs, E, k, p)
+    w1p = torch.empty(E * lib.tp_moe_expert_w1_bytes(desc) // 2, dtype=torch.bfloat16, device=g)
+    w2p = torch.empty(E * lib.tp_moe_expert_w2_bytes(desc) // 2, dtype=torch.bfloat16, device=g)
+    w1s = w2s = None
+    if Fs:
+        w1s = torch.empty(lib.tp_moe_shared_w1_bytes(desc) // 2, dtype=torch.bfloat16, device=g)
+        w2s = torch.empty(lib.tp_moe_shared_w2_bytes(desc) // 2, dtype=torch.bfloat16, device=g)
+    dex = [tuple(t.to(g) for t in e) for e in ex]
+    lib.tp_moe_pack(desc, [e[0] for e in dex], [e[1] for e in dex], [e[2] for e in dex], w1p, w2p,
+                    shared=None if sh is None else tuple(t.to(g) for t in sh), w1p_s=w1s, w2p_s=w2s)
+    ws = torch.empty(lib.tp_moe_fwd_workspace(desc), dtype=torch.uint8, device=g)
+    st = dict(desc=desc, x=x, wr=wr, ex=ex, sh=sh, bias=bias, res=res, w1p=w1p, w2p=w2p, w1s=w1s,
+              w2s=w2s, ws=ws, T=T, d=d, k=k)
+    return st
+
+
+def _run(lib, st):
+    g = dev()
+    T, d, k = st["T"], st["d"], st["k"]
+    y = torch.empty(T, d, dtype=torch.bfloat16, device=g)
+    idx = torch.empty(T, k, dtype=torch.int32, device=g)
+    w = torch.empty(T, k, dtype=torch.float32, device=g)
+    lib.tp_moe_fwd(st["desc"], st["x"].to(g), st["wr"].to(g), st["w1p"], st["w2p"], y,
+                   w1p_s=st["w1s"], w2p_s=st["w2s"],
+                   bias=None if st["bias"] is None else st["bias"].to(g),
+                   residual=None if st["res"] is None else st["res"].to(g),
+                   route_idx=idx, route_w=w, workspace=st["ws"])
+    return y, idx, w
+
+
+def _check(st, y, idx, w):
+    x, wr = f64(st["x"]), f64(st["wr"])
+    k = st["k"]
+    logits = x @ wr
+    ref_idx, ref_w = omoe.route(x, wr, k)
+    srt = -np.sort(-logits, axis=1)
+    gap = srt[:, k - 1] - srt[:, k] if k < logits.shape[1] else np.full(len(srt), np.inf)
+    clear = gap > 1e-2
+    assert clear.mean() > 0.8
+    gi, gw = idx.cpu().numpy(), w.cpu().numpy()
+    assert np.array_equal(gi[clear], ref_idx[clear])
+    assert rel_l2(gw[clear], ref_w[clear]) <= 1e-3
+    assert ((gi >= 0) & (gi < wr.shape[1])).all()
+    assert np.allclose(gw.sum(axis=1), 1.0, atol=1e-5)
+    experts = [tuple(f64(t) for t in e) for e in st["ex"]]
+    sh = None if st["sh"] is None else tuple(f64(t) for t in st["sh"])
+    ref = omoe.moe_forward(x, wr, experts, k, shared=sh,
+                           bias=None if st["bias"] is None else f64(st["bias"]),
+                           routing=(gi.astype(np.int64), gw.astype(np.float64)))
+    if st["res"] is not None:
+        ref = ref + f64(st["res"])
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("T,d,E,k,F,Fs,p", [
+    (200, 256, 16, 2, 512, 256, 2),    # few experts (SIMT router), shared expert, bias, residual
+    (150, 512, 64, 4, 256, 0, 4),      # tensor-core router, no shared expert
+    (1, 256, 64, 8, 256, 256, 2),      # one token (decode), eight experts
+    (300, 264, 128, 2, 384, 128, 1),   # ragged d, 128 experts, p = 1
+])
+def test_moe_forward_parity(lib, T, d, E, k, F, Fs, p):
+    st = _setup(lib, T, d, E, k, F, Fs, p, seed=50 + T)
+    lib.tp_reset_reduction_count()
+    y, idx, w = _run(lib, st)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    _check(st, y, idx, w)
+
+
+def test_moe_deterministic(lib):
+    st = _setup(lib, 180, 256, 64, 2, 256, 128, 2, seed=60)
+    a = [t.clone() for t in _run(lib, st)]
+    b = _run(lib, st)
+    torch.cuda.synchronize()
+    for u, v in zip(a, b):
+        assert torch.equal(u, v)
+
+
+def test_moe_rejects(lib):
+    assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 512, 0, 12, 2, 2)) == 0   # E % 8
+    assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 512, 0, 16, 9, 2)) == 0   # top_k > 8
+    assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 510, 0, 16, 2, 4)) == 0   # p | d_ff
