@@ -805,7 +805,7 @@ def main():
     ap.add_argument("--no-extras", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--extra-steps", type=int, default=20)
-    ap.add_argument("--extras", default="tiny,prefill,attention,stack,seqpar",
+    ap.add_argument("--extras", default="tiny,prefill,attention,stack,seqpar,moe",
                     help="comma list of extra workloads to measure at N=1")
     ap.add_argument("--reduce-mode", choices=["separate", "fused"], default="separate",
                     help="how the p partial sums are added in the decode workloads")
