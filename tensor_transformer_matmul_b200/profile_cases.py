@@ -7,6 +7,8 @@ to capture with the profiler's skip count).
 
     python -m tensor_transformer_matmul_b200.profile_cases mlp_fwd --tokens 1024
     python -m tensor_transformer_matmul_b200.profile_cases attn_fwd --tokens 2048 --fused
+    python -m tensor_transformer_matmul_b200.profile_cases attn_bwd --tokens 2048
+    python -m tensor_transformer_matmul_b200.profile_cases moe_fwd --tokens 1024
 """
 import argparse
 
@@ -50,7 +52,53 @@ def attn_fwd(tokens, reps, fused, h=8192, n_q=64, n_kv=8, hd=128, p=8):
     return y
 
 
-CASES = {"mlp_fwd": mlp_fwd, "attn_fwd": attn_fwd}
+def attn_bwd(tokens, reps, fused, h=8192, n_q=64, n_kv=8, hd=128, p=8):
+    """GQA attention block backward (b=1, causal) with the attention configuration's heads."""
+    mode = tp.TP_REDUCE_FUSED if fused else tp.TP_REDUCE_SEPARATE
+    desc = tp.attn_desc(1, tokens, h, n_q, n_kv, hd, p, reduce_mode=mode)
+    ai = inputs.attn_inputs(1, tokens, h, n_q, n_kv, hd, "bf16", seed=0, device="cuda")
+    wqkv = torch.empty(tp.tp_attn_wqkv_packed_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+    wo = torch.empty(tp.tp_attn_wo_packed_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+    tp.tp_attn_pack(desc, ai["wq"], ai["wk"], ai["wv"], ai["wo"], wqkv, wo)
+    dy = inputs.normal((1, tokens, h), 1.0, 0, 97, "bf16", "cuda")
+    dx = torch.empty_like(ai["x"])
+    dwqkv = torch.empty(wqkv.numel(), dtype=torch.float32, device="cuda")
+    dwo = torch.empty(wo.numel(), dtype=torch.float32, device="cuda")
+    ws = torch.empty(tp.tp_attn_bwd_workspace(desc), dtype=torch.uint8, device="cuda")
+    for _ in range(reps):
+        tp.tp_attn_bwd(desc, ai["x"], wqkv, wo, dy, dx, dwqkv, dwo, workspace=ws)
+    torch.cuda.synchronize()
+    return dx
+
+
+def moe_fwd(tokens, reps, fused, d=7168, n_experts=32, top_k=8, d_ff=2048, p=8):
+    """MoE block forward with DeepSeek-V3-shaped experts (d=7168, width 2048, top-8, a shared
+    expert of width 2048, p=8) but 32 experts, so that the weights take about 3 GB."""
+    desc = tp.moe_desc(tokens, d, d_ff, d_ff, n_experts, top_k, p)
+    e1, e2 = tp.tp_moe_expert_w1_bytes(desc) // 2, tp.tp_moe_expert_w2_bytes(desc) // 2
+    w1p = torch.empty(n_experts * e1, dtype=torch.bfloat16, device="cuda")
+    w2p = torch.empty(n_experts * e2, dtype=torch.bfloat16, device="cuda")
+    ed = tp.mlp_desc(1, d, d_ff, p, "swiglu", "bf16")
+    for e in range(n_experts):
+        g, u, o = (inputs.normal(s, 0.02, 0, 1000 + 3 * e + j, "bf16", "cuda")
+                   for j, s in enumerate(((d, d_ff), (d, d_ff), (d_ff, d))))
+        tp.tp_mlp_pack(ed, g, u, o, w1p[e * e1:(e + 1) * e1], w2p[e * e2:(e + 1) * e2])
+    w1s = torch.empty(tp.tp_moe_shared_w1_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+    w2s = torch.empty(tp.tp_moe_shared_w2_bytes(desc) // 2, dtype=torch.bfloat16, device="cuda")
+    g, u, o = (inputs.normal(s, 0.02, 0, 900 + j, "bf16", "cuda")
+               for j, s in enumerate(((d, d_ff), (d, d_ff), (d_ff, d))))
+    tp.tp_mlp_pack(ed, g, u, o, w1s, w2s)
+    wr = inputs.normal((d, n_experts), d ** -0.5, 0, 901, "bf16", "cuda")
+    x = inputs.normal((tokens, d), 1.0, 0, 902, "bf16", "cuda")
+    y = torch.empty_like(x)
+    ws = torch.empty(tp.tp_moe_fwd_workspace(desc), dtype=torch.uint8, device="cuda")
+    for _ in range(reps):
+        tp.tp_moe_fwd(desc, x, wr, w1p, w2p, y, w1p_s=w1s, w2p_s=w2s, workspace=ws)
+    torch.cuda.synchronize()
+    return y
+
+
+CASES = {"mlp_fwd": mlp_fwd, "attn_fwd": attn_fwd, "attn_bwd": attn_bwd, "moe_fwd": moe_fwd}
 
 
 def main(argv=None):

@@ -95,6 +95,22 @@ def test_moe_forward_parity(lib, T, d, E, k, F, Fs, p):
     _check(st, y, idx, w)
 
 
+def test_moe_skewed_routing(lib):
+    # a router column pair that dominates every token: experts 0 and 1 each receive all 300
+    # tokens (three 128-row blocks apiece) and the other 62 experts none
+    st = _setup(lib, 300, 256, 64, 2, 256, 128, 2, seed=61)
+    wr = st["wr"].float()
+    wr[:, 0] += 0.5 * torch.sign(st["x"].float().sum(0))
+    wr[:, 1] += 0.45 * torch.sign(st["x"].float().sum(0))
+    st["wr"] = wr.to(torch.bfloat16)
+    st["x"] = (st["x"].float() + torch.sign(st["x"].float().sum(0))).to(torch.bfloat16)
+    y, idx, w = _run(lib, st)
+    torch.cuda.synchronize()
+    counts = torch.bincount(idx.flatten().long().cpu(), minlength=64)
+    assert counts[0] == 300 and counts[1] == 300 and counts[2:].sum() == 0
+    _check(st, y, idx, w)
+
+
 def test_moe_deterministic(lib):
     st = _setup(lib, 180, 256, 64, 2, 256, 128, 2, seed=60)
     a = [t.clone() for t in _run(lib, st)]
