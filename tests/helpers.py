@@ -5,7 +5,7 @@ import torch
 
 from tensor_transformer_matmul_b200 import inputs
 
-# tolerances of the benchmark spec: rel-L2 <= 2e-2 for bf16, <= 1e-5 for fp32
+# parity tolerances: rel-L2 <= 2e-2 for bf16, <= 1e-5 for fp32
 TOL = {"bf16": 2e-2, "f32": 1e-5}
 
 
