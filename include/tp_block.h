@@ -286,7 +286,9 @@ size_t tp_moe_shared_w2_bytes(const tp_moe_desc* desc);
 
 /* Pack the experts.  wg, wu, w2: HOST arrays of E device pointers to expert e's Wg, Wu [d][d_ff]
  * and W2 [d_ff][d] (bf16, input-major); wg_s, wu_s, w2_s: the shared expert (ignored when
- * d_ff_shared == 0).  w1p, w2p: E * tp_moe_expert_w{1,2}_bytes; w1p_s, w2p_s: the shared sizes. */
+ * d_ff_shared == 0).  w1p, w2p: E * tp_moe_expert_w{1,2}_bytes; w1p_s, w2p_s: the shared sizes.
+ * The experts are packed in order; a null pointer inside the arrays is found when its expert
+ * is reached (TP_ERR_INVALID_ARG), after the experts before it were enqueued. */
 tp_status tp_moe_pack(const tp_moe_desc* desc, const void* const* wg, const void* const* wu,
                       const void* const* w2, const void* wg_s, const void* wu_s, const void* w2_s,
                       void* w1p, void* w2p, void* w1p_s, void* w2p_s, void* stream);

@@ -203,3 +203,29 @@ def test_moe_layout_and_argument_errors(lib):
     assert so.tp_moe_fwd(ctypes.byref(d), None, fake, fake, fake, fake, fake, None, None, fake,
                          None, None, fake, 1 << 40, None) == lib.TP_ERR_INVALID_ARG
     lib.tp_reset_reduction_count()
+
+
+def test_moe_pack_and_sp_backward_argument_errors(lib):
+    # host-side checks only: nothing is enqueued when they fail
+    so = lib.load()
+    fake = ctypes.c_void_p(0x1000)
+    d = lib.moe_desc(8, 256, 512, 0, 8, 2, 2)
+    ok8 = (ctypes.c_void_p * 8)(*([0x1000] * 8))
+    arr = lambda a: ctypes.cast(a, ctypes.c_void_p)
+    assert so.tp_moe_pack(ctypes.byref(d), None, arr(ok8), arr(ok8), None, None, None, fake, fake,
+                          None, None, None) == lib.TP_ERR_INVALID_ARG
+    ds = lib.moe_desc(8, 256, 512, 256, 8, 2, 2)   # a shared expert needs its weights
+    assert so.tp_moe_fwd(ctypes.byref(ds), fake, fake, fake, fake, None, None, None, None, fake,
+                         None, None, fake, 1 << 40, None) == lib.TP_ERR_INVALID_ARG
+    # workspace too small
+    assert so.tp_moe_fwd(ctypes.byref(d), fake, fake, fake, fake, None, None, None, None, fake,
+                         None, None, fake, 16, None) == lib.TP_ERR_WORKSPACE
+    two = (ctypes.c_void_p * 2)(0x1000, 0x2000)
+    dm = lib.mlp_desc(8, 64, 256, 2, "swiglu", "bf16")
+    # the backward needs the forward's saved activations and every slice
+    assert so.tp_mlp_bwd_sp(ctypes.byref(dm), arr(two), arr(two), None, fake, fake, arr(two), fake,
+                            fake, fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_mlp_bwd_sp(ctypes.byref(dm), arr(two), None, fake, fake, fake, arr(two), fake,
+                            fake, fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_mlp_bwd_sp(ctypes.byref(dm), arr(two), arr(two), fake, fake, fake, arr(two), fake,
+                            fake, fake, 16, None) == lib.TP_ERR_WORKSPACE
