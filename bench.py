@@ -608,7 +608,32 @@ def extra_prefill(tp, inputs, torch, stream, peaks, steps):
     res["reduce_fused"] = {k: fused[k] for k in ("ms_fwd", "ms_bwd", "TFLOP_per_s",
                                                   "frac_of_burst_peak", "frac_of_sustained_peak",
                                                   "tokens_per_s", "kernels")}
+    res["cublas_context"] = _cublas_context(torch, stream, steps)
     return res
+
+
+def _cublas_context(torch, stream, steps):
+    """Context only, not this library's path: torch.matmul (cuBLAS) bf16 on the prefill MLP's
+    two forward GEMM shapes, all shards at once (T x d by d x 2 d_ff, T x d_ff by d_ff x d)."""
+    try:
+        c = PREFILL
+        dev = torch.device("cuda", torch.cuda.current_device())
+        g = torch.Generator(device=dev)
+        g.manual_seed(7)
+        out = {}
+        for name, (m, k, n) in (("up", (c["T"], c["d"], 2 * c["F"])),
+                                ("down", (c["T"], c["F"], c["d"]))):
+            a = torch.randn(m, k, generator=g, device=dev).to(torch.bfloat16)
+            b = torch.randn(k, n, generator=g, device=dev).to(torch.bfloat16)
+            for _ in range(3):
+                torch.matmul(a, b)
+            ms = _cuda_time(lambda: torch.matmul(a, b), steps, stream) / steps
+            out[name] = {"ms": round(ms, 3), "TFLOP_per_s": round(2.0 * m * k * n / (ms / 1e3) / 1e12, 1)}
+            del a, b
+        torch.cuda.empty_cache()
+        return out
+    except Exception as e:  # context only: never fail the bench over it
+        return {"error": f"{type(e).__name__}: {e}"[:200]}
 
 
 def _prefill_mode(tp, inputs, torch, stream, peaks, steps, mode):
