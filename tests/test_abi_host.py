@@ -229,3 +229,23 @@ def test_moe_pack_and_sp_backward_argument_errors(lib):
                             fake, fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
     assert so.tp_mlp_bwd_sp(ctypes.byref(dm), arr(two), arr(two), fake, fake, fake, arr(two), fake,
                             fake, fake, 16, None) == lib.TP_ERR_WORKSPACE
+
+
+def test_product_and_oracle_are_independent():
+    # the product package never imports the oracle, and the oracle never imports the product
+    # (they share only the seeded input generators, which hold none of the block's arithmetic)
+    pkg = os.path.join(ROOT, "tensor_transformer_matmul_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith(".py"):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, re.M), f
+    for f in os.listdir(os.path.join(ROOT, "oracle")):
+        if f.endswith(".py"):
+            src = open(os.path.join(ROOT, "oracle", f)).read()
+            assert "tensor_transformer_matmul_b200" not in src, f
+            assert "libtpblock" not in src, f
+    # no CUDA source names the oracle
+    csrc = os.path.join(pkg, "csrc")
+    for f in os.listdir(csrc):
+        assert "oracle" not in open(os.path.join(csrc, f)).read().lower(), f
