@@ -320,9 +320,10 @@ tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr, con
 
 /* Reduce-scatter: out_slices[i][r] = residual_slices[i][r] + sum_{s=0}^{p-1} partials[s][i*T/p + r]
  * (fp32 in shard order, residual last, one rounding to out_dtype); with norm_slices, also
- * norm_slices[i][r] = RMSNorm(out_slices[i][r]) (unit weight, eps; norm_dtype) computed from the
- * stored values.  partials: [p][T][d] fp32.  residual_slices and norm_slices may be NULL.
- * Adds 1 to the reduction counter. */
+ * norm_slices[i][r] = RMSNorm(out_slices[i][r]) (unit weight; norm_dtype) computed from the
+ * stored values.  eps is used exactly as given, as in tp_rmsnorm (0 is allowed and means no eps;
+ * a negative or NaN eps returns TP_ERR_INVALID_ARG).  partials: [p][T][d] fp32.  residual_slices
+ * and norm_slices may be NULL.  Adds 1 to the reduction counter. */
 tp_status tp_reduce_scatter_partials(const void* partials, int32_t p, int64_t T, int64_t d,
                                      void* const* residual_slices, void* const* out_slices,
                                      int32_t out_dtype, void* const* norm_slices,

@@ -53,6 +53,44 @@ def route(x, wr, k):
     return idx, w
 
 
+def weights_for(x, wr, idx):
+    """The routing weights that go with a given choice of experts: for each token, the softmax of
+    its logits at the chosen experts ``idx[t]`` (in the order given).  With idx from route() this
+    equals route()'s weights; for another valid top-k set (a near tie broken the other way) it
+    gives that set's weights from the exact logits."""
+    logits = _f64(x) @ _f64(wr)
+    idx = np.asarray(idx, dtype=np.int64)
+    w = np.zeros(idx.shape)
+    for t in range(idx.shape[0]):
+        sel = logits[t, idx[t]]
+        e = np.exp(sel - sel.max())
+        w[t] = e / e.sum()
+    return w
+
+
+def topk_margin(x, wr, idx):
+    """For each token, the smallest chosen logit minus the largest unchosen one (exact logits).
+
+    ``idx[t]`` is a true top-k set exactly when the margin is >= 0.  A router that computes its
+    logits with an error of at most eps per logit picks a set whose exact margin is >= -2 eps, so
+    a caller checks a rounded router's choice against that bound.  With k = E every logit is
+    chosen and the margin is +inf."""
+    logits = _f64(x) @ _f64(wr)
+    idx = np.asarray(idx, dtype=np.int64)
+    T, E = logits.shape
+    out = np.full(T, np.inf)
+    for t in range(T):
+        chosen = np.zeros(E, dtype=bool)
+        chosen[idx[t]] = True
+        if chosen.sum() != idx.shape[1]:
+            out[t] = -np.inf          # an expert chosen twice is never a valid top-k set
+            continue
+        if chosen.all():
+            continue
+        out[t] = logits[t, chosen].min() - logits[t, ~chosen].max()
+    return out
+
+
 def moe_forward(x, wr, experts, k, shared=None, bias=None, routing=None):
     """Unsharded MoE block.  experts: list of (wg, wu, w2) per expert; shared: (wg, wu, w2) or
     None; routing: (idx, weights) to use instead of route(x, wr, k)."""

@@ -52,8 +52,8 @@ extern "C" tp_status tp_reduce_scatter_partials(const void* partials, int32_t p,
   if (!(eps >= 0.f)) return tp::set_error(TP_ERR_INVALID_ARG, "eps must be >= 0");
   if (T > 0 && !partials) return tp::set_error(TP_ERR_INVALID_ARG, "partials is null");
   st = tp::seqpar::reduce_scatter(static_cast<const float*>(partials), p, T, d, residual_slices,
-                                  out_slices, out_dtype, norm_slices, norm_dtype,
-                                  eps > 0.f ? eps : 1e-5f, static_cast<cudaStream_t>(stream));
+                                  out_slices, out_dtype, norm_slices, norm_dtype, eps,
+                                  static_cast<cudaStream_t>(stream));
   if (st == TP_OK) tp::count_reduction();
   return st;
 }

@@ -15,6 +15,18 @@ def rel_l2(got, ref):
     return float(np.linalg.norm(got - ref) / max(np.linalg.norm(ref), 1e-300))
 
 
+def rel_l2_rows(got, ref):
+    """The largest rel-L2 over the rows (the last axis) of got against ref: a wrong tile or a
+    wrong shard's block shows up in its own rows even when the whole-tensor norm hides it."""
+    got = np.asarray(got, dtype=np.float64)
+    ref = np.asarray(ref, dtype=np.float64)
+    g = got.reshape(-1, got.shape[-1])
+    r = ref.reshape(-1, ref.shape[-1])
+    num = np.linalg.norm(g - r, axis=1)
+    den = np.maximum(np.linalg.norm(r, axis=1), 1e-300)
+    return float((num / den).max()) if len(r) else 0.0
+
+
 def f64(t):
     return inputs.to_f64(t)
 

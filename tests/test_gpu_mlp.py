@@ -9,7 +9,7 @@ import torch
 
 from oracle import mlp as omlp
 from tensor_transformer_matmul_b200 import inputs
-from tests.helpers import TOL, Mlp, dev, f64, rel_l2
+from tests.helpers import TOL, Mlp, dev, f64, rel_l2, rel_l2_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -153,23 +153,33 @@ def test_deterministic(lib):
     assert torch.equal(a, b)
 
 
-def test_full_size_decode_mlp_sampled(lib):
-    # T=64 (batch 64, s=1), d=8192, d_ff=28672, p=8, bf16 x ~ N(0,1), W ~ N(0, 0.02)
+def test_full_size_decode_mlp(lib):
+    # T=64 (batch 64, s=1), d=8192, d_ff=28672, p=8, bf16 x ~ N(0,1), W ~ N(0, 0.02): every row
+    # against the oracle, whole tensor and row by row
     T, d, F, p = 64, 8192, 28672, 8
     inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02)
     m = Mlp(lib, inp, p, "swiglu", "bf16")
     y = m.forward(inp["x"], save=False)
     torch.cuda.synchronize()
-    rows = [0, 1, 31, 63]
-    ref = omlp.mlp_forward_rows(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu", rows,
-                                f64(inp["w_up"]))
-    assert rel_l2(f64(y)[rows], ref) <= TOL["bf16"]
+    ref = omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu",
+                           f64(inp["w_up"]))
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
+    assert rel_l2_rows(f64(y), ref) <= TOL["bf16"]
+
+
+def _one_per_block(n, block, salt):
+    """One index in every ``block``-wide block of range(n), at a different offset in each."""
+    return [b * block + (salt * (b + 1) * 37) % min(block, n - b * block)
+            for b in range((n + block - 1) // block)]
 
 
 @pytest.mark.parametrize("mode", [0, 1])
 def test_full_size_prefill_mlp_sampled(lib, mode):
-    # T=4096 (b=1, s=4096), d=8192, d_ff=28672, p=8: forward rows, then backward samples;
-    # mode 1 adds the 8 shard partials of y and of dx inside the GEMM accumulators
+    # T=4096 (b=1, s=4096), d=8192, d_ff=28672, p=8: one row of y and dx in every 256-row tile
+    # (the SM-pair GEMM's token tile), and one hidden feature of every shard for the dWg / dWu
+    # columns and the dW2 row, each computed by the oracle over its full contraction and checked
+    # as a whole and row by row (column by column for dW1); mode 1 adds the 8 shard partials of
+    # y and of dx inside the GEMM accumulators
     T, d, F, p = 4096, 8192, 28672, 8
     inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02,
                             backward=True)
@@ -178,13 +188,20 @@ def test_full_size_prefill_mlp_sampled(lib, mode):
     dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
     torch.cuda.synchronize()
     x, wg, wu, w2, dy = (f64(inp[k]) for k in ("x", "w1", "w_up", "w2", "dy"))
-    rows, cols, w2rows = [0, 777, 2048, 4095], [0, 3583, 3584, 28671], [5, 14000]
-    assert rel_l2(f64(y)[rows], omlp.mlp_forward_rows(x, wg, w2, "swiglu", rows, wu)) <= TOL["bf16"]
+    rows = _one_per_block(T, 256, 3)
+    cols = _one_per_block(F, F // p, 5)        # one feature per shard
+    w2rows = _one_per_block(F, F // p, 7)
+    ref_y = omlp.mlp_forward_rows(x, wg, w2, "swiglu", rows, wu)
+    got_y = f64(y)[rows]
+    assert rel_l2(got_y, ref_y) <= TOL["bf16"] and rel_l2_rows(got_y, ref_y) <= TOL["bf16"]
     s = omlp.mlp_backward_samples(x, wg, w2, dy, "swiglu", rows, cols, w2rows, wu)
-    assert rel_l2(f64(dx)[rows], s["dx"]) <= TOL["bf16"]
-    assert rel_l2(f64(dw1)[:, cols], s["dw1_cols"]) <= TOL["bf16"]
-    assert rel_l2(f64(dwu)[:, cols], s["dw_up_cols"]) <= TOL["bf16"]
-    assert rel_l2(f64(dw2)[w2rows], s["dw2_rows"]) <= TOL["bf16"]
+    checks = ((f64(dx)[rows], s["dx"]),
+              (f64(dw1)[:, cols].T, s["dw1_cols"].T),
+              (f64(dwu)[:, cols].T, s["dw_up_cols"].T),
+              (f64(dw2)[w2rows], s["dw2_rows"]))
+    for got, ref in checks:
+        assert rel_l2(got, ref) <= TOL["bf16"]
+        assert rel_l2_rows(got, ref) <= TOL["bf16"]
 
 
 def test_f32_residual_stream(lib):

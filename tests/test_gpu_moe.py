@@ -1,9 +1,12 @@
 """Tensor-parallel MoE block on the GPU through the C ABI, against the float64 oracle.
 
-The routing (which experts, a discrete decision) is compared where it is unique: tokens whose k-th
-and (k+1)-th oracle logits are apart by more than the fp32/bf16 rounding of the router.  The
-block's output is then compared with the oracle run on the GPU's own routing (the decision passed
-in), rel-L2 <= 2e-2 (bf16).
+Routing is a discrete decision taken from fp32 logits, so near ties may break either way.  It is
+checked for every token: the GPU's chosen set must be a top-k set of the exact (float64) logits
+within the router's rounding bound, listed in descending logit order within that bound, and where
+the choice is unique (a clear gap between the k-th and (k+1)-th logit) it must be the oracle's.  Only the GPU's expert indices
+go to the oracle: the oracle computes their weights from its own float64 logits, the GPU's
+weights are compared with those, and the block's output is compared with the oracle's output on
+those experts, rel-L2 <= 2e-2 (bf16) for the whole tensor and for every row.
 """
 import numpy as np
 import pytest
@@ -11,7 +14,7 @@ import torch
 
 from oracle import moe as omoe
 from tensor_transformer_matmul_b200 import inputs
-from tests.helpers import TOL, dev, f64, rel_l2
+from tests.helpers import TOL, dev, f64, rel_l2, rel_l2_rows
 
 pytestmark = pytest.mark.gpu
 
@@ -56,28 +59,48 @@ def _run(lib, st):
     return y, idx, w
 
 
+def router_eps(x, wr):
+    """Per-token bound on how far apart the GPU's and the exact logits of two experts can be.
+
+    The router forms each logit as a sum of d products of bf16 values, each exact in fp32, added
+    in fp32 in some order; the error of such a sum is at most d * u * sum_k |x_k w_ke|
+    (u = 2^-23 also covers an accumulator that truncates).  Two logits: twice that, with 1%
+    slack for the bound's higher-order term."""
+    d = x.shape[1]
+    return 2.0 * 1.01 * d * 2.0 ** -23 * (np.abs(x) @ np.abs(wr)).max(axis=1)
+
+
 def _check(st, y, idx, w):
     x, wr = f64(st["x"]), f64(st["wr"])
-    k = st["k"]
+    k, E = st["k"], wr.shape[1]
+    gi, gw = idx.cpu().numpy().astype(np.int64), w.cpu().numpy().astype(np.float64)
+    assert ((gi >= 0) & (gi < E)).all()
+    # every token: a valid top-k set of the exact logits, within the router's rounding
+    assert (omoe.topk_margin(x, wr, gi) >= -router_eps(x, wr)).all()
+    # where the choice is unique it is the oracle's set; the order is descending in the exact
+    # logits, within the same rounding bound
+    eps = router_eps(x, wr)
     logits = x @ wr
-    ref_idx, ref_w = omoe.route(x, wr, k)
+    ref_idx, _ = omoe.route(x, wr, k)
     srt = -np.sort(-logits, axis=1)
-    gap = srt[:, k - 1] - srt[:, k] if k < logits.shape[1] else np.full(len(srt), np.inf)
-    clear = gap > 1e-2
+    gap = srt[:, k - 1] - srt[:, k] if k < E else np.full(len(srt), np.inf)
+    clear = gap > eps
     assert clear.mean() > 0.8
-    gi, gw = idx.cpu().numpy(), w.cpu().numpy()
-    assert np.array_equal(gi[clear], ref_idx[clear])
-    assert rel_l2(gw[clear], ref_w[clear]) <= 1e-3
-    assert ((gi >= 0) & (gi < wr.shape[1])).all()
-    assert np.allclose(gw.sum(axis=1), 1.0, atol=1e-5)
+    assert np.array_equal(np.sort(gi[clear], axis=1), np.sort(ref_idx[clear], axis=1))
+    chosen = np.take_along_axis(logits, gi, axis=1)
+    assert (chosen[:, :-1] >= chosen[:, 1:] - eps[:, None]).all()
+    # the weights of the chosen experts come from the oracle's own logits
+    ow = omoe.weights_for(x, wr, gi)
+    assert np.abs(gw - ow).max() <= 1e-4
     experts = [tuple(f64(t) for t in e) for e in st["ex"]]
     sh = None if st["sh"] is None else tuple(f64(t) for t in st["sh"])
     ref = omoe.moe_forward(x, wr, experts, k, shared=sh,
                            bias=None if st["bias"] is None else f64(st["bias"]),
-                           routing=(gi.astype(np.int64), gw.astype(np.float64)))
+                           routing=(gi, ow))
     if st["res"] is not None:
         ref = ref + f64(st["res"])
     assert rel_l2(f64(y), ref) <= TOL["bf16"]
+    assert rel_l2_rows(f64(y), ref) <= TOL["bf16"]
 
 
 @pytest.mark.parametrize("T,d,E,k,F,Fs,p", [

@@ -52,6 +52,22 @@ def test_reduce_scatter(lib, p, T, d, out_dtype, with_res, with_norm):
             assert rel_l2(f64(norms[i]), odec.rmsnorm(f64(outs[i]))) <= TOL["bf16"], i
 
 
+@pytest.mark.parametrize("eps", [0.0, 1e-5])
+def test_reduce_scatter_eps_is_used_as_given(lib, eps):
+    # rows of size ~1e-3 (mean square ~1e-6), so eps = 1e-5 changes the norm by a factor ~3 and
+    # eps = 0 must give x / sqrt(mean(x^2)) exactly as tp_rmsnorm does with the same eps
+    p, T, d = 2, 4, 64
+    part = inputs.normal((p, T, d), 1e-3, 42, 1, "f32", "cpu")
+    outs = [torch.empty(T // p, d, device=dev()) for _ in range(p)]
+    norms = [torch.empty(T // p, d, device=dev()) for _ in range(p)]
+    lib.tp_reduce_scatter_partials(part.to(dev()), p, outs, norm=norms, eps=eps)
+    torch.cuda.synchronize()
+    for i in range(p):
+        assert rel_l2(f64(norms[i]), odec.rmsnorm(f64(outs[i]), eps=eps)) <= TOL["f32"], i
+        other = 1e-5 if eps == 0.0 else 0.0
+        assert rel_l2(f64(norms[i]), odec.rmsnorm(f64(outs[i]), eps=other)) > 0.1, i
+
+
 @pytest.mark.parametrize("p,R,d,dtype", [(4, 3, 8192, "bf16"), (3, 5, 7, "bf16"), (2, 4, 6, "f32"),
                                          (8, 8, 8192, "f32")])
 def test_all_gather_exact(lib, p, R, d, dtype):

@@ -112,3 +112,48 @@ def test_given_routing_is_used():
     y = moe.moe_forward(x, wr, experts, 2, routing=(idx, w))
     f = lambda e: mlp.mlp_forward(x, experts[e][0], experts[e][2], "swiglu", experts[e][1])
     np.testing.assert_allclose(y, 0.75 * f(3) + 0.25 * f(0), rtol=1e-13)
+
+
+def test_weights_for_a_given_choice_by_hand():
+    # the weights of a given expert set are the softmax of those logits, in the order given
+    wr = np.array([[1.0, 3.0, 2.0, 0.0]])
+    x = np.array([[1.0]])
+    w = moe.weights_for(x, wr, np.array([[2, 0]]))
+    assert abs(w[0, 0] - math.e / (math.e + 1.0)) < 1e-15
+    assert abs(w[0, 1] - 1.0 / (math.e + 1.0)) < 1e-15
+    idx, wref = moe.route(x, wr, 2)
+    assert np.array_equal(moe.weights_for(x, wr, idx), wref)
+
+
+def test_weights_for_route_equals_scipy_renormalised_softmax():
+    # softmax over all experts, renormalised over the chosen k (scipy), for a random case
+    x, wr, _, _ = _case(T=9, d=8, E=16, seed=7)
+    idx, _ = moe.route(x, wr, 3)
+    g = softmax(x @ wr, axis=1)
+    want = np.take_along_axis(g, idx, axis=1)
+    want = want / want.sum(axis=1, keepdims=True)
+    np.testing.assert_allclose(moe.weights_for(x, wr, idx), want, rtol=1e-13)
+
+
+def test_topk_margin_by_hand():
+    # logits [1, 3, 2, 0]: the top-2 set {1, 2} has margin 2 - 1 = 1; swapping in expert 0 for
+    # expert 2 gives a set that is not a top-2 set, margin 1 - 2 = -1; a repeated expert is never
+    # valid; k = E has nothing unchosen
+    wr = np.array([[1.0, 3.0, 2.0, 0.0]])
+    x = np.array([[1.0]])
+    assert moe.topk_margin(x, wr, np.array([[1, 2]]))[0] == 1.0
+    assert moe.topk_margin(x, wr, np.array([[2, 1]]))[0] == 1.0
+    assert moe.topk_margin(x, wr, np.array([[1, 0]]))[0] == -1.0
+    assert moe.topk_margin(x, wr, np.array([[1, 1]]))[0] == -np.inf
+    assert moe.topk_margin(x, wr, np.array([[0, 1, 2, 3]]))[0] == np.inf
+
+
+def test_topk_margin_of_route_is_the_logit_gap():
+    # brute force: for the oracle's own choice the margin is the k-th minus the (k+1)-th largest
+    # logit, >= 0 for every token
+    x, wr, _, _ = _case(T=20, d=8, E=12, seed=8)
+    k = 4
+    idx, _ = moe.route(x, wr, k)
+    srt = -np.sort(-(x @ wr), axis=1)
+    np.testing.assert_allclose(moe.topk_margin(x, wr, idx), srt[:, k - 1] - srt[:, k], rtol=1e-14)
+    assert (moe.topk_margin(x, wr, idx) >= 0).all()
