@@ -92,6 +92,17 @@ def job_throughput(dist, ms_local, units_per_rank):
     return ms, units_per_rank * dist.world / (ms / 1e3)
 
 
+def smi_id(local):
+    """The nvidia-smi -i argument for CUDA device ``local``: with CUDA_VISIBLE_DEVICES set, CUDA
+    ordinals are positions in that list, not nvidia-smi indices."""
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").strip()
+    if vis:
+        ids = [v.strip() for v in vis.split(",") if v.strip()]
+        if 0 <= local < len(ids):
+            return ids[local]
+    return str(local)
+
+
 class ClockSampler:
     """nvidia-smi samples of SM clock and throttle reasons while a timed region runs."""
 
@@ -109,7 +120,7 @@ class ClockSampler:
             fd, self.path = tempfile.mkstemp(suffix=".csv")
             os.close(fd)
             self.proc = subprocess.Popen(
-                ["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.FIELDS}",
+                ["nvidia-smi", "-i", smi_id(self.gpu), f"--query-gpu={self.FIELDS}",
                  "--format=csv,noheader,nounits", "-lms", "100"],
                 stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
         except Exception:
@@ -390,41 +401,188 @@ def run_ours(args, dist):
         del st
         torch.cuda.empty_cache()
         out["extras"] = run_extras(args, tp, inputs, torch, stream, peaks)
+    elif dist.world > 1 and not args.no_extras:
+        # every rank runs this, in the same order (its collectives must match across ranks)
+        del st
+        torch.cuda.empty_cache()
+        tpm = tp_multi_gpu(args, dist, tp, inputs, torch, stream)
+        if dist.rank == 0:
+            out["extras"] = {"tp_one_shard_per_gpu": tpm}
 
+    cpu = None
     if dist.world == 1 and dist.rank == 0 and not args.no_cpu_baseline:
-        out["cpu_baseline"] = cpu_baseline(seconds=args.cpu_seconds)
+        cpu = cpu_config_baselines(seconds=args.cpu_seconds)
+        out["cpu_baseline"] = {"value": cpu["2"]["value"], "unit": "tokens/s",
+                               "cores": cpu["cores"], "kind": "oracle",
+                               "sample": cpu["2"]["sample"] + " (the whole decode MLP), "
+                                         f"{args.cpu_seconds:.0f} s"}
     elif dist.rank == 0:
         out["cpu_baseline"] = None
     dist.close()
     if dist.rank == 0:
+        # the compact per-configuration summary goes last, so that it survives in the tail of
+        # the output even when the line is cut
+        out["configs"] = config_summary(out, cpu, peaks)
         print(json.dumps(out), flush=True)
+
+
+def tp_multi_gpu(args, dist, tp, inputs, torch, stream):
+    """The decode MLP (T=64, d=8192, d_ff=28672) with one shard per GPU, p = N: rank r packs and
+    holds only shard r (1/N of the weights), computes its partial, and the 1 MiB bf16 partials
+    are summed by an NCCL all-reduce over NVLink, one per step (the pages' decode payload).
+    Reports the step time (max over ranks) and the latency of every all-reduce."""
+    from tensor_transformer_matmul_b200 import tp_dist
+    c = DECODE
+    dev = torch.device("cuda", torch.cuda.current_device())
+    g = tp_dist.TPGroup(timing=False)
+    m = tp_dist.ShardedMLP(g, c["T"], c["d"], c["F"], act="swiglu", dtype="bf16",
+                           partial_dtype=torch.bfloat16, device=dev)
+    # every rank draws the same full weights, packs its own shard, then drops the rest
+    inp = inputs.mlp_inputs(c["T"], c["d"], c["F"], "swiglu", "bf16", seed=0, device=dev,
+                            w_std=0.02)
+    m.pack(inp["w1"], inp["w_up"], inp["w2"])
+    x = inp["x"]
+    del inp
+    torch.cuda.empty_cache()
+
+    def step():
+        m.forward(x)
+
+    for _ in range(max(3, args.warmup)):
+        step()
+    torch.cuda.synchronize()
+    steps = max(3, min(args.steps, 500))
+    dist.barrier()
+    torch.cuda.synchronize()
+    ms = _cuda_time(step, steps, stream)
+    dist.barrier()
+    ms = dist.max(ms) / steps
+    g.timing = True
+    g.count = 0
+    n_lat = min(steps, 200)
+    for _ in range(n_lat):
+        step()
+    lat = g.latencies_ms()
+    q = _quantiles_us(lat)
+    p50_max = dist.max(q["p50"] if q else 0.0)
+    return {"workload": f"decode TP SwiGLU MLP: T=64, d=8192, d_ff=28672, one shard per GPU "
+                        f"(p={dist.world}), bf16 partials summed by an NCCL all-reduce",
+            "ms_per_step": round(ms, 5), "tokens_per_s": round(c["T"] / (ms / 1e3), 1),
+            "allreduce_bytes": c["T"] * c["d"] * 2, "allreduces_per_step": g.count // n_lat,
+            "allreduce_us": q, "allreduce_us_p50_max_over_ranks": round(p50_max, 2),
+            "steps": steps}
+
+
+def _clocked(gpu, fn, *a, **k):
+    """Run one extra workload with the SM clock sampled while it runs; the median under load
+    and the throttle reasons go into its result."""
+    clk = ClockSampler(gpu)
+    clk.start()
+    r = fn(*a, **k)
+    c = clk.stop()
+    if isinstance(r, dict):
+        r["clocks"] = c
+    return r
+
+
+def _mhz(d):
+    c = (d or {}).get("clocks") or {}
+    return c.get("sm_mhz")
+
+
+def _dom_short(dom):
+    if not dom:
+        return None
+    r = {"k": dom["kernel"]}
+    if "frac" in dom:
+        r.update({"work": dom["work_per_launch"], "ach": dom["achieved"], "frac": dom["frac"]})
+    return r
+
+
+def config_summary(out, cpu, peaks):
+    """Compact per-configuration summary (well under 1.5 KB): value and unit, the dominant
+    kernel with its algorithmic work per launch (bytes or flops), achieved rate and fraction of
+    the measured peak, the median SM clock while that workload ran, and the oracle's time on the
+    host cores for the same configuration."""
+    ex = out.get("extras") or {}
+    cpu = cpu or {}
+    cb = lambda i: [cpu[i]["value"], cpu[i]["unit"]] if i in cpu else None
+    r = {"peaks": {"hbm": peaks["hbm_gbs"], "bf16": peaks["bf16_tflops"],
+                   "bf16_sust": peaks["bf16_tflops_sustained"], "src": peaks["source"]},
+         "cpu_cores": cpu.get("cores")}
+    t = ex.get("tiny_mlp")
+    if t:
+        r["1_tiny"] = {"v": t["us_per_call"], "u": "us/call", "bound": "launch latency",
+                       "launches": t["launches_per_call"], "mhz": _mhz(t), "cpu": cb("1")}
+    rf = out.get("roofline") or {}
+    r["2_decode_mlp"] = {"v": out["value"], "u": "tokens/s",
+                         "dom": {"k": rf.get("kernel"),
+                                 "work": rf.get("algorithmic_bytes_per_launch"),
+                                 "ach": rf.get("achieved"), "frac": rf.get("frac")},
+                         "step_frac_hbm": out["config"].get("step_frac_of_hbm"),
+                         "mhz": (out.get("clocks") or {}).get("sm_mhz"), "cpu": cb("2")}
+    p = ex.get("prefill_mlp_fwd_bwd")
+    if p:
+        f = p.get("reduce_fused") or p
+        r["3_prefill_fwd_bwd"] = {"v": f["TFLOP_per_s"], "u": "TFLOP/s", "mode": "fused",
+                                  "frac_burst": f["frac_of_burst_peak"],
+                                  "v_separate": p["TFLOP_per_s"],
+                                  "dom": _dom_short(f.get("dominant")), "mhz": _mhz(p),
+                                  "cpu": cb("3"), "cpu_note": "extrapolated" if "3" in cpu else None}
+    a = ex.get("attention_block")
+    if a:
+        f = a.get("reduce_fused") or a
+        r["4_attention"] = {"v": f["TFLOP_per_s"], "u": "TFLOP/s", "mode": "fused",
+                            "frac_burst": f.get("frac_of_burst_peak"), "v_separate": a["TFLOP_per_s"],
+                            "dom": _dom_short(f.get("dominant")), "mhz": _mhz(a), "cpu": cb("4")}
+    tpm = ex.get("tp_one_shard_per_gpu")
+    if tpm:
+        q = tpm.get("allreduce_us") or {}
+        r["tp_one_shard_per_gpu"] = {"v": tpm["tokens_per_s"], "u": "tokens/s",
+                                     "ms": tpm["ms_per_step"],
+                                     "allreduce_us": [q.get("p10"), q.get("p50"), q.get("p90"),
+                                                      q.get("max")]}
+    st = ex.get("decode_stack")
+    if st:
+        q = st.get("reduce_us_quantiles") or {}
+        r["5_decode_stack"] = {"v": st["tokens_per_s"], "u": "tokens/s",
+                               "frac_hbm": st["frac_of_hbm"], "dom": _dom_short(st.get("dominant")),
+                               "reduce_us": [q.get("p10"), q.get("p50"), q.get("p90"), q.get("max")],
+                               "reduces": st.get("reductions_per_step"), "mhz": _mhz(st),
+                               "cpu": cb("5")}
+    return r
 
 
 def run_extras(args, tp, inputs, torch, stream, peaks):
     ex = {}
     which = set(args.extras.split(","))
     steps = max(3, min(args.steps, args.extra_steps))
+    gpu = torch.cuda.current_device()
     if "tiny" in which:
-        ex["tiny_mlp"] = extra_tiny(tp, inputs, torch, stream)
+        ex["tiny_mlp"] = _clocked(gpu, extra_tiny, tp, inputs, torch, stream)
     # lightest first, with a short idle gap between workloads, so that no extra is timed at the
     # power-capped clocks a previous seconds-long tensor-core run leaves behind
     if "stack" in which:
-        ex["decode_stack"] = extra_stack(tp, torch, stream, peaks, steps, args.reduce_mode)
+        ex["decode_stack"] = _clocked(gpu, extra_stack, tp, torch, stream, peaks, steps,
+                                      args.reduce_mode)
         time.sleep(1.0)
     if "attention" in which:
-        ex["attention_block"] = extra_attention(tp, inputs, torch, stream, peaks, steps)
+        ex["attention_block"] = _clocked(gpu, extra_attention, tp, inputs, torch, stream, peaks,
+                                         steps)
         time.sleep(1.0)
-        ex["attention_block_bwd"] = extra_attention_bwd(tp, inputs, torch, stream, peaks,
-                                                        max(3, steps // 4))
+        ex["attention_block_bwd"] = _clocked(gpu, extra_attention_bwd, tp, inputs, torch, stream,
+                                             peaks, max(3, steps // 4))
         time.sleep(1.0)
     if "prefill" in which:
-        ex["prefill_mlp_fwd_bwd"] = extra_prefill(tp, inputs, torch, stream, peaks, steps)
+        ex["prefill_mlp_fwd_bwd"] = _clocked(gpu, extra_prefill, tp, inputs, torch, stream, peaks,
+                                             steps)
     if "seqpar" in which:
         time.sleep(1.0)
-        ex["seqpar_prefill_mlp_fwd"] = extra_seqpar(tp, inputs, torch, stream, peaks, steps)
+        ex["seqpar_prefill_mlp_fwd"] = _clocked(gpu, extra_seqpar, tp, inputs, torch, stream,
+                                                peaks, steps)
     if "moe" in which:
         time.sleep(1.0)
-        ex["moe_layer"] = extra_moe(tp, inputs, torch, stream, peaks, steps)
+        ex["moe_layer"] = _clocked(gpu, extra_moe, tp, inputs, torch, stream, peaks, steps)
     return ex
 
 
@@ -562,6 +720,33 @@ def extra_tiny(tp, inputs, torch, stream, calls=2000):
             "calls": calls}
 
 
+def _dominant(prof, work, peak, unit):
+    """The kernel with the largest summed time in ``prof`` ({label: (launches, ms)}), with its
+    algorithmic work per launch (``work``: label -> bytes or flops), achieved rate and fraction of
+    ``peak``."""
+    if not prof:
+        return None
+    k = max(prof, key=lambda q: prof[q][1])
+    n, ms = prof[k]
+    out = {"kernel": k, "ms_per_launch": round(ms / n, 5), "share": round(ms / sum(v[1] for v in prof.values()), 3)}
+    if k in work:
+        scale = 1e9 if unit == "GB/s" else 1e12
+        ach = work[k] / (ms / n / 1e3) / scale
+        out.update({"work_per_launch": work[k], "achieved": round(ach, 1), "unit": unit,
+                    "frac": round(ach / peak, 4)})
+    return out
+
+
+def _quantiles_us(ms_list):
+    """p10 / p50 / p90 / max of a list of durations in ms, in microseconds."""
+    if not ms_list:
+        return None
+    v = sorted(ms_list)
+    q = lambda f: round(v[int(f * (len(v) - 1))] * 1e3, 2)
+    return {"p10": q(0.1), "p50": q(0.5), "p90": q(0.9), "max": round(v[-1] * 1e3, 2),
+            "n": len(v)}
+
+
 def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
     """16 Llama-70B-shaped decode layers, b=1, KV length 4096, replayed as one CUDA graph."""
     from tensor_transformer_matmul_b200.decode_stack import DecodeStack
@@ -576,24 +761,45 @@ def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
         st.replay()
     torch.cuda.synchronize()
     ms = _cuda_time(st.replay, steps, stream) / steps
-    # eager steps with the event profiler: per-kernel split and per-reduction latency
+    # eager steps with the event profiler: per-kernel split and the latency of every reduction
+    # (the on-device stand-in for the per-collective latency of a replayed iteration)
     tp.tp_reset_reduction_count()
-    prof = _profile(tp, lambda: st.step(x), max(3, steps // 4))
+    n_prof = max(3, steps // 4)
+    tp.tp_profile_reset()
+    tp.tp_profile_enable(True)
+    for _ in range(n_prof):
+        st.step(x)
+    torch.cuda.synchronize()
+    tp.tp_profile_enable(False)
+    prof = tp.tp_profile_read()
+    red_ms = sorted(tp.tp_profile_launch_ms("reduce_partials"))
+    tp.tp_profile_reset()
     per_layer_w = (tp.tp_attn_wqkv_packed_bytes(st.adesc) + tp.tp_attn_wo_packed_bytes(st.adesc)
                    + tp.tp_mlp_w1_packed_bytes(st.mdesc) + tp.tp_mlp_w2_packed_bytes(st.mdesc))
     kv = 2 * c["n_kv"] * (c["kv_len"] + 1) * c["hd"] * 2
     nbytes = c["layers"] * (per_layer_w + kv)
     gbs = nbytes / (ms / 1e3) / 1e9
     red = prof.get("reduce_partials", (0, 0.0))
+    h, Fsp = c["h"], -(-c["F"] // c["p"] // 128) * 128
+    qkv = (c["n_q"] + 2 * c["n_kv"]) * c["hd"]
+    work = {"mlp_up_gemm": tp.tp_mlp_w1_packed_bytes(st.mdesc) + 2 * h + 2 * c["p"] * 2 * Fsp,
+            "mlp_down_gemm": tp.tp_mlp_w2_packed_bytes(st.mdesc) + 2 * c["p"] * Fsp + 4 * c["p"] * h,
+            "attn_qkv_gemm": tp.tp_attn_wqkv_packed_bytes(st.adesc) + 2 * h + 2 * qkv,
+            "attn_out_gemm": tp.tp_attn_wo_packed_bytes(st.adesc) + 2 * c["n_q"] * c["hd"]
+            + 4 * c["p"] * h,
+            "attn_decode": kv}
     out = {"workload": "decode stack: 16 layers (GQA attention s=1 over KV 4096+1, SwiGLU MLP "
                        "d_ff=28672), b=1, p=8, 2 reductions of 1x8192 per layer, CUDA graph",
            "ms_per_token": round(ms, 4), "tokens_per_s": round(1e3 / ms, 1),
            "GB_per_s": round(gbs, 1), "frac_of_hbm": round(gbs / peaks["hbm_gbs"], 4),
            "bytes_per_step": nbytes,
-           "reductions_per_step": red[0] // max(1, max(3, steps // 4)),
+           "reductions_per_step": red[0] // n_prof,
            "reduce_us_mean": round(red[1] / max(1, red[0]) * 1e3, 2),
-           "kernels": {k: {"launches_per_step": v[0] / max(3, steps // 4),
-                           "ms_per_step": round(v[1] / max(3, steps // 4), 4)}
+           "reduce_us_quantiles": _quantiles_us(red_ms),
+           "dominant": _dominant(prof, work, peaks["hbm_gbs"], "GB/s"),
+           "kernels": {k: {"launches_per_step": v[0] / n_prof,
+                           "ms_per_step": round(v[1] / n_prof, 4),
+                           "ms_per_launch": round(v[1] / v[0], 5)}
                        for k, v in prof.items()},
            "steps": steps}
     del st
@@ -607,7 +813,7 @@ def extra_prefill(tp, inputs, torch, stream, peaks, steps):
     fused = _prefill_mode(tp, inputs, torch, stream, peaks, steps, tp.TP_REDUCE_FUSED)
     res["reduce_fused"] = {k: fused[k] for k in ("ms_fwd", "ms_bwd", "TFLOP_per_s",
                                                   "frac_of_burst_peak", "frac_of_sustained_peak",
-                                                  "tokens_per_s", "kernels")}
+                                                  "tokens_per_s", "dominant", "kernels")}
     res["cublas_context"] = _cublas_context(torch, stream, steps)
     return res
 
@@ -676,6 +882,7 @@ def _prefill_mode(tp, inputs, torch, stream, peaks, steps, mode):
             e["frac_of_sustained_peak"] = round(tf / peaks["bf16_tflops_sustained"], 3)
         kern[k] = e
     tot = (ms_f + ms_b)
+    dom = _dominant(prof, gemm_fl, peaks["bf16_tflops"], "TFLOP/s")
     res = {
         "workload": "prefill TP SwiGLU MLP fwd+bwd: T=4096, d=8192, d_ff=28672, p=8, bf16",
         "ms_fwd": round(ms_f, 3), "ms_bwd": round(ms_b, 3),
@@ -684,7 +891,8 @@ def _prefill_mode(tp, inputs, torch, stream, peaks, steps, mode):
         "TFLOP_per_s_bwd": round(b_fl / (ms_b / 1e3) / 1e12, 1),
         "frac_of_burst_peak": round((f_fl + b_fl) / (tot / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "frac_of_sustained_peak": round((f_fl + b_fl) / (tot / 1e3) / 1e12 / peaks["bf16_tflops_sustained"], 3),
-        "tokens_per_s": round(c["T"] / (tot / 1e3), 1), "kernels": kern, "steps": steps}
+        "tokens_per_s": round(c["T"] / (tot / 1e3), 1), "dominant": dom, "kernels": kern,
+        "steps": steps}
     del st
     torch.cuda.empty_cache()
     return res
@@ -722,17 +930,24 @@ def extra_attention(tp, inputs, torch, stream, peaks, steps):
     fl_att = 2.0 * 2 * a["n_q"] * a["hd"] * s * (s + 1) / 2
     fl_o = 2.0 * s * a["n_q"] * a["hd"] * h
     prof = _profile(tp, attn, steps)
+    prof_f = _profile(tp, attn_fused, steps)
+    work = {"attn_qkv_gemm": fl_qkv, "attn_prefill": fl_att, "attn_out_gemm": fl_o}
+    pk = peaks["bf16_tflops"]
     return {
         "workload": "TP GQA attention: b=1, s=2048, h=8192, 64 Q / 8 KV heads, hd=128, p=8, causal",
         "ms": round(ms_a, 3),
         "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12, 1),
         "frac_of_burst_peak": round((fl_qkv + fl_att + fl_o) / (ms_a / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
         "tokens_per_s": round(s / (ms_a / 1e3), 1),
+        "dominant": _dominant(prof, work, pk, "TFLOP/s"),
         "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)} for k, v in prof.items()},
         "reduce_fused": {"ms": round(ms_af, 3),
                          "TFLOP_per_s": round((fl_qkv + fl_att + fl_o) / (ms_af / 1e3) / 1e12, 1),
+                         "frac_of_burst_peak": round((fl_qkv + fl_att + fl_o) / (ms_af / 1e3)
+                                                     / 1e12 / pk, 3),
+                         "dominant": _dominant(prof_f, work, pk, "TFLOP/s"),
                          "kernels": {k: {"ms_per_launch": round(v[1] / v[0], 4)}
-                                     for k, v in _profile(tp, attn_fused, steps).items()}},
+                                     for k, v in prof_f.items()}},
         "steps": steps}
 
 
@@ -827,6 +1042,97 @@ def cpu_baseline(seconds=10.0, arrays=None):
             "cores": _threads(), "kind": "oracle",
             "sample": f"{n} oracle calls, each all 64 tokens through a {ORACLE_CHUNK}-feature slice "
                       f"of d_ff ({TOKENS_PER_ORACLE_STEP:.3f} token-equivalents), {el:.1f} s"}
+
+
+def _timed(fn, seconds, min_calls=1):
+    """Call fn until ``seconds`` have passed (at least ``min_calls`` times); (calls, seconds)."""
+    n, t0 = 0, time.perf_counter()
+    while True:
+        fn()
+        n += 1
+        el = time.perf_counter() - t0
+        if n >= min_calls and el >= seconds:
+            return n, el
+
+
+def cpu_config_baselines(seconds=10.0):
+    """The oracle (float64 numpy, as it stands) on the host cores for every configuration, in the
+    unit the GPU number of that configuration is reported in.
+
+    * tiny MLP (T=4, d=8, d_ff=32, GELU): full calls, us per call;
+    * decode MLP (T=64, d=8192, d_ff=28672): full calls, tokens/s;
+    * prefill MLP forward + backward (T=4096): a 64-token sample of forward + backward (every
+      GEMM's flops scale with the tokens), TFLOP/s and the step time extrapolated by the token
+      ratio -- labelled "extrapolated";
+    * attention block (s=2048, 64/8 heads): full calls, TFLOP/s (causal half counted, as for
+      the GPU);
+    * decode stack (16 layers, KV 4096): one layer timed in full, x 16 (the layers have the same
+      shapes), tokens/s.
+    Inputs are the configurations' seeded draws made on the host.  The returned dict maps
+    "1".."5" to {value, unit, sample}, plus the thread count."""
+    from oracle import attention as oattn
+    from oracle import decode as odec
+    from oracle import mlp as omlp
+    from tensor_transformer_matmul_b200 import inputs
+    f64 = inputs.to_f64
+    out = {"cores": _threads()}
+
+    tiny = inputs.mlp_inputs(4, 8, 32, "gelu", "f32", seed=0)
+    t = {k: f64(v) for k, v in tiny.items() if v is not None}
+    n, el = _timed(lambda: omlp.mlp_forward(t["x"], t["w1"], t["w2"], "gelu"), min(1.0, seconds))
+    out["1"] = {"value": round(el / n * 1e6, 2), "unit": "us/call", "sample": f"{n} full calls"}
+
+    c = DECODE
+    m = inputs.mlp_inputs(c["T"], c["d"], c["F"], "swiglu", "bf16", seed=0, device="cpu",
+                          w_std=0.02)
+    W = {k: f64(v) for k, v in m.items() if v is not None}
+    del m
+    n, el = _timed(lambda: omlp.mlp_forward(W["x"], W["w1"], W["w2"], "swiglu", W["w_up"]),
+                   seconds)
+    out["2"] = {"value": round(n * c["T"] / el, 2), "unit": "tokens/s",
+                "sample": f"{n} full calls of T=64"}
+
+    P, S = PREFILL, 64
+    x3 = f64(inputs.normal((S, P["d"]), 1.0, 0, inputs.S_X, "bf16"))
+    dy3 = f64(inputs.normal((S, P["d"]), 1.0, 0, inputs.S_DY, "bf16"))
+
+    def fb():
+        omlp.mlp_forward(x3, W["w1"], W["w2"], "swiglu", W["w_up"])
+        omlp.mlp_backward(x3, W["w1"], W["w2"], dy3, "swiglu", W["w_up"])
+
+    n, el = _timed(fb, seconds / 2)
+    fl = 6.0 * S * P["d"] * P["F"] * 3
+    out["3"] = {"value": round(fl * n / el / 1e12, 4), "unit": "TFLOP/s",
+                "ms_per_step": round(el / n * (P["T"] / S) * 1e3, 1),
+                "sample": f"{n} forward+backward calls of {S} of the {P['T']} tokens; step time "
+                          f"extrapolated by the token ratio"}
+
+    a = ATTN
+    ai = inputs.attn_inputs(a["b"], a["s"], a["h"], a["n_q"], a["n_kv"], a["hd"], "bf16", seed=0)
+    A = {k: f64(v) for k, v in ai.items()}
+    del ai
+    n, el = _timed(lambda: oattn.attention_forward(A["x"], A["wq"], A["wk"], A["wv"], A["wo"],
+                                                   a["n_q"], a["n_kv"], a["hd"], causal=True), 0.0)
+    s_, h_ = a["s"], a["h"]
+    fl = (2.0 * s_ * h_ * (a["n_q"] + 2 * a["n_kv"]) * a["hd"] + 2.0 * s_ * a["n_q"] * a["hd"] * h_
+          + 4.0 * a["n_q"] * a["hd"] * s_ * (s_ + 1) / 2)
+    out["4"] = {"value": round(fl * n / el / 1e12, 4), "unit": "TFLOP/s",
+                "sample": f"{n} full calls"}
+
+    k = STACK
+    cache = inputs.attn_inputs(1, 1, k["h"], k["n_q"], k["n_kv"], k["hd"], "bf16", seed=0,
+                               kv_len=k["kv_len"])
+    kc = f64(cache["k_cache"])[:, :, :k["kv_len"]]
+    vc = f64(cache["v_cache"])[:, :, :k["kv_len"]]
+    xd = f64(cache["x"])[:, 0]
+    del cache
+    lw = {"wq": A["wq"], "wk": A["wk"], "wv": A["wv"], "wo": A["wo"], "wg": W["w1"],
+          "wu": W["w_up"], "w2": W["w2"]}
+    n, el = _timed(lambda: odec.decode_layer(xd, lw, kc, vc, k["n_q"], k["n_kv"], k["hd"]),
+                   seconds / 2)
+    out["5"] = {"value": round(1.0 / (el / n * k["layers"]), 3), "unit": "tokens/s",
+                "sample": f"one layer timed over {n} calls, x {k['layers']} layers"}
+    return out
 
 
 def run_reference(args, dist):

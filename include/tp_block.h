@@ -368,6 +368,71 @@ tp_status tp_attn_fwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
                          void* stream);
 
 /* ------------------------------------------------------------------------------------------ */
+/* One shard per device                                                                        */
+/* ------------------------------------------------------------------------------------------ */
+/* "Tensor Parallelism" (klaylearn), Notes, and "How does tensor parallelism split a transformer
+ * feed-forward block's two matmuls", "One collective" and "The backward pass": with one shard per
+ * GPU, device i holds only shard i's slices -- the columns i*F_s .. of W1 (and Wu) and the
+ * matching rows of W2; its n_q/p query heads and n_kv/p KV heads (columns of Wq, Wk, Wv, rows of
+ * Wo) and its own KV cache -- computes its full-shape partial, and the devices' all-reduce (the
+ * caller's collective, e.g. NCCL) adds the p partials.  Backward: dy is replicated, each device
+ * keeps its weight gradients (no exchange) and its dx partial is all-reduced.
+ * Shard i is the block with p = 1 and d_ff/p features (n_q/p, n_kv/p heads); its packed layout
+ * equals shard i's slice of the p-shard packing above (so w1p + i * size and the like also work
+ * on one device).  desc describes the whole block (its p, d_ff, heads); `shard` is in 0 .. p-1;
+ * desc.flags must be 0.  The partial ([T][d], or [b][s][h]) is written in partial_dtype: TP_F32
+ * or TP_BF16 (TP_F32 only for fp32 blocks).  These calls do no reduction and add nothing to the
+ * reduction counter; the residual add that follows the all-reduce is tp_reduce_partials with
+ * p = 1 on the summed partial. */
+typedef struct {
+  size_t col_weight_bytes;  /* packed column-parallel weights of one shard (w1p / wqkv slice)  */
+  size_t row_weight_bytes;  /* packed row-parallel weights of one shard (w2p / wo slice)       */
+  size_t saved_bytes;       /* MLP: activations tp_mlp_fwd_shard saves for tp_mlp_bwd_shard     */
+  size_t fwd_workspace;     /* workspace of the *_fwd_shard call                              */
+  size_t bwd_workspace;     /* workspace of the *_bwd_shard call (0: not supported)           */
+  size_t partial_bytes;     /* one partial                                                    */
+} tp_shard_sizes;
+
+tp_status tp_mlp_shard_sizes(const tp_mlp_desc* desc, int32_t partial_dtype, tp_shard_sizes* out);
+/* Pack shard `shard`'s slice from the user's full W1 / Wu [d][d_ff] and W2 [d_ff][d] (device
+ * pointers, dtype) into w1p_shard / w2p_shard (col/row_weight_bytes). */
+tp_status tp_mlp_pack_shard(const tp_mlp_desc* desc, int32_t shard, const void* w1,
+                            const void* w_up, const void* w2, void* w1p_shard, void* w2p_shard,
+                            void* stream);
+/* partial = act(x W1_i) W2_i  [T][d].  saved_shard: NULL or saved_bytes for tp_mlp_bwd_shard. */
+tp_status tp_mlp_fwd_shard(const tp_mlp_desc* desc, int32_t shard, int32_t partial_dtype,
+                           const void* x, const void* w1p_shard, const void* w2p_shard,
+                           void* partial, void* saved_shard, void* workspace, size_t ws_bytes,
+                           void* stream);
+/* dx_partial = dx_i [T][d] (partial_dtype); dw1p_shard / dw2p_shard: this shard's fp32 weight
+ * gradients in its packed layout (no exchange). */
+tp_status tp_mlp_bwd_shard(const tp_mlp_desc* desc, int32_t shard, int32_t partial_dtype,
+                           const void* dy, const void* x, const void* saved_shard,
+                           const void* w1p_shard, const void* w2p_shard, void* dx_partial,
+                           void* dw1p_shard, void* dw2p_shard, void* workspace, size_t ws_bytes,
+                           void* stream);
+
+tp_status tp_attn_shard_sizes(const tp_attn_desc* desc, int32_t partial_dtype,
+                              tp_shard_sizes* out);
+/* Pack shard `shard`'s slice from the user's full wq [h][n_q*hd], wk, wv [h][n_kv*hd] and
+ * wo [n_q*hd][h]. */
+tp_status tp_attn_pack_shard(const tp_attn_desc* desc, int32_t shard, const void* wq,
+                             const void* wk, const void* wv, const void* wo, void* wqkv_shard,
+                             void* wo_shard, void* stream);
+/* partial = Attn_i(x) Wo_i  [b][s][h].  Decode (desc.kv_len > 0): k_cache_shard / v_cache_shard
+ * are this shard's caches [b][n_kv/p][kv_cap][hd]; the new token is appended there. */
+tp_status tp_attn_fwd_shard(const tp_attn_desc* desc, int32_t shard, int32_t partial_dtype,
+                            const void* x, const void* wqkv_shard, const void* wo_shard,
+                            void* k_cache_shard, void* v_cache_shard, void* partial,
+                            void* workspace, size_t ws_bytes, void* stream);
+/* Self-attention backward of one shard (bf16; as tp_attn_bwd): dx_partial [b][s][h] bf16,
+ * dwqkv_shard / dwo_shard fp32 in the shard's packed layout. */
+tp_status tp_attn_bwd_shard(const tp_attn_desc* desc, int32_t shard, const void* x,
+                            const void* wqkv_shard, const void* wo_shard, const void* dy,
+                            void* dx_partial, void* dwqkv_shard, void* dwo_shard,
+                            void* workspace, size_t ws_bytes, void* stream);
+
+/* ------------------------------------------------------------------------------------------ */
 /* Diagnostics                                                                                 */
 /* ------------------------------------------------------------------------------------------ */
 
@@ -408,6 +473,10 @@ tp_status tp_selftest_wait_timeout(uint32_t limit_us, void* stream);
 void tp_profile_enable(int32_t on);
 int32_t tp_profile_read(int32_t i, char* label, int32_t label_len, uint64_t* launches,
                         double* total_ms);
+/* Duration in ms of launch j (0-based, in launch order) of entry i of tp_profile_read; returns 1,
+ * or 0 when i or j is out of range.  Synchronizes the device.  Gives the distribution of one
+ * kernel's launches, e.g. the latency of every reduction in a decoded token. */
+int32_t tp_profile_read_launch(int32_t i, int64_t j, double* ms);
 void tp_profile_reset(void);
 
 /* Library version, major*10000 + minor*100 + patch. */

@@ -190,6 +190,25 @@ int32_t tp_profile_read(int32_t i, char* label, int32_t label_len, uint64_t* lau
   return 1;
 }
 
+int32_t tp_profile_read_launch(int32_t i, int64_t j, double* ms) {
+  cudaDeviceSynchronize();
+  std::lock_guard<std::mutex> g(tp::g_prof_mu);
+  std::vector<std::string> order;
+  for (auto& r : tp::g_prof)
+    if (std::find(order.begin(), order.end(), r.label) == order.end()) order.push_back(r.label);
+  if (i < 0 || i >= static_cast<int32_t>(order.size()) || j < 0) return 0;
+  int64_t k = 0;
+  for (auto& r : tp::g_prof) {
+    if (r.label != order[i]) continue;
+    if (k++ != j) continue;
+    float t = 0.f;
+    if (cudaEventElapsedTime(&t, r.a, r.b) != cudaSuccess) return 0;
+    if (ms) *ms = t;
+    return 1;
+  }
+  return 0;
+}
+
 uint64_t tp_reduction_count(void) { return tp::g_reductions.load(); }
 void tp_reset_reduction_count(void) { tp::g_reductions.store(0); }
 uint64_t tp_launch_count(void) { return tp::g_launches.load(); }

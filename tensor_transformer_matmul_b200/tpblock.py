@@ -33,12 +33,15 @@ EXPORTS = (
     "tp_reduction_count", "tp_reset_reduction_count", "tp_launch_count", "tp_last_error",
     "tp_status_string", "tp_check_device_error", "tp_tensor_core_path_available", "tp_version",
     "tp_profile_enable", "tp_profile_read", "tp_profile_reset", "tp_mlp_fwd_static_ws",
+    "tp_profile_read_launch",
     "tp_selftest_wait_timeout", "tp_attn_bwd_workspace", "tp_attn_bwd", "tp_attn_unpack_grads",
     "tp_reduce_scatter_partials", "tp_all_gather_slices", "tp_mlp_fwd_sp_workspace",
     "tp_mlp_fwd_sp", "tp_mlp_bwd_sp_workspace", "tp_mlp_bwd_sp", "tp_attn_fwd_sp_workspace",
     "tp_attn_fwd_sp", "tp_moe_expert_w1_bytes", "tp_moe_expert_w2_bytes",
     "tp_moe_shared_w1_bytes", "tp_moe_shared_w2_bytes", "tp_moe_pack", "tp_moe_fwd_workspace",
-    "tp_moe_fwd",
+    "tp_moe_fwd", "tp_mlp_shard_sizes", "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
+    "tp_mlp_bwd_shard", "tp_attn_shard_sizes", "tp_attn_pack_shard", "tp_attn_fwd_shard",
+    "tp_attn_bwd_shard",
 )
 
 
@@ -69,6 +72,12 @@ class tp_attn_desc(ctypes.Structure):
                 ("kv_len", ctypes.c_int64), ("kv_cap", ctypes.c_int64),
                 ("reduce_mode", ctypes.c_int32), ("flags", ctypes.c_int32),
                 ("norm_eps", ctypes.c_float), ("reserved", ctypes.c_int32)]
+
+
+class tp_shard_sizes(ctypes.Structure):
+    _fields_ = [("col_weight_bytes", ctypes.c_size_t), ("row_weight_bytes", ctypes.c_size_t),
+                ("saved_bytes", ctypes.c_size_t), ("fwd_workspace", ctypes.c_size_t),
+                ("bwd_workspace", ctypes.c_size_t), ("partial_bytes", ctypes.c_size_t)]
 
 
 _lib = None
@@ -122,8 +131,17 @@ def load():
         "tp_moe_fwd_workspace": (S, [ED]),
         "tp_moe_fwd": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
+        "tp_mlp_shard_sizes": (I32, [MD, I32, ctypes.POINTER(tp_shard_sizes)]),
+        "tp_mlp_pack_shard": (I32, [MD, I32, P, P, P, P, P, P]),
+        "tp_mlp_fwd_shard": (I32, [MD, I32, I32, P, P, P, P, P, P, S, P]),
+        "tp_mlp_bwd_shard": (I32, [MD, I32, I32, P, P, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_shard_sizes": (I32, [AD, I32, ctypes.POINTER(tp_shard_sizes)]),
+        "tp_attn_pack_shard": (I32, [AD, I32, P, P, P, P, P, P, P]),
+        "tp_attn_fwd_shard": (I32, [AD, I32, I32, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_bwd_shard": (I32, [AD, I32, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
+        "tp_profile_read_launch": (I32, [I32, ctypes.c_int64, ctypes.POINTER(ctypes.c_double)]),
     }
     for name, (res, args) in sig.items():
         fn = getattr(lib, name)
@@ -286,6 +304,69 @@ def tp_rmsnorm(x, out, eps=1e-5, stream=None):
     rows = x.numel() // x.shape[-1] if x.numel() else 0
     _check(load().tp_rmsnorm(_ptr(x), xt, int(rows), int(x.shape[-1]), float(eps), _ptr(out), ot,
                              _stream(stream)))
+
+
+# ------------------------------------------------------------------ one shard per device
+def _pdt(partial_dtype):
+    if isinstance(partial_dtype, str):
+        return DTYPE[partial_dtype]
+    if partial_dtype in (torch.float32, torch.bfloat16):
+        return TP_BF16 if partial_dtype == torch.bfloat16 else TP_F32
+    return int(partial_dtype)
+
+
+def tp_mlp_shard_sizes(desc, partial_dtype="f32"):
+    out = tp_shard_sizes()
+    _check(load().tp_mlp_shard_sizes(ctypes.byref(desc), _pdt(partial_dtype), ctypes.byref(out)))
+    return out
+
+
+def tp_mlp_pack_shard(desc, shard, w1, w_up, w2, w1p_shard, w2p_shard, stream=None):
+    _check(load().tp_mlp_pack_shard(ctypes.byref(desc), int(shard), _ptr(w1), _ptr(w_up),
+                                    _ptr(w2), _ptr(w1p_shard), _ptr(w2p_shard), _stream(stream)))
+
+
+def tp_mlp_fwd_shard(desc, shard, x, w1p_shard, w2p_shard, partial, saved=None, workspace=None,
+                     stream=None):
+    """partial ([T][d], its dtype is the partial dtype) = act(x W1_shard) W2_shard."""
+    _check(load().tp_mlp_fwd_shard(ctypes.byref(desc), int(shard), _dt(partial), _ptr(x),
+                                   _ptr(w1p_shard), _ptr(w2p_shard), _ptr(partial), _ptr(saved),
+                                   _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def tp_mlp_bwd_shard(desc, shard, dy, x, saved, w1p_shard, w2p_shard, dx_partial, dw1p_shard,
+                     dw2p_shard, workspace=None, stream=None):
+    _check(load().tp_mlp_bwd_shard(ctypes.byref(desc), int(shard), _dt(dx_partial), _ptr(dy),
+                                   _ptr(x), _ptr(saved), _ptr(w1p_shard), _ptr(w2p_shard),
+                                   _ptr(dx_partial), _ptr(dw1p_shard), _ptr(dw2p_shard),
+                                   _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def tp_attn_shard_sizes(desc, partial_dtype="f32"):
+    out = tp_shard_sizes()
+    _check(load().tp_attn_shard_sizes(ctypes.byref(desc), _pdt(partial_dtype), ctypes.byref(out)))
+    return out
+
+
+def tp_attn_pack_shard(desc, shard, wq, wk, wv, wo, wqkv_shard, wo_shard, stream=None):
+    _check(load().tp_attn_pack_shard(ctypes.byref(desc), int(shard), _ptr(wq), _ptr(wk), _ptr(wv),
+                                     _ptr(wo), _ptr(wqkv_shard), _ptr(wo_shard), _stream(stream)))
+
+
+def tp_attn_fwd_shard(desc, shard, x, wqkv_shard, wo_shard, partial, k_cache=None, v_cache=None,
+                      workspace=None, stream=None):
+    _check(load().tp_attn_fwd_shard(ctypes.byref(desc), int(shard), _dt(partial), _ptr(x),
+                                    _ptr(wqkv_shard), _ptr(wo_shard), _ptr(k_cache), _ptr(v_cache),
+                                    _ptr(partial), _ptr(workspace), _nbytes(workspace),
+                                    _stream(stream)))
+
+
+def tp_attn_bwd_shard(desc, shard, x, wqkv_shard, wo_shard, dy, dx_partial, dwqkv_shard,
+                      dwo_shard, workspace=None, stream=None):
+    _check(load().tp_attn_bwd_shard(ctypes.byref(desc), int(shard), _ptr(x), _ptr(wqkv_shard),
+                                    _ptr(wo_shard), _ptr(dy), _ptr(dx_partial), _ptr(dwqkv_shard),
+                                    _ptr(dwo_shard), _ptr(workspace), _nbytes(workspace),
+                                    _stream(stream)))
 
 
 # ------------------------------------------------------------------- sequence parallelism
@@ -466,4 +547,19 @@ def tp_profile_read():
     while lib.tp_profile_read(i, buf, 128, ctypes.byref(n), ctypes.byref(ms)):
         out[buf.value.decode()] = (int(n.value), float(ms.value))
         i += 1
+    return out
+
+
+def tp_profile_launch_ms(label):
+    """Per-launch durations (ms, in launch order) of the kernel ``label`` recorded while profiling
+    was enabled; [] if it was not launched."""
+    lib = load()
+    names = list(tp_profile_read())
+    if label not in names:
+        return []
+    i = names.index(label)
+    out = []
+    ms = ctypes.c_double()
+    while lib.tp_profile_read_launch(i, len(out), ctypes.byref(ms)):
+        out.append(float(ms.value))
     return out
