@@ -69,6 +69,13 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
 }
 
 
+// Decode shapes the MMA decode kernel takes (the rest use the SIMT split kernel).
+inline bool decode_mma_eligible(const AttnLayout& L, const tp_attn_desc* d) {
+  const int group = d->n_q / d->n_kv;
+  return d->dtype == TP_BF16 && (L.hd == 64 || L.hd == 128) &&
+         (group == 1 || group == 2 || group == 4 || group == 8);
+}
+
 inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (!d) return set_error(TP_ERR_INVALID_ARG, "desc is null");
   if (d->b < 0 || d->s < 0) return set_error(TP_ERR_SHAPE, "b and s must be >= 0");
@@ -104,8 +111,12 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
     const int64_t n_keys = L->kv_len + 1;
     // at most one wave: splits * n_kv * b <= SMs when possible; a split's K and V rows must fit
     // in shared memory (staged by bulk copies)
-    const int64_t max_chunk = std::min<int64_t>(
+    int64_t max_chunk = std::min<int64_t>(
         512, (200 * 1024) / (2 * static_cast<int64_t>(L->hd) * L->eb + 4 * (L->n_q / L->n_kv)) / 16 * 16);
+    // the MMA decode kernel (bf16, head_dim 64/128, <= 8 query heads per KV head) stages at most
+    // 256 (head_dim 128) or 512 (head_dim 64) keys per split
+    if (decode_mma_eligible(*L, d))
+      max_chunk = std::min<int64_t>(max_chunk, L->hd == 128 ? 256 : 512);
     const int64_t want = std::max<int64_t>(1, num_sms() / std::max<int64_t>(1, L->b * L->n_kv));
     int64_t splits = std::min<int64_t>(std::min<int64_t>(want, 64), ceil_div(n_keys, 16));
     splits = std::max<int64_t>(splits, ceil_div(n_keys, max_chunk));
@@ -136,17 +147,20 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   return TP_OK;
 }
 
+// ``ldq`` / ``ldkv``: row lengths of the user's Wq and Wk / Wv when they exceed this layout's
+// (L is one shard's layout and the pointers sit at that shard's first column).
 template <typename T>
 inline tp_status attn_pack_t(const AttnLayout& L, const void* wq, const void* wk, const void* wv,
-                             const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s) {
+                             const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s,
+                             int64_t ldq = 0, int64_t ldkv = 0) {
   pack::ColMap cm{};
   cm.kind = 2;
   cm.R = L.R_a;
   cm.q_rows = static_cast<int64_t>(L.qh) * L.hd;
   cm.k_rows = static_cast<int64_t>(L.kh) * L.hd;
   cm.src[0] = wq; cm.src[1] = wk; cm.src[2] = wv;
-  cm.ld[0] = static_cast<int64_t>(L.n_q) * L.hd;
-  cm.ld[1] = cm.ld[2] = static_cast<int64_t>(L.n_kv) * L.hd;
+  cm.ld[0] = ldq > 0 ? ldq : static_cast<int64_t>(L.n_q) * L.hd;
+  cm.ld[1] = cm.ld[2] = ldkv > 0 ? ldkv : static_cast<int64_t>(L.n_kv) * L.hd;
   const int64_t rows = L.p * L.R_a;
   dim3 blk(32, 8);
   dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.h, 32)), 1);
@@ -164,9 +178,11 @@ inline tp_status attn_pack_t(const AttnLayout& L, const void* wq, const void* wk
 }
 
 inline tp_status attn_pack(const AttnLayout& L, const void* wq, const void* wk, const void* wv,
-                           const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s) {
-  return L.dtype == TP_BF16 ? attn_pack_t<__nv_bfloat16>(L, wq, wk, wv, wo, wqkv_p, wo_p, s)
-                            : attn_pack_t<float>(L, wq, wk, wv, wo, wqkv_p, wo_p, s);
+                           const void* wo, void* wqkv_p, void* wo_p, cudaStream_t s,
+                           int64_t ldq = 0, int64_t ldkv = 0) {
+  return L.dtype == TP_BF16
+             ? attn_pack_t<__nv_bfloat16>(L, wq, wk, wv, wo, wqkv_p, wo_p, s, ldq, ldkv)
+             : attn_pack_t<float>(L, wq, wk, wv, wo, wqkv_p, wo_p, s, ldq, ldkv);
 }
 
 namespace attn {
@@ -257,6 +273,84 @@ __global__ void __launch_bounds__(128) prefill_simt_kernel(const T* qkv, T* o, Q
 // holds it patches them into its staged rows and stores them into cache slot kv_len.
 // Output per (bi, q head, split): a record of hd + 4 floats, o[hd] then m (log2 units) and l
 // (16-byte aligned records, so the merge reads o with vector loads).
+// The last block of a (sequence, KV head) to finish merges all splits of its query heads, in
+// split order: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c, from the per-split records
+// (o[HD], m in log2 units, l) in ``ml``.  No block waits for another: a counter per (sequence,
+// KV head) tells each block whether it is the last, and the last one resets it.
+template <typename T, int GROUP, int HD>
+__device__ __forceinline__ void merge_splits_if_last(const float* ml, int* counters, T* o,
+                                                     int64_t bi, int g, int n_q, int n_kv) {
+  constexpr int kWarps = 8;
+  constexpr int kRec = HD + 4;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  __shared__ int s_last;
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int* cnt = counters + bi * n_kv + g;
+    const int last = atomicAdd(cnt, 1) == static_cast<int>(gridDim.x) - 1;
+    if (last) *cnt = 0;
+    s_last = last;
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  // weights w[a][c] = exp(m_c - M_a) / L_a of every split: all (m, l) pairs are loaded at once,
+  // then one warp per query head reduces over the splits with shuffles; then independent loads
+  // of the o_c
+  constexpr int kMaxSplits = 64;
+  __shared__ float s_w[GROUP][kMaxSplits], s_lc[GROUP][kMaxSplits];
+  const int splits = gridDim.x;   // <= kMaxSplits (host)
+  const float* recs = ml + (bi * n_q + static_cast<int64_t>(g) * GROUP) * splits * kRec;
+  for (int idx = threadIdx.x; idx < GROUP * splits; idx += blockDim.x) {
+    const int a = idx / splits, sp = idx - a * splits;
+    const float* r = recs + (static_cast<int64_t>(a) * splits + sp) * kRec;
+    s_w[a][sp] = __ldcg(r + HD);        // m (log2 units)
+    s_lc[a][sp] = __ldcg(r + HD + 1);   // l
+  }
+  __syncthreads();
+  for (int a = warp; a < GROUP; a += kWarps) {
+    // splits <= 64: lane handles splits lane and lane + 32
+    const float m0 = lane < splits ? s_w[a][lane] : -INFINITY;
+    const float m1 = lane + 32 < splits ? s_w[a][lane + 32] : -INFINITY;
+    float M = fmaxf(m0, m1);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
+    const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
+    const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
+    float Ls = (lane < splits ? s_lc[a][lane] * f0 : 0.f) +
+               (lane + 32 < splits ? s_lc[a][lane + 32] * f1 : 0.f);
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
+    const float inv = 1.f / Ls;
+    if (lane < splits) s_w[a][lane] = f0 * inv;
+    if (lane + 32 < splits) s_w[a][lane + 32] = f1 * inv;
+  }
+  __syncthreads();
+  // o: four consecutive dims per thread, every split's 16-byte load issued before the adds,
+  // which run in split order
+  constexpr int V4 = HD / 4;
+  for (int idx = threadIdx.x; idx < GROUP * V4; idx += blockDim.x) {
+    const int a = idx / V4, e4 = idx - a * V4;
+    const float4* r = reinterpret_cast<const float4*>(recs + static_cast<int64_t>(a) * splits * kRec) + e4;
+    float4 acc2 = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll 16
+    for (int sp = 0; sp < splits; ++sp) {
+      const float4 v = __ldcg(r + static_cast<int64_t>(sp) * (kRec / 4));
+      const float w = s_w[a][sp];
+      acc2.x += w * v.x;
+      acc2.y += w * v.y;
+      acc2.z += w * v.z;
+      acc2.w += w * v.w;
+    }
+    T* op = o + bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + 4 * e4;
+    op[0] = from_f<T>(acc2.x);
+    op[1] = from_f<T>(acc2.y);
+    op[2] = from_f<T>(acc2.z);
+    op[3] = from_f<T>(acc2.w);
+  }
+}
+
 template <int HD, int GROUP, typename T>
 struct DecodeSmem {
   static size_t bytes(int chunk) {
@@ -437,74 +531,283 @@ __global__ void __launch_bounds__(256) decode_split_kernel(const T* qkv, QkvIdx 
       }
     }
   }
-  // the last block of this (sequence, KV head) to finish merges all splits (fixed order):
-  // o = sum_c exp(m_c - M) o_c / sum_c exp(m_c - M) l_c   (no block waits for another)
-  __shared__ int s_last;
-  __threadfence();
-  __syncthreads();
+  merge_splits_if_last<T, GROUP, HD>(ml, counters, o, bi, g, n_q, n_kv);
+}
+
+
+// ---------------------------------------------------------------------------------------------
+// Decode attention for bf16 with head_dim 64 or 128 and up to 8 query heads per KV head.
+//
+// The same (split, KV head, sequence) blocks and split records as decode_split_kernel, with the
+// split's K and V rows streamed instead of staged whole:
+//   * the split is cut into sub-chunks of 32 keys; each sub-chunk's K and V arrive as 128B-swizzled
+//     TMA tiles [32 keys][64 dims] (the cache seen as [b*n_kv][kv_len][hd]; rows past the cached
+//     positions are out of bounds and arrive as zeros) on an mbarrier of their own, all issued
+//     at the start, so computing starts as soon as the first tiles land;
+//   * warp w takes the 16-key blocks w, w + 8, ...: per block, S = Q K^T for the group's query
+//     heads (rows of a 16-row MMA, the unused rows zero) and then O += P V with warp-level bf16
+//     MMAs (m16n8k16, fp32 accumulate); the fragments come from the swizzled tiles through
+//     ldmatrix, so neither product meets a shared-memory bank conflict;
+//   * each warp keeps an online softmax (running max in log2 units, running sum, rescaled O);
+//     the 8 warps' states are then combined in shared memory into the split's record;
+//   * the block holding the new token (position kv_len) patches its K and V rows into the staged
+//     tiles from the projection and stores them into cache slot kv_len.
+// The per-block contraction is tiny (at most 8 heads share a K/V row), so the MMAs only take the
+// arithmetic off the path of the HBM stream.
+template <int HD>
+struct DecodeMmaCfg {
+  static constexpr int kSub = 32;                       // keys per TMA tile / barrier
+  static constexpr int kHalves = HD / 64;               // 64-dim tiles per row
+  static constexpr int kTileBytes = kSub * 128;         // one [32][64] bf16 tile
+  static constexpr int kSubBytes = 2 * kHalves * kTileBytes;   // K and V of one sub-chunk
+  static constexpr int kMaxSub = HD == 128 ? 8 : 16;    // at most 256 (128) or 512 (64) keys
+  static constexpr int kMaxChunk = kMaxSub * kSub;
+  static constexpr size_t kSmem = static_cast<size_t>(kMaxSub) * kSubBytes + 1024;
+};
+
+__device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                        uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+__device__ __forceinline__ void ldsm_x4_t(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2,
+                                          uint32_t& r3) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.trans.shared.b16 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r0), "=r"(r1), "=r"(r2), "=r"(r3)
+               : "r"(addr));
+}
+// D (16x8, fp32) += A (16x16 bf16, row) * B (16x8 bf16, col)
+__device__ __forceinline__ void mma_16816(float (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2,
+                                          uint32_t a3, uint32_t b0, uint32_t b1) {
+  asm volatile(
+      "mma.sync.aligned.m16n8k16.row.col.f32.bf16.bf16.f32 {%0, %1, %2, %3}, "
+      "{%4, %5, %6, %7}, {%8, %9}, {%0, %1, %2, %3};"
+      : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+      : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+__device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
+  const __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+  return *reinterpret_cast<const uint32_t*>(&v);
+}
+
+template <int GROUP, int HD>
+__global__ void __launch_bounds__(256) decode_mma_kernel(
+    const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
+    const __nv_bfloat16* qkv, QkvIdx ix, __nv_bfloat16* kc, __nv_bfloat16* vc, int64_t kv_cap,
+    int64_t kv_len, int chunk, int n_q, int n_kv, float scale, float* ml, int* counters,
+    __nv_bfloat16* o, uint32_t* err) {
+  using C = DecodeMmaCfg<HD>;
+  constexpr int kWarps = 8;
+  constexpr int kRec = HD + 4;
+  constexpr int KS = HD / 16;          // k-steps of S = Q K^T
+  static_assert(GROUP >= 1 && GROUP <= 8, "at most 8 query heads per KV head");
+  extern __shared__ __align__(1024) uint8_t dsm_raw[];
+  uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
+  __shared__ __align__(8) uint64_t bars[C::kMaxSub];
+  __shared__ int s_abort;
+  const int c = blockIdx.x, g = blockIdx.y;
+  const int64_t bi = blockIdx.z;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int qr = lane >> 2, qc = lane & 3;    // MMA fragment row (query head) and column pair
+  const int64_t n_keys = kv_len + 1;
+  const int64_t k0 = static_cast<int64_t>(c) * chunk;
+  const int nk = static_cast<int>(min(n_keys, k0 + chunk) - k0);
+  const int nsub = (nk + C::kSub - 1) / C::kSub;
+  const int nblk = (nk + 15) / 16;
+  const float sl2 = scale * 1.4426950408889634f;
+  // tile (sub, kind 0 = K / 1 = V, half) of the staging area
+  auto tile = [&](int sub, int kind, int half) -> uint8_t* {
+    return dsm + static_cast<size_t>(sub) * C::kSubBytes + (kind * C::kHalves + half) * C::kTileBytes;
+  };
   if (threadIdx.x == 0) {
-    int* cnt = counters + bi * n_kv + g;
-    const int last = atomicAdd(cnt, 1) == static_cast<int>(gridDim.x) - 1;
-    if (last) *cnt = 0;
-    s_last = last;
+    for (int i = 0; i < nsub; ++i) sm100::mbar_init(&bars[i], 1);
+    s_abort = 0;
+    sm100::fence_barrier_init();
   }
   __syncthreads();
-  if (!s_last) return;
-  __threadfence();
-  // weights w[a][c] = exp(m_c - M_a) / L_a of every split: all (m, l) pairs are loaded at once,
-  // then one warp per query head reduces over the splits with shuffles; then independent loads
-  // of the o_c
-  constexpr int kMaxSplits = 64;
-  __shared__ float s_w[GROUP][kMaxSplits], s_lc[GROUP][kMaxSplits];
-  const int splits = gridDim.x;   // <= kMaxSplits (host)
-  const float* recs = ml + (bi * n_q + static_cast<int64_t>(g) * GROUP) * splits * kRec;
-  for (int idx = threadIdx.x; idx < GROUP * splits; idx += blockDim.x) {
-    const int a = idx / splits, sp = idx - a * splits;
-    const float* r = recs + (static_cast<int64_t>(a) * splits + sp) * kRec;
-    s_w[a][sp] = __ldcg(r + HD);        // m (log2 units)
-    s_lc[a][sp] = __ldcg(r + HD + 1);   // l
+  pdl_wait();   // global memory only from here on (programmatic dependent launch)
+  pdl_trigger();
+  if (threadIdx.x == 0) {
+    const int32_t z = static_cast<int32_t>(bi * n_kv + g);
+    for (int i = 0; i < nsub; ++i) {
+      sm100::mbar_arrive_expect_tx(&bars[i], C::kSubBytes);
+      const int32_t y = static_cast<int32_t>(k0 + i * C::kSub);
+      for (int hf = 0; hf < C::kHalves; ++hf) {
+        sm100::tma_load_3d(&kmap, &bars[i], tile(i, 0, hf), hf * 64, y, z);
+        sm100::tma_load_3d(&vmap, &bars[i], tile(i, 1, hf), hf * 64, y, z);
+      }
+    }
   }
-  __syncthreads();
-  for (int a = warp; a < GROUP; a += kWarps) {
-    // splits <= 64: lane handles splits lane and lane + 32
-    const float m0 = lane < splits ? s_w[a][lane] : -INFINITY;
-    const float m1 = lane + 32 < splits ? s_w[a][lane + 32] : -INFINITY;
-    float M = fmaxf(m0, m1);
+
+  // the group's query rows as MMA A fragments (rows >= GROUP and rows 8..15 are zero)
+  uint32_t qa[KS][2];
+  {
+    const __nv_bfloat16* qrow = qkv + ix.q(bi, g * GROUP + (qr < GROUP ? qr : 0));
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, off));
-    const float f0 = m0 == -INFINITY ? 0.f : exp2f(m0 - M);
-    const float f1 = m1 == -INFINITY ? 0.f : exp2f(m1 - M);
-    float Ls = (lane < splits ? s_lc[a][lane] * f0 : 0.f) +
-               (lane + 32 < splits ? s_lc[a][lane + 32] * f1 : 0.f);
+    for (int kk = 0; kk < KS; ++kk) {
+      const uint32_t lo = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qc);
+      const uint32_t hi = *reinterpret_cast<const uint32_t*>(qrow + kk * 16 + 2 * qc + 8);
+      qa[kk][0] = qr < GROUP ? lo : 0u;
+      qa[kk][1] = qr < GROUP ? hi : 0u;
+    }
+  }
+  float oacc[HD / 8][4];
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, off);
-    const float inv = 1.f / Ls;
-    if (lane < splits) s_w[a][lane] = f0 * inv;
-    if (lane + 32 < splits) s_w[a][lane + 32] = f1 * inv;
+  for (int nt = 0; nt < HD / 8; ++nt) oacc[nt][0] = oacc[nt][1] = oacc[nt][2] = oacc[nt][3] = 0.f;
+  float m_run = -INFINITY, l_run = 0.f;
+  const bool owns_new = kv_len >= k0 && kv_len < k0 + nk;
+  const int r_new = static_cast<int>(kv_len - k0);
+  int abort_local = 0;
+
+  for (int kb = warp; kb < nblk; kb += kWarps) {
+    const int sub = kb >> 1, ro = (kb & 1) * 16;
+    if (!sm100::mbar_wait(&bars[sub], 0, &s_abort, err, DEVERR_WAIT_FULL)) {
+      abort_local = 1;
+      break;
+    }
+    if (owns_new && (r_new >> 4) == kb) {
+      // the new token's key and value: from the projection into the staged tiles and the cache
+      const __nv_bfloat16* knew = qkv + ix.k(bi, g);
+      const __nv_bfloat16* vnew = qkv + ix.v(bi, g);
+      __nv_bfloat16* kdst = kc + ((bi * n_kv + g) * kv_cap + kv_len) * HD;
+      __nv_bfloat16* vdst = vc + ((bi * n_kv + g) * kv_cap + kv_len) * HD;
+      const int r = r_new & 31;
+      for (int e = lane * 4; e < HD; e += 128) {
+        const uint2 kv4 = *reinterpret_cast<const uint2*>(knew + e);
+        const uint2 vv4 = *reinterpret_cast<const uint2*>(vnew + e);
+        const int half = e >> 6, ch = (e & 63) >> 3;
+        const size_t off = static_cast<size_t>(r) * 128 + ((ch ^ (r & 7)) << 4) + (e & 7) * 2;
+        *reinterpret_cast<uint2*>(tile(sub, 0, half) + off) = kv4;
+        *reinterpret_cast<uint2*>(tile(sub, 1, half) + off) = vv4;
+        *reinterpret_cast<uint2*>(kdst + e) = kv4;
+        *reinterpret_cast<uint2*>(vdst + e) = vv4;
+      }
+      __syncwarp();
+    }
+    // ---- S = Q K^T for keys kb*16 .. kb*16+15: two n-tiles of 8 keys
+    float sacc[2][4] = {{0.f, 0.f, 0.f, 0.f}, {0.f, 0.f, 0.f, 0.f}};
+    {
+      const int mi = lane >> 3, rr = lane & 7;
+      const int r = ro + (mi >> 1) * 8 + rr;       // staged row (key) this lane addresses
+#pragma unroll
+      for (int kk = 0; kk < KS; ++kk) {
+        const int half = kk >> 2, ch = ((kk & 3) << 1) + (mi & 1);
+        const uint32_t addr = sm100::smem_addr(tile(sub, 0, half)) + r * 128 + ((ch ^ (r & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4(addr, b0, b1, b2, b3);
+        mma_16816(sacc[0], qa[kk][0], 0u, qa[kk][1], 0u, b0, b1);
+        mma_16816(sacc[1], qa[kk][0], 0u, qa[kk][1], 0u, b2, b3);
+      }
+    }
+    // ---- online softmax for query head qr over these 16 keys (log2 units)
+    float sv[2][2];
+    float mblk = -INFINITY;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        const int key = kb * 16 + n * 8 + 2 * qc + j;
+        sv[n][j] = key < nk ? sacc[n][j] * sl2 : -INFINITY;
+        mblk = fmaxf(mblk, sv[n][j]);
+      }
+    mblk = fmaxf(mblk, __shfl_xor_sync(0xffffffffu, mblk, 1));
+    mblk = fmaxf(mblk, __shfl_xor_sync(0xffffffffu, mblk, 2));
+    const float m_new = fmaxf(m_run, mblk);       // finite: the block's first key is valid
+    const float corr = exp2f(m_run - m_new);      // 0 on the first block (m_run = -inf)
+    float p[2][2];
+    float psum = 0.f;
+#pragma unroll
+    for (int n = 0; n < 2; ++n)
+#pragma unroll
+      for (int j = 0; j < 2; ++j) {
+        p[n][j] = exp2f(sv[n][j] - m_new);
+        psum += p[n][j];
+      }
+    l_run = l_run * corr + psum;
+    m_run = m_new;
+#pragma unroll
+    for (int nt = 0; nt < HD / 8; ++nt) {
+      oacc[nt][0] *= corr;
+      oacc[nt][1] *= corr;
+    }
+    // ---- O += P V: P (head rows, 16 keys) as the A fragment straight from the S layout
+    const uint32_t pa0 = pack_bf16x2(p[0][0], p[0][1]);
+    const uint32_t pa2 = pack_bf16x2(p[1][0], p[1][1]);
+    {
+      const int mi = lane >> 3, rr = lane & 7;
+      const int r = ro + (mi & 1) * 8 + rr;
+#pragma unroll
+      for (int np = 0; np < HD / 16; ++np) {
+        const int half = np >> 2, ch = ((np & 3) << 1) + (mi >> 1);
+        const uint32_t addr = sm100::smem_addr(tile(sub, 1, half)) + r * 128 + ((ch ^ (r & 7)) << 4);
+        uint32_t b0, b1, b2, b3;
+        ldsm_x4_t(addr, b0, b1, b2, b3);
+        mma_16816(oacc[2 * np], pa0, 0u, pa2, 0u, b0, b1);
+        mma_16816(oacc[2 * np + 1], pa0, 0u, pa2, 0u, b2, b3);
+      }
+    }
+  }
+  // the row sum over the quad's lanes
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
+  l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
+
+  // ---- abort path: every tile must land before the block leaves (bounded), then return
+  if (abort_local) s_abort = 1;
+  __syncthreads();
+  if (s_abort) {
+    if (threadIdx.x < nsub) {
+      const uint64_t t0 = globaltimer_ns();
+      while (!sm100::mbar_try_wait(&bars[threadIdx.x], 0) && globaltimer_ns() - t0 < kWaitTimeoutNs) {
+      }
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- combine the 8 warps' states (the staging area is free now)
+  float* wo = reinterpret_cast<float*>(dsm);                       // [warp][GROUP][HD]
+  float* wm = wo + kWarps * GROUP * HD;                             // [warp][GROUP]
+  float* wl = wm + kWarps * GROUP;
+  if (qr < GROUP) {
+#pragma unroll
+    for (int nt = 0; nt < HD / 8; ++nt)
+      *reinterpret_cast<float2*>(&wo[(warp * GROUP + qr) * HD + nt * 8 + 2 * qc]) =
+          make_float2(oacc[nt][0], oacc[nt][1]);
+    if (qc == 0) {
+      wm[warp * GROUP + qr] = m_run;
+      wl[warp * GROUP + qr] = l_run;
+    }
   }
   __syncthreads();
-  // o: four consecutive dims per thread, every split's 16-byte load issued before the adds,
-  // which run in split order
   constexpr int V4 = HD / 4;
   for (int idx = threadIdx.x; idx < GROUP * V4; idx += blockDim.x) {
     const int a = idx / V4, e4 = idx - a * V4;
-    const float4* r = reinterpret_cast<const float4*>(recs + static_cast<int64_t>(a) * splits * kRec) + e4;
-    float4 acc2 = make_float4(0.f, 0.f, 0.f, 0.f);
-#pragma unroll 16
-    for (int sp = 0; sp < splits; ++sp) {
-      const float4 v = __ldcg(r + static_cast<int64_t>(sp) * (kRec / 4));
-      const float w = s_w[a][sp];
-      acc2.x += w * v.x;
-      acc2.y += w * v.y;
-      acc2.z += w * v.z;
-      acc2.w += w * v.w;
+    float M = -INFINITY;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) M = fmaxf(M, wm[w * GROUP + a]);
+    float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+    float L = 0.f;
+#pragma unroll
+    for (int w = 0; w < kWarps; ++w) {
+      const float mw = wm[w * GROUP + a];
+      const float f = mw == -INFINITY ? 0.f : exp2f(mw - M);
+      const float4 v = *reinterpret_cast<const float4*>(&wo[(w * GROUP + a) * HD + 4 * e4]);
+      acc.x += f * v.x;
+      acc.y += f * v.y;
+      acc.z += f * v.z;
+      acc.w += f * v.w;
+      L += f * wl[w * GROUP + a];
     }
-    T* op = o + bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + 4 * e4;
-    op[0] = from_f<T>(acc2.x);
-    op[1] = from_f<T>(acc2.y);
-    op[2] = from_f<T>(acc2.z);
-    op[3] = from_f<T>(acc2.w);
+    const int j = g * GROUP + a;
+    float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * kRec;
+    *reinterpret_cast<float4*>(rec + 4 * e4) = acc;
+    if (e4 == 0) {
+      rec[HD] = M;
+      rec[HD + 1] = L;
+    }
   }
+  merge_splits_if_last<__nv_bfloat16, GROUP, HD>(ml, counters, o, bi, g, n_q, n_kv);
 }
 
 }  // namespace attn
@@ -545,6 +848,46 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
     const int64_t words = L.b * L.n_kv;
     TP_LAUNCH_PDL(zero_words_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words, 256), 64))),
                   dim3(256), 0, s, reinterpret_cast<uint32_t*>(counters), words);
+  }
+  if constexpr (sizeof(T) == 2) {
+    const bool mma = tensor_cores_usable() && (L.hd == 64 || L.hd == 128) &&
+                     (group == 1 || group == 2 || group == 4 || group == 8) &&
+                     L.kv_chunk <= (L.hd == 128 ? attn::DecodeMmaCfg<128>::kMaxChunk
+                                                : attn::DecodeMmaCfg<64>::kMaxChunk) &&
+                     L.kv_len <= INT32_MAX - 512 && L.b * L.n_kv <= INT32_MAX;
+    if (mma) {
+      // the caches as [b*n_kv][kv_len][hd]: the new token's slot and any slot past it read as zeros
+      CUtensorMap km, vm;
+      const uint64_t hd = static_cast<uint64_t>(L.hd);
+      tp_status r = encode_tmap_bf16_3d(&km, kc, hd, static_cast<uint64_t>(L.kv_len),
+                                        static_cast<uint64_t>(L.b * L.n_kv), hd * 2,
+                                        static_cast<uint64_t>(L.kv_cap) * hd * 2, 64,
+                                        attn::DecodeMmaCfg<128>::kSub);
+      if (r != TP_OK) return r;
+      r = encode_tmap_bf16_3d(&vm, vc, hd, static_cast<uint64_t>(L.kv_len),
+                              static_cast<uint64_t>(L.b * L.n_kv), hd * 2,
+                              static_cast<uint64_t>(L.kv_cap) * hd * 2, 64,
+                              attn::DecodeMmaCfg<128>::kSub);
+      if (r != TP_OK) return r;
+#define TP_DECODE_MMA_CASE(G, H)                                                              \
+      if (group == G && L.hd == H) {                                                          \
+        auto* kern = attn::decode_mma_kernel<G, H>;                                           \
+        const size_t smem = attn::DecodeMmaCfg<H>::kSmem;                                     \
+        TP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
+                                         static_cast<int>(smem)));                            \
+        ProfScope prof(s, "attn_decode");                                                     \
+        TP_LAUNCH_PDL(kern, grid, dim3(256), smem, s, km, vm,                                 \
+                      reinterpret_cast<const __nv_bfloat16*>(qkv), ix,                        \
+                      static_cast<__nv_bfloat16*>(kc), static_cast<__nv_bfloat16*>(vc),       \
+                      L.kv_cap, L.kv_len, L.kv_chunk, L.n_q, L.n_kv, scale, ml, counters,     \
+                      reinterpret_cast<__nv_bfloat16*>(o), device_error_word());             \
+        return TP_OK;                                                                         \
+      }
+      TP_DECODE_MMA_CASE(8, 128) TP_DECODE_MMA_CASE(4, 128) TP_DECODE_MMA_CASE(2, 128)
+      TP_DECODE_MMA_CASE(1, 128) TP_DECODE_MMA_CASE(8, 64) TP_DECODE_MMA_CASE(4, 64)
+      TP_DECODE_MMA_CASE(2, 64) TP_DECODE_MMA_CASE(1, 64)
+#undef TP_DECODE_MMA_CASE
+    }
   }
 #define TP_DECODE_CASE(G, H)                                                                  \
   if (group == G && L.hd == H) {                                                              \

@@ -91,6 +91,39 @@ def test_decode(lib, dtype, b, kv_len, h, n_q, n_kv, hd, p, mode):
     assert np.array_equal(f64(kc)[:, :, :kv_len], kc0)
 
 
+@pytest.mark.parametrize("b,kv_len,n_q,n_kv,hd,spare", [
+    (1, 64, 4, 4, 128, 0),     # one query head per KV head; the new token opens a 32-key tile
+    (2, 31, 8, 4, 128, 7),     # two per KV head; the new token closes a tile; spare slots
+    (1, 4111, 16, 2, 128, 0),  # eight per KV head, a last split of a few keys
+    (2, 700, 8, 2, 64, 33),    # head_dim 64, four per KV head, spare slots past the new token
+    (3, 17, 16, 2, 64, 0),     # one split holding 18 keys
+])
+def test_decode_edges(lib, b, kv_len, n_q, n_kv, hd, spare):
+    # slots past the new token (kv_cap > kv_len + 1) hold NaN: they must never be read
+    h, p = 256, 2
+    inp = inputs.attn_inputs(b, 1, h, n_q, n_kv, hd, "bf16", seed=5, w_std=0.05, kv_len=kv_len)
+    cap = kv_len + 1 + spare
+    kc = torch.full((b, n_kv, cap, hd), float("nan"), dtype=torch.bfloat16, device=dev())
+    vc = torch.full_like(kc, float("nan"))
+    kc[:, :, :kv_len] = inp["k_cache"][:, :, :kv_len].to(dev())
+    vc[:, :, :kv_len] = inp["v_cache"][:, :, :kv_len].to(dev())
+    a = Attn(lib, inp, p, "bf16", True, kv_len=kv_len, n_q=n_q, n_kv=n_kv, hd=hd)
+    desc = lib.attn_desc(b, 1, h, n_q, n_kv, hd, p, True, "bf16", kv_len, kv_cap=cap)
+    ws = torch.empty(lib.tp_attn_fwd_workspace(desc), dtype=torch.uint8, device=dev())
+    y = torch.empty(b, 1, h, dtype=torch.bfloat16, device=dev())
+    lib.tp_attn_fwd(desc, inp["x"].to(dev()), a.wqkv, a.wo, y, k_cache=kc, v_cache=vc, workspace=ws)
+    torch.cuda.synchronize()
+    kc0, vc0 = f64(inp["k_cache"])[:, :, :kv_len], f64(inp["v_cache"])[:, :, :kv_len]
+    ref, kn, vn = oattn.attention_decode(f64(inp["x"])[:, 0], *(f64(inp[k]) for k in ("wq", "wk", "wv", "wo")),
+                                         kc0, vc0, n_q, n_kv, hd)
+    assert rel_l2(f64(y)[:, 0], ref) <= TOL["bf16"]
+    assert rel_l2_rows(f64(y)[:, 0], ref) <= TOL["bf16"]
+    assert rel_l2(f64(kc)[:, :, kv_len], kn) <= TOL["bf16"]
+    assert rel_l2(f64(vc)[:, :, kv_len], vn) <= TOL["bf16"]
+    assert np.array_equal(f64(kc)[:, :, :kv_len], kc0)
+    assert torch.isnan(kc[:, :, kv_len + 1:].float()).all()
+
+
 def test_decode_matches_prefill_last_row(lib):
     # decoding position L over a cache holding the keys/values of positions 0..L-1 equals the
     # last row of causal prefill over L+1 tokens (both through the library)
