@@ -185,3 +185,127 @@ extern "C" tp_status tp_attn_unpack_grads(const tp_attn_desc* desc, const void* 
                                static_cast<float*>(dwk), static_cast<float*>(dwv),
                                static_cast<float*>(dwo), static_cast<cudaStream_t>(stream));
 }
+
+// ------------------------------------------------------------------------ one shard per device
+// "Tensor Parallelism" (klaylearn), Notes: with one shard per GPU, device i owns n_q/p query heads
+// and n_kv/p KV heads (its column slices of Wq, Wk, Wv and its KV cache), runs attention over
+// them locally, and turns its heads' output into a full-width partial through its row slice of
+// Wo; the devices' all-reduce adds the partials.  Shard i on its own is the block with p = 1 and
+// n_q/p, n_kv/p heads, whose packed layout is exactly shard i's slice of the p-shard packing;
+// these calls run that problem and leave the sum to the caller's collective (nothing is added to
+// the reduction counter).
+namespace {
+tp_status attn_shard_desc(const tp_attn_desc* desc, int32_t shard, int32_t partial_dtype,
+                          tp_attn_desc* sd, tp::AttnLayout* LS) {
+  tp::AttnLayout L;
+  tp_status st = tp::attn_layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (shard < 0 || shard >= L.p) return tp::set_error(TP_ERR_INVALID_ARG, "shard must be in 0 .. p-1");
+  if (partial_dtype != TP_F32 && partial_dtype != TP_BF16)
+    return tp::set_error(TP_ERR_INVALID_ARG, "partial_dtype must be TP_F32 or TP_BF16");
+  if (L.dtype == TP_F32 && partial_dtype != TP_F32)
+    return tp::set_error(TP_ERR_UNSUPPORTED, "fp32 blocks give fp32 partials");
+  if (desc->flags != 0)
+    return tp::set_error(TP_ERR_INVALID_ARG, "shard calls take no flags (partial_dtype sets the type)");
+  *sd = *desc;
+  sd->n_q = desc->n_q / desc->p;
+  sd->n_kv = desc->n_kv / desc->p;
+  sd->p = 1;
+  sd->flags = (L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0;
+  sd->reduce_mode = L.tc ? TP_REDUCE_FUSED : TP_REDUCE_SEPARATE;
+  return tp::attn_layout_of(sd, LS);
+}
+}  // namespace
+
+extern "C" tp_status tp_attn_shard_sizes(const tp_attn_desc* desc, int32_t partial_dtype,
+                                         tp_shard_sizes* out) {
+  tp::clear_error();
+  if (!out) return tp::set_error(TP_ERR_INVALID_ARG, "out is null");
+  tp_attn_desc sd;
+  tp::AttnLayout L;
+  tp_status st = attn_shard_desc(desc, 0, partial_dtype, &sd, &L);
+  if (st != TP_OK) return st;
+  out->col_weight_bytes = L.wqkv_bytes;
+  out->row_weight_bytes = L.wo_bytes;
+  out->saved_bytes = 0;
+  out->fwd_workspace = L.ws_bytes;
+  tp::AttnLayout LB;
+  const bool bwd_ok = partial_dtype == TP_BF16 && attn_bwd_check(&sd, &LB) == TP_OK;
+  tp::clear_error();
+  out->bwd_workspace = bwd_ok ? tp::attn_bwd_layout(LB).bytes : 0;
+  out->partial_bytes = static_cast<size_t>(L.tokens * L.h) * tp::elem_bytes(partial_dtype);
+  return TP_OK;
+}
+
+extern "C" tp_status tp_attn_pack_shard(const tp_attn_desc* desc, int32_t shard, const void* wq,
+                                        const void* wk, const void* wv, const void* wo,
+                                        void* wqkv_shard, void* wo_shard, void* stream) {
+  tp::clear_error();
+  tp_attn_desc sd;
+  tp::AttnLayout L;
+  tp_status st = attn_shard_desc(desc, shard, desc ? desc->dtype : TP_F32, &sd, &L);
+  if (st != TP_OK) return st;
+  if (!wq || !wk || !wv || !wo || !wqkv_shard || !wo_shard)
+    return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  const size_t eb = static_cast<size_t>(L.eb);
+  const int64_t qcols = static_cast<int64_t>(L.n_q) * L.hd;    // this shard's Wq columns
+  const int64_t kcols = static_cast<int64_t>(L.n_kv) * L.hd;
+  const int64_t q0 = static_cast<int64_t>(shard) * qcols, k0 = static_cast<int64_t>(shard) * kcols;
+  return tp::attn_pack(L, static_cast<const uint8_t*>(wq) + q0 * eb,
+                       static_cast<const uint8_t*>(wk) + k0 * eb,
+                       static_cast<const uint8_t*>(wv) + k0 * eb,
+                       static_cast<const uint8_t*>(wo) + q0 * L.h * eb, wqkv_shard, wo_shard,
+                       static_cast<cudaStream_t>(stream), static_cast<int64_t>(desc->n_q) * L.hd,
+                       static_cast<int64_t>(desc->n_kv) * L.hd);
+}
+
+extern "C" tp_status tp_attn_fwd_shard(const tp_attn_desc* desc, int32_t shard,
+                                       int32_t partial_dtype, const void* x,
+                                       const void* wqkv_shard, const void* wo_shard,
+                                       void* k_cache_shard, void* v_cache_shard, void* partial,
+                                       void* workspace, size_t ws_bytes, void* stream) {
+  tp::clear_error();
+  tp_attn_desc sd;
+  tp::AttnLayout L;
+  tp_status st = attn_shard_desc(desc, shard, partial_dtype, &sd, &L);
+  if (st != TP_OK) return st;
+  if (L.tokens == 0) return TP_OK;
+  if (!x || !wqkv_shard || !wo_shard || !partial) return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (L.kv_len > 0 && (!k_cache_shard || !v_cache_shard))
+    return tp::set_error(TP_ERR_INVALID_ARG, "decode needs k_cache and v_cache");
+  if (L.kv_len > 0 &&
+      ((reinterpret_cast<uintptr_t>(k_cache_shard) | reinterpret_cast<uintptr_t>(v_cache_shard)) & 15))
+    return tp::set_error(TP_ERR_INVALID_ARG, "k_cache and v_cache must be 16-byte aligned");
+  if (!workspace) return tp::set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < L.ws_bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
+  return tp::attn_forward(L, x, wqkv_shard, wo_shard, k_cache_shard, v_cache_shard, nullptr,
+                          partial, nullptr, workspace, static_cast<cudaStream_t>(stream));
+}
+
+extern "C" tp_status tp_attn_bwd_shard(const tp_attn_desc* desc, int32_t shard, const void* x,
+                                       const void* wqkv_shard, const void* wo_shard,
+                                       const void* dy, void* dx_partial, void* dwqkv_shard,
+                                       void* dwo_shard, void* workspace, size_t ws_bytes,
+                                       void* stream) {
+  tp::clear_error();
+  tp_attn_desc sd;
+  tp::AttnLayout L0;
+  tp_status st = attn_shard_desc(desc, shard, TP_BF16, &sd, &L0);
+  if (st != TP_OK) return st;
+  tp::AttnLayout L;
+  if ((st = attn_bwd_check(&sd, &L)) != TP_OK) return st;
+  if (L.tokens == 0) return TP_OK;
+  if (!x || !wqkv_shard || !wo_shard || !dy || !dx_partial || !dwqkv_shard || !dwo_shard || !workspace)
+    return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  for (const void* q : {x, wqkv_shard, wo_shard, dy, static_cast<const void*>(dx_partial),
+                        static_cast<const void*>(dwqkv_shard), static_cast<const void*>(dwo_shard)})
+    if (reinterpret_cast<uintptr_t>(q) & 15)
+      return tp::set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const tp::AttnBwdLayout B = tp::attn_bwd_layout(L);
+  if (ws_bytes < B.bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tp::tensor_cores_usable())
+    return tp::set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  return tp::attn_backward(L, x, wqkv_shard, wo_shard, dy, dx_partial,
+                           static_cast<float*>(dwqkv_shard), static_cast<float*>(dwo_shard),
+                           workspace, static_cast<cudaStream_t>(stream));
+}

@@ -232,7 +232,7 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
 // (``dx``); otherwise it writes the fp32 partials to ``part`` for the separate reduce.
 tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const void* z,
                       const void* h, const void* w1p, const void* w2p, void* dz, float* dw1p,
-                      float* dw2p, float* part, void* dx, cudaStream_t s) {
+                      float* dw2p, float* part, void* dx, bool dx_f32, cudaStream_t s) {
   const int64_t P = L.p;
   tp_status st;
   // (1) dH_i = dY W2_i^T with the activation backward fused: dz in w1p row order
@@ -299,7 +299,7 @@ tp_status tc_backward(const MlpLayout& L, const void* dy, const void* x, const v
       ep.ld = L.d;
       ep.rows_valid = static_cast<int32_t>(L.T);
       ep.cols_valid = static_cast<int32_t>(L.d);
-      ep.out_bf16 = 1;
+      ep.out_bf16 = dx_f32 ? 0 : 1;
       ep.swap = 0;
       return tc::run_gemm_pair<PP<false, true>, tc::EpiReduceOut>(a, b, L.T, L.d, L.R, P, ep, s,
                                                                   "mlp_dx_gemm", -1, true);
@@ -397,14 +397,18 @@ pack::ColMap w1_colmap(const MlpLayout& L, const void* w1, const void* wu) {
   return cm;
 }
 
+// ``ld1`` is the row length of the user's W1 / Wu (their d_ff; larger than L.F when L is one
+// shard's layout and w1 / wu / w2 already point at that shard's first column / row).
 template <typename T>
 tp_status pack_t(const MlpLayout& L, const void* w1, const void* wu, const void* w2, void* w1p,
-                 void* w2p, cudaStream_t s) {
+                 void* w2p, cudaStream_t s, int64_t ld1 = 0) {
   const int64_t rows = L.p * L.R;
   dim3 blk(32, 8);
   dim3 g1(static_cast<unsigned>(ceil_div(rows, 32)), static_cast<unsigned>(ceil_div(L.d, 32)), 1);
   if (!pack::grid_ok(g1.x, g1.y, 1)) return set_error(TP_ERR_UNSUPPORTED, "pack grid too large");
-  pack::pack_cols_kernel<T><<<g1, blk, 0, s>>>(static_cast<T*>(w1p), rows, L.d, w1_colmap(L, w1, wu));
+  pack::ColMap cm = w1_colmap(L, w1, wu);
+  if (ld1 > 0) cm.ld[0] = cm.ld[1] = ld1;
+  pack::pack_cols_kernel<T><<<g1, blk, 0, s>>>(static_cast<T*>(w1p), rows, L.d, cm);
   TP_LAUNCH_CHECK();
   dim3 g2(static_cast<unsigned>(ceil_div(L.d, 32)), static_cast<unsigned>(ceil_div(L.Fsp, 32)),
           static_cast<unsigned>(L.p));
@@ -481,24 +485,24 @@ extern "C" tp_status tp_mlp_unpack_grads(const tp_mlp_desc* desc, const void* dw
   return TP_OK;
 }
 
-extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p,
-                                const void* w2p, const void* residual, void* y, void* y_norm,
-                                void* saved, void* workspace, size_t ws_bytes, void* stream) {
-  clear_error();
-  MlpLayout L;
-  tp_status st = layout_of(desc, &L);
-  if (st != TP_OK) return st;
+namespace tp {
+namespace {
+// The forward on layout L.  ``count``: add the reduction to the counter (not for a shard's
+// partial, whose reduction is the caller's collective).
+tp_status mlp_forward(const MlpLayout& L, const tp_mlp_desc* desc, const void* x, const void* w1p,
+                      const void* w2p, const void* residual, void* y, void* y_norm, void* saved,
+                      void* workspace, size_t ws_bytes, cudaStream_t s, bool count) {
+  tp_status st;
   if (desc->reduce_mode == TP_REDUCE_FUSED && !L.tc)
     return set_error(TP_ERR_UNSUPPORTED,
                      "TP_REDUCE_FUSED needs the tensor-core path (bf16, d a multiple of 8)");
   if (L.T == 0) {
-    count_reduction();
+    if (count) count_reduction();
     return TP_OK;
   }
   if (!x || !w1p || !w2p || !y) return set_error(TP_ERR_INVALID_ARG, "null pointer");
   if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
   if (ws_bytes < L.fwd_ws) return set_error(TP_ERR_WORKSPACE, "workspace too small");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   void* z = saved ? off(saved, L.saved_z_off) : off(workspace, L.fz_off);
   void* h = saved ? off(saved, L.saved_h_off) : off(workspace, L.fh_off);
   float* part = reinterpret_cast<float*>(off(workspace, L.fpart_off));
@@ -516,7 +520,7 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
     if (L.reduce_mode == TP_REDUCE_FUSED) {
       if (y_norm && (st = reduce::rmsnorm(y, L.y_dtype, L.T, L.d, L.norm_eps, y_norm, L.dtype, s)) != TP_OK)
         return st;
-      count_reduction();
+      if (count) count_reduction();
       return TP_OK;
     }
   } else if (L.dtype == TP_BF16) {
@@ -527,24 +531,21 @@ extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const vo
   st = y_norm ? reduce::reduce_norm(part, L.p, L.T, L.d, residual, y, L.y_dtype, y_norm, L.dtype,
                                     L.norm_eps, s)
               : reduce::launch(part, TP_F32, L.p, L.T * L.d, residual, y, L.y_dtype, s);
-  if (st == TP_OK) count_reduction();
+  if (st == TP_OK && count) count_reduction();
   return st;
 }
 
-extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const void* x,
-                                const void* saved, const void* w1p, const void* w2p, void* dx,
-                                void* dw1p, void* dw2p, void* workspace, size_t ws_bytes,
-                                void* stream) {
-  clear_error();
-  MlpLayout L;
-  tp_status st = layout_of(desc, &L);
-  if (st != TP_OK) return st;
+// The backward on layout L; dx in L.dtype, or fp32 when ``dx_f32``.
+tp_status mlp_backward(const MlpLayout& L, const void* dy, const void* x, const void* saved,
+                       const void* w1p, const void* w2p, void* dx, void* dw1p, void* dw2p,
+                       void* workspace, size_t ws_bytes, cudaStream_t s, bool dx_f32,
+                       bool count) {
+  tp_status st;
   if (!w1p || !w2p || !dw1p || !dw2p) return set_error(TP_ERR_INVALID_ARG, "null pointer");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (L.T == 0) {  // no tokens: zero weight gradients, nothing else
     TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(L.p * L.R * L.d) * 4, s));
     TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(L.p * L.d * L.Fsp) * 4, s));
-    count_reduction();
+    if (count) count_reduction();
     return TP_OK;
   }
   if (!dy || !x || !saved || !dx) return set_error(TP_ERR_INVALID_ARG, "null pointer");
@@ -562,9 +563,9 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
       return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {dy, x, saved, w1p, w2p, static_cast<const void*>(dx)})
       if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, dx, s);
+    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, dx, dx_f32, s);
     if (st == TP_OK && L.reduce_mode == TP_REDUCE_FUSED) {   // dx already summed
-      count_reduction();
+      if (count) count_reduction();
       return TP_OK;
     }
   } else if (L.dtype == TP_BF16) {
@@ -573,9 +574,135 @@ extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const v
     st = simt_backward<float>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
   }
   if (st != TP_OK) return st;
-  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, nullptr, dx, L.dtype, s);
-  if (st == TP_OK) count_reduction();
+  st = reduce::launch(part, TP_F32, L.p, L.T * L.d, nullptr, dx, dx_f32 ? TP_F32 : L.dtype, s);
+  if (st == TP_OK && count) count_reduction();
   return st;
+}
+}  // namespace
+}  // namespace tp
+
+extern "C" tp_status tp_mlp_fwd(const tp_mlp_desc* desc, const void* x, const void* w1p,
+                                const void* w2p, const void* residual, void* y, void* y_norm,
+                                void* saved, void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  return mlp_forward(L, desc, x, w1p, w2p, residual, y, y_norm, saved, workspace, ws_bytes,
+                     static_cast<cudaStream_t>(stream), true);
+}
+
+extern "C" tp_status tp_mlp_bwd(const tp_mlp_desc* desc, const void* dy, const void* x,
+                                const void* saved, const void* w1p, const void* w2p, void* dx,
+                                void* dw1p, void* dw2p, void* workspace, size_t ws_bytes,
+                                void* stream) {
+  clear_error();
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  return mlp_backward(L, dy, x, saved, w1p, w2p, dx, dw1p, dw2p, workspace, ws_bytes,
+                      static_cast<cudaStream_t>(stream), false, true);
+}
+
+// ------------------------------------------------------------------------ one shard per device
+// "Tensor Parallelism" (klaylearn), Notes, and "How does tensor parallelism split a transformer
+// feed-forward block's two matmuls", "One collective": with one shard per GPU, device i holds
+// the column slice W1_i (and Wu_i) and the row slice W2_i, computes h_i = act(x W1_i) and the
+// full-shape partial y_i = h_i W2_i, and the devices' all-reduce adds the partials.  Shard i on
+// its own is the block with p = 1 and d_ff / p features, whose packed layout is exactly shard i's
+// slice of the p-shard packing; these calls run that problem and leave the sum to the caller's
+// collective (so they add nothing to the reduction counter).
+namespace tp {
+namespace {
+tp_status shard_desc_of(const tp_mlp_desc* desc, int32_t shard, int32_t partial_dtype,
+                        tp_mlp_desc* sd, MlpLayout* LS) {
+  MlpLayout L;
+  tp_status st = layout_of(desc, &L);
+  if (st != TP_OK) return st;
+  if (shard < 0 || shard >= L.p) return set_error(TP_ERR_INVALID_ARG, "shard must be in 0 .. p-1");
+  if (partial_dtype != TP_F32 && partial_dtype != TP_BF16)
+    return set_error(TP_ERR_INVALID_ARG, "partial_dtype must be TP_F32 or TP_BF16");
+  if (L.dtype == TP_F32 && partial_dtype != TP_F32)
+    return set_error(TP_ERR_UNSUPPORTED, "fp32 blocks give fp32 partials");
+  if (desc->flags != 0)
+    return set_error(TP_ERR_INVALID_ARG, "shard calls take no flags (partial_dtype sets the type)");
+  *sd = *desc;
+  sd->d_ff = L.Fs;
+  sd->p = 1;
+  sd->flags = (L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0;
+  sd->reduce_mode = L.tc ? TP_REDUCE_FUSED : TP_REDUCE_SEPARATE;
+  return layout_of(sd, LS);
+}
+}  // namespace
+}  // namespace tp
+
+extern "C" tp_status tp_mlp_shard_sizes(const tp_mlp_desc* desc, int32_t partial_dtype,
+                                        tp_shard_sizes* out) {
+  clear_error();
+  if (!out) return set_error(TP_ERR_INVALID_ARG, "out is null");
+  tp_mlp_desc sd;
+  MlpLayout L;
+  tp_status st = shard_desc_of(desc, 0, partial_dtype, &sd, &L);
+  if (st != TP_OK) return st;
+  out->col_weight_bytes = L.w1p_bytes;
+  out->row_weight_bytes = L.w2p_bytes;
+  out->saved_bytes = L.saved_bytes;
+  out->fwd_workspace = L.fwd_ws;
+  out->bwd_workspace = L.bwd_ws;
+  out->partial_bytes = static_cast<size_t>(L.T * L.d) * elem_bytes(partial_dtype);
+  return TP_OK;
+}
+
+extern "C" tp_status tp_mlp_pack_shard(const tp_mlp_desc* desc, int32_t shard, const void* w1,
+                                       const void* w_up, const void* w2, void* w1p_shard,
+                                       void* w2p_shard, void* stream) {
+  clear_error();
+  tp_mlp_desc sd;
+  MlpLayout L;
+  tp_status st = shard_desc_of(desc, shard, desc ? desc->dtype : TP_F32, &sd, &L);
+  if (st != TP_OK) return st;
+  if (!w1 || !w2 || !w1p_shard || !w2p_shard) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if ((L.act == TP_ACT_SWIGLU) != (w_up != nullptr))
+    return set_error(TP_ERR_INVALID_ARG, "w_up must be given exactly for TP_ACT_SWIGLU");
+  // shard i's first column of W1 / Wu and first row of W2 in the user's full matrices
+  const int64_t col0 = static_cast<int64_t>(shard) * L.Fs;
+  const size_t eb = static_cast<size_t>(L.eb);
+  const uint8_t* w1s = static_cast<const uint8_t*>(w1) + col0 * eb;
+  const uint8_t* wus = w_up ? static_cast<const uint8_t*>(w_up) + col0 * eb : nullptr;
+  const uint8_t* w2s = static_cast<const uint8_t*>(w2) + col0 * L.d * eb;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return L.dtype == TP_BF16
+             ? pack_t<__nv_bfloat16>(L, w1s, wus, w2s, w1p_shard, w2p_shard, s, desc->d_ff)
+             : pack_t<float>(L, w1s, wus, w2s, w1p_shard, w2p_shard, s, desc->d_ff);
+}
+
+extern "C" tp_status tp_mlp_fwd_shard(const tp_mlp_desc* desc, int32_t shard,
+                                      int32_t partial_dtype, const void* x, const void* w1p_shard,
+                                      const void* w2p_shard, void* partial, void* saved_shard,
+                                      void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  tp_mlp_desc sd;
+  MlpLayout L;
+  tp_status st = shard_desc_of(desc, shard, partial_dtype, &sd, &L);
+  if (st != TP_OK) return st;
+  return mlp_forward(L, &sd, x, w1p_shard, w2p_shard, nullptr, partial, nullptr, saved_shard,
+                     workspace, ws_bytes, static_cast<cudaStream_t>(stream), false);
+}
+
+extern "C" tp_status tp_mlp_bwd_shard(const tp_mlp_desc* desc, int32_t shard,
+                                      int32_t partial_dtype, const void* dy, const void* x,
+                                      const void* saved_shard, const void* w1p_shard,
+                                      const void* w2p_shard, void* dx_partial, void* dw1p_shard,
+                                      void* dw2p_shard, void* workspace, size_t ws_bytes,
+                                      void* stream) {
+  clear_error();
+  tp_mlp_desc sd;
+  MlpLayout L;
+  tp_status st = shard_desc_of(desc, shard, partial_dtype, &sd, &L);
+  if (st != TP_OK) return st;
+  return mlp_backward(L, dy, x, saved_shard, w1p_shard, w2p_shard, dx_partial, dw1p_shard,
+                      dw2p_shard, workspace, ws_bytes, static_cast<cudaStream_t>(stream),
+                      partial_dtype == TP_F32, false);
 }
 
 // ------------------------------------------------------------------ sequence-parallel variant
@@ -703,7 +830,7 @@ extern "C" tp_status tp_mlp_bwd_sp(const tp_mlp_desc* desc, const void* const* d
       return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
     for (const void* q : {saved, w1p, w2p})
       if (!aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
-    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, nullptr, s);
+    st = tc_backward(L, dy, x, z, h, w1p, w2p, dz, g1, g2, part, nullptr, false, s);
   } else if (L.dtype == TP_BF16) {
     st = simt_backward<__nv_bfloat16>(L, dy, x, z, h, w1p, w2p, dh, dz, g1, g2, part, s);
   } else {

@@ -249,3 +249,54 @@ def test_product_and_oracle_are_independent():
     csrc = os.path.join(pkg, "csrc")
     for f in os.listdir(csrc):
         assert "oracle" not in open(os.path.join(csrc, f)).read().lower(), f
+
+
+def test_shard_sizes_are_one_pth_of_the_packing(lib):
+    # one shard per device: its packed weights are exactly its slice of the p-shard packing
+    d = lib.mlp_desc(64, 8192, 28672, 8, "swiglu", "bf16")
+    s = lib.tp_mlp_shard_sizes(d, "bf16")
+    assert s.col_weight_bytes * 8 == lib.tp_mlp_w1_packed_bytes(d)
+    assert s.row_weight_bytes * 8 == lib.tp_mlp_w2_packed_bytes(d)
+    assert s.partial_bytes == 64 * 8192 * 2          # the pages' 1 MiB decode all-reduce payload
+    assert lib.tp_mlp_shard_sizes(d, "f32").partial_bytes == 64 * 8192 * 4
+    a = lib.attn_desc(1, 2048, 8192, 64, 8, 128, 8)
+    sa = lib.tp_attn_shard_sizes(a, "f32")
+    assert sa.col_weight_bytes * 8 == lib.tp_attn_wqkv_packed_bytes(a)
+    assert sa.row_weight_bytes * 8 == lib.tp_attn_wo_packed_bytes(a)
+    # per shard Wq 8192x1024, Wk and Wv 8192x128, Wo 1024x8192 (bf16)
+    assert sa.col_weight_bytes == 8192 * (1024 + 2 * 128) * 2
+    assert sa.row_weight_bytes == 1024 * 8192 * 2
+    assert sa.bwd_workspace == 0                      # the attention backward takes bf16 partials
+    assert lib.tp_attn_shard_sizes(a, "bf16").bwd_workspace > 0
+
+
+def test_shard_argument_checks(lib):
+    so = lib.load()
+    fake = ctypes.c_void_p(0x1000)           # never dereferenced: each call fails its checks first
+    d = lib.mlp_desc(8, 64, 256, 4, "swiglu", "bf16")
+    for shard in (-1, 4):
+        assert so.tp_mlp_fwd_shard(ctypes.byref(d), shard, lib.TP_F32, fake, fake, fake, fake,
+                                   None, fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
+        assert so.tp_mlp_pack_shard(ctypes.byref(d), shard, fake, fake, fake, fake, fake,
+                                    None) == lib.TP_ERR_INVALID_ARG
+    # a bad partial dtype, and bf16 partials of an fp32 block
+    assert so.tp_mlp_fwd_shard(ctypes.byref(d), 0, 7, fake, fake, fake, fake, None, fake,
+                               1 << 30, None) == lib.TP_ERR_INVALID_ARG
+    with pytest.raises(lib.TpError) as e:
+        lib.tp_mlp_shard_sizes(lib.mlp_desc(8, 64, 256, 4, "swiglu", "f32"), "bf16")
+    assert e.value.status == lib.TP_ERR_UNSUPPORTED
+    with pytest.raises(lib.TpError) as e:     # the partial dtype replaces the flags
+        lib.tp_mlp_shard_sizes(lib.mlp_desc(8, 64, 256, 4, "swiglu", "bf16",
+                                            flags=lib.TP_FLAG_F32_RESIDUAL), "f32")
+    assert e.value.status == lib.TP_ERR_INVALID_ARG
+    with pytest.raises(lib.TpError) as e:     # p must divide the heads
+        lib.tp_attn_shard_sizes(lib.attn_desc(1, 4, 64, 6, 3, 8, 2), "f32")
+    assert e.value.status == lib.TP_ERR_SHAPE
+    a = lib.attn_desc(1, 4, 64, 4, 2, 8, 2)
+    assert so.tp_attn_fwd_shard(ctypes.byref(a), 2, lib.TP_F32, fake, fake, fake, None, None,
+                                fake, fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
+    assert so.tp_attn_bwd_shard(ctypes.byref(a), -1, fake, fake, fake, fake, fake, fake, fake,
+                                fake, 1 << 30, None) == lib.TP_ERR_INVALID_ARG
+    # too small a workspace: refused before anything is enqueued
+    assert so.tp_mlp_fwd_shard(ctypes.byref(d), 1, lib.TP_F32, fake, fake, fake, fake, None,
+                               fake, 16, None) == lib.TP_ERR_WORKSPACE
