@@ -367,6 +367,18 @@ tp_status tp_attn_fwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
                          void* const* y_norm_slices, void* workspace, size_t ws_bytes,
                          void* stream);
 
+/* Attention backward, sequence-parallel (self-attention, bf16, as tp_attn_bwd).  The x and dy
+ * slices ([b*s/p][h]) are all-gathered (the reduce-scatter's gradient is an all-gather), the
+ * backward runs as in tp_attn_bwd, and the dx partials are reduce-scattered into dx_slices (the
+ * all-gather's gradient).  dwqkv_p and dwo_p as in tp_attn_bwd.  Takes TP_REDUCE_SEPARATE only.
+ * workspace: tp_attn_bwd_sp_workspace(desc) bytes (0 for an unsupported descriptor).  Adds 1 to
+ * the reduction counter. */
+size_t tp_attn_bwd_sp_workspace(const tp_attn_desc* desc);
+tp_status tp_attn_bwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
+                         const void* wqkv_p, const void* wo_p, const void* const* dy_slices,
+                         void* const* dx_slices, void* dwqkv_p, void* dwo_p, void* workspace,
+                         size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* One shard per device                                                                        */
 /* ------------------------------------------------------------------------------------------ */

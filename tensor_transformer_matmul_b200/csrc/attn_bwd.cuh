@@ -195,9 +195,12 @@ inline AttnBwdLayout attn_bwd_layout(const AttnLayout& L) {
   return B;
 }
 
+// ``sp``: the sequence-parallel form -- the dx partials are reduce-scattered into
+// sp->y (the shards' token slices) instead of summed into dx.
 inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* wqkv,
                                const void* wo_p, const void* dy, void* dx, float* dwqkv_p,
-                               float* dwo_p, void* ws, cudaStream_t s) {
+                               float* dwo_p, void* ws, cudaStream_t s,
+                               const seqpar::SpOut* sp = nullptr) {
   using tc::Operand;
   using tc::TileCfg;
   using BF = __nv_bfloat16;
@@ -309,7 +312,7 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
   {
     const Operand a{dqkv, false, T, L.R_a, P, P * L.R_a, L.R_a};
     const Operand bw{wqkv, true, L.h, L.R_a, P, L.h, L.R_a * L.h};
-    if (L.reduce_mode == TP_REDUCE_FUSED) {
+    if (L.reduce_mode == TP_REDUCE_FUSED && !sp) {
       tc::EpiReduceOut::Params ep;
       ep.out = dx;
       ep.residual = nullptr;
@@ -332,6 +335,9 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
         a, bw, T, L.h, L.R_a, P, ep, s, "attn_dx_gemm");
     if (st != TP_OK) return st;
   }
+  if (sp)   // the all-gather's gradient: dx reduce-scattered into the token slices
+    return seqpar::reduce_scatter(part, L.p, T, L.h, nullptr, sp->y, TP_BF16, nullptr,
+                                  TP_BF16, L.norm_eps, s);
   return reduce::launch(part, TP_F32, L.p, T * L.h, nullptr, dx, TP_BF16, s);
 }
 

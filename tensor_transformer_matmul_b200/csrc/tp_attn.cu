@@ -171,6 +171,60 @@ extern "C" tp_status tp_attn_bwd(const tp_attn_desc* desc, const void* x, const 
   return st;
 }
 
+// Sequence-parallel backward: x and dy arrive as the p shards' token slices and are all-gathered
+// (the reduce-scatter's gradient is an all-gather); the dx partials are reduce-scattered into the
+// slices (the all-gather's gradient).  "Why tensor parallelism has to stay in scale-up",
+// "Where the 320 comes from".
+extern "C" size_t tp_attn_bwd_sp_workspace(const tp_attn_desc* desc) {
+  tp::AttnLayout L;
+  if (attn_bwd_check(desc, &L) != TP_OK || sp_layout(desc, &L) != TP_OK) return 0;
+  return 2 * sp_act_bytes(L) + tp::attn_bwd_layout(L).bytes;
+}
+
+extern "C" tp_status tp_attn_bwd_sp(const tp_attn_desc* desc, const void* const* x_slices,
+                                    const void* wqkv_p, const void* wo_p,
+                                    const void* const* dy_slices, void* const* dx_slices,
+                                    void* dwqkv_p, void* dwo_p, void* workspace, size_t ws_bytes,
+                                    void* stream) {
+  tp::clear_error();
+  tp::AttnLayout L;
+  tp_status st = attn_bwd_check(desc, &L);
+  if (st != TP_OK) return st;
+  if ((st = sp_layout(desc, &L)) != TP_OK) return st;
+  if (L.tokens == 0) {
+    tp::count_reduction();
+    return TP_OK;
+  }
+  using tp::seqpar::check_slices;
+  if ((st = check_slices(L.p, L.tokens, const_cast<void* const*>(x_slices), "x_slices")) != TP_OK ||
+      (st = check_slices(L.p, L.tokens, const_cast<void* const*>(dy_slices), "dy_slices")) != TP_OK ||
+      (st = check_slices(L.p, L.tokens, dx_slices, "dx_slices")) != TP_OK)
+    return st;
+  if (!wqkv_p || !wo_p || !dwqkv_p || !dwo_p || !workspace)
+    return tp::set_error(TP_ERR_INVALID_ARG, "null pointer");
+  for (const void* q : {wqkv_p, wo_p, static_cast<const void*>(dwqkv_p),
+                        static_cast<const void*>(dwo_p), static_cast<const void*>(workspace)})
+    if (reinterpret_cast<uintptr_t>(q) & 15)
+      return tp::set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  const size_t act = sp_act_bytes(L);
+  const tp::AttnBwdLayout B = tp::attn_bwd_layout(L);
+  if (ws_bytes < 2 * act + B.bytes) return tp::set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tp::tensor_cores_usable())
+    return tp::set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* w = static_cast<uint8_t*>(workspace);
+  void* x = w;
+  void* dy = w + act;
+  const int64_t slice_bytes = (L.tokens / L.p) * L.h * tp::elem_bytes(L.dtype);
+  if ((st = tp::seqpar::all_gather(x_slices, L.p, slice_bytes, x, s)) != TP_OK) return st;
+  if ((st = tp::seqpar::all_gather(dy_slices, L.p, slice_bytes, dy, s)) != TP_OK) return st;
+  const tp::seqpar::SpOut sp{nullptr, dx_slices, nullptr};
+  st = tp::attn_backward(L, x, wqkv_p, wo_p, dy, nullptr, static_cast<float*>(dwqkv_p),
+                         static_cast<float*>(dwo_p), w + 2 * act, s, &sp);
+  if (st == TP_OK) tp::count_reduction();
+  return st;
+}
+
 extern "C" tp_status tp_attn_unpack_grads(const tp_attn_desc* desc, const void* dwqkv_p,
                                           const void* dwo_p, void* dwq, void* dwk, void* dwv,
                                           void* dwo, void* stream) {

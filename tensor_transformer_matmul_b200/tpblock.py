@@ -41,7 +41,7 @@ EXPORTS = (
     "tp_moe_shared_w1_bytes", "tp_moe_shared_w2_bytes", "tp_moe_pack", "tp_moe_fwd_workspace",
     "tp_moe_fwd", "tp_mlp_shard_sizes", "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
     "tp_mlp_bwd_shard", "tp_attn_shard_sizes", "tp_attn_pack_shard", "tp_attn_fwd_shard",
-    "tp_attn_bwd_shard",
+    "tp_attn_bwd_shard", "tp_attn_bwd_sp_workspace", "tp_attn_bwd_sp",
 )
 
 
@@ -139,6 +139,8 @@ def load():
         "tp_attn_pack_shard": (I32, [AD, I32, P, P, P, P, P, P, P]),
         "tp_attn_fwd_shard": (I32, [AD, I32, I32, P, P, P, P, P, P, P, S, P]),
         "tp_attn_bwd_shard": (I32, [AD, I32, P, P, P, P, P, P, P, P, S, P]),
+        "tp_attn_bwd_sp_workspace": (S, [AD]),
+        "tp_attn_bwd_sp": (I32, [AD, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_read": (I32, [I32, ctypes.c_char_p, I32, ctypes.POINTER(ctypes.c_uint64),
                                   ctypes.POINTER(ctypes.c_double)]),
         "tp_profile_read_launch": (I32, [I32, ctypes.c_int64, ctypes.POINTER(ctypes.c_double)]),
@@ -450,6 +452,18 @@ def tp_attn_fwd_sp(desc, x_slices, wqkv_p, wo_p, y_slices, k_cache=None, v_cache
     _check(load().tp_attn_fwd_sp(ctypes.byref(desc), xs.ptr, _ptr(wqkv_p), _ptr(wo_p),
                                  _ptr(k_cache), _ptr(v_cache), _sp(rs), ys.ptr, _sp(ns),
                                  _ptr(workspace), _nbytes(workspace), _stream(stream)))
+
+
+def tp_attn_bwd_sp_workspace(desc):
+    return load().tp_attn_bwd_sp_workspace(ctypes.byref(desc))
+
+
+def tp_attn_bwd_sp(desc, x_slices, wqkv_p, wo_p, dy_slices, dx_slices, dwqkv_p, dwo_p,
+                   workspace=None, stream=None):
+    xs, dys, dxs = _Slices(x_slices), _Slices(dy_slices), _Slices(dx_slices)
+    _check(load().tp_attn_bwd_sp(ctypes.byref(desc), xs.ptr, _ptr(wqkv_p), _ptr(wo_p), dys.ptr,
+                                 dxs.ptr, _ptr(dwqkv_p), _ptr(dwo_p), _ptr(workspace),
+                                 _nbytes(workspace), _stream(stream)))
 
 
 # ------------------------------------------------------------------------ mixture of experts

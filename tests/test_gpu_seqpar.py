@@ -171,3 +171,40 @@ def test_attention_forward_sp(lib):
                                   n_q, n_kv, hd, causal=True).reshape(T, h) + f64(res.cpu()).reshape(T, h)
     for i, rows in enumerate(osp.token_slices(T, p)):
         assert rel_l2(f64(ys[i]), ref[rows]) <= TOL["bf16"], i
+
+
+def test_attention_backward_sp(lib):
+    # x and dy as 2 slices of 150 token rows, dx out as slices: equal to tp_attn_bwd's rows bit for
+    # bit (the same shard-order fp32 sum and rounding), and to the oracle; the weight gradients
+    # equal tp_attn_bwd's
+    b, s, h, n_q, n_kv, hd, p = 2, 150, 256, 4, 2, 128, 2
+    inp = inputs.attn_inputs(b, s, h, n_q, n_kv, hd, "bf16", seed=45, w_std=0.05)
+    a = Attn(lib, inp, p, "bf16", True, n_q=n_q, n_kv=n_kv, hd=hd)
+    dy = inputs.normal((b, s, h), 1.0, 45, 97, "bf16", "cpu").to(dev())
+    g = dev()
+    dx = torch.empty(b, s, h, dtype=torch.bfloat16, device=g)
+    dwqkv = torch.empty(a.wqkv.numel(), dtype=torch.float32, device=g)
+    dwo = torch.empty(a.wo.numel(), dtype=torch.float32, device=g)
+    ws = torch.empty(lib.tp_attn_bwd_workspace(a.desc), dtype=torch.uint8, device=g)
+    lib.tp_attn_bwd(a.desc, inp["x"].to(g), a.wqkv, a.wo, dy, dx, dwqkv, dwo, workspace=ws)
+    T = b * s
+    xs = _split(inp["x"].to(g).reshape(T, h), p)
+    dys = _split(dy.reshape(T, h), p)
+    dxs = [torch.empty(T // p, h, dtype=torch.bfloat16, device=g) for _ in range(p)]
+    dwqkv_sp = torch.empty_like(dwqkv)
+    dwo_sp = torch.empty_like(dwo)
+    ws_sp = torch.empty(lib.tp_attn_bwd_sp_workspace(a.desc), dtype=torch.uint8, device=g)
+    lib.tp_reset_reduction_count()
+    lib.tp_attn_bwd_sp(a.desc, xs, a.wqkv, a.wo, dys, dxs, dwqkv_sp, dwo_sp, workspace=ws_sp)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    assert torch.equal(torch.cat(dxs), dx.reshape(T, h))
+    assert torch.equal(dwqkv_sp, dwqkv) and torch.equal(dwo_sp, dwo)
+    ref = oattn.attention_backward(*(f64(inp[k]) for k in ("x", "wq", "wk", "wv", "wo")),
+                                   f64(dy.cpu()), n_q, n_kv, hd, causal=True)[0].reshape(T, h)
+    for i, rows in enumerate(osp.token_slices(T, p)):
+        assert rel_l2(f64(dxs[i]), ref[rows]) <= TOL["bf16"], i
+    # fused reduce mode and ragged token counts are refused
+    fused = lib.attn_desc(b, s, h, n_q, n_kv, hd, p, reduce_mode=lib.TP_REDUCE_FUSED)
+    assert lib.tp_attn_bwd_sp_workspace(fused) == 0
+    assert lib.tp_attn_bwd_sp_workspace(lib.attn_desc(1, 5, h, n_q, n_kv, hd, p)) == 0
