@@ -528,6 +528,8 @@ def config_summary(out, cpu, peaks):
                                   "frac_burst": f["frac_of_burst_peak"],
                                   "v_separate": p["TFLOP_per_s"],
                                   "dom": _dom_short(f.get("dominant")), "mhz": _mhz(p),
+                                  "fwd_vs_cublas": [(p.get("cublas_context") or {}).get(k) for k in
+                                                    ("ratio_TFLOP_per_s", "ratio_per_clock")],
                                   "cpu": cb("3"), "cpu_note": "extrapolated" if "3" in cpu else None}
     a = ex.get("attention_block")
     if a:
@@ -814,28 +816,68 @@ def extra_prefill(tp, inputs, torch, stream, peaks, steps):
     res["reduce_fused"] = {k: fused[k] for k in ("ms_fwd", "ms_bwd", "TFLOP_per_s",
                                                   "frac_of_burst_peak", "frac_of_sustained_peak",
                                                   "tokens_per_s", "dominant", "kernels")}
-    res["cublas_context"] = _cublas_context(torch, stream, steps)
+    res["cublas_context"] = _cublas_context(tp, inputs, torch, stream)
     return res
 
 
-def _cublas_context(torch, stream, steps):
-    """Context only, not this library's path: torch.matmul (cuBLAS) bf16 on the prefill MLP's
-    two forward GEMM shapes, all shards at once (T x d by d x 2 d_ff, T x d_ff by d_ff x d)."""
+def _cublas_context(tp, inputs, torch, stream, region_s=1.0):
+    """Context only, not this library's path: the prefill forward's two GEMM shapes (all shards at
+    once: T x d by d x 2 d_ff with the SwiGLU epilogue, then T x d_ff by d_ff x d with the shard
+    sum) run by this library (tp_mlp_fwd, TP_REDUCE_FUSED) and by torch.matmul (cuBLAS), in
+    alternating timed regions of about ``region_s`` seconds each, with the SM clock sampled in
+    every region.  Both are reported as TFLOP/s and as flop per clock per SM, so that a gap that
+    comes from the power-capped clock is told apart from one in the kernels."""
     try:
         c = PREFILL
         dev = torch.device("cuda", torch.cuda.current_device())
+        gpu = torch.cuda.current_device()
+        nsm = torch.cuda.get_device_properties(dev).multi_processor_count
+        st = setup_mlp(tp, inputs, torch, c, reduce_mode=tp.TP_REDUCE_FUSED)
         g = torch.Generator(device=dev)
         g.manual_seed(7)
-        out = {}
-        for name, (m, k, n) in (("up", (c["T"], c["d"], 2 * c["F"])),
-                                ("down", (c["T"], c["F"], c["d"]))):
-            a = torch.randn(m, k, generator=g, device=dev).to(torch.bfloat16)
-            b = torch.randn(k, n, generator=g, device=dev).to(torch.bfloat16)
+        a1 = torch.randn(c["T"], c["d"], generator=g, device=dev).to(torch.bfloat16)
+        b1 = torch.randn(c["d"], 2 * c["F"], generator=g, device=dev).to(torch.bfloat16)
+        a2 = torch.randn(c["T"], c["F"], generator=g, device=dev).to(torch.bfloat16)
+        b2 = torch.randn(c["F"], c["d"], generator=g, device=dev).to(torch.bfloat16)
+        flops = 2.0 * c["T"] * c["d"] * 2 * c["F"] + 2.0 * c["T"] * c["F"] * c["d"]
+
+        def ours():
+            tp.tp_mlp_fwd(st["desc"], st["x"], st["w1p"], st["w2p"], st["y"], workspace=st["ws"])
+
+        def cublas():
+            torch.matmul(a1, b1)
+            torch.matmul(a2, b2)
+
+        for fn in (ours, cublas):
             for _ in range(3):
-                torch.matmul(a, b)
-            ms = _cuda_time(lambda: torch.matmul(a, b), steps, stream) / steps
-            out[name] = {"ms": round(ms, 3), "TFLOP_per_s": round(2.0 * m * k * n / (ms / 1e3) / 1e12, 1)}
-            del a, b
+                fn()
+        torch.cuda.synchronize()
+        ms1 = {"ours": _cuda_time(ours, 5, stream) / 5, "cublas": _cuda_time(cublas, 5, stream) / 5}
+        reps = {k: max(5, int(region_s * 1e3 / v)) for k, v in ms1.items()}
+        rows = {"ours": [], "cublas": []}
+        for _ in range(2):
+            for name, fn in (("ours", ours), ("cublas", cublas)):
+                time.sleep(0.5)
+                clk = ClockSampler(gpu)
+                clk.start()
+                ms = _cuda_time(fn, reps[name], stream) / reps[name]
+                ck = clk.stop() or {}
+                rows[name].append((ms, ck.get("sm_mhz")))
+        out = {"shapes": "T=4096: [4096x8192]x[8192x57344] + [4096x28672]x[28672x8192]",
+               "region_s": region_s}
+        for name, r in rows.items():
+            ms = min(x[0] for x in r)
+            mhz = [x[1] for x in r if x[1]]
+            mhz_med = statistics.median(mhz) if mhz else None
+            tf = flops / (ms / 1e3) / 1e12
+            out[name] = {"ms": round(ms, 3), "TFLOP_per_s": round(tf, 1), "sm_mhz": mhz_med,
+                         "flop_per_clk_per_sm": round(tf * 1e12 / (mhz_med * 1e6) / nsm, 1)
+                         if mhz_med else None}
+        if out["ours"]["flop_per_clk_per_sm"] and out["cublas"]["flop_per_clk_per_sm"]:
+            out["ratio_TFLOP_per_s"] = round(out["ours"]["TFLOP_per_s"] / out["cublas"]["TFLOP_per_s"], 3)
+            out["ratio_per_clock"] = round(out["ours"]["flop_per_clk_per_sm"]
+                                           / out["cublas"]["flop_per_clk_per_sm"], 3)
+        del st, a1, b1, a2, b2
         torch.cuda.empty_cache()
         return out
     except Exception as e:  # context only: never fail the bench over it

@@ -9,6 +9,7 @@ to capture with the profiler's skip count).
     python -m tensor_transformer_matmul_b200.profile_cases attn_fwd --tokens 2048 --fused
     python -m tensor_transformer_matmul_b200.profile_cases attn_bwd --tokens 2048
     python -m tensor_transformer_matmul_b200.profile_cases moe_fwd --tokens 1024
+    python -m tensor_transformer_matmul_b200.profile_cases decode_layer --tokens 1
 """
 import argparse
 
@@ -98,7 +99,23 @@ def moe_fwd(tokens, reps, fused, d=7168, n_experts=32, top_k=8, d_ff=2048, p=8):
     return y
 
 
-CASES = {"mlp_fwd": mlp_fwd, "attn_fwd": attn_fwd, "attn_bwd": attn_bwd, "moe_fwd": moe_fwd}
+def decode_layer(tokens, reps, fused, h=8192, d_ff=28672, n_q=64, n_kv=8, hd=128, p=8,
+                 kv_len=4096):
+    """One layer of the decode stack (b = ``tokens`` single-token sequences, KV length 4096):
+    the attention block (QKV GEMM, split-KV decode attention with the KV append, O projection,
+    reduce + RMSNorm) then the SwiGLU MLP block, fp32 residual stream."""
+    from tensor_transformer_matmul_b200.decode_stack import DecodeStack
+    mode = tp.TP_REDUCE_FUSED if fused else tp.TP_REDUCE_SEPARATE
+    st = DecodeStack(1, h, d_ff, n_q, n_kv, hd, p, kv_len, b=tokens, reduce_mode=mode)
+    x = torch.randn(tokens, 1, h, device="cuda")
+    for _ in range(reps):
+        st.step(x)
+    torch.cuda.synchronize()
+    return x
+
+
+CASES = {"mlp_fwd": mlp_fwd, "attn_fwd": attn_fwd, "attn_bwd": attn_bwd, "moe_fwd": moe_fwd,
+         "decode_layer": decode_layer}
 
 
 def main(argv=None):

@@ -262,3 +262,51 @@ def test_y_norm_output(lib, reduce_mode, T):
     ref = _oracle_fwd(inp, "swiglu") + f64(res)
     assert rel_l2(f64(y), ref) <= TOL["bf16"]
     assert rel_l2(f64(yn), odec.rmsnorm(ref)) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("reduce_mode", [0, 1])
+@pytest.mark.parametrize("act", ["swiglu", "gelu", "relu", "identity"])
+@pytest.mark.parametrize("T", [1, 2, 3, 4])
+def test_gemv_decode_path(lib, act, T, reduce_mode):
+    # 1..4 tokens with d and the padded shard width multiples of 256 run the decode GEMV path
+    # (streaming matrix-vector products, the shard sum in the reduce kernel in both modes):
+    # d = 512, d_ff = 1536 over p = 3 (512 features per shard), residual and RMSNorm output
+    from oracle import decode as odec
+    d, F, p = 512, 1536, 3
+    inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=30 + T, w_std=0.05, backward=True)
+    m = Mlp(lib, inp, p, act, "bf16", reduce_mode)
+    res = inputs.normal((T, d), 1.0, 30, 99, "bf16", "cpu").to(dev())
+    y = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+    yn = torch.empty_like(y)
+    lib.tp_reset_reduction_count()
+    lib.tp_mlp_fwd(m.desc, inp["x"].to(dev()), m.w1p, m.w2p, y, residual=res, saved=m.saved,
+                   workspace=m.ws_f, y_norm=yn)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    ref = _oracle_fwd(inp, act) + f64(res)
+    assert rel_l2(f64(y), ref) <= TOL["bf16"] and rel_l2_rows(f64(y), ref) <= TOL["bf16"]
+    assert rel_l2(f64(yn), odec.rmsnorm(ref)) <= TOL["bf16"]
+    # the saved pre-activations feed the backward pass
+    dx, dw1, dwu, dw2, _, _ = m.backward(inp["dy"], inp["x"])
+    torch.cuda.synchronize()
+    wu = None if inp["w_up"] is None else f64(inp["w_up"])
+    rb = omlp.mlp_backward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), f64(inp["dy"]), act, wu)
+    assert rel_l2(f64(dx), rb["dx"]) <= TOL["bf16"]
+    assert rel_l2(f64(dw2), rb["dw2"]) <= TOL["bf16"]
+    # deterministic: a second call gives the same bytes
+    y2 = torch.empty_like(y)
+    lib.tp_mlp_fwd(m.desc, inp["x"].to(dev()), m.w1p, m.w2p, y2, residual=res, workspace=m.ws_f)
+    torch.cuda.synchronize()
+    assert torch.equal(y, y2)
+
+
+def test_gemv_decode_full_size_one_token(lib):
+    # the decode stack's MLP shape at b = 1: d=8192, d_ff=28672, p=8, one token
+    T, d, F, p = 1, 8192, 28672, 8
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    y = m.forward(inp["x"], save=False)
+    torch.cuda.synchronize()
+    ref = omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu",
+                           f64(inp["w_up"]))
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
