@@ -148,58 +148,64 @@ inline tp_status launch(const void* part, int in_dtype, int p, int64_t n, const 
   return launch_t<__nv_bfloat16, __nv_bfloat16>(part, p, n, res, out, s);
 }
 
-// Reduce and normalize one row per block (512 threads): out = res + sum_s part[s] (in order,
-// fp32, one rounding), then norm = out / sqrt(mean(out^2) + eps) from the stored out values.
-// VEC (p <= 8): 8 consecutive elements per thread, all p loads issued before the in-order adds.
+// One row of "reduce, then normalise": out = res + sum_s part[s] (fp32, shards in order, one
+// rounding), then norm = out / sqrt(mean(out^2) + eps) of the stored (rounded) out values.  The
+// block's threads split the row; ``prow`` is the row in partial 0 (partial s at + s*n).
+// VEC (d % 8 == 0, 16-byte aligned rows): 8 consecutive elements per thread and access; the
+// partials are loaded four at a time, every load of a group issued before its adds, which run in
+// the order 0..p-1.  Used by the plain and the sequence-parallel reduce-and-norm kernels,
+// so that both give the same bits for the same row.
+constexpr int kRowThreads = 256;
 template <typename Tin, typename Tout, typename Tn, bool VEC>
-__global__ void __launch_bounds__(512) reduce_norm_rows_kernel(const Tin* __restrict__ part, int p,
-                                                                int64_t rows, int64_t d,
-                                                                const Tout* res, Tout* out,
-                                                                Tn* norm, float eps) {
-  pdl_wait();   // programmatic dependent launch: global memory only from here on
-  pdl_trigger();
-  __shared__ float red[16];
-  const int64_t n = rows * d;
-  const int64_t base = static_cast<int64_t>(blockIdx.x) * d;
+__device__ __forceinline__ void reduce_norm_row(const Tin* __restrict__ prow, int p, int64_t n,
+                                                int64_t d, const Tout* rrow, Tout* orow,
+                                                Tn* nrow, float eps, float* red) {
   float ss = 0.f;
   if (VEC) {
     for (int64_t j = 8 * static_cast<int64_t>(threadIdx.x); j < d; j += 8 * blockDim.x) {
-      float v[8][8];
-#pragma unroll
-      for (int q = 0; q < 8; ++q)
-        if (q < p) Vec8<Tin>::load(part + static_cast<int64_t>(q) * n + base + j, v[q]);
       float acc[8];
+      for (int g = 0; g < p; g += 4) {
+        float v[4][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = v[0][e];
+        for (int q = 0; q < 4; ++q)
+          if (g + q < p) Vec8<Tin>::load(prow + static_cast<int64_t>(g + q) * n + j, v[q]);
 #pragma unroll
-      for (int t = 1; t < 8; ++t)
-        if (t < p) {
+        for (int q = 0; q < 4; ++q) {
+          if (g + q >= p) break;
+          if (g + q == 0) {
 #pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] += v[t][e];
+            for (int e = 0; e < 8; ++e) acc[e] = v[0][e];
+          } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) acc[e] += v[q][e];
+          }
         }
-      if (res) {
+      }
+      if (rrow) {
         float r[8];
-        Vec8<Tout>::load(res + base + j, r);
+        Vec8<Tout>::load(rrow + j, r);
 #pragma unroll
         for (int e = 0; e < 8; ++e) acc[e] = r[e] + acc[e];
       }
-      Vec8<Tout>::store(out + base + j, acc);
-      float st[8];
-      Vec8<Tout>::load(out + base + j, st);   // the stored (rounded) values
+      Vec8<Tout>::store(orow + j, acc);
 #pragma unroll
-      for (int e = 0; e < 8; ++e) ss = fmaf(st[e], st[e], ss);
+      for (int e = 0; e < 8; ++e) {   // the stored, rounded value
+        const float y = to_f(from_f<Tout>(acc[e]));
+        ss = fmaf(y, y, ss);
+      }
     }
   } else {
     for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
-      float acc = to_f(part[base + j]);
-      for (int q = 1; q < p; ++q) acc += to_f(part[static_cast<int64_t>(q) * n + base + j]);
-      if (res) acc = to_f(res[base + j]) + acc;
+      float acc = to_f(prow[j]);
+      for (int q = 1; q < p; ++q) acc += to_f(prow[static_cast<int64_t>(q) * n + j]);
+      if (rrow) acc = to_f(rrow[j]) + acc;
       const Tout y = from_f<Tout>(acc);
-      out[base + j] = y;
+      orow[j] = y;
       const float yv = to_f(y);
       ss = fmaf(yv, yv, ss);
     }
   }
+  if (!nrow) return;   // block-uniform
 #pragma unroll
   for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
   if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
@@ -212,8 +218,32 @@ __global__ void __launch_bounds__(512) reduce_norm_rows_kernel(const Tin* __rest
   }
   __syncthreads();
   const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
-  for (int64_t j = threadIdx.x; j < d; j += blockDim.x)
-    norm[base + j] = from_f<Tn>(to_f(out[base + j]) * scale);
+  if (VEC) {
+    // the same elements this thread stored: its own writes, read back in order
+    for (int64_t j = 8 * static_cast<int64_t>(threadIdx.x); j < d; j += 8 * blockDim.x) {
+      float y[8];
+      Vec8<Tout>::load(orow + j, y);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) y[e] *= scale;
+      Vec8<Tn>::store(nrow + j, y);
+    }
+  } else {
+    for (int64_t j = threadIdx.x; j < d; j += blockDim.x)
+      nrow[j] = from_f<Tn>(to_f(orow[j]) * scale);
+  }
+}
+
+// One row per block: reduce_norm_row over rows of [rows][d].
+template <typename Tin, typename Tout, typename Tn, bool VEC>
+__global__ void __launch_bounds__(kRowThreads, 3) reduce_norm_rows_kernel(
+    const Tin* __restrict__ part, int p, int64_t rows, int64_t d, const Tout* res, Tout* out,
+    Tn* norm, float eps) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
+  __shared__ float red[kRowThreads / 32];
+  const int64_t base = static_cast<int64_t>(blockIdx.x) * d;
+  reduce_norm_row<Tin, Tout, Tn, VEC>(part + base, p, rows * d, d, res ? res + base : nullptr,
+                                      out + base, norm + base, eps, red);
 }
 
 template <typename Tin, typename Tout, typename Tn>
@@ -224,12 +254,12 @@ inline void reduce_norm_launch(const void* part, int p, int64_t rows, int64_t d,
                    (!res || (reinterpret_cast<uintptr_t>(res) & 15) == 0);
   if (vec)
     (void)launch_pdl(reduce_norm_rows_kernel<Tin, Tout, Tn, true>, dim3(static_cast<unsigned>(rows)),
-                     dim3(512), 0, s, static_cast<const Tin*>(part), p, rows, d,
+                     dim3(kRowThreads), 0, s, static_cast<const Tin*>(part), p, rows, d,
                      static_cast<const Tout*>(res), static_cast<Tout*>(out),
                      static_cast<Tn*>(norm), eps);
   else
     (void)launch_pdl(reduce_norm_rows_kernel<Tin, Tout, Tn, false>,
-                     dim3(static_cast<unsigned>(rows)), dim3(512), 0, s,
+                     dim3(static_cast<unsigned>(rows)), dim3(kRowThreads), 0, s,
                      static_cast<const Tin*>(part), p, rows, d, static_cast<const Tout*>(res),
                      static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
 }

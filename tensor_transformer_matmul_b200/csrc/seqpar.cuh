@@ -30,13 +30,11 @@ struct Slices {
   void* p[kMaxSlices];
 };
 
-// One block (512 threads) per token row.  VEC: d % 8 == 0 and 16-byte aligned rows, 8 elements
-// per access, and (p <= 8) all p loads issued before the in-order adds -- the same arithmetic,
-// work split and reduction tree as the plain reduce-and-norm kernel, so a slice equals the plain
-// call's rows bit for bit when that kernel runs (one block per row).
-constexpr int kRsThreads = 512;
+// One block per token row, written into its shard's slice: reduce::reduce_norm_row (the plain
+// reduce-and-norm kernel's row routine), so a slice equals the plain call's rows bit for bit.
+constexpr int kRsThreads = reduce::kRowThreads;
 template <typename Tout, typename Tn, bool VEC>
-__global__ void __launch_bounds__(kRsThreads) reduce_scatter_rows_kernel(
+__global__ void __launch_bounds__(kRsThreads, 3) reduce_scatter_rows_kernel(
     const float* __restrict__ part, int p, int64_t rows, int64_t d, int64_t R, Slices res,
     int has_res, Slices out, Slices norm, int has_norm, float eps) {
   pdl_wait();   // programmatic dependent launch: global memory only from here on
@@ -45,76 +43,11 @@ __global__ void __launch_bounds__(kRsThreads) reduce_scatter_rows_kernel(
   const int64_t r = blockIdx.x;
   const int sl = static_cast<int>(r / R);
   const int64_t lr = r - static_cast<int64_t>(sl) * R;
-  const int64_t n = rows * d;
-  const float* prow = part + r * d;
   Tout* orow = static_cast<Tout*>(out.p[sl]) + lr * d;
   const Tout* rrow = has_res ? static_cast<const Tout*>(res.p[sl]) + lr * d : nullptr;
-  float ss = 0.f;
-  if (VEC) {
-    for (int64_t j = 8 * static_cast<int64_t>(threadIdx.x); j < d; j += 8 * blockDim.x) {
-      float acc[8];
-      if (p <= 8) {
-        float v[8][8];
-#pragma unroll
-        for (int q = 0; q < 8; ++q)
-          if (q < p) reduce::Vec8<float>::load(prow + static_cast<int64_t>(q) * n + j, v[q]);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = v[0][e];
-#pragma unroll
-        for (int q = 1; q < 8; ++q)
-          if (q < p) {
-#pragma unroll
-            for (int e = 0; e < 8; ++e) acc[e] += v[q][e];
-          }
-      } else {
-        reduce::Vec8<float>::load(prow + j, acc);
-        for (int q = 1; q < p; ++q) {
-          float v[8];
-          reduce::Vec8<float>::load(prow + static_cast<int64_t>(q) * n + j, v);
-#pragma unroll
-          for (int e = 0; e < 8; ++e) acc[e] += v[e];
-        }
-      }
-      if (rrow) {
-        float v[8];
-        reduce::Vec8<Tout>::load(rrow + j, v);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) acc[e] = v[e] + acc[e];
-      }
-      reduce::Vec8<Tout>::store(orow + j, acc);
-      if (has_norm) {
-        float st[8];
-        reduce::Vec8<Tout>::load(orow + j, st);   // the stored (rounded) values
-#pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(st[e], st[e], ss);
-      }
-    }
-  } else {
-    for (int64_t j = threadIdx.x; j < d; j += blockDim.x) {
-      float acc = prow[j];
-      for (int q = 1; q < p; ++q) acc += prow[static_cast<int64_t>(q) * n + j];
-      if (rrow) acc = to_f(rrow[j]) + acc;
-      const Tout y = from_f<Tout>(acc);
-      orow[j] = y;
-      const float yv = to_f(y);
-      ss = fmaf(yv, yv, ss);
-    }
-  }
-  if (!has_norm) return;   // block-uniform
-#pragma unroll
-  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
-  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
-  __syncthreads();
-  if (threadIdx.x < 32) {
-    float v = threadIdx.x < (blockDim.x >> 5) ? red[threadIdx.x] : 0.f;
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
-    if (threadIdx.x == 0) red[0] = v;
-  }
-  __syncthreads();
-  const float scale = rsqrtf(red[0] / static_cast<float>(d) + eps);
-  Tn* nrow = static_cast<Tn*>(norm.p[sl]) + lr * d;
-  for (int64_t j = threadIdx.x; j < d; j += blockDim.x) nrow[j] = from_f<Tn>(to_f(orow[j]) * scale);
+  Tn* nrow = has_norm ? static_cast<Tn*>(norm.p[sl]) + lr * d : nullptr;
+  reduce::reduce_norm_row<float, Tout, Tn, VEC>(part + r * d, p, rows * d, d, rrow, orow, nrow,
+                                                eps, red);
 }
 
 // full[i*R + r] = slice_i[r]: block (x, i) copies 16-byte words of slice i (W: the slice's size
