@@ -140,9 +140,10 @@ def test_attention_shards_sum_to_the_block(lib, b, s, kv_len, h, n_q, n_kv, hd, 
         lib.tp_attn_fwd_shard(desc, i, inp["x"].to(g), wqkv, wo, part, k_cache=kc, v_cache=vc,
                               workspace=ws)
         parts.append(part)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 0     # the shard calls reduce nothing
     y = _sum(lib, parts)
     torch.cuda.synchronize()
-    assert lib.tp_reduction_count() == 0
     args = [f64(inp[k]) for k in ("wq", "wk", "wv", "wo")]
     if kv_len:
         ref, kn, vn = oattn.attention_decode(f64(inp["x"])[:, 0], *args,
