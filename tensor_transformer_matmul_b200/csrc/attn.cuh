@@ -95,7 +95,8 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (d->dtype != TP_F32 && d->dtype != TP_BF16) return set_error(TP_ERR_INVALID_ARG, "dtype");
   if (d->reduce_mode != TP_REDUCE_SEPARATE && d->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
-  if (d->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  if (d->flags & ~(TP_FLAG_F32_RESIDUAL | TP_FLAG_DECODE_TILES))
+    return set_error(TP_ERR_INVALID_ARG, "unknown flags");
   if (d->kv_len < 0) return set_error(TP_ERR_SHAPE, "kv_len must be >= 0");
   if (d->kv_len > 0 && d->s != 1) return set_error(TP_ERR_SHAPE, "decode (kv_len > 0) needs s == 1");
   L->b = d->b; L->s = d->s; L->h = d->h; L->tokens = d->b * d->s;
@@ -141,7 +142,7 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (L->hd + 4) * 4;
   L->reduce_mode = d->reduce_mode;
   L->tc = d->dtype == TP_BF16 && d->h % 8 == 0;
-  L->gemv = L->tc && gemv::usable(L->tokens, L->h) &&
+  L->gemv = L->tc && !(d->flags & TP_FLAG_DECODE_TILES) && gemv::usable(L->tokens, L->h) &&
             (static_cast<int64_t>(L->qh) * L->hd) % gemv::kStep == 0;
   L->qkv_off = 0;
   L->o_off = align256(qkvb);
@@ -635,8 +636,10 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
     sm100::fence_barrier_init();
   }
   __syncthreads();
-  pdl_wait();   // global memory only from here on (programmatic dependent launch)
-  pdl_trigger();
+  // The cached rows 0 .. kv_len-1 are written only by earlier decode steps' calls of this kernel,
+  // never by the kernels just before it on the stream (the projection writes q, k, v of the new
+  // token; this kernel itself writes slot kv_len, which the tensor maps leave out), so their
+  // streaming starts before the programmatic-launch wait and overlaps the previous kernel's tail.
   if (threadIdx.x == 0) {
     const int32_t z = static_cast<int32_t>(bi * n_kv + g);
     for (int i = 0; i < nsub; ++i) {
@@ -648,6 +651,8 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
       }
     }
   }
+  pdl_wait();   // everything else in global memory only from here on
+  pdl_trigger();
 
   // the group's query rows as MMA A fragments (rows >= GROUP and rows 8..15 are zero)
   uint32_t qa[KS][2];

@@ -26,6 +26,7 @@ constexpr int kMaxT = 4;              // tokens handled here
 constexpr int kThreads = 256;
 constexpr int kBlocksPerSm = 4;       // resident together (launch bounds cap the registers)
 constexpr int kStep = 256;            // elements of one warp step (16 bytes per lane)
+constexpr size_t kMaxStagedX = 48 * 1024;   // x staged per block (fp32): K <= 12288
 // weight steps whose loads a lane keeps in flight: 128 (T <= 2) or 64 bytes per lane, i.e.
 // 128 or 64 KB per SM
 template <int T>
@@ -157,6 +158,101 @@ __global__ void __launch_bounds__(kThreads, kBlocksPerSm) gemv_kernel(Args a) {
   flush(cur_row);
 }
 
+// One token and one batch (the column-parallel projections): x is staged once per block in shared
+// memory as fp32, so a step costs one 16-byte weight load, its bf16 -> fp32 unpacking, two shared
+// loads and four packed fp32 FMAs (fma.rn.f32x2).
+__device__ __forceinline__ uint64_t pair_of(float a, float b) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(a), "f"(b));
+  return r;
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ float pair_sum(uint64_t v) {
+  float a, b;
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(a), "=f"(b) : "l"(v));
+  return a + b;
+}
+
+static __global__ void __launch_bounds__(kThreads, kBlocksPerSm) gemv_x1_kernel(Args a) {
+  constexpr int kUnroll = 8;
+  extern __shared__ __align__(16) float xs[];          // [K] fp32
+  pdl_wait();
+  pdl_trigger();
+  for (int64_t k = threadIdx.x * 8; k < a.K; k += kThreads * 8) {
+    float f[8];
+    bf16x8_to_f32(__ldg(reinterpret_cast<const uint4*>(a.x + k)), f);
+    *reinterpret_cast<float4*>(xs + k) = make_float4(f[0], f[1], f[2], f[3]);
+    *reinterpret_cast<float4*>(xs + k + 4) = make_float4(f[4], f[5], f[6], f[7]);
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int64_t warp = (static_cast<int64_t>(blockIdx.x) * kThreads + threadIdx.x) >> 5;
+  const int64_t spr = a.K / kStep;
+  const int64_t s_begin = warp * a.steps_per_warp;
+  const int64_t total = a.rows * spr;
+  const int64_t s_end = min(total, s_begin + a.steps_per_warp);
+  if (s_begin >= s_end) return;
+  uint64_t acc = 0;                                     // a packed pair of fp32 partial sums
+  int64_t cur_row = s_begin / spr;
+  auto flush = [&](int64_t row) {
+    float v = pair_sum(acc);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+    acc = 0;
+    if (lane == 0) {
+      const int64_t first = (row * spr) / a.steps_per_warp;
+      a.pieces[row * a.max_pieces + (warp - first)] = v;
+    }
+  };
+  int64_t row = cur_row;
+  int kst = static_cast<int>(s_begin - cur_row * spr);
+  const int spr32 = static_cast<int>(spr);
+  const float* xl = xs + lane * 8;
+  for (int64_t left = s_end - s_begin; left > 0; left -= kUnroll) {
+    uint4 wv[kUnroll];
+    const int64_t row0 = row;
+    const int kst0 = kst;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (u < left) {
+        wv[u] = __ldcs(reinterpret_cast<const uint4*>(a.w + row * a.K + kst * kStep + lane * 8));
+        if (++kst == spr32) {
+          kst = 0;
+          ++row;
+        }
+      }
+    }
+    int64_t r = row0;
+    int kc = kst0;
+#pragma unroll
+    for (int u = 0; u < kUnroll; ++u) {
+      if (u >= left) break;                                // warp-uniform
+      if (r != cur_row) {
+        flush(cur_row);
+        cur_row = r;
+      }
+      const float4 x0 = *reinterpret_cast<const float4*>(xl + kc * kStep);
+      const float4 x1 = *reinterpret_cast<const float4*>(xl + kc * kStep + 4);
+      const uint32_t w4[4] = {wv[u].x, wv[u].y, wv[u].z, wv[u].w};
+      const float xv[8] = {x0.x, x0.y, x0.z, x0.w, x1.x, x1.y, x1.z, x1.w};
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const uint64_t wp = pair_of(__uint_as_float(w4[i] << 16), __uint_as_float(w4[i] & 0xFFFF0000u));
+        acc = ffma2(wp, pair_of(xv[2 * i], xv[2 * i + 1]), acc);
+      }
+      if (++kc == spr32) {
+        kc = 0;
+        ++r;
+      }
+    }
+  }
+  flush(cur_row);
+}
+
 // Sum of a row's pieces in warp order.
 __device__ __forceinline__ float row_sum(const float* pieces, int64_t row, int64_t spr,
                                          int64_t steps_per_warp, int max_pieces, int T, int t) {
@@ -241,6 +337,19 @@ inline tp_status run(const Args& a0, const Plan& P, cudaStream_t s, const char* 
   a.steps_per_warp = P.steps_per_warp;
   a.max_pieces = P.max_pieces;
   ProfScope prof(s, label);
+  const size_t xs_bytes = static_cast<size_t>(a.K) * sizeof(float);
+  if (a.T == 1 && a.batch == 1 && xs_bytes <= kMaxStagedX) {
+    static int attr_set[64] = {0};
+    int dev = 0;
+    TP_CUDA_TRY(cudaGetDevice(&dev));
+    if (dev < 64 && !attr_set[dev]) {
+      TP_CUDA_TRY(cudaFuncSetAttribute(gemv_x1_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(kMaxStagedX)));
+      attr_set[dev] = 1;
+    }
+    TP_LAUNCH_PDL(gemv_x1_kernel, dim3(P.blocks), dim3(kThreads), xs_bytes, s, a);
+    return TP_OK;
+  }
   switch (a.T) {
     case 1: TP_LAUNCH_PDL(gemv_kernel<1>, dim3(P.blocks), dim3(kThreads), 0, s, a); break;
     case 2: TP_LAUNCH_PDL(gemv_kernel<2>, dim3(P.blocks), dim3(kThreads), 0, s, a); break;

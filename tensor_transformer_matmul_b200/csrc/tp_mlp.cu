@@ -97,7 +97,8 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
     return set_error(TP_ERR_INVALID_ARG, "dtype must be TP_F32 or TP_BF16");
   if (desc->reduce_mode != TP_REDUCE_SEPARATE && desc->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
-  if (desc->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  if (desc->flags & ~(TP_FLAG_F32_RESIDUAL | TP_FLAG_DECODE_TILES))
+    return set_error(TP_ERR_INVALID_ARG, "unknown flags");
   L->y_dtype = (desc->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : desc->dtype;
   L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
   L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
@@ -113,7 +114,8 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   const size_t zb = static_cast<size_t>(L->T * P * L->R) * L->eb;
   const size_t hb = static_cast<size_t>(L->T * P * L->Fsp) * L->eb;
   const size_t partb = static_cast<size_t>(P * L->T * L->d) * 4;
-  L->gemv = L->tc && gemv::usable(L->T, L->d) && L->Fsp % gemv::kStep == 0;
+  L->gemv = L->tc && !(desc->flags & TP_FLAG_DECODE_TILES) && gemv::usable(L->T, L->d) &&
+            L->Fsp % gemv::kStep == 0;
   L->saved_z_off = 0;
   L->saved_h_off = align256(zb);
   L->saved_bytes = L->saved_h_off + align256(hb);
@@ -661,12 +663,13 @@ tp_status shard_desc_of(const tp_mlp_desc* desc, int32_t shard, int32_t partial_
     return set_error(TP_ERR_INVALID_ARG, "partial_dtype must be TP_F32 or TP_BF16");
   if (L.dtype == TP_F32 && partial_dtype != TP_F32)
     return set_error(TP_ERR_UNSUPPORTED, "fp32 blocks give fp32 partials");
-  if (desc->flags != 0)
-    return set_error(TP_ERR_INVALID_ARG, "shard calls take no flags (partial_dtype sets the type)");
+  if (desc->flags & ~TP_FLAG_DECODE_TILES)
+    return set_error(TP_ERR_INVALID_ARG, "shard calls take no residual flag (partial_dtype sets the type)");
   *sd = *desc;
   sd->d_ff = L.Fs;
   sd->p = 1;
-  sd->flags = (L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0;
+  sd->flags = ((L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0) |
+              (desc->flags & TP_FLAG_DECODE_TILES);
   sd->reduce_mode = L.tc ? TP_REDUCE_FUSED : TP_REDUCE_SEPARATE;
   return layout_of(sd, LS);
 }

@@ -310,3 +310,21 @@ def test_gemv_decode_full_size_one_token(lib):
     ref = omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu",
                            f64(inp["w_up"]))
     assert rel_l2(f64(y), ref) <= TOL["bf16"]
+
+
+@pytest.mark.parametrize("T", [1, 4])
+def test_decode_tiles_flag(lib, T):
+    # TP_FLAG_DECODE_TILES runs 1-4 tokens on the tensor-core tiles instead of the GEMV path:
+    # both match the oracle
+    d, F, p = 512, 1536, 3
+    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=40 + T, w_std=0.05)
+    m = Mlp(lib, inp, p, "swiglu", "bf16")
+    ref = _oracle_fwd(inp, "swiglu")
+    for flags in (0, lib.TP_FLAG_DECODE_TILES):
+        desc = lib.mlp_desc(T, d, F, p, "swiglu", "bf16", flags=flags)
+        ws = torch.empty(lib.tp_mlp_fwd_workspace(desc), dtype=torch.uint8, device=dev())
+        y = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+        lib.tp_mlp_fwd(desc, inp["x"].to(dev()), m.w1p, m.w2p, y, workspace=ws)
+        torch.cuda.synchronize()
+        assert rel_l2(f64(y), ref) <= TOL["bf16"] and rel_l2_rows(f64(y), ref) <= TOL["bf16"]
+
