@@ -74,10 +74,6 @@ typedef enum { TP_REDUCE_SEPARATE = 0, TP_REDUCE_FUSED = 1 } tp_reduce_mode;
  *   weights stay in dtype.  The residual plus the sum of the partials is then rounded to fp32
  *   instead of bf16, so a deep stack of bf16 layers never rounds its skip path to bf16. */
 #define TP_FLAG_F32_RESIDUAL 1
-/*   TP_FLAG_DECODE_TILES: with 1-4 tokens, run the projections on the tensor-core tiles instead
- *   of the streaming matrix-vector kernels the library picks for so few tokens (same results
- *   within rounding; a tuning choice). */
-#define TP_FLAG_DECODE_TILES 2
 
 /* ------------------------------------------------------------------------------------------ */
 /* MLP block                                                                                   */

@@ -7,7 +7,6 @@
 #include "flash_attn.cuh"
 #include "gemm_launch.cuh"
 #include "gemm_pair.cuh"
-#include "gemv.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
 #include "seqpar.cuh"
@@ -28,7 +27,6 @@ struct AttnLayout {
   size_t cnt_off;       // decode: arrival counters [b][n_kv]
   int reduce_mode;
   bool tc;              // bf16 with 16-byte rows: tensor-core projections
-  bool gemv;            // 1..4 tokens, h and qh*hd multiples of 256: the decode GEMV projections
 };
 
 namespace attn_tc {
@@ -67,10 +65,6 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
       return tc::plan_stream_k<typename decltype(t)::type>(L.h, L.tokens, K, L.p, fused, num_sms()).bytes();
     });
   }
-  if (L.gemv)   // the GEMV pieces of the QKV and output projections (one after the other)
-    return std::max({a, b,
-                     gemv::plan(rows, L.h, 1, static_cast<int>(L.tokens), num_sms()).pieces_bytes,
-                     gemv::plan(L.h, K, L.p, static_cast<int>(L.tokens), num_sms()).pieces_bytes});
   return std::max(a, b);
 }
 
@@ -95,8 +89,7 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   if (d->dtype != TP_F32 && d->dtype != TP_BF16) return set_error(TP_ERR_INVALID_ARG, "dtype");
   if (d->reduce_mode != TP_REDUCE_SEPARATE && d->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
-  if (d->flags & ~(TP_FLAG_F32_RESIDUAL | TP_FLAG_DECODE_TILES))
-    return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  if (d->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
   if (d->kv_len < 0) return set_error(TP_ERR_SHAPE, "kv_len must be >= 0");
   if (d->kv_len > 0 && d->s != 1) return set_error(TP_ERR_SHAPE, "decode (kv_len > 0) needs s == 1");
   L->b = d->b; L->s = d->s; L->h = d->h; L->tokens = d->b * d->s;
@@ -142,13 +135,10 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
   const size_t mlb = static_cast<size_t>(L->b * L->n_q * L->kv_splits) * (L->hd + 4) * 4;
   L->reduce_mode = d->reduce_mode;
   L->tc = d->dtype == TP_BF16 && d->h % 8 == 0;
-  L->gemv = L->tc && !(d->flags & TP_FLAG_DECODE_TILES) && gemv::usable(L->tokens, L->h) &&
-            (static_cast<int64_t>(L->qh) * L->hd) % gemv::kStep == 0;
   L->qkv_off = 0;
   L->o_off = align256(qkvb);
   L->part_off = L->o_off + align256(ob);
-  // the GEMV path always materialises the partials (its shard sum is the reduce kernel's)
-  const size_t pb = (L->tc && L->reduce_mode == TP_REDUCE_FUSED && !L->gemv) ? 0 : partb;
+  const size_t pb = (L->tc && L->reduce_mode == TP_REDUCE_FUSED) ? 0 : partb;
   L->ml_off = L->part_off + align256(pb);
   L->cnt_off = L->ml_off + align256(mlb);
   const size_t cntb = L->kv_len > 0 ? static_cast<size_t>(L->b * L->n_kv) * sizeof(int32_t) : 0;
@@ -939,20 +929,6 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
   ep.tokens = static_cast<int32_t>(L.tokens);
   ep.rows = static_cast<int32_t>(rows);
   ep.act = TP_ACT_IDENTITY;
-  if (L.gemv) {
-    // a few tokens: a streaming matrix-vector product over all shards' packed rows
-    const gemv::Plan P = gemv::plan(rows, L.h, 1, static_cast<int>(L.tokens), num_sms());
-    if (P.pieces_bytes > sk_bytes) return set_error(TP_ERR_WORKSPACE, "GEMV scratch too small");
-    gemv::Args a{static_cast<const __nv_bfloat16*>(wqkv), static_cast<const __nv_bfloat16*>(x),
-                 rows, L.h, 1, 0, L.h, static_cast<int>(L.tokens), 0, 0, static_cast<float*>(sk_ws)};
-    tp_status st = gemv::run(a, P, s, "attn_qkv_gemm");
-    if (st != TP_OK) return st;
-    ProfScope prof(s, "attn_qkv_fixup");
-    TP_LAUNCH_PDL(gemv::fix_store_kernel, dim3(gemv::fix_grid(rows * L.tokens)), dim3(256), 0, s,
-                  gemv::fix_args(a, P), static_cast<int64_t>(1), rows, static_cast<float*>(nullptr),
-                  static_cast<__nv_bfloat16*>(qkv), rows);
-    return TP_OK;
-  }
   const Operand xo{x, false, L.tokens, L.h, 1, L.h, 0};
   const Operand wo{wqkv, false, rows, L.h, 1, L.h, 0};
   if (L.tokens <= kSwapMaxT) {
@@ -977,22 +953,6 @@ inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, 
                           const void* residual, void* y, void* sk_ws, size_t sk_bytes,
                           cudaStream_t s) {
   const int64_t K = static_cast<int64_t>(L.qh) * L.hd;
-  if (L.gemv) {
-    // a few tokens: shard i's partial o_i Wo_i as a streaming matrix-vector product over all
-    // shards' rows, written as the fp32 partials [p][tokens][h] that the reduce kernel adds
-    const gemv::Plan P = gemv::plan(L.h, K, L.p, static_cast<int>(L.tokens), num_sms());
-    if (P.pieces_bytes > sk_bytes) return set_error(TP_ERR_WORKSPACE, "GEMV scratch too small");
-    gemv::Args a{static_cast<const __nv_bfloat16*>(wo_p), static_cast<const __nv_bfloat16*>(o),
-                 L.h, K, L.p, K, static_cast<int64_t>(L.n_q) * L.hd, static_cast<int>(L.tokens), 0, 0,
-                 static_cast<float*>(sk_ws)};
-    tp_status st = gemv::run(a, P, s, "attn_out_gemm");
-    if (st != TP_OK) return st;
-    ProfScope prof(s, "attn_out_fixup");
-    TP_LAUNCH_PDL(gemv::fix_store_kernel, dim3(gemv::fix_grid(L.p * L.h * L.tokens)), dim3(256), 0,
-                  s, gemv::fix_args(a, P), static_cast<int64_t>(L.p), L.h, part,
-                  static_cast<__nv_bfloat16*>(nullptr), static_cast<int64_t>(0));
-    return TP_OK;
-  }
   const Operand ao{o, false, L.tokens, K, L.p, static_cast<int64_t>(L.n_q) * L.hd, K};
   const Operand wo{wo_p, false, L.h, K, L.p, K, L.h * K};
   const bool swap = L.tokens <= kSwapMaxT;
@@ -1087,7 +1047,7 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
     if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, sk, skb, s)) != TP_OK) return st;
     if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
     if ((st = attn_tc::out_proj(L, o, wo_p, part, residual, y, sk, skb, s)) != TP_OK) return st;
-    if (L.reduce_mode == TP_REDUCE_FUSED && !L.gemv)
+    if (L.reduce_mode == TP_REDUCE_FUSED)
       return y_norm ? reduce::rmsnorm(y, L.y_dtype, L.tokens, L.h, L.norm_eps, y_norm, L.dtype, s)
                     : TP_OK;
   } else if (L.dtype == TP_BF16) {

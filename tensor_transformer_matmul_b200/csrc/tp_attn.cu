@@ -133,8 +133,7 @@ tp_status attn_bwd_check(const tp_attn_desc* desc, tp::AttnLayout* L) {
   if (L->kv_len != 0) return tp::set_error(TP_ERR_UNSUPPORTED, "backward is for self-attention (kv_len == 0)");
   if (!L->tc) return tp::set_error(TP_ERR_UNSUPPORTED, "backward needs bf16 with h a multiple of 8");
   if (L->hd > 256) return tp::set_error(TP_ERR_UNSUPPORTED, "backward needs head_dim <= 256");
-  if (desc->flags & ~TP_FLAG_DECODE_TILES)
-    return tp::set_error(TP_ERR_UNSUPPORTED, "backward takes no residual flag");
+  if (desc->flags != 0) return tp::set_error(TP_ERR_UNSUPPORTED, "backward takes no flags");
   return TP_OK;
 }
 }  // namespace
@@ -260,14 +259,13 @@ tp_status attn_shard_desc(const tp_attn_desc* desc, int32_t shard, int32_t parti
     return tp::set_error(TP_ERR_INVALID_ARG, "partial_dtype must be TP_F32 or TP_BF16");
   if (L.dtype == TP_F32 && partial_dtype != TP_F32)
     return tp::set_error(TP_ERR_UNSUPPORTED, "fp32 blocks give fp32 partials");
-  if (desc->flags & ~TP_FLAG_DECODE_TILES)
-    return tp::set_error(TP_ERR_INVALID_ARG, "shard calls take no residual flag (partial_dtype sets the type)");
+  if (desc->flags != 0)
+    return tp::set_error(TP_ERR_INVALID_ARG, "shard calls take no flags (partial_dtype sets the type)");
   *sd = *desc;
   sd->n_q = desc->n_q / desc->p;
   sd->n_kv = desc->n_kv / desc->p;
   sd->p = 1;
-  sd->flags = ((L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0) |
-              (desc->flags & TP_FLAG_DECODE_TILES);
+  sd->flags = (L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0;
   sd->reduce_mode = L.tc ? TP_REDUCE_FUSED : TP_REDUCE_SEPARATE;
   return tp::attn_layout_of(sd, LS);
 }

@@ -14,7 +14,6 @@
 
 #include "gemm_launch.cuh"
 #include "gemm_pair.cuh"
-#include "gemv.cuh"
 #include "moe.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
@@ -37,7 +36,6 @@ struct MlpLayout {
   int p, act, dtype, eb, y_dtype, reduce_mode;
   float norm_eps;
   bool tc;                      // bf16 with 16-byte rows: the tensor-core path
-  bool gemv;                    // 1..4 tokens, d and F_sp multiples of 256: the decode GEMV path
   size_t w1p_bytes, w2p_bytes;
   size_t saved_z_off, saved_h_off, saved_bytes;
   size_t fz_off, fh_off, fpart_off, fsk_off, fwd_ws;
@@ -97,8 +95,7 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
     return set_error(TP_ERR_INVALID_ARG, "dtype must be TP_F32 or TP_BF16");
   if (desc->reduce_mode != TP_REDUCE_SEPARATE && desc->reduce_mode != TP_REDUCE_FUSED)
     return set_error(TP_ERR_INVALID_ARG, "unknown reduce_mode");
-  if (desc->flags & ~(TP_FLAG_F32_RESIDUAL | TP_FLAG_DECODE_TILES))
-    return set_error(TP_ERR_INVALID_ARG, "unknown flags");
+  if (desc->flags & ~TP_FLAG_F32_RESIDUAL) return set_error(TP_ERR_INVALID_ARG, "unknown flags");
   L->y_dtype = (desc->flags & TP_FLAG_F32_RESIDUAL) ? TP_F32 : desc->dtype;
   L->T = desc->T; L->d = desc->d; L->F = desc->d_ff; L->p = desc->p;
   L->act = desc->act; L->dtype = desc->dtype; L->eb = elem_bytes(desc->dtype);
@@ -114,8 +111,6 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
   const size_t zb = static_cast<size_t>(L->T * P * L->R) * L->eb;
   const size_t hb = static_cast<size_t>(L->T * P * L->Fsp) * L->eb;
   const size_t partb = static_cast<size_t>(P * L->T * L->d) * 4;
-  L->gemv = L->tc && !(desc->flags & TP_FLAG_DECODE_TILES) && gemv::usable(L->T, L->d) &&
-            L->Fsp % gemv::kStep == 0;
   L->saved_z_off = 0;
   L->saved_h_off = align256(zb);
   L->saved_bytes = L->saved_h_off + align256(hb);
@@ -125,13 +120,9 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
     L->fz_off = 0;
     L->fh_off = 0;
     L->fsk_off = align256(hb);
-    size_t sk = L->T > 0 ? std::max(up_sk_bytes(*L), down_sk_bytes(*L)) : 0;
-    if (L->gemv)   // the GEMV pieces of the up and down projections (one after the other)
-      sk = std::max({sk, gemv::plan(P * L->R, L->d, 1, static_cast<int>(L->T), num_sms()).pieces_bytes,
-                     gemv::plan(L->d, L->Fsp, P, static_cast<int>(L->T), num_sms()).pieces_bytes});
+    const size_t sk = L->T > 0 ? std::max(up_sk_bytes(*L), down_sk_bytes(*L)) : 0;
     L->fpart_off = L->fsk_off + align256(sk);
-    // the GEMV path always materialises the partials (its shard sum is the reduce kernel's)
-    const size_t pb = (L->reduce_mode == TP_REDUCE_FUSED && !L->gemv) ? 0 : partb;
+    const size_t pb = L->reduce_mode == TP_REDUCE_FUSED ? 0 : partb;
     L->fwd_ws = L->fpart_off + align256(pb);
   } else {
     L->fz_off = 0;
@@ -165,20 +156,6 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
   ep.tokens = static_cast<int32_t>(L.T);
   ep.rows = static_cast<int32_t>(rows);
   ep.act = L.act;
-  if (L.gemv) {
-    // a few tokens: a streaming matrix-vector product, then the activation epilogue
-    const gemv::Plan P = gemv::plan(rows, L.d, 1, static_cast<int>(L.T), num_sms());
-    if (P.pieces_bytes > sk_bytes) return set_error(TP_ERR_WORKSPACE, "GEMV scratch too small");
-    gemv::Args a{static_cast<const __nv_bfloat16*>(w1p), static_cast<const __nv_bfloat16*>(x),
-                 rows, L.d, 1, 0, L.d, static_cast<int>(L.T), 0, 0, static_cast<float*>(sk_ws)};
-    tp_status st = gemv::run(a, P, s, "mlp_up_gemm");
-    if (st != TP_OK) return st;
-    ProfScope prof(s, "mlp_up_fixup");
-    TP_LAUNCH_PDL(gemv::fix_hidden_kernel, dim3(gemv::fix_grid(L.p * L.Fsp * L.T)), dim3(256), 0,
-                  s, gemv::fix_args(a, P), L.p, L.R, L.Fsp, L.act,
-                  static_cast<__nv_bfloat16*>(h), static_cast<__nv_bfloat16*>(z));
-    return TP_OK;
-  }
   const Operand xo{x, false, L.T, L.d, 1, L.d, 0};
   const Operand wo{w1p, false, rows, L.d, 1, L.d, 0};
   if (L.T <= kSwapMaxT) {
@@ -203,22 +180,6 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
 // Fused reduce: y = residual + sum_i h_i W2_i written directly (shards added in order).
 tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* part,
                   const void* residual, void* y, void* sk_ws, size_t sk_bytes, cudaStream_t s) {
-  if (L.gemv) {
-    // a few tokens: shard i's partial y_i = h_i W2_i as a streaming matrix-vector product over
-    // all shards' rows, written as the fp32 partials [p][T][d] that the reduce kernel adds
-    const gemv::Plan P = gemv::plan(L.d, L.Fsp, L.p, static_cast<int>(L.T), num_sms());
-    if (P.pieces_bytes > sk_bytes) return set_error(TP_ERR_WORKSPACE, "GEMV scratch too small");
-    gemv::Args a{static_cast<const __nv_bfloat16*>(w2p), static_cast<const __nv_bfloat16*>(h),
-                 L.d, L.Fsp, L.p, L.Fsp, L.p * L.Fsp, static_cast<int>(L.T), 0, 0,
-                 static_cast<float*>(sk_ws)};
-    tp_status st = gemv::run(a, P, s, "mlp_down_gemm");
-    if (st != TP_OK) return st;
-    ProfScope prof(s, "mlp_down_fixup");
-    TP_LAUNCH_PDL(gemv::fix_store_kernel, dim3(gemv::fix_grid(L.p * L.d * L.T)), dim3(256), 0, s,
-                  gemv::fix_args(a, P), static_cast<int64_t>(L.p), L.d, part,
-                  static_cast<__nv_bfloat16*>(nullptr), static_cast<int64_t>(0));
-    return TP_OK;
-  }
   const Operand ho{h, false, L.T, L.Fsp, L.p, L.p * L.Fsp, L.Fsp};
   const Operand wo{w2p, false, L.d, L.Fsp, L.p, L.Fsp, L.d * L.Fsp};
   const bool swap = L.T <= kSwapMaxT;
@@ -556,7 +517,7 @@ tp_status mlp_forward(const MlpLayout& L, const tp_mlp_desc* desc, const void* x
     const size_t skb = L.fpart_off - L.fsk_off;
     if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
     if ((st = tc_down(L, h, w2p, part, residual, y, sk, skb, s)) != TP_OK) return st;
-    if (L.reduce_mode == TP_REDUCE_FUSED && !L.gemv) {
+    if (L.reduce_mode == TP_REDUCE_FUSED) {
       if (y_norm && (st = reduce::rmsnorm(y, L.y_dtype, L.T, L.d, L.norm_eps, y_norm, L.dtype, s)) != TP_OK)
         return st;
       if (count) count_reduction();
@@ -663,13 +624,12 @@ tp_status shard_desc_of(const tp_mlp_desc* desc, int32_t shard, int32_t partial_
     return set_error(TP_ERR_INVALID_ARG, "partial_dtype must be TP_F32 or TP_BF16");
   if (L.dtype == TP_F32 && partial_dtype != TP_F32)
     return set_error(TP_ERR_UNSUPPORTED, "fp32 blocks give fp32 partials");
-  if (desc->flags & ~TP_FLAG_DECODE_TILES)
-    return set_error(TP_ERR_INVALID_ARG, "shard calls take no residual flag (partial_dtype sets the type)");
+  if (desc->flags != 0)
+    return set_error(TP_ERR_INVALID_ARG, "shard calls take no flags (partial_dtype sets the type)");
   *sd = *desc;
   sd->d_ff = L.Fs;
   sd->p = 1;
-  sd->flags = ((L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0) |
-              (desc->flags & TP_FLAG_DECODE_TILES);
+  sd->flags = (L.dtype == TP_BF16 && partial_dtype == TP_F32) ? TP_FLAG_F32_RESIDUAL : 0;
   sd->reduce_mode = L.tc ? TP_REDUCE_FUSED : TP_REDUCE_SEPARATE;
   return layout_of(sd, LS);
 }
@@ -920,7 +880,6 @@ tp_status moe_layout(const tp_moe_desc* desc, MoeLayout* M) {
     tp_mlp_desc ms{M->T, M->d, M->Fsh, M->p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_FUSED,
                    TP_FLAG_F32_RESIDUAL, 0.f};
     if ((st = layout_of(&ms, &M->sh)) != TP_OK) return st;
-    M->sh.gemv = false;   // its down GEMM writes the summed [T][d] itself (no partials buffer)
   }
   size_t o = 0;
   auto take = [&](size_t& field, size_t bytes) {

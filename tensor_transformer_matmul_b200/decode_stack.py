@@ -32,14 +32,13 @@ from . import tpblock as tp
 
 class DecodeStack:
     def __init__(self, layers, h, d_ff, n_q, n_kv, head_dim, p, kv_len, b=1, seed=0,
-                 w_std=0.02, device=None, reduce_mode=tp.TP_REDUCE_SEPARATE, flags=0):
-        """``flags``: extra descriptor flags for every block (e.g. TP_FLAG_DECODE_TILES)."""
+                 w_std=0.02, device=None, reduce_mode=tp.TP_REDUCE_SEPARATE):
         self.device = device or torch.device("cuda", torch.cuda.current_device())
         self.L, self.h, self.b = layers, h, b
         self.adesc = tp.attn_desc(b, 1, h, n_q, n_kv, head_dim, p, True, "bf16", kv_len,
-                                  reduce_mode=reduce_mode, flags=tp.TP_FLAG_F32_RESIDUAL | flags)
+                                  reduce_mode=reduce_mode, flags=tp.TP_FLAG_F32_RESIDUAL)
         self.mdesc = tp.mlp_desc(b, h, d_ff, p, "swiglu", "bf16", reduce_mode,
-                                 flags=tp.TP_FLAG_F32_RESIDUAL | flags)
+                                 flags=tp.TP_FLAG_F32_RESIDUAL)
         self.layers = []
         for l in range(layers):
             a = inputs.attn_inputs(b, 1, h, n_q, n_kv, head_dim, "bf16", seed=seed,

@@ -100,14 +100,13 @@ def moe_fwd(tokens, reps, fused, d=7168, n_experts=32, top_k=8, d_ff=2048, p=8):
 
 
 def decode_layer(tokens, reps, fused, h=8192, d_ff=28672, n_q=64, n_kv=8, hd=128, p=8,
-                 kv_len=4096, flags=0):
+                 kv_len=4096):
     """One layer of the decode stack (b = ``tokens`` single-token sequences, KV length 4096):
     the attention block (QKV GEMM, split-KV decode attention with the KV append, O projection,
     reduce + RMSNorm) then the SwiGLU MLP block, fp32 residual stream."""
     from tensor_transformer_matmul_b200.decode_stack import DecodeStack
     mode = tp.TP_REDUCE_FUSED if fused else tp.TP_REDUCE_SEPARATE
-    st = DecodeStack(1, h, d_ff, n_q, n_kv, hd, p, kv_len, b=tokens, reduce_mode=mode,
-                     flags=flags)
+    st = DecodeStack(1, h, d_ff, n_q, n_kv, hd, p, kv_len, b=tokens, reduce_mode=mode)
     x = torch.randn(tokens, 1, h, device="cuda")
     for _ in range(reps):
         st.step(x)
@@ -125,13 +124,8 @@ def main(argv=None):
     ap.add_argument("--tokens", type=int, default=1024)
     ap.add_argument("--reps", type=int, default=4)
     ap.add_argument("--fused", action="store_true", help="TP_REDUCE_FUSED instead of SEPARATE")
-    ap.add_argument("--tiles", action="store_true",
-                    help="decode_layer: TP_FLAG_DECODE_TILES (tensor-core tiles at 1-4 tokens)")
     a = ap.parse_args(argv)
-    if a.case == "decode_layer":
-        y = decode_layer(a.tokens, a.reps, a.fused, flags=tp.TP_FLAG_DECODE_TILES if a.tiles else 0)
-    else:
-        y = CASES[a.case](a.tokens, a.reps, a.fused)
+    y = CASES[a.case](a.tokens, a.reps, a.fused)
     print(f"{a.case} tokens={a.tokens} reps={a.reps} fused={a.fused} ok, mean|y|="
           f"{float(y.float().abs().mean()):.4f}")
 

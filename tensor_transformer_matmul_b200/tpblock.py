@@ -23,7 +23,6 @@ DTYPE = {"f32": TP_F32, "bf16": TP_BF16}
 TORCH_OF = {TP_F32: torch.float32, TP_BF16: torch.bfloat16}
 TP_REDUCE_SEPARATE, TP_REDUCE_FUSED = 0, 1
 TP_FLAG_F32_RESIDUAL = 1
-TP_FLAG_DECODE_TILES = 2
 
 # every symbol the header declares
 EXPORTS = (

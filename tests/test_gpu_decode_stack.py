@@ -62,21 +62,6 @@ def test_small_stack(lib, graph):
     assert rel_l2(f64(out)[:, 0], ref) <= TOL["bf16"]
 
 
-def test_small_stack_decode_tiles(lib):
-    # the same stack with the projections on the tensor-core tiles (TP_FLAG_DECODE_TILES)
-    cfg = dict(layers=2, b=1, h=512, F=1536, n_q=8, n_kv=2, hd=64, p=2, kv_len=200, seed=4)
-    st = DecodeStack(cfg["layers"], cfg["h"], cfg["F"], cfg["n_q"], cfg["n_kv"], cfg["hd"],
-                     cfg["p"], cfg["kv_len"], b=cfg["b"], seed=cfg["seed"], device=dev(),
-                     flags=lib.TP_FLAG_DECODE_TILES)
-    caches = [(f64(l["k_cache"])[:, :, :cfg["kv_len"]], f64(l["v_cache"])[:, :, :cfg["kv_len"]])
-              for l in st.layers]
-    x0 = inputs.normal((cfg["b"], 1, cfg["h"]), 1.0, cfg["seed"], 97, "bf16", "cpu")
-    out = st.step(x0.to(dev()).float())
-    torch.cuda.synchronize()
-    ref, _ = _oracle_stack(cfg, f64(x0)[:, 0], caches, dev())
-    assert rel_l2(f64(out)[:, 0], ref) <= TOL["bf16"]
-
-
 def test_full_size_stack(lib):
     # 16 Llama-70B-shaped layers: h=8192, d_ff=28672, 64 Q / 8 KV heads, hd=128, p=8,
     # b=1, s=1, KV length 4096; 2 reductions of 1 x 8192 per layer

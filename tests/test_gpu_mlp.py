@@ -267,9 +267,8 @@ def test_y_norm_output(lib, reduce_mode, T):
 @pytest.mark.parametrize("reduce_mode", [0, 1])
 @pytest.mark.parametrize("act", ["swiglu", "gelu", "relu", "identity"])
 @pytest.mark.parametrize("T", [1, 2, 3, 4])
-def test_gemv_decode_path(lib, act, T, reduce_mode):
-    # 1..4 tokens with d and the padded shard width multiples of 256 run the decode GEMV path
-    # (streaming matrix-vector products, the shard sum in the reduce kernel in both modes):
+def test_few_tokens_decode_path(lib, act, T, reduce_mode):
+    # 1..4 tokens (the decode stack's batch sizes) on the swapped decode tiles, both reduce modes:
     # d = 512, d_ff = 1536 over p = 3 (512 features per shard), residual and RMSNorm output
     from oracle import decode as odec
     d, F, p = 512, 1536, 3
@@ -300,7 +299,7 @@ def test_gemv_decode_path(lib, act, T, reduce_mode):
     assert torch.equal(y, y2)
 
 
-def test_gemv_decode_full_size_one_token(lib):
+def test_decode_full_size_one_token(lib):
     # the decode stack's MLP shape at b = 1: d=8192, d_ff=28672, p=8, one token
     T, d, F, p = 1, 8192, 28672, 8
     inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=0, device="cuda", w_std=0.02)
@@ -310,21 +309,3 @@ def test_gemv_decode_full_size_one_token(lib):
     ref = omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "swiglu",
                            f64(inp["w_up"]))
     assert rel_l2(f64(y), ref) <= TOL["bf16"]
-
-
-@pytest.mark.parametrize("T", [1, 4])
-def test_decode_tiles_flag(lib, T):
-    # TP_FLAG_DECODE_TILES runs 1-4 tokens on the tensor-core tiles instead of the GEMV path:
-    # both match the oracle
-    d, F, p = 512, 1536, 3
-    inp = inputs.mlp_inputs(T, d, F, "swiglu", "bf16", seed=40 + T, w_std=0.05)
-    m = Mlp(lib, inp, p, "swiglu", "bf16")
-    ref = _oracle_fwd(inp, "swiglu")
-    for flags in (0, lib.TP_FLAG_DECODE_TILES):
-        desc = lib.mlp_desc(T, d, F, p, "swiglu", "bf16", flags=flags)
-        ws = torch.empty(lib.tp_mlp_fwd_workspace(desc), dtype=torch.uint8, device=dev())
-        y = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
-        lib.tp_mlp_fwd(desc, inp["x"].to(dev()), m.w1p, m.w2p, y, workspace=ws)
-        torch.cuda.synchronize()
-        assert rel_l2(f64(y), ref) <= TOL["bf16"] and rel_l2_rows(f64(y), ref) <= TOL["bf16"]
-
