@@ -976,8 +976,8 @@ inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, 
       });
     // prefill: each 256 x 256 tile runs the k-blocks of shard 0, 1, ..., p-1 into one
     // accumulator, so the shard sum never leaves TMEM
-    return tc::run_gemm_pair_fit<false, false, tc::EpiReduceOut>(ao, wo, L.tokens, L.h, K, L.p,
-                                                                 ep, s, "attn_out_gemm", true);
+    return tc::run_gemm_pair<PP<false, false>, tc::EpiReduceOut>(ao, wo, L.tokens, L.h, K, L.p, ep,
+                                                                 s, "attn_out_gemm", -1, true);
   }
   tc::EpiStoreF32::Params ep;
   ep.out = part;

@@ -321,8 +321,8 @@ inline tp_status attn_backward(const AttnLayout& L, const void* x, const void* w
       ep.cols_valid = static_cast<int32_t>(L.h);
       ep.out_bf16 = 1;
       ep.swap = 0;
-      return tc::run_gemm_pair_fit<false, true, tc::EpiReduceOut>(
-          a, bw, T, L.h, L.R_a, P, ep, s, "attn_dx_gemm", true);
+      return tc::run_gemm_pair<attn_tc::PP<false, true>, tc::EpiReduceOut>(
+          a, bw, T, L.h, L.R_a, P, ep, s, "attn_dx_gemm", -1, true);
     }
     tc::EpiStoreF32::Params ep;
     ep.out = part;

@@ -2,8 +2,8 @@
 //
 //   D[b][m][n] = sum_k A_b(m, k) * B_b(n, k)      (bf16 operands, fp32 accumulator in TMEM)
 //
-// A cluster of two CTAs on a pair of SMs computes one 256 x 256 (or 256 x 128) output tile with
-// tcgen05.mma.cta_group::2 (M = 256, N = 256 or 128).  CTA r (its rank in the cluster) keeps rows
+// A cluster of two CTAs on a pair of SMs computes one 256 x 256 output tile with
+// tcgen05.mma.cta_group::2 (M = 256, N = 256).  CTA r (its rank in the cluster) keeps rows
 // 128 r .. 128 r + 127 of the tile's A block and rows 128 r .. 128 r + 127 of its B block in its
 // own shared memory; its TMEM receives the accumulator rows of its own A rows, all 256 columns.
 // Per SM this is the MMA work of a one-CTA 128 x 256 tile with half of that tile's B traffic:
@@ -35,31 +35,26 @@
 namespace tp {
 namespace tc {
 
-// Compile-time configuration of the pair tile: TILE (256) rows of the output by TILE_N (256 or
-// 128) columns; per CTA and stage, 128 A rows and TILE_N / 2 B rows.  The 256 x 128 tile doubles
-// the tile count of a GEMM whose 256 x 256 tiles would fill only a few waves of the SM pairs.
-template <bool A_MN_, bool B_MN_, int STAGES_, int TILE_N_ = 256>
+// Compile-time configuration of the pair tile (per CTA: 128 A rows, 128 B rows per stage).
+template <bool A_MN_, bool B_MN_, int STAGES_>
 struct PairCfg {
   static constexpr bool A_MN = A_MN_;
   static constexpr bool B_MN = B_MN_;
   static constexpr int STAGES = STAGES_;
-  static constexpr int TILE = 256;                 // output tile rows (M)
-  static constexpr int TILE_N = TILE_N_;           // output tile columns (N)
-  static constexpr int HALF = 128;                 // rows of A held by each CTA
-  static constexpr int B_HALF = TILE_N / 2;        // rows of B held by each CTA
+  static constexpr int TILE = 256;                 // output tile is TILE x TILE
+  static constexpr int HALF = 128;                 // rows of A and of B held by each CTA
   static constexpr int A_STAGE_BYTES = HALF * kBK * 2;
-  static constexpr int B_STAGE_BYTES = B_HALF * kBK * 2;
+  static constexpr int B_STAGE_BYTES = HALF * kBK * 2;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
-  static constexpr int ACC_COLS = TILE_N;          // accumulator columns in each CTA's TMEM
+  static constexpr int ACC_COLS = TILE;            // accumulator columns in each CTA's TMEM
   static constexpr int TMEM_COLS = 2 * ACC_COLS;   // two accumulators
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 32;
   static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
-  static constexpr uint32_t IDESC = sm100::make_idesc_bf16(2 * HALF, TILE_N, A_MN, B_MN);
-  // what the epilogues see: a 128-row x TILE_N-column accumulator, as a one-CTA tile
-  static constexpr int BN = TILE_N;
+  static constexpr uint32_t IDESC = sm100::make_idesc_bf16(2 * HALF, TILE, A_MN, B_MN);
+  // what the epilogues see: a 128-row x 256-column accumulator, as a one-CTA 128 x 256 tile
+  static constexpr int BN = TILE;
   static constexpr int A_SUB = 1;
   static constexpr int A_ROWS = HALF;
-  static_assert(TILE_N == 256 || TILE_N == 128, "pair tiles are 256 x 256 or 256 x 128");
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
 
@@ -222,7 +217,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         int b, mb, nb;
         pair::decode_tile(t, gp, b, mb, nb);
         const int m0 = mb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
-        const int n0 = nb * Cfg::TILE_N + Cfg::B_HALF * static_cast<int>(rank);
+        const int n0 = nb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
         int bu = b, kb = 0;   // problem and k-block of step u
         for (int u = 0; u < nk; ++u, ++kb) {
           if (kb == gp.k_blocks) {   // sum_batch: on to the next problem's k-blocks
@@ -249,7 +244,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           if (Cfg::B_MN) {
 #pragma unroll
-            for (int j = 0; j < Cfg::B_HALF / 64; ++j)
+            for (int j = 0; j < Cfg::HALF / 64; ++j)
               pair::tma_load_3d_pair(&tma_b, fb, sb + j * 64 * kBK * 2, n0 + 64 * j, k0, zb);
           } else {
             pair::tma_load_3d_pair(&tma_b, fb, sb, k0, n0, zb);
@@ -364,7 +359,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctx.row = row;
       ctx.b = b;
       ctx.m0 = mb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
-      ctx.n0 = nb * Cfg::TILE_N;
+      ctx.n0 = nb * Cfg::TILE;
       Epi::template run<Cfg>(ep, gp, ctx, tsrc);
       tc_fence_before();
       __syncwarp();
@@ -430,7 +425,7 @@ tp_status run_gemm_pair(const Operand& a, const Operand& b, int64_t M, int64_t N
   CUtensorMap ta, tb;
   tp_status st = encode_operand(&ta, a, Cfg::HALF);
   if (st != TP_OK) return st;
-  st = encode_operand(&tb, b, Cfg::B_HALF);
+  st = encode_operand(&tb, b, Cfg::HALF);
   if (st != TP_OK) return st;
 
   GemmParams gp = {};
@@ -439,7 +434,7 @@ tp_status run_gemm_pair(const Operand& a, const Operand& b, int64_t M, int64_t N
   gp.K = static_cast<int32_t>(K);
   gp.batch = static_cast<int32_t>(batch);
   gp.m_blocks = static_cast<int32_t>(ceil_div(M, Cfg::TILE));
-  gp.n_blocks = static_cast<int32_t>(ceil_div(N, Cfg::TILE_N));
+  gp.n_blocks = static_cast<int32_t>(ceil_div(N, Cfg::TILE));
   gp.k_blocks = static_cast<int32_t>(ceil_div(K, kBK));
   gp.m_fastest = m_fastest >= 0 ? m_fastest : (gp.m_blocks <= gp.n_blocks ? 1 : 0);
   gp.a_batched = a.batch > 1 ? 1 : 0;
@@ -476,30 +471,6 @@ tp_status run_gemm_pair(const Operand& a, const Operand& b, int64_t M, int64_t N
     return set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
   count_launch();
   return TP_OK;
-}
-
-// Run on 256 x 256 pair tiles, or on 256 x 128 ones when those fill the resident SM pairs'
-// waves enough better to pay for their narrower tile (about 7% less MMA work per shared-memory
-// byte, so a 256 x 128 tile is assumed 0.93 as efficient).  With sum_batch the tile count drops
-// the problem index, as in run_gemm_pair.
-template <bool A_MN, bool B_MN, class Epi>
-tp_status run_gemm_pair_fit(const Operand& a, const Operand& b, int64_t M, int64_t N, int64_t K,
-                            int64_t batch, const typename Epi::Params& ep, cudaStream_t stream,
-                            const char* label, bool sum_batch = false) {
-  using Wide = PairCfg<A_MN, B_MN, 6, 256>;
-  using Narrow = PairCfg<A_MN, B_MN, 8, 128>;
-  int resident = 0;
-  tp_status st = pair_clusters<Wide, Epi>(&resident);
-  if (st != TP_OK) return st;
-  const int64_t per = sum_batch ? 1 : batch;
-  const int64_t t_wide = per * ceil_div(M, 256) * ceil_div(N, 256);
-  const int64_t t_narrow = per * ceil_div(M, 256) * ceil_div(N, 128);
-  auto fill = [&](int64_t t) {
-    return static_cast<double>(t) / static_cast<double>(ceil_div(t, resident) * resident);
-  };
-  if (0.93 * fill(t_narrow) > fill(t_wide))
-    return run_gemm_pair<Narrow, Epi>(a, b, M, N, K, batch, ep, stream, label, -1, sum_batch);
-  return run_gemm_pair<Wide, Epi>(a, b, M, N, K, batch, ep, stream, label, -1, sum_batch);
 }
 
 }  // namespace tc
