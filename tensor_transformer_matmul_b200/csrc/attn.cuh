@@ -818,7 +818,8 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
 
 template <typename T>
 inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, void* kc, void* vc,
-                           float* ml, int* counters, cudaStream_t s, float* lse = nullptr) {
+                           float* ml, int* counters, cudaStream_t s, float* lse = nullptr,
+                           bool counters_zeroed = false) {
   const T* qkv = static_cast<const T*>(qkv_v);
   T* o = static_cast<T*>(o_v);
   attn::QkvIdx ix{L.p * L.R_a, L.R_a, L.qh, L.kh, L.hd, L.n_q / L.n_kv};
@@ -848,7 +849,7 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
   dim3 grid(static_cast<unsigned>(L.kv_splits), static_cast<unsigned>(L.n_kv),
             static_cast<unsigned>(L.b));
   if (L.b > 65535) return set_error(TP_ERR_UNSUPPORTED, "decode batch above 65535");
-  {
+  if (!counters_zeroed) {   // else the projection's launch cleared them
     const int64_t words = L.b * L.n_kv;
     TP_LAUNCH_PDL(zero_words_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words, 256), 64))),
                   dim3(256), 0, s, reinterpret_cast<uint32_t*>(counters), words);
@@ -919,7 +920,8 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
 namespace attn_tc {
 
 inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, void* qkv,
-                          void* sk_ws, size_t sk_bytes, cudaStream_t s) {
+                          void* sk_ws, size_t sk_bytes, cudaStream_t s,
+                          int* zero_also = nullptr, int64_t zero_also_words = 0) {
   const int64_t rows = L.p * L.R_a;
   tc::EpiHidden::Params ep;
   ep.h = static_cast<__nv_bfloat16*>(qkv);
@@ -937,11 +939,17 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
     tc::GemmOpts opt;
     opt.sk = decode_stream_k(qkv_tiles(L)) ? &sk : nullptr;
     opt.rotate_k = true;
+    opt.zero_also = reinterpret_cast<uint32_t*>(zero_also);
+    opt.zero_also_words = zero_also ? zero_also_words : 0;
     return by_tokens(L.tokens, [&](auto t) {
       return tc::run_gemm<typename decltype(t)::type, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1,
                                                                      ep, s, "attn_qkv_gemm", opt);
     });
   }
+  if (zero_also && zero_also_words > 0)
+    TP_LAUNCH_PDL(zero_words_kernel,
+                  dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(zero_also_words, 256), 64))),
+                  dim3(256), 0, s, reinterpret_cast<uint32_t*>(zero_also), zero_also_words);
   ep.swap = 0;
   return tc::run_gemm_pair<PP<false, false>, tc::EpiHidden>(xo, wo, L.tokens, rows, L.h, 1, ep, s,
                                                             "attn_qkv_gemm");
@@ -1044,8 +1052,13 @@ inline tp_status attn_forward(const AttnLayout& L, const void* x, const void* wq
         return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
     void* sk = w + L.sk_off;
     const size_t skb = L.ws_bytes - L.sk_off;
-    if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, sk, skb, s)) != TP_OK) return st;
-    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, counters, s)) != TP_OK) return st;
+    // decode: the projection's launch also clears the split-merge counters of the attention
+    const bool dec = L.kv_len > 0;
+    if ((st = attn_tc::qkv_proj(L, x, wqkv, qkv, sk, skb, s, dec ? counters : nullptr,
+                                dec ? L.b * L.n_kv : 0)) != TP_OK)
+      return st;
+    if ((st = attn_core<__nv_bfloat16>(L, qkv, o, kc, vc, ml, counters, s, nullptr, dec)) != TP_OK)
+      return st;
     if ((st = attn_tc::out_proj(L, o, wo_p, part, residual, y, sk, skb, s)) != TP_OK) return st;
     if (L.reduce_mode == TP_REDUCE_FUSED)
       return y_norm ? reduce::rmsnorm(y, L.y_dtype, L.tokens, L.h, L.norm_eps, y_norm, L.dtype, s)

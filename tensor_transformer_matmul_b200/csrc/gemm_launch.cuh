@@ -114,6 +114,10 @@ struct GemmOpts {
   int grp_n = 0;
   int grp_div = 1;
   bool grp_sum = false;   // sum each group's grp_div problems into one output (in order)
+  // words that the kernel after this GEMM needs zeroed: cleared by the launch that zeroes the
+  // stream-K counters (one kernel for both), or by a small kernel of their own
+  uint32_t* zero_also = nullptr;
+  int64_t zero_also_words = 0;
 };
 
 // Launch gemm_kernel<Cfg, Epi> over ``batch`` problems of D = A B^T (M x N, contraction K).
@@ -182,8 +186,16 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
     gp.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(sk->ws) + pl.counter_bytes);
     grid_sk = pl.grid;
     const int64_t words = static_cast<int64_t>(pl.counter_bytes / 4);
-    TP_LAUNCH_PDL(zero_words_kernel, dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words, 256), 64))),
-                  dim3(256), 0, stream, static_cast<uint32_t*>(sk->ws), words);
+    const int64_t extra = opts.zero_also ? opts.zero_also_words : 0;
+    TP_LAUNCH_PDL(zero_words2_kernel,
+                  dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(words + extra, 256), 64))),
+                  dim3(256), 0, stream, static_cast<uint32_t*>(sk->ws), words, opts.zero_also,
+                  extra);
+  } else if (opts.zero_also && opts.zero_also_words > 0) {
+    const int64_t extra = opts.zero_also_words;
+    TP_LAUNCH_PDL(zero_words_kernel,
+                  dim3(static_cast<unsigned>(std::min<int64_t>(ceil_div(extra, 256), 64))),
+                  dim3(256), 0, stream, opts.zero_also, extra);
   }
 
   static int attr_set[64] = {0};

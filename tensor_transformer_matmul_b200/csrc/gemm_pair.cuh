@@ -60,21 +60,6 @@ struct PairCfg {
 
 namespace pair {
 
-__device__ __forceinline__ uint32_t cluster_rank() {
-  uint32_t r;
-  asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
-  return r;
-}
-// shared::cluster address of the same shared variable in the CTA of the given rank
-__device__ __forceinline__ uint32_t map_to_rank(uint32_t smem_cta_addr, uint32_t rank) {
-  uint32_t r;
-  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_cta_addr), "r"(rank));
-  return r;
-}
-// every thread of both CTAs: arrive (release) and wait (acquire)
-__device__ __forceinline__ void cluster_sync() {
-  asm volatile("barrier.cluster.arrive.release;\n\tbarrier.cluster.wait.acquire;" ::: "memory");
-}
 // arrive on an mbarrier given by its shared::cluster address (possibly in the peer CTA)
 __device__ __forceinline__ void mbar_arrive_cluster(uint32_t bar_cluster_addr) {
   asm volatile("mbarrier.arrive.release.cluster.shared::cluster.b64 _, [%0];" ::"r"(
@@ -169,7 +154,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const uint32_t rank = pair::cluster_rank();
+  const uint32_t rank = cluster_rank();
   const int cluster = static_cast<int>(blockIdx.x >> 1);
   const int nclusters = static_cast<int>(gridDim.x >> 1);
   const int tiles = (gp.sum_batch ? 1 : gp.batch) * gp.m_blocks * gp.n_blocks;
@@ -198,7 +183,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   }
   // barrier initialisation and the TMEM address are visible to both CTAs from here on
   tc_fence_before();
-  pair::cluster_sync();
+  cluster_sync();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   pdl_wait();
@@ -212,7 +197,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t issued_mask = 0;
       uint32_t last_parity = 0;
       bool ok = true;
-      const uint32_t full0 = pair::map_to_rank(smem_addr(full), 0);
+      const uint32_t full0 = map_to_rank(smem_addr(full), 0);
       for (int t = cluster; ok && t < tiles; t += nclusters) {
         int b, mb, nb;
         pair::decode_tile(t, gp, b, mb, nb);
@@ -339,7 +324,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // ------------------------------------------------------------------ epilogue warps
     const int quarter = warp & 3;   // TMEM lanes 32*quarter .. +31
     const int row = quarter * 32 + lane;
-    const uint32_t acc_empty0 = pair::map_to_rank(smem_addr(acc_empty), 0);
+    const uint32_t acc_empty0 = map_to_rank(smem_addr(acc_empty), 0);
     int it_n = 0;
     for (int t = cluster; t < tiles; t += nclusters) {
       const int acc = it_n & 1;
@@ -369,7 +354,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   tc_fence_before();
   __syncthreads();
-  pair::cluster_sync();
+  cluster_sync();
   tc_fence_after();
   if (warp == 1) {
     __syncwarp();

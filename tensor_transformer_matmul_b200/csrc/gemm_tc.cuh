@@ -238,6 +238,24 @@ struct SegIter {
   }
 };
 
+// TMA coordinates of the i-th k step of segment sg (its k loop starts at kb0 + rot and wraps):
+// the K offset and the A and B batch coordinates (with sum_batch, k steps past the first
+// problem's k-blocks belong to the next problems).
+struct KStep {
+  int k0, za, zb;
+};
+__device__ __forceinline__ KStep k_step(const GemmParams& gp, const Seg& sg, int i) {
+  const int nk = sg.kb1 - sg.kb0;
+  int kb = sg.kb0 + i + sg.rot;
+  if (kb >= sg.kb1) kb -= nk;
+  const int pi = kb / gp.k_blocks;
+  KStep r;
+  r.k0 = (kb - pi * gp.k_blocks) * kBK;
+  r.za = gp.a_batched ? sg.ab + pi : 0;
+  r.zb = gp.b_batched ? sg.b + pi : 0;
+  return r;
+}
+
 // All segments of output tile g, in k order: slot pointer and problem index of each.  Returns the
 // count (0 if more than kMaxGroupSegs, which the host rules out).
 template <int SLOT_FLOATS>
@@ -426,22 +444,15 @@ __global__ void __launch_bounds__(kThreads, 1)
       while (ok && it.next(gp, grid, sg)) {
         const int m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
         const int n0 = sg.nb * Cfg::BN;
-        const int za = gp.a_batched ? sg.ab : 0;
-        const int zb = gp.b_batched ? sg.b : 0;
         const int nk = sg.kb1 - sg.kb0;
         for (int i = 0; i < nk; ++i) {
-          int kb = sg.kb0 + i + sg.rot;
-          if (kb >= sg.kb1) kb -= nk;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
             ok = false;
             break;
           }
           mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
-          // grouped sum: k steps past the first problem's k-blocks belong to the next problems
-          const int pi = kb / gp.k_blocks;
-          const int k0 = (kb - pi * gp.k_blocks) * kBK;
-          const int zai = gp.a_batched ? za + pi : 0;
-          const int zbi = gp.b_batched ? zb + pi : 0;
+          const KStep ks = k_step(gp, sg, i);
+          const int k0 = ks.k0, zai = ks.za, zbi = ks.zb;
           uint8_t* sa = a_smem + stage * Cfg::A_STAGE_BYTES;
           uint8_t* sb = b_smem + stage * Cfg::B_STAGE_BYTES;
           if (Cfg::A_MN) {

@@ -1,6 +1,7 @@
 // Partial-sum reduce and RMSNorm kernels (HBM-bound, vectorised, coalesced).
 #pragma once
 
+#include "sm100.cuh"
 #include "tp_common.cuh"
 
 namespace tp {
@@ -264,6 +265,126 @@ inline void reduce_norm_launch(const void* part, int p, int64_t rows, int64_t d,
                      static_cast<Tout*>(out), static_cast<Tn*>(norm), eps);
 }
 
+// Few rows: "reduce, then normalise" with one cluster of kNormCluster CTAs per row.  CTA c of
+// the cluster takes columns [c*w, (c+1)*w) of the row: it adds the partials in shard order and then
+// the residual (fp32, one rounding), stores y, and sums the squares of its stored values.  The CTAs
+// exchange these sums through distributed shared memory; each adds all of them in rank order, so
+// every CTA gets the same scale, and normalises its own columns from registers.  One kernel
+// replaces the sum over all rows*d elements followed by the row-split RMSNorm.
+constexpr int kNormCluster = 8;
+constexpr int kNormThreads = 128;
+constexpr int kNormVecs = 2;   // 8-element vectors per thread: d <= 8 * 128 * 8 * 2 = 16384
+template <typename Tout, typename Tn>
+__global__ void __launch_bounds__(kNormThreads) reduce_norm_cluster_kernel(
+    const float* __restrict__ part, int p, int64_t n, int64_t d, int w, const Tout* res, Tout* out,
+    Tn* norm, float eps) {
+  pdl_wait();   // programmatic dependent launch: global memory only from here on
+  pdl_trigger();
+  __shared__ float red[kNormThreads / 32];
+  __shared__ float s_part;
+  __shared__ float s_all[kNormCluster];
+  const uint32_t rank = sm100::cluster_rank();
+  const int64_t base = static_cast<int64_t>(blockIdx.y) * d;
+  const int64_t c0 = static_cast<int64_t>(rank) * w;
+  const int64_t c1 = c0 + w < d ? c0 + w : d;
+  float y[kNormVecs][8];
+  float ss = 0.f;
+#pragma unroll
+  for (int v = 0; v < kNormVecs; ++v) {
+    const int64_t j = c0 + 8 * (static_cast<int64_t>(threadIdx.x) + v * kNormThreads);
+    if (j >= c1) continue;
+    float acc[8];
+    for (int g = 0; g < p; g += 8) {   // up to 8 partials in flight, added in order 0..p-1
+      float pv[8][8];
+#pragma unroll
+      for (int q = 0; q < 8; ++q)
+        if (g + q < p) Vec8<float>::load(part + static_cast<int64_t>(g + q) * n + base + j, pv[q]);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) {
+        if (g + q >= p) break;
+        if (g + q == 0) {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] = pv[0][e];
+        } else {
+#pragma unroll
+          for (int e = 0; e < 8; ++e) acc[e] += pv[q][e];
+        }
+      }
+    }
+    if (res) {
+      float r[8];
+      Vec8<Tout>::load(res + base + j, r);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] = r[e] + acc[e];
+    }
+    Vec8<Tout>::store(out + base + j, acc);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {   // the stored, rounded value
+      y[v][e] = to_f(from_f<Tout>(acc[e]));
+      ss = fmaf(y[v][e], y[v][e], ss);
+    }
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) ss += __shfl_xor_sync(0xffffffffu, ss, o);
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = ss;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    float t = 0.f;
+#pragma unroll
+    for (int i = 0; i < kNormThreads / 32; ++i) t += red[i];
+    s_part = t;
+  }
+  sm100::cluster_sync();   // every CTA's s_part is written and visible to the cluster
+  if (threadIdx.x < kNormCluster)
+    s_all[threadIdx.x] =
+        sm100::ld_shared_cluster_f32(sm100::map_to_rank(sm100::smem_addr(&s_part), threadIdx.x));
+  sm100::cluster_sync();   // every peer has read this CTA's s_part (it may exit after this)
+  float tot = 0.f;
+#pragma unroll
+  for (int i = 0; i < kNormCluster; ++i) tot += s_all[i];
+  const float scale = rsqrtf(tot / static_cast<float>(d) + eps);
+#pragma unroll
+  for (int v = 0; v < kNormVecs; ++v) {
+    const int64_t j = c0 + 8 * (static_cast<int64_t>(threadIdx.x) + v * kNormThreads);
+    if (j >= c1) continue;
+#pragma unroll
+    for (int e = 0; e < 8; ++e) y[v][e] *= scale;
+    Vec8<Tn>::store(norm + base + j, y[v]);
+  }
+}
+
+inline bool reduce_norm_cluster_ok(const void* part, int64_t rows, int64_t d, const void* res,
+                                   const void* out, const void* norm) {
+  return rows > 0 && rows < num_sms() && rows <= 65535 && d % 8 == 0 &&
+         d <= static_cast<int64_t>(kNormCluster) * kNormThreads * 8 * kNormVecs &&
+         ((reinterpret_cast<uintptr_t>(part) | reinterpret_cast<uintptr_t>(res) |
+           reinterpret_cast<uintptr_t>(out) | reinterpret_cast<uintptr_t>(norm)) & 15) == 0;
+}
+
+template <typename Tout, typename Tn>
+inline cudaError_t reduce_norm_cluster_launch(const float* part, int p, int64_t rows, int64_t d,
+                                              const void* res, void* out, void* norm, float eps,
+                                              cudaStream_t s) {
+  const int w = static_cast<int>(round_up(ceil_div(d, kNormCluster), 8));
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(kNormCluster, static_cast<unsigned>(rows));
+  cfg.blockDim = dim3(kNormThreads);
+  cfg.dynamicSmemBytes = 0;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = kNormCluster;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 2;
+  return cudaLaunchKernelEx(&cfg, reduce_norm_cluster_kernel<Tout, Tn>, part, p, rows * d, d, w,
+                            static_cast<const Tout*>(res), static_cast<Tout*>(out),
+                            static_cast<Tn*>(norm), eps);
+}
+
 inline tp_status rmsnorm(const void* x, int in_dtype, int64_t rows, int64_t d, float eps,
                          void* out, int out_dtype, cudaStream_t s);
 inline bool rmsnorm_split_ok(const void* x, int64_t rows, int64_t d, const void* out);
@@ -274,10 +395,25 @@ inline tp_status reduce_norm(const float* part, int p, int64_t rows, int64_t d, 
                              cudaStream_t s) {
   if (rows == 0) return TP_OK;
   if (rows > INT32_MAX) return set_error(TP_ERR_UNSUPPORTED, "too many rows");
+  if (reduce_norm_cluster_ok(part, rows, d, res, out, norm)) {
+    // few rows: one row per block would leave most SMs idle, so each row is spread over a
+    // cluster of CTAs that share the row's sum of squares
+    ProfScope prof(s, "reduce_partials");
+    const bool ob = out_dtype == TP_BF16, nb = norm_dtype == TP_BF16;
+    cudaError_t e;
+    if (ob && nb) e = reduce_norm_cluster_launch<__nv_bfloat16, __nv_bfloat16>(part, p, rows, d, res, out, norm, eps, s);
+    else if (ob) e = reduce_norm_cluster_launch<__nv_bfloat16, float>(part, p, rows, d, res, out, norm, eps, s);
+    else if (nb) e = reduce_norm_cluster_launch<float, __nv_bfloat16>(part, p, rows, d, res, out, norm, eps, s);
+    else e = reduce_norm_cluster_launch<float, float>(part, p, rows, d, res, out, norm, eps, s);
+    if (e != cudaSuccess)
+      return set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
+    count_launch();
+    return TP_OK;
+  }
   if (rmsnorm_split_ok(out, rows, d, norm)) {
-    // few rows: one row per block would leave most SMs idle, so the sum runs as the plain
-    // vectorised reduce over all rows*d elements and the norm as the row-split kernel (both read
-    // the stored, rounded y, as the one-kernel path does)
+    // few rows with a shape the cluster kernel does not take: the plain vectorised reduce over
+    // all rows*d elements, then the row-split norm (both read the stored, rounded y, as the
+    // one-kernel path does)
     tp_status st = launch(part, TP_F32, p, rows * d, res, out, out_dtype, s);
     if (st != TP_OK) return st;
     return rmsnorm(out, out_dtype, rows, d, eps, norm, norm_dtype, s);

@@ -80,6 +80,17 @@ static __global__ void zero_words_kernel(uint32_t* p, int64_t n) {
        i += static_cast<int64_t>(gridDim.x) * blockDim.x)
     p[i] = 0u;
 }
+// The same for two arrays in one launch (a GEMM's counters and those of the kernel after it).
+static __global__ void zero_words2_kernel(uint32_t* p, int64_t n, uint32_t* q, int64_t m) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; i < n + m;
+       i += stride) {
+    if (i < n) p[i] = 0u;
+    else q[i - n] = 0u;
+  }
+}
 
 
 // Brackets one kernel launch with CUDA events when tp_profile_enable(1) is in effect.

@@ -62,3 +62,39 @@ def test_empty(lib):
     out = torch.empty(0, device=dev())
     lib.tp_reduce_partials(torch.empty(0, device=dev()), 4, 0, out)
     torch.cuda.synchronize()
+
+
+@pytest.mark.parametrize("T,d,p", [
+    (1, 8192, 8),      # a decode row of the workload: one cluster, one vector per thread
+    (3, 776, 12),      # ragged column split, 12 partials (two groups of loads)
+    (147, 512, 2),     # the most rows that still take the few-rows path (fewer than the SMs)
+    (2, 16384, 4),     # two vectors per thread: the widest row of the cluster kernel
+    (2, 16392, 4),     # one vector too wide: the two-kernel path
+    (1, 8, 1),         # one shard, one vector: seven of the eight CTAs hold no columns
+])
+def test_reduce_norm_few_rows(lib, T, d, p):
+    # reduce + RMSNorm of fewer rows than SMs (the decode reductions): y must equal, bit for bit,
+    # the plain reduce of the same partials (the same in-order sum and rounding), and y_norm must
+    # be the RMSNorm of the stored y rows
+    from oracle import decode as odec
+    from oracle import mlp as omlp
+    from tensor_transformer_matmul_b200 import inputs
+    from tests.helpers import Mlp, rel_l2_rows
+    F = 128 * p
+    inp = inputs.mlp_inputs(T, d, F, "gelu", "bf16", seed=60 + T, w_std=0.05)
+    m = Mlp(lib, inp, p, "gelu", "bf16", 0)
+    res = inputs.normal((T, d), 1.0, 60, 99, "bf16", "cpu").to(dev())
+    x = inp["x"].to(dev())
+    y_plain = torch.empty(T, d, dtype=torch.bfloat16, device=dev())
+    lib.tp_mlp_fwd(m.desc, x, m.w1p, m.w2p, y_plain, residual=res, workspace=m.ws_f)
+    y = torch.empty_like(y_plain)
+    yn = torch.empty_like(y_plain)
+    lib.tp_reset_reduction_count()
+    lib.tp_mlp_fwd(m.desc, x, m.w1p, m.w2p, y, residual=res, workspace=m.ws_f, y_norm=yn)
+    torch.cuda.synchronize()
+    assert lib.tp_reduction_count() == 1
+    assert torch.equal(y, y_plain)
+    ref_norm = odec.rmsnorm(f64(y))
+    assert rel_l2(f64(yn), ref_norm) <= 4e-3 and rel_l2_rows(f64(yn), ref_norm) <= 4e-3
+    ref = omlp.mlp_forward(f64(inp["x"]), f64(inp["w1"]), f64(inp["w2"]), "gelu") + f64(res)
+    assert rel_l2(f64(y), ref) <= TOL["bf16"]
