@@ -58,10 +58,10 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
   const bool fused = L.reduce_mode == TP_REDUCE_FUSED;
   size_t a = 0, b = 0;
   if (L.tokens <= kSwapMaxT) {
-    if (decode_stream_k(qkv_tiles(L))) a = by_tokens(L.tokens, [&](auto t) {
+    if (decode_stream_k(qkv_tiles(L), L.tokens, ceil_div(L.h, 64))) a = by_tokens(L.tokens, [&](auto t) {
       return tc::plan_stream_k<typename decltype(t)::type>(rows, L.tokens, L.h, 1, false, num_sms()).bytes();
     });
-    if (decode_stream_k(out_tiles(L)) || fused) b = by_tokens(L.tokens, [&](auto t) {
+    if (decode_stream_k(out_tiles(L), L.tokens, ceil_div(static_cast<int64_t>(L.qh) * L.hd, 64)) || fused) b = by_tokens(L.tokens, [&](auto t) {
       return tc::plan_stream_k<typename decltype(t)::type>(L.h, L.tokens, K, L.p, fused, num_sms()).bytes();
     });
   }
@@ -937,12 +937,12 @@ inline tp_status qkv_proj(const AttnLayout& L, const void* x, const void* wqkv, 
     ep.swap = 1;
     const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
     tc::GemmOpts opt;
-    opt.sk = decode_stream_k(qkv_tiles(L)) ? &sk : nullptr;
+    opt.sk = decode_stream_k(qkv_tiles(L), L.tokens, ceil_div(L.h, 64)) ? &sk : nullptr;
     opt.rotate_k = true;
     opt.zero_also = reinterpret_cast<uint32_t*>(zero_also);
     opt.zero_also_words = zero_also ? zero_also_words : 0;
     return by_tokens(L.tokens, [&](auto t) {
-      return tc::run_gemm<typename decltype(t)::type, tc::EpiHidden>(wo, xo, rows, L.tokens, L.h, 1,
+      return tc::run_gemm<typename decltype(t)::type, tc::EpiHiddenSwap>(wo, xo, rows, L.tokens, L.h, 1,
                                                                      ep, s, "attn_qkv_gemm", opt);
     });
   }
@@ -997,7 +997,7 @@ inline tp_status out_proj(const AttnLayout& L, const void* o, const void* wo_p, 
     ep.swap = 1;
     const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
     tc::GemmOpts opt;
-    opt.sk = decode_stream_k(out_tiles(L)) ? &sk : nullptr;
+    opt.sk = decode_stream_k(out_tiles(L), L.tokens, ceil_div(static_cast<int64_t>(L.qh) * L.hd, 64)) ? &sk : nullptr;
     opt.rotate_k = true;
     return by_tokens(L.tokens, [&](auto t) {
       return tc::run_gemm<typename decltype(t)::type, tc::EpiStoreF32>(wo, ao, L.h, L.tokens, K, L.p,

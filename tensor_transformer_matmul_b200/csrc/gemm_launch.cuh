@@ -48,8 +48,9 @@ struct SkPlan {
   int grid = 0;             // CTAs (<= SMs, <= k-blocks)
   int slots_per_cta = 0;    // partial-tile slots per CTA
   int max_group_segs = 0;   // most segments any output tile is cut into
-  int64_t units = 0;        // k-blocks over all output tiles
+  int64_t units = 0;        // k-blocks over the split tiles
   int64_t groups = 0;       // output tiles
+  int64_t sk_groups = 0;    // the first sk_groups tiles are split; the rest run whole
   size_t counter_bytes = 0; // arrival counters (256-aligned)
   size_t slot_bytes = 0;    // partial slots
   size_t bytes() const { return counter_bytes + slot_bytes; }
@@ -62,11 +63,20 @@ SkPlan plan_stream_k(int64_t M, int64_t N, int64_t K, int64_t batch, bool sum_ba
   if (M <= 0 || N <= 0 || K <= 0 || batch <= 0) return pl;
   pl.groups = sum_batch ? mb * nb : batch * mb * nb;
   const int64_t U = sum_batch ? batch * kb : kb;
-  pl.units = pl.groups * U;
-  std::vector<int> per_group(static_cast<size_t>(pl.groups), 0);
+  // With at least a wave of tiles, the whole waves run as whole tiles after the split ranges and
+  // only the remainder is split (plus one wave when the remainder alone would be cut into too
+  // many pieces).  The fused shard sum splits every tile (each shard's k-range is a segment).
+  pl.sk_groups = pl.groups;
+  if (!sum_batch && pl.groups > sms) {
+    const int64_t r = pl.groups % sms;
+    pl.sk_groups = r == 0 ? 0 : (r * 14 >= sms) ? r : r + sms;
+  }
+  pl.units = pl.sk_groups * U;
+  std::vector<int> per_group(static_cast<size_t>(pl.sk_groups), 0);
   // fewer, longer ranges when a tile would otherwise be cut into too many segments (tiny
-  // problems spread over many SMs)
-  for (int grid = static_cast<int>(std::min<int64_t>(sms, pl.units)); grid >= 1; grid = grid / 2) {
+  // problems spread over many SMs); with whole tiles after the split ones the grid stays at sms
+  const int grid0 = pl.sk_groups < pl.groups ? sms : static_cast<int>(std::min<int64_t>(sms, pl.units));
+  for (int grid = grid0; grid >= 1; grid = grid / 2) {
     std::fill(per_group.begin(), per_group.end(), 0);
     int spc = 0;
     for (int c = 0; c < grid; ++c) {
@@ -88,7 +98,7 @@ SkPlan plan_stream_k(int64_t M, int64_t N, int64_t K, int64_t batch, bool sum_ba
     pl.grid = grid;
     pl.slots_per_cta = spc;
     pl.max_group_segs = mx;
-    if (mx <= kMaxGroupSegs || grid == 1) break;
+    if (mx <= kMaxGroupSegs || grid == 1 || pl.sk_groups < pl.groups) break;
   }
   pl.counter_bytes = align256(static_cast<size_t>(pl.groups) * sizeof(int32_t));
   pl.slot_bytes = static_cast<size_t>(pl.grid) * pl.slots_per_cta * Cfg::SLOT_FLOATS * sizeof(float);
@@ -157,6 +167,7 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   gp.stream_k = 0;
   gp.sum_batch = 0;
   gp.units = 0;
+  gp.sk_groups = 0;
   gp.slots_per_cta = 0;
   gp.slots = nullptr;
   gp.counters = nullptr;
@@ -181,6 +192,7 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
     gp.stream_k = 1;
     gp.sum_batch = sk->sum_batch ? 1 : 0;
     gp.units = pl.units;
+    gp.sk_groups = static_cast<int32_t>(pl.sk_groups);
     gp.slots_per_cta = pl.slots_per_cta;
     gp.counters = static_cast<int32_t*>(sk->ws);
     gp.slots = reinterpret_cast<float*>(static_cast<uint8_t*>(sk->ws) + pl.counter_bytes);

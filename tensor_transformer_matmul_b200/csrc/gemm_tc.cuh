@@ -10,11 +10,14 @@
 //
 // Work is cut into segments, each one accumulator's worth of k-blocks.  Two schedules:
 //   * tiles: segment = one whole output tile (all of K); tile = blockIdx.x + i * gridDim.x.
-//   * stream-K: the k-blocks of all tiles, in order, are split into gridDim.x equal contiguous
-//     ranges, one per CTA, so every SM streams the same number of k-blocks.  A tile whose
-//     k-blocks fall in several segments ("split") is finished by whichever CTA arrives last:
-//     each writes its fp32 partial to a slot, and the last one adds the slots in k order and
-//     applies the epilogue.  No CTA ever waits for another.
+//   * stream-K: the k-blocks of the first sk_groups tiles, in order, are split into gridDim.x
+//     equal contiguous ranges, one per CTA.  A tile whose k-blocks fall in several segments
+//     ("split") is finished by whichever CTA arrives last: each writes its fp32 partial to a
+//     slot, and the last one adds the slots in k order and applies the epilogue.  No CTA ever
+//     waits for another.  The remaining tiles (a whole number of waves) follow as whole tiles,
+//     tile sk_groups + c + i * gridDim.x on CTA c, after the CTA's split range: so every SM
+//     streams the same number of k-blocks, and the fix-ups of the split tiles overlap the
+//     streaming of the whole ones instead of trailing the kernel.
 //   With sum_batch, the problem index (the shard) is part of the k space of an output tile:
 //   each shard's k-range is its own segment, and the finishing CTA adds the shards' partial
 //   tiles in shard order 0..p-1 -- the partial-sum reduce fused into the GEMM.
@@ -32,6 +35,8 @@
 
 #include <cuda.h>
 #include <stdint.h>
+
+#include <type_traits>
 
 #include "sm100.cuh"
 #include "tp_common.cuh"
@@ -86,7 +91,8 @@ struct GemmParams {
   // stream-K schedule
   int32_t stream_k;       // 0: whole tiles; 1: equal contiguous k-block ranges per CTA
   int32_t sum_batch;      // stream-K: the problems are summed into one output (fused reduce)
-  int64_t units;          // total k-blocks over all output tiles
+  int64_t units;          // stream-K: k-blocks over the split tiles (the first sk_groups tiles)
+  int32_t sk_groups;      // stream-K: tiles cut into ranges; the tiles after them run whole
   int32_t slots_per_cta;  // partial-tile slots reserved per CTA
   float* slots;           // [gridDim.x][slots_per_cta][SLOT_FLOATS]
   int32_t* counters;      // [output tiles] arrivals of split tiles (zero before the launch)
@@ -160,9 +166,11 @@ __device__ __forceinline__ int cta_of(int64_t u, const GemmParams& gp, int grid)
 // Segment iterator over one CTA's work (both schedules); all roles walk the same sequence.
 struct SegIter {
   int64_t u, end;   // stream-K: unit cursor and end; tiles: tile cursor and count
-  int local;
+  int local;        // segments so far (stream-K: split segments only; the slot index)
+  int dp;           // stream-K: the CTA's next whole tile (after its split range)
   __device__ __forceinline__ void init(const GemmParams& gp, int cta, int grid) {
     local = 0;
+    dp = gp.sk_groups + cta;
     if (gp.stream_k) {
       u = cta_start(cta, gp, grid);
       end = cta_start(cta + 1, gp, grid);
@@ -176,6 +184,23 @@ struct SegIter {
     }
   }
   __device__ __forceinline__ bool next(const GemmParams& gp, int grid, Seg& s) {
+    if (gp.stream_k && u >= end) {
+      // the whole tiles after the split range (never with sum_batch: the host keeps them out)
+      if (dp >= num_groups(gp)) return false;
+      s.g = dp;
+      dp += grid;
+      const int per = gp.m_blocks * gp.n_blocks;
+      s.b = s.g / per;
+      decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
+      s.ab = s.b;
+      s.row0 = 0;
+      s.row_end = 0x7fffffff;
+      s.kb0 = 0;
+      s.kb1 = gp.k_blocks;
+      s.local = -1;   // whole: no slot
+      s.rot = gp.rotate_k ? static_cast<int>((static_cast<int64_t>(s.g) * 37) % gp.k_blocks) : 0;
+      return true;
+    }
     if (u >= end) return false;
     if (!gp.stream_k) {
       s.g = static_cast<int>(u);
@@ -271,7 +296,7 @@ __device__ __forceinline__ int group_segments(const GemmParams& gp, int grid, in
     it.init(gp, c, grid);
     Seg s;
     while (it.next(gp, grid, s)) {
-      if (s.g < g) continue;
+      if (s.local < 0 || s.g < g) continue;   // a whole tile, or a split tile before g
       if (s.g > g) break;
       if (n == kMaxGroupSegs) return 0;
       ptr[n] = gp.slots + (static_cast<int64_t>(c) * gp.slots_per_cta + s.local) * SLOT_FLOATS;
@@ -333,8 +358,10 @@ struct TmemSrc {
 };
 
 // From the partial slots of a split tile: the sum over its segments, in k order; with several
-// problems (shards), each shard's segments are added first, then the shards in order.
-template <int ACC_COLS>
+// problems (shards), each shard's segments are added first, then the shards in order.  For
+// 16-column pieces the loads of up to G16 segments are issued before their adds (one L2 round
+// trip per G16 segments, not per segment); the additions keep the order above.
+template <int ACC_COLS, int G16>
 struct FixupSrc {
   const float* const* ptr;
   const int* bs;
@@ -342,6 +369,7 @@ struct FixupSrc {
   int row;
   template <int W>
   __device__ __forceinline__ void load(int col, float (&v)[W]) const {
+    constexpr int G = W <= 16 ? G16 : 1;
     float tot[W], cur[W];
 #pragma unroll
     for (int e = 0; e < W; ++e) {
@@ -349,25 +377,35 @@ struct FixupSrc {
       cur[e] = 0.f;
     }
     int cur_b = -1;
-    for (int s = 0; s < n; ++s) {
-      const float4* p4 = reinterpret_cast<const float4*>(ptr[s] + row * ACC_COLS + col);
-      float x[W];
+#pragma unroll 1
+    for (int s0 = 0; s0 < n; s0 += G) {
+      float x[G][W];
 #pragma unroll
-      for (int q = 0; q < W / 4; ++q) {
-        const float4 f = __ldcg(p4 + q);
-        x[4 * q] = f.x; x[4 * q + 1] = f.y; x[4 * q + 2] = f.z; x[4 * q + 3] = f.w;
-      }
-      if (bs[s] != cur_b) {
-        if (cur_b >= 0) {
+      for (int j = 0; j < G; ++j) {
+        if (s0 + j < n) {
+          const float4* p4 = reinterpret_cast<const float4*>(ptr[s0 + j] + row * ACC_COLS + col);
 #pragma unroll
-          for (int e = 0; e < W; ++e) tot[e] += cur[e];
+          for (int q = 0; q < W / 4; ++q) {
+            const float4 f = __ldcg(p4 + q);
+            x[j][4 * q] = f.x; x[j][4 * q + 1] = f.y; x[j][4 * q + 2] = f.z; x[j][4 * q + 3] = f.w;
+          }
         }
+      }
 #pragma unroll
-        for (int e = 0; e < W; ++e) cur[e] = x[e];
-        cur_b = bs[s];
-      } else {
+      for (int j = 0; j < G; ++j) {
+        if (s0 + j >= n) break;
+        if (bs[s0 + j] != cur_b) {
+          if (cur_b >= 0) {
 #pragma unroll
-        for (int e = 0; e < W; ++e) cur[e] += x[e];
+            for (int e = 0; e < W; ++e) tot[e] += cur[e];
+          }
+#pragma unroll
+          for (int e = 0; e < W; ++e) cur[e] = x[j][e];
+          cur_b = bs[s0 + j];
+        } else {
+#pragma unroll
+          for (int e = 0; e < W; ++e) cur[e] += x[j][e];
+        }
       }
     }
 #pragma unroll
@@ -375,6 +413,17 @@ struct FixupSrc {
   }
   __device__ __forceinline__ void load32(int col, float (&v)[32]) const { load<32>(col, v); }
   __device__ __forceinline__ void load16(int col, float (&v)[16]) const { load<16>(col, v); }
+};
+
+// Segments whose loads a fix-up issues together (FixupSrc): 3 unless the epilogue asks for fewer
+// (a kernel that also carries another epilogue path with high register demand).
+template <class E, class = void>
+struct FixupGroup {
+  static constexpr int value = 3;
+};
+template <class E>
+struct FixupGroup<E, std::void_t<decltype(E::kFixupGroup)>> {
+  static constexpr int value = E::kFixupGroup;
 };
 
 template <class Cfg, class Epi>
@@ -577,7 +626,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctx.row_end = sg.row_end;
       // the tile is whole when all its k-blocks lie in this CTA's range (then it is one segment)
       const int64_t g0 = static_cast<int64_t>(sg.g) * U;
-      const bool whole = !gp.stream_k ||
+      const bool whole = !gp.stream_k || sg.g >= gp.sk_groups ||
                          (g0 >= my_start && g0 + U <= my_end && (!gp.sum_batch || gp.batch == 1));
       if (whole) {
         Epi::template run<Cfg>(ep, gp, ctx, tsrc);
@@ -618,7 +667,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       epi_bar();   // every thread has read the flag before it can be rewritten
       if (last) {
         __threadfence();
-        FixupSrc<Cfg::ACC_COLS> fsrc{ptrs, bs, nseg, row};
+        FixupSrc<Cfg::ACC_COLS, FixupGroup<Epi>::value> fsrc{ptrs, bs, nseg, row};
         Epi::template run<Cfg>(ep, gp, ctx, fsrc);
       }
     }
@@ -670,22 +719,28 @@ __device__ __forceinline__ float fast_sigmoid(float z) { return 1.0f / (1.0f + _
 // gate in columns 0..127 and up in 128..255; swapped A_SUB = 2 with gate in sub-tile 0 and up in
 // sub-tile 1.  h column of feature (block j, offset o) is j*128 + o in the padded layout.
 // ---------------------------------------------------------------------------------------------
-struct EpiHidden {
-  struct Params {
-    __nv_bfloat16* h;   // [tokens][ld_h]
-    __nv_bfloat16* z;   // [tokens][ld_z] or null
-    int64_t ld_h, ld_z;
-    int32_t tokens;     // valid tokens
-    int32_t rows;       // valid packed rows (columns of z)
-    int32_t act;        // tp_act
-    int32_t swap;       // 1: A = weights, B = tokens
-  };
+struct EpiHiddenParams {
+  __nv_bfloat16* h;   // [tokens][ld_h]
+  __nv_bfloat16* z;   // [tokens][ld_z] or null
+  int64_t ld_h, ld_z;
+  int32_t tokens;     // valid tokens
+  int32_t rows;       // valid packed rows (columns of z)
+  int32_t act;        // tp_act
+  int32_t swap;       // 1: A = weights, B = tokens
+};
+
+// MODE 0: p.swap chooses the orientation at run time; MODE 1: swapped only (the decode GEMMs),
+// so their kernels carry neither the other path's code nor its register demand.
+template <int MODE>
+struct EpiHiddenT {
+  using Params = EpiHiddenParams;
+  static constexpr int kFixupGroup = MODE == 1 ? 3 : 1;
 
   template <class Cfg, class Src>
   __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
                                              const Src& src) {
     const bool swiglu = p.act == TP_ACT_SWIGLU;
-    if (!p.swap) {
+    if (MODE == 0 && !p.swap) {
       const int t = c.m0 + c.row;
       const bool live = t < p.tokens && t < c.row_end;
       if (swiglu) {
@@ -774,6 +829,8 @@ struct EpiHidden {
     }
   }
 };
+using EpiHidden = EpiHiddenT<0>;
+using EpiHiddenSwap = EpiHiddenT<1>;
 
 // ---------------------------------------------------------------------------------------------
 // fp32 store of the accumulator: out[b][i][j] = D (or D^T when swapped), with i < rows_valid and

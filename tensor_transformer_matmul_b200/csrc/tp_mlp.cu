@@ -67,7 +67,7 @@ int64_t up_tiles(const MlpLayout& L) {
 int64_t down_tiles(const MlpLayout& L) { return L.p * ceil_div(L.d, 128); }
 
 size_t up_sk_bytes(const MlpLayout& L) {
-  if (L.T > kSwapMaxT || !decode_stream_k(up_tiles(L))) return 0;
+  if (L.T > kSwapMaxT || !decode_stream_k(up_tiles(L), L.T, ceil_div(L.d, 64))) return 0;
   const int64_t rows = L.p * L.R;
   auto f = [&](auto tag) {
     return tc::plan_stream_k<typename decltype(tag)::type>(rows, L.T, L.d, 1, false, num_sms()).bytes();
@@ -77,7 +77,7 @@ size_t up_sk_bytes(const MlpLayout& L) {
 size_t down_sk_bytes(const MlpLayout& L) {
   const bool fused = L.reduce_mode == TP_REDUCE_FUSED;
   if (L.T > kSwapMaxT) return 0;   // prefill: whole pair tiles, the fused sum in the accumulator
-  if (!fused && !decode_stream_k(down_tiles(L))) return 0;
+  if (!fused && !decode_stream_k(down_tiles(L), L.T, ceil_div(L.Fsp, 64))) return 0;
   return by_tokens<1>(L.T, [&](auto tag) {
     return tc::plan_stream_k<typename decltype(tag)::type>(L.d, L.T, L.Fsp, L.p, fused, num_sms()).bytes();
   });
@@ -163,10 +163,10 @@ tp_status tc_up(const MlpLayout& L, const void* x, const void* w1p, void* h, voi
     ep.swap = 1;
     const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
     tc::GemmOpts opt;
-    opt.sk = decode_stream_k(up_tiles(L)) ? &sk : nullptr;
+    opt.sk = decode_stream_k(up_tiles(L), L.T, ceil_div(L.d, 64)) ? &sk : nullptr;
     opt.rotate_k = true;
     auto f = [&](auto tag) {
-      return tc::run_gemm<typename decltype(tag)::type, tc::EpiHidden>(wo, xo, rows, L.T, L.d, 1, ep,
+      return tc::run_gemm<typename decltype(tag)::type, tc::EpiHiddenSwap>(wo, xo, rows, L.T, L.d, 1, ep,
                                                                        s, "mlp_up_gemm", opt);
     };
     return L.act == TP_ACT_SWIGLU ? by_tokens<2>(L.T, f) : by_tokens<1>(L.T, f);
@@ -216,7 +216,7 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
     ep.swap = 1;
     const tc::StreamKArgs sk{false, sk_ws, sk_bytes};
     tc::GemmOpts opt;
-    opt.sk = decode_stream_k(down_tiles(L)) ? &sk : nullptr;
+    opt.sk = decode_stream_k(down_tiles(L), L.T, ceil_div(L.Fsp, 64)) ? &sk : nullptr;
     opt.rotate_k = true;
     return by_tokens<1>(L.T, [&](auto tag) {
       return tc::run_gemm<typename decltype(tag)::type, tc::EpiStoreF32>(

@@ -236,6 +236,26 @@ def test_stream_k_splits_fused_vs_separate(lib, T, d, F, p):
     assert rel_l2(f64(outs[0]), f64(outs[1])) <= 1e-2
 
 
+@pytest.mark.parametrize("T,d,F,p,act", [
+    (2, 5504, 14336, 7, "gelu"),     # down: 7 x 43 = 301 tiles of 32 k-blocks = 2 waves + 5: the
+                                     # 5 are split together with one more wave, then whole tiles
+    (3, 2048, 19072, 1, "swiglu"),   # up: 149 tiles of 256 packed rows, one more than the SMs
+    (5, 4096, 22400, 5, "swiglu"),   # up: 175 tiles (27 split, 148 whole); down: 160 (12, 148)
+])
+def test_decode_split_then_whole_tiles(lib, T, d, F, p, act):
+    # weight-streaming GEMMs with more tiles than SMs: the remainder after whole waves is split
+    # into equal k-ranges (fixed up by the last CTA to arrive), then every CTA runs whole tiles;
+    # checked against the oracle row by row, and two runs give the same bits
+    inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=11 + T, w_std=0.03)
+    m = Mlp(lib, inp, p, act, "bf16", 0)
+    a = m.forward(inp["x"], save=False).clone()
+    b = m.forward(inp["x"], save=False)
+    torch.cuda.synchronize()
+    assert torch.equal(a, b)
+    ref = _oracle_fwd(inp, act)
+    assert rel_l2(f64(a), ref) <= TOL["bf16"] and rel_l2_rows(f64(a), ref) <= TOL["bf16"]
+
+
 def test_fused_reduce_deterministic(lib):
     inp = inputs.mlp_inputs(64, 1024, 4096, "swiglu", "bf16", seed=9, w_std=0.02)
     m = Mlp(lib, inp, 8, "swiglu", "bf16", 1)
