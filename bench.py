@@ -227,6 +227,7 @@ def decode_mlp_bytes():
     part = c["p"] * c["T"] * c["d"] * 4
     y = c["T"] * c["d"] * 2
     return {"mlp_up_gemm": w1 + x + h, "mlp_down_gemm": w2 + h + part,
+            "mlp_decode_gemm": w1 + x + h + w2 + h + part,   # both projections in one launch
             "mlp_down_gemm_fused": w2 + h + y,
             "reduce_partials": part + y, "step": w1 + w2 + x + y, "weights": w1 + w2, "Fs": Fs}
 
@@ -786,6 +787,8 @@ def extra_stack(tp, torch, stream, peaks, steps, reduce_mode="separate"):
     qkv = (c["n_q"] + 2 * c["n_kv"]) * c["hd"]
     work = {"mlp_up_gemm": tp.tp_mlp_w1_packed_bytes(st.mdesc) + 2 * h + 2 * c["p"] * 2 * Fsp,
             "mlp_down_gemm": tp.tp_mlp_w2_packed_bytes(st.mdesc) + 2 * c["p"] * Fsp + 4 * c["p"] * h,
+            "mlp_decode_gemm": tp.tp_mlp_w1_packed_bytes(st.mdesc) + tp.tp_mlp_w2_packed_bytes(st.mdesc)
+            + 2 * h + 2 * 2 * c["p"] * Fsp + 4 * c["p"] * h,
             "attn_qkv_gemm": tp.tp_attn_wqkv_packed_bytes(st.adesc) + 2 * h + 2 * qkv,
             "attn_out_gemm": tp.tp_attn_wo_packed_bytes(st.adesc) + 2 * c["n_q"] * c["hd"]
             + 4 * c["p"] * h,

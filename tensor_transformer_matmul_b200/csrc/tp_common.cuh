@@ -138,6 +138,7 @@ enum : uint32_t {
   DEVERR_WAIT_ACC_FULL = 1u << 2,  // epilogue waited too long for an accumulator
   DEVERR_WAIT_ACC_EMPTY = 1u << 3, // MMA warp waited too long for the epilogue
   DEVERR_WAIT_DRAIN = 1u << 4,     // abort path: in-flight copies did not land in time
+  DEVERR_WAIT_FLAG = 1u << 5,      // a tile waited too long for another CTA's tiles (decode MLP)
 };
 
 // Device address of the error word of the current device (owned by tp_abi.cu).  Kernels get

@@ -14,6 +14,7 @@
 
 #include "gemm_launch.cuh"
 #include "gemm_pair.cuh"
+#include "mlp_decode.cuh"
 #include "moe.cuh"
 #include "pack.cuh"
 #include "reduce.cuh"
@@ -65,6 +66,16 @@ int64_t up_tiles(const MlpLayout& L) {
   return ceil_div(L.p * L.R, L.act == TP_ACT_SWIGLU ? 256 : 128);
 }
 int64_t down_tiles(const MlpLayout& L) { return L.p * ceil_div(L.d, 128); }
+
+// The one-launch decode MLP (csrc/mlp_decode.cuh): tensor-core path, 1..64 tokens, separate
+// shard reduce.  Its counters (next work item, finished up tiles per shard) sit in the stream-K
+// region, which the separate up and down GEMMs would otherwise use.
+bool fused_decode_ok(const MlpLayout& L) {
+  return L.tc && L.T >= 1 && L.T <= 64 && L.reduce_mode == TP_REDUCE_SEPARATE;
+}
+size_t fused_decode_bytes(const MlpLayout& L) {
+  return fused_decode_ok(L) ? align256(static_cast<size_t>(1 + L.p) * sizeof(int32_t)) : 0;
+}
 
 size_t up_sk_bytes(const MlpLayout& L) {
   if (L.T > kSwapMaxT || !decode_stream_k(up_tiles(L), L.T, ceil_div(L.d, 64))) return 0;
@@ -120,7 +131,9 @@ tp_status layout_of(const tp_mlp_desc* desc, MlpLayout* L) {
     L->fz_off = 0;
     L->fh_off = 0;
     L->fsk_off = align256(hb);
-    const size_t sk = L->T > 0 ? std::max(up_sk_bytes(*L), down_sk_bytes(*L)) : 0;
+    const size_t sk = L->T > 0 ? std::max({up_sk_bytes(*L), down_sk_bytes(*L),
+                                           fused_decode_bytes(*L)})
+                               : 0;
     L->fpart_off = L->fsk_off + align256(sk);
     const size_t pb = L->reduce_mode == TP_REDUCE_FUSED ? 0 : partb;
     L->fwd_ws = L->fpart_off + align256(pb);
@@ -226,6 +239,79 @@ tp_status tc_down(const MlpLayout& L, const void* h, const void* w2p, float* par
   ep.swap = 0;
   return tc::run_gemm_pair<PP<false, false>, tc::EpiStoreF32>(ho, wo, L.T, L.d, L.Fsp, L.p, ep, s,
                                                               "mlp_down_gemm");
+}
+
+// Up and down projections of a decode call as one persistent launch (mlp_decode.cuh): h (and z
+// when saved) as tc_up writes them, fp32 partials [p][T][d] as tc_down writes them.
+template <int BN, int UP_SUB>
+tp_status run_mlp_decode(const MlpLayout& L, const void* x, const void* w1p, const void* w2p,
+                         void* h, void* z, float* part, void* counters, cudaStream_t s) {
+  using C = mlpdec::Cfg<BN, UP_SUB>;
+  const int64_t rows = L.p * L.R;
+  const uint64_t d = static_cast<uint64_t>(L.d), Fsp = static_cast<uint64_t>(L.Fsp);
+  const uint64_t P = static_cast<uint64_t>(L.p), T = static_cast<uint64_t>(L.T);
+  CUtensorMap m_w1, m_x, m_w2, m_h;
+  tp_status st;
+  // packed W1 [p*R][d] (K-major), one box = the tile's 128 * UP_SUB rows
+  if ((st = encode_tmap_bf16_3d(&m_w1, w1p, d, static_cast<uint64_t>(rows), 1, d * 2,
+                                d * 2 * static_cast<uint64_t>(rows), 64, 128 * UP_SUB)) != TP_OK)
+    return st;
+  // x [T][d]: token rows past T read as zeros
+  if ((st = encode_tmap_bf16_3d(&m_x, x, d, T, 1, d * 2, d * 2 * T, 64, BN)) != TP_OK) return st;
+  // packed W2 [p][d][Fsp]
+  if ((st = encode_tmap_bf16_3d(&m_w2, w2p, Fsp, d, P, Fsp * 2, d * Fsp * 2, 64, 128)) != TP_OK)
+    return st;
+  // h [T][p*Fsp] seen as [p][T][Fsp]: shard i's columns are its k range
+  if ((st = encode_tmap_bf16_3d(&m_h, h, Fsp, T, P, P * Fsp * 2, Fsp * 2, 64, BN)) != TP_OK)
+    return st;
+  mlpdec::Params pr;
+  pr.n_up = static_cast<int32_t>(rows / (128 * UP_SUB));
+  pr.up_kb = static_cast<int32_t>(ceil_div(L.d, 64));
+  pr.up_per_shard = static_cast<int32_t>(L.Fsp / 128);
+  pr.dn_mb = static_cast<int32_t>(ceil_div(L.d, 128));
+  pr.n_dn = static_cast<int32_t>(L.p * pr.dn_mb);
+  pr.dn_kb = static_cast<int32_t>(L.Fsp / 64);
+  pr.counters = static_cast<int32_t*>(counters);
+  pr.err = device_error_word();
+  pr.up.h = static_cast<__nv_bfloat16*>(h);
+  pr.up.z = static_cast<__nv_bfloat16*>(z);
+  pr.up.ld_h = L.p * L.Fsp;
+  pr.up.ld_z = rows;
+  pr.up.tokens = static_cast<int32_t>(L.T);
+  pr.up.rows = static_cast<int32_t>(rows);
+  pr.up.act = L.act;
+  pr.up.swap = 1;
+  pr.dn.out = part;
+  pr.dn.ld = L.d;
+  pr.dn.batch_stride = L.T * L.d;
+  pr.dn.rows_valid = static_cast<int32_t>(L.T);
+  pr.dn.cols_valid = static_cast<int32_t>(L.d);
+  pr.dn.swap = 1;
+  TP_LAUNCH_PDL(zero_words_kernel, dim3(1), dim3(256), 0, s, static_cast<uint32_t*>(counters),
+                static_cast<int64_t>(1 + L.p));
+  auto* kern = mlpdec::mlp_decode_kernel<C>;
+  static int attr_set[64] = {0};
+  int dev = 0;
+  TP_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev < 64 && !attr_set[dev]) {
+    TP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                     C::SMEM_BYTES));
+    attr_set[dev] = 1;
+  }
+  ProfScope prof(s, "mlp_decode_gemm");
+  TP_LAUNCH_PDL(kern, dim3(static_cast<unsigned>(num_sms())), dim3(tc::kThreads),
+                static_cast<size_t>(C::SMEM_BYTES), s, m_w1, m_x, m_w2, m_h, pr);
+  return TP_OK;
+}
+
+tp_status mlp_decode(const MlpLayout& L, const void* x, const void* w1p, const void* w2p, void* h,
+                     void* z, float* part, void* counters, cudaStream_t s) {
+  const bool swiglu = L.act == TP_ACT_SWIGLU;
+  if (L.T <= 16)
+    return swiglu ? run_mlp_decode<16, 2>(L, x, w1p, w2p, h, z, part, counters, s)
+                  : run_mlp_decode<16, 1>(L, x, w1p, w2p, h, z, part, counters, s);
+  return swiglu ? run_mlp_decode<64, 2>(L, x, w1p, w2p, h, z, part, counters, s)
+                : run_mlp_decode<64, 1>(L, x, w1p, w2p, h, z, part, counters, s);
 }
 
 // With TP_REDUCE_FUSED the dx GEMM sums the shards in its accumulator and writes dx itself
@@ -515,8 +601,13 @@ tp_status mlp_forward(const MlpLayout& L, const tp_mlp_desc* desc, const void* x
         return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
     void* sk = off(workspace, L.fsk_off);
     const size_t skb = L.fpart_off - L.fsk_off;
-    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
-    if ((st = tc_down(L, h, w2p, part, residual, y, sk, skb, s)) != TP_OK) return st;
+    if (fused_decode_ok(L)) {
+      if ((st = mlp_decode(L, x, w1p, w2p, h, saved ? z : nullptr, part, sk, s)) != TP_OK)
+        return st;
+    } else {
+      if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
+      if ((st = tc_down(L, h, w2p, part, residual, y, sk, skb, s)) != TP_OK) return st;
+    }
     if (L.reduce_mode == TP_REDUCE_FUSED) {
       if (y_norm && (st = reduce::rmsnorm(y, L.y_dtype, L.T, L.d, L.norm_eps, y_norm, L.dtype, s)) != TP_OK)
         return st;
