@@ -39,12 +39,19 @@ using tc::kUmmaK;
 using tc::kEpiWarps;
 using tc::kThreads;
 
+// A stage holds two 128 x 64 weight boxes and up to two token boxes: an up tile of SwiGLU loads its
+// gate and up rows of one k-block, every other item two k-blocks of 128 rows, so each stage keeps
+// 32 KB of weights in flight whatever the item.
 template <int BN_, int UP_SUB_>
 struct Cfg {
   static constexpr int BN = BN_;            // tokens per tile (N of the MMAs)
   static constexpr int UP_SUB = UP_SUB_;    // 128-row MMAs per up tile (2: SwiGLU gate + up)
-  static constexpr int A_STAGE_BYTES = 128 * UP_SUB * kBK * 2;   // a down stage uses 128 rows
-  static constexpr int B_STAGE_BYTES = BN * kBK * 2;
+  static constexpr int UP_KPACK = 2 / UP_SUB;   // k-blocks per stage of an up tile
+  static constexpr int DN_KPACK = 2;            // k-blocks per stage of a down tile
+  static constexpr int BOX_A = 128 * kBK * 2;   // one 128 x 64 weight box
+  static constexpr int BOX_B = BN * kBK * 2;    // one BN x 64 token box
+  static constexpr int A_STAGE_BYTES = 2 * BOX_A;
+  static constexpr int B_STAGE_BYTES = 2 * BOX_B;
   static constexpr int STAGE_BYTES = A_STAGE_BYTES + B_STAGE_BYTES;
   static constexpr int STAGES = (200 * 1024) / STAGE_BYTES < 8 ? (200 * 1024) / STAGE_BYTES : 8;
   static constexpr int ACC_COLS = UP_SUB * BN;
@@ -192,9 +199,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int t = up ? item : item - pr.n_up;
         const int shard = up ? 0 : t / pr.dn_mb;
         const int m0 = up ? t * 128 * C::UP_SUB : (t - shard * pr.dn_mb) * 128;
-        const int nk = up ? pr.up_kb : pr.dn_kb;
-        const int rot = static_cast<int>((static_cast<int64_t>(item) * 37) % nk);
-        const uint32_t bytes = up ? C::STAGE_BYTES : 128 * kBK * 2 + C::B_STAGE_BYTES;
+        const int kb_all = up ? pr.up_kb : pr.dn_kb;
+        const int kpack = up ? C::UP_KPACK : C::DN_KPACK;
+        const int nst = (kb_all + kpack - 1) / kpack;   // stages of this item
+        const int rot = static_cast<int>((static_cast<int64_t>(item) * 37) % nst);
         if (!up) {
           // h of this shard must be complete before its tensor loads
           if (!wait_shard_ready(pr, shard, pr.up_per_shard, abort_flag)) {
@@ -203,22 +211,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           fence_proxy_async_global();
         }
-        for (int i = 0; i < nk; ++i) {
-          int kb = i + rot;
-          if (kb >= nk) kb -= nk;
+        for (int i = 0; i < nst; ++i) {
+          int si = i + rot;
+          if (si >= nst) si -= nst;
+          const int kb0 = si * kpack;
+          const int nkb = kb_all - kb0 < kpack ? kb_all - kb0 : kpack;
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, pr.err, DEVERR_WAIT_EMPTY)) {
             ok = false;
             break;
           }
-          mbar_arrive_expect_tx(&full[stage], bytes);
           uint8_t* sa = a_smem + stage * C::A_STAGE_BYTES;
           uint8_t* sb = b_smem + stage * C::B_STAGE_BYTES;
-          if (up) {
-            tma_load_3d(&tma_w1, &full[stage], sa, kb * kBK, m0, 0);
-            tma_load_3d(&tma_x, &full[stage], sb, kb * kBK, 0, 0);
+          if (up && C::UP_SUB == 2) {
+            // gate and up rows of one k-block: one 256-row box
+            mbar_arrive_expect_tx(&full[stage], 2 * C::BOX_A + C::BOX_B);
+            tma_load_3d(&tma_w1, &full[stage], sa, kb0 * kBK, m0, 0);
+            tma_load_3d(&tma_x, &full[stage], sb, kb0 * kBK, 0, 0);
           } else {
-            tma_load_3d(&tma_w2, &full[stage], sa, kb * kBK, m0, shard);
-            tma_load_3d(&tma_h, &full[stage], sb, kb * kBK, 0, shard);
+            mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nkb * (C::BOX_A + C::BOX_B)));
+            for (int j = 0; j < nkb; ++j) {
+              const int k0 = (kb0 + j) * kBK;
+              if (up) {
+                tma_load_3d(&tma_w1, &full[stage], sa + j * C::BOX_A, k0, m0, 0);
+                tma_load_3d(&tma_x, &full[stage], sb + j * C::BOX_B, k0, 0, 0);
+              } else {
+                tma_load_3d(&tma_w2, &full[stage], sa + j * C::BOX_A, k0, m0, shard);
+                tma_load_3d(&tma_h, &full[stage], sb + j * C::BOX_B, k0, 0, shard);
+              }
+            }
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
@@ -253,8 +273,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         if (item < 0) break;
         const bool up = item < pr.n_up;
-        const int nk = up ? pr.up_kb : pr.dn_kb;
-        const int subs = up ? C::UP_SUB : 1;
+        const int kb_all = up ? pr.up_kb : pr.dn_kb;
+        const int kpack = up ? C::UP_KPACK : C::DN_KPACK;
+        const int nst = (kb_all + kpack - 1) / kpack;
+        const int rot = static_cast<int>((static_cast<int64_t>(item) * 37) % nst);
         const int acc = it_n & 1;
         const uint32_t acc_phase = (it_n >> 1) & 1;
         ++it_n;
@@ -265,7 +287,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
         tc_fence_after();
         const uint32_t d_base = tmem_base + acc * C::ACC_COLS;
-        for (int i = 0; i < nk; ++i) {
+        for (int i = 0; i < nst; ++i) {
           if (!mbar_wait(&full[stage], phase, abort_flag, pr.err, DEVERR_WAIT_FULL)) {
             ok = false;
             break;
@@ -273,15 +295,31 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_after();
           const uint32_t a_addr = smem_addr(a_smem + stage * C::A_STAGE_BYTES);
           const uint32_t b_addr = smem_addr(b_smem + stage * C::B_STAGE_BYTES);
+          int si = i + rot;
+          if (si >= nst) si -= nst;
+          const int kb0 = si * kpack;
+          const int nkb = kb_all - kb0 < kpack ? kb_all - kb0 : kpack;
+          if (up && C::UP_SUB == 2) {
+            // gate rows accumulate in columns [0, BN), up rows in [BN, 2 BN)
 #pragma unroll
-          for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
-            const uint64_t bdesc = make_sdesc_sw128(b_addr + kk * (kUmmaK * 2), 16, 1024);
+            for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+              const uint64_t bdesc = make_sdesc_sw128(b_addr + kk * (kUmmaK * 2), 16, 1024);
 #pragma unroll
-            for (int s = 0; s < C::UP_SUB; ++s) {
-              if (s < subs) {
+              for (int s = 0; s < 2; ++s) {
                 const uint64_t adesc =
-                    make_sdesc_sw128(a_addr + s * 128 * kBK * 2 + kk * (kUmmaK * 2), 16, 1024);
+                    make_sdesc_sw128(a_addr + s * C::BOX_A + kk * (kUmmaK * 2), 16, 1024);
                 umma_f16(d_base + s * C::BN, adesc, bdesc, C::IDESC, (i > 0 || kk != 0) ? 1u : 0u);
+              }
+            }
+          } else {
+            for (int j = 0; j < nkb; ++j) {
+#pragma unroll
+              for (int kk = 0; kk < kBK / kUmmaK; ++kk) {
+                const uint64_t bdesc =
+                    make_sdesc_sw128(b_addr + j * C::BOX_B + kk * (kUmmaK * 2), 16, 1024);
+                const uint64_t adesc =
+                    make_sdesc_sw128(a_addr + j * C::BOX_A + kk * (kUmmaK * 2), 16, 1024);
+                umma_f16(d_base, adesc, bdesc, C::IDESC, (i > 0 || j > 0 || kk != 0) ? 1u : 0u);
               }
             }
           }

@@ -860,8 +860,13 @@ extern "C" tp_status tp_mlp_fwd_sp(const tp_mlp_desc* desc, const void* const* x
       if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "bf16 pointers must be 16-byte aligned");
     void* sk = off(ws, L.fsk_off);
     const size_t skb = L.fpart_off - L.fsk_off;
-    if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
-    if ((st = tc_down(L, h, w2p, part, nullptr, nullptr, sk, skb, s)) != TP_OK) return st;
+    if (fused_decode_ok(L)) {
+      if ((st = mlp_decode(L, x, w1p, w2p, h, saved ? z : nullptr, part, sk, s)) != TP_OK)
+        return st;
+    } else {
+      if ((st = tc_up(L, x, w1p, h, saved ? z : nullptr, sk, skb, s)) != TP_OK) return st;
+      if ((st = tc_down(L, h, w2p, part, nullptr, nullptr, sk, skb, s)) != TP_OK) return st;
+    }
   } else if (L.dtype == TP_BF16) {
     if ((st = simt_forward<__nv_bfloat16>(L, x, w1p, w2p, z, h, part, s)) != TP_OK) return st;
   } else {

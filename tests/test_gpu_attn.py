@@ -73,6 +73,9 @@ def test_residual(lib):
     ("bf16", 1, 4096, 512, 16, 2, 128, 2, 1),  # 33 chunks, group of 8 query heads per KV head
     ("bf16", 2, 1, 128, 4, 4, 32, 4, 0),       # a single cached key
     ("f32", 2, 37, 64, 4, 2, 32, 2, 0),
+    # output projection of 4 x 40 = 160 tiles of 32 k-blocks: the 12 past a wave are split,
+    # then every CTA runs whole tiles
+    ("bf16", 2, 64, 5120, 64, 8, 128, 4, 0),
 ])
 def test_decode(lib, dtype, b, kv_len, h, n_q, n_kv, hd, p, mode):
     inp = inputs.attn_inputs(b, 1, h, n_q, n_kv, hd, dtype, seed=4, w_std=0.05, kv_len=kv_len)

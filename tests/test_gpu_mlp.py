@@ -237,15 +237,16 @@ def test_stream_k_splits_fused_vs_separate(lib, T, d, F, p):
 
 
 @pytest.mark.parametrize("T,d,F,p,act", [
-    (2, 5504, 14336, 7, "gelu"),     # down: 7 x 43 = 301 tiles of 32 k-blocks = 2 waves + 5: the
-                                     # 5 are split together with one more wave, then whole tiles
-    (3, 2048, 19072, 1, "swiglu"),   # up: 149 tiles of 256 packed rows, one more than the SMs
-    (5, 4096, 22400, 5, "swiglu"),   # up: 175 tiles (27 split, 148 whole); down: 160 (12, 148)
+    (2, 5568, 14336, 7, "gelu"),     # 87 k-blocks per up tile (two per stage, one left over), a
+                                     # ragged last block of 64 output rows, 7 shards
+    (3, 2048, 19072, 1, "swiglu"),   # one shard, 149 up tiles of 256 packed rows
+    (5, 4096, 22400, 5, "swiglu"),   # 175 up tiles, 160 down tiles
+    (40, 1024, 3072, 3, "relu"),     # 64-token tiles, three shards
 ])
-def test_decode_split_then_whole_tiles(lib, T, d, F, p, act):
-    # weight-streaming GEMMs with more tiles than SMs: the remainder after whole waves is split
-    # into equal k-ranges (fixed up by the last CTA to arrive), then every CTA runs whole tiles;
-    # checked against the oracle row by row, and two runs give the same bits
+def test_decode_one_launch_shapes(lib, T, d, F, p, act):
+    # the one-launch decode MLP (up tiles, then down tiles taken from a device counter once their
+    # shard's h is complete): checked against the oracle row by row, and two runs give the same
+    # bits
     inp = inputs.mlp_inputs(T, d, F, act, "bf16", seed=11 + T, w_std=0.03)
     m = Mlp(lib, inp, p, act, "bf16", 0)
     a = m.forward(inp["x"], save=False).clone()
