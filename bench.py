@@ -178,7 +178,7 @@ def _profile(tp, fn, steps):
     return prof
 
 
-GEMM_SOURCES = ("gemm_tc.cuh", "sm100.cuh", "gemm_launch.cuh", "tp_mlp.cu")
+GEMM_SOURCES = ("gemm_tc.cuh", "sm100.cuh", "gemm_launch.cuh", "tp_mlp.cu", "mlp_decode.cuh")
 
 
 def _gemm_source_hash():

@@ -3,6 +3,7 @@
 #pragma once
 
 #include <algorithm>
+#include <tuple>
 
 #include "flash_attn.cuh"
 #include "gemm_launch.cuh"
@@ -70,6 +71,10 @@ inline size_t attn_sk_bytes(const AttnLayout& L) {
 
 
 // Decode shapes the MMA decode kernel takes (the rest use the SIMT split kernel).
+// Most splits of one KV head merged through distributed shared memory (a non-portable cluster
+// size on sm_100; the launch checks that such clusters fit and otherwise merges through memory).
+constexpr int64_t kDecodeClusterMax = 16;
+
 inline bool decode_mma_eligible(const AttnLayout& L, const tp_attn_desc* d) {
   const int group = d->n_q / d->n_kv;
   return d->dtype == TP_BF16 && (L.hd == 64 || L.hd == 128) &&
@@ -114,10 +119,13 @@ inline tp_status attn_layout_of(const tp_attn_desc* d, AttnLayout* L) {
     int64_t max_chunk = std::min<int64_t>(
         512, (200 * 1024) / (2 * static_cast<int64_t>(L->hd) * L->eb + 4 * (L->n_q / L->n_kv)) / 16 * 16);
     // the MMA decode kernel (bf16, head_dim 64/128, <= 8 query heads per KV head) stages at most
-    // 256 (head_dim 128) or 512 (head_dim 64) keys per split
-    if (decode_mma_eligible(*L, d))
-      max_chunk = std::min<int64_t>(max_chunk, L->hd == 128 ? 256 : 512);
-    const int64_t want = std::max<int64_t>(1, num_sms() / std::max<int64_t>(1, L->b * L->n_kv));
+    // 384 (head_dim 128) or 768 (head_dim 64) keys per split, and merges the splits of a KV head
+    // inside a cluster when there are at most kDecodeClusterMax of them
+    int64_t want = std::max<int64_t>(1, num_sms() / std::max<int64_t>(1, L->b * L->n_kv));
+    if (decode_mma_eligible(*L, d)) {
+      max_chunk = std::min<int64_t>(max_chunk, L->hd == 128 ? 384 : 768);
+      want = std::min<int64_t>(want, kDecodeClusterMax);
+    }
     int64_t splits = std::min<int64_t>(std::min<int64_t>(want, 64), ceil_div(n_keys, 16));
     splits = std::max<int64_t>(splits, ceil_div(n_keys, max_chunk));
     L->kv_chunk = static_cast<int>(round_up(ceil_div(n_keys, splits), 16));
@@ -560,7 +568,7 @@ struct DecodeMmaCfg {
   static constexpr int kHalves = HD / 64;               // 64-dim tiles per row
   static constexpr int kTileBytes = kSub * 128;         // one [32][64] bf16 tile
   static constexpr int kSubBytes = 2 * kHalves * kTileBytes;   // K and V of one sub-chunk
-  static constexpr int kMaxSub = HD == 128 ? 8 : 16;    // at most 256 (128) or 512 (64) keys
+  static constexpr int kMaxSub = HD == 128 ? 12 : 24;   // at most 384 (128) or 768 (64) keys
   static constexpr int kMaxChunk = kMaxSub * kSub;
   static constexpr size_t kSmem = static_cast<size_t>(kMaxSub) * kSubBytes + 1024;
 };
@@ -591,7 +599,7 @@ __device__ __forceinline__ uint32_t pack_bf16x2(float lo, float hi) {
   return *reinterpret_cast<const uint32_t*>(&v);
 }
 
-template <int GROUP, int HD>
+template <int GROUP, int HD, bool CLUSTER>
 __global__ void __launch_bounds__(256) decode_mma_kernel(
     const __grid_constant__ CUtensorMap kmap, const __grid_constant__ CUtensorMap vmap,
     const __nv_bfloat16* qkv, QkvIdx ix, __nv_bfloat16* kc, __nv_bfloat16* vc, int64_t kv_cap,
@@ -606,6 +614,9 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
   uint8_t* dsm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(dsm_raw) + 1023) & ~uintptr_t(1023));
   __shared__ __align__(8) uint64_t bars[C::kMaxSub];
   __shared__ int s_abort;
+  // this split's merged result (cluster merge): o[GROUP][HD], m (log2 units) and l per head
+  __shared__ __align__(16) float s_res_o[CLUSTER ? GROUP : 1][CLUSTER ? HD : 4];
+  __shared__ float s_res_m[GROUP], s_res_l[GROUP];
   const int c = blockIdx.x, g = blockIdx.y;
   const int64_t bi = blockIdx.z;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -756,7 +767,8 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 1);
   l_run += __shfl_xor_sync(0xffffffffu, l_run, 2);
 
-  // ---- abort path: every tile must land before the block leaves (bounded), then return
+  // ---- abort path: every tile must land before the block leaves (bounded), then return (in a
+  // cluster, only after the two cluster barriers every CTA of the cluster takes)
   if (abort_local) s_abort = 1;
   __syncthreads();
   if (s_abort) {
@@ -766,6 +778,10 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
       }
     }
     __syncthreads();
+    if constexpr (CLUSTER) {
+      sm100::cluster_sync();
+      sm100::cluster_sync();
+    }
     return;
   }
 
@@ -803,18 +819,130 @@ __global__ void __launch_bounds__(256) decode_mma_kernel(
       acc.w += f * v.w;
       L += f * wl[w * GROUP + a];
     }
-    const int j = g * GROUP + a;
-    float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * kRec;
-    *reinterpret_cast<float4*>(rec + 4 * e4) = acc;
-    if (e4 == 0) {
-      rec[HD] = M;
-      rec[HD + 1] = L;
+    if constexpr (CLUSTER) {
+      *reinterpret_cast<float4*>(&s_res_o[a][4 * e4]) = acc;
+      if (e4 == 0) {
+        s_res_m[a] = M;
+        s_res_l[a] = L;
+      }
+    } else {
+      const int j = g * GROUP + a;
+      float* rec = ml + ((bi * n_q + j) * gridDim.x + c) * kRec;
+      *reinterpret_cast<float4*>(rec + 4 * e4) = acc;
+      if (e4 == 0) {
+        rec[HD] = M;
+        rec[HD + 1] = L;
+      }
     }
   }
-  merge_splits_if_last<__nv_bfloat16, GROUP, HD>(ml, counters, o, bi, g, n_q, n_kv);
+  if constexpr (CLUSTER) {
+    // The splits of this KV head are the cluster's CTAs (rank = split).  After the barrier, CTA r
+    // merges its share of the GROUP x HD outputs from every split's shared memory, in split
+    // order: o = sum_c 2^(m_c - M) o_c / sum_c 2^(m_c - M) l_c.
+    sm100::cluster_sync();
+    const int splits = static_cast<int>(gridDim.x);
+    const int rank = static_cast<int>(sm100::cluster_rank());
+    constexpr int kOut = GROUP * HD;
+    const int per = (kOut + splits - 1) / splits;
+    const int i0 = rank * per;
+    const int i1 = i0 + per < kOut ? i0 + per : kOut;
+    for (int idx = i0 + threadIdx.x; idx < i1; idx += blockDim.x) {
+      const int a = idx / HD, e = idx - a * HD;
+      const uint32_t am = sm100::smem_addr(&s_res_m[a]);
+      const uint32_t al = sm100::smem_addr(&s_res_l[a]);
+      const uint32_t ao = sm100::smem_addr(&s_res_o[a][e]);
+      float mc[kDecodeClusterMax], lc[kDecodeClusterMax], oc[kDecodeClusterMax];
+#pragma unroll
+      for (int cc = 0; cc < kDecodeClusterMax; ++cc) {
+        if (cc < splits) {
+          mc[cc] = sm100::ld_shared_cluster_f32(sm100::map_to_rank(am, cc));
+          lc[cc] = sm100::ld_shared_cluster_f32(sm100::map_to_rank(al, cc));
+          oc[cc] = sm100::ld_shared_cluster_f32(sm100::map_to_rank(ao, cc));
+        }
+      }
+      float Mx = -INFINITY;
+#pragma unroll
+      for (int cc = 0; cc < kDecodeClusterMax; ++cc)
+        if (cc < splits) Mx = fmaxf(Mx, mc[cc]);
+      float Ls = 0.f, acc = 0.f;
+#pragma unroll
+      for (int cc = 0; cc < kDecodeClusterMax; ++cc) {
+        if (cc < splits) {
+          const float f = mc[cc] == -INFINITY ? 0.f : exp2f(mc[cc] - Mx);
+          Ls += f * lc[cc];
+          acc += f * oc[cc];
+        }
+      }
+      o[bi * static_cast<int64_t>(n_q) * HD + (g * GROUP + a) * HD + e] = from_f<__nv_bfloat16>(acc / Ls);
+    }
+    sm100::cluster_sync();   // no CTA leaves while a peer may still read its shared memory
+  } else {
+    merge_splits_if_last<__nv_bfloat16, GROUP, HD>(ml, counters, o, bi, g, n_q, n_kv);
+  }
 }
 
 }  // namespace attn
+
+// Decode attention with the splits of each KV head merged inside a cluster (one CTA per split).
+// Tries the layout's split count, then fewer splits (longer chunks, up to the kernel's limit),
+// and launches with the largest count whose clusters all fit on the device at once (one per
+// sequence and KV head); *done tells the caller whether it launched.
+template <int MAX_CHUNK, class Kern, class Args>
+inline tp_status launch_decode_cluster(Kern kern, dim3 grid, size_t smem, const AttnLayout& L,
+                                       cudaStream_t s, Args args, bool* done) {
+  *done = false;
+  if (L.kv_splits < 2) return TP_OK;
+  static int fits[64][kDecodeClusterMax + 1];   // per device and cluster size; 0 = not queried
+  int dev = 0;
+  TP_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 64) return TP_OK;
+  TP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                   static_cast<int>(smem)));
+  TP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeNonPortableClusterSizeAllowed, 1));
+  cudaLaunchConfig_t cfg = {};
+  cfg.blockDim = dim3(256);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[2];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  attr[1].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[1].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  const int64_t n_keys = L.kv_len + 1;
+  for (int64_t c = std::min<int64_t>(L.kv_splits, kDecodeClusterMax); c >= 2; --c) {
+    const int64_t chunk = round_up(ceil_div(n_keys, c), 16);
+    if (chunk > MAX_CHUNK) break;              // fewer splits only make the chunks longer
+    if (ceil_div(n_keys, chunk) != c) continue;   // c splits of this chunk leave one empty
+    int& fit = fits[dev][c];
+    if (fit == 0) {
+      cfg.gridDim = dim3(static_cast<unsigned>(c), grid.y, grid.z);
+      attr[0].val.clusterDim.x = static_cast<unsigned>(c);
+      cfg.numAttrs = 1;
+      int n = 0;
+      if (cudaOccupancyMaxActiveClusters(&n, kern, &cfg) != cudaSuccess) {
+        (void)cudaGetLastError();
+        n = 0;
+      }
+      fit = n > 0 ? n : -1;
+    }
+    if (fit < L.b * L.n_kv) continue;
+    cfg.gridDim = dim3(static_cast<unsigned>(c), grid.y, grid.z);
+    attr[0].val.clusterDim.x = static_cast<unsigned>(c);
+    cfg.numAttrs = 2;
+    std::get<8>(args) = static_cast<int>(chunk);   // the kernel's chunk argument
+    ProfScope prof(s, "attn_decode");
+    const cudaError_t e = std::apply(
+        [&](auto... a) { return cudaLaunchKernelEx(&cfg, kern, a...); }, args);
+    if (e != cudaSuccess)
+      return set_error(TP_ERR_CUDA, std::string("kernel launch: ") + cudaGetErrorString(e));
+    count_launch();
+    *done = true;
+    return TP_OK;
+  }
+  return TP_OK;
+}
 
 template <typename T>
 inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, void* kc, void* vc,
@@ -876,8 +1004,18 @@ inline tp_status attn_core(const AttnLayout& L, const void* qkv_v, void* o_v, vo
       if (r != TP_OK) return r;
 #define TP_DECODE_MMA_CASE(G, H)                                                              \
       if (group == G && L.hd == H) {                                                          \
-        auto* kern = attn::decode_mma_kernel<G, H>;                                           \
         const size_t smem = attn::DecodeMmaCfg<H>::kSmem;                                     \
+        auto args = std::make_tuple(km, vm, reinterpret_cast<const __nv_bfloat16*>(qkv), ix,  \
+                                    static_cast<__nv_bfloat16*>(kc),                          \
+                                    static_cast<__nv_bfloat16*>(vc), L.kv_cap, L.kv_len,      \
+                                    L.kv_chunk, L.n_q, L.n_kv, scale, ml, counters,           \
+                                    reinterpret_cast<__nv_bfloat16*>(o), device_error_word()); \
+        bool done = false;                                                                    \
+        tp_status cst = launch_decode_cluster<attn::DecodeMmaCfg<H>::kMaxChunk>(                \
+            attn::decode_mma_kernel<G, H, true>, grid, smem, L, s, args, &done);               \
+        if (cst != TP_OK) return cst;                                                         \
+        if (done) return TP_OK;                                                               \
+        auto* kern = attn::decode_mma_kernel<G, H, false>;                                    \
         TP_CUDA_TRY(cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,   \
                                          static_cast<int>(smem)));                            \
         ProfScope prof(s, "attn_decode");                                                     \

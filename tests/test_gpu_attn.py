@@ -100,6 +100,7 @@ def test_decode(lib, dtype, b, kv_len, h, n_q, n_kv, hd, p, mode):
     (1, 4111, 16, 2, 128, 0),  # eight per KV head, a last split of a few keys
     (2, 700, 8, 2, 64, 33),    # head_dim 64, four per KV head, spare slots past the new token
     (3, 17, 16, 2, 64, 0),     # one split holding 18 keys
+    (1, 6000, 16, 2, 128, 0),  # 19 splits, more than a cluster takes: merged through memory
 ])
 def test_decode_edges(lib, b, kv_len, n_q, n_kv, hd, spare):
     # slots past the new token (kv_cap > kv_len + 1) hold NaN: they must never be read
