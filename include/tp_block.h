@@ -470,9 +470,10 @@ int32_t tp_tensor_core_path_available(void);
 
 /* Failure-detection self-test (the pages have no counterpart; it exercises the timeout path
  * behind TP_ERR_TIMEOUT without any fault).  Enqueues one small kernel that waits, through the
- * same bounded mbarrier wait the tensor-core kernels use, on a barrier that nothing completes;
- * after limit_us microseconds (1 .. 1000000) the wait gives up, records the timeout in the device
- * error word and the kernel returns.  A following tp_check_device_error() reports TP_ERR_TIMEOUT
+ * same bounded mbarrier wait the tensor-core kernels use, on a barrier that nothing completes,
+ * then through the bounded cross-CTA counter wait of the one-launch decode MLP on a counter that
+ * nothing increments; after limit_us microseconds (1 .. 1000000) each wait gives up and records
+ * its site in the device error word (bits 1 and 32), and the kernel returns.  A following tp_check_device_error() reports TP_ERR_TIMEOUT
  * and clears the word; the CUDA context stays usable.  Returns TP_ERR_INVALID_ARG for a limit
  * out of range (checked before anything is enqueued). */
 tp_status tp_selftest_wait_timeout(uint32_t limit_us, void* stream);

@@ -81,34 +81,9 @@ struct Params {
   tc::EpiStoreF32::Params dn;  // fp32 partials [p][T][d], swapped
 };
 
-__device__ __forceinline__ int ld_acquire_gpu(const int32_t* p) {
-  int32_t v;
-  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
-  return v;
-}
 // orders this thread's generic-proxy accesses with its tensor (async-proxy) accesses
 __device__ __forceinline__ void fence_proxy_async_global() {
   asm volatile("fence.proxy.async.global;" ::: "memory");
-}
-
-// Bounded wait until counters[1 + shard] reaches need (the up tiles of a shard have stored h).
-__device__ __forceinline__ bool wait_shard_ready(const Params& pr, int shard, int need,
-                                                 volatile int* abort_flag) {
-  const int32_t* c = pr.counters + 1 + shard;
-  if (ld_acquire_gpu(c) >= need) return true;
-  const uint64_t t0 = globaltimer_ns();
-  uint32_t n = 0;
-  while (ld_acquire_gpu(c) < need) {
-    if ((++n & 15u) == 0) {
-      if (*abort_flag) return false;
-      if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-        *abort_flag = 1;
-        record_device_error(pr.err, DEVERR_WAIT_FLAG);
-        return false;
-      }
-    }
-  }
-  return true;
 }
 
 template <class C>
@@ -205,7 +180,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int rot = static_cast<int>((static_cast<int64_t>(item) * 37) % nst);
         if (!up) {
           // h of this shard must be complete before its tensor loads
-          if (!wait_shard_ready(pr, shard, pr.up_per_shard, abort_flag)) {
+          if (!wait_counter_at_least(pr.counters + 1 + shard, pr.up_per_shard, abort_flag,
+                                     pr.err, DEVERR_WAIT_FLAG)) {
             ok = false;
             break;
           }

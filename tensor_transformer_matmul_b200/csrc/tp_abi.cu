@@ -138,6 +138,9 @@ namespace tp {
 // One warp waits, through the same bounded mbarrier wait the tensor-core kernels use, on a
 // barrier that nothing ever completes; after limit_ns the wait gives up, raises the abort flag
 // and records DEVERR_WAIT_FULL in the device error word, and the kernel returns.
+// A counter that no kernel ever increments (the self-test's cross-CTA wait).
+__device__ int32_t g_selftest_counter = 0;
+
 __global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
   __shared__ uint64_t bar;
   __shared__ int abort_flag;
@@ -147,8 +150,12 @@ __global__ void wait_selftest_kernel(uint64_t limit_ns, uint32_t* err) {
     sm100::fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0)
+  if (threadIdx.x == 0) {
+    // the mbarrier wait of the pipelines, then the counter wait of the one-launch decode MLP
     sm100::mbar_wait(&bar, 0, &abort_flag, err, DEVERR_WAIT_FULL, limit_ns);
+    abort_flag = 0;
+    wait_counter_at_least(&g_selftest_counter, 1, &abort_flag, err, DEVERR_WAIT_FLAG, limit_ns);
+  }
   __syncthreads();
 }
 }  // namespace tp

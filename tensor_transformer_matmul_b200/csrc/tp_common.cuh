@@ -158,6 +158,36 @@ __device__ __forceinline__ void record_device_error(uint32_t* word, uint32_t bit
   if (word) atomicOr(word, bits);
 }
 
+// Acquire load of a 32-bit word at GPU scope (a counter other CTAs publish with a release).
+__device__ __forceinline__ int32_t ld_acquire_gpu(const int32_t* p) {
+  int32_t v;
+  asm volatile("ld.acquire.gpu.global.b32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *c >= need (another CTA's progress counter).  Gives up when *abort is set
+// or after limit_ns; a timeout sets *abort, records site in the device error word and returns
+// false.
+__device__ __forceinline__ bool wait_counter_at_least(const int32_t* c, int32_t need,
+                                                      volatile int* abort, uint32_t* err,
+                                                      uint32_t site,
+                                                      uint64_t limit_ns = kWaitTimeoutNs) {
+  if (ld_acquire_gpu(c) >= need) return true;
+  const uint64_t t0 = globaltimer_ns();
+  uint32_t n = 0;
+  while (ld_acquire_gpu(c) < need) {
+    if ((++n & 15u) == 0) {
+      if (*abort) return false;
+      if (globaltimer_ns() - t0 > limit_ns) {
+        *abort = 1;
+        record_device_error(err, site);
+        return false;
+      }
+    }
+  }
+  return true;
+}
+
 // ----------------------------------------------------------------------------------------------
 // element conversions
 // ----------------------------------------------------------------------------------------------

@@ -21,6 +21,9 @@ def test_wait_timeout_is_reported_and_cleared(lib):
     with pytest.raises(lib.TpError) as e:
         lib.tp_check_device_error()
     assert e.value.status == lib.TP_ERR_TIMEOUT
+    # both waits ran out: the pipeline's mbarrier wait (bit 1) and the cross-CTA counter wait of
+    # the one-launch decode MLP (bit 32)
+    assert "site bits 33" in str(e.value)
     lib.tp_check_device_error()              # the report cleared the word
 
 
