@@ -630,9 +630,21 @@ def extra_moe(tp, inputs, torch, stream, peaks, steps):
         ms = _cuda_time(fwd, steps, stream) / steps
         prof = _profile(tp, fwd, steps)
         flops = T * k * fl_per_row + T * 2.0 * d * 3 * Fs + 2.0 * T * d * E
+        # the weights every call must stream: the experts the router picks (counted here from the
+        # same logits, outside the timed calls) and the shared expert, plus x and y
+        with torch.no_grad():
+            picked = torch.topk(x.float() @ wr.float(), k, dim=1).indices.unique().numel()
+        nbytes = 2 * (picked * (e1 + e2) + w1s.numel() + w2s.numel()) + 2 * 2 * T * d
+        t_hbm = nbytes / (peaks["hbm_gbs"] * 1e9) * 1e3
+        t_tc = flops / (peaks["bf16_tflops"] * 1e12) * 1e3
         out[name] = {"T": T, "ms": round(ms, 3),
                      "TFLOP_per_s": round(flops / (ms / 1e3) / 1e12, 1),
                      "frac_of_burst_peak": round(flops / (ms / 1e3) / 1e12 / peaks["bf16_tflops"], 3),
+                     "experts_hit": picked, "weight_bytes": nbytes,
+                     "GB_per_s": round(nbytes / (ms / 1e3) / 1e9, 1),
+                     "bound": "hbm" if t_hbm >= t_tc else "tensor",
+                     "roofline_ms": round(max(t_hbm, t_tc), 3),
+                     "frac_of_roofline": round(max(t_hbm, t_tc) / ms, 3),
                      "tokens_per_s": round(T / (ms / 1e3), 1),
                      "kernels": {kk: {"ms_per_launch": round(v[1] / v[0], 4)} for kk, v in prof.items()}}
         del ws, x, y

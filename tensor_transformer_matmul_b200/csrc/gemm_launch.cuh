@@ -124,6 +124,7 @@ struct GemmOpts {
   int grp_n = 0;
   int grp_div = 1;
   bool grp_sum = false;   // sum each group's grp_div problems into one output (in order)
+  bool grp_swap = false;  // the group ranges run along N (B rows); grp_mbp counts BN-row blocks
   // words that the kernel after this GEMM needs zeroed: cleared by the launch that zeroes the
   // stream-K counters (one kernel for both), or by a small kernel of their own
   uint32_t* zero_also = nullptr;
@@ -177,11 +178,17 @@ tp_status run_gemm(const Operand& a, const Operand& b, int64_t M, int64_t N, int
   gp.grp_mbp = opts.grp_mbp;
   gp.grp_n = opts.grp_n;
   gp.grp_div = opts.grp_div > 0 ? opts.grp_div : 1;
+  gp.grp_swap = opts.grp_swap ? 1 : 0;
   if (opts.grp_cnt && opts.grp_sum) gp.sum_batch = 1;
-  if (opts.grp_cnt && (sk || Cfg::A_MN || Cfg::A_ROWS != 128 || !opts.grp_off || !opts.grp_mbp ||
-                       opts.grp_n < 1 || batch != static_cast<int64_t>(opts.grp_n) * gp.grp_div))
+  if (opts.grp_cnt && (sk || Cfg::A_MN || !opts.grp_off || !opts.grp_mbp || opts.grp_n < 1 ||
+                       batch != static_cast<int64_t>(opts.grp_n) * gp.grp_div))
     return set_error(TP_ERR_INVALID_ARG,
-                     "grouped GEMM: whole 128-row tiles, K-major A, n groups x grp_div problems");
+                     "grouped GEMM: whole tiles, K-major A, n groups x grp_div problems");
+  if (opts.grp_cnt && !opts.grp_swap && Cfg::A_ROWS != 128)
+    return set_error(TP_ERR_INVALID_ARG, "grouped GEMM: the groups' rows come in 128-row tiles");
+  if (opts.grp_cnt && opts.grp_swap && (Cfg::BN != 128 || Cfg::B_MN))
+    return set_error(TP_ERR_INVALID_ARG,
+                     "swapped grouped GEMM: the groups' rows come in 128-row K-major B tiles");
   int grid_sk = 0;
   if (sk) {
     const SkPlan pl = plan_stream_k<Cfg>(M, N, K, batch, sk->sum_batch, num_sms());

@@ -114,6 +114,11 @@ struct GemmParams {
   const int32_t* grp_mbp;
   int32_t grp_n;
   int32_t grp_div;
+  // Swapped grouped problems: the group ranges run along N (B = the gathered rows, A = problem
+  // b's weights at A batch coordinate b); grp_mbp then counts BN-row blocks, the tile space is
+  // (block of all groups' blocks, [problem of the group,] m block), and each tile's MMAs take
+  // N = its block's rows rounded up to 16.
+  int32_t grp_swap;
 };
 
 // One accumulator's worth of work.
@@ -126,7 +131,9 @@ struct Seg {
   int rot;        // the k loop visits kb0 + (i + rot) % (kb1 - kb0), i = 0, 1, ...
   int ab;         // A batch coordinate
   int row0;       // first A row of the problem (grouped), else 0
-  int row_end;    // end of the problem's A rows (grouped), else INT32_MAX
+  int n_off;      // first B row of the problem (swapped grouped), else 0
+  int row_end;    // end of the problem's gathered rows (A rows, or B rows when swapped);
+                  // INT32_MAX when ungrouped
 };
 
 // What the epilogue of one tile sees.
@@ -135,7 +142,8 @@ struct EpiCtx {
   int b;            // problem index (0 when the problems were summed; A batch when grouped)
   int m0;           // first A row of the tile
   int n0;           // first B row of the tile
-  int row_end = 0x7fffffff;   // A rows at or past this belong to no problem of the tile
+  int row_end = 0x7fffffff;   // gathered rows (A rows, or B rows when swapped) at or past this
+                              // belong to no problem of the tile
 };
 
 __device__ __forceinline__ void decode_mn(int r, const GemmParams& gp, int& mb, int& nb) {
@@ -177,7 +185,7 @@ struct SegIter {
     } else if (gp.grp_cnt) {
       u = cta;
       end = static_cast<int64_t>(gp.grp_mbp[gp.grp_n]) * (gp.sum_batch ? 1 : gp.grp_div) *
-            gp.n_blocks;
+            (gp.grp_swap ? gp.m_blocks : gp.n_blocks);
     } else {
       u = cta;
       end = num_groups(gp);
@@ -194,6 +202,7 @@ struct SegIter {
       decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
       s.ab = s.b;
       s.row0 = 0;
+      s.n_off = 0;
       s.row_end = 0x7fffffff;
       s.kb0 = 0;
       s.kb1 = gp.k_blocks;
@@ -206,27 +215,41 @@ struct SegIter {
       s.g = static_cast<int>(u);
       u += grid;
       if (gp.grp_cnt) {
-        s.nb = s.g % gp.n_blocks;
-        const int r = s.g / gp.n_blocks;
+        const int other = gp.grp_swap ? gp.m_blocks : gp.n_blocks;
+        const int ob = s.g % other;
+        const int r = s.g / other;
         const int i = gp.sum_batch ? 0 : r % gp.grp_div;
-        const int mbg = gp.sum_batch ? r : r / gp.grp_div;
-        int lo = 0, hi = gp.grp_n;   // the last group whose first block is <= mbg
+        const int bg = gp.sum_batch ? r : r / gp.grp_div;   // block among all groups' blocks
+        int lo = 0, hi = gp.grp_n;   // the last group whose first block is <= bg
         while (hi - lo > 1) {
           const int mid = (lo + hi) >> 1;
-          if (gp.grp_mbp[mid] <= mbg) lo = mid;
+          if (gp.grp_mbp[mid] <= bg) lo = mid;
           else hi = mid;
         }
-        s.mb = mbg - gp.grp_mbp[lo];
-        s.b = lo * gp.grp_div + i;
-        s.ab = i;
-        s.row0 = gp.grp_off[lo];
-        s.row_end = s.row0 + gp.grp_cnt[lo];
+        if (gp.grp_swap) {
+          // A = problem (lo, i)'s weights, B = the group's gathered rows (batch: i)
+          s.mb = ob;
+          s.nb = bg - gp.grp_mbp[lo];
+          s.b = i;
+          s.ab = lo * gp.grp_div + i;
+          s.row0 = 0;
+          s.n_off = gp.grp_off[lo];
+        } else {
+          s.nb = ob;
+          s.mb = bg - gp.grp_mbp[lo];
+          s.b = lo * gp.grp_div + i;
+          s.ab = i;
+          s.row0 = gp.grp_off[lo];
+          s.n_off = 0;
+        }
+        s.row_end = gp.grp_off[lo] + gp.grp_cnt[lo];
       } else {
         const int per = gp.m_blocks * gp.n_blocks;
         s.b = s.g / per;
         decode_mn(s.g - s.b * per, gp, s.mb, s.nb);
         s.ab = s.b;
         s.row0 = 0;
+        s.n_off = 0;
         s.row_end = 0x7fffffff;
       }
       s.kb0 = 0;
@@ -236,6 +259,7 @@ struct SegIter {
       return true;
     }
     s.row0 = 0;
+    s.n_off = 0;
     s.row_end = 0x7fffffff;
     const int64_t U = units_per_group(gp);
     const int64_t g = u / U, o = u - g * U;
@@ -492,7 +516,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       Seg sg;
       while (ok && it.next(gp, grid, sg)) {
         const int m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
-        const int n0 = sg.nb * Cfg::BN;
+        const int n0 = sg.n_off + sg.nb * Cfg::BN;
         const int nk = sg.kb1 - sg.kb0;
         for (int i = 0; i < nk; ++i) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
@@ -555,6 +579,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         tc_fence_after();
         const uint32_t d_base = tmem_base + acc * Cfg::ACC_COLS;
         const int nk = sg.kb1 - sg.kb0;
+        uint32_t idesc = Cfg::IDESC;
+        if (gp.grp_swap) {
+          // only the block's rows of the group: N = those rows rounded up to 16
+          const int left = sg.row_end - (sg.n_off + sg.nb * Cfg::BN);
+          const int n_mma = left >= Cfg::BN ? Cfg::BN : ((left + 15) & ~15);
+          idesc = make_idesc_bf16(128, n_mma < 16 ? 16 : n_mma, Cfg::A_MN, Cfg::B_MN);
+        }
         for (int i = 0; i < nk; ++i) {
           if (!mbar_wait(&full[stage], phase, abort_flag, gp.err, DEVERR_WAIT_FULL)) {
             ok = false;
@@ -574,8 +605,7 @@ __global__ void __launch_bounds__(kThreads, 1)
               const uint64_t adesc =
                   Cfg::A_MN ? make_sdesc_sw128(a_sub + kk * (kUmmaK * 128), 64 * kBK * 2, 1024)
                             : make_sdesc_sw128(a_sub + kk * (kUmmaK * 2), 16, 1024);
-              umma_f16(d_base + s * Cfg::BN, adesc, bdesc, Cfg::IDESC,
-                       (i > 0 || kk != 0) ? 1u : 0u);
+              umma_f16(d_base + s * Cfg::BN, adesc, bdesc, idesc, (i > 0 || kk != 0) ? 1u : 0u);
             }
           }
           issued_any = true;
@@ -622,7 +652,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctx.row = row;
       ctx.b = gp.sum_batch ? 0 : (gp.grp_cnt ? sg.ab : sg.b);
       ctx.m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
-      ctx.n0 = sg.nb * Cfg::BN;
+      ctx.n0 = sg.n_off + sg.nb * Cfg::BN;
       ctx.row_end = sg.row_end;
       // the tile is whole when all its k-blocks lie in this CTA's range (then it is one segment)
       const int64_t g0 = static_cast<int64_t>(sg.g) * U;
@@ -799,7 +829,7 @@ struct EpiHiddenT {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int t = c.n0 + col + e;
-            if (t < p.tokens) {
+            if (t < p.tokens && t < c.row_end) {
               p.h[t * p.ld_h + feat] = __float2bfloat16_rn(fast_silu(g[e]) * u[e]);
               if (p.z) {
                 p.z[t * p.ld_z + zg] = __float2bfloat16_rn(g[e]);
@@ -819,7 +849,7 @@ struct EpiHiddenT {
 #pragma unroll
           for (int e = 0; e < 16; ++e) {
             const int t = c.n0 + col + e;
-            if (t < p.tokens) {
+            if (t < p.tokens && t < c.row_end) {
               p.h[t * p.ld_h + r] = __float2bfloat16_rn(act_f(p.act, v[e]));
               if (p.z) p.z[t * p.ld_z + r] = __float2bfloat16_rn(v[e]);
             }
@@ -838,7 +868,7 @@ using EpiHiddenSwap = EpiHiddenT<1>;
 // gradients.  Non-swapped: i = m (A row), j = n.  Swapped: i = n (token), j = m (feature).
 // ---------------------------------------------------------------------------------------------
 struct EpiStoreF32 {
-  // requires Cfg::A_SUB == 1
+  // not swapped: requires Cfg::A_SUB == 1; swapped: sub-tile s holds A rows m0 + 128 s + row
   struct Params {
     float* out;
     int64_t ld;            // elements between rows
@@ -874,17 +904,20 @@ struct EpiStoreF32 {
         }
       }
     } else {
-      const int j = c.m0 + c.row;
-      const bool live = j < p.cols_valid;
 #pragma unroll 1
-      for (int col = 0; col < Cfg::BN; col += 16) {
-        float v[16];
-        src.load16(col, v);
-        if (live) {
+      for (int sub = 0; sub < Cfg::A_SUB; ++sub) {
+        const int j = c.m0 + sub * 128 + c.row;
+        const bool live = j < p.cols_valid;
+#pragma unroll 1
+        for (int col = 0; col < Cfg::BN; col += 16) {
+          float v[16];
+          src.load16(sub * Cfg::BN + col, v);
+          if (live) {
 #pragma unroll
-          for (int e = 0; e < 16; ++e) {
-            const int i = c.n0 + col + e;
-            if (i < p.rows_valid) base[i * p.ld + j] = v[e];
+            for (int e = 0; e < 16; ++e) {
+              const int i = c.n0 + col + e;
+              if (i < p.rows_valid && i < c.row_end) base[i * p.ld + j] = v[e];
+            }
           }
         }
       }

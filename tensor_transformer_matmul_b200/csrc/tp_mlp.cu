@@ -1119,10 +1119,13 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
                   static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(perm), M.k,
                   M.d, xs);
   }
-  // (5) grouped up GEMM + SwiGLU over all experts: rows of expert e are xs[off[e] .. +cnt[e])
+  // (5) grouped up GEMM + SwiGLU over all experts: rows of expert e are xs[off[e] .. +cnt[e]).
+  // Swapped: each tile is 256 packed rows of one expert's W1 (128 gate + 128 up features) times
+  // up to 128 of its routed rows, the MMA width cut to that block's rows rounded up to 16, so an
+  // expert's last block costs its rows rather than a full tile.
   {
     const int64_t rows = L.p * L.R;
-    tc::EpiHidden::Params ep;
+    tc::EpiHiddenParams ep;
     ep.h = hs;
     ep.z = nullptr;
     ep.ld_h = L.p * L.Fsp;
@@ -1130,21 +1133,24 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
     ep.tokens = static_cast<int32_t>(M.n_rows);
     ep.rows = static_cast<int32_t>(rows);
     ep.act = TP_ACT_SWIGLU;
-    ep.swap = 0;
-    const Operand ao{xs, false, M.n_rows, M.d, 1, M.d, 0};
-    const Operand bo{w1p, false, rows, M.d, M.E, M.d, rows * M.d};
+    ep.swap = 1;
+    const Operand wo{w1p, false, rows, M.d, M.E, M.d, rows * M.d};
+    const Operand xo{xs, false, M.n_rows, M.d, 1, M.d, 0};
     tc::GemmOpts opt;
     opt.grp_cnt = cnt;
     opt.grp_off = offs;
     opt.grp_mbp = mbp;
     opt.grp_n = M.E;
     opt.grp_div = 1;
-    st = tc::run_gemm<KK<256, 1>, tc::EpiHidden>(ao, bo, M.T, rows, M.d, M.E, ep, s,
-                                                 "moe_up_gemm", opt);
+    opt.grp_swap = true;
+    st = tc::run_gemm<TileCfg<128, 2, false, false, stages_for(128, 2)>, tc::EpiHiddenSwap>(
+        wo, xo, rows, M.T, M.d, M.E, ep, s, "moe_up_gemm", opt);
     if (st != TP_OK) return st;
   }
   // (6) grouped down GEMM: problem e * p + i = expert e, shard i; each tile runs shard 0..p-1's
-  // k-blocks into one accumulator, so the routed rows leave with their shards summed: [row][d]
+  // k-blocks into one accumulator, so the routed rows leave with their shards summed: [row][d].
+  // Swapped like the up GEMM: 256 rows of W2 (output features, two 128-row MMAs) times up to 128
+  // routed rows.
   {
     const Operand ho{hs, false, M.n_rows, L.Fsp, L.p, L.p * L.Fsp, L.Fsp};
     const Operand wo{w2p, false, M.d, L.Fsp, static_cast<int64_t>(M.E) * L.p, L.Fsp, M.d * L.Fsp};
@@ -1154,7 +1160,7 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
     ep.batch_stride = 0;
     ep.rows_valid = static_cast<int32_t>(M.n_rows);
     ep.cols_valid = static_cast<int32_t>(M.d);
-    ep.swap = 0;
+    ep.swap = 1;
     tc::GemmOpts opt;
     opt.grp_cnt = cnt;
     opt.grp_off = offs;
@@ -1162,9 +1168,9 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
     opt.grp_n = M.E;
     opt.grp_div = L.p;
     opt.grp_sum = true;
-    st = tc::run_gemm<KK<256, 1>, tc::EpiStoreF32>(ho, wo, M.T, M.d, L.Fsp,
-                                                   static_cast<int64_t>(M.E) * L.p, ep, s,
-                                                   "moe_down_gemm", opt);
+    opt.grp_swap = true;
+    st = tc::run_gemm<TileCfg<128, 2, false, false, stages_for(128, 2)>, tc::EpiStoreF32>(
+        wo, ho, M.d, M.T, L.Fsp, static_cast<int64_t>(M.E) * L.p, ep, s, "moe_down_gemm", opt);
     if (st != TP_OK) return st;
   }
   // (7) the shared expert over all tokens, its p shards summed in its down GEMM: [T][d] fp32
