@@ -48,28 +48,28 @@ __global__ void __launch_bounds__(256) router_simt_kernel(const __nv_bfloat16* _
   }
 }
 
-// One thread per token: the k largest logits (descending; among equal logits the lower expert
-// index first) and their softmax.
+// One warp per token: the k largest logits (descending; among equal logits the lower expert
+// index first) and their softmax.  Lane L reads logits L, L + 32, ... (coalesced across the warp)
+// and keeps its own k largest in that order; then k rounds of a warp-wide maximum (ties: the
+// lower index) take the next entry from the lane that holds it.  The result, and the softmax
+// computed from it by lane 0 in choice order, are those of a sequential scan over all E logits.
 __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ logits, int64_t T,
                                                    int E, int k, int32_t* __restrict__ idx,
                                                    float* __restrict__ w) {
   pdl_wait();
   pdl_trigger();
-  const int64_t t = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (t >= T) return;
+  const int lane = threadIdx.x & 31;
+  const int64_t t = static_cast<int64_t>(blockIdx.x) * (blockDim.x >> 5) + (threadIdx.x >> 5);
+  if (t >= T) return;   // warp-uniform
   const float* l = logits + t * E;
   float best[kMaxTopK];
   int bi[kMaxTopK];
-#pragma unroll
-  for (int j = 0; j < kMaxTopK; ++j) {
-    best[j] = -INFINITY;
-    bi[j] = j;
-  }
-  for (int e = 0; e < E; ++e) {
+  int nkept = 0;
+  for (int e = lane; e < E; e += 32) {
     const float v = l[e];
-    if (!(v > best[k - 1]) && e >= k) continue;   // not above the k-th (ties keep the lower index)
-    // insertion: after every kept entry with a logit >= v
-    int pos = k - 1;
+    if (nkept == k && !(v > best[k - 1])) continue;   // not above this lane's k-th
+    // insertion after every kept entry with a logit >= v (this lane's indices ascend)
+    int pos = nkept < k ? nkept : k - 1;
     while (pos > 0 && best[pos - 1] < v) {
       best[pos] = best[pos - 1];
       bi[pos] = bi[pos - 1];
@@ -77,15 +77,37 @@ __global__ void __launch_bounds__(256) topk_kernel(const float* __restrict__ log
     }
     best[pos] = v;
     bi[pos] = e;
+    if (nkept < k) ++nkept;
   }
-  float s = 0.f, ex[kMaxTopK];
+  int head = 0;
+  float ch_v[kMaxTopK];
+  int ch_i[kMaxTopK];
   for (int j = 0; j < k; ++j) {
-    ex[j] = expf(best[j] - best[0]);
-    s += ex[j];
+    float v = head < nkept ? best[head] : -INFINITY;
+    int i = head < nkept ? bi[head] : 0x7fffffff;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float ov = __shfl_xor_sync(0xffffffffu, v, o);
+      const int oi = __shfl_xor_sync(0xffffffffu, i, o);
+      if (ov > v || (ov == v && oi < i)) {
+        v = ov;
+        i = oi;
+      }
+    }
+    ch_v[j] = v;
+    ch_i[j] = i;
+    if (head < nkept && bi[head] == i) ++head;   // the lane that held it moves on
   }
-  for (int j = 0; j < k; ++j) {
-    idx[t * k + j] = bi[j];
-    w[t * k + j] = ex[j] / s;
+  if (lane == 0) {
+    float s = 0.f, ex[kMaxTopK];
+    for (int j = 0; j < k; ++j) {
+      ex[j] = expf(ch_v[j] - ch_v[0]);
+      s += ex[j];
+    }
+    for (int j = 0; j < k; ++j) {
+      idx[t * k + j] = ch_i[j];
+      w[t * k + j] = ex[j] / s;
+    }
   }
 }
 

@@ -1108,7 +1108,7 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
   // (2) top-k and weights; (3) per-expert counts, offsets and stable positions; (4) gather
   {
     ProfScope prof(s, "moe_route");
-    TP_LAUNCH_PDL(moe::topk_kernel, dim3(static_cast<unsigned>(ceil_div(M.T, 256))), dim3(256), 0,
+    TP_LAUNCH_PDL(moe::topk_kernel, dim3(static_cast<unsigned>(ceil_div(M.T, 8))), dim3(256), 0,
                   s, logits, M.T, M.E, M.k, idx, wts);
     TP_LAUNCH_PDL(moe::count_kernel, dim3(static_cast<unsigned>(M.E)), dim3(1024), 0, s,
                   static_cast<const int32_t*>(idx), M.n_rows, cnt);
