@@ -13,10 +13,13 @@
 // 128 threads, thread t owning query row t of the tile (TMEM lane t).  Thread 0 also issues the
 // TMA loads and the MMAs.  Key blocks are 128 keys, so every MMA is 128 x 128.  S and P share 128
 // TMEM columns (the bf16 P of a block is written over its S and read from there as the A operand
-// of P V, so P never touches shared memory) and O takes the other 128.  Q, K and V each have one
-// shared-memory buffer: K(kb+1) is fetched as soon as S(kb) is done, V(kb+1) as soon as P(kb)
-// V(kb) is done, each well ahead of its use.  A CTA needs 96 KB of shared memory and 256 TMEM
-// columns, so two CTAs share an SM and one's softmax runs while the other's MMAs do.
+// of P V, so P never touches shared memory) and O takes the other 128.  Thread 0 issues
+// S(kb+1) = Q K(kb+1)^T right behind P(kb) V(kb): the MMAs of a CTA run in issue order, so S(kb+1)
+// overwrites P(kb) only after P(kb) V(kb) has read it, and S(kb+1) done means P(kb) V(kb) is done
+// too.  Q, K and V each have one shared-memory buffer: K(kb+1) is fetched as soon as S(kb) is
+// done, V(kb+1) as soon as S(kb+1) is, each well ahead of its use.  A CTA needs 96 KB of shared
+// memory and 256 TMEM columns, so two CTAs share an SM and one's softmax runs while the other's
+// MMAs do.
 //
 // The special-function unit computes 16 exponentials per clock per SM, which for this tile shape
 // is as slow as the tensor core, so three pairs of P values in eight are computed on the FMA pipe:
@@ -208,6 +211,9 @@ __global__ void __launch_bounds__(kThreads, 2)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
+  // everything above may overlap the previous kernel's tail; global memory only from here on
+  pdl_wait();
+  pdl_trigger();
   const uint32_t tS = tmem, tO = tmem + 128;
   const uint32_t lane_base = static_cast<uint32_t>(warp * 32) << 16;
 
@@ -268,15 +274,20 @@ __global__ void __launch_bounds__(kThreads, 2)
   float m_run = -INFINITY, l_run = 0.f;
   for (int kb = 0; kb < nkb; ++kb) {
     const uint32_t par = kb & 1;
+    // S(kb) done: the MMAs run in issue order, so P(kb-1) V(kb-1) is done too and O is final
+    // for a rescale
     ok = __all_sync(0xffffffffu, wait(s_full, par, DEVERR_WAIT_ACC_FULL));
-    // O holds P(kb-1) V(kb-1) (S(kb) was issued after it completed; waited here for ordering)
-    if (ok && kb > 0)
-      ok = __all_sync(0xffffffffu, wait(pv_done, par ^ 1, DEVERR_WAIT_ACC_EMPTY));
     if (!ok) break;
     tc_fence_after();
-    if (tid == 0 && kb + 1 < nkb) {   // K buffer is free once S(kb) is done
-      load_block(k_full, sK, k_col, (kb + 1) * kKeys);
-      ++n_k;
+    if (tid == 0) {
+      if (kb + 1 < nkb) {   // the K buffer is free once S(kb) is done
+        load_block(k_full, sK, k_col, (kb + 1) * kKeys);
+        ++n_k;
+      }
+      if (kb > 0) {         // and the V buffer once P(kb-1) V(kb-1) is
+        load_block(v_full, sV, v_col, kb * kKeys);
+        ++n_v;
+      }
     }
     float sv[kKeys];
     {
@@ -359,19 +370,11 @@ __global__ void __launch_bounds__(kThreads, 2)
     tc_fence_before();
     mbar_arrive(p_full);
     if (tid == 0) {
-      // every row has stored P(kb) and rescaled O: O += P(kb) V(kb); then, once that is done
-      // (it reads P from the S columns), V(kb+1) and S(kb+1)
+      // every row has stored P(kb) and rescaled O: O += P(kb) V(kb), and right behind it S(kb+1),
+      // which overwrites P(kb) only after P(kb) V(kb) has read it (issue order)
       bool t = wait(p_full, par, DEVERR_WAIT_ACC_FULL) && wait(v_full, par, DEVERR_WAIT_FULL);
       if (t) issue_pv(kb);
-      if (t && kb + 1 < nkb) {
-        t = wait(pv_done, par, DEVERR_WAIT_ACC_EMPTY) &&
-            wait(k_full, (kb + 1) & 1, DEVERR_WAIT_FULL);
-        if (t) {
-          issue_s();
-          load_block(v_full, sV, v_col, (kb + 1) * kKeys);   // V is free once P(kb) V(kb) is done
-          ++n_v;
-        }
-      }
+      if (t && kb + 1 < nkb && wait(k_full, (kb + 1) & 1, DEVERR_WAIT_FULL)) issue_s();
     }
   }
   tmem_wait_st();
@@ -462,8 +465,8 @@ inline tp_status launch(const void* qkv, int64_t b, int64_t s, int n_q, int qh, 
   P.err = device_error_word();
   dim3 grid(static_cast<unsigned>(n_q), static_cast<unsigned>(P.n_qt), static_cast<unsigned>(b));
   ProfScope prof(st, "attn_prefill");
-  flash_fwd_kernel<HD><<<grid, kThreads, L::BYTES, st>>>(map, P);
-  TP_LAUNCH_CHECK();
+  TP_LAUNCH_PDL(flash_fwd_kernel<HD>, grid, dim3(kThreads), static_cast<size_t>(L::BYTES), st,
+                map, P);
   return TP_OK;
 }
 
