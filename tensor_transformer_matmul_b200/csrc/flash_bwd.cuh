@@ -20,6 +20,9 @@
 //     and one half of the 128 keys each) write dS back over S, and dQ += dS K accumulates in
 //     TMEM (K read MN-major).  K and V are double buffered.
 // Thread 0 issues the TMA loads and the MMAs; TMEM holds four (three) 128-column fp32 tiles.
+// The next step's S^T/dP^T (S/dP) MMAs are issued right behind this step's dV/dK (dQ) MMAs: the
+// MMAs run in issue order, so they overwrite P^T and dS^T (dS) only after those have been read,
+// and their completion also means the previous step's MMAs are done.
 // The two thread halves (warps 0-3 and 4-7) read the same TMEM lanes, columns 0-63 and 64-127;
 // half h packs its 64 bf16 results into columns 64 h .. 64 h + 31, which only it reads, so the
 // halves need no ordering between them.  The MMA that consumes them takes queries (keys)
@@ -192,6 +195,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ++nq[b];
   };
+  // S^T = K Q(it)^T and dP^T = V dO(it)^T (thread 0)
+  auto issue_s = [&](int it) {
+    const int b = it & 1;
+    const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ + b * L::BLOCK),
+                   da = smem_addr(sDO + b * L::BLOCK);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
+      umma_f16(tS, make_sdesc_sw128(ka + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
+               IDESC_KK, kk > 0 ? 1u : 0u);
+      umma_f16(tdP, make_sdesc_sw128(va + off, 16, 1024), make_sdesc_sw128(da + off, 16, 1024),
+               IDESC_KK, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(s_full);
+    any_mma = true;
+  };
+  bool ok = true;
   if (tid == 0) {
     mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
 #pragma unroll
@@ -201,14 +221,17 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     load_qd(0);
     if (n_iter > 1) load_qd(1);
+    ok = wait(&qd_full[0], 0, DEVERR_WAIT_FULL) && wait(kv_full, 0, DEVERR_WAIT_FULL);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+    }
   }
-  bool ok = true;
   for (int it = 0; it < n_iter; ++it) {
     if (!__syncthreads_and(ok ? 1 : 0)) {   // everyone is done with the previous step
       ok = false;
       break;
     }
-    const int b = it & 1;
     const int j = head_of(it);
     const int q0 = block_of(it) * kBlk;
     if (tid < kBlk) {
@@ -219,33 +242,13 @@ __global__ void __launch_bounds__(kThreads, 1)
       D_s[tid] = valid ? P.D[ri] : 0.f;
     }
     __syncthreads();
-    if (tid == 0 && ok) {
-      // S^T and dP^T overwrite P^T, dS^T of the previous step: wait for its MMAs (which also
-      // frees the other Q/dO buffer for the step after this one)
-      if (it > 0) ok = wait(m_done, (it - 1) & 1, DEVERR_WAIT_ACC_EMPTY);
-      if (ok && it >= 1 && it + 1 < n_iter) load_qd(it + 1);
-      if (ok) ok = wait(&qd_full[b], (it >> 1) & 1, DEVERR_WAIT_FULL) &&
-                   (it > 0 || wait(kv_full, 0, DEVERR_WAIT_FULL));
-      if (ok) {
-        tc_fence_after();
-        const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ + b * L::BLOCK),
-                       da = smem_addr(sDO + b * L::BLOCK);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
-          umma_f16(tS, make_sdesc_sw128(ka + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
-                   IDESC_KK, kk > 0 ? 1u : 0u);
-          umma_f16(tdP, make_sdesc_sw128(va + off, 16, 1024),
-                   make_sdesc_sw128(da + off, 16, 1024), IDESC_KK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
-        any_mma = true;
-      }
-    }
     // ---- P^T and dS^T for this key row against this thread's 64 of the block's queries,
     // written as bf16 over the first half of this half's TMEM columns (chunks in ascending
     // order: a chunk's S and dP are read before any later chunk's columns are overwritten)
+    // S^T(it) done: the MMAs run in issue order, so dV/dK of the previous step are done too and
+    // the other Q/dO buffer is free for step it+1
     ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
+    if (ok && tid == 0 && it >= 1 && it + 1 < n_iter) load_qd(it + 1);
     if (ok) {
       tc_fence_after();
       // no mask inside the block: every query is valid and (causal) after every key
@@ -283,6 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait(p_ready, it & 1, DEVERR_WAIT_ACC_FULL);
       if (ok) {
         tc_fence_after();
+        const int b = it & 1;
         const uint32_t qa = smem_addr(sQ + b * L::BLOCK), da = smem_addr(sDO + b * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
@@ -296,6 +300,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                               (it > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
+        // the next step's S^T and dP^T right behind: they overwrite P^T and dS^T only after
+        // these MMAs have read them (issue order)
+        if (it + 1 < n_iter) {
+          ok = wait(&qd_full[(it + 1) & 1], ((it + 1) >> 1) & 1, DEVERR_WAIT_FULL);
+          if (ok) {
+            tc_fence_after();
+            issue_s(it + 1);
+          }
+        }
       }
     }
   }
@@ -439,6 +452,23 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     ++nk[b];
   };
+  // S = Q K(kb)^T and dP = dO V(kb)^T (thread 0)
+  auto issue_s = [&](int kb) {
+    const int b = kb & 1;
+    const uint32_t qa = smem_addr(sQ), da = smem_addr(sDO), ka = smem_addr(sK + b * L::BLOCK),
+                   va = smem_addr(sV + b * L::BLOCK);
+#pragma unroll
+    for (int kk = 0; kk < HD / 16; ++kk) {
+      const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
+      umma_f16(tS, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
+               IDESC_KK, kk > 0 ? 1u : 0u);
+      umma_f16(tdP, make_sdesc_sw128(da + off, 16, 1024), make_sdesc_sw128(va + off, 16, 1024),
+               IDESC_KK, kk > 0 ? 1u : 0u);
+    }
+    umma_commit(s_full);
+    any_mma = true;
+  };
+  bool ok = true;
   if (tid == 0) {
     mbar_arrive_expect_tx(qd_full, 2 * L::BLOCK);
 #pragma unroll
@@ -448,42 +478,25 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
     load_kv(0);
     if (nkb > 1) load_kv(1);
+    ok = wait(&kv_full[0], 0, DEVERR_WAIT_FULL) && wait(qd_full, 0, DEVERR_WAIT_FULL);
+    if (ok) {
+      tc_fence_after();
+      issue_s(0);
+    }
   }
-  bool ok = true;
   for (int kb = 0; kb < nkb; ++kb) {
     if (!__syncthreads_and(ok ? 1 : 0)) {
       ok = false;
       break;
     }
-    const int b = kb & 1;
     const int k0 = kb * kBlk;
-    if (tid == 0 && ok) {
-      // S and dP overwrite dS of the previous step: wait for its MMA (which also frees the
-      // other K/V buffer for the step after this one)
-      if (kb > 0) ok = wait(m_done, (kb - 1) & 1, DEVERR_WAIT_ACC_EMPTY);
-      if (ok && kb >= 1 && kb + 1 < nkb) load_kv(kb + 1);
-      if (ok) ok = wait(&kv_full[b], (kb >> 1) & 1, DEVERR_WAIT_FULL) &&
-                   (kb > 0 || wait(qd_full, 0, DEVERR_WAIT_FULL));
-      if (ok) {
-        tc_fence_after();
-        const uint32_t qa = smem_addr(sQ), da = smem_addr(sDO), ka = smem_addr(sK + b * L::BLOCK),
-                       va = smem_addr(sV + b * L::BLOCK);
-#pragma unroll
-        for (int kk = 0; kk < HD / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
-          umma_f16(tS, make_sdesc_sw128(qa + off, 16, 1024), make_sdesc_sw128(ka + off, 16, 1024),
-                   IDESC_KK, kk > 0 ? 1u : 0u);
-          umma_f16(tdP, make_sdesc_sw128(da + off, 16, 1024),
-                   make_sdesc_sw128(va + off, 16, 1024), IDESC_KK, kk > 0 ? 1u : 0u);
-        }
-        umma_commit(s_full);
-        any_mma = true;
-      }
-    }
     // ---- dS for this query row against this thread's 64 of the block's 128 keys, bf16 over
     // the first half of this half's S columns (ascending chunks: a chunk is read before any
     // later chunk is overwritten)
+    // S(kb) done: the MMAs run in issue order, so dQ of the previous step is done too and the
+    // other K/V buffer is free for step kb+1
     ok = __all_sync(0xffffffffu, ok && wait(s_full, kb & 1, DEVERR_WAIT_ACC_FULL));
+    if (ok && tid == 0 && kb >= 1 && kb + 1 < nkb) load_kv(kb + 1);
     if (ok) {
       tc_fence_after();
       // no mask inside the block: every key is valid and (causal) before every query
@@ -518,7 +531,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ok = wait(p_ready, kb & 1, DEVERR_WAIT_ACC_FULL);
       if (ok) {
         tc_fence_after();
-        const uint32_t ka = smem_addr(sK + b * L::BLOCK);
+        const uint32_t ka = smem_addr(sK + (kb & 1) * L::BLOCK);
 #pragma unroll
         for (int kk = 0; kk < kBlk / 16; ++kk) {
           // A: 16 keys = 8 TMEM columns of dS; B: the [key][dim] K tile read MN-major
@@ -527,6 +540,15 @@ __global__ void __launch_bounds__(kThreads, 1)
                               (kb > 0 || kk > 0) ? 1u : 0u);
         }
         umma_commit(m_done);
+        // the next step's S and dP right behind: they overwrite dS only after this MMA has read
+        // it (issue order)
+        if (kb + 1 < nkb) {
+          ok = wait(&kv_full[(kb + 1) & 1], ((kb + 1) >> 1) & 1, DEVERR_WAIT_FULL);
+          if (ok) {
+            tc_fence_after();
+            issue_s(kb + 1);
+          }
+        }
       }
     }
   }
