@@ -123,16 +123,15 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* sV = sK + L::BLOCK;
   uint8_t* sQ = sV + L::BLOCK;        // [2] buffers
   uint8_t* sDO = sQ + 2 * L::BLOCK;   // [2] buffers
-  float* lse_s = reinterpret_cast<float*>(sDO + 2 * L::BLOCK);
-  float* D_s = lse_s + kBlk;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + kBlk);
+  float* lse_s = reinterpret_cast<float*>(sDO + 2 * L::BLOCK);   // [2][kBlk]
+  float* D_s = lse_s + 2 * kBlk;                                   // [2][kBlk]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + 2 * kBlk);
   uint64_t* kv_full = bar + 0;
   uint64_t* qd_full = bar + 1;   // [2]
   uint64_t* s_full = bar + 3;
-  uint64_t* p_ready = bar + 4;
-  uint64_t* m_done = bar + 5;
-  uint64_t* drain = bar + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 7);
+  uint64_t* m_done = bar + 4;
+  uint64_t* drain = bar + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -152,7 +151,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&qd_full[0], 1);
     mbar_init(&qd_full[1], 1);
     mbar_init(s_full, 1);
-    mbar_init(p_ready, kThreads);
     mbar_init(m_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -211,6 +209,21 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma_commit(s_full);
     any_mma = true;
   };
+  // log-sum-exp and D of a step's 128 queries, double-buffered in shared memory: thread t < 128
+  // loads step it+1's pair while step it runs and stores it before the step's barrier
+  auto row_data = [&](int it, float& l, float& dd) {
+    const int t_abs = block_of(it) * kBlk + tid;
+    const bool valid = t_abs < P.s;
+    const int64_t ri = (static_cast<int64_t>(bi) * P.s + t_abs) * P.n_q + head_of(it);
+    l = valid ? P.lse[ri] : 0.f;
+    dd = valid ? P.D[ri] : 0.f;
+  };
+  if (tid < kBlk) {
+    float l, dd;
+    row_data(0, l, dd);
+    lse_s[tid] = l;
+    D_s[tid] = dd;
+  }
   bool ok = true;
   if (tid == 0) {
     mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
@@ -227,87 +240,101 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_s(0);
     }
   }
+  __syncthreads();
   for (int it = 0; it < n_iter; ++it) {
-    if (!__syncthreads_and(ok ? 1 : 0)) {   // everyone is done with the previous step
-      ok = false;
-      break;
-    }
-    const int j = head_of(it);
     const int q0 = block_of(it) * kBlk;
-    if (tid < kBlk) {
-      const int t_abs = q0 + tid;
-      const bool valid = t_abs < P.s;
-      const int64_t ri = (static_cast<int64_t>(bi) * P.s + t_abs) * P.n_q + j;
-      lse_s[tid] = valid ? P.lse[ri] : 0.f;
-      D_s[tid] = valid ? P.D[ri] : 0.f;
-    }
-    __syncthreads();
-    // ---- P^T and dS^T for this key row against this thread's 64 of the block's queries,
-    // written as bf16 over the first half of this half's TMEM columns (chunks in ascending
-    // order: a chunk's S and dP are read before any later chunk's columns are overwritten)
+    const float* lse_c = lse_s + (it & 1) * kBlk;
+    const float* D_c = D_s + (it & 1) * kBlk;
+    float nl = 0.f, nd = 0.f;
+    if (tid < kBlk && it + 1 < n_iter) row_data(it + 1, nl, nd);
     // S^T(it) done: the MMAs run in issue order, so dV/dK of the previous step are done too and
     // the other Q/dO buffer is free for step it+1
     ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
     if (ok && tid == 0 && it >= 1 && it + 1 < n_iter) load_qd(it + 1);
+    // ---- P^T and dS^T for this key row against this thread's 64 of the block's queries,
+    // written as bf16 over the first half of this half's TMEM columns (all of this thread's S
+    // and dP are read before any of them is overwritten)
     if (ok) {
       tc_fence_after();
       // no mask inside the block: every query is valid and (causal) after every key
       const bool plain = q0 + kBlk <= P.s && k0 + kBlk <= P.s && (!P.causal || q0 > k0);
-#pragma unroll 1
-      for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-        float sv[32], dp[32];
-        ld32(tS + lane_base + c0, sv);
-        ld32(tdP + lane_base + c0, dp);
+      float sv[64], dp[64];
+      {
+        uint32_t r[4][32];
+        tmem_ld_32x32b_x32(tS + lane_base + 64 * half, r[0]);
+        tmem_ld_32x32b_x32(tS + lane_base + 64 * half + 32, r[1]);
+        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half, r[2]);
+        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half + 32, r[3]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          sv[e] = __uint_as_float(r[e >> 5][e & 31]);
+          dp[e] = __uint_as_float(r[2 + (e >> 5)][e & 31]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int c0 = 64 * half + 32 * c;
         uint32_t pw[16], dw[16];
 #pragma unroll
-        for (int e = 0; e < 32; e += 2) {
-          float pr[2], ds[2];
+        for (int e = 0; e < 32; e += 4) {
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_c + c0 + e);
+          const float4 d4 = *reinterpret_cast<const float4*>(D_c + c0 + e);
+          const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
+          float pr[4], ds[4];
 #pragma unroll
-          for (int u = 0; u < 2; ++u) {
+          for (int u = 0; u < 4; ++u) {
             const int qi = c0 + e + u;
-            pr[u] = exp2_fast(sv[e + u] * P.scale_log2 - lse_s[qi]);
+            pr[u] = exp2_fast(sv[32 * c + e + u] * P.scale_log2 - lv[u]);
             if (!plain) {
               const int q_abs = q0 + qi;
               if (q_abs >= P.s || k_abs >= P.s || (P.causal && k_abs > q_abs)) pr[u] = 0.f;
             }
-            ds[u] = pr[u] * (dp[e + u] - D_s[qi]);
+            ds[u] = pr[u] * (dp[32 * c + e + u] - dv[u]);
           }
           pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
+          pw[(e >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
+          dw[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
         st16(tS + lane_base + packed_col(c0 / 2), pw);
         st16(tdP + lane_base + packed_col(c0 / 2), dw);
       }
       fa::tmem_wait_st();
     }
+    if (tid < kBlk && it + 1 < n_iter) {
+      lse_s[((it + 1) & 1) * kBlk + tid] = nl;
+      D_s[((it + 1) & 1) * kBlk + tid] = nd;
+    }
     tc_fence_before();
-    mbar_arrive(p_ready);
-    if (tid == 0 && ok) {
-      ok = wait(p_ready, it & 1, DEVERR_WAIT_ACC_FULL);
-      if (ok) {
-        tc_fence_after();
-        const int b = it & 1;
-        const uint32_t qa = smem_addr(sQ + b * L::BLOCK), da = smem_addr(sDO + b * L::BLOCK);
+    // every thread's P^T and dS^T (and the next step's row data) are stored; all agree on ok
+    if (!__syncthreads_and(ok ? 1 : 0)) {
+      ok = false;
+      break;
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      const int b = it & 1;
+      const uint32_t qa = smem_addr(sQ + b * L::BLOCK), da = smem_addr(sDO + b * L::BLOCK);
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
-          // MN-major (N = dim), 16 query rows per MMA
-          fa::umma_f16_tmem_a(tdV, tS + packed_col(kk * 8),
-                              make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                              (it > 0 || kk > 0) ? 1u : 0u);
-          fa::umma_f16_tmem_a(tdK, tdP + packed_col(kk * 8),
-                              make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                              (it > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(m_done);
-        // the next step's S^T and dP^T right behind: they overwrite P^T and dS^T only after
-        // these MMAs have read them (issue order)
-        if (it + 1 < n_iter) {
-          ok = wait(&qd_full[(it + 1) & 1], ((it + 1) >> 1) & 1, DEVERR_WAIT_FULL);
-          if (ok) {
-            tc_fence_after();
-            issue_s(it + 1);
-          }
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
+        // MN-major (N = dim), 16 query rows per MMA
+        fa::umma_f16_tmem_a(tdV, tS + packed_col(kk * 8),
+                            make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                            (it > 0 || kk > 0) ? 1u : 0u);
+        fa::umma_f16_tmem_a(tdK, tdP + packed_col(kk * 8),
+                            make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                            (it > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(m_done);
+      // the next step's S^T and dP^T right behind: they overwrite P^T and dS^T only after
+      // these MMAs have read them (issue order)
+      if (it + 1 < n_iter) {
+        ok = wait(&qd_full[(it + 1) & 1], ((it + 1) >> 1) & 1, DEVERR_WAIT_FULL);
+        if (ok) {
+          tc_fence_after();
+          issue_s(it + 1);
         }
       }
     }
@@ -385,10 +412,9 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* qd_full = bar + 0;
   uint64_t* kv_full = bar + 1;       // [2]
   uint64_t* s_full = bar + 3;
-  uint64_t* p_ready = bar + 4;
-  uint64_t* m_done = bar + 5;
-  uint64_t* drain = bar + 6;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 7);
+  uint64_t* m_done = bar + 4;
+  uint64_t* drain = bar + 5;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -407,7 +433,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     mbar_init(&kv_full[0], 1);
     mbar_init(&kv_full[1], 1);
     mbar_init(s_full, 1);
-    mbar_init(p_ready, kThreads);
     mbar_init(m_done, 1);
     mbar_init(drain, 1);
     *abort_flag = 0;
@@ -484,40 +509,49 @@ __global__ void __launch_bounds__(kThreads, 1)
       issue_s(0);
     }
   }
+  __syncthreads();
   for (int kb = 0; kb < nkb; ++kb) {
-    if (!__syncthreads_and(ok ? 1 : 0)) {
-      ok = false;
-      break;
-    }
     const int k0 = kb * kBlk;
-    // ---- dS for this query row against this thread's 64 of the block's 128 keys, bf16 over
-    // the first half of this half's S columns (ascending chunks: a chunk is read before any
-    // later chunk is overwritten)
     // S(kb) done: the MMAs run in issue order, so dQ of the previous step is done too and the
     // other K/V buffer is free for step kb+1
     ok = __all_sync(0xffffffffu, ok && wait(s_full, kb & 1, DEVERR_WAIT_ACC_FULL));
     if (ok && tid == 0 && kb >= 1 && kb + 1 < nkb) load_kv(kb + 1);
+    // ---- dS for this query row against this thread's 64 of the block's 128 keys, bf16 over
+    // the first half of this half's S columns (all of this thread's S and dP are read before
+    // any of them is overwritten)
     if (ok) {
       tc_fence_after();
       // no mask inside the block: every key is valid and (causal) before every query
       const bool plain = q0 + kBlk <= P.s && k0 + kBlk <= P.s && (!P.causal || k0 < q0);
-#pragma unroll 1
-      for (int c0 = 64 * half; c0 < 64 * half + 64; c0 += 32) {
-        float sv[32], dp[32];
-        ld32(tS + lane_base + c0, sv);
-        ld32(tdP + lane_base + c0, dp);
+      float sv[64], dp[64];
+      {
+        uint32_t r[4][32];
+        tmem_ld_32x32b_x32(tS + lane_base + 64 * half, r[0]);
+        tmem_ld_32x32b_x32(tS + lane_base + 64 * half + 32, r[1]);
+        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half, r[2]);
+        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half + 32, r[3]);
+        tmem_wait_ld();
+#pragma unroll
+        for (int e = 0; e < 64; ++e) {
+          sv[e] = __uint_as_float(r[e >> 5][e & 31]);
+          dp[e] = __uint_as_float(r[2 + (e >> 5)][e & 31]);
+        }
+      }
+#pragma unroll
+      for (int c = 0; c < 2; ++c) {
+        const int c0 = 64 * half + 32 * c;
         uint32_t dw[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 2) {
           float ds[2];
 #pragma unroll
           for (int u = 0; u < 2; ++u) {
-            float pr = exp2_fast(sv[e + u] * P.scale_log2 - lse_r);
+            float pr = exp2_fast(sv[32 * c + e + u] * P.scale_log2 - lse_r);
             if (!plain) {
               const int k_abs = k0 + c0 + e + u;
               if (!q_live || k_abs >= P.s || (P.causal && k_abs > q_abs)) pr = 0.f;
             }
-            ds[u] = pr * (dp[e + u] - D_r);
+            ds[u] = pr * (dp[32 * c + e + u] - D_r);
           }
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
         }
@@ -526,28 +560,29 @@ __global__ void __launch_bounds__(kThreads, 1)
       fa::tmem_wait_st();
     }
     tc_fence_before();
-    mbar_arrive(p_ready);
-    if (tid == 0 && ok) {
-      ok = wait(p_ready, kb & 1, DEVERR_WAIT_ACC_FULL);
-      if (ok) {
-        tc_fence_after();
-        const uint32_t ka = smem_addr(sK + (kb & 1) * L::BLOCK);
+    // every thread's dS is stored; all agree on ok
+    if (!__syncthreads_and(ok ? 1 : 0)) {
+      ok = false;
+      break;
+    }
+    if (tid == 0) {
+      tc_fence_after();
+      const uint32_t ka = smem_addr(sK + (kb & 1) * L::BLOCK);
 #pragma unroll
-        for (int kk = 0; kk < kBlk / 16; ++kk) {
-          // A: 16 keys = 8 TMEM columns of dS; B: the [key][dim] K tile read MN-major
-          fa::umma_f16_tmem_a(tdQ, tS + packed_col(kk * 8),
-                              make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                              (kb > 0 || kk > 0) ? 1u : 0u);
-        }
-        umma_commit(m_done);
-        // the next step's S and dP right behind: they overwrite dS only after this MMA has read
-        // it (issue order)
-        if (kb + 1 < nkb) {
-          ok = wait(&kv_full[(kb + 1) & 1], ((kb + 1) >> 1) & 1, DEVERR_WAIT_FULL);
-          if (ok) {
-            tc_fence_after();
-            issue_s(kb + 1);
-          }
+      for (int kk = 0; kk < kBlk / 16; ++kk) {
+        // A: 16 keys = 8 TMEM columns of dS; B: the [key][dim] K tile read MN-major
+        fa::umma_f16_tmem_a(tdQ, tS + packed_col(kk * 8),
+                            make_sdesc_sw128(ka + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
+                            (kb > 0 || kk > 0) ? 1u : 0u);
+      }
+      umma_commit(m_done);
+      // the next step's S and dP right behind: they overwrite dS only after this MMA has read
+      // it (issue order)
+      if (kb + 1 < nkb) {
+        ok = wait(&kv_full[(kb + 1) & 1], ((kb + 1) >> 1) & 1, DEVERR_WAIT_FULL);
+        if (ok) {
+          tc_fence_after();
+          issue_s(kb + 1);
         }
       }
     }
@@ -612,7 +647,7 @@ __global__ void __launch_bounds__(256) combine_kv_kernel(const float* part, int 
 }
 
 template <int HD>
-constexpr int dkv_smem() { return 6 * Tiles<HD>::BLOCK + 2 * kBlk * 4 + 128 + 1024; }
+constexpr int dkv_smem() { return 6 * Tiles<HD>::BLOCK + 4 * kBlk * 4 + 128 + 1024; }
 // at least 120 KB, so that no second CTA (which would wait for the 512 TMEM columns) shares an SM
 template <int HD>
 constexpr int dq_smem() {
