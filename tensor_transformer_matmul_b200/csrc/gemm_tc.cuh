@@ -500,7 +500,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // everything above may overlap the previous kernel's tail; global memory only from here on
-  pdl_wait();
+  // (the TMA producer waits below, after requesting the weight tiles no earlier kernel writes)
+  if (threadIdx.x != 0) pdl_wait();
   pdl_trigger();
 
   if (warp == 0) {
@@ -513,28 +514,53 @@ __global__ void __launch_bounds__(kThreads, 1)
       bool ok = true;
       SegIter it;
       it.init(gp, blockIdx.x, grid);
+      auto load_a = [&](int st, const Seg& sg, const KStep& ks) {
+        const int m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
+        uint8_t* sa = a_smem + st * Cfg::A_STAGE_BYTES;
+        if (Cfg::A_MN) {
+#pragma unroll
+          for (int j = 0; j < Cfg::A_ROWS / 64; ++j)
+            tma_load_3d(&tma_a, &full[st], sa + j * 64 * kBK * 2, m0 + 64 * j, ks.k0, ks.za);
+        } else {
+          tma_load_3d(&tma_a, &full[st], sa, ks.k0, m0, ks.za);
+        }
+      };
+      // Weight-streaming GEMMs (rotate_k: A is a weight that no earlier kernel writes, and the
+      // schedule is plain arithmetic): the first ring's worth of A tiles is requested before the
+      // programmatic-launch wait, so it streams while the previous kernel finishes; B (the
+      // activations) is loaded only after the wait.
+      int pre = 0;
+      if (gp.rotate_k && !gp.grp_cnt) {
+        SegIter it0 = it;
+        Seg s0;
+        if (it0.next(gp, grid, s0)) {
+          pre = min(Cfg::STAGES, s0.kb1 - s0.kb0);
+          for (int i = 0; i < pre; ++i) {
+            mbar_arrive_expect_tx(&full[i], Cfg::STAGE_BYTES);
+            load_a(i, s0, k_step(gp, s0, i));
+            issued_mask |= 1u << i;   // phase 0
+          }
+        }
+      }
+      pdl_wait();
       Seg sg;
       while (ok && it.next(gp, grid, sg)) {
-        const int m0 = sg.row0 + sg.mb * Cfg::A_ROWS;
         const int n0 = sg.n_off + sg.nb * Cfg::BN;
         const int nk = sg.kb1 - sg.kb0;
         for (int i = 0; i < nk; ++i) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
-            ok = false;
-            break;
-          }
-          mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
           const KStep ks = k_step(gp, sg, i);
-          const int k0 = ks.k0, zai = ks.za, zbi = ks.zb;
-          uint8_t* sa = a_smem + stage * Cfg::A_STAGE_BYTES;
-          uint8_t* sb = b_smem + stage * Cfg::B_STAGE_BYTES;
-          if (Cfg::A_MN) {
-#pragma unroll
-            for (int j = 0; j < Cfg::A_ROWS / 64; ++j)
-              tma_load_3d(&tma_a, &full[stage], sa + j * 64 * kBK * 2, m0 + 64 * j, k0, zai);
+          const int k0 = ks.k0, zbi = ks.zb;
+          if (pre > 0) {
+            --pre;   // this stage's A tile and byte count went out before the wait
           } else {
-            tma_load_3d(&tma_a, &full[stage], sa, k0, m0, zai);
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, gp.err, DEVERR_WAIT_EMPTY)) {
+              ok = false;
+              break;
+            }
+            mbar_arrive_expect_tx(&full[stage], Cfg::STAGE_BYTES);
+            load_a(stage, sg, ks);
           }
+          uint8_t* sb = b_smem + stage * Cfg::B_STAGE_BYTES;
           if (Cfg::B_MN) {
 #pragma unroll
             for (int j = 0; j < Cfg::BN / 64; ++j)

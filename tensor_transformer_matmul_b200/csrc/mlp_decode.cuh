@@ -75,7 +75,8 @@ struct Params {
   int32_t n_dn;           // down tiles: p shards x dn_mb blocks of 128 output features
   int32_t dn_mb;          // 128-row blocks of d
   int32_t dn_kb;          // k-blocks of a down tile (Fsp / 64)
-  int32_t* counters;      // [0]: next work item; [1 + i]: finished up tiles of shard i (zeroed)
+  int32_t* counters;      // [0]: items handed out after the first gridDim.x (each CTA starts at
+                          // its index); [1 + i]: finished up tiles of shard i (zeroed)
   uint32_t* err;          // device error word
   tc::EpiHiddenParams up;      // h (and the saved pre-activations), swapped
   tc::EpiStoreF32::Params dn;  // fp32 partials [p][T][d], swapped
@@ -145,7 +146,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
   // everything above may overlap the previous kernel's tail; global memory only from here on
-  pdl_wait();
+  // (the TMA producer waits below, after requesting its first weight tiles)
+  if (threadIdx.x != 0) pdl_wait();
   pdl_trigger();
 
   if (warp == 0) {
@@ -155,9 +157,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0, qphase = 0;
       uint32_t issued_mask = 0, last_parity = 0;
       bool ok = true;
+      // Item of step i of a tile: stage count, k-rotation, first k-block and k-block count.
+      auto up_stage = [&](int item, int i, int& kb0, int& nkb) {
+        const int nst = (pr.up_kb + C::UP_KPACK - 1) / C::UP_KPACK;
+        const int rot = static_cast<int>((static_cast<int64_t>(item) * 37) % nst);
+        int si = i + rot;
+        if (si >= nst) si -= nst;
+        kb0 = si * C::UP_KPACK;
+        nkb = pr.up_kb - kb0 < C::UP_KPACK ? pr.up_kb - kb0 : C::UP_KPACK;
+      };
+      auto up_bytes = [&](int nkb) {
+        return C::UP_SUB == 2 ? static_cast<uint32_t>(2 * C::BOX_A + C::BOX_B)
+                              : static_cast<uint32_t>(nkb * (C::BOX_A + C::BOX_B));
+      };
+      auto load_w1 = [&](int st, int kb0, int nkb, int m0) {
+        uint8_t* sa = a_smem + st * C::A_STAGE_BYTES;
+        if (C::UP_SUB == 2) {
+          tma_load_3d(&tma_w1, &full[st], sa, kb0 * kBK, m0, 0);   // gate and up rows: one box
+        } else {
+          for (int j = 0; j < nkb; ++j)
+            tma_load_3d(&tma_w1, &full[st], sa + j * C::BOX_A, (kb0 + j) * kBK, m0, 0);
+        }
+      };
+      // The first item is this CTA's index (the counter hands out the rest).  When it is an up
+      // tile, its first stages of W1 -- a weight no earlier kernel writes -- are requested
+      // before the programmatic-launch wait and stream while the previous kernel finishes; x
+      // follows after the wait.
+      const int first = static_cast<int>(blockIdx.x) < n_items ? static_cast<int>(blockIdx.x) : -1;
+      int pre = 0;
+      if (first >= 0 && first < pr.n_up) {
+        const int nst = (pr.up_kb + C::UP_KPACK - 1) / C::UP_KPACK;
+        pre = nst < C::STAGES ? nst : C::STAGES;
+        for (int i = 0; i < pre; ++i) {
+          int kb0, nkb;
+          up_stage(first, i, kb0, nkb);
+          mbar_arrive_expect_tx(&full[i], up_bytes(nkb));
+          load_w1(i, kb0, nkb, first * 128 * C::UP_SUB);
+          issued_mask |= 1u << i;   // phase 0
+        }
+      }
+      pdl_wait();
+      bool first_taken = false;
       while (ok) {
-        int item = atomicAdd(pr.counters, 1);
-        if (item >= n_items) item = -1;
+        int item = first;
+        if (first_taken) {
+          item = static_cast<int>(gridDim.x) + atomicAdd(pr.counters, 1);
+          if (item >= n_items) item = -1;
+        }
+        first_taken = true;
         // publish the item to the MMA issuer and the epilogue warps
         if (!mbar_wait(&q_empty[slot], qphase ^ 1u, abort_flag, pr.err, DEVERR_WAIT_EMPTY)) {
           ok = false;
@@ -192,29 +239,35 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (si >= nst) si -= nst;
           const int kb0 = si * kpack;
           const int nkb = kb_all - kb0 < kpack ? kb_all - kb0 : kpack;
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, pr.err, DEVERR_WAIT_EMPTY)) {
-            ok = false;
-            break;
-          }
-          uint8_t* sa = a_smem + stage * C::A_STAGE_BYTES;
           uint8_t* sb = b_smem + stage * C::B_STAGE_BYTES;
-          if (up && C::UP_SUB == 2) {
-            // gate and up rows of one k-block: one 256-row box
-            mbar_arrive_expect_tx(&full[stage], 2 * C::BOX_A + C::BOX_B);
-            tma_load_3d(&tma_w1, &full[stage], sa, kb0 * kBK, m0, 0);
-            tma_load_3d(&tma_x, &full[stage], sb, kb0 * kBK, 0, 0);
+          if (pre > 0) {
+            --pre;   // this stage's W1 tile and byte count went out before the wait
           } else {
-            mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nkb * (C::BOX_A + C::BOX_B)));
-            for (int j = 0; j < nkb; ++j) {
-              const int k0 = (kb0 + j) * kBK;
-              if (up) {
-                tma_load_3d(&tma_w1, &full[stage], sa + j * C::BOX_A, k0, m0, 0);
-                tma_load_3d(&tma_x, &full[stage], sb + j * C::BOX_B, k0, 0, 0);
-              } else {
-                tma_load_3d(&tma_w2, &full[stage], sa + j * C::BOX_A, k0, m0, shard);
-                tma_load_3d(&tma_h, &full[stage], sb + j * C::BOX_B, k0, 0, shard);
-              }
+            if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, pr.err, DEVERR_WAIT_EMPTY)) {
+              ok = false;
+              break;
             }
+            if (up) {
+              mbar_arrive_expect_tx(&full[stage], up_bytes(nkb));
+              load_w1(stage, kb0, nkb, m0);
+            } else {
+              uint8_t* sa = a_smem + stage * C::A_STAGE_BYTES;
+              mbar_arrive_expect_tx(&full[stage], static_cast<uint32_t>(nkb * (C::BOX_A + C::BOX_B)));
+              for (int j = 0; j < nkb; ++j)
+                tma_load_3d(&tma_w2, &full[stage], sa + j * C::BOX_A, (kb0 + j) * kBK, m0, shard);
+            }
+          }
+          if (up) {
+            // x: one box per k-block of the stage
+            if (C::UP_SUB == 2) {
+              tma_load_3d(&tma_x, &full[stage], sb, kb0 * kBK, 0, 0);
+            } else {
+              for (int j = 0; j < nkb; ++j)
+                tma_load_3d(&tma_x, &full[stage], sb + j * C::BOX_B, (kb0 + j) * kBK, 0, 0);
+            }
+          } else {
+            for (int j = 0; j < nkb; ++j)
+              tma_load_3d(&tma_h, &full[stage], sb + j * C::BOX_B, (kb0 + j) * kBK, 0, shard);
           }
           issued_mask |= 1u << stage;
           last_parity = (last_parity & ~(1u << stage)) | (phase << stage);
