@@ -135,10 +135,39 @@ __global__ void __launch_bounds__(1024) count_kernel(const int32_t* __restrict__
   if (threadIdx.x == 0) cnt[e] = c;
 }
 
+// Exclusive prefix sum of v over the block (threads in index order); red holds 32 ints.
+__device__ __forceinline__ int block_exclusive_scan_int(int v, int* red) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int inc = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int u = __shfl_up_sync(0xffffffffu, inc, o);
+    if (lane >= o) inc += u;
+  }
+  if (lane == 31) red[warp] = inc;
+  __syncthreads();
+  if (warp == 0) {
+    const int nw = static_cast<int>(blockDim.x >> 5);
+    int w = lane < nw ? red[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int u = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += u;
+    }
+    if (lane < nw) red[lane] = w;   // inclusive totals of warps 0..lane
+  }
+  __syncthreads();
+  const int before = (warp > 0 ? red[warp - 1] : 0) + inc - v;
+  __syncthreads();   // red is reused by the caller
+  return before;
+}
+
 // Block e: off[e] = sum of the counts of experts < e and mbp[e] = sum of their block_rows-row
 // blocks (the last block also writes mbp[E], the total); then every entry routed to e gets the
 // next position in entry order: perm[off + pos] = entry, inv[entry] = off + pos (a stable order,
-// so the dispatch is deterministic).
+// so the dispatch is deterministic).  Thread t owns a contiguous range of the entries: it counts
+// its hits, an exclusive scan over the block gives its first position, and a second pass over
+// the same range writes them.
 __global__ void __launch_bounds__(1024) position_kernel(const int32_t* __restrict__ idx,
                                                         int64_t n_entries,
                                                         const int32_t* __restrict__ cnt,
@@ -150,7 +179,6 @@ __global__ void __launch_bounds__(1024) position_kernel(const int32_t* __restric
   pdl_wait();
   pdl_trigger();
   __shared__ int red[32];
-  __shared__ int warp_pre[32];
   const int e = blockIdx.x;
   int o = 0, nb = 0;
   for (int i = threadIdx.x; i < e; i += blockDim.x) {
@@ -164,41 +192,35 @@ __global__ void __launch_bounds__(1024) position_kernel(const int32_t* __restric
     mbp[e] = blocks0;
     if (e == static_cast<int>(gridDim.x) - 1) mbp[e + 1] = blocks0 + (cnt[e] + block_rows - 1) / block_rows;
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
-  int base = base0;
-  for (int64_t c0 = 0; c0 < n_entries; c0 += blockDim.x) {
-    const int64_t i = c0 + threadIdx.x;
-    const bool hit = i < n_entries && idx[i] == e;
-    const unsigned m = __ballot_sync(0xffffffffu, hit);
-    if (lane == 0) warp_pre[warp] = __popc(m);
-    __syncthreads();
-    int before = 0, total = 0;
-    for (int q = 0; q < nw; ++q) {
-      const int v = warp_pre[q];
-      if (q < warp) before += v;
-      total += v;
-    }
-    if (hit) {
-      const int slot = base + before + __popc(m & ((1u << lane) - 1u));
-      perm[slot] = static_cast<int32_t>(i);
-      inv[i] = slot;
-    }
-    base += total;
-    __syncthreads();   // warp_pre is rewritten by the next chunk
-  }
+  const int64_t per = (n_entries + blockDim.x - 1) / blockDim.x;
+  const int64_t i0 = static_cast<int64_t>(threadIdx.x) * per;
+  const int64_t i1 = i0 + per < n_entries ? i0 + per : n_entries;
+  int c = 0;
+  for (int64_t i = i0; i < i1; ++i) c += idx[i] == e ? 1 : 0;
+  int slot = base0 + block_exclusive_scan_int(c, red);
+  if (c > 0)
+    for (int64_t i = i0; i < i1; ++i)
+      if (idx[i] == e) {
+        perm[slot] = static_cast<int32_t>(i);
+        inv[i] = slot;
+        ++slot;
+      }
 }
 
-// xs[r] = x[perm[r] / k] for the n_rows routed rows: one block per row, 16-byte words (d % 8 == 0).
-__global__ void __launch_bounds__(128) gather_kernel(const __nv_bfloat16* __restrict__ x,
-                                                     const int32_t* __restrict__ perm, int k,
-                                                     int64_t d, __nv_bfloat16* __restrict__ xs) {
+// xs[r] = x[perm[r] / k] for the n_rows routed rows: one warp per row, 16-byte words
+// (d % 8 == 0).
+constexpr int kGatherRowsPerBlock = 8;
+__global__ void __launch_bounds__(32 * kGatherRowsPerBlock) gather_kernel(
+    const __nv_bfloat16* __restrict__ x, const int32_t* __restrict__ perm, int k, int64_t d,
+    int64_t n_rows, __nv_bfloat16* __restrict__ xs) {
   pdl_wait();
   pdl_trigger();
-  const int64_t r = blockIdx.x;
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * kGatherRowsPerBlock + (threadIdx.x >> 5);
+  if (r >= n_rows) return;
   const int64_t t = perm[r] / k;
   const uint4* src = reinterpret_cast<const uint4*>(x + t * d);
   uint4* dst = reinterpret_cast<uint4*>(xs + r * d);
-  for (int64_t j = threadIdx.x; j < d / 8; j += blockDim.x) dst[j] = src[j];
+  for (int64_t j = threadIdx.x & 31; j < d / 8; j += 32) dst[j] = src[j];
 }
 
 // y[t] = residual[t] + ((shared[t] + sum_{j<k} w[t][j] * routed[inv[t k + j]]) + bias): the

@@ -1115,9 +1115,10 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
     TP_LAUNCH_PDL(moe::position_kernel, dim3(static_cast<unsigned>(M.E)), dim3(1024), 0, s,
                   static_cast<const int32_t*>(idx), M.n_rows, static_cast<const int32_t*>(cnt), 128,
                   offs, mbp, perm, inv);
-    TP_LAUNCH_PDL(moe::gather_kernel, dim3(static_cast<unsigned>(M.n_rows)), dim3(128), 0, s,
-                  static_cast<const __nv_bfloat16*>(x), static_cast<const int32_t*>(perm), M.k,
-                  M.d, xs);
+    TP_LAUNCH_PDL(moe::gather_kernel,
+                  dim3(static_cast<unsigned>(ceil_div(M.n_rows, moe::kGatherRowsPerBlock))),
+                  dim3(32 * moe::kGatherRowsPerBlock), 0, s, static_cast<const __nv_bfloat16*>(x),
+                  static_cast<const int32_t*>(perm), M.k, M.d, M.n_rows, xs);
   }
   // (5) grouped up GEMM + SwiGLU over all experts: rows of expert e are xs[off[e] .. +cnt[e]).
   // Swapped: each tile is 256 packed rows of one expert's W1 (128 gate + 128 up features) times
