@@ -142,3 +142,57 @@ def moe_forward_sharded(x, wr, experts, k, p, shared=None, bias=None, routing=No
     if bias is not None:
         y = y + _f64(bias)[None, :]
     return y, partials
+
+
+def moe_backward(x, wr, experts, k, dy, shared=None, routing=None):
+    """Gradients of moe_forward's output y against an upstream gradient dy, with the choice of
+    experts held fixed (the top-k selection is constant wherever the k-th and (k+1)-th logits
+    differ, so it carries no gradient there).  The residual and the bias pass dy through and are
+    not part of the result.
+
+    Chain rule, with l_t = x_t Wr, the chosen experts e_tj = idx[t, j], the routed outputs
+    o_tj = expert_{e_tj}(x_t) and the weights w_t = softmax(l_t[idx_t]):
+      y_t = sum_j w_tj o_tj + shared(x_t)
+      d o_tj = w_tj dy_t           -> expert e_tj's MLP backward on row t
+      dw_tj = <dy_t, o_tj>
+      dl_t[e_tj] = w_tj (dw_tj - sum_i w_ti dw_ti), 0 at the experts not chosen
+      dWr = x^T dl,  dx += dl Wr^T
+      the shared expert: its MLP backward with dy.
+    ``routing``: (idx, weights) as moe_forward takes them; else route(x, wr, k).
+    Returns a dict: dx (T, d), dwr (d, E), experts (per expert a dict dwg, dwu, dw2; zeros for
+    an expert no token chose) and shared (dwg, dwu, dw2, or None)."""
+    x, wr, dy = _f64(x), _f64(wr), _f64(dy)
+    idx, w = routing if routing is not None else route(x, wr, k)
+    idx = np.asarray(idx, dtype=np.int64)
+    w = _f64(w)
+    T, d = x.shape
+    E = wr.shape[1]
+    dx = np.zeros((T, d))
+    grads = [{"dwg": np.zeros_like(_f64(ex[0])), "dwu": np.zeros_like(_f64(ex[1])),
+              "dw2": np.zeros_like(_f64(ex[2]))} for ex in experts]
+    dl = np.zeros((T, E))
+    for t in range(T):
+        dwt = np.zeros(idx.shape[1])
+        for j in range(idx.shape[1]):
+            wg, wu, w2 = experts[int(idx[t, j])]
+            xt = x[t:t + 1]
+            o = mlp.mlp_forward(xt, wg, w2, "swiglu", wu)[0]
+            dwt[j] = dy[t] @ o
+            b = mlp.mlp_backward(xt, wg, w2, w[t, j] * dy[t:t + 1], "swiglu", wu)
+            g = grads[int(idx[t, j])]
+            g["dwg"] += b["dw1"]
+            g["dwu"] += b["dw_up"]
+            g["dw2"] += b["dw2"]
+            dx[t] += b["dx"][0]
+        s = w[t] @ dwt
+        for j in range(idx.shape[1]):
+            dl[t, int(idx[t, j])] = w[t, j] * (dwt[j] - s)
+    dwr = x.T @ dl
+    dx += dl @ wr.T
+    out = {"dx": dx, "dwr": dwr, "experts": grads, "shared": None}
+    if shared is not None:
+        wg, wu, w2 = shared
+        b = mlp.mlp_backward(x, wg, w2, dy, "swiglu", wu)
+        out["dx"] = out["dx"] + b["dx"]
+        out["shared"] = {"dwg": b["dw1"], "dwu": b["dw_up"], "dw2": b["dw2"]}
+    return out

@@ -157,3 +157,76 @@ def test_topk_margin_of_route_is_the_logit_gap():
     srt = -np.sort(-(x @ wr), axis=1)
     np.testing.assert_allclose(moe.topk_margin(x, wr, idx), srt[:, k - 1] - srt[:, k], rtol=1e-14)
     assert (moe.topk_margin(x, wr, idx) >= 0).all()
+
+
+# --- backward: central finite differences of the forward (itself pinned above), with the choice
+# of experts held at the base point's and the weights recomputed from the perturbed logits
+
+def _fd_case(seed=3, T=5, d=6, E=5, F=4, k=2):
+    r = np.random.default_rng(seed)
+    for _ in range(200):
+        x = r.standard_normal((T, d))
+        wr = r.standard_normal((d, E))
+        idx, _ = moe.route(x, wr, k)
+        if moe.topk_margin(x, wr, idx).min() > 0.3:   # no choice flips under a 1e-6 step
+            break
+    experts = [tuple(r.standard_normal(s) / math.sqrt(s[0]) for s in ((d, F), (d, F), (F, d)))
+               for _ in range(E)]
+    sh = tuple(r.standard_normal(s) / math.sqrt(s[0]) for s in ((d, F), (d, F), (F, d)))
+    dy = r.standard_normal((T, d))
+    return x, wr, experts, sh, dy, idx, k
+
+
+def _loss(x, wr, experts, sh, dy, idx, k):
+    w = moe.weights_for(x, wr, idx)
+    return float(np.sum(dy * moe.moe_forward(x, wr, experts, k, shared=sh, routing=(idx, w))))
+
+
+def _fd(fun, a, entries, e=1e-6):
+    out = []
+    for ij in entries:
+        keep = a[ij]
+        a[ij] = keep + e
+        up = fun()
+        a[ij] = keep - e
+        dn = fun()
+        a[ij] = keep
+        out.append((up - dn) / (2 * e))
+    return np.array(out)
+
+
+def test_backward_matches_finite_differences():
+    x, wr, experts, sh, dy, idx, k = _fd_case()
+    g = moe.moe_backward(x, wr, experts, k, dy, shared=sh)
+    f = lambda: _loss(x, wr, experts, sh, dy, idx, k)
+    ent = [(t, c) for t in range(x.shape[0]) for c in range(x.shape[1])]
+    np.testing.assert_allclose(g["dx"][tuple(np.array(ent).T)], _fd(f, x, ent), rtol=1e-6, atol=1e-7)
+    ent = [(c, e) for c in range(wr.shape[0]) for e in range(wr.shape[1])]
+    np.testing.assert_allclose(g["dwr"][tuple(np.array(ent).T)], _fd(f, wr, ent), rtol=1e-6, atol=1e-7)
+    used = sorted(set(int(e) for e in idx.ravel()))
+    for e in used[:2]:
+        for name, a in zip(("dwg", "dwu", "dw2"), experts[e]):
+            ent = [(i, j) for i in range(a.shape[0]) for j in range(a.shape[1])][:7]
+            np.testing.assert_allclose(g["experts"][e][name][tuple(np.array(ent).T)], _fd(f, a, ent),
+                                       rtol=1e-6, atol=1e-7)
+    for name, a in zip(("dwg", "dwu", "dw2"), sh):
+        ent = [(i, j) for i in range(a.shape[0]) for j in range(a.shape[1])][:7]
+        np.testing.assert_allclose(g["shared"][name][tuple(np.array(ent).T)], _fd(f, a, ent),
+                                   rtol=1e-6, atol=1e-7)
+    # an expert no token chose gets no gradient
+    for e in set(range(len(experts))) - set(used):
+        assert all(not g["experts"][e][n].any() for n in ("dwg", "dwu", "dw2"))
+
+
+def test_backward_one_expert_is_the_dense_mlp_backward():
+    # k = E = 1: the weight is 1 whatever the logit, so the router gets no gradient and the
+    # block's gradients are the dense MLP oracle's
+    x, wr, experts, _ = _case(E=1, shared=False)
+    dy = np.random.default_rng(7).standard_normal(x.shape)
+    g = moe.moe_backward(x, wr, experts, 1, dy)
+    wg, wu, w2 = experts[0]
+    b = mlp.mlp_backward(x, wg, w2, dy, "swiglu", wu)
+    np.testing.assert_allclose(g["dx"], b["dx"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["experts"][0]["dwg"], b["dw1"], rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(g["experts"][0]["dw2"], b["dw2"], rtol=1e-12, atol=1e-12)
+    assert not g["dwr"].any()
