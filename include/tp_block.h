@@ -305,6 +305,28 @@ tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr, con
                      const void* residual, void* y, void* route_idx, void* route_w,
                      void* workspace, size_t ws_bytes, void* stream);
 
+/* Backward of the MoE block: the chain rule through the forward above with the routing held
+ * fixed (the top-k choice is constant wherever the k-th and (k+1)-th logits differ).
+ *   routed row (t, j): d o = w_tj dy_t through expert e_tj; dw_tj = <dy_t, o_tj>;
+ *   router: dl_t[e_tj] = w_tj (dw_tj - sum_i w_ti dw_ti), dWr = x^T dl, dx += dl Wr^T;
+ *   shared expert: its MLP backward with dy.
+ * dy [T][d] bf16, the gradient of y.  dx [T][d] bf16 receives the gradient through the routed
+ * experts, the shared expert and the router, summed in that order in fp32 with one rounding (the
+ * residual passes dy straight through and is not added; the bias gradient, the column sum of dy,
+ * is not computed).  dwr [d][E] fp32.  dw1p, dw2p: fp32 gradients of the packed expert weights,
+ * E * 2 * tp_moe_expert_w{1,2}_bytes bytes, expert e's at element offset e * w{1,2}p elements in
+ * the packed layout of its weights (tp_mlp_unpack_grads with the dense desc {d, d_ff, p, SWIGLU}
+ * unpacks it); an expert no token chose gets zeros.  dw1p_s, dw2p_s: the shared expert's, the
+ * same way (ignored when d_ff_shared == 0).  The routing and the expert activations are
+ * recomputed from x.  The routed experts' GEMMs run expert by expert, so the call reads the E
+ * per-expert row counts back to the host once (it synchronises the stream and cannot be
+ * captured in a CUDA graph).  workspace: tp_moe_bwd_workspace(desc) bytes. */
+size_t tp_moe_bwd_workspace(const tp_moe_desc* desc);
+tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const void* wr, const void* w1p,
+                     const void* w2p, const void* w1p_s, const void* w2p_s, const void* dy,
+                     void* dx, float* dwr, float* dw1p, float* dw2p, float* dw1p_s,
+                     float* dw2p_s, void* workspace, size_t ws_bytes, void* stream);
+
 /* ------------------------------------------------------------------------------------------ */
 /* Sequence parallelism                                                                        */
 /* ------------------------------------------------------------------------------------------ */

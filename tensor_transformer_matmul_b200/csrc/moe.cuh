@@ -15,6 +15,7 @@
 //   expert + weighted routed rows (choices in order) + bias, then the residual.
 #pragma once
 
+#include "reduce.cuh"
 #include "tp_common.cuh"
 
 namespace tp {
@@ -276,6 +277,105 @@ __global__ void __launch_bounds__(256) combine_kernel(
     o.z = pack_bf16x2(acc[4], acc[5]);
     o.w = pack_bf16x2(acc[6], acc[7]);
     *reinterpret_cast<uint4*>(y + t * d + c) = o;
+  }
+}
+
+// ------------------------------------------------------------------------------ backward
+// dw[t k + j] = <dy_t, o[inv[t k + j]]>: the gradient of routing weight w_tj (o: the routed
+// rows' outputs, fp32 [row][d]).  One warp per (token, choice); fp32 sum.
+__global__ void __launch_bounds__(256) route_weight_grad_kernel(
+    const __nv_bfloat16* __restrict__ dy, const float* __restrict__ o,
+    const int32_t* __restrict__ inv, int k, int64_t T, int64_t d, float* __restrict__ dw) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t q = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  if (q >= T * k) return;
+  const int64_t t = q / k;
+  const __nv_bfloat16* g = dy + t * d;
+  const float* r = o + static_cast<int64_t>(inv[q]) * d;
+  float acc = 0.f;
+  for (int64_t c = 8 * lane; c < d; c += 256) {
+    float gv[8], rv[8];
+    reduce::Vec8<__nv_bfloat16>::load(g + c, gv);
+    reduce::Vec8<float>::load(r + c, rv);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc = fmaf(gv[e], rv[e], acc);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  if (lane == 0) dw[q] = acc;
+}
+
+// dl[t][e] = w_tj (dw_tj - sum_i w_ti dw_ti) when e = idx[t][j], else 0: the gradient of the
+// router logits through the softmax over each token's k chosen logits (bf16 [T][E]).
+__global__ void __launch_bounds__(256) router_logit_grad_kernel(
+    const int32_t* __restrict__ idx, const float* __restrict__ w, const float* __restrict__ dw,
+    int k, int64_t T, int E, __nv_bfloat16* __restrict__ dl) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (q >= T * E) return;
+  const int64_t t = q / E;
+  const int e = static_cast<int>(q - t * E);
+  float s = 0.f, v = 0.f;
+  for (int j = 0; j < k; ++j) s = fmaf(w[t * k + j], dw[t * k + j], s);
+  for (int j = 0; j < k; ++j)
+    if (idx[t * k + j] == e) v = w[t * k + j] * (dw[t * k + j] - s);
+  dl[q] = __float2bfloat16_rn(v);
+}
+
+// gs[r] = w[perm[r]] * dy[perm[r] / k] (bf16), the routed rows' output gradients in expert
+// order: one warp per row, 8 columns per lane and step (d % 8 == 0).
+__global__ void __launch_bounds__(32 * kGatherRowsPerBlock) gather_scaled_kernel(
+    const __nv_bfloat16* __restrict__ dy, const int32_t* __restrict__ perm,
+    const float* __restrict__ w, int k, int64_t d, int64_t n_rows,
+    __nv_bfloat16* __restrict__ gs) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t r = static_cast<int64_t>(blockIdx.x) * kGatherRowsPerBlock + (threadIdx.x >> 5);
+  if (r >= n_rows) return;
+  const int32_t entry = perm[r];
+  const float sc = w[entry];
+  const __nv_bfloat16* src = dy + static_cast<int64_t>(entry / k) * d;
+  __nv_bfloat16* dst = gs + r * d;
+  for (int64_t c = 8 * (threadIdx.x & 31); c < d; c += 256) {
+    float v[8];
+    reduce::Vec8<__nv_bfloat16>::load(src + c, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) v[e] *= sc;
+    reduce::Vec8<__nv_bfloat16>::store(dst + c, v);
+  }
+}
+
+// dx[t] = (sum_{j<k} dxs[inv[t k + j]] + dxr[t]) + dxsh[t]: the routed rows' input gradients
+// (choices in order), the router's and the shared expert's (optional), fp32, one rounding.
+__global__ void __launch_bounds__(256) dx_combine_kernel(
+    const float* __restrict__ dxs, const float* __restrict__ dxr, const float* __restrict__ dxsh,
+    const int32_t* __restrict__ inv, int k, int64_t T, int64_t d, __nv_bfloat16* __restrict__ dx) {
+  pdl_wait();
+  pdl_trigger();
+  const int64_t nv = T * (d / 8);
+  const int64_t stride = static_cast<int64_t>(gridDim.x) * blockDim.x;
+  for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < nv; q += stride) {
+    const int64_t t = q / (d / 8);
+    const int64_t c = (q - t * (d / 8)) * 8;
+    float acc[8], v[8];
+    reduce::Vec8<float>::load(dxs + static_cast<int64_t>(inv[t * k]) * d + c, acc);
+    for (int j = 1; j < k; ++j) {
+      reduce::Vec8<float>::load(dxs + static_cast<int64_t>(inv[t * k + j]) * d + c, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    }
+    reduce::Vec8<float>::load(dxr + t * d + c, v);
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    if (dxsh) {
+      reduce::Vec8<float>::load(dxsh + t * d + c, v);
+#pragma unroll
+      for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    }
+    reduce::Vec8<__nv_bfloat16>::store(dx + t * d + c, acc);
   }
 }
 

@@ -1046,33 +1046,15 @@ extern "C" tp_status tp_moe_pack(const tp_moe_desc* desc, const void* const* wg,
   return TP_OK;
 }
 
-extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr,
-                                const void* w1p, const void* w2p, const void* w1p_s,
-                                const void* w2p_s, const void* bias, const void* residual,
-                                void* y, void* route_idx, void* route_w, void* workspace,
-                                size_t ws_bytes, void* stream) {
-  clear_error();
-  MoeLayout M;
-  tp_status st = moe_layout(desc, &M);
-  if (st != TP_OK) return st;
-  if (M.T == 0) {
-    count_reduction();
-    return TP_OK;
-  }
-  if (!x || !wr || !w1p || !w2p || !y) return set_error(TP_ERR_INVALID_ARG, "null pointer");
-  if (M.Fsh > 0 && (!w1p_s || !w2p_s))
-    return set_error(TP_ERR_INVALID_ARG, "the shared expert's packed weights are null");
-  for (const void* q : {x, wr, w1p, w2p, w1p_s, w2p_s, bias, residual, static_cast<const void*>(y)})
-    if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
-  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
-  if (ws_bytes < M.bytes) return set_error(TP_ERR_WORKSPACE, "workspace too small");
-  if (!tensor_cores_usable())
-    return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+// Steps (1)-(6) of the forward: router logits, top-k routing, dispatch (counts, stable
+// positions, gather) and the two grouped expert GEMMs, in M's workspace regions; the routing goes
+// to idx / wts, the routed rows' outputs (shards summed) to the part region, and with ``zs`` the
+// routed rows' gate/up pre-activations ([row][p R], as the dense MLP saves them) to zs.
+tp_status moe_routed(const MoeLayout& M, const void* x, const void* wr, const void* w1p,
+                     const void* w2p, void* workspace, int32_t* idx, float* wts, void* zs,
+                     cudaStream_t s) {
+  tp_status st;
   float* logits = reinterpret_cast<float*>(off(workspace, M.logits_off));
-  int32_t* idx = route_idx ? static_cast<int32_t*>(route_idx)
-                           : reinterpret_cast<int32_t*>(off(workspace, M.idx_off));
-  float* wts = route_w ? static_cast<float*>(route_w) : reinterpret_cast<float*>(off(workspace, M.w_off));
   int32_t* cnt = reinterpret_cast<int32_t*>(off(workspace, M.cnt_off));
   int32_t* offs = reinterpret_cast<int32_t*>(off(workspace, M.off_off));
   int32_t* mbp = reinterpret_cast<int32_t*>(off(workspace, M.mbp_off));
@@ -1128,9 +1110,9 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
     const int64_t rows = L.p * L.R;
     tc::EpiHiddenParams ep;
     ep.h = hs;
-    ep.z = nullptr;
+    ep.z = static_cast<__nv_bfloat16*>(zs);
     ep.ld_h = L.p * L.Fsp;
-    ep.ld_z = 0;
+    ep.ld_z = zs ? rows : 0;
     ep.tokens = static_cast<int32_t>(M.n_rows);
     ep.rows = static_cast<int32_t>(rows);
     ep.act = TP_ACT_SWIGLU;
@@ -1174,6 +1156,38 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
         wo, ho, M.d, M.T, L.Fsp, static_cast<int64_t>(M.E) * L.p, ep, s, "moe_down_gemm", opt);
     if (st != TP_OK) return st;
   }
+  return TP_OK;
+}
+
+extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const void* wr,
+                                const void* w1p, const void* w2p, const void* w1p_s,
+                                const void* w2p_s, const void* bias, const void* residual,
+                                void* y, void* route_idx, void* route_w, void* workspace,
+                                size_t ws_bytes, void* stream) {
+  clear_error();
+  MoeLayout M;
+  tp_status st = moe_layout(desc, &M);
+  if (st != TP_OK) return st;
+  if (M.T == 0) {
+    count_reduction();
+    return TP_OK;
+  }
+  if (!x || !wr || !w1p || !w2p || !y) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (M.Fsh > 0 && (!w1p_s || !w2p_s))
+    return set_error(TP_ERR_INVALID_ARG, "the shared expert's packed weights are null");
+  for (const void* q : {x, wr, w1p, w2p, w1p_s, w2p_s, bias, residual, static_cast<const void*>(y)})
+    if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < M.bytes) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tensor_cores_usable())
+    return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  int32_t* idx = route_idx ? static_cast<int32_t*>(route_idx)
+                           : reinterpret_cast<int32_t*>(off(workspace, M.idx_off));
+  float* wts = route_w ? static_cast<float*>(route_w) : reinterpret_cast<float*>(off(workspace, M.w_off));
+  if ((st = moe_routed(M, x, wr, w1p, w2p, workspace, idx, wts, nullptr, s)) != TP_OK) return st;
+  int32_t* inv = reinterpret_cast<int32_t*>(off(workspace, M.inv_off));
+  float* part = reinterpret_cast<float*>(off(workspace, M.part_off));
   // (7) the shared expert over all tokens, its p shards summed in its down GEMM: [T][d] fp32
   const float* shared_sum = nullptr;
   if (M.Fsh > 0) {
@@ -1199,5 +1213,180 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
                   static_cast<const __nv_bfloat16*>(residual), static_cast<__nv_bfloat16*>(y));
   }
   count_reduction();
+  return TP_OK;
+}
+
+// ------------------------------------------------------------------ MoE backward
+namespace {
+// Backward workspace: the forward's regions, then the backward's own.
+struct MoeBwdLayout {
+  size_t zs_off, dw_off, dl_off, dxr_off, gs_off, dz_off, dxs_off, zsh_off, hsh_off, dzs_off,
+      dxsh_off, bytes;
+};
+MoeBwdLayout moe_bwd_layout(const MoeLayout& M) {
+  MoeBwdLayout B;
+  size_t o = M.bytes;
+  auto take = [&](size_t& field, size_t bytes) {
+    field = o;
+    o += align256(bytes);
+  };
+  const size_t R = static_cast<size_t>(M.n_rows), T = static_cast<size_t>(M.T);
+  const size_t d = static_cast<size_t>(M.d);
+  const size_t zrow = static_cast<size_t>(M.ex.p * M.ex.R);
+  take(B.zs_off, R * zrow * 2);       // routed rows' gate/up pre-activations
+  take(B.dw_off, R * 4);              // routing-weight gradients [T][k]
+  take(B.dl_off, T * M.E * 2);        // router-logit gradients [T][E] bf16
+  take(B.dxr_off, T * d * 4);         // dx through the router
+  take(B.gs_off, R * d * 2);          // w * dy per routed row, expert order
+  take(B.dz_off, R * zrow * 2);       // dz of the expert being differentiated
+  take(B.dxs_off, R * d * 4);         // routed rows' input gradients
+  const size_t zsh = M.Fsh > 0 ? T * static_cast<size_t>(M.sh.p * M.sh.R) * 2 : 0;
+  take(B.zsh_off, zsh);               // the shared expert's z, h and dz
+  take(B.hsh_off, M.Fsh > 0 ? T * static_cast<size_t>(M.sh.p * M.sh.Fsp) * 2 : 0);
+  take(B.dzs_off, zsh);
+  take(B.dxsh_off, M.Fsh > 0 ? T * d * 4 : 0);
+  B.bytes = o;
+  return B;
+}
+}  // namespace
+
+extern "C" size_t tp_moe_bwd_workspace(const tp_moe_desc* desc) {
+  MoeLayout M;
+  return moe_layout(desc, &M) == TP_OK ? moe_bwd_layout(M).bytes : 0;
+}
+
+extern "C" tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const void* wr,
+                                const void* w1p, const void* w2p, const void* w1p_s,
+                                const void* w2p_s, const void* dy, void* dx, float* dwr,
+                                float* dw1p, float* dw2p, float* dw1p_s, float* dw2p_s,
+                                void* workspace, size_t ws_bytes, void* stream) {
+  clear_error();
+  MoeLayout M;
+  tp_status st = moe_layout(desc, &M);
+  if (st != TP_OK) return st;
+  const MoeBwdLayout B = moe_bwd_layout(M);
+  const MlpLayout& L = M.ex;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (!dwr || !dw1p || !dw2p || (M.Fsh > 0 && (!dw1p_s || !dw2p_s)))
+    return set_error(TP_ERR_INVALID_ARG, "null gradient pointer");
+  // every gradient starts at zero: an expert no token chose keeps it
+  TP_CUDA_TRY(cudaMemsetAsync(dwr, 0, static_cast<size_t>(M.d) * M.E * 4, s));
+  TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(M.E) * L.w1p_bytes * 2, s));
+  TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(M.E) * L.w2p_bytes * 2, s));
+  if (M.Fsh > 0) {
+    TP_CUDA_TRY(cudaMemsetAsync(dw1p_s, 0, M.sh.w1p_bytes * 2, s));
+    TP_CUDA_TRY(cudaMemsetAsync(dw2p_s, 0, M.sh.w2p_bytes * 2, s));
+  }
+  if (M.T == 0) return TP_OK;
+  if (!x || !wr || !w1p || !w2p || !dy || !dx) return set_error(TP_ERR_INVALID_ARG, "null pointer");
+  if (M.Fsh > 0 && (!w1p_s || !w2p_s))
+    return set_error(TP_ERR_INVALID_ARG, "the shared expert's packed weights are null");
+  for (const void* q : {x, wr, w1p, w2p, w1p_s, w2p_s, dy, static_cast<const void*>(dx),
+                        static_cast<const void*>(dw1p), static_cast<const void*>(dw2p),
+                        static_cast<const void*>(dw1p_s), static_cast<const void*>(dw2p_s)})
+    if (q && !aligned16(q)) return set_error(TP_ERR_INVALID_ARG, "pointers must be 16-byte aligned");
+  if (!workspace) return set_error(TP_ERR_INVALID_ARG, "workspace is null");
+  if (ws_bytes < B.bytes) return set_error(TP_ERR_WORKSPACE, "workspace too small");
+  if (!tensor_cores_usable())
+    return set_error(TP_ERR_UNSUPPORTED, "bf16 tensor-core path needs an sm_100 device");
+  using BF = __nv_bfloat16;
+  int32_t* idx = reinterpret_cast<int32_t*>(off(workspace, M.idx_off));
+  float* wts = reinterpret_cast<float*>(off(workspace, M.w_off));
+  const int32_t* cnt = reinterpret_cast<const int32_t*>(off(workspace, M.cnt_off));
+  const int32_t* offs = reinterpret_cast<const int32_t*>(off(workspace, M.off_off));
+  const int32_t* perm = reinterpret_cast<const int32_t*>(off(workspace, M.perm_off));
+  const int32_t* inv = reinterpret_cast<const int32_t*>(off(workspace, M.inv_off));
+  BF* xs = reinterpret_cast<BF*>(off(workspace, M.xs_off));
+  BF* hs = reinterpret_cast<BF*>(off(workspace, M.hs_off));
+  float* o = reinterpret_cast<float*>(off(workspace, M.part_off));
+  BF* zs = reinterpret_cast<BF*>(off(workspace, B.zs_off));
+  float* dwk = reinterpret_cast<float*>(off(workspace, B.dw_off));
+  BF* dl = reinterpret_cast<BF*>(off(workspace, B.dl_off));
+  float* dxr = reinterpret_cast<float*>(off(workspace, B.dxr_off));
+  BF* gs = reinterpret_cast<BF*>(off(workspace, B.gs_off));
+  BF* dz = reinterpret_cast<BF*>(off(workspace, B.dz_off));
+  float* dxs = reinterpret_cast<float*>(off(workspace, B.dxs_off));
+  // (1) the forward's routing, dispatch and expert activations again, keeping z
+  if ((st = moe_routed(M, x, wr, w1p, w2p, workspace, idx, wts, zs, s)) != TP_OK) return st;
+  // (2) routing-weight gradients, then the router logits' through the softmax over the chosen k
+  {
+    ProfScope prof(s, "moe_bwd_route");
+    const int64_t warps = M.n_rows;
+    TP_LAUNCH_PDL(moe::route_weight_grad_kernel, dim3(static_cast<unsigned>(ceil_div(warps * 32, 256))),
+                  dim3(256), 0, s, static_cast<const BF*>(dy), static_cast<const float*>(o), inv,
+                  M.k, M.T, M.d, dwk);
+    const int64_t n = M.T * M.E;
+    TP_LAUNCH_PDL(moe::router_logit_grad_kernel, dim3(static_cast<unsigned>(ceil_div(n, 256))),
+                  dim3(256), 0, s, static_cast<const int32_t*>(idx), static_cast<const float*>(wts),
+                  static_cast<const float*>(dwk), M.k, M.T, M.E, dl);
+    // w * dy of every routed row, in expert order
+    TP_LAUNCH_PDL(moe::gather_scaled_kernel,
+                  dim3(static_cast<unsigned>(ceil_div(M.n_rows, moe::kGatherRowsPerBlock))),
+                  dim3(32 * moe::kGatherRowsPerBlock), 0, s, static_cast<const BF*>(dy), perm,
+                  static_cast<const float*>(wts), M.k, M.d, M.n_rows, gs);
+  }
+  // (3) dWr = x^T dl [d][E] and dx through the router dl Wr^T [T][d] (fp32)
+  {
+    simt::GemmArgs g{};
+    g.a = x; g.a_bs = 0; g.a_sm = 1; g.a_sk = M.d;
+    g.b = dl; g.b_bs = 0; g.b_sm = 1; g.b_sk = M.E;
+    g.out = dwr; g.o_bs = 0; g.o_sm = M.E; g.o_sn = 1;
+    g.M = M.d; g.N = M.E; g.K = M.T; g.batch = 1; g.out_f32 = 1;
+    if ((st = simt::gemm<BF>(g, s)) != TP_OK) return st;
+    simt::GemmArgs h{};
+    h.a = dl; h.a_bs = 0; h.a_sm = M.E; h.a_sk = 1;
+    h.b = wr; h.b_bs = 0; h.b_sm = M.E; h.b_sk = 1;
+    h.out = dxr; h.o_bs = 0; h.o_sm = M.d; h.o_sn = 1;
+    h.M = M.T; h.N = M.d; h.K = M.E; h.batch = 1; h.out_f32 = 1;
+    if ((st = simt::gemm<BF>(h, s)) != TP_OK) return st;
+  }
+  // (4) every chosen expert's MLP backward on its routed rows (their gradient w * dy): dW1, dW2
+  // into its slice of dw1p / dw2p, dx of the rows (shards summed in the accumulator) into dxs.
+  // The per-expert row counts come back to the host once.
+  {
+    std::vector<int32_t> hcnt(static_cast<size_t>(M.E)), hoff(static_cast<size_t>(M.E));
+    TP_CUDA_TRY(cudaMemcpyAsync(hcnt.data(), cnt, hcnt.size() * 4, cudaMemcpyDeviceToHost, s));
+    TP_CUDA_TRY(cudaMemcpyAsync(hoff.data(), offs, hoff.size() * 4, cudaMemcpyDeviceToHost, s));
+    TP_CUDA_TRY(cudaStreamSynchronize(s));
+    const int64_t zrow = L.p * L.R, hrow = L.p * L.Fsp;
+    for (int e = 0; e < M.E; ++e) {
+      const int64_t n = hcnt[static_cast<size_t>(e)], r0 = hoff[static_cast<size_t>(e)];
+      if (n == 0) continue;
+      tp_mlp_desc me{n, M.d, M.F, M.p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_FUSED, 0, 0.f};
+      MlpLayout Le;
+      if ((st = layout_of(&me, &Le)) != TP_OK) return st;
+      if ((st = tc_backward(Le, gs + r0 * M.d, xs + r0 * M.d, zs + r0 * zrow, hs + r0 * hrow,
+                            off(const_cast<void*>(w1p), e * L.w1p_bytes),
+                            off(const_cast<void*>(w2p), e * L.w2p_bytes), dz,
+                            dw1p + e * (L.w1p_bytes / 2), dw2p + e * (L.w2p_bytes / 2), nullptr,
+                            dxs + r0 * M.d, true, s)) != TP_OK)
+        return st;
+    }
+  }
+  // (5) the shared expert: its forward again (keeping z and h), then its MLP backward with dy
+  const float* dxsh = nullptr;
+  if (M.Fsh > 0) {
+    void* ws = off(workspace, M.shared_off);
+    void* h = off(workspace, B.hsh_off);
+    void* z = off(workspace, B.zsh_off);
+    void* sk = off(ws, M.sh.fsk_off);
+    const size_t skb = M.sh.fpart_off - M.sh.fsk_off;
+    float* dxs_sh = reinterpret_cast<float*>(off(workspace, B.dxsh_off));
+    if ((st = tc_up(M.sh, x, w1p_s, h, z, sk, skb, s)) != TP_OK) return st;
+    if ((st = tc_backward(M.sh, dy, x, z, h, w1p_s, w2p_s, off(workspace, B.dzs_off), dw1p_s,
+                          dw2p_s, nullptr, dxs_sh, true, s)) != TP_OK)
+      return st;
+    dxsh = dxs_sh;
+  }
+  // (6) dx = sum over the choices of the routed rows' input gradients + the router's + the
+  // shared expert's
+  {
+    ProfScope prof(s, "moe_bwd_combine");
+    const int64_t nv = M.T * (M.d / 8);
+    const int64_t blocks = std::min<int64_t>(ceil_div(nv, 256), static_cast<int64_t>(num_sms()) * 8);
+    TP_LAUNCH_PDL(moe::dx_combine_kernel, dim3(static_cast<unsigned>(blocks)), dim3(256), 0, s,
+                  static_cast<const float*>(dxs), static_cast<const float*>(dxr), dxsh, inv, M.k,
+                  M.T, M.d, static_cast<BF*>(dx));
+  }
   return TP_OK;
 }

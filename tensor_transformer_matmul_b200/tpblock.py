@@ -39,7 +39,7 @@ EXPORTS = (
     "tp_mlp_fwd_sp", "tp_mlp_bwd_sp_workspace", "tp_mlp_bwd_sp", "tp_attn_fwd_sp_workspace",
     "tp_attn_fwd_sp", "tp_moe_expert_w1_bytes", "tp_moe_expert_w2_bytes",
     "tp_moe_shared_w1_bytes", "tp_moe_shared_w2_bytes", "tp_moe_pack", "tp_moe_fwd_workspace",
-    "tp_moe_fwd", "tp_mlp_shard_sizes", "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
+    "tp_moe_fwd", "tp_moe_bwd_workspace", "tp_moe_bwd", "tp_mlp_shard_sizes", "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
     "tp_mlp_bwd_shard", "tp_attn_shard_sizes", "tp_attn_pack_shard", "tp_attn_fwd_shard",
     "tp_attn_bwd_shard", "tp_attn_bwd_sp_workspace", "tp_attn_bwd_sp",
 )
@@ -130,6 +130,8 @@ def load():
         "tp_moe_pack": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P]),
         "tp_moe_fwd_workspace": (S, [ED]),
         "tp_moe_fwd": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
+        "tp_moe_bwd_workspace": (S, [ED]),
+        "tp_moe_bwd": (I32, [ED, P, P, P, P, P, P, P, P, P, P, P, P, P, P, S, P]),
         "tp_profile_enable": (None, [I32]), "tp_profile_reset": (None, []),
         "tp_mlp_shard_sizes": (I32, [MD, I32, ctypes.POINTER(tp_shard_sizes)]),
         "tp_mlp_pack_shard": (I32, [MD, I32, P, P, P, P, P, P]),
@@ -507,6 +509,19 @@ def tp_moe_fwd(desc, x, wr, w1p, w2p, y, w1p_s=None, w2p_s=None, bias=None, resi
                              _ptr(w1p_s), _ptr(w2p_s), _ptr(bias), _ptr(residual), _ptr(y),
                              _ptr(route_idx), _ptr(route_w), _ptr(workspace), _nbytes(workspace),
                              _stream(stream)))
+
+
+def tp_moe_bwd_workspace(desc):
+    return load().tp_moe_bwd_workspace(ctypes.byref(desc))
+
+
+def tp_moe_bwd(desc, x, wr, w1p, w2p, dy, dx, dwr, dw1p, dw2p, w1p_s=None, w2p_s=None,
+               dw1p_s=None, dw2p_s=None, workspace=None, stream=None):
+    """dwr [d][E], dw1p / dw2p (E experts' packed layouts) and dw1p_s / dw2p_s: float32."""
+    _check(load().tp_moe_bwd(ctypes.byref(desc), _ptr(x), _ptr(wr), _ptr(w1p), _ptr(w2p),
+                             _ptr(w1p_s), _ptr(w2p_s), _ptr(dy), _ptr(dx), _ptr(dwr), _ptr(dw1p),
+                             _ptr(dw2p), _ptr(dw1p_s), _ptr(dw2p_s), _ptr(workspace),
+                             _nbytes(workspace), _stream(stream)))
 
 
 # ------------------------------------------------------------------------------ diagnostics

@@ -147,3 +147,63 @@ def test_moe_rejects(lib):
     assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 512, 0, 12, 2, 2)) == 0   # E % 8
     assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 512, 0, 16, 9, 2)) == 0   # top_k > 8
     assert lib.tp_moe_fwd_workspace(lib.moe_desc(8, 256, 510, 0, 16, 2, 4)) == 0   # p | d_ff
+
+
+@pytest.mark.parametrize("T,d,E,k,F,Fs,p", [
+    (200, 256, 16, 2, 512, 256, 2),    # few experts, shared expert
+    (150, 512, 64, 4, 256, 0, 4),      # no shared expert, four shards
+    (1, 256, 64, 8, 256, 256, 2),      # one token: eight experts of one row each
+    (300, 264, 128, 2, 384, 128, 1),   # ragged d, 128 experts (some chosen by no token), p = 1
+])
+def test_moe_backward_parity(lib, T, d, E, k, F, Fs, p):
+    # the backward recomputes the routing; the forward's routing of the same x gives the GPU's
+    # choice, and the oracle differentiates the block on that choice with its own weights
+    st = _setup(lib, T, d, E, k, F, Fs, p, seed=70 + T, with_bias=False, with_res=False)
+    _, idx, _ = _run(lib, st)
+    g = dev()
+    dy = inputs.normal((T, d), 1.0, 70 + T, 13, "bf16", "cpu")
+    desc = st["desc"]
+    dx = torch.empty(T, d, dtype=torch.bfloat16, device=g)
+    dwr = torch.empty(d, E, dtype=torch.float32, device=g)
+    dw1p = torch.full((st["w1p"].numel(),), float("nan"), dtype=torch.float32, device=g)
+    dw2p = torch.full((st["w2p"].numel(),), float("nan"), dtype=torch.float32, device=g)
+    dw1s = dw2s = None
+    if Fs:
+        dw1s = torch.empty(st["w1s"].numel(), dtype=torch.float32, device=g)
+        dw2s = torch.empty(st["w2s"].numel(), dtype=torch.float32, device=g)
+    ws = torch.empty(lib.tp_moe_bwd_workspace(desc), dtype=torch.uint8, device=g)
+    lib.tp_moe_bwd(desc, st["x"].to(g), st["wr"].to(g), st["w1p"], st["w2p"], dy.to(g), dx, dwr,
+                   dw1p, dw2p, w1p_s=st["w1s"], w2p_s=st["w2s"], dw1p_s=dw1s, dw2p_s=dw2s,
+                   workspace=ws)
+    torch.cuda.synchronize()
+    x, wr = f64(st["x"]), f64(st["wr"])
+    gi = idx.cpu().numpy().astype(np.int64)
+    experts = [tuple(f64(t) for t in e) for e in st["ex"]]
+    sh = None if st["sh"] is None else tuple(f64(t) for t in st["sh"])
+    ref = omoe.moe_backward(x, wr, experts, k, f64(dy), shared=sh,
+                            routing=(gi, omoe.weights_for(x, wr, gi)))
+    assert rel_l2(f64(dx), ref["dx"]) <= TOL["bf16"] and rel_l2_rows(f64(dx), ref["dx"]) <= TOL["bf16"]
+    assert rel_l2(f64(dwr), ref["dwr"]) <= TOL["bf16"]
+    # each expert's gradient, unpacked from its slice of the packed gradients
+    md = lib.mlp_desc(T, d, F, p, "swiglu", "bf16")
+    n1, n2 = st["w1p"].numel() // E, st["w2p"].numel() // E
+    used = set(gi.ravel().tolist())
+    for e in range(E):
+        a = (torch.empty(d, F, dtype=torch.float32, device=g), torch.empty(d, F, dtype=torch.float32, device=g),
+             torch.empty(F, d, dtype=torch.float32, device=g))
+        lib.tp_mlp_unpack_grads(md, dw1p[e * n1:(e + 1) * n1], dw2p[e * n2:(e + 1) * n2], *a)
+        torch.cuda.synchronize()
+        r = ref["experts"][e]
+        if e not in used:
+            assert all(not t.any() for t in a), e   # zeros, not left over
+            continue
+        for t, name in zip(a, ("dwg", "dwu", "dw2")):
+            assert rel_l2(f64(t), r[name]) <= TOL["bf16"], (e, name)
+    if Fs:
+        ms = lib.mlp_desc(T, d, Fs, p, "swiglu", "bf16")
+        a = (torch.empty(d, Fs, dtype=torch.float32, device=g), torch.empty(d, Fs, dtype=torch.float32, device=g),
+             torch.empty(Fs, d, dtype=torch.float32, device=g))
+        lib.tp_mlp_unpack_grads(ms, dw1s, dw2s, *a)
+        torch.cuda.synchronize()
+        for t, name in zip(a, ("dwg", "dwu", "dw2")):
+            assert rel_l2(f64(t), ref["shared"][name]) <= TOL["bf16"], name
