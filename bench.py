@@ -647,7 +647,38 @@ def extra_moe(tp, inputs, torch, stream, peaks, steps):
                      "frac_of_roofline": round(max(t_hbm, t_tc) / ms, 3),
                      "tokens_per_s": round(T / (ms / 1e3), 1),
                      "kernels": {kk: {"ms_per_launch": round(v[1] / v[0], 4)} for kk, v in prof.items()}}
-        del ws, x, y
+        if name == "prefill":
+            # the backward: routing and expert activations recomputed, then every chosen expert's
+            # MLP backward (expert by expert after one read-back of the row counts), the router's
+            # and the shared expert's; fp32 gradients of all 22.7 GB of weights
+            del ws
+            torch.cuda.empty_cache()
+            wsb = torch.empty(tp.tp_moe_bwd_workspace(desc), dtype=torch.uint8, device=dev)
+            dy = inputs.normal((T, d), 1.0, 0, 903, "bf16", dev)
+            dx = torch.empty(T, d, dtype=torch.bfloat16, device=dev)
+            dwr = torch.empty(d, E, dtype=torch.float32, device=dev)
+            dw1 = torch.empty(w1p.numel(), dtype=torch.float32, device=dev)
+            dw2 = torch.empty(w2p.numel(), dtype=torch.float32, device=dev)
+            dws1 = torch.empty(w1s.numel(), dtype=torch.float32, device=dev)
+            dws2 = torch.empty(w2s.numel(), dtype=torch.float32, device=dev)
+
+            def bwd():
+                tp.tp_moe_bwd(desc, x, wr, w1p, w2p, dy, dx, dwr, dw1, dw2, w1p_s=w1s, w2p_s=w2s,
+                              dw1p_s=dws1, dw2p_s=dws2, workspace=wsb)
+
+            bwd()
+            nb = 3
+            ms_b = _cuda_time(bwd, nb, stream) / nb
+            # recomputed forward (without the combine) + the backward GEMMs (2x the forward's)
+            out[name]["backward"] = {
+                "ms": round(ms_b, 2), "steps": nb,
+                "TFLOP_per_s": round(3 * flops / (ms_b / 1e3) / 1e12, 1),
+                "grad_bytes_written": 4 * (dw1.numel() + dw2.numel() + dws1.numel() + dws2.numel()),
+                "note": "routed experts differentiated one by one (host loop over the 256 experts)"}
+            del wsb, dy, dx, dwr, dw1, dw2, dws1, dws2
+        else:
+            del ws
+        del x, y
         torch.cuda.empty_cache()
     out["steps"] = steps
     del w1p, w2p, w1s, w2s

@@ -1269,15 +1269,16 @@ extern "C" tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const vo
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   if (!dwr || !dw1p || !dw2p || (M.Fsh > 0 && (!dw1p_s || !dw2p_s)))
     return set_error(TP_ERR_INVALID_ARG, "null gradient pointer");
-  // every gradient starts at zero: an expert no token chose keeps it
-  TP_CUDA_TRY(cudaMemsetAsync(dwr, 0, static_cast<size_t>(M.d) * M.E * 4, s));
-  TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(M.E) * L.w1p_bytes * 2, s));
-  TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(M.E) * L.w2p_bytes * 2, s));
-  if (M.Fsh > 0) {
-    TP_CUDA_TRY(cudaMemsetAsync(dw1p_s, 0, M.sh.w1p_bytes * 2, s));
-    TP_CUDA_TRY(cudaMemsetAsync(dw2p_s, 0, M.sh.w2p_bytes * 2, s));
+  if (M.T == 0) {   // no tokens: every gradient is zero
+    TP_CUDA_TRY(cudaMemsetAsync(dwr, 0, static_cast<size_t>(M.d) * M.E * 4, s));
+    TP_CUDA_TRY(cudaMemsetAsync(dw1p, 0, static_cast<size_t>(M.E) * L.w1p_bytes * 2, s));
+    TP_CUDA_TRY(cudaMemsetAsync(dw2p, 0, static_cast<size_t>(M.E) * L.w2p_bytes * 2, s));
+    if (M.Fsh > 0) {
+      TP_CUDA_TRY(cudaMemsetAsync(dw1p_s, 0, M.sh.w1p_bytes * 2, s));
+      TP_CUDA_TRY(cudaMemsetAsync(dw2p_s, 0, M.sh.w2p_bytes * 2, s));
+    }
+    return TP_OK;
   }
-  if (M.T == 0) return TP_OK;
   if (!x || !wr || !w1p || !w2p || !dy || !dx) return set_error(TP_ERR_INVALID_ARG, "null pointer");
   if (M.Fsh > 0 && (!w1p_s || !w2p_s))
     return set_error(TP_ERR_INVALID_ARG, "the shared expert's packed weights are null");
@@ -1351,7 +1352,11 @@ extern "C" tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const vo
     const int64_t zrow = L.p * L.R, hrow = L.p * L.Fsp;
     for (int e = 0; e < M.E; ++e) {
       const int64_t n = hcnt[static_cast<size_t>(e)], r0 = hoff[static_cast<size_t>(e)];
-      if (n == 0) continue;
+      if (n == 0) {   // an expert no token chose: zero gradients
+        TP_CUDA_TRY(cudaMemsetAsync(dw1p + e * (L.w1p_bytes / 2), 0, L.w1p_bytes * 2, s));
+        TP_CUDA_TRY(cudaMemsetAsync(dw2p + e * (L.w2p_bytes / 2), 0, L.w2p_bytes * 2, s));
+        continue;
+      }
       tp_mlp_desc me{n, M.d, M.F, M.p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_FUSED, 0, 0.f};
       MlpLayout Le;
       if ((st = layout_of(&me, &Le)) != TP_OK) return st;
