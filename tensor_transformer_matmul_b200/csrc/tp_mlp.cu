@@ -1218,6 +1218,21 @@ extern "C" tp_status tp_moe_fwd(const tp_moe_desc* desc, const void* x, const vo
 
 // ------------------------------------------------------------------ MoE backward
 namespace {
+// Streams on which the routed experts' backward GEMMs run side by side (created once per
+// device, non-blocking; forked from and joined back to the caller's stream with events).
+constexpr int kMoeStreams = 8;
+tp_status moe_streams(cudaStream_t (&out)[kMoeStreams]) {
+  static cudaStream_t pool[64][kMoeStreams] = {};
+  int dev = 0;
+  TP_CUDA_TRY(cudaGetDevice(&dev));
+  if (dev >= 64) return set_error(TP_ERR_UNSUPPORTED, "device index above 63");
+  for (int j = 0; j < kMoeStreams; ++j) {
+    if (!pool[dev][j]) TP_CUDA_TRY(cudaStreamCreateWithFlags(&pool[dev][j], cudaStreamNonBlocking));
+    out[j] = pool[dev][j];
+  }
+  return TP_OK;
+}
+
 // Backward workspace: the forward's regions, then the backward's own.
 struct MoeBwdLayout {
   size_t zs_off, dw_off, dl_off, dxr_off, gs_off, dz_off, dxs_off, zsh_off, hsh_off, dzs_off,
@@ -1343,30 +1358,47 @@ extern "C" tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const vo
   }
   // (4) every chosen expert's MLP backward on its routed rows (their gradient w * dy): dW1, dW2
   // into its slice of dw1p / dw2p, dx of the rows (shards summed in the accumulator) into dxs.
-  // The per-expert row counts come back to the host once.
+  // The per-expert row counts come back to the host once.  Each expert works on its own rows of
+  // every buffer (dz included), so the experts run side by side on kMoeStreams streams.
   {
     std::vector<int32_t> hcnt(static_cast<size_t>(M.E)), hoff(static_cast<size_t>(M.E));
     TP_CUDA_TRY(cudaMemcpyAsync(hcnt.data(), cnt, hcnt.size() * 4, cudaMemcpyDeviceToHost, s));
     TP_CUDA_TRY(cudaMemcpyAsync(hoff.data(), offs, hoff.size() * 4, cudaMemcpyDeviceToHost, s));
     TP_CUDA_TRY(cudaStreamSynchronize(s));
+    cudaStream_t pool[kMoeStreams];
+    if ((st = moe_streams(pool)) != TP_OK) return st;
+    cudaEvent_t ev[kMoeStreams + 1];
+    for (auto& e : ev) TP_CUDA_TRY(cudaEventCreateWithFlags(&e, cudaEventDisableTiming));
+    TP_CUDA_TRY(cudaEventRecord(ev[kMoeStreams], s));
+    for (int j = 0; j < kMoeStreams; ++j) TP_CUDA_TRY(cudaStreamWaitEvent(pool[j], ev[kMoeStreams], 0));
     const int64_t zrow = L.p * L.R, hrow = L.p * L.Fsp;
-    for (int e = 0; e < M.E; ++e) {
+    int next = 0;
+    for (int e = 0; e < M.E && st == TP_OK; ++e) {
       const int64_t n = hcnt[static_cast<size_t>(e)], r0 = hoff[static_cast<size_t>(e)];
+      cudaStream_t se = pool[next];
+      next = next + 1 == kMoeStreams ? 0 : next + 1;
       if (n == 0) {   // an expert no token chose: zero gradients
-        TP_CUDA_TRY(cudaMemsetAsync(dw1p + e * (L.w1p_bytes / 2), 0, L.w1p_bytes * 2, s));
-        TP_CUDA_TRY(cudaMemsetAsync(dw2p + e * (L.w2p_bytes / 2), 0, L.w2p_bytes * 2, s));
+        if (cudaMemsetAsync(dw1p + e * (L.w1p_bytes / 2), 0, L.w1p_bytes * 2, se) != cudaSuccess ||
+            cudaMemsetAsync(dw2p + e * (L.w2p_bytes / 2), 0, L.w2p_bytes * 2, se) != cudaSuccess)
+          st = set_error(TP_ERR_CUDA, "cudaMemsetAsync of an unchosen expert's gradients");
         continue;
       }
       tp_mlp_desc me{n, M.d, M.F, M.p, TP_ACT_SWIGLU, TP_BF16, TP_REDUCE_FUSED, 0, 0.f};
       MlpLayout Le;
-      if ((st = layout_of(&me, &Le)) != TP_OK) return st;
-      if ((st = tc_backward(Le, gs + r0 * M.d, xs + r0 * M.d, zs + r0 * zrow, hs + r0 * hrow,
-                            off(const_cast<void*>(w1p), e * L.w1p_bytes),
-                            off(const_cast<void*>(w2p), e * L.w2p_bytes), dz,
-                            dw1p + e * (L.w1p_bytes / 2), dw2p + e * (L.w2p_bytes / 2), nullptr,
-                            dxs + r0 * M.d, true, s)) != TP_OK)
-        return st;
+      if ((st = layout_of(&me, &Le)) != TP_OK) break;
+      st = tc_backward(Le, gs + r0 * M.d, xs + r0 * M.d, zs + r0 * zrow, hs + r0 * hrow,
+                       off(const_cast<void*>(w1p), e * L.w1p_bytes),
+                       off(const_cast<void*>(w2p), e * L.w2p_bytes), dz + r0 * zrow,
+                       dw1p + e * (L.w1p_bytes / 2), dw2p + e * (L.w2p_bytes / 2), nullptr,
+                       dxs + r0 * M.d, true, se);
     }
+    // join: the caller's stream waits for every expert's work (also on an error, so that nothing
+    // of this call is left running unordered behind it)
+    for (int j = 0; j < kMoeStreams; ++j) {
+      if (cudaEventRecord(ev[j], pool[j]) == cudaSuccess) (void)cudaStreamWaitEvent(s, ev[j], 0);
+    }
+    for (auto& e : ev) (void)cudaEventDestroy(e);
+    if (st != TP_OK) return st;
   }
   // (5) the shared expert: its forward again (keeping z and h), then its MLP backward with dy
   const float* dxsh = nullptr;
