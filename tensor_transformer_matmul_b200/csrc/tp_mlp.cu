@@ -1341,20 +1341,30 @@ extern "C" tp_status tp_moe_bwd(const tp_moe_desc* desc, const void* x, const vo
                   dim3(32 * moe::kGatherRowsPerBlock), 0, s, static_cast<const BF*>(dy), perm,
                   static_cast<const float*>(wts), M.k, M.d, M.n_rows, gs);
   }
-  // (3) dWr = x^T dl [d][E] and dx through the router dl Wr^T [T][d] (fp32)
+  // (3) dWr = x^T dl [d][E] (x and dl read MN-major) and dx through the router dl Wr^T [T][d]
+  // (dl and Wr read K-major), fp32, on the tensor cores
   {
-    simt::GemmArgs g{};
-    g.a = x; g.a_bs = 0; g.a_sm = 1; g.a_sk = M.d;
-    g.b = dl; g.b_bs = 0; g.b_sm = 1; g.b_sk = M.E;
-    g.out = dwr; g.o_bs = 0; g.o_sm = M.E; g.o_sn = 1;
-    g.M = M.d; g.N = M.E; g.K = M.T; g.batch = 1; g.out_f32 = 1;
-    if ((st = simt::gemm<BF>(g, s)) != TP_OK) return st;
-    simt::GemmArgs h{};
-    h.a = dl; h.a_bs = 0; h.a_sm = M.E; h.a_sk = 1;
-    h.b = wr; h.b_bs = 0; h.b_sm = M.E; h.b_sk = 1;
-    h.out = dxr; h.o_bs = 0; h.o_sm = M.d; h.o_sn = 1;
-    h.M = M.T; h.N = M.d; h.K = M.E; h.batch = 1; h.out_f32 = 1;
-    if ((st = simt::gemm<BF>(h, s)) != TP_OK) return st;
+    const Operand xa{x, true, M.d, M.T, 1, M.d, 0};
+    const Operand lb{dl, true, M.E, M.T, 1, M.E, 0};
+    tc::EpiStoreF32::Params ep;
+    ep.out = dwr;
+    ep.ld = M.E;
+    ep.batch_stride = 0;
+    ep.rows_valid = static_cast<int32_t>(M.d);
+    ep.cols_valid = M.E;
+    ep.swap = 0;
+    st = tc::run_gemm<TileCfg<128, 1, true, true, stages_for(128, 1)>, tc::EpiStoreF32>(
+        xa, lb, M.d, M.E, M.T, 1, ep, s, "moe_bwd_dwr_gemm");
+    if (st != TP_OK) return st;
+    const Operand la{dl, false, M.T, M.E, 1, M.E, 0};
+    const Operand wb{wr, false, M.d, M.E, 1, M.E, 0};
+    ep.out = dxr;
+    ep.ld = M.d;
+    ep.rows_valid = static_cast<int32_t>(M.T);
+    ep.cols_valid = static_cast<int32_t>(M.d);
+    st = tc::run_gemm<TileCfg<128, 1, false, false, stages_for(128, 1)>, tc::EpiStoreF32>(
+        la, wb, M.T, M.d, M.E, 1, ep, s, "moe_bwd_dxr_gemm");
+    if (st != TP_OK) return st;
   }
   // (4) every chosen expert's MLP backward on its routed rows (their gradient w * dy): dW1, dW2
   // into its slice of dw1p / dw2p, dx of the rows (shards summed in the accumulator) into dxs.
