@@ -39,7 +39,8 @@ EXPORTS = (
     "tp_mlp_fwd_sp", "tp_mlp_bwd_sp_workspace", "tp_mlp_bwd_sp", "tp_attn_fwd_sp_workspace",
     "tp_attn_fwd_sp", "tp_moe_expert_w1_bytes", "tp_moe_expert_w2_bytes",
     "tp_moe_shared_w1_bytes", "tp_moe_shared_w2_bytes", "tp_moe_pack", "tp_moe_fwd_workspace",
-    "tp_moe_fwd", "tp_moe_bwd_workspace", "tp_moe_bwd", "tp_mlp_shard_sizes", "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
+    "tp_moe_fwd", "tp_moe_bwd_workspace", "tp_moe_bwd", "tp_mlp_shard_sizes",
+    "tp_mlp_pack_shard", "tp_mlp_fwd_shard",
     "tp_mlp_bwd_shard", "tp_attn_shard_sizes", "tp_attn_pack_shard", "tp_attn_fwd_shard",
     "tp_attn_bwd_shard", "tp_attn_bwd_sp_workspace", "tp_attn_bwd_sp",
 )

@@ -203,6 +203,17 @@ def test_moe_layout_and_argument_errors(lib):
     assert so.tp_moe_fwd(ctypes.byref(d), None, fake, fake, fake, fake, fake, None, None, fake,
                          None, None, fake, 1 << 40, None) == lib.TP_ERR_INVALID_ARG
     lib.tp_reset_reduction_count()
+    # the backward: its workspace holds the forward's and more; argument errors before any enqueue
+    assert lib.tp_moe_bwd_workspace(d) > lib.tp_moe_fwd_workspace(d)
+    assert lib.tp_moe_bwd_workspace(lib.moe_desc(64, 256, 512, 0, 12, 2, 2)) == 0
+    args = [fake] * 6 + [fake, fake]          # x, wr, w1p, w2p, w1p_s, w2p_s, dy, dx
+    grads = [fake, fake, fake, fake, fake]    # dwr, dw1p, dw2p, dw1p_s, dw2p_s
+    assert so.tp_moe_bwd(ctypes.byref(d), *args, None, *grads[1:], fake, 1 << 40,
+                         None) == lib.TP_ERR_INVALID_ARG          # dwr null
+    assert so.tp_moe_bwd(ctypes.byref(d), *args, *grads[:3], None, fake, fake, 1 << 40,
+                         None) == lib.TP_ERR_INVALID_ARG          # the shared expert's dw1p null
+    assert so.tp_moe_bwd(ctypes.byref(d), *args, *grads, fake, 64,
+                         None) == lib.TP_ERR_WORKSPACE            # workspace too small
 
 
 def test_moe_pack_and_sp_backward_argument_errors(lib):
