@@ -108,6 +108,8 @@ def _check(st, y, idx, w):
     (150, 512, 64, 4, 256, 0, 4),      # tensor-core router, no shared expert
     (1, 256, 64, 8, 256, 256, 2),      # one token (decode), eight experts
     (300, 264, 128, 2, 384, 128, 1),   # ragged d, 128 experts, p = 1
+    (400, 256, 8, 2, 256, 128, 2),     # ~100 rows per expert, some with two row blocks
+    (600, 256, 8, 4, 512, 0, 4),       # ~300 rows per expert: three 128-row blocks
 ])
 def test_moe_forward_parity(lib, T, d, E, k, F, Fs, p):
     st = _setup(lib, T, d, E, k, F, Fs, p, seed=50 + T)
@@ -134,6 +136,22 @@ def test_moe_skewed_routing(lib):
     _check(st, y, idx, w)
 
 
+def test_moe_skewed_routing_many_blocks(lib):
+    # as above with few experts: experts 0 and 1 each receive all 600 tokens (five 128-row
+    # blocks apiece, the last part-filled)
+    st = _setup(lib, 600, 256, 8, 2, 256, 128, 2, seed=62)
+    wr = st["wr"].float()
+    wr[:, 0] += 0.5 * torch.sign(st["x"].float().sum(0))
+    wr[:, 1] += 0.45 * torch.sign(st["x"].float().sum(0))
+    st["wr"] = wr.to(torch.bfloat16)
+    st["x"] = (st["x"].float() + torch.sign(st["x"].float().sum(0))).to(torch.bfloat16)
+    y, idx, w = _run(lib, st)
+    torch.cuda.synchronize()
+    counts = torch.bincount(idx.flatten().long().cpu(), minlength=8)
+    assert counts[0] == 600 and counts[1] == 600 and counts[2:].sum() == 0
+    _check(st, y, idx, w)
+
+
 def test_moe_deterministic(lib):
     st = _setup(lib, 180, 256, 64, 2, 256, 128, 2, seed=60)
     a = [t.clone() for t in _run(lib, st)]
@@ -154,6 +172,7 @@ def test_moe_rejects(lib):
     (150, 512, 64, 4, 256, 0, 4),      # no shared expert, four shards
     (1, 256, 64, 8, 256, 256, 2),      # one token: eight experts of one row each
     (300, 264, 128, 2, 384, 128, 1),   # ragged d, 128 experts (some chosen by no token), p = 1
+    (600, 256, 8, 4, 256, 128, 2),     # ~300 rows per expert: several row blocks each
 ])
 def test_moe_backward_parity(lib, T, d, E, k, F, Fs, p):
     # the backward recomputes the routing; the forward's routing of the same x gives the GPU's
