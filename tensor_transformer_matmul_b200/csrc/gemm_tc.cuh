@@ -978,17 +978,52 @@ struct EpiReduceOut {
   __device__ __forceinline__ static void run(const Params& p, const GemmParams&, const EpiCtx& c,
                                              const Src& src) {
     if (!p.swap) {
+      // one thread per output row: a whole 32-column chunk goes out as 16-byte stores (and the
+      // residual comes in as 16-byte loads); chunks at the right edge or off 16-byte alignment
+      // take the element path.  Both add the residual in fp32 and round the same way.
       const int i = c.m0 + c.row;
       const bool live = i < p.rows_valid;
+      const int eb = p.out_bf16 ? 2 : 4;
 #pragma unroll 1
       for (int col = 0; col < Cfg::BN; col += 32) {
         float v[32];
         src.load32(col, v);
         if (!live) continue;
         const int j0 = c.n0 + col;
+        const int64_t idx0 = static_cast<int64_t>(i) * p.ld + j0;
+        const uintptr_t oa = reinterpret_cast<uintptr_t>(p.out) + idx0 * eb;
+        const uintptr_t ra = reinterpret_cast<uintptr_t>(p.residual) + idx0 * eb;
+        if (j0 + 32 <= p.cols_valid && (oa & 15) == 0 && (ra & 15) == 0) {
+          if (p.out_bf16) {
+            if (p.residual) {
+              float r[32];
+              load_bf16x32(reinterpret_cast<const __nv_bfloat16*>(ra), r);
+#pragma unroll
+              for (int e = 0; e < 32; ++e) v[e] = r[e] + v[e];
+            }
+            store_bf16x32(reinterpret_cast<__nv_bfloat16*>(oa), v);
+          } else {
+            if (p.residual) {
+              const float4* r4 = reinterpret_cast<const float4*>(ra);
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                const float4 r = r4[q];
+                v[4 * q] = r.x + v[4 * q];
+                v[4 * q + 1] = r.y + v[4 * q + 1];
+                v[4 * q + 2] = r.z + v[4 * q + 2];
+                v[4 * q + 3] = r.w + v[4 * q + 3];
+              }
+            }
+            float4* d4 = reinterpret_cast<float4*>(oa);
+#pragma unroll
+            for (int q = 0; q < 8; ++q)
+              d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          }
+          continue;
+        }
 #pragma unroll
         for (int e = 0; e < 32; ++e)
-          if (j0 + e < p.cols_valid) put(p, static_cast<int64_t>(i) * p.ld + j0 + e, v[e]);
+          if (j0 + e < p.cols_valid) put(p, idx0 + e, v[e]);
       }
     } else {
       const int j = c.m0 + c.row;
