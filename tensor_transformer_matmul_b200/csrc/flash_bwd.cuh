@@ -9,24 +9,26 @@
 //
 // Two kernels, neither with atomics (each output tile is summed by one CTA in a fixed order):
 //   * dK/dV: one CTA per (128-key block, KV head, query head of its group, sequence).  It walks
-//     the query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in TMEM,
-//     the 256 threads (one key row and one half of the 128 queries each) turn them into P^T and
-//     dS^T, written back as bf16 over their own TMEM columns, and dV += P^T dO, dK += dS^T Q
-//     accumulate in TMEM with P^T and dS^T as the TMEM A operands (dO and Q read MN-major).
-//     Q and dO are double buffered, so the next step's tiles load during this one.  The
-//     per-head shares are added afterwards.
+//     the 64-query blocks that see its keys; per step S^T = K Q^T and dP^T = V dO^T land in one
+//     of two TMEM buffers, the 256 compute threads (one key row and one half of the 64 queries
+//     each) turn them into P^T and dS^T, written back as bf16 over their own TMEM columns, and
+//     dV += P^T dO, dK += dS^T Q accumulate in TMEM with P^T and dS^T as the TMEM A operands
+//     (dO and Q read MN-major).  A ninth warp issues the MMAs and loads, so the next step's
+//     S^T/dP^T are ready while the threads work on this one; Q and dO stream through a ring of
+//     four 64-row slots.  The per-head shares are added afterwards.
 //   * dQ: one CTA per (128-query block, query head, sequence).  It walks the key blocks its
 //     queries see; per step S = Q K^T and dP = dO V^T land in TMEM, the threads (one query row
 //     and one half of the 128 keys each) write dS back over S, and dQ += dS K accumulates in
 //     TMEM (K read MN-major).  K and V are double buffered.
-// Thread 0 issues the TMA loads and the MMAs; TMEM holds four (three) 128-column fp32 tiles.
-// The next step's S^T/dP^T (S/dP) MMAs are issued right behind this step's dV/dK (dQ) MMAs: the
-// MMAs run in issue order, so they overwrite P^T and dS^T (dS) only after those have been read,
-// and their completion also means the previous step's MMAs are done.
-// The two thread halves (warps 0-3 and 4-7) read the same TMEM lanes, columns 0-63 and 64-127;
-// half h packs its 64 bf16 results into columns 64 h .. 64 h + 31, which only it reads, so the
-// halves need no ordering between them.  The MMA that consumes them takes queries (keys)
-// 0-63 from columns 0-31 and 64-127 from columns 64-95.
+// In the dQ kernel thread 0 issues the TMA loads and the MMAs; TMEM holds three 128-column fp32
+// tiles.  The next step's S/dP MMAs are issued right behind this step's dQ MMAs: the MMAs run
+// in issue order, so they overwrite dS only after it has been read, and their completion also
+// means the previous step's MMAs are done.  The dK/dV kernel's issuing warp uses the same
+// order, two steps ahead: step it's dV/dK MMAs, then step it+2's S^T/dP^T into the buffer they
+// have just read.
+// The two thread halves (warps 0-3 and 4-7) read the same TMEM lanes and split a step's columns
+// in two; half h packs its bf16 results into the first half of its own columns, which only it
+// reads, so the halves need no ordering between them.
 // Every wait is bounded; a timeout sets the abort flag, drains what was issued and leaves, and
 // the loop exit is CTA-uniform.
 #pragma once
@@ -110,28 +112,68 @@ struct Drain {
 };
 
 // ================================================================================ dK and dV
+// Steps of 64 queries.  S^T/dP^T have two TMEM buffers of 64 + 64 columns next to dV and dK
+// (128 each), so the MMAs of step it+1 are already done while the 256 compute threads turn step
+// it into P^T/dS^T.  A ninth warp issues: when all 256 threads have stored step it's P^T/dS^T
+// (an mbarrier of 256 arrivals) its elected thread issues step it's dV/dK MMAs and then step
+// it+2's S^T/dP^T into the same buffer (issue order keeps the overwrite behind the reads), so
+// the compute threads never wait for the issue.  Q and dO stream through a ring of kRing 64-row
+// slots, loaded three steps ahead.
+constexpr int kQStep = 64;   // queries per step of the dK/dV kernel (keys per step of dQ)
+constexpr int kRing = 4;     // 64-row Q/dO (K/V) slots
+constexpr int kThreadsIssue = kThreads + 32;   // compute threads plus the issuing warp
+constexpr int kIssuer = kThreads;              // the issuing thread
+
+// barrier 1 over the 256 compute threads (the issuing warp does not take part), returning the
+// AND of v over them
+__device__ __forceinline__ int compute_bar_and(int v) {
+  int out;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\tsetp.ne.s32 p, %1, 0;\n\t"
+      "bar.red.and.pred q, 1, %2, p;\n\tselp.s32 %0, 1, 0, q;\n\t}\n"
+      : "=r"(out)
+      : "r"(v), "n"(kThreads)
+      : "memory");
+  return out;
+}
+
 template <int HD>
-__global__ void __launch_bounds__(kThreads, 1)
+struct Tiles64 {
+  static constexpr int TILE = kQStep * 128;           // one 64-row, 128-byte-wide sub-tile
+  static constexpr int BLOCK = Tiles<HD>::SUB * TILE; // one 64-row head tile
+};
+
+// TMEM column, from a 64-column buffer's start, of the packed bf16 pairs that the k-th
+// 16-row MMA step reads: half h of the threads packs its 32 rows into columns 32 h .. 32 h + 15
+__device__ __forceinline__ uint32_t packed_col64(int kk) {
+  return static_cast<uint32_t>(32 * (kk >> 1) + 8 * (kk & 1));
+}
+
+template <int HD>
+__global__ void __launch_bounds__(kThreadsIssue, 1)
     flash_bwd_dkv_kernel(const __grid_constant__ CUtensorMap tma_qkv,
-                         const __grid_constant__ CUtensorMap tma_do, const Params P) {
+                         const __grid_constant__ CUtensorMap tma_q64,
+                         const __grid_constant__ CUtensorMap tma_do64, const Params P) {
   using namespace sm100;
   using L = Tiles<HD>;
+  using Q = Tiles64<HD>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~static_cast<uintptr_t>(1023));
   uint8_t* sK = smem;
   uint8_t* sV = sK + L::BLOCK;
-  uint8_t* sQ = sV + L::BLOCK;        // [2] buffers
-  uint8_t* sDO = sQ + 2 * L::BLOCK;   // [2] buffers
-  float* lse_s = reinterpret_cast<float*>(sDO + 2 * L::BLOCK);   // [2][kBlk]
-  float* D_s = lse_s + 2 * kBlk;                                   // [2][kBlk]
-  uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + 2 * kBlk);
+  uint8_t* sQ = sV + L::BLOCK;            // [kRing] slots
+  uint8_t* sDO = sQ + kRing * Q::BLOCK;   // [kRing] slots
+  float* lse_s = reinterpret_cast<float*>(sDO + kRing * Q::BLOCK);   // [2][kQStep]
+  float* D_s = lse_s + 2 * kQStep;                                     // [2][kQStep]
+  uint64_t* bar = reinterpret_cast<uint64_t*>(D_s + 2 * kQStep);
   uint64_t* kv_full = bar + 0;
-  uint64_t* qd_full = bar + 1;   // [2]
-  uint64_t* s_full = bar + 3;
-  uint64_t* m_done = bar + 4;
-  uint64_t* drain = bar + 5;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(bar + 6);
+  uint64_t* qd_full = bar + 1;            // [kRing]
+  uint64_t* s_full = qd_full + kRing;     // [2]
+  uint64_t* m_done = s_full + 2;          // [2]
+  uint64_t* p_ready = m_done + 2;         // [2]: the 256 threads' P^T/dS^T of a step stored
+  uint64_t* drain = p_ready + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5;
@@ -142,21 +184,25 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int k_col = shard * P.R_a + (P.qh + gl) * HD;
   const int v_col = shard * P.R_a + (P.qh + P.kh + gl) * HD;
   const int k0 = kb * kBlk;
-  const int qb0 = P.causal ? kb : 0;
-  const int nqb = P.n_blk - qb0;
+  const int n64 = (P.s + kQStep - 1) / kQStep;
+  const int qb0 = P.causal ? k0 / kQStep : 0;   // first 64-query block that sees these keys
+  const int nqb = n64 - qb0;
   const int n_iter = heads * nqb;
 
   if (tid == 0) {
     mbar_init(kv_full, 1);
-    mbar_init(&qd_full[0], 1);
-    mbar_init(&qd_full[1], 1);
-    mbar_init(s_full, 1);
-    mbar_init(m_done, 1);
+    for (int i = 0; i < kRing; ++i) mbar_init(&qd_full[i], 1);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(&s_full[i], 1);
+      mbar_init(&m_done[i], 1);
+      mbar_init(&p_ready[i], kThreads);
+    }
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_barrier_init();
     tma_prefetch_desc(&tma_qkv);
-    tma_prefetch_desc(&tma_do);
+    tma_prefetch_desc(&tma_q64);
+    tma_prefetch_desc(&tma_do64);
   }
   if (warp == 0) {
     tmem_alloc(tmem_slot, 512);
@@ -166,182 +212,193 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  const uint32_t tS = tmem, tdP = tmem + 128, tdV = tmem + 256, tdK = tmem + 384;
+  // buffer b: S^T at 128 b, dP^T at 128 b + 64; dV at 256, dK at 384
+  const uint32_t tdV = tmem + 256, tdK = tmem + 384;
   const uint32_t lane_base = static_cast<uint32_t>((warp & 3) * 32) << 16;
   const int row = tid & (kBlk - 1);
-  const int half = tid >> 7;   // columns 64 half .. 64 half + 63
+  const int half = tid >> 7;   // queries 32 half .. 32 half + 31 of a step
   const int k_abs = k0 + row;
   auto wait = [&](uint64_t* b, uint32_t par, uint32_t site) {
     return mbar_wait(b, par, abort_flag, P.err, site);
   };
-  constexpr uint32_t IDESC_KK = make_idesc_bf16(128, 128, false, false);   // S^T, dP^T
-  constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);     // dV, dK
+  constexpr uint32_t IDESC_S = make_idesc_bf16(128, kQStep, false, false);   // S^T, dP^T
+  constexpr uint32_t IDESC_KN = make_idesc_bf16(128, HD, false, true);       // dV, dK
 
-  // step it -> (query head, query block)
+  // step it -> (query head, 64-query block)
   auto head_of = [&](int it) { return g * P.group + a0 + it / nqb; };
   auto block_of = [&](int it) { return qb0 + it % nqb; };
-  uint32_t nq[2] = {0, 0};   // Q/dO loads issued per buffer (thread 0)
+  uint32_t nq[kRing] = {0, 0, 0, 0};   // Q/dO loads issued per slot (issuing thread)
   bool any_mma = false;
   auto load_qd = [&](int it) {
-    const int b = it & 1, j = head_of(it), jl = j - shard * P.qh;
-    const int q_col = shard * P.R_a + jl * HD, q0 = block_of(it) * kBlk;
-    mbar_arrive_expect_tx(&qd_full[b], 2 * L::BLOCK);
+    const int r = it % kRing, j = head_of(it), jl = j - shard * P.qh;
+    const int q_col = shard * P.R_a + jl * HD, q0 = block_of(it) * kQStep;
+    mbar_arrive_expect_tx(&qd_full[r], 2 * Q::BLOCK);
 #pragma unroll
     for (int c = 0; c < L::SUB; ++c) {
-      tma_load_3d(&tma_qkv, &qd_full[b], sQ + b * L::BLOCK + c * L::TILE, q_col + 64 * c, q0, bi);
-      tma_load_3d(&tma_do, &qd_full[b], sDO + b * L::BLOCK + c * L::TILE, j * HD + 64 * c, q0, bi);
+      tma_load_3d(&tma_q64, &qd_full[r], sQ + r * Q::BLOCK + c * Q::TILE, q_col + 64 * c, q0, bi);
+      tma_load_3d(&tma_do64, &qd_full[r], sDO + r * Q::BLOCK + c * Q::TILE, j * HD + 64 * c, q0,
+                  bi);
     }
-    ++nq[b];
+    ++nq[r];
   };
-  // S^T = K Q(it)^T and dP^T = V dO(it)^T (thread 0)
+  // S^T = K Q(it)^T and dP^T = V dO(it)^T into buffer it & 1 (issuing thread)
   auto issue_s = [&](int it) {
-    const int b = it & 1;
-    const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ + b * L::BLOCK),
-                   da = smem_addr(sDO + b * L::BLOCK);
+    const int b = it & 1, r = it % kRing;
+    const uint32_t tS = tmem + 128 * b, tdP = tS + 64;
+    const uint32_t ka = smem_addr(sK), va = smem_addr(sV), qa = smem_addr(sQ + r * Q::BLOCK),
+                   da = smem_addr(sDO + r * Q::BLOCK);
 #pragma unroll
     for (int kk = 0; kk < HD / 16; ++kk) {
-      const uint32_t off = (kk >> 2) * L::TILE + (kk & 3) * 32;
-      umma_f16(tS, make_sdesc_sw128(ka + off, 16, 1024), make_sdesc_sw128(qa + off, 16, 1024),
-               IDESC_KK, kk > 0 ? 1u : 0u);
-      umma_f16(tdP, make_sdesc_sw128(va + off, 16, 1024), make_sdesc_sw128(da + off, 16, 1024),
-               IDESC_KK, kk > 0 ? 1u : 0u);
+      const uint32_t ok_ = (kk >> 2) * L::TILE + (kk & 3) * 32;
+      const uint32_t oq = (kk >> 2) * Q::TILE + (kk & 3) * 32;
+      umma_f16(tS, make_sdesc_sw128(ka + ok_, 16, 1024), make_sdesc_sw128(qa + oq, 16, 1024),
+               IDESC_S, kk > 0 ? 1u : 0u);
+      umma_f16(tdP, make_sdesc_sw128(va + ok_, 16, 1024), make_sdesc_sw128(da + oq, 16, 1024),
+               IDESC_S, kk > 0 ? 1u : 0u);
     }
-    umma_commit(s_full);
+    umma_commit(&s_full[b]);
     any_mma = true;
   };
-  // log-sum-exp and D of a step's 128 queries, double-buffered in shared memory: thread t < 128
+  // log-sum-exp and D of a step's 64 queries, double-buffered in shared memory: thread t < 64
   // loads step it+1's pair while step it runs and stores it before the step's barrier
   auto row_data = [&](int it, float& l, float& dd) {
-    const int t_abs = block_of(it) * kBlk + tid;
+    const int t_abs = block_of(it) * kQStep + tid;
     const bool valid = t_abs < P.s;
     const int64_t ri = (static_cast<int64_t>(bi) * P.s + t_abs) * P.n_q + head_of(it);
     l = valid ? P.lse[ri] : 0.f;
     dd = valid ? P.D[ri] : 0.f;
   };
-  if (tid < kBlk) {
+  if (tid < kQStep) {
     float l, dd;
     row_data(0, l, dd);
     lse_s[tid] = l;
     D_s[tid] = dd;
   }
   bool ok = true;
-  if (tid == 0) {
-    mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
+  __syncthreads();   // step 0's row data is in shared memory
+  if (tid >= kThreads) {
+    // ------------------------------------------------------------------ issuing warp
+    if (tid == kIssuer) {
+      mbar_arrive_expect_tx(kv_full, 2 * L::BLOCK);
 #pragma unroll
-    for (int c = 0; c < L::SUB; ++c) {
-      tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
-      tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
-    }
-    load_qd(0);
-    if (n_iter > 1) load_qd(1);
-    ok = wait(&qd_full[0], 0, DEVERR_WAIT_FULL) && wait(kv_full, 0, DEVERR_WAIT_FULL);
-    if (ok) {
-      tc_fence_after();
-      issue_s(0);
-    }
-  }
-  __syncthreads();
-  for (int it = 0; it < n_iter; ++it) {
-    const int q0 = block_of(it) * kBlk;
-    const float* lse_c = lse_s + (it & 1) * kBlk;
-    const float* D_c = D_s + (it & 1) * kBlk;
-    float nl = 0.f, nd = 0.f;
-    if (tid < kBlk && it + 1 < n_iter) row_data(it + 1, nl, nd);
-    // S^T(it) done: the MMAs run in issue order, so dV/dK of the previous step are done too and
-    // the other Q/dO buffer is free for step it+1
-    ok = __all_sync(0xffffffffu, ok && wait(s_full, it & 1, DEVERR_WAIT_ACC_FULL));
-    if (ok && tid == 0 && it >= 1 && it + 1 < n_iter) load_qd(it + 1);
-    // ---- P^T and dS^T for this key row against this thread's 64 of the block's queries,
-    // written as bf16 over the first half of this half's TMEM columns (all of this thread's S
-    // and dP are read before any of them is overwritten)
-    if (ok) {
-      tc_fence_after();
-      // no mask inside the block: every query is valid and (causal) after every key
-      const bool plain = q0 + kBlk <= P.s && k0 + kBlk <= P.s && (!P.causal || q0 > k0);
-      float sv[64], dp[64];
-      {
-        uint32_t r[4][32];
-        tmem_ld_32x32b_x32(tS + lane_base + 64 * half, r[0]);
-        tmem_ld_32x32b_x32(tS + lane_base + 64 * half + 32, r[1]);
-        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half, r[2]);
-        tmem_ld_32x32b_x32(tdP + lane_base + 64 * half + 32, r[3]);
-        tmem_wait_ld();
-#pragma unroll
-        for (int e = 0; e < 64; ++e) {
-          sv[e] = __uint_as_float(r[e >> 5][e & 31]);
-          dp[e] = __uint_as_float(r[2 + (e >> 5)][e & 31]);
+      for (int c = 0; c < L::SUB; ++c) {
+        tma_load_3d(&tma_qkv, kv_full, sK + c * L::TILE, k_col + 64 * c, k0, bi);
+        tma_load_3d(&tma_qkv, kv_full, sV + c * L::TILE, v_col + 64 * c, k0, bi);
+      }
+      for (int m = 0; m < kRing - 1 && m < n_iter; ++m) load_qd(m);
+      ok = wait(&qd_full[0], 0, DEVERR_WAIT_FULL) && wait(kv_full, 0, DEVERR_WAIT_FULL);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      if (ok && n_iter > 1) {
+        ok = wait(&qd_full[1], 0, DEVERR_WAIT_FULL);
+        if (ok) {
+          tc_fence_after();
+          issue_s(1);
         }
       }
+      for (int it = 0; ok && it < n_iter; ++it) {
+        const int b = it & 1, r = it % kRing;
+        const uint32_t tS = tmem + 128 * b, tdP = tS + 64;
+        ok = wait(&p_ready[b], (it >> 1) & 1, DEVERR_WAIT_ACC_EMPTY);
+        if (!ok) break;
+        tc_fence_after();
+        const uint32_t qa = smem_addr(sQ + r * Q::BLOCK), da = smem_addr(sDO + r * Q::BLOCK);
 #pragma unroll
-      for (int c = 0; c < 2; ++c) {
-        const int c0 = 64 * half + 32 * c;
+        for (int kk = 0; kk < kQStep / 16; ++kk) {
+          // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
+          // MN-major (N = dim), 16 query rows per MMA
+          fa::umma_f16_tmem_a(tdV, tS + packed_col64(kk),
+                              make_sdesc_sw128(da + kk * 16 * 128, Q::TILE, 1024), IDESC_KN,
+                              (it > 0 || kk > 0) ? 1u : 0u);
+          fa::umma_f16_tmem_a(tdK, tdP + packed_col64(kk),
+                              make_sdesc_sw128(qa + kk * 16 * 128, Q::TILE, 1024), IDESC_KN,
+                              (it > 0 || kk > 0) ? 1u : 0u);
+        }
+        umma_commit(&m_done[b]);
+        // step it+2's S^T and dP^T into this buffer, behind the MMAs that read it
+        if (it + 2 < n_iter) {
+          ok = wait(&qd_full[(it + 2) % kRing], ((it + 2) / kRing) & 1, DEVERR_WAIT_FULL);
+          if (!ok) break;
+          tc_fence_after();
+          issue_s(it + 2);
+        }
+        // step it+3's Q and dO into the slot of step it-1, whose dV/dK MMAs are then done
+        if (it + kRing - 1 < n_iter) {
+          if (it >= 1) ok = wait(&m_done[b ^ 1], ((it - 1) >> 1) & 1, DEVERR_WAIT_ACC_EMPTY);
+          if (!ok) break;
+          load_qd(it + kRing - 1);
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ compute threads
+    for (int it = 0; it < n_iter; ++it) {
+      const int b = it & 1;
+      const uint32_t tS = tmem + 128 * b, tdP = tS + 64;
+      const int q0 = block_of(it) * kQStep;
+      const float* lse_c = lse_s + b * kQStep;
+      const float* D_c = D_s + b * kQStep;
+      float nl = 0.f, nd = 0.f;
+      if (tid < kQStep && it + 1 < n_iter) row_data(it + 1, nl, nd);
+      // S^T(it) done (issued two steps back, or before the loop)
+      ok = __all_sync(0xffffffffu, ok && wait(&s_full[b], (it >> 1) & 1, DEVERR_WAIT_ACC_FULL));
+      // ---- P^T and dS^T for this key row against this thread's 32 of the step's queries,
+      // written as bf16 over the first half of its own S^T / dP^T columns (read before
+      // overwrite)
+      if (ok) {
+        tc_fence_after();
+        // no mask: every query is valid and (causal) at or after every key of the block
+        const bool plain =
+            q0 + kQStep <= P.s && k0 + kBlk <= P.s && (!P.causal || q0 >= k0 + kBlk);
+        uint32_t rs[32], rd[32];
+        tmem_ld_32x32b_x32(tS + lane_base + 32 * half, rs);
+        tmem_ld_32x32b_x32(tdP + lane_base + 32 * half, rd);
+        tmem_wait_ld();
         uint32_t pw[16], dw[16];
 #pragma unroll
         for (int e = 0; e < 32; e += 4) {
-          const float4 l4 = *reinterpret_cast<const float4*>(lse_c + c0 + e);
-          const float4 d4 = *reinterpret_cast<const float4*>(D_c + c0 + e);
+          const int c0 = 32 * half + e;
+          const float4 l4 = *reinterpret_cast<const float4*>(lse_c + c0);
+          const float4 d4 = *reinterpret_cast<const float4*>(D_c + c0);
           const float lv[4] = {l4.x, l4.y, l4.z, l4.w}, dv[4] = {d4.x, d4.y, d4.z, d4.w};
           float pr[4], ds[4];
 #pragma unroll
           for (int u = 0; u < 4; ++u) {
-            const int qi = c0 + e + u;
-            pr[u] = exp2_fast(sv[32 * c + e + u] * P.scale_log2 - lv[u]);
+            pr[u] = exp2_fast(__uint_as_float(rs[e + u]) * P.scale_log2 - lv[u]);
             if (!plain) {
-              const int q_abs = q0 + qi;
+              const int q_abs = q0 + c0 + u;
               if (q_abs >= P.s || k_abs >= P.s || (P.causal && k_abs > q_abs)) pr[u] = 0.f;
             }
-            ds[u] = pr[u] * (dp[32 * c + e + u] - dv[u]);
+            ds[u] = pr[u] * (__uint_as_float(rd[e + u]) - dv[u]);
           }
           pw[e >> 1] = pack_bf16x2(pr[0], pr[1]);
           pw[(e >> 1) + 1] = pack_bf16x2(pr[2], pr[3]);
           dw[e >> 1] = pack_bf16x2(ds[0], ds[1]);
           dw[(e >> 1) + 1] = pack_bf16x2(ds[2], ds[3]);
         }
-        st16(tS + lane_base + packed_col(c0 / 2), pw);
-        st16(tdP + lane_base + packed_col(c0 / 2), dw);
+        st16(tS + lane_base + 32 * half, pw);
+        st16(tdP + lane_base + 32 * half, dw);
+        fa::tmem_wait_st();
+        tc_fence_before();
+        mbar_arrive(&p_ready[b]);
       }
-      fa::tmem_wait_st();
-    }
-    if (tid < kBlk && it + 1 < n_iter) {
-      lse_s[((it + 1) & 1) * kBlk + tid] = nl;
-      D_s[((it + 1) & 1) * kBlk + tid] = nd;
-    }
-    tc_fence_before();
-    // every thread's P^T and dS^T (and the next step's row data) are stored; all agree on ok
-    if (!__syncthreads_and(ok ? 1 : 0)) {
-      ok = false;
-      break;
-    }
-    if (tid == 0) {
-      tc_fence_after();
-      const int b = it & 1;
-      const uint32_t qa = smem_addr(sQ + b * L::BLOCK), da = smem_addr(sDO + b * L::BLOCK);
-#pragma unroll
-      for (int kk = 0; kk < kBlk / 16; ++kk) {
-        // A: 16 queries = 8 TMEM columns of P^T / dS^T; B: the [query][dim] tiles read
-        // MN-major (N = dim), 16 query rows per MMA
-        fa::umma_f16_tmem_a(tdV, tS + packed_col(kk * 8),
-                            make_sdesc_sw128(da + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                            (it > 0 || kk > 0) ? 1u : 0u);
-        fa::umma_f16_tmem_a(tdK, tdP + packed_col(kk * 8),
-                            make_sdesc_sw128(qa + kk * 16 * 128, L::TILE, 1024), IDESC_KN,
-                            (it > 0 || kk > 0) ? 1u : 0u);
+      if (tid < kQStep && it + 1 < n_iter) {
+        lse_s[(b ^ 1) * kQStep + tid] = nl;
+        D_s[(b ^ 1) * kQStep + tid] = nd;
       }
-      umma_commit(m_done);
-      // the next step's S^T and dP^T right behind: they overwrite P^T and dS^T only after
-      // these MMAs have read them (issue order)
-      if (it + 1 < n_iter) {
-        ok = wait(&qd_full[(it + 1) & 1], ((it + 1) >> 1) & 1, DEVERR_WAIT_FULL);
-        if (ok) {
-          tc_fence_after();
-          issue_s(it + 1);
-        }
+      // the next step's row data is stored, this step's is read by all; all agree on ok
+      if (!compute_bar_and(ok ? 1 : 0)) {
+        ok = false;
+        break;
       }
     }
+    if (ok)
+      ok = __all_sync(0xffffffffu, wait(&m_done[(n_iter - 1) & 1], ((n_iter - 1) >> 1) & 1,
+                                        DEVERR_WAIT_ACC_EMPTY));
   }
-  if (!__syncthreads_and(ok ? 1 : 0)) ok = false;
-  if (ok) ok = __all_sync(0xffffffffu, wait(m_done, (n_iter - 1) & 1, DEVERR_WAIT_ACC_EMPTY));
-  if (ok) {
+  if (ok && tid < kThreads) {
     tc_fence_after();
     const bool live = k_abs < P.s;
     const int64_t t = static_cast<int64_t>(bi) * P.s + k_abs;
@@ -378,11 +435,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   }
   __syncthreads();
-  if (*abort_flag && tid == 0) {
+  if (*abort_flag && tid == kIssuer) {
     const Drain dr{globaltimer_ns(), P.err};
     dr(kv_full, 0);
-    for (int b = 0; b < 2; ++b)
-      if (nq[b]) dr(&qd_full[b], (nq[b] - 1) & 1);
+    for (int r = 0; r < kRing; ++r)
+      if (nq[r]) dr(&qd_full[r], (nq[r] - 1) & 1);
     if (any_mma) {
       umma_commit(drain);
       dr(drain, 0);
@@ -647,7 +704,9 @@ __global__ void __launch_bounds__(256) combine_kv_kernel(const float* part, int 
 }
 
 template <int HD>
-constexpr int dkv_smem() { return 6 * Tiles<HD>::BLOCK + 4 * kBlk * 4 + 128 + 1024; }
+constexpr int dkv_smem() {
+  return 2 * Tiles<HD>::BLOCK + 2 * kRing * Tiles64<HD>::BLOCK + 4 * kQStep * 4 + 128 + 1024;
+}
 // at least 120 KB, so that no second CTA (which would wait for the 512 TMEM columns) shares an SM
 template <int HD>
 constexpr int dq_smem() {
@@ -672,6 +731,14 @@ inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, c
   const uint64_t dcols = static_cast<uint64_t>(n_q) * HD;
   r = encode_tmap_bf16_3d(&md, dO, dcols, static_cast<uint64_t>(s), static_cast<uint64_t>(b),
                           dcols * 2, dcols * 2 * static_cast<uint64_t>(s), 64, kBlk);
+  if (r != TP_OK) return r;
+  // 64-row boxes of the same tensors: the dK/dV kernel's query steps
+  CUtensorMap mq64, md64;
+  r = encode_tmap_bf16_3d(&mq64, qkv, cols, static_cast<uint64_t>(s), static_cast<uint64_t>(b),
+                          cols * 2, cols * 2 * static_cast<uint64_t>(s), 64, kQStep);
+  if (r != TP_OK) return r;
+  r = encode_tmap_bf16_3d(&md64, dO, dcols, static_cast<uint64_t>(s), static_cast<uint64_t>(b),
+                          dcols * 2, dcols * 2 * static_cast<uint64_t>(s), 64, kQStep);
   if (r != TP_OK) return r;
   static int attr_set[64] = {0};
   int dev = 0;
@@ -704,7 +771,7 @@ inline tp_status launch_bwd(const void* qkv, const void* dO, const float* lse, c
   ProfScope prof(st, "attn_bwd_flash");
   flash_bwd_dkv_kernel<HD><<<dim3(static_cast<unsigned>(P.n_blk),
                                   static_cast<unsigned>(n_kv * P.split), static_cast<unsigned>(b)),
-                             kThreads, dkv_smem_padded<HD>(), st>>>(mq, md, P);
+                             kThreadsIssue, dkv_smem_padded<HD>(), st>>>(mq, mq64, md64, P);
   TP_LAUNCH_CHECK();
   if (P.split > 1) {
     const int64_t n_tok = b * s;
