@@ -49,7 +49,10 @@ struct PairCfg {
   static constexpr int ACC_COLS = TILE;            // accumulator columns in each CTA's TMEM
   static constexpr int TMEM_COLS = 2 * ACC_COLS;   // two accumulators
   static constexpr int BAR_BYTES = 8 * (2 * STAGES + 5) + 32;
-  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_BYTES;
+  static constexpr int BAR_SPAN = (BAR_BYTES + 127) / 128 * 128;
+  static constexpr int EPI_STAGE_FLOATS = 32 * 32;   // per epilogue warp: 32 rows x 32 fp32
+  static constexpr int EPI_STAGE_BYTES = 4 * EPI_STAGE_FLOATS * 4;
+  static constexpr int SMEM_BYTES = 1024 + STAGES * STAGE_BYTES + BAR_SPAN + EPI_STAGE_BYTES;
   static constexpr uint32_t IDESC = sm100::make_idesc_bf16(2 * HALF, TILE, A_MN, B_MN);
   // what the epilogues see: a 128-row x 256-column accumulator, as a one-CTA 128 x 256 tile
   static constexpr int BN = TILE;
@@ -57,6 +60,9 @@ struct PairCfg {
   static constexpr int A_ROWS = HALF;
   static_assert(SMEM_BYTES <= 227 * 1024, "shared memory");
 };
+
+// Tiles of at most this many k-blocks store fp32 accumulators through the staging tiles.
+constexpr int kStageMaxKBlocks = 48;
 
 namespace pair {
 
@@ -151,6 +157,12 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* drain = acc_empty + 2;           // [1]
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  // the epilogue warps' staging tiles, after the barriers: used when a tile's k loop is short
+  // (the epilogue's stores then bound the kernel); with a long k loop the epilogue is hidden
+  // behind the next tile's MMAs and its direct stores measured faster
+  float* epi_stage = pair::tile_k_blocks(gp) <= kStageMaxKBlocks
+                         ? reinterpret_cast<float*>(reinterpret_cast<uint8_t*>(full) + Cfg::BAR_SPAN)
+                         : nullptr;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -345,6 +357,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       ctx.b = b;
       ctx.m0 = mb * Cfg::TILE + Cfg::HALF * static_cast<int>(rank);
       ctx.n0 = nb * Cfg::TILE;
+      ctx.stage = epi_stage ? epi_stage + quarter * Cfg::EPI_STAGE_FLOATS : nullptr;
       Epi::template run<Cfg>(ep, gp, ctx, tsrc);
       tc_fence_before();
       __syncwarp();

@@ -144,6 +144,7 @@ struct EpiCtx {
   int n0;           // first B row of the tile
   int row_end = 0x7fffffff;   // gathered rows (A rows, or B rows when swapped) at or past this
                               // belong to no problem of the tile
+  float* stage = nullptr;     // this warp's 32 x 32 fp32 shared-memory staging tile, if any
 };
 
 __device__ __forceinline__ void decode_mn(int r, const GemmParams& gp, int& mb, int& nb) {
@@ -910,11 +911,47 @@ struct EpiStoreF32 {
     if (!p.swap) {
       const int i = c.m0 + c.row;
       const bool live = i < p.rows_valid && i < c.row_end;
+      // With a staging tile, each 32-column chunk of the warp's 32 rows goes through shared
+      // memory so that the global stores are whole 128-byte row segments (8 lanes per row, 4
+      // rows per instruction) instead of 16 bytes in each of 32 rows.  Float4 slots are XOR
+      // swizzled by row, so both the row-wise writes and the transposed reads are conflict-free.
+      const bool staged = c.stage != nullptr && (p.ld & 3) == 0 &&
+                          (reinterpret_cast<uintptr_t>(base) & 15) == 0;
+      const int lane = threadIdx.x & 31;
+      const int i_warp = i - lane;   // the warp's first row
 #pragma unroll 1
       for (int col = 0; col < Cfg::BN; col += 32) {
         float v[32];
         src.load32(col, v);
         const int j0 = c.n0 + col;
+        if (staged) {
+          float4* mine = reinterpret_cast<float4*>(c.stage + lane * 32);
+#pragma unroll
+          for (int q = 0; q < 8; ++q)
+            mine[q ^ (lane & 7)] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          __syncwarp();
+          const int jq = lane & 7;
+          const int jc = j0 + 4 * jq;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const int r = 4 * k + (lane >> 3);
+            const float4 val = reinterpret_cast<const float4*>(c.stage + r * 32)[jq ^ (r & 7)];
+            const int ir = i_warp + r;
+            if (ir < p.rows_valid && ir < c.row_end) {
+              float* dst = base + static_cast<int64_t>(ir) * p.ld + jc;
+              if (jc + 4 <= p.cols_valid) {
+                *reinterpret_cast<float4*>(dst) = val;
+              } else {
+                const float e4[4] = {val.x, val.y, val.z, val.w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e)
+                  if (jc + e < p.cols_valid) dst[e] = e4[e];
+              }
+            }
+          }
+          __syncwarp();
+          continue;
+        }
         if (live) {
           float* dst = base + i * p.ld + j0;
           if (j0 + 32 <= p.cols_valid && (reinterpret_cast<uintptr_t>(dst) & 15) == 0) {
