@@ -248,14 +248,31 @@ __global__ void __launch_bounds__(256) combine_kernel(
       acc[0] = a.x; acc[1] = a.y; acc[2] = a.z; acc[3] = a.w;
       acc[4] = b.x; acc[5] = b.y; acc[6] = b.z; acc[7] = b.w;
     }
-    for (int j = 0; j < k; ++j) {
-      const float wt = w[t * k + j];
-      const int64_t rr = inv[t * k + j];
-      const float4* r4 = reinterpret_cast<const float4*>(routed + rr * d + c);
-      const float4 a = r4[0], b = r4[1];
-      const float v[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+    // all choices' indices and weights first, then all their rows, so that the loads of the
+    // k rows are in flight together; the sum still runs over the choices in order
+    float wt[kMaxTopK];
+    int64_t rr[kMaxTopK];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] = fmaf(wt, v[e], acc[e]);
+    for (int j = 0; j < kMaxTopK; ++j) {
+      wt[j] = j < k ? w[t * k + j] : 0.f;
+      rr[j] = j < k ? inv[t * k + j] : 0;
+    }
+    float4 ra[kMaxTopK], rb[kMaxTopK];
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
+        const float4* r4 = reinterpret_cast<const float4*>(routed + rr[j] * d + c);
+        ra[j] = r4[0];
+        rb[j] = r4[1];
+      }
+    }
+#pragma unroll
+    for (int j = 0; j < kMaxTopK; ++j) {
+      if (j < k) {
+        const float v[8] = {ra[j].x, ra[j].y, ra[j].z, ra[j].w, rb[j].x, rb[j].y, rb[j].z, rb[j].w};
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] = fmaf(wt[j], v[e], acc[e]);
+      }
     }
     if (bias) {
       const uint4 bw = *reinterpret_cast<const uint4*>(bias + c);
