@@ -377,12 +377,20 @@ __global__ void __launch_bounds__(256) dx_combine_kernel(
   for (int64_t q = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x; q < nv; q += stride) {
     const int64_t t = q / (d / 8);
     const int64_t c = (q - t * (d / 8)) * 8;
-    float acc[8], v[8];
-    reduce::Vec8<float>::load(dxs + static_cast<int64_t>(inv[t * k]) * d + c, acc);
-    for (int j = 1; j < k; ++j) {
-      reduce::Vec8<float>::load(dxs + static_cast<int64_t>(inv[t * k + j]) * d + c, v);
+    // every choice's row is loaded before the in-order sum, so the k loads are in flight together
+    float vr[kMaxTopK][8];
 #pragma unroll
-      for (int e = 0; e < 8; ++e) acc[e] += v[e];
+    for (int j = 0; j < kMaxTopK; ++j)
+      if (j < k) reduce::Vec8<float>::load(dxs + static_cast<int64_t>(inv[t * k + j]) * d + c, vr[j]);
+    float acc[8], v[8];
+#pragma unroll
+    for (int e = 0; e < 8; ++e) acc[e] = vr[0][e];
+#pragma unroll
+    for (int j = 1; j < kMaxTopK; ++j) {
+      if (j < k) {
+#pragma unroll
+        for (int e = 0; e < 8; ++e) acc[e] += vr[j][e];
+      }
     }
     reduce::Vec8<float>::load(dxr + t * d + c, v);
 #pragma unroll
