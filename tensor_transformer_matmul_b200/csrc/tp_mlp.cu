@@ -1064,8 +1064,10 @@ tp_status moe_routed(const MoeLayout& M, const void* x, const void* wr, const vo
   auto* hs = reinterpret_cast<__nv_bfloat16*>(off(workspace, M.hs_off));
   float* part = reinterpret_cast<float*>(off(workspace, M.part_off));
   const MlpLayout& L = M.ex;
-  // (1) router logits = x Wr (Wr [d][E] read MN-major), fp32
-  if (M.E % 64) {
+  // (1) router logits = x Wr (Wr [d][E] read MN-major), fp32: on the tensor cores when Wr's rows
+  // are whole 16-byte units (E a multiple of 8; the 64-wide loads past E read zeros and the
+  // epilogue writes the E valid columns), else one block per token on the SIMT core
+  if (M.E % 8) {
     ProfScope prof(s, "moe_router");
     const int threads = (256 / M.E) * M.E;
     TP_LAUNCH_PDL(moe::router_simt_kernel, dim3(static_cast<unsigned>(M.T)), dim3(threads), 0, s,
@@ -1081,7 +1083,7 @@ tp_status moe_routed(const MoeLayout& M, const void* x, const void* wr, const vo
     ep.rows_valid = static_cast<int32_t>(M.T);
     ep.cols_valid = M.E;
     ep.swap = 0;
-    st = M.E == 64 ? tc::run_gemm<TileCfg<64, 1, false, true, stages_for(64, 1)>, tc::EpiStoreF32>(
+    st = M.E <= 64 ? tc::run_gemm<TileCfg<64, 1, false, true, stages_for(64, 1)>, tc::EpiStoreF32>(
                          xo, ro, M.T, M.E, M.d, 1, ep, s, "moe_router")
                    : tc::run_gemm<TileCfg<128, 1, false, true, stages_for(128, 1)>, tc::EpiStoreF32>(
                          xo, ro, M.T, M.E, M.d, 1, ep, s, "moe_router");
